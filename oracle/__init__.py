@@ -1,0 +1,368 @@
+"""CPU oracle for block-scaled FP4 quantization -- TEST INFRASTRUCTURE ONLY.
+
+This package is the plain, slow, obviously-correct definition that the CUDA
+library is checked against.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import it; the library
+(``fp4_block_scaled_04_b200``) never does, and the two share no code.
+
+The arithmetic lives in ``fp4q_oracle.c`` (plain C, binary32, no FMA
+contraction); this module compiles it on first use (``gcc -O2
+-ffp-contract=off``) and wraps it for numpy arrays.  All arrays here are host
+numpy arrays; BF16 tensors are passed as their uint16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp4q_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+BF16, FP32 = 0, 1
+ROWWISE, COLWISE = 1, 2
+RNE, SR = 0, 1
+SCALE_LINEAR, SCALE_SWIZZLED = 0, 1
+E8M0_RNE, E8M0_CEIL, E8M0_OCP_FLOOR = 0, 1, 2
+FMT_NVFP4, FMT_MXFP4, FMT_IF4 = 0, 1, 2
+
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+
+def build(force: bool = False) -> str:
+    """Compile fp4q_oracle.c into liboracle.so (idempotent)."""
+    with _lock:
+        stale = (not os.path.exists(_LIB_PATH)
+                 or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+        if force or stale:
+            tmp = _LIB_PATH + f".{os.getpid()}.tmp"
+            subprocess.check_call(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"])
+            os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I64, I, U, U64, F = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                ctypes.c_uint, ctypes.c_uint64, ctypes.c_float)
+        sig = {
+            "orc_bf16_to_f32": (F, [ctypes.c_uint16]),
+            "orc_f32_to_bf16": (ctypes.c_uint16, [F]),
+            "orc_e2m1_value": (F, [ctypes.c_uint8]),
+            "orc_e2m1_rne": (ctypes.c_uint8, [F]),
+            "orc_e2m1_sr": (ctypes.c_uint8, [F, ctypes.c_uint32]),
+            "orc_e4m3_value": (F, [ctypes.c_uint8]),
+            "orc_e4m3_rne_sat": (ctypes.c_uint8, [F]),
+            "orc_e8m0_exponent": (I, [F, I]),
+            "orc_philox4x32_10": (None, [P, P, P]),
+            "orc_sr_bits16": (ctypes.c_uint32, [U64, U64]),
+            "orc_rht_signs": (None, [U64, I, P]),
+            "orc_scale_bytes": (I64, [I64, I64, I]),
+            "orc_scale_offset": (I64, [I64, I64, I64, I64, I]),
+            "orc_amax": (F, [P, I, I64, I64, I64]),
+            "orc_tensor_scales": (None, [F, P, P]),
+            "orc_quantize_nvfp4": (I, [P, I, I64, I64, I64, U, I, U64, P, P, P, P, P, P, I]),
+            "orc_quantize_mxfp4": (I, [P, I, I64, I64, I64, U, I, P, P, P, P, I]),
+            "orc_quantize_2d": (I, [P, I, I64, I64, I64, P, P, P, P, P, P, P, I]),
+            "orc_rht_norm": (F, [I]),
+            "orc_rht": (I, [P, I, I64, I64, I64, I, U64, P]),
+            "orc_quantize_rht": (I, [P, I, I64, I64, I64, I, I, U64, P, P, P, P, I, P]),
+            "orc_if4_c76": (F, []),
+            "orc_if4_c67": (F, []),
+            "orc_quantize_if4": (I, [P, I, I64, I64, I64, P, P, P, P, I, I]),
+            "orc_dequantize": (I, [I, P, P, I, I, I, P, I64, I64, P, I]),
+            "orc_glossary_mae": (ctypes.c_double, [P, I64, I64]),
+            "orc_e2m1_rne_n": (None, [P, P, I64]),
+            "orc_e2m1_sr_n": (None, [P, P, P, I64]),
+            "orc_e4m3_rne_sat_n": (None, [P, P, I64]),
+            "orc_e8m0_exponent_n": (None, [P, I, P, I64]),
+            "orc_sr_bits16_n": (None, [U64, U64, P, I64]),
+            "orc_f32_to_bf16_n": (None, [P, P, I64]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------------------
+# numpy helpers
+# ---------------------------------------------------------------------------
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_code(x: np.ndarray) -> int:
+    if x.dtype == np.uint16:
+        return BF16
+    if x.dtype == np.float32:
+        return FP32
+    raise TypeError("oracle inputs are BF16 bit patterns (uint16) or float32")
+
+
+def _f32(v) -> ctypes.c_float:
+    return ctypes.c_float(float(v))
+
+
+def scale_bytes(rows: int, cols: int, layout: int) -> int:
+    return int(lib().orc_scale_bytes(rows, cols, layout))
+
+
+def scale_offset(r: int, c: int, rows: int, cols: int, layout: int) -> int:
+    return int(lib().orc_scale_offset(r, c, rows, cols, layout))
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def e2m1_rne(v: float) -> int:
+    return int(lib().orc_e2m1_rne(float(np.float32(v))))
+
+
+def e2m1_rne_array(v: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.zeros(v.shape, np.uint8)
+    lib().orc_e2m1_rne_n(_ptr(v), _ptr(out), v.size)
+    return out
+
+
+def e2m1_sr_array(v: np.ndarray, u16: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    u = np.ascontiguousarray(u16, dtype=np.uint32)
+    assert u.shape == v.shape
+    out = np.zeros(v.shape, np.uint8)
+    lib().orc_e2m1_sr_n(_ptr(v), _ptr(u), _ptr(out), v.size)
+    return out
+
+
+def e4m3_rne_sat_array(s: np.ndarray) -> np.ndarray:
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    out = np.zeros(s.shape, np.uint8)
+    lib().orc_e4m3_rne_sat_n(_ptr(s), _ptr(out), s.size)
+    return out
+
+
+def e8m0_exponent_array(m: np.ndarray, mode: int = E8M0_RNE) -> np.ndarray:
+    m = np.ascontiguousarray(m, dtype=np.float32)
+    out = np.zeros(m.shape, np.int32)
+    lib().orc_e8m0_exponent_n(_ptr(m), mode, _ptr(out), m.size)
+    return out
+
+
+def sr_bits16_array(seed: int, first_index: int, n: int) -> np.ndarray:
+    out = np.zeros(n, np.uint32)
+    lib().orc_sr_bits16_n(seed, first_index, _ptr(out), n)
+    return out
+
+
+def f32_to_bf16_array(v: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.zeros(v.shape, np.uint16)
+    lib().orc_f32_to_bf16_n(_ptr(v), _ptr(out), v.size)
+    return out
+
+
+def e2m1_sr(v: float, u16: int) -> int:
+    return int(lib().orc_e2m1_sr(float(np.float32(v)), int(u16)))
+
+
+def e2m1_value(code: int) -> float:
+    return float(lib().orc_e2m1_value(int(code)))
+
+
+def e4m3_rne_sat(s: float) -> int:
+    return int(lib().orc_e4m3_rne_sat(float(np.float32(s))))
+
+
+def e4m3_value(code: int) -> float:
+    return float(lib().orc_e4m3_value(int(code)))
+
+
+def e8m0_exponent(block_amax: float, mode: int = E8M0_RNE) -> int:
+    return int(lib().orc_e8m0_exponent(float(np.float32(block_amax)), mode))
+
+
+def philox4x32_10(counter, key) -> np.ndarray:
+    c = np.asarray(counter, dtype=np.uint32).copy()
+    k = np.asarray(key, dtype=np.uint32).copy()
+    out = np.zeros(4, dtype=np.uint32)
+    lib().orc_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def sr_bits16(seed: int, index: int) -> int:
+    return int(lib().orc_sr_bits16(seed, index))
+
+
+def rht_signs(seed: int, n: int) -> np.ndarray:
+    out = np.zeros(n, dtype=np.float32)
+    lib().orc_rht_signs(seed, n, _ptr(out))
+    return out
+
+
+def rht_norm(n: int) -> float:
+    return float(lib().orc_rht_norm(n))
+
+
+def amax(x: np.ndarray) -> float:
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    return float(lib().orc_amax(_ptr(x), _dtype_code(x), rows, cols, cols))
+
+
+def tensor_scales(a: float):
+    e, d = ctypes.c_float(), ctypes.c_float()
+    lib().orc_tensor_scales(float(np.float32(a)), ctypes.byref(e), ctypes.byref(d))
+    return e.value, d.value
+
+
+def _amax_arg(a):
+    if a is None:
+        return None, None
+    buf = np.array([a], dtype=np.float32)
+    return buf, _ptr(buf)
+
+
+def quantize_nvfp4(x: np.ndarray, layouts: int = ROWWISE, round: int = RNE, seed: int = 0,
+                   amax: float | None = None, scale_layout: int = SCALE_LINEAR) -> dict:
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    out = {"s_dec": np.zeros(1, np.float32)}
+    if layouts & ROWWISE:
+        out["q_row"] = np.zeros((rows, cols // 2), np.uint8)
+        out["sf_row"] = np.zeros(scale_bytes(rows, cols // 16, scale_layout), np.uint8)
+    if layouts & COLWISE:
+        out["q_col"] = np.zeros((cols, rows // 2), np.uint8)
+        out["sf_col"] = np.zeros(scale_bytes(cols, rows // 16, scale_layout), np.uint8)
+    keep, ap = _amax_arg(amax)
+    rc = lib().orc_quantize_nvfp4(_ptr(x), _dtype_code(x), rows, cols, cols, layouts, round,
+                                  seed, ap, _ptr(out["s_dec"]), _ptr(out.get("q_row")),
+                                  _ptr(out.get("sf_row")), _ptr(out.get("q_col")),
+                                  _ptr(out.get("sf_col")), scale_layout)
+    if rc != 0:
+        raise ValueError(f"oracle rejected shape {x.shape}")
+    return out
+
+
+def quantize_mxfp4(x: np.ndarray, layouts: int = ROWWISE, e8m0_mode: int = E8M0_RNE,
+                   scale_layout: int = SCALE_LINEAR) -> dict:
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    out = {}
+    if layouts & ROWWISE:
+        out["q_row"] = np.zeros((rows, cols // 2), np.uint8)
+        out["sf_row"] = np.zeros(scale_bytes(rows, cols // 32, scale_layout), np.uint8)
+    if layouts & COLWISE:
+        out["q_col"] = np.zeros((cols, rows // 2), np.uint8)
+        out["sf_col"] = np.zeros(scale_bytes(cols, rows // 32, scale_layout), np.uint8)
+    rc = lib().orc_quantize_mxfp4(_ptr(x), _dtype_code(x), rows, cols, cols, layouts,
+                                  e8m0_mode, _ptr(out.get("q_row")), _ptr(out.get("sf_row")),
+                                  _ptr(out.get("q_col")), _ptr(out.get("sf_col")), scale_layout)
+    if rc != 0:
+        raise ValueError(f"oracle rejected shape {x.shape}")
+    return out
+
+
+def quantize_2d(w: np.ndarray, amax: float | None = None, with_1x16: bool = False,
+                scale_layout: int = SCALE_LINEAR) -> dict:
+    w = np.ascontiguousarray(w)
+    rows, cols = w.shape
+    out = {"s_dec": np.zeros(1, np.float32),
+           "q_w": np.zeros((rows, cols // 2), np.uint8),
+           "q_wt": np.zeros((cols, rows // 2), np.uint8),
+           "sf_tiles": np.zeros((rows // 16, cols // 16), np.uint8)}
+    if with_1x16:
+        out["sf_w_1x16"] = np.zeros(scale_bytes(rows, cols // 16, scale_layout), np.uint8)
+        out["sf_wt_1x16"] = np.zeros(scale_bytes(cols, rows // 16, scale_layout), np.uint8)
+    keep, ap = _amax_arg(amax)
+    rc = lib().orc_quantize_2d(_ptr(w), _dtype_code(w), rows, cols, cols, ap,
+                               _ptr(out["s_dec"]), _ptr(out["q_w"]), _ptr(out["q_wt"]),
+                               _ptr(out["sf_tiles"]), _ptr(out.get("sf_w_1x16")),
+                               _ptr(out.get("sf_wt_1x16")), scale_layout)
+    if rc != 0:
+        raise ValueError(f"oracle rejected shape {w.shape}")
+    return out
+
+
+def rht(dy: np.ndarray, n: int, seed: int = 0) -> np.ndarray:
+    dy = np.ascontiguousarray(dy)
+    tokens, cols = dy.shape
+    out = np.zeros((tokens, cols), np.float32)
+    rc = lib().orc_rht(_ptr(dy), _dtype_code(dy), tokens, cols, cols, n, seed, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected RHT arguments")
+    return out
+
+
+def quantize_rht(dy: np.ndarray, n: int, round: int = SR, seed: int = 0,
+                 amax_rht: float | None = None, scale_layout: int = SCALE_LINEAR,
+                 want_rht: bool = False) -> dict:
+    dy = np.ascontiguousarray(dy)
+    tokens, cols = dy.shape
+    out = {"s_dec": np.zeros(1, np.float32),
+           "q_t": np.zeros((cols, tokens // 2), np.uint8),
+           "sf_t": np.zeros(scale_bytes(cols, tokens // 16, scale_layout), np.uint8)}
+    if want_rht:
+        out["rht"] = np.zeros((tokens, cols), np.float32)
+    keep, ap = _amax_arg(amax_rht)
+    rc = lib().orc_quantize_rht(_ptr(dy), _dtype_code(dy), tokens, cols, cols, n, round, seed,
+                                ap, _ptr(out["s_dec"]), _ptr(out["q_t"]), _ptr(out["sf_t"]),
+                                scale_layout, _ptr(out.get("rht")))
+    if rc != 0:
+        raise ValueError("oracle rejected RHT arguments")
+    return out
+
+
+def if4_constants():
+    return float(lib().orc_if4_c76()), float(lib().orc_if4_c67())
+
+
+def quantize_if4(x: np.ndarray, amax: float | None = None, scale_layout: int = SCALE_LINEAR,
+                 allow_int4: bool = True) -> dict:
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    out = {"s_dec": np.zeros(1, np.float32),
+           "q": np.zeros((rows, cols // 2), np.uint8),
+           "sf": np.zeros(scale_bytes(rows, cols // 16, scale_layout), np.uint8)}
+    keep, ap = _amax_arg(amax)
+    rc = lib().orc_quantize_if4(_ptr(x), _dtype_code(x), rows, cols, cols, ap,
+                                _ptr(out["s_dec"]), _ptr(out["q"]), _ptr(out["sf"]),
+                                scale_layout, 1 if allow_int4 else 0)
+    if rc != 0:
+        raise ValueError(f"oracle rejected shape {x.shape}")
+    return out
+
+
+def dequantize(fmt: int, q: np.ndarray, sf: np.ndarray, rows: int, cols: int,
+               block_rows: int = 1, block_cols: int = 16, s_dec: float | None = None,
+               scale_layout: int = SCALE_LINEAR, out_dtype: int = FP32) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    y = np.zeros((rows, cols), np.float32 if out_dtype == FP32 else np.uint16)
+    keep, sp = _amax_arg(s_dec)
+    rc = lib().orc_dequantize(fmt, _ptr(q), _ptr(sf), scale_layout, block_rows, block_cols, sp,
+                              rows, cols, _ptr(y), out_dtype)
+    if rc != 0:
+        raise ValueError("oracle rejected dequant arguments")
+    return y
+
+
+def glossary_mae(x: np.ndarray, block: int) -> float:
+    x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1)
+    return float(lib().orc_glossary_mae(_ptr(x), x.size, block))

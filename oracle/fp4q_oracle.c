@@ -1,0 +1,732 @@
+/*
+ * fp4q_oracle.c -- plain CPU definition of block-scaled FP4 quantization.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the oracle that the CUDA library is
+ * checked against.  Only the tests, the smoke check and the benchmark's CPU
+ * baseline may load it; the library itself never does, and the two share no
+ * code, headers, tables or constants.
+ *
+ * Every result is written out step by step, in IEEE binary32, in the order
+ * stated next to each function.  Build with -O2 -ffp-contract=off and without
+ * -ffast-math on x86-64 (SSE arithmetic, no excess precision), so that each
+ * C float operation below is one correctly rounded binary32 operation
+ * ("RN(.)" in the comments).  Speed is not a goal: scale and element codes are
+ * found by enumerating the format's values.
+ *
+ * Sources (the pages this follows):
+ *   [Q]  Qiita note on the NVFP4 pre-training paper (nishiha): sections
+ *        "NVFP4データの変換" (E2M1 definition), "2D scaling", "ランダム
+ *        アダマール変換" (RHT), "確率的丸め" (stochastic rounding),
+ *        "NVFP4の表現できる最大値" (2688), "scaleの導出" (scale derivation).
+ *   [G]  Ultralytics glossary "FP4": "FP4の仕組み" (MXFP4 / NVFP4 and the
+ *        block-size worked example).
+ *   [I]  gist.science explainer of "Adaptive Block-Scaled Data Types":
+ *        section 2 "提案手法：IF4" (IF4 selection, sign-bit flag, 6/7 method).
+ *   [F]  blog.ast.moe "FP6から考えるLLM量子化": remark that round-to-nearest-
+ *        even matters when converting the shared scale to E8M0.
+ * Where the pages are silent the plainest reading is taken; each such place is
+ * marked READING below.
+ */
+#include <float.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_BF16 0
+#define ORC_FP32 1
+#define ORC_ROWWISE 1u
+#define ORC_COLWISE 2u
+#define ORC_RNE 0
+#define ORC_SR 1
+#define ORC_SCALE_LINEAR 0
+#define ORC_SCALE_SWIZZLED 1
+#define ORC_E8M0_RNE 0
+#define ORC_E8M0_CEIL 1
+#define ORC_E8M0_OCP_FLOOR 2
+#define ORC_FMT_NVFP4 0
+#define ORC_FMT_MXFP4 1
+#define ORC_FMT_IF4 2
+
+/* ------------------------------------------------------------------------ */
+/* Scalar helpers                                                            */
+/* ------------------------------------------------------------------------ */
+
+static float f32_from_bits(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t bits_from_f32(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+/* BF16 -> FP32 is exact: the 16 bits are the high half of the FP32 word. */
+float orc_bf16_to_f32(uint16_t b) { return f32_from_bits((uint32_t)b << 16); }
+
+/* FP32 -> BF16, round to nearest even (finite inputs; NaN kept quiet). */
+uint16_t orc_f32_to_bf16(float f) {
+  uint32_t u = bits_from_f32(f);
+  if (isnan(f)) return (uint16_t)((u >> 16) | 0x40);
+  uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7FFFu + lsb;
+  return (uint16_t)(u >> 16);
+}
+
+static float load_elem(const void *x, int dtype, int64_t ld, int64_t r, int64_t c) {
+  if (dtype == ORC_BF16) return orc_bf16_to_f32(((const uint16_t *)x)[r * ld + c]);
+  return ((const float *)x)[r * ld + c];
+}
+
+/* ------------------------------------------------------------------------ */
+/* E2M1 (FP4) element format  [Q] "NVFP4データの変換", [G] "FP4の仕組み"       */
+/*   value = (-1)^s (0 + m/2) 2^e           for e = 0                        */
+/*   value = (-1)^s (1 + m/2) 2^(e-1)       for e > 0                        */
+/* giving magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 for codes 0..7; bit 3 = sign.*/
+/* ------------------------------------------------------------------------ */
+
+float orc_e2m1_value(uint8_t code) {
+  int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+  double mag = (e == 0) ? (0.0 + 0.5 * m) : (1.0 + 0.5 * m) * ldexp(1.0, e - 1);
+  return (float)(s ? -mag : mag);
+}
+
+/* Nearest E2M1 value to v; a tie goes to the even code (round to nearest
+ * even); magnitudes beyond 6 saturate to 6.  READING: the sign bit copies the
+ * sign of v, so a negative value that rounds to zero gives code 0x8. */
+uint8_t orc_e2m1_rne(float v) {
+  double a = fabs((double)v);
+  int best = 0;
+  double best_d = INFINITY;
+  if (a >= 6.0) /* saturate: 6 is the nearest value to anything above it */
+    return (uint8_t)(7 | (signbit(v) ? 8 : 0));
+  for (int c = 0; c < 8; ++c) {
+    double d = fabs(a - (double)orc_e2m1_value((uint8_t)c));
+    if (d < best_d || (d == best_d && (c % 2) == 0)) { best = c; best_d = d; }
+  }
+  return (uint8_t)(best | (signbit(v) ? 8 : 0));
+}
+
+/* Stochastic rounding onto the E2M1 grid  [Q] "確率的丸め".
+ * The page rounds x + U(-1/2, 1/2) on a unit grid, i.e. it rounds up with
+ * probability equal to the distance from the lower neighbour.  READING: the
+ * same rule on the non-uniform E2M1 grid with 16 random bits: between adjacent
+ * magnitudes lo <= |v| < hi, t = (|v| - lo)/(hi - lo) (exact: Sterbenz and a
+ * power-of-two divisor) and the magnitude rounds up iff u < t * 2^16.
+ * |v| >= 6 saturates to 6.  The sign is copied. */
+uint8_t orc_e2m1_sr(float v, uint32_t u16) {
+  float a = fabsf(v);
+  int code;
+  if (a >= 6.0f) {
+    code = 7;
+  } else {
+    int lo = 0;
+    for (int c = 0; c < 8; ++c)
+      if (orc_e2m1_value((uint8_t)c) <= a) lo = c;
+    float lo_v = orc_e2m1_value((uint8_t)lo);
+    float hi_v = orc_e2m1_value((uint8_t)(lo + 1));
+    float t = (a - lo_v) / (hi_v - lo_v);
+    int up = (float)(u16 & 0xFFFFu) < t * 65536.0f;
+    code = lo + up;
+  }
+  return (uint8_t)(code | (signbit(v) ? 8 : 0));
+}
+
+/* ------------------------------------------------------------------------ */
+/* E4M3 (FP8, "fn": no infinities, 0x7F/0xFF = NaN) block-scale format       */
+/* [Q] "NVFP4の表現できる最大値": the largest E4M3 value is 448.             */
+/* ------------------------------------------------------------------------ */
+
+float orc_e4m3_value(uint8_t code) {
+  int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+  if (e == 15 && m == 7) return NAN;
+  double mag = (e == 0) ? m * ldexp(1.0, -9) : (1.0 + m / 8.0) * ldexp(1.0, e - 7);
+  return (float)(s ? -mag : mag);
+}
+
+/* Nearest non-negative E4M3 value to s >= 0, ties to the even code, values
+ * at or above 448 saturate to 448 (code 0x7E). */
+uint8_t orc_e4m3_rne_sat(float s) {
+  if (s >= 448.0f) return 0x7E;
+  int best = 0;
+  double best_d = INFINITY;
+  for (int c = 0; c <= 0x7E; ++c) {
+    double d = fabs((double)s - (double)orc_e4m3_value((uint8_t)c));
+    if (d < best_d || (d == best_d && (c % 2) == 0)) { best = c; best_d = d; }
+  }
+  return (uint8_t)best;
+}
+
+/* ------------------------------------------------------------------------ */
+/* E8M0 shared scale (MXFP4)  [G] "FP4の仕組み", [F] E8M0 rounding remark     */
+/* Returns the unbiased exponent e of the scale 2^e, e in [-127, 127];       */
+/* the stored byte is e + 127.                                               */
+/* ------------------------------------------------------------------------ */
+
+/* split a positive float into f * 2^E with f in [1, 2) (exact) */
+static void split_pow2(float a, double *f, int *E) {
+  int e2;
+  double fr = frexp((double)a, &e2); /* fr in [0.5, 1) */
+  *f = fr * 2.0;
+  *E = e2 - 1;
+}
+
+int orc_e8m0_exponent(float block_amax, int mode) {
+  int e;
+  if (!(block_amax > 0.0f)) return -127;
+  if (mode == ORC_E8M0_OCP_FLOOR) {
+    /* floor(log2(amax)) - 2: the largest E2M1 magnitude is 1.5 * 2^2 */
+    double f; int E;
+    split_pow2(block_amax, &f, &E);
+    e = E - 2;
+  } else {
+    /* map the block maximum to 6: the scale before rounding is RN(amax/6) */
+    float target = block_amax / 6.0f;
+    if (!(target > 0.0f)) return -127;
+    double f; int E;
+    split_pow2(target, &f, &E);
+    if (mode == ORC_E8M0_CEIL) {
+      e = (f > 1.0) ? E + 1 : E;             /* smallest 2^e >= target */
+    } else {
+      /* nearest power of two (linear distance: the midpoint of 2^E and
+       * 2^(E+1) is 1.5 * 2^E); at the exact midpoint take the even biased
+       * exponent.  READING of "round-to-nearest-even" for E8M0. */
+      if (f > 1.5) e = E + 1;
+      else if (f < 1.5) e = E;
+      else e = (((E + 127) & 1) == 0) ? E : E + 1;
+    }
+  }
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return e;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As   */
+/* Easy as 1, 2, 3", SC'11): 10 rounds of the 4x32 S-box with multipliers    */
+/* 0xD2511F53 / 0xCD9E8D57 and Weyl key increments 0x9E3779B9 / 0xBB67AE85.  */
+/* ------------------------------------------------------------------------ */
+
+void orc_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4]) {
+  uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+  uint32_t k0 = key_in[0], k1 = key_in[1];
+  for (int round = 0; round < 10; ++round) {
+    if (round > 0) { k0 += 0x9E3779B9u; k1 += 0xBB67AE85u; }
+    uint64_t p0 = (uint64_t)0xD2511F53u * (uint64_t)c0;
+    uint64_t p1 = (uint64_t)0xCD9E8D57u * (uint64_t)c2;
+    uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+    uint32_t n0 = hi1 ^ c1 ^ k0, n1 = lo1, n2 = hi0 ^ c3 ^ k1, n3 = lo0;
+    c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+  }
+  out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* READING (the pages give no bit mapping): the 16 random bits of the element
+ * with flat row-major index i of the input tensor come from the Philox call
+ * with counter (g mod 2^32, g div 2^32, 0, 0), g = i div 8, keyed by
+ * (seed mod 2^32, seed div 2^32); element i takes bits 16*(i mod 2) .. +15 of
+ * output word (i mod 8) div 2. */
+uint32_t orc_sr_bits16(uint64_t seed, uint64_t i) {
+  uint64_t g = i / 8;
+  uint32_t ctr[4] = {(uint32_t)g, (uint32_t)(g >> 32), 0u, 0u};
+  uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  uint32_t w[4];
+  orc_philox4x32_10(ctr, key, w);
+  return (w[(i % 8) / 2] >> (16 * (i % 2))) & 0xFFFFu;
+}
+
+/* READING: the random diagonal S of the Hadamard transform is one sign vector
+ * of length n per call, drawn from the Philox call with counter (0, 0, 1, 0):
+ * S_k = -1 when bit k of the 128-bit output (word k div 32, bit k mod 32) is
+ * set, else +1.  [Q] "ランダムアダマール変換": S_d has {1, -1} on its diagonal. */
+void orc_rht_signs(uint64_t seed, int n, float *signs) {
+  uint32_t ctr[4] = {0u, 0u, 1u, 0u};
+  uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  uint32_t w[4];
+  orc_philox4x32_10(ctr, key, w);
+  for (int k = 0; k < n; ++k) signs[k] = ((w[k / 32] >> (k % 32)) & 1u) ? -1.0f : 1.0f;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Scale-factor layouts                                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Size in bytes of a [rows, cols] scale matrix in the given layout.  The
+ * swizzled layout is the 128 x 4 block-scale tile layout that NVIDIA
+ * documents for block-scaled tensor-core operands: rows padded to 128, scale
+ * columns padded to 4, each 128 x 4 tile stored as 512 contiguous bytes. */
+int64_t orc_scale_bytes(int64_t rows, int64_t cols, int layout) {
+  if (layout == ORC_SCALE_LINEAR) return rows * cols;
+  int64_t rp = (rows + 127) / 128 * 128, cp = (cols + 3) / 4 * 4;
+  return rp * cp;
+}
+
+int64_t orc_scale_offset(int64_t r, int64_t c, int64_t rows, int64_t cols, int layout) {
+  (void)rows;
+  if (layout == ORC_SCALE_LINEAR) return r * cols + c;
+  int64_t col_tiles = (cols + 3) / 4;
+  int64_t tile = (r / 128) * col_tiles + (c / 4);
+  return tile * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + (c % 4);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Tensor amax and the two-level NVFP4 tensor scale                          */
+/* [Q] "scaleの導出": global_scale = 6*448 / max|x|                          */
+/* ------------------------------------------------------------------------ */
+
+float orc_amax(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld) {
+  float m = 0.0f;
+  int any_nan = 0;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < cols; ++c) {
+      float a = fabsf(load_elem(x, dtype, ld, r, c));
+      if (isnan(a)) any_nan = 1;
+      else if (a > m) m = a;
+    }
+  return any_nan ? NAN : m;
+}
+
+/* global (encode) scale s_enc = RN(2688 / amax), clamped to FLT_MAX, and
+ * the stored (decode) scale s_dec = RN(amax / 2688).  amax == 0 gives 1, 1.
+ * 2688 = 6 * 448 is the largest NVFP4 magnitude ([Q] "NVFP4の表現できる最大値"). */
+void orc_tensor_scales(float amax, float *s_enc, float *s_dec) {
+  if (amax == 0.0f) { *s_enc = 1.0f; *s_dec = 1.0f; return; }
+  float e = 2688.0f / amax;
+  if (e > FLT_MAX) e = FLT_MAX;
+  *s_enc = e;
+  *s_dec = amax / 2688.0f;
+}
+
+/* One NVFP4 block scale  [Q] "scaleの導出": x2 = x * global_scale, the
+ * block's local scale is max|x2| / 6 cast to E4M3.  Because RN is monotone,
+ * max|RN(x * s)| = RN(max|x| * s), so the block maximum is taken on x. */
+static uint8_t nvfp4_block_scale(float block_amax, float s_enc) {
+  float x2_max = block_amax * s_enc;
+  float local = x2_max / 6.0f;
+  return orc_e4m3_rne_sat(local);
+}
+
+/* READING: the element step divides by the block scale once per block:
+ * r = RN(s_enc / S) (0 when S == 0), then v = RN(x * r). */
+static float nvfp4_block_factor(uint8_t sf, float s_enc) {
+  float S = orc_e4m3_value((uint8_t)(sf & 0x7F));
+  return (S == 0.0f) ? 0.0f : s_enc / S;
+}
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 1x16 quantization, row-wise and/or column-wise                      */
+/* [Q] "Blockwise" (16 values per 8-bit scale), "2D scaling" (activations    */
+/* and gradients use 1x16), "誤差逆伝播と転置" (the backward pass needs the   */
+/* transposed operand, hence the column-wise copy).                          */
+/* Row-wise: blocks are 16 consecutive columns of a row; codes [rows, cols/2]*/
+/*   (element 2j in the low nibble), scales [rows, cols/16].                 */
+/* Column-wise: blocks are 16 consecutive rows of a column, written as the   */
+/*   transposed matrix: codes [cols, rows/2], scales [cols, rows/16].        */
+/* SR bits use the element's flat row-major index r*cols + c in the input.   */
+/* ------------------------------------------------------------------------ */
+
+static uint8_t encode_elem(float v, int round, uint64_t seed, uint64_t index) {
+  return (round == ORC_SR) ? orc_e2m1_sr(v, orc_sr_bits16(seed, index)) : orc_e2m1_rne(v);
+}
+
+static void put_nibble(uint8_t *q, int64_t byte_index, int high, uint8_t code) {
+  if (high) q[byte_index] = (uint8_t)((q[byte_index] & 0x0F) | ((code & 0xF) << 4));
+  else q[byte_index] = (uint8_t)((q[byte_index] & 0xF0) | (code & 0xF));
+}
+
+int orc_quantize_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                       unsigned layouts, int round, uint64_t seed, const float *amax_in,
+                       float *s_dec_out, uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col,
+                       uint8_t *sf_col, int scale_layout) {
+  if ((layouts & ORC_ROWWISE) && cols % 16 != 0) return 1;
+  if ((layouts & ORC_COLWISE) && rows % 16 != 0) return 1;
+  float amax = amax_in ? *amax_in : orc_amax(x, dtype, rows, cols, ld);
+  float s_enc, s_dec;
+  orc_tensor_scales(amax, &s_enc, &s_dec);
+  if (s_dec_out) *s_dec_out = s_dec;
+
+  if (layouts & ORC_ROWWISE) {
+    for (int64_t r = 0; r < rows; ++r)
+      for (int64_t b = 0; b < cols / 16; ++b) {
+        float m = 0.0f;
+        for (int k = 0; k < 16; ++k) {
+          float a = fabsf(load_elem(x, dtype, ld, r, b * 16 + k));
+          if (a > m) m = a;
+        }
+        uint8_t sf = nvfp4_block_scale(m, s_enc);
+        float rf = nvfp4_block_factor(sf, s_enc);
+        sf_row[orc_scale_offset(r, b, rows, cols / 16, scale_layout)] = sf;
+        for (int k = 0; k < 16; ++k) {
+          int64_t c = b * 16 + k;
+          float v = load_elem(x, dtype, ld, r, c) * rf;
+          uint8_t code = encode_elem(v, round, seed, (uint64_t)(r * cols + c));
+          put_nibble(q_row, r * (cols / 2) + c / 2, (int)(c & 1), code);
+        }
+      }
+  }
+  if (layouts & ORC_COLWISE) {
+    for (int64_t c = 0; c < cols; ++c)
+      for (int64_t b = 0; b < rows / 16; ++b) {
+        float m = 0.0f;
+        for (int k = 0; k < 16; ++k) {
+          float a = fabsf(load_elem(x, dtype, ld, b * 16 + k, c));
+          if (a > m) m = a;
+        }
+        uint8_t sf = nvfp4_block_scale(m, s_enc);
+        float rf = nvfp4_block_factor(sf, s_enc);
+        sf_col[orc_scale_offset(c, b, cols, rows / 16, scale_layout)] = sf;
+        for (int k = 0; k < 16; ++k) {
+          int64_t r = b * 16 + k;
+          float v = load_elem(x, dtype, ld, r, c) * rf;
+          uint8_t code = encode_elem(v, round, seed, (uint64_t)(r * cols + c));
+          put_nibble(q_col, c * (rows / 2) + r / 2, (int)(r & 1), code);
+        }
+      }
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4: 32 values share one E8M0 power-of-two scale, no tensor scale.      */
+/* [G] "FP4の仕組み" (MXFP4 bullet; scale chosen so the block max is near 6) */
+/* Elements: v = RN(x * 2^-e) (exact except below the normal range), then    */
+/* E2M1 round to nearest even with saturation.                               */
+/* ------------------------------------------------------------------------ */
+
+static float pow2f_exact(int e) { return (float)ldexp(1.0, e); } /* e in [-149, 127] */
+
+int orc_quantize_mxfp4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                       unsigned layouts, int e8m0_mode, uint8_t *q_row, uint8_t *sf_row,
+                       uint8_t *q_col, uint8_t *sf_col, int scale_layout) {
+  if ((layouts & ORC_ROWWISE) && cols % 32 != 0) return 1;
+  if ((layouts & ORC_COLWISE) && rows % 32 != 0) return 1;
+  if (layouts & ORC_ROWWISE) {
+    for (int64_t r = 0; r < rows; ++r)
+      for (int64_t b = 0; b < cols / 32; ++b) {
+        float m = 0.0f;
+        for (int k = 0; k < 32; ++k) {
+          float a = fabsf(load_elem(x, dtype, ld, r, b * 32 + k));
+          if (a > m) m = a;
+        }
+        int e = orc_e8m0_exponent(m, e8m0_mode);
+        sf_row[orc_scale_offset(r, b, rows, cols / 32, scale_layout)] = (uint8_t)(e + 127);
+        float inv = pow2f_exact(-e);
+        for (int k = 0; k < 32; ++k) {
+          int64_t c = b * 32 + k;
+          put_nibble(q_row, r * (cols / 2) + c / 2, (int)(c & 1),
+                     orc_e2m1_rne(load_elem(x, dtype, ld, r, c) * inv));
+        }
+      }
+  }
+  if (layouts & ORC_COLWISE) {
+    for (int64_t c = 0; c < cols; ++c)
+      for (int64_t b = 0; b < rows / 32; ++b) {
+        float m = 0.0f;
+        for (int k = 0; k < 32; ++k) {
+          float a = fabsf(load_elem(x, dtype, ld, b * 32 + k, c));
+          if (a > m) m = a;
+        }
+        int e = orc_e8m0_exponent(m, e8m0_mode);
+        sf_col[orc_scale_offset(c, b, cols, rows / 32, scale_layout)] = (uint8_t)(e + 127);
+        float inv = pow2f_exact(-e);
+        for (int k = 0; k < 32; ++k) {
+          int64_t r = b * 32 + k;
+          put_nibble(q_col, c * (rows / 2) + r / 2, (int)(r & 1),
+                     orc_e2m1_rne(load_elem(x, dtype, ld, r, c) * inv));
+        }
+      }
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 with 16x16 2D block scaling for weights  [Q] "2D scaling":          */
+/* one scale per 16x16 square tile, so quantizing W and quantizing W^T give  */
+/* the same numbers: q(W) = q(W^T)^T.                                         */
+/* Outputs: q_w [rows, cols/2], q_wt [cols, rows/2] (the same nibbles,       */
+/* transposed), tile scales [rows/16, cols/16] (always linear), and          */
+/* optionally the tile scale replicated into 1x16-block form for W           */
+/* ([rows, cols/16]) and for W^T ([cols, rows/16]) in scale_layout.          */
+/* ------------------------------------------------------------------------ */
+
+int orc_quantize_2d(const void *w, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                    const float *amax_in, float *s_dec_out, uint8_t *q_w, uint8_t *q_wt,
+                    uint8_t *sf_tiles, uint8_t *sf_w_1x16, uint8_t *sf_wt_1x16,
+                    int scale_layout) {
+  if (rows % 16 != 0 || cols % 16 != 0) return 1;
+  float amax = amax_in ? *amax_in : orc_amax(w, dtype, rows, cols, ld);
+  float s_enc, s_dec;
+  orc_tensor_scales(amax, &s_enc, &s_dec);
+  if (s_dec_out) *s_dec_out = s_dec;
+  for (int64_t tr = 0; tr < rows / 16; ++tr)
+    for (int64_t tc = 0; tc < cols / 16; ++tc) {
+      float m = 0.0f;
+      for (int i = 0; i < 16; ++i)
+        for (int j = 0; j < 16; ++j) {
+          float a = fabsf(load_elem(w, dtype, ld, tr * 16 + i, tc * 16 + j));
+          if (a > m) m = a;
+        }
+      uint8_t sf = nvfp4_block_scale(m, s_enc);
+      float rf = nvfp4_block_factor(sf, s_enc);
+      sf_tiles[tr * (cols / 16) + tc] = sf;
+      for (int i = 0; i < 16; ++i) {
+        int64_t r = tr * 16 + i;
+        if (sf_w_1x16) sf_w_1x16[orc_scale_offset(r, tc, rows, cols / 16, scale_layout)] = sf;
+        for (int j = 0; j < 16; ++j) {
+          int64_t c = tc * 16 + j;
+          uint8_t code = orc_e2m1_rne(load_elem(w, dtype, ld, r, c) * rf);
+          if (q_w) put_nibble(q_w, r * (cols / 2) + c / 2, (int)(c & 1), code);
+          if (q_wt) put_nibble(q_wt, c * (rows / 2) + r / 2, (int)(r & 1), code);
+        }
+      }
+      if (sf_wt_1x16)
+        for (int j = 0; j < 16; ++j)
+          sf_wt_1x16[orc_scale_offset(tc * 16 + j, tr, cols, rows / 16, scale_layout)] = sf;
+    }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Random Hadamard transform  [Q] "ランダムアダマール変換":                   */
+/*   Wgrad' = q(dY H) q(H^T x), H H^T = I, and the random version multiplies  */
+/*   H by a diagonal S of random signs.                                      */
+/* Per column j of dY [tokens, cols] and per group of n consecutive tokens:  */
+/*   u_k = S_k * x_k;                                                        */
+/*   FWHT in natural (Sylvester) order, stages h = 1, 2, 4, ..., n/2 in this */
+/*   order; at each stage every pair (i, i+h) with (i & h) == 0 becomes      */
+/*   (RN(u_i + u_{i+h}), RN(u_i - u_{i+h}));                                 */
+/*   t_k = RN(u_k * c_n), c_n = RN(1/sqrt(n)) (0.25 for n = 16), so that the */
+/*   transform is orthonormal (H H^T = I).                                   */
+/* READING: the sign flip comes first (H times diag(S)); one S per call.     */
+/* ------------------------------------------------------------------------ */
+
+float orc_rht_norm(int n) { return (float)(1.0 / sqrt((double)n)); }
+
+int orc_rht(const void *dy, int dtype, int64_t tokens, int64_t cols, int64_t ld, int n,
+            uint64_t seed, float *t_out /* [tokens, cols] */) {
+  if (n != 16 && n != 128) return 1;
+  if (tokens % n != 0) return 1;
+  float S[128], u[128];
+  orc_rht_signs(seed, n, S);
+  float cn = orc_rht_norm(n);
+  for (int64_t j = 0; j < cols; ++j)
+    for (int64_t g = 0; g < tokens / n; ++g) {
+      for (int k = 0; k < n; ++k) u[k] = S[k] * load_elem(dy, dtype, ld, g * n + k, j);
+      for (int h = 1; h < n; h *= 2)
+        for (int i = 0; i < n; ++i)
+          if ((i & h) == 0) {
+            float a = u[i], b = u[i + h];
+            u[i] = a + b;
+            u[i + h] = a - b;
+          }
+      for (int k = 0; k < n; ++k) t_out[(g * n + k) * cols + j] = u[k] * cn;
+    }
+  return 0;
+}
+
+/* RHT followed by column-wise NVFP4 1x16 quantization of the transformed
+ * tensor (blocks of 16 tokens; the tensor amax is taken over the transformed
+ * values), written as dY^T codes [cols, tokens/2] and scales [cols, tokens/16].
+ * SR bits use the flat input index token*cols + col.  [Q] "確率的丸め": SR
+ * is what helps gradient quantization. */
+int orc_quantize_rht(const void *dy, int dtype, int64_t tokens, int64_t cols, int64_t ld,
+                     int n, int round, uint64_t seed, const float *amax_rht_in,
+                     float *s_dec_out, uint8_t *q_t, uint8_t *sf_t, int scale_layout,
+                     float *rht_out) {
+  if (n != 16 && n != 128) return 1;
+  if (tokens % n != 0 || tokens % 16 != 0) return 1;
+  float *t = (float *)malloc(sizeof(float) * (size_t)(tokens * cols));
+  if (!t) return 2;
+  orc_rht(dy, dtype, tokens, cols, ld, n, seed, t);
+  if (rht_out) memcpy(rht_out, t, sizeof(float) * (size_t)(tokens * cols));
+  float amax = amax_rht_in ? *amax_rht_in : orc_amax(t, ORC_FP32, tokens, cols, cols);
+  float s_enc, s_dec;
+  orc_tensor_scales(amax, &s_enc, &s_dec);
+  if (s_dec_out) *s_dec_out = s_dec;
+  for (int64_t c = 0; c < cols; ++c)
+    for (int64_t b = 0; b < tokens / 16; ++b) {
+      float m = 0.0f;
+      for (int k = 0; k < 16; ++k) {
+        float a = fabsf(t[(b * 16 + k) * cols + c]);
+        if (a > m) m = a;
+      }
+      uint8_t sf = nvfp4_block_scale(m, s_enc);
+      float rf = nvfp4_block_factor(sf, s_enc);
+      sf_t[orc_scale_offset(c, b, cols, tokens / 16, scale_layout)] = sf;
+      for (int k = 0; k < 16; ++k) {
+        int64_t r = b * 16 + k;
+        float v = t[r * cols + c] * rf;
+        uint8_t code = encode_elem(v, round, seed, (uint64_t)(r * cols + c));
+        put_nibble(q_t, c * (tokens / 2) + r / 2, (int)(r & 1), code);
+      }
+    }
+  free(t);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* IF4: per 16-value block, quantize both as FP4 (E2M1) and as INT4 with the  */
+/* 6/7 method, keep the one with the smaller squared error, and record the   */
+/* choice in the (otherwise unused) sign bit of the E4M3 scale.              */
+/* [I] section 2 "提案手法：IF4" (selection by MSE, sign-bit indicator, 6/7). */
+/* Steps per block (scale S and factor r exactly as NVFP4):                   */
+/*   v_i = RN(x_i * r)                                                        */
+/*   FP4:  g_i = E2M1 value of e2m1_rne(v_i)                                  */
+/*   INT4: k_i = clamp(rint(RN(v_i * C76)), -7, 7), h_i = RN(k_i * C67)       */
+/*         with C76 = RN(7/6), C67 = RN(6/7)                                  */
+/*   e_fp = sum_i (v_i - g_i)^2, e_int = sum_i (v_i - h_i)^2, each summed in  */
+/*         order i = 0..15 as e = fma(d, d, e) with d = RN(v_i - q_i)         */
+/*   INT4 iff e_int < e_fp (ties keep FP4).                                   */
+/* READING: INT4 nibbles hold k_i in two's complement; scale bit 7 set means  */
+/* INT4.  With allow_int4 = 0 the result is NVFP4 row-wise byte for byte.    */
+/* ------------------------------------------------------------------------ */
+
+float orc_if4_c76(void) { return 7.0f / 6.0f; }
+float orc_if4_c67(void) { return 6.0f / 7.0f; }
+
+int orc_quantize_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                     const float *amax_in, float *s_dec_out, uint8_t *q, uint8_t *sf_out,
+                     int scale_layout, int allow_int4) {
+  if (cols % 16 != 0) return 1;
+  float amax = amax_in ? *amax_in : orc_amax(x, dtype, rows, cols, ld);
+  float s_enc, s_dec;
+  orc_tensor_scales(amax, &s_enc, &s_dec);
+  if (s_dec_out) *s_dec_out = s_dec;
+  const float C76 = orc_if4_c76(), C67 = orc_if4_c67();
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < cols / 16; ++b) {
+      float xv[16], v[16];
+      float m = 0.0f;
+      for (int k = 0; k < 16; ++k) {
+        xv[k] = load_elem(x, dtype, ld, r, b * 16 + k);
+        if (fabsf(xv[k]) > m) m = fabsf(xv[k]);
+      }
+      uint8_t sf = nvfp4_block_scale(m, s_enc);
+      float rf = nvfp4_block_factor(sf, s_enc);
+      uint8_t fp_code[16], int_code[16];
+      float e_fp = 0.0f, e_int = 0.0f;
+      for (int k = 0; k < 16; ++k) {
+        v[k] = xv[k] * rf;
+        fp_code[k] = orc_e2m1_rne(v[k]);
+        float g = orc_e2m1_value(fp_code[k]);
+        float kk = rintf(v[k] * C76);
+        if (kk > 7.0f) kk = 7.0f;
+        if (kk < -7.0f) kk = -7.0f;
+        int ki = (int)kk;
+        int_code[k] = (uint8_t)(ki & 0xF);
+        float h = (float)ki * C67;
+        float d_fp = v[k] - g;
+        float d_int = v[k] - h;
+        e_fp = fmaf(d_fp, d_fp, e_fp);
+        e_int = fmaf(d_int, d_int, e_int);
+      }
+      int use_int = allow_int4 && (e_int < e_fp);
+      sf_out[orc_scale_offset(r, b, rows, cols / 16, scale_layout)] =
+          (uint8_t)(sf | (use_int ? 0x80 : 0x00));
+      for (int k = 0; k < 16; ++k) {
+        int64_t c = b * 16 + k;
+        put_nibble(q, r * (cols / 2) + c / 2, (int)(c & 1), use_int ? int_code[k] : fp_code[k]);
+      }
+    }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Dequantization  [G] "FP4の仕組み" (reconstruct = grid value * sign * scale)*/
+/* NVFP4:  y = RN(RN(g * S) * s_dec)   (g * S is exact)                       */
+/* IF4 INT4 blocks: h = RN(k * C67), y = RN(RN(h * S) * s_dec)                */
+/* MXFP4:  y = RN(g * 2^e)                                                    */
+/* Block shape: block_rows x block_cols (1x16, 1x32, or 16x16 for 2D tiles,  */
+/* whose scales are [rows/16, cols/16] linear).  Output FP32 or BF16 (RNE of */
+/* the FP32 result).                                                         */
+/* ------------------------------------------------------------------------ */
+
+int orc_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,
+                   int block_rows, int block_cols, const float *s_dec_in, int64_t rows,
+                   int64_t cols, void *y, int y_dtype) {
+  if (cols % block_cols != 0 || rows % block_rows != 0) return 1;
+  float s_dec = s_dec_in ? *s_dec_in : 1.0f;
+  int64_t srows = rows / block_rows, scols = cols / block_cols;
+  const float C67 = orc_if4_c67();
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < cols; ++c) {
+      uint8_t byte = q[r * (cols / 2) + c / 2];
+      uint8_t code = (c & 1) ? (byte >> 4) : (byte & 0xF);
+      int64_t sr = r / block_rows, sc = c / block_cols;
+      int64_t off = (block_rows == 1) ? orc_scale_offset(sr, sc, srows, scols, scale_layout)
+                                      : sr * scols + sc;
+      uint8_t s = sf[off];
+      float out;
+      if (format == ORC_FMT_MXFP4) {
+        out = orc_e2m1_value(code) * pow2f_exact((int)s - 127);
+      } else {
+        float S = orc_e4m3_value((uint8_t)(s & 0x7F));
+        if (format == ORC_FMT_IF4 && (s & 0x80)) {
+          int k = (code & 0x8) ? (int)code - 16 : (int)code;
+          float h = (float)k * C67;
+          out = (h * S) * s_dec;
+        } else {
+          out = (orc_e2m1_value(code) * S) * s_dec;
+        }
+      }
+      if (y_dtype == ORC_BF16) ((uint16_t *)y)[r * cols + c] = orc_f32_to_bf16(out);
+      else ((float *)y)[r * cols + c] = out;
+    }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Glossary mode  [G] "FP4の仕組み", the block-size worked example:           */
+/* scale = amax_b / 6 in FP32 (no E4M3 rounding), v = |x| / scale per        */
+/* element, nearest E2M1 magnitude with ties to the FIRST (smaller) one       */
+/* (argmin), dequantized value = grid * sign(x) * scale; returns the mean     */
+/* absolute error over the n values (accumulated in double).                  */
+/* ------------------------------------------------------------------------ */
+
+double orc_glossary_mae(const float *x, int64_t n, int64_t block) {
+  static const float grid[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  double err = 0.0;
+  for (int64_t b = 0; b < n / block; ++b) {
+    float m = 0.0f;
+    for (int64_t k = 0; k < block; ++k)
+      if (fabsf(x[b * block + k]) > m) m = fabsf(x[b * block + k]);
+    float scale = m / 6.0f;
+    for (int64_t k = 0; k < block; ++k) {
+      float xv = x[b * block + k];
+      float v = fabsf(xv) / scale;
+      int best = 0;
+      float best_d = fabsf(v - grid[0]);
+      for (int c = 1; c < 8; ++c) {
+        float d = fabsf(v - grid[c]);
+        if (d < best_d) { best = c; best_d = d; }
+      }
+      float sgn = (xv > 0.0f) ? 1.0f : (xv < 0.0f ? -1.0f : 0.0f);
+      float deq = (grid[best] * sgn) * scale;
+      err += fabs((double)deq - (double)xv);
+    }
+  }
+  return err / (double)n;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Array forms of the scalar format functions (for tests over many values).  */
+/* ------------------------------------------------------------------------ */
+
+void orc_e2m1_rne_n(const float *v, uint8_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m1_rne(v[i]);
+}
+
+void orc_e2m1_sr_n(const float *v, const uint32_t *u16, uint8_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m1_sr(v[i], u16[i]);
+}
+
+void orc_e4m3_rne_sat_n(const float *s, uint8_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_rne_sat(s[i]);
+}
+
+void orc_e8m0_exponent_n(const float *m, int mode, int32_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e8m0_exponent(m[i], mode);
+}
+
+void orc_sr_bits16_n(uint64_t seed, uint64_t first_index, uint32_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_sr_bits16(seed, first_index + (uint64_t)i);
+}
+
+void orc_f32_to_bf16_n(const float *v, uint16_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_f32_to_bf16(v[i]);
+}

@@ -1,0 +1,400 @@
+"""Pins for the oracle's quantization recipes (CPU only).
+
+Each check ties the oracle to something outside itself: numbers the pages
+print, invariants the pages state (q(W) = q(W^T)^T under 2D scaling,
+H H^T = I, W'x' = Wx for an invertible transform, IF4 keeps the smaller
+error), exact round trips of constructed representable inputs, scipy's
+Hadamard matrix, exact float64 arithmetic, and error bounds.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+from fp4_block_scaled_04_b200 import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+GRID = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+
+
+def bf16_bits(x) -> np.ndarray:
+    t = torch.as_tensor(x)
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).copy()
+
+
+def code_values(codes: np.ndarray) -> np.ndarray:
+    mag = GRID[codes & 7]
+    return np.where(codes & 8, -mag, mag)
+
+
+def unpack(q: np.ndarray) -> np.ndarray:
+    """[R, C/2] packed bytes -> [R, C] codes (element 2j in the low nibble)."""
+    out = np.empty((q.shape[0], q.shape[1] * 2), np.uint8)
+    out[:, 0::2] = q & 0xF
+    out[:, 1::2] = q >> 4
+    return out
+
+
+def pack(codes: np.ndarray) -> np.ndarray:
+    return (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+
+
+# ---------------------------------------------------------------- pages' numbers
+
+def test_glossary_worked_example(orc):
+    gold = json.load(open(os.path.join(GOLDEN, "glossary_mae.json")))
+    x = workloads.glossary_example().numpy()
+    for block, want in gold["mae"].items():
+        got = orc.glossary_mae(x, int(block))
+        assert round(got, gold["decimals"]) == want, (block, got, want)
+
+
+def test_small_matrix_starts_with_glossary_tensor():
+    x = workloads.small_matrix().float().numpy().reshape(-1)[:4096]
+    g = workloads.glossary_example().to(torch.bfloat16).float().numpy()
+    assert np.array_equal(x, g)
+
+
+def test_qiita_scale_derivation(orc):
+    """The printed local scales [448, 6.5, 16, 13]: the outlier block maps to
+    the E4M3 maximum, the others follow max|x * 6*448/amax| / 6 -> E4M3."""
+    gold = json.load(open(os.path.join(GOLDEN, "qiita_scale_derivation.json")))
+    big = gold["outlier_value"]
+    gs = 6.0 * 448.0 / big
+    x = np.clip(np.random.default_rng(0).standard_normal(64) * 100.0, -120, 120)
+    x[0] = big
+    for b, L in enumerate(gold["printed_local_scales"][1:], start=1):
+        x[16 * b + 3] = L * 6.0 / gs               # this block's max lands on L
+    out = orc.quantize_nvfp4(x.astype(np.float32)[None, :], orc.ROWWISE)
+    got = [orc.e4m3_value(int(s)) for s in out["sf_row"]]
+    assert got == gold["printed_local_scales"]
+
+
+def test_tensor_amax_block_gets_e4m3_max(orc):
+    rng = np.random.default_rng(1)
+    for trial in range(5):
+        x = (rng.standard_normal((64, 128)) * 10.0 ** rng.uniform(-3, 3)).astype(np.float32)
+        out = orc.quantize_nvfp4(x, orc.ROWWISE | orc.COLWISE)
+        r, c = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+        assert out["sf_row"].reshape(64, 8)[r, c // 16] == 0x7E
+        assert out["sf_col"].reshape(128, 4)[c, r // 16] == 0x7E
+        assert out["s_dec"][0] == np.float32(np.abs(x).max()) / np.float32(2688.0)
+
+
+# ---------------------------------------------------------------- NVFP4 1x16
+
+def _representable_blocks(rng, rows, cols, block=16):
+    """x = g(q) * S with one |q| = 6 per block and one block at S = 448, so
+    amax = 2688, s_enc = s_dec = 1 and quantization must give back q and S."""
+    codes = rng.integers(0, 16, (rows, cols)).astype(np.uint8)
+    nb = cols // block
+    sf = rng.integers(8, 0x7E, (rows, nb)).astype(np.uint8)     # normal E4M3 scales
+    sf[0, 0] = 0x7E
+    for r in range(rows):
+        for b in range(nb):
+            pos = b * block + rng.integers(0, block)
+            codes[r, pos] = 7 | (codes[r, pos] & 8)
+    S = np.array([[orcS for orcS in row] for row in sf], np.float64)
+    return codes, sf, S
+
+
+def test_nvfp4_round_trip_of_representable_values(orc):
+    rng = np.random.default_rng(2)
+    rows, cols = 32, 64
+    codes, sf, _ = _representable_blocks(rng, rows, cols)
+    S = np.vectorize(orc.e4m3_value)(sf).astype(np.float64)
+    x = code_values(codes) * np.repeat(S, 16, axis=1)
+    x[codes == 8] = -0.0
+    xb = bf16_bits(torch.from_numpy(x.astype(np.float32)))
+    assert np.array_equal(orc.bf16_bits_to_f32(xb), x.astype(np.float32))   # exact in BF16
+    out = orc.quantize_nvfp4(xb, orc.ROWWISE)
+    assert out["s_dec"][0] == 1.0
+    assert np.array_equal(out["sf_row"].reshape(rows, cols // 16), sf)
+    assert np.array_equal(out["q_row"], pack(codes))
+    y = orc.dequantize(orc.FMT_NVFP4, out["q_row"], out["sf_row"], rows, cols, s_dec=1.0)
+    assert np.array_equal(y, x.astype(np.float32))
+    # the same blocks laid out down the columns come back through COLWISE
+    outc = orc.quantize_nvfp4(np.ascontiguousarray(xb.T), orc.COLWISE)
+    assert np.array_equal(outc["q_col"], pack(codes))
+    assert np.array_equal(outc["sf_col"].reshape(rows, cols // 16), sf)
+
+
+def test_nvfp4_colwise_is_rowwise_of_transpose(orc):
+    x = bf16_bits(workloads.activation(seed=3, rows=64, cols=96, n_outlier_cols=3))
+    for layout in (orc.SCALE_LINEAR, orc.SCALE_SWIZZLED):
+        a = orc.quantize_nvfp4(x, orc.COLWISE, scale_layout=layout)
+        b = orc.quantize_nvfp4(np.ascontiguousarray(x.T), orc.ROWWISE, scale_layout=layout)
+        assert np.array_equal(a["q_col"], b["q_row"])
+        assert np.array_equal(a["sf_col"], b["sf_row"])
+
+
+def test_nvfp4_swizzle_is_a_permutation_of_linear(orc):
+    x = bf16_bits(workloads.activation(seed=4, rows=256, cols=128, n_outlier_cols=2))
+    lin = orc.quantize_nvfp4(x, orc.ROWWISE | orc.COLWISE, scale_layout=orc.SCALE_LINEAR)
+    swz = orc.quantize_nvfp4(x, orc.ROWWISE | orc.COLWISE, scale_layout=orc.SCALE_SWIZZLED)
+    assert np.array_equal(lin["q_row"], swz["q_row"]) and np.array_equal(lin["q_col"], swz["q_col"])
+    for key, (R, C) in (("sf_row", (256, 8)), ("sf_col", (128, 16))):
+        for r in range(R):
+            for c in range(C):
+                assert swz[key][orc.scale_offset(r, c, R, C, orc.SCALE_SWIZZLED)] == lin[key][r * C + c]
+
+
+def test_nvfp4_dequant_error_bound(orc):
+    """|x - dequant(q(x))| <= (half the E2M1 gap at v) * S * s_dec for blocks with
+    a normal E4M3 scale; the gap is at most 2, and saturation (block max
+    slightly above 6 after E4M3 rounding) costs at most 6/16."""
+    x = bf16_bits(workloads.activation(seed=5, rows=128, cols=256, n_outlier_cols=4))
+    xf = orc.bf16_bits_to_f32(x).astype(np.float64)
+    out = orc.quantize_nvfp4(x, orc.ROWWISE)
+    s_dec = float(out["s_dec"][0])
+    y = orc.dequantize(orc.FMT_NVFP4, out["q_row"], out["sf_row"], 128, 256, s_dec=s_dec)
+    S = np.repeat(np.vectorize(orc.e4m3_value)(out["sf_row"].reshape(128, 16)), 16, axis=1)
+    normal = S >= 2.0 ** -6
+    err = np.abs(xf - y)
+    assert np.all(err[normal] <= 1.0 * S[normal] * s_dec * (1 + 1e-5))
+    # a dropped tensor scale or a transposed layout would blow this up
+    assert err.mean() < 0.2 * np.abs(xf).mean()
+
+
+def test_nvfp4_sr_uses_input_index_and_is_unbiased(orc):
+    """SR over many seeds averages to the value (in the scaled domain)."""
+    rng = np.random.default_rng(6)
+    x = np.zeros((1, 16), np.float32)
+    x[0, 0] = 6.0 * 448.0                         # amax 2688: s_enc = 1
+    x[0, 1:] = rng.uniform(-6 * 448, 6 * 448, 15)
+    det = orc.quantize_nvfp4(x, orc.ROWWISE, orc.RNE)
+    S = orc.e4m3_value(int(det["sf_row"][0]))
+    acc = np.zeros(16)
+    n = 4000
+    for seed in range(n):
+        out = orc.quantize_nvfp4(x, orc.ROWWISE, orc.SR, seed=seed)
+        acc += code_values(unpack(out["q_row"]))[0]
+    v = x[0].astype(np.float64) * np.float32(1.0 / S)
+    mean = acc / n
+    # each element is a two-point draw with spread <= 2: sd of the mean <= 1/sqrt(n)
+    assert np.all(np.abs(mean - np.clip(v, -6, 6)) < 5.0 / np.sqrt(n))
+
+
+# ---------------------------------------------------------------- MXFP4
+
+def test_mxfp4_round_trip_and_scale(orc):
+    rng = np.random.default_rng(7)
+    rows, cols = 16, 128
+    codes = rng.integers(0, 16, (rows, cols)).astype(np.uint8)
+    e = rng.integers(-30, 30, (rows, cols // 32))
+    for r in range(rows):
+        for b in range(cols // 32):
+            pos = b * 32 + rng.integers(0, 32)
+            codes[r, pos] = 7 | (codes[r, pos] & 8)
+    x = code_values(codes) * np.exp2(np.repeat(e, 32, axis=1).astype(np.float64))
+    x[codes == 8] = -0.0
+    x32 = x.astype(np.float32)
+    for mode in (orc.E8M0_RNE, orc.E8M0_CEIL):
+        out = orc.quantize_mxfp4(x32, orc.ROWWISE, mode)
+        assert np.array_equal(out["sf_row"].reshape(rows, -1), (e + 127).astype(np.uint8))
+        assert np.array_equal(out["q_row"], pack(codes))
+        y = orc.dequantize(orc.FMT_MXFP4, out["q_row"], out["sf_row"], rows, cols, 1, 32)
+        assert np.array_equal(y, x32)
+    outc = orc.quantize_mxfp4(np.ascontiguousarray(x32.T), orc.COLWISE)
+    assert np.array_equal(outc["q_col"], pack(codes))
+
+
+def test_mxfp4_error_bounds(orc):
+    x = bf16_bits(workloads.activation(seed=8, rows=64, cols=256, n_outlier_cols=4))
+    xf = orc.bf16_bits_to_f32(x).astype(np.float64)
+    for mode, sat in ((orc.E8M0_RNE, 3.0), (orc.E8M0_CEIL, 1.0)):
+        out = orc.quantize_mxfp4(x, orc.ROWWISE | orc.COLWISE, mode)
+        y = orc.dequantize(orc.FMT_MXFP4, out["q_row"], out["sf_row"], 64, 256, 1, 32)
+        scale = np.exp2(np.repeat(out["sf_row"].reshape(64, 8).astype(np.float64) - 127, 32, axis=1))
+        # RNE can round the scale down by up to 1.5x (block max up to 9 -> 6)
+        assert np.all(np.abs(xf - y) <= sat * scale)
+        yc = orc.dequantize(orc.FMT_MXFP4, out["q_col"], out["sf_col"], 256, 64, 1, 32)
+        assert np.abs(xf.T - yc).mean() < 0.15 * np.abs(xf).mean()
+
+
+# ---------------------------------------------------------------- 2D 16x16
+
+def test_2d_transpose_invariance(orc):
+    """Qiita note "2D scaling": with 16x16 tiles, q(W) = q(W^T)^T; with 1x16
+    blocks the two generally differ."""
+    w = workloads.weight(seed=9, rows=64, cols=96).numpy()
+    a = orc.quantize_2d(w)
+    b = orc.quantize_2d(np.ascontiguousarray(w.T))
+    assert np.array_equal(a["q_w"], b["q_wt"]) and np.array_equal(a["q_wt"], b["q_w"])
+    assert np.array_equal(a["sf_tiles"], b["sf_tiles"].T)
+    assert np.array_equal(unpack(a["q_w"]), unpack(a["q_wt"]).T)
+    r1 = orc.quantize_nvfp4(w, orc.ROWWISE)
+    r2 = orc.quantize_nvfp4(np.ascontiguousarray(w.T), orc.ROWWISE)
+    assert not np.array_equal(unpack(r1["q_row"]), unpack(r2["q_row"]).T)
+
+
+def test_2d_round_trip_and_replicated_scales(orc):
+    rng = np.random.default_rng(10)
+    rows, cols = 48, 64
+    codes = rng.integers(0, 16, (rows, cols)).astype(np.uint8)
+    sf = rng.integers(8, 0x7E, (rows // 16, cols // 16)).astype(np.uint8)
+    sf[0, 0] = 0x7E
+    for i in range(rows // 16):
+        for j in range(cols // 16):
+            r, c = 16 * i + rng.integers(0, 16), 16 * j + rng.integers(0, 16)
+            codes[r, c] = 7 | (codes[r, c] & 8)
+    S = np.vectorize(orc.e4m3_value)(sf).astype(np.float64)
+    x = (code_values(codes) * np.kron(S, np.ones((16, 16)))).astype(np.float32)
+    x[codes == 8] = -0.0
+    out = orc.quantize_2d(x, with_1x16=True)
+    assert np.array_equal(out["sf_tiles"], sf)
+    assert np.array_equal(out["q_w"], pack(codes))
+    assert np.array_equal(out["q_wt"], pack(np.ascontiguousarray(codes.T)))
+    assert np.array_equal(out["sf_w_1x16"].reshape(rows, cols // 16), np.repeat(sf, 16, axis=0))
+    assert np.array_equal(out["sf_wt_1x16"].reshape(cols, rows // 16), np.repeat(sf.T, 16, axis=0))
+    y = orc.dequantize(orc.FMT_NVFP4, out["q_w"], out["sf_tiles"], rows, cols, 16, 16, s_dec=1.0)
+    assert np.array_equal(y, x)
+
+
+# ---------------------------------------------------------------- RHT
+
+@pytest.mark.parametrize("n", [16, 128])
+def test_rht_of_unit_vectors_is_scaled_signed_sylvester_hadamard(orc, n):
+    """Columns of the transform of e_k are c_n * S_k * H[:, k] with H the
+    natural-order (Sylvester) Hadamard matrix from scipy; the +-1 matrix
+    satisfies H H^T = n I (Qiita note: H H^T = I after normalisation)."""
+    seed = 1234
+    eye = np.eye(n, dtype=np.float32)
+    t = orc.rht(bf16_bits(torch.from_numpy(eye)), n, seed).astype(np.float64)
+    S = orc.rht_signs(seed, n).astype(np.float64)
+    c = float(np.float32(orc.rht_norm(n)))
+    H = scipy.linalg.hadamard(n).astype(np.float64)
+    assert np.array_equal(t, c * H @ np.diag(S))
+    M = np.rint(t / c)
+    assert np.array_equal(M @ M.T, n * np.eye(n))
+
+
+@pytest.mark.parametrize("n", [16, 128])
+def test_rht_exact_on_small_integers(orc, n):
+    """Integer inputs keep every butterfly exact, so the FP32 result equals
+    one rounding of the float64 product c_n * H diag(S) x."""
+    rng = np.random.default_rng(11)
+    x = rng.integers(-8, 9, (2 * n, 24)).astype(np.float32)
+    seed = 5
+    t = orc.rht(bf16_bits(torch.from_numpy(x)), n, seed)
+    Hs = scipy.linalg.hadamard(n).astype(np.float64) @ np.diag(orc.rht_signs(seed, n).astype(np.float64))
+    c = np.float64(np.float32(orc.rht_norm(n)))
+    for g in range(2):
+        blk = x[g * n:(g + 1) * n].astype(np.float64)
+        want = (c * (Hs @ blk)).astype(np.float32)
+        assert np.array_equal(t[g * n:(g + 1) * n], want)
+
+
+@pytest.mark.parametrize("n", [16, 128])
+def test_rht_preserves_inner_products(orc, n):
+    """FP6 essay, invertible-transform identity: W'x' = Wx when x' = Tx and
+    W' = W T^-1; for the orthonormal RHT T^-1 = T^T, so column inner products
+    over each group of n tokens are kept (to FP32 rounding)."""
+    a = workloads.gradient(seed=12, tokens=4 * n, cols=32)
+    b = workloads.gradient(seed=13, tokens=4 * n, cols=32)
+    ta = orc.rht(bf16_bits(a), n, 3).astype(np.float64)
+    tb = orc.rht(bf16_bits(b), n, 3).astype(np.float64)
+    af, bf = a.float().numpy().astype(np.float64), b.float().numpy().astype(np.float64)
+    for g in range(4):
+        s = slice(g * n, (g + 1) * n)
+        lhs = (ta[s] * tb[s]).sum(0)
+        rhs = (af[s] * bf[s]).sum(0)
+        scale = np.sqrt((af[s] ** 2).sum(0) * (bf[s] ** 2).sum(0))
+        assert np.all(np.abs(lhs - rhs) <= 1e-5 * scale)
+        assert np.allclose((ta[s] ** 2).sum(0), (af[s] ** 2).sum(0), rtol=1e-5)
+
+
+@pytest.mark.parametrize("rnd", [0, 1])
+def test_rht_quantize_is_rht_then_colwise_nvfp4(orc, rnd):
+    dy = bf16_bits(workloads.gradient(seed=14, tokens=256, cols=48))
+    for n in (16, 128):
+        out = orc.quantize_rht(dy, n, round=rnd, seed=77, want_rht=True)
+        t = orc.rht(dy, n, 77)
+        assert np.array_equal(out["rht"], t)
+        ref = orc.quantize_nvfp4(t, orc.COLWISE, round=rnd, seed=77)
+        assert np.array_equal(out["q_t"], ref["q_col"]) and np.array_equal(out["sf_t"], ref["sf_col"])
+        assert out["s_dec"][0] == ref["s_dec"][0]
+
+
+# ---------------------------------------------------------------- IF4
+
+def test_if4_without_int4_is_nvfp4(orc):
+    x = bf16_bits(workloads.if4_blocks(seed=15, rows=32, cols=256))
+    a = orc.quantize_if4(x, allow_int4=False)
+    b = orc.quantize_nvfp4(x, orc.ROWWISE)
+    assert np.array_equal(a["q"], b["q_row"]) and np.array_equal(a["sf"], b["sf_row"])
+
+
+def _if4_candidates(orc, x):
+    """Dequantized scaled-domain values of both candidates per element."""
+    fp = orc.quantize_if4(x, allow_int4=False)
+    both = orc.quantize_if4(x, allow_int4=True)
+    return fp, both
+
+
+def test_if4_keeps_the_smaller_error(orc):
+    """IF4 explainer, section 2: per block keep whichever of FP4 / INT4 has the
+    smaller MSE; the sign bit of the E4M3 scale flags INT4 (6/7 method).
+    Errors here are recomputed in float64 from the dequantized outputs."""
+    x = bf16_bits(workloads.if4_blocks(seed=16, rows=64, cols=512))
+    rows, cols = x.shape
+    xf = orc.bf16_bits_to_f32(x).astype(np.float64)
+    fp, ifq = _if4_candidates(orc, x)
+    s_dec = float(ifq["s_dec"][0])
+    flags = (ifq["sf"].reshape(rows, -1) & 0x80) != 0
+    assert 0.05 < flags.mean() < 0.95          # both formats get used on this mix
+    y_if = orc.dequantize(orc.FMT_IF4, ifq["q"], ifq["sf"], rows, cols, s_dec=s_dec)
+    y_fp = orc.dequantize(orc.FMT_NVFP4, fp["q"], fp["sf"], rows, cols, s_dec=s_dec)
+    # force-INT4 reconstruction of every block: k = nearest integer of v*7/6
+    S = np.repeat(np.vectorize(orc.e4m3_value)(fp["sf"].reshape(rows, -1) & 0x7F), 16, axis=1)
+    scale = S * s_dec
+    v = xf / scale
+    k = np.clip(np.rint(v * 7.0 / 6.0), -7, 7)
+    y_int = k * (6.0 / 7.0) * scale
+    e_if = ((xf - y_if) ** 2).reshape(rows, -1, 16).sum(-1)
+    e_fp = ((xf - y_fp) ** 2).reshape(rows, -1, 16).sum(-1)
+    e_int = ((xf - y_int) ** 2).reshape(rows, -1, 16).sum(-1)
+    assert np.all(e_if <= e_fp * (1 + 1e-5) + 1e-30)
+    clear = np.abs(e_int - e_fp) > 1e-3 * np.maximum(e_int, e_fp)
+    assert np.array_equal(flags[clear], (e_int < e_fp)[clear])
+    # INT4 blocks: codes are k in two's complement, |k| <= 7
+    codes = unpack(ifq["q"]).astype(np.int64)
+    kk = np.where(codes >= 8, codes - 16, codes)
+    blk = np.repeat(flags, 16, axis=1)
+    assert np.all(np.abs(kk[blk]) <= 7)
+    near = np.abs(np.abs(v * 7 / 6 - np.rint(v * 7 / 6)) - 0.5) > 1e-4
+    assert np.array_equal(kk[blk & near], k[blk & near].astype(np.int64))
+
+
+def test_if4_gaussian_mse_ratio(orc):
+    """IF4 explainer, Table 1: on normal data IF4 lowers the quantization MSE
+    from 9.0 (NVFP4) to 6.2 in the paper's units; only the ratio is checked,
+    loosely, because the setting is not stated."""
+    x = bf16_bits(torch.randn(256, 1024, generator=torch.Generator().manual_seed(17)))
+    xf = orc.bf16_bits_to_f32(x).astype(np.float64)
+    fp, ifq = _if4_candidates(orc, x)
+    s = float(ifq["s_dec"][0])
+    y_if = orc.dequantize(orc.FMT_IF4, ifq["q"], ifq["sf"], 256, 1024, s_dec=s)
+    y_fp = orc.dequantize(orc.FMT_NVFP4, fp["q"], fp["sf"], 256, 1024, s_dec=s)
+    ratio = ((xf - y_if) ** 2).mean() / ((xf - y_fp) ** 2).mean()
+    assert 0.5 < ratio < 0.9, ratio          # 6.2 / 9.0 = 0.69
+
+
+# ---------------------------------------------------------------- dequant
+
+def test_dequant_single_rounding(orc):
+    """y = RN(RN(g*S)*s_dec) with g*S exact equals one rounding of g*S*s_dec."""
+    rng = np.random.default_rng(18)
+    rows, cols = 8, 64
+    q = rng.integers(0, 256, (rows, cols // 2)).astype(np.uint8)
+    sf = rng.integers(0, 0x7F, rows * cols // 16).astype(np.uint8)
+    s_dec = float(np.float32(rng.uniform(1e-4, 10)))
+    y = orc.dequantize(orc.FMT_NVFP4, q, sf, rows, cols, s_dec=s_dec)
+    S = np.repeat(np.vectorize(orc.e4m3_value)(sf).reshape(rows, -1), 16, axis=1).astype(np.float64)
+    want = (code_values(unpack(q)) * S * np.float64(np.float32(s_dec))).astype(np.float32)
+    assert np.array_equal(y, want)
+    yb = orc.dequantize(orc.FMT_NVFP4, q, sf, rows, cols, s_dec=s_dec, out_dtype=orc.BF16)
+    assert np.array_equal(yb, bf16_bits(torch.from_numpy(want)))
