@@ -1,0 +1,555 @@
+#!/usr/bin/env python3
+"""Benchmark: block-scaled FP4 quantization throughput on B200.
+
+Metric: GB/s = (algorithmic bytes in + out) / kernel time, and % of the
+measured HBM copy bandwidth.  One "step" is one pass of the whole hot path
+over the benchmark workloads (each kernel with the tensor amax already on the
+device, as with delayed scaling or a fused producer):
+
+  activation 8192x4096 BF16   NVFP4 1x16 row + col from one read
+  activation 8192x4096 BF16   MXFP4 1x32 row + col
+  weight    14336x4096 FP32   NVFP4 16x16 2D, W and W^T codes
+  gradient   8192x5120 BF16   RHT-16 / RHT-128 + NVFP4 of dY^T, SR and RNE
+  if4       16384x8192 BF16   IF4 quantize, and IF4 -> BF16 dequantize
+
+Each kernel is timed with CUDA events on the launching stream; the L2 is
+flushed (256 MiB write) before every kernel, outside the timed events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs the suite on its own tensors (the work
+shards into independent tensors; no collective on the data path), the step
+time is the max over ranks and ``value`` is all ranks' bytes over that time.
+``--impl reference`` times the CPU oracle on a bounded sample instead (rank 0
+only).  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "quantize throughput GB/s (bytes in+out) and % of B200 HBM peak per config"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# jobs: one kernel launch each, with its algorithmic byte count
+# ---------------------------------------------------------------------------
+
+class Job:
+    def __init__(self, name, src, bytes_moved, launches, run, e2e=None, oracle=None):
+        self.name = name            # workload / variant
+        self.src = src              # CUDA source file of the kernel
+        self.bytes = bytes_moved    # algorithmic bytes (input once + outputs)
+        self.launches = launches    # our kernels per call
+        self.run = run              # device call (inputs resident)
+        self.e2e = e2e              # host-buffer call: returns (h2d_bytes, d2h_bytes)
+        self.oracle = oracle        # CPU oracle on a row fraction: returns bytes done
+
+
+def build_jobs(device, fq, inputs):
+    """The benchmark suite on `device`.  Inputs and outputs are allocated once."""
+    import torch
+
+    jobs = []
+    SW = fq.SCALE_SWIZZLED
+
+    def pinned_like(t):
+        return torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+
+    def to_host(outs, hosts):
+        n = 0
+        for k, v in outs.items():
+            hosts[k].copy_(v, non_blocking=True)
+            n += v.numel() * v.element_size()
+        return n
+
+    # ---- activation: NVFP4 row + col, MXFP4 row + col -------------------
+    xa_cpu = inputs["activation"]
+    xa = xa_cpu.to(device)
+    amax_a = fq.fp4q_amax(xa)
+    out_nv = fq.fp4q_quantize_nvfp4(xa, layouts=3, amax=amax_a, scale_layout=SW)
+    out_mx = fq.fp4q_quantize_mxfp4(xa, layouts=3, scale_layout=SW)
+    R, C = xa.shape
+    nb_nv = R * C * 2 + 2 * (R * C // 2) + 2 * (R * C // 16) + 4
+    nb_mx = R * C * 2 + 2 * (R * C // 2) + 2 * (R * C // 32)
+    xa_h = pinned_like(xa_cpu).copy_(xa_cpu)
+    hn = {k: pinned_like(v.cpu()) for k, v in out_nv.items()}
+    hm = {k: pinned_like(v.cpu()) for k, v in out_mx.items()}
+
+    def e2e_nv():
+        x = xa_h.to(device, non_blocking=True)
+        o = fq.fp4q_quantize_nvfp4(x, layouts=3, scale_layout=SW, out=out_nv)
+        return xa_h.numel() * 2, to_host(o, hn)
+
+    def e2e_mx():
+        x = xa_h.to(device, non_blocking=True)
+        o = fq.fp4q_quantize_mxfp4(x, layouts=3, scale_layout=SW, out=out_mx)
+        return xa_h.numel() * 2, to_host(o, hm)
+
+    jobs.append(Job("activation 8192x4096 bf16 nvfp4 row+col", "nvfp4.cu", nb_nv, 1,
+                    lambda: fq.fp4q_quantize_nvfp4(xa, layouts=3, amax=amax_a, scale_layout=SW,
+                                                   out=out_nv), e2e_nv))
+    jobs.append(Job("activation 8192x4096 bf16 mxfp4 row+col", "nvfp4.cu", nb_mx, 1,
+                    lambda: fq.fp4q_quantize_mxfp4(xa, layouts=3, scale_layout=SW, out=out_mx),
+                    e2e_mx))
+
+    # ---- weight: 2D 16x16 ------------------------------------------------
+    w_cpu = inputs["weight"]
+    w = w_cpu.to(device)
+    amax_w = fq.fp4q_amax(w)
+    out_w = fq.fp4q_quantize_2d(w, amax=amax_w)
+    R, C = w.shape
+    nb_w = R * C * 4 + 2 * (R * C // 2) + (R // 16) * (C // 16) + 4
+    w_h = pinned_like(w_cpu).copy_(w_cpu)
+    hw = {k: pinned_like(v.cpu()) for k, v in out_w.items()}
+
+    def e2e_w():
+        x = w_h.to(device, non_blocking=True)
+        o = fq.fp4q_quantize_2d(x, out=out_w)
+        return w_h.numel() * 4, to_host(o, hw)
+
+    jobs.append(Job("weight 14336x4096 fp32 2d16x16 w+wt", "quant2d.cu", nb_w, 1,
+                    lambda: fq.fp4q_quantize_2d(w, amax=amax_w, out=out_w), e2e_w))
+
+    # ---- gradient: RHT + NVFP4 of dY^T ----------------------------------
+    g_cpu = inputs["gradient"]
+    g = g_cpu.to(device)
+    T, C = g.shape
+    nb_g = T * C * 2 + (T * C // 2) + (T * C // 16) + 4
+    g_h = pinned_like(g_cpu).copy_(g_cpu)
+    for n in (16, 128):
+        amax_g = fq.fp4q_rht_amax(g, n, seed=0)
+        for rnd, rname in ((fq.SR, "sr"), (fq.RNE, "rne")):
+            out_g = fq.fp4q_quantize_rht_sr(g, n, round=rnd, seed=0, amax_rht=amax_g,
+                                            scale_layout=SW)
+            hg = {k: pinned_like(v.cpu()) for k, v in out_g.items()}
+
+            def e2e_g(n=n, rnd=rnd, out_g=out_g, hg=hg):
+                x = g_h.to(device, non_blocking=True)
+                o = fq.fp4q_quantize_rht_sr(x, n, round=rnd, seed=0, scale_layout=SW, out=out_g)
+                return g_h.numel() * 2, to_host(o, hg)
+
+            jobs.append(Job(f"gradient 8192x5120 bf16 rht{n}+{rname}", "rht.cu", nb_g, 1,
+                            lambda n=n, rnd=rnd, a=amax_g, o=out_g: fq.fp4q_quantize_rht_sr(
+                                g, n, round=rnd, seed=0, amax_rht=a, scale_layout=SW, out=o),
+                            e2e_g))
+
+    # ---- IF4: quantize and dequantize -----------------------------------
+    x5_cpu = inputs["if4"]
+    x5 = x5_cpu.to(device)
+    amax5 = fq.fp4q_amax(x5)
+    out5 = fq.fp4q_quantize_if4(x5, amax=amax5, scale_layout=SW)
+    R, C = x5.shape
+    nb_q5 = R * C * 2 + R * C // 2 + R * C // 16 + 4
+    # the dequant reads its own copy of the codes so it never sees them in L2
+    q5 = out5["q"].clone()
+    sf5 = out5["sf"].clone()
+    s5 = out5["s_dec"].clone()
+    y5 = torch.empty((R, C), dtype=torch.bfloat16, device=device)
+    nb_d5 = R * C // 2 + R * C // 16 + 4 + R * C * 2
+    x5_h = pinned_like(x5_cpu).copy_(x5_cpu)
+    h5 = {k: pinned_like(v.cpu()) for k, v in out5.items()}
+    q5_h, sf5_h, s5_h = q5.cpu().pin_memory(), sf5.cpu().pin_memory(), s5.cpu().pin_memory()
+    y5_h = torch.empty((R, C), dtype=torch.bfloat16, pin_memory=True)
+
+    def e2e_q5():
+        x = x5_h.to(device, non_blocking=True)
+        o = fq.fp4q_quantize_if4(x, scale_layout=SW, out=out5)
+        return x5_h.numel() * 2, to_host(o, h5)
+
+    def e2e_d5():
+        q = q5_h.to(device, non_blocking=True)
+        sf = sf5_h.to(device, non_blocking=True)
+        s = s5_h.to(device, non_blocking=True)
+        fq.fp4q_dequantize(fq.FMT_IF4, q, sf, R, C, tensor_scale=s, scale_layout=SW, out=y5)
+        y5_h.copy_(y5, non_blocking=True)
+        return q5_h.numel() + sf5_h.numel() + 4, y5_h.numel() * 2
+
+    jobs.append(Job("if4 16384x8192 bf16 quantize", "if4.cu", nb_q5, 1,
+                    lambda: fq.fp4q_quantize_if4(x5, amax=amax5, scale_layout=SW, out=out5),
+                    e2e_q5))
+    jobs.append(Job("if4 16384x8192 dequantize to bf16", "dequant.cu", nb_d5, 1,
+                    lambda: fq.fp4q_dequantize(fq.FMT_IF4, q5, sf5, R, C, tensor_scale=s5,
+                                               scale_layout=SW, out=y5), e2e_d5))
+    torch.cuda.synchronize(device)
+    return jobs
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, read only)
+# ---------------------------------------------------------------------------
+
+_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _handle(self, idx):
+        import torch
+        nv = self._nv
+        try:
+            p = torch.cuda.get_device_properties(idx)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                try:
+                    return nv.nvmlDeviceGetHandleByIndex(int(vis.split(",")[idx]))
+                except Exception:
+                    pass
+            return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        nv = self._nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = get_r(self._h)
+                for bit, name in _REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.005)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle on a bounded sample (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+
+def suite_inputs():
+    """CPU copies of the suite's inputs (activation, weight, gradient, if4)."""
+    from fp4_block_scaled_04_b200 import workloads
+    return {"activation": workloads.activation(), "weight": workloads.weight(),
+            "gradient": workloads.gradient(), "if4": workloads.if4_blocks()}
+
+
+def oracle_sample(rows_fraction: float, inputs=None):
+    """Run the oracle over the first rows_fraction of every workload of the
+    suite; returns (algorithmic bytes of the sample, seconds, description)."""
+    import numpy as np
+    import torch
+    import oracle as orc
+
+    def bits(t):
+        t = t.contiguous()
+        if t.dtype == torch.bfloat16:
+            return t.view(torch.int16).numpy().view(np.uint16)
+        return t.numpy()
+
+    def rows_of(n, align):
+        return max(align, int(n * rows_fraction) // align * align)
+
+    inputs = inputs or suite_inputs()
+    xa, w, g, x5 = inputs["activation"], inputs["weight"], inputs["gradient"], inputs["if4"]
+    total_b, total_s = 0, 0.0
+    ra = rows_of(xa.shape[0], 32)
+    a = np.ascontiguousarray(bits(xa[:ra]))
+    C = xa.shape[1]
+    t0 = time.perf_counter()
+    orc.quantize_nvfp4(a, layouts=3, scale_layout=orc.SCALE_SWIZZLED if ra % 128 == 0 else 0)
+    orc.quantize_mxfp4(a, layouts=3)
+    total_s += time.perf_counter() - t0
+    total_b += ra * C * 2 + 2 * (ra * C // 2) + 2 * (ra * C // 16) + 4
+    total_b += ra * C * 2 + 2 * (ra * C // 2) + 2 * (ra * C // 32)
+    rw = rows_of(w.shape[0], 16)
+    ww = np.ascontiguousarray(bits(w[:rw]))
+    C = w.shape[1]
+    t0 = time.perf_counter()
+    orc.quantize_2d(ww)
+    total_s += time.perf_counter() - t0
+    total_b += rw * C * 4 + 2 * (rw * C // 2) + (rw // 16) * (C // 16) + 4
+    rg = rows_of(g.shape[0], 128)
+    gg = np.ascontiguousarray(bits(g[:rg]))
+    C = g.shape[1]
+    t0 = time.perf_counter()
+    for n in (16, 128):
+        for rnd in (orc.SR, orc.RNE):
+            orc.quantize_rht(gg, n, round=rnd, seed=0)
+    total_s += time.perf_counter() - t0
+    total_b += 4 * (rg * C * 2 + rg * C // 2 + rg * C // 16 + 4)
+    r5 = rows_of(x5.shape[0], 16)
+    xx = np.ascontiguousarray(bits(x5[:r5]))
+    C = x5.shape[1]
+    t0 = time.perf_counter()
+    o = orc.quantize_if4(xx)
+    orc.dequantize(orc.FMT_IF4, o["q"], o["sf"], r5, C, s_dec=float(o["s_dec"][0]),
+                   out_dtype=orc.BF16)
+    total_s += time.perf_counter() - t0
+    total_b += 2 * (r5 * C * 2 + r5 * C // 2 + r5 * C // 16 + 4)
+    desc = (f"oracle (plain C, 1 thread) on the first {rows_fraction:.4g} of the rows of every "
+            f"workload of the suite: activation {ra} rows, weight {rw}, gradient {rg}, "
+            f"if4 {r5}")
+    return total_b, total_s, desc
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def traffic_for(job_src: str, job_name: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel's
+    source is unchanged since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path))[job_name]
+    except Exception:
+        return None
+    src = os.path.join(ROOT, "fp4_block_scaled_04_b200", "csrc", job_src)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["dram_bytes_per_launch"] if rec.get("src_sha256_16") == h else None
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    frac = args.reference_fraction
+    times, nbytes, desc = [], 0, ""
+    inputs = suite_inputs()
+    for i in range(args.warmup + args.steps):
+        b, s, desc = oracle_sample(frac, inputs)
+        if i >= args.warmup:
+            times.append(s)
+            nbytes = b
+    total = sum(times)
+    value = nbytes * len(times) / total / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / len(times), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": "fp4 quantization suite (bounded row sample per step)",
+                   "rows_fraction": frac, "l2": "n/a (CPU)", "parallelism": "rank 0 only"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--reference-fraction", type=float, default=1.0 / 32)
+    ap.add_argument("--cpu-baseline-fraction", type=float, default=1.0 / 8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    import fp4_block_scaled_04_b200 as fq
+
+    ws, rank, local = dist_env()
+    if ws != args.gpus and ws > 1:
+        print(f"warning: WORLD_SIZE={ws} but --gpus {args.gpus}", file=sys.stderr)
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    fq.lib()
+    inputs = suite_inputs()
+    jobs = build_jobs(device, fq, inputs)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(record):
+        for j, job in enumerate(jobs):
+            flush.fill_(float(j))
+            if record is not None:
+                record[j][0].record(stream)
+            job.run()
+            if record is not None:
+                record[j][1].record(stream)
+
+    for _ in range(args.warmup):
+        step(None)
+    torch.cuda.synchronize(device)
+
+    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+               for _ in jobs] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(device)
+    wall0 = time.perf_counter()
+    with ClockSampler(local) as clocks:
+        for s in range(args.steps):
+            step(events[s])
+        torch.cuda.synchronize(device)
+    barrier()
+    wall = time.perf_counter() - wall0
+    per_job_ms = [sum(events[s][j][0].elapsed_time(events[s][j][1]) for s in range(args.steps))
+                  for j in range(len(jobs))]
+    total_ms = sum(per_job_ms)
+    if ws > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms_max = float(t.item())
+    else:
+        total_ms_max = total_ms
+
+    step_bytes = sum(j.bytes for j in jobs)
+    value = ws * step_bytes * args.steps / (total_ms_max * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+
+    per_config = []
+    for job, ms in zip(jobs, per_job_ms):
+        avg_s = ms * 1e-3 / args.steps
+        gbs = job.bytes / avg_s / 1e9
+        per_config.append({"workload": job.name, "bytes": job.bytes,
+                           "us": round(avg_s * 1e6, 2), "GB/s": round(gbs, 1),
+                           "pct_of_peak": round(100 * gbs / peak, 1),
+                           "share": round(ms / total_ms, 4)})
+    dom = max(range(len(jobs)), key=lambda j: per_job_ms[j])
+    dom_avg_s = per_job_ms[dom] * 1e-3 / args.steps
+    dom_achieved = jobs[dom].bytes / dom_avg_s / 1e9
+    roofline = {"bound": "hbm", "achieved": round(dom_achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(dom_achieved / peak, 4),
+                "traffic": traffic_for(jobs[dom].src, jobs[dom].name),
+                "kernel": jobs[dom].name, "peak_kind": f"{peak_kind} (HBM copy bandwidth)"}
+
+    # ---- end to end through the public API with host buffers -------------
+    e2e = None
+    if not args.no_e2e:
+        k = args.e2e_steps or max(1, min(args.steps, 10))
+        for job in jobs:
+            job.e2e()
+        torch.cuda.synchronize(device)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        h2d = d2h = 0
+        e0.record(stream)
+        for _ in range(k):
+            h2d = d2h = 0
+            for job in jobs:
+                a, b = job.e2e()
+                h2d += a
+                d2h += b
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = e0.elapsed_time(e1)
+        if ws > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": round(ws * step_bytes * k / (e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k,
+               "path": "pinned host -> device copy, C-ABI call (tensor amax computed inside), "
+                       "device -> pinned host copy of every output"}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        b, s, desc = oracle_sample(args.cpu_baseline_fraction, inputs)
+        cpu = {"value": round(b / s / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": desc, "seconds": round(s, 2)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "fp4 quantization suite: activation 8192x4096 nvfp4 row+col "
+                                   "and mxfp4 row+col; weight 14336x4096 fp32 2d16x16; gradient "
+                                   "8192x5120 rht16/rht128 x sr/rne; if4 16384x8192 quant + "
+                                   "bf16 dequant",
+                       "l2": "flushed before every kernel (256 MiB write, untimed)",
+                       "amax": "precomputed on the device (headline); e2e computes it",
+                       "parallelism": f"replicas x{ws}" if ws > 1 else "single gpu"},
+            "pct_of_peak": round(100 * value / (ws * peak), 2),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": sum(j.launches for j in jobs) * args.steps,
+            "clocks": clocks.summary(), "wall_s_timed_region": round(wall, 4),
+            "per_config": per_config,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,275 @@
+// common.cuh -- device helpers shared by the fp4q kernels (sm_100a only).
+//
+// Every floating-point step that decides a code uses an explicitly rounded
+// intrinsic (__fmul_rn, __fadd_rn, __fdiv_rn, __fmaf_rn) or a hand-written
+// PTX conversion, and the translation units are compiled with -fmad=false
+// -ftz=false -prec-div=true, so the result is the same binary32 value the
+// library documents in include/fp4q.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "fp4q.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "fp4q kernels target sm_100a only"
+#endif
+
+namespace fp4q {
+
+constexpr float kNvfp4Max = 2688.0f;   // 6 (E2M1 max) * 448 (E4M3 max)
+
+// ---------------------------------------------------------------------------
+// element loads
+// ---------------------------------------------------------------------------
+
+// BF16 pair packed in a 32-bit word: the low half is the lower address.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Load 8 consecutive elements starting at p (16-byte aligned for BF16, 32 for FP32).
+template <typename T> struct Vec8;
+template <> struct Vec8<__nv_bfloat16> {
+  __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&v)[8]) {
+    uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+    v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+    v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
+  }
+};
+template <> struct Vec8<float> {
+  __device__ __forceinline__ static void load(const float *p, float (&v)[8]) {
+    float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+    float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+
+__device__ __forceinline__ float to_f32(__nv_bfloat16 h) { return __bfloat162float(h); }
+__device__ __forceinline__ float to_f32(float f) { return f; }
+
+// ---------------------------------------------------------------------------
+// E2M1 encode / decode
+// ---------------------------------------------------------------------------
+
+// Round two floats to E2M1 (nearest, ties to even, saturating at +-6, sign
+// kept) with the sm_100a conversion instruction; `lo` lands in bits 0..3.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+      "cvt.u16.u8 %0, t;\n\t}"
+      : "=h"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+// Eight floats -> eight nibbles in one word, v[0] in bits 0..3.
+__device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+        "f"(v[7]));
+  return r;
+}
+
+// E2M1 magnitude of a 3-bit code: 0, .5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ float e2m1_magnitude(uint32_t c3) {
+  // codes 2..7 are normal: exponent (c3 >> 1) - 1, one mantissa bit (c3 & 1)
+  uint32_t normal = ((((c3 >> 1) + 126u) << 23) | ((c3 & 1u) << 22));
+  float v = __uint_as_float(normal);
+  return c3 >= 2 ? v : (c3 == 1 ? 0.5f : 0.0f);
+}
+
+__device__ __forceinline__ float e2m1_value(uint32_t code) {
+  float m = e2m1_magnitude(code & 7u);
+  return (code & 8u) ? -m : m;
+}
+
+// ---------------------------------------------------------------------------
+// E4M3 encode / decode (block scales)
+// ---------------------------------------------------------------------------
+
+// s >= 0 -> E4M3 code, round to nearest even, saturating at 448 (0x7E).
+__device__ __forceinline__ uint32_t e4m3_code(float s) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(s));
+  return r & 0xFFu;
+}
+
+// Value of a 7-bit E4M3 magnitude code (sign bit ignored).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  uint32_t e = (code >> 3) & 15u, m = code & 7u;
+  if (e == 0) return __fmul_rn(static_cast<float>(m), 0.001953125f);  // m * 2^-9
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4 tensor and block scales
+// ---------------------------------------------------------------------------
+
+struct TensorScale {
+  float enc;  // RN(2688 / amax), clamped to FLT_MAX; 1 if amax == 0
+  float dec;  // RN(amax / 2688); 1 if amax == 0
+};
+
+__device__ __forceinline__ TensorScale tensor_scale(float amax) {
+  TensorScale t;
+  if (amax == 0.0f) {
+    t.enc = 1.0f;
+    t.dec = 1.0f;
+  } else {
+    t.enc = fminf(__fdiv_rn(kNvfp4Max, amax), 3.402823466e+38f);
+    t.dec = __fdiv_rn(amax, kNvfp4Max);
+  }
+  return t;
+}
+
+// E4M3 code of the block scale: RN(RN(m * s_enc) / 6).
+__device__ __forceinline__ uint32_t nvfp4_scale_code(float block_amax, float s_enc) {
+  return e4m3_code(__fdiv_rn(__fmul_rn(block_amax, s_enc), 6.0f));
+}
+
+// Per-CTA table of r = RN(s_enc / S) for the 128 non-negative E4M3 codes
+// (0 for S == 0); one IEEE division per code instead of one per block.
+__device__ __forceinline__ void fill_factor_table(float *tab, float s_enc) {
+  for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+    float S = e4m3_value(static_cast<uint32_t>(c));
+    tab[c] = (S == 0.0f) ? 0.0f : __fdiv_rn(s_enc, S);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// E8M0 shared exponent (MXFP4)
+// ---------------------------------------------------------------------------
+
+// Unbiased exponent e in [-127, 127] of the power-of-two scale of a block
+// whose maximum magnitude is m.  Modes as in fp4q_e8m0_mode.
+__device__ __forceinline__ int e8m0_exponent(float m, int mode) {
+  if (!(m > 0.0f)) return -127;
+  int e;
+  if (mode == FP4Q_E8M0_OCP_FLOOR) {
+    uint32_t b = __float_as_uint(m);
+    int E = static_cast<int>(b >> 23) - 127;
+    if ((b >> 23) == 0) E = -127 - (__clz(static_cast<int>(b)) - 9);  // subnormal
+    e = E - 2;
+  } else {
+    float t = __fdiv_rn(m, 6.0f);
+    if (!(t > 0.0f)) return -127;
+    uint32_t b = __float_as_uint(t);
+    int E;
+    uint32_t frac;  // fraction bits below the leading one, left-aligned to 23 bits
+    if ((b >> 23) != 0) {
+      E = static_cast<int>(b >> 23) - 127;
+      frac = b & 0x7FFFFFu;
+    } else {  // subnormal: b = mant * 2^-149, leading one at bit p
+      int p = 31 - __clz(static_cast<int>(b));
+      E = p - 149;
+      frac = (b << (23 - p)) & 0x7FFFFFu;
+    }
+    if (mode == FP4Q_E8M0_CEIL) {
+      e = (frac != 0) ? E + 1 : E;
+    } else {  // nearest power of two; midpoint 1.5 * 2^E -> even biased exponent
+      if (frac > 0x400000u) e = E + 1;
+      else if (frac < 0x400000u) e = E;
+      else e = (((E + 127) & 1) == 0) ? E : E + 1;
+    }
+  }
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// 2^-e as a float, e in [-127, 127] (2^-127 is subnormal, the rest normal).
+__device__ __forceinline__ float exp2_neg(int e) {
+  int k = -e;
+  if (k >= -126) return __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+  return __uint_as_float(0x00400000u);  // 2^-127
+}
+
+// 2^e as a float for a stored E8M0 byte (e = byte - 127, e <= 127).
+__device__ __forceinline__ float e8m0_value(uint32_t byte) {
+  if (byte == 0) return __uint_as_float(0x00400000u);
+  return __uint_as_float(byte << 23);
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., SC'11) and stochastic rounding
+// ---------------------------------------------------------------------------
+
+struct U32x4 { uint32_t x, y, z, w; };
+
+__device__ __forceinline__ U32x4 philox4x32_10(U32x4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+    uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+    U32x4 n = {hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0};
+    c = n;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+
+// 16 random bits for elements 8g .. 8g+7 (flat input index) of a seed.
+__device__ __forceinline__ U32x4 sr_bits_group(uint64_t seed, uint64_t g) {
+  U32x4 c = {static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u};
+  return philox4x32_10(c, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+}
+
+__device__ __forceinline__ uint32_t half16(const U32x4 &w, int j) {
+  uint32_t word = (j >> 1) == 0 ? w.x : (j >> 1) == 1 ? w.y : (j >> 1) == 2 ? w.z : w.w;
+  return (j & 1) ? (word >> 16) : (word & 0xFFFFu);
+}
+
+// Stochastic rounding of v onto E2M1: between adjacent magnitudes
+// lo <= |v| < hi round up iff u < (|v| - lo) / (hi - lo) * 2^16; |v| >= 6 -> 6;
+// the sign is copied.  Returns the 4-bit code.
+__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t u16) {
+  float a = fabsf(v);
+  uint32_t sign = (__float_as_uint(v) >> 28) & 8u;
+  uint32_t code;
+  if (a >= 6.0f) {
+    code = 7u;
+  } else {
+    // lower neighbour: codes 0..7 at 0, .5, 1, 1.5, 2, 3, 4, 6
+    uint32_t lo = (a >= 0.5f) + (a >= 1.0f) + (a >= 1.5f) + (a >= 2.0f) + (a >= 3.0f) +
+                  (a >= 4.0f);
+    float lo_v = e2m1_magnitude(lo);
+    // spacing to the next value: .5 below 2, 1 in [2, 4), 2 in [4, 6)
+    float inv_gap_2p16 = lo >= 6 ? 32768.0f : (lo >= 4 ? 65536.0f : 131072.0f);
+    float t16 = __fmul_rn(__fsub_rn(a, lo_v), inv_gap_2p16);  // exact
+    code = lo + (static_cast<float>(u16) < t16 ? 1u : 0u);
+  }
+  return code | sign;
+}
+
+// ---------------------------------------------------------------------------
+// scale-factor layouts
+// ---------------------------------------------------------------------------
+
+// Byte offset of scale (r, c) in an [rows, cols] scale matrix.
+__device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t c, int64_t cols,
+                                                int layout) {
+  if (layout == FP4Q_SCALE_LINEAR) return r * cols + c;
+  int64_t tile = (r >> 7) * (cols >> 2) + (c >> 2);
+  return tile * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+// ---------------------------------------------------------------------------
+// misc
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+}  // namespace fp4q

@@ -1,0 +1,50 @@
+// launch.h -- internal host-side launchers (one per kernel family).  The
+// extern "C" entry points in api.cu validate arguments and call these.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp4q {
+
+struct Launch {
+  cudaStream_t stream;
+  int num_sms;
+};
+
+cudaError_t launch_amax(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                        float *amax_out, const Launch &L);
+
+cudaError_t launch_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                         unsigned layouts, int round, uint64_t seed, const float *amax,
+                         float *s_dec_out, uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col,
+                         uint8_t *sf_col, int scale_layout, const Launch &L);
+
+cudaError_t launch_mxfp4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                         unsigned layouts, int e8m0_mode, uint8_t *q_row, uint8_t *sf_row,
+                         uint8_t *q_col, uint8_t *sf_col, int scale_layout, const Launch &L);
+
+cudaError_t launch_2d(const void *w, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                      const float *amax, float *s_dec_out, uint8_t *q_w, uint8_t *q_wt,
+                      uint8_t *sf_tiles, uint8_t *sf_w_1x16, uint8_t *sf_wt_1x16,
+                      int scale_layout, const Launch &L);
+
+cudaError_t launch_rht_amax(const void *dy, int dtype, int64_t tokens, int64_t cols,
+                            int64_t ld, int n, uint64_t seed, float *amax_out,
+                            const Launch &L);
+
+cudaError_t launch_rht_quant(const void *dy, int dtype, int64_t tokens, int64_t cols,
+                             int64_t ld, int n, int round, uint64_t seed, const float *amax,
+                             float *s_dec_out, uint8_t *q_t, uint8_t *sf_t, int scale_layout,
+                             float *rht_out, const Launch &L);
+
+cudaError_t launch_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                       const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,
+                       int scale_layout, const Launch &L);
+
+cudaError_t launch_dequant(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,
+                           int block_rows, int block_cols, const float *s_dec, int64_t rows,
+                           int64_t cols, void *y, int y_dtype, const Launch &L);
+
+}  // namespace fp4q

@@ -1,0 +1,227 @@
+/*
+ * fp4q.h -- C ABI of the block-scaled FP4 quantization library (libfp4q.so).
+ *
+ * What is computed.  Each entry point quantizes (or dequantizes) one tensor
+ * into a block-scaled 4-bit format, bit for bit as the CPU oracle in this
+ * repository defines it:
+ *
+ *   NVFP4  E2M1 codes (magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 plus a sign bit),
+ *          one E4M3 scale per 16 values and one FP32 scale per tensor.
+ *          Qiita note on the NVFP4 pre-training paper (nishiha): "NVFP4データ
+ *          の変換" (E2M1), "Blockwise" (16 values per 8-bit scale), "scaleの
+ *          導出" (global_scale = 6*448/amax, local scale = block max / 6 as
+ *          E4M3), "NVFP4の表現できる最大値" (2688 = 6 * 448).
+ *   MXFP4  E2M1 codes, one E8M0 power-of-two scale per 32 values, no tensor
+ *          scale.  Ultralytics glossary "FP4", section "FP4の仕組み".
+ *   2D     NVFP4 with one scale per 16x16 tile, so q(W) = q(W^T)^T.
+ *          Qiita note, section "2D scaling".
+ *   RHT    random Hadamard transform H diag(S) along tokens ahead of the
+ *          Wgrad operand, with stochastic rounding.  Qiita note, sections
+ *          "ランダムアダマール変換" and "確率的丸め".
+ *   IF4    per 16-value block, FP4 or INT4 (6/7 method), whichever has the
+ *          smaller squared error, flagged in bit 7 of the E4M3 scale.
+ *          "Adaptive Block-Scaled Data Types" explainer, section 2 (IF4).
+ *
+ * Arithmetic, per 16-value NVFP4 block (all binary32, RN = round to nearest
+ * even, no fused operations):
+ *   amax = max |x| over the tensor;  s_enc = RN(2688 / amax) (1 if amax = 0),
+ *   s_dec = RN(amax / 2688) (1 if amax = 0);
+ *   block scale S = E4M3_rne_sat(RN(RN(m * s_enc) / 6)), m = block max |x|;
+ *   r = RN(s_enc / S) (0 if S = 0);  v = RN(x * r);  code = E2M1_rne_sat(v)
+ *   (or stochastic rounding); dequant y = RN(RN(E2M1(code) * S) * s_dec).
+ *
+ * Conventions (all entry points):
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless
+ *     stated otherwise.  The library allocates nothing and keeps no state
+ *     between calls.  Inputs, outputs and workspace of one call must be on
+ *     the same device; the call runs on that device.
+ *   - Matrices are row-major.  `ld` is the input's leading dimension in
+ *     elements (ld >= cols); ld * element size must be a multiple of 16 bytes
+ *     and every pointer must be 16-byte aligned.
+ *   - Packed codes: two 4-bit codes per byte, element 2j in the low nibble.
+ *     Row-wise output of a [rows, cols] input: codes [rows, cols/2], scales
+ *     [rows, cols/block].  Column-wise ("transposed") output: codes
+ *     [cols, rows/2], scales [cols, rows/block] -- i.e. the row-wise layout
+ *     of the transpose.
+ *   - Scale layout FP4Q_SCALE_LINEAR stores scales row-major.
+ *     FP4Q_SCALE_SWIZZLED_128x4 stores them in the 128 x 4 tile layout that
+ *     block-scaled tensor-core GEMMs read: byte (r, c) of an [R, C] scale
+ *     matrix lives at ((r/128)*(C/4) + c/4)*512 + (r%32)*16 + ((r/32)%4)*4
+ *     + c%4.  It requires R % 128 == 0 and C % 4 == 0.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and is asynchronous.  Argument errors are detected on
+ *     the host and returned before anything is enqueued.  A failed launch
+ *     returns FP4Q_ERR_CUDA.  No call traps on the device.
+ *   - Inputs must be finite; a NaN or Inf input makes the tensor amax
+ *     non-finite and the outputs unspecified.
+ */
+#ifndef FP4Q_H_
+#define FP4Q_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP4Q_OK = 0,
+  FP4Q_ERR_INVALID_ARG = 1,        /* null pointer, bad enum, host pointer, ld < cols */
+  FP4Q_ERR_UNSUPPORTED_SHAPE = 2,  /* shape not a multiple of the block / tile size */
+  FP4Q_ERR_MISALIGNED = 3,         /* pointer or row stride not 16-byte aligned */
+  FP4Q_ERR_WORKSPACE_TOO_SMALL = 4,
+  FP4Q_ERR_CUDA = 5                /* a CUDA runtime call or launch failed */
+} fp4q_status;
+
+typedef enum { FP4Q_BF16 = 0, FP4Q_FP32 = 1 } fp4q_dtype;
+typedef enum { FP4Q_RNE = 0, FP4Q_SR = 1 } fp4q_round;
+typedef enum { FP4Q_SCALE_LINEAR = 0, FP4Q_SCALE_SWIZZLED_128x4 = 1 } fp4q_scale_layout;
+typedef enum { FP4Q_E8M0_RNE = 0, FP4Q_E8M0_CEIL = 1, FP4Q_E8M0_OCP_FLOOR = 2 } fp4q_e8m0_mode;
+typedef enum { FP4Q_FMT_NVFP4 = 0, FP4Q_FMT_MXFP4 = 1, FP4Q_FMT_IF4 = 2 } fp4q_format;
+
+#define FP4Q_ROWWISE 1u
+#define FP4Q_COLWISE 2u
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *fp4q_status_string(int status);
+
+/* Library version string (static). */
+const char *fp4q_version(void);
+
+/* Bytes of device workspace the quantize calls need when they compute the
+ * tensor amax themselves (amax argument NULL).  Constant. */
+size_t fp4q_workspace_bytes(void);
+
+/* Bytes of a scale matrix for a [rows, cols] tensor quantized in blocks of
+ * `block` values along cols: [rows, cols/block] in the given layout (the
+ * swizzled layout rounds rows up to 128 and cols/block up to 4).  For a
+ * column-wise output pass (cols, rows, block, layout).  Returns 0 on bad
+ * arguments. */
+size_t fp4q_scale_bytes(int64_t rows, int64_t cols, int block, int scale_layout);
+
+/* Tensor amax: *amax_out = max |x| over x[rows, cols] (FP32, exact).
+ * Qiita note, "scaleの導出": max|x| sets the global scale.
+ * amax_out: device float, overwritten.  Shape: cols % 16 == 0. */
+fp4q_status fp4q_amax(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                      float *amax_out, void *stream);
+
+/* NVFP4 1x16 quantization of an activation or gradient, row-wise and/or
+ * column-wise from one read of x.  Qiita note: "Blockwise", "誤差逆伝播と
+ * 転置" (backprop needs the transposed operand), "2D scaling" (activations
+ * and gradients use 1x16), "確率的丸め" (round = FP4Q_SR).
+ *   layouts      FP4Q_ROWWISE | FP4Q_COLWISE (at least one)
+ *   round        FP4Q_RNE, or FP4Q_SR: stochastic rounding whose 16 random
+ *                bits per element come from Philox4x32-10 keyed on `seed`,
+ *                counter = (flat input index r*cols + c) / 8
+ *   amax         device float with the tensor amax, or NULL: then it is
+ *                computed first into `workspace`
+ *   tensor_scale_out  device float <- s_dec (may be NULL)
+ *   q_row, sf_row     row-wise codes [rows, cols/2], scales [rows, cols/16]
+ *   q_col, sf_col     column-wise codes [cols, rows/2], scales [cols, rows/16]
+ *                (pointers of a layout not requested may be NULL)
+ *   workspace, ws_bytes  >= fp4q_workspace_bytes() when amax == NULL
+ * Shape: cols % 16 == 0; COLWISE also needs rows % 16 == 0. */
+fp4q_status fp4q_quantize_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols,
+                                int64_t ld, unsigned layouts, int round, uint64_t seed,
+                                const float *amax, float *tensor_scale_out, uint8_t *q_row,
+                                uint8_t *sf_row, uint8_t *q_col, uint8_t *sf_col,
+                                int scale_layout, void *workspace, size_t ws_bytes,
+                                void *stream);
+
+/* MXFP4 1x32 quantization, row-wise and/or column-wise from one read.
+ * Ultralytics glossary "FP4", "FP4の仕組み": 32 values share an 8-bit
+ * power-of-two (E8M0) scale chosen so the block maximum lands near 6.
+ * e8m0_mode: FP4Q_E8M0_RNE (default reading: RN(m/6) rounded to the nearest
+ * power of two, exact midpoints to the even biased exponent -- the FP6 essay
+ * on blog.ast.moe notes that round-to-nearest-even in the E8M0 conversion
+ * matters), FP4Q_E8M0_CEIL (smallest power of two >= RN(m/6): never clips),
+ * FP4Q_E8M0_OCP_FLOOR (2^(floor(log2 m) - 2), the OCP MX rule).
+ * Elements: v = RN(x * 2^-e), E2M1 round to nearest even with saturation.
+ * Scale byte = e + 127.  Outputs as for NVFP4 with blocks of 32.
+ * Shape: cols % 32 == 0; COLWISE also needs rows % 32 == 0. */
+fp4q_status fp4q_quantize_mxfp4(const void *x, int dtype, int64_t rows, int64_t cols,
+                                int64_t ld, unsigned layouts, int e8m0_mode, uint8_t *q_row,
+                                uint8_t *sf_row, uint8_t *q_col, uint8_t *sf_col,
+                                int scale_layout, void *stream);
+
+/* NVFP4 with 16x16 2D block scaling of a weight (Qiita note, "2D scaling":
+ * square 16x16 tiles make q(W) = q(W^T)^T), emitting W and W^T codes from
+ * the same scales in one pass.
+ *   q_w   [rows, cols/2]   codes of W      (may be NULL)
+ *   q_wt  [cols, rows/2]   codes of W^T    (may be NULL)
+ *   sf_tiles [rows/16, cols/16]  one E4M3 scale per tile, linear (required)
+ *   sf_w_1x16  [rows, cols/16] (nullable)  the tile scale repeated for each
+ *   sf_wt_1x16 [cols, rows/16] (nullable)  1x16 block of W / W^T, in
+ *              scale_layout -- the form a 1x16 block-scaled GEMM reads
+ *   amax, tensor_scale_out, workspace as for fp4q_quantize_nvfp4.
+ * Shape: rows % 16 == 0, cols % 16 == 0. */
+fp4q_status fp4q_quantize_2d(const void *w, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                             const float *amax, float *tensor_scale_out, uint8_t *q_w,
+                             uint8_t *q_wt, uint8_t *sf_tiles, uint8_t *sf_w_1x16,
+                             uint8_t *sf_wt_1x16, int scale_layout, void *workspace,
+                             size_t ws_bytes, void *stream);
+
+/* amax of the random-Hadamard-transformed gradient (see below), the tensor
+ * amax that fp4q_quantize_rht_sr needs.  amax_out: device float, overwritten. */
+fp4q_status fp4q_rht_amax(const void *dy, int dtype, int64_t tokens, int64_t cols, int64_t ld,
+                          int hadamard_n, uint64_t seed, float *amax_out, void *stream);
+
+/* Random Hadamard transform of a gradient dY [tokens, cols] along tokens,
+ * fused with column-wise NVFP4 1x16 quantization (blocks of 16 tokens) of
+ * the transformed values, written as the Wgrad operand dY^T.
+ * Qiita note, "ランダムアダマール変換": Wgrad' = q(dY H) q(H^T x), with H a
+ * Hadamard matrix (H H^T = I) times a random +-1 diagonal S; "確率的丸め":
+ * stochastic rounding helps gradient quantization.
+ * Per column and per group of n = hadamard_n (16 or 128) tokens:
+ *   u = S * x (signs from Philox4x32-10(counter (0,0,1,0), key seed), bit k
+ *   of the 128-bit output -> S_k = -1), a natural-order fast Walsh-Hadamard
+ *   transform with stages h = 1, 2, ..., n/2 in that order (each butterfly
+ *   (a, b) -> (RN(a+b), RN(a-b))), then t = RN(u * RN(1/sqrt(n))).
+ *   round  FP4Q_SR (bits keyed on seed and the input index token*cols+col)
+ *          or FP4Q_RNE
+ *   amax_rht  device float: amax of t (from fp4q_rht_amax), or NULL: then
+ *          it is computed first into `workspace`
+ *   q_t [cols, tokens/2], sf_t [cols, tokens/16] (scale_layout)
+ *   rht_debug_out  nullable device float [tokens, cols] <- t itself
+ * Shape: tokens % hadamard_n == 0, cols % 8 == 0. */
+fp4q_status fp4q_quantize_rht_sr(const void *dy, int dtype, int64_t tokens, int64_t cols,
+                                 int64_t ld, int hadamard_n, int round, uint64_t seed,
+                                 const float *amax_rht, float *tensor_scale_out, uint8_t *q_t,
+                                 uint8_t *sf_t, int scale_layout, float *rht_debug_out,
+                                 void *workspace, size_t ws_bytes, void *stream);
+
+/* IF4 adaptive quantization, row-wise 1x16 ("Adaptive Block-Scaled Data
+ * Types" explainer, section 2): per block the NVFP4 scale S and factor r,
+ * v = RN(x*r); FP4 candidate E2M1_rne(v); INT4 candidate
+ * k = clamp(rint(RN(v * RN(7/6))), -7, 7) decoded as RN(k * RN(6/7)) (the 6/7
+ * method); squared errors summed in order with fused multiply-add; INT4 iff
+ * its error is strictly smaller.  INT4 nibbles hold k in two's complement;
+ * bit 7 of the scale byte is set for INT4 blocks.
+ *   q [rows, cols/2], sf [rows, cols/16]; amax / tensor_scale_out / workspace
+ *   as for fp4q_quantize_nvfp4.   Shape: cols % 16 == 0. */
+fp4q_status fp4q_quantize_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                              const float *amax, float *tensor_scale_out, uint8_t *q,
+                              uint8_t *sf, int scale_layout, void *workspace, size_t ws_bytes,
+                              void *stream);
+
+/* Dequantization of packed codes [rows, cols/2] back to y [rows, cols]
+ * (FP32 or BF16 = RNE of the FP32 value), Ultralytics glossary "FP4の仕組み"
+ * (grid value * sign * scale):
+ *   NVFP4  y = RN(RN(g * S) * s_dec)           block 1x16 or 16x16
+ *   IF4    INT4 blocks (scale bit 7): y = RN(RN(RN(k * RN(6/7)) * S) * s_dec)
+ *   MXFP4  y = g * 2^(scale - 127)             block 1x32
+ *   block_rows x block_cols: 1x16 (NVFP4, IF4), 16x16 (NVFP4 2D tiles; then
+ *   sf is the linear [rows/16, cols/16] tile matrix), 1x32 (MXFP4).
+ *   tensor_scale: device float s_dec (NVFP4 / IF4), ignored for MXFP4.
+ *   Column-wise outputs are dequantized as the [cols, rows] matrices they are.
+ * Shape: cols % block_cols == 0, rows % block_rows == 0. */
+fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,
+                            int block_rows, int block_cols, const float *tensor_scale,
+                            int64_t rows, int64_t cols, void *y, int y_dtype, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4Q_H_ */

@@ -1,0 +1,105 @@
+"""The C ABI on the CPU: the library builds for sm_100a, loads, exports every
+entry point include/fp4q.h declares, and rejects bad arguments on the host
+with the documented status codes before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp4_block_scaled_04_b200 as fq
+from fp4_block_scaled_04_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp4q.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return fq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp4q_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ["fp4q_amax", "fp4q_quantize_nvfp4", "fp4q_quantize_mxfp4", "fp4q_quantize_2d",
+              "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
+              "fp4q_scale_bytes", "fp4q_workspace_bytes", "fp4q_status_string", "fp4q_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings_and_constants(L):
+    assert fq.fp4q_status_string(0) == "FP4Q_OK"
+    assert fq.fp4q_status_string(2) == "FP4Q_ERR_UNSUPPORTED_SHAPE"
+    assert fq.fp4q_status_string(99) == "FP4Q_ERR_UNKNOWN"
+    assert "sm_100a" in fq.fp4q_version()
+    assert fq.fp4q_workspace_bytes() >= 4
+
+
+def test_scale_bytes(L):
+    assert fq.fp4q_scale_bytes(8192, 4096, 16, fq.SCALE_LINEAR) == 8192 * 256
+    assert fq.fp4q_scale_bytes(8192, 4096, 16, fq.SCALE_SWIZZLED) == 8192 * 256
+    assert fq.fp4q_scale_bytes(130, 80, 16, fq.SCALE_SWIZZLED) == 256 * 8
+    assert fq.fp4q_scale_bytes(130, 80, 16, fq.SCALE_LINEAR) == 130 * 5
+    assert fq.fp4q_scale_bytes(16, 24, 16, fq.SCALE_LINEAR) == 0      # cols % block
+    assert fq.fp4q_scale_bytes(16, 32, 16, 7) == 0                    # bad layout
+
+
+FAKE = ctypes.c_void_p(0x7F0000000000)          # 16-byte aligned, never dereferenced
+
+
+def nv(L, **kw):
+    a = dict(x=FAKE, dtype=0, rows=32, cols=64, ld=64, layouts=1, round=0, seed=0, amax=FAKE,
+             s=FAKE, q_row=FAKE, sf_row=FAKE, q_col=FAKE, sf_col=FAKE, layout=0, ws=None,
+             ws_bytes=0, stream=None)
+    a.update(kw)
+    return L.fp4q_quantize_nvfp4(a["x"], a["dtype"], a["rows"], a["cols"], a["ld"], a["layouts"],
+                                 a["round"], a["seed"], a["amax"], a["s"], a["q_row"],
+                                 a["sf_row"], a["q_col"], a["sf_col"], a["layout"], a["ws"],
+                                 a["ws_bytes"], a["stream"])
+
+
+def test_host_side_argument_checks(L):
+    assert nv(L, dtype=5) == 1                       # bad dtype
+    assert nv(L, ld=32) == 1                         # ld < cols
+    assert nv(L, layouts=0) == 1 and nv(L, layouts=4) == 1
+    assert nv(L, round=2) == 1
+    assert nv(L, layout=3) == 1
+    assert nv(L, cols=24, ld=24) == 2                # cols % 16
+    assert nv(L, rows=24, layouts=2) == 2            # COLWISE needs rows % 16
+    assert nv(L, layout=1) == 2                      # swizzle needs rows % 128
+    assert nv(L, x=ctypes.c_void_p(0x7F0000000008)) == 3
+    assert nv(L, ld=68) == 3                         # row stride not 16-byte aligned (BF16)
+    assert nv(L, q_row=None) == 1
+    assert L.fp4q_quantize_mxfp4(FAKE, 0, 32, 48, 48, 1, 0, FAKE, FAKE, None, None, 0, None) == 2
+    assert L.fp4q_quantize_mxfp4(FAKE, 0, 32, 64, 64, 1, 9, FAKE, FAKE, None, None, 0, None) == 1
+    assert L.fp4q_quantize_2d(FAKE, 1, 24, 64, 64, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 0,
+                              None, 0, None) == 2
+    assert L.fp4q_quantize_rht_sr(FAKE, 0, 128, 64, 64, 32, 1, 0, FAKE, FAKE, FAKE, FAKE, 0,
+                                  None, None, 0, None) == 1      # n must be 16 or 128
+    assert L.fp4q_quantize_rht_sr(FAKE, 0, 120, 64, 64, 16, 1, 0, FAKE, FAKE, FAKE, FAKE, 0,
+                                  None, None, 0, None) == 2      # tokens % n
+    assert L.fp4q_quantize_rht_sr(FAKE, 0, 128, 68, 72, 16, 1, 0, FAKE, FAKE, FAKE, FAKE, 0,
+                                  None, None, 0, None) == 2      # cols % 8
+    assert L.fp4q_quantize_if4(FAKE, 0, 16, 40, 40, FAKE, FAKE, FAKE, FAKE, 0, None, 0, None) == 2
+    assert L.fp4q_quantize_if4(FAKE, 0, 16, 48, 52, FAKE, FAKE, FAKE, FAKE, 0, None, 0, None) == 3
+    assert L.fp4q_dequantize(0, FAKE, FAKE, 0, 1, 32, FAKE, 16, 64, FAKE, 1, None) == 1
+    assert L.fp4q_dequantize(1, FAKE, FAKE, 0, 1, 32, None, 16, 48, FAKE, 1, None) == 2
+    assert L.fp4q_dequantize(0, FAKE, FAKE, 0, 1, 16, None, 16, 64, FAKE, 1, None) == 1
+
+
+def test_python_binding_refuses_cpu_tensors(L):
+    import torch
+    with pytest.raises(ValueError):
+        fq.fp4q_quantize_nvfp4(torch.zeros(16, 16, dtype=torch.bfloat16))
