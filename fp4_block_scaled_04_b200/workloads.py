@@ -92,8 +92,10 @@ def if4_blocks(seed: int = 0, rows: int = 16384, cols: int = 8192,
     nb = rows * cols // 16
     is_laplace = torch.rand(nb, generator=g) < 0.5
     u = torch.rand(nb, 16, generator=g, dtype=torch.float32) * 2.0 - 1.0       # U(-1, 1)
-    w = torch.rand(nb, 16, generator=g, dtype=torch.float32) - 0.5            # U(-1/2, 1/2)
-    lap = -torch.sign(w) * torch.log1p(-2.0 * w.abs())                        # Laplace(0, 1)
+    # Laplace(0, 1) = random sign * Exp(1); Exp(1) = -log(1 - U) with U in [0, 1)
+    # stays finite (1 - U >= 2^-24)
+    e = -torch.log1p(-torch.rand(nb, 16, generator=g, dtype=torch.float32))
+    lap = torch.where(torch.rand(nb, 16, generator=g) < 0.5, -e, e)
     x = torch.where(is_laplace[:, None], lap, u)
     pos = torch.randint(0, 16, (nb,), generator=g)
     x[torch.arange(nb), pos] *= outlier_scale

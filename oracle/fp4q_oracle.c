@@ -302,10 +302,15 @@ static uint8_t nvfp4_block_scale(float block_amax, float s_enc) {
 }
 
 /* READING: the element step divides by the block scale once per block:
- * r = RN(s_enc / S) (0 when S == 0), then v = RN(x * r). */
+ * r = RN(s_enc / S) (0 when S == 0), then v = RN(x * r).  READING (the
+ * pages do not consider overflow): like s_enc, r is clamped to FLT_MAX; it
+ * can only overflow when the whole tensor is tiny (amax < ~4e-33), and the
+ * clamp keeps v finite (x = 0 would otherwise give 0 * inf = NaN). */
 static float nvfp4_block_factor(uint8_t sf, float s_enc) {
   float S = orc_e4m3_value((uint8_t)(sf & 0x7F));
-  return (S == 0.0f) ? 0.0f : s_enc / S;
+  if (S == 0.0f) return 0.0f;
+  float r = s_enc / S;
+  return (r > FLT_MAX) ? FLT_MAX : r;
 }
 
 /* ------------------------------------------------------------------------ */
