@@ -132,17 +132,33 @@ __device__ __forceinline__ TensorScale tensor_scale(float amax) {
   return t;
 }
 
-// E4M3 code of the block scale: RN(RN(m * s_enc) / 6).
+// RN(y / 6) in three instructions: Markstein's correction of RN(y * RN(1/6))
+// with an exact FMA remainder (P. Markstein, IBM J. Res. Dev. 34(1), 1990).
+// Equal to the IEEE quotient for every float y in [2^-125, 4096] (checked
+// exhaustively on the host by tests/div6_check.c); below that the quotient
+// is subnormal, where callers either do not care (E4M3 rounds it to 0) or
+// use the IEEE division.
+__device__ __forceinline__ float div6(float y) {
+  constexpr float kInv6 = 1.0f / 6.0f;   // RN(1/6)
+  const float q0 = __fmul_rn(y, kInv6);
+  const float r = __fmaf_rn(-q0, 6.0f, y);
+  return __fmaf_rn(r, kInv6, q0);
+}
+
+// E4M3 code of the block scale: RN(RN(m * s_enc) / 6).  RN(m * s_enc) is at
+// most 2688 (1 + 2^-23); where it is below 2^-125 both quotients lie far
+// below the smallest E4M3 subnormal and give code 0.
 __device__ __forceinline__ uint32_t nvfp4_scale_code(float block_amax, float s_enc) {
-  return e4m3_code(__fdiv_rn(__fmul_rn(block_amax, s_enc), 6.0f));
+  return e4m3_code(div6(__fmul_rn(block_amax, s_enc)));
 }
 
 // Per-CTA table of r = RN(s_enc / S) for the 128 non-negative E4M3 codes
-// (0 for S == 0); one IEEE division per code instead of one per block.
+// (0 for S == 0, clamped to FLT_MAX like s_enc); one IEEE division per code
+// instead of one per block.
 __device__ __forceinline__ void fill_factor_table(float *tab, float s_enc) {
   for (int c = threadIdx.x; c < 128; c += blockDim.x) {
     float S = e4m3_value(static_cast<uint32_t>(c));
-    tab[c] = (S == 0.0f) ? 0.0f : __fdiv_rn(s_enc, S);
+    tab[c] = (S == 0.0f) ? 0.0f : fminf(__fdiv_rn(s_enc, S), 3.402823466e+38f);
   }
 }
 
@@ -161,7 +177,7 @@ __device__ __forceinline__ int e8m0_exponent(float m, int mode) {
     if ((b >> 23) == 0) E = -127 - (__clz(static_cast<int>(b)) - 9);  // subnormal
     e = E - 2;
   } else {
-    float t = __fdiv_rn(m, 6.0f);
+    float t = m >= 2.4e-37f ? div6(m) : __fdiv_rn(m, 6.0f);
     if (!(t > 0.0f)) return -127;
     uint32_t b = __float_as_uint(t);
     int E;
@@ -265,6 +281,121 @@ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t c, int64_t co
 // ---------------------------------------------------------------------------
 // misc
 // ---------------------------------------------------------------------------
+
+// ---------------------------------------------------------------------------
+// packed arithmetic (sm_100a f32x2 and bf16x2)
+// ---------------------------------------------------------------------------
+
+// (a.x * b.x, a.y * b.y), each rounded to nearest even
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+// (fma(a.x, b.x, c.x), fma(a.y, b.y, c.y)), single rounding each
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+
+// per 16-bit lane: max(|a|, |b|) of two BF16 pairs (the sign bits of the
+// result are meaningless; mask with 0x7FFF7FFF)
+__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// the larger magnitude of the two BF16 lanes of a max.xorsign.abs result,
+// as an FP32 value
+__device__ __forceinline__ float bf16x2_hmax(uint32_t m) {
+  m &= 0x7FFF7FFFu;
+  return __uint_as_float(max(m << 16, m & 0xFFFF0000u));
+}
+
+// |x| max over 8 BF16 in a uint4 -> FP32
+__device__ __forceinline__ float absmax8(uint4 u) {
+  return bf16x2_hmax(maxabs_bf16x2(maxabs_bf16x2(u.x, u.y), maxabs_bf16x2(u.z, u.w)));
+}
+
+// E2M1 codes of two floats as the low byte of a 32-bit register
+__device__ __forceinline__ uint32_t e2m1_byte(float lo, float hi) { return e2m1x2(lo, hi); }
+
+// Stochastic rounding onto E2M1 by integer comparisons (same rule as
+// e2m1_sr): for |v| in [1, 6) the grid has one mantissa bit and t * 2^16 is
+// the low 22 mantissa bits / 64; in [0.5, 1) the spacing is 0.5 and t * 2^16
+// is the 23 mantissa bits / 128; below 0.5, t * 2^16 = |v| * 2^17.
+__device__ __forceinline__ uint32_t e2m1_sr_bits(float v, uint32_t u16) {
+  const uint32_t raw = __float_as_uint(v);
+  const uint32_t sign = (raw >> 28) & 8u;
+  const uint32_t b = raw & 0x7FFFFFFFu;
+  const bool ge1 = b >= 0x3F800000u;
+  const uint32_t shifted = ge1 ? (u16 << 6) : (u16 << 7);
+  const uint32_t frac = ge1 ? (b & 0x3FFFFFu) : (b & 0x7FFFFFu);
+  const uint32_t base = ge1 ? (b >> 22) - 252u : 1u;
+  uint32_t code = base + (shifted < frac ? 1u : 0u);
+  const uint32_t small =
+      (static_cast<float>(u16) < __fmul_rn(__uint_as_float(b), 131072.0f)) ? 1u : 0u;
+  code = b >= 0x3F000000u ? code : small;
+  code = b >= 0x40C00000u ? 7u : code;
+  return code | sign;
+}
+
+// Philox4x32-10 with the round keys held by the caller (they depend only on
+// the seed).
+struct PhiloxKey {
+  uint32_t k0[10], k1[10];
+  __device__ __forceinline__ explicit PhiloxKey(uint64_t seed) {
+    uint32_t a = static_cast<uint32_t>(seed), b = static_cast<uint32_t>(seed >> 32);
+#pragma unroll
+    for (int i = 0; i < 10; ++i) {
+      k0[i] = a;
+      k1[i] = b;
+      a += 0x9E3779B9u;
+      b += 0xBB67AE85u;
+    }
+  }
+};
+
+__device__ __forceinline__ U32x4 philox(const PhiloxKey &K, uint32_t c0, uint32_t c1,
+                                        uint32_t c2, uint32_t c3) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c0;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c2;
+    const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ K.k0[i];
+    const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ K.k1[i];
+    c1 = static_cast<uint32_t>(p1);
+    c3 = static_cast<uint32_t>(p0);
+    c0 = n0;
+    c2 = n2;
+  }
+  return U32x4{c0, c1, c2, c3};
+}
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll

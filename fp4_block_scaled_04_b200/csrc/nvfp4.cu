@@ -7,70 +7,119 @@
 // E4M3).  Ultralytics glossary "FP4", "FP4の仕組み" (MXFP4: 32 values per
 // power-of-two E8M0 scale).
 //
-// Two kernels:
-//   rowwise_kernel  one thread per block of 16 (NVFP4) or 32 (MXFP4) values
-//                   along a row; 128-bit loads, 64/128-bit code stores.
-//   tile_kernel     a 64 x 64 tile staged in shared memory; row blocks and
-//                   column blocks are quantized from the same staged copy.
+// rowwise_kernel  one thread per block of 16 (NVFP4) or 32 (MXFP4) values of
+//                 a row, two blocks per iteration; 128-bit loads.
+// rowcol_kernel   register-tiled, no shared memory.  A thread owns 16 rows x
+//                 one 16-byte column chunk (8 BF16 or 4 FP32 columns); a warp
+//                 owns 64 rows x 8 chunks (lane = chunk + 8 * row band).
+//                 Pass 1 takes row and column block maxima on the packed
+//                 data (row blocks span 2..8 lanes: shuffle), pass 2 scales
+//                 and encodes every element twice.  Row codes of a warp
+//                 instruction are 8 lanes x 4 bytes of one row, column codes
+//                 4 lanes x 8 bytes of one column: whole 32-byte sectors.
 #include "common.cuh"
 #include "launch.h"
 
 namespace fp4q {
 namespace {
 
-constexpr int kThreads = 256;
-
-// Quantize BLK values already scaled into the E2M1 domain (RNE), packed
-// nibbles in words (8 values per word).
-template <int BLK>
-__device__ __forceinline__ void encode_rne(const float *v, uint32_t *words) {
-#pragma unroll
-  for (int w = 0; w < BLK / 8; ++w) {
-    float t[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) t[k] = v[w * 8 + k];
-    words[w] = e2m1x8(t);
-  }
-}
-
-// Stochastic rounding of 16 values whose flat input indices are
-// first + k * step (k = 0..15).
-__device__ __forceinline__ void encode_sr16(const float *v, uint64_t seed, uint64_t first,
-                                            uint64_t step, uint32_t *words) {
-  words[0] = words[1] = 0u;
-  if (step == 1 && (first % 8) == 0) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      U32x4 bits = sr_bits_group(seed, first / 8 + h);
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        words[h] |= e2m1_sr(v[h * 8 + k], half16(bits, k)) << (4 * k);
-    }
-  } else {
-#pragma unroll 1
-    for (int k = 0; k < 16; ++k) {
-      uint64_t i = first + static_cast<uint64_t>(k) * step;
-      U32x4 bits = sr_bits_group(seed, i / 8);
-      words[k >> 3] |= e2m1_sr(v[k], half16(bits, static_cast<int>(i % 8))) << (4 * (k & 7));
-    }
-  }
-}
-
-template <typename T>
-__device__ __forceinline__ void load_row_block(const T *p, float *v, int blk) {
-  for (int c = 0; c < blk; c += 8) Vec8<T>::load(p + c, *reinterpret_cast<float(*)[8]>(v + c));
-}
-
 // ----------------------------------------------------------------------------
 // row-wise only
 // ----------------------------------------------------------------------------
+constexpr int kRowThreads = 256;
+
+template <typename T, int BLK>
+__device__ __forceinline__ void load_block(const T *p, uint4 (&u)[BLK * sizeof(T) / 16]) {
+#pragma unroll
+  for (int i = 0; i < BLK * static_cast<int>(sizeof(T)) / 16; ++i)
+    u[i] = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+}
+
+template <typename T, int BLK>
+__device__ __forceinline__ void unpack_block(const uint4 (&u)[BLK * sizeof(T) / 16],
+                                             float (&v)[BLK]) {
+  if (sizeof(T) == 2) {
+#pragma unroll
+    for (int i = 0; i < BLK / 8; ++i) {
+      v[8 * i + 0] = bf16_lo(u[i].x); v[8 * i + 1] = bf16_hi(u[i].x);
+      v[8 * i + 2] = bf16_lo(u[i].y); v[8 * i + 3] = bf16_hi(u[i].y);
+      v[8 * i + 4] = bf16_lo(u[i].z); v[8 * i + 5] = bf16_hi(u[i].z);
+      v[8 * i + 6] = bf16_lo(u[i].w); v[8 * i + 7] = bf16_hi(u[i].w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < BLK / 4; ++i) {
+      v[4 * i + 0] = __uint_as_float(u[i].x); v[4 * i + 1] = __uint_as_float(u[i].y);
+      v[4 * i + 2] = __uint_as_float(u[i].z); v[4 * i + 3] = __uint_as_float(u[i].w);
+    }
+  }
+}
+
+template <typename T, int BLK>
+__device__ __forceinline__ float block_absmax(const uint4 (&u)[BLK * sizeof(T) / 16]) {
+  constexpr int N = BLK * sizeof(T) / 16;
+  if (sizeof(T) == 2) {
+    uint32_t m = maxabs_bf16x2(u[0].x, u[0].y);
+    m = maxabs_bf16x2(m, maxabs_bf16x2(u[0].z, u[0].w));
+#pragma unroll
+    for (int i = 1; i < N; ++i)
+      m = maxabs_bf16x2(m, maxabs_bf16x2(maxabs_bf16x2(u[i].x, u[i].y),
+                                         maxabs_bf16x2(u[i].z, u[i].w)));
+    return bf16x2_hmax(m);
+  } else {
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      m = fmaxf(m, fmaxf(fabsf(__uint_as_float(u[i].x)), fabsf(__uint_as_float(u[i].y))));
+      m = fmaxf(m, fmaxf(fabsf(__uint_as_float(u[i].z)), fabsf(__uint_as_float(u[i].w))));
+    }
+    return m;
+  }
+}
+
+// 16 values scaled by f, stochastic rounding with the bits of one Philox call
+// per 8 values: calls g0 and g0 + 1
+__device__ __forceinline__ void encode_sr16(const float (&v)[16], float f, const PhiloxKey &K,
+                                            uint64_t g0, uint32_t (&w)[2]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint64_t g = g0 + h;
+    const U32x4 bits = philox(K, static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u);
+    const uint32_t words[4] = {bits.x, bits.y, bits.z, bits.w};
+    uint32_t acc = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t u16 = (k & 1) ? (words[k >> 1] >> 16) : (words[k >> 1] & 0xFFFFu);
+      acc |= e2m1_sr_bits(__fmul_rn(v[8 * h + k], f), u16) << (4 * k);
+    }
+    w[h] = acc;
+  }
+}
+
+template <int BLK>
+__device__ __forceinline__ void encode_rne(const float (&v)[BLK], float f,
+                                           uint32_t (&w)[BLK / 8]) {
+#pragma unroll
+  for (int i = 0; i < BLK / 8; ++i) {
+    float t[8];
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) {
+      const float2 p = mul2(make_float2(v[8 * i + k], v[8 * i + k + 1]), make_float2(f, f));
+      t[k] = p.x;
+      t[k + 1] = p.y;
+    }
+    w[i] = e2m1x8(t);
+  }
+}
+
 template <typename T, bool MX, bool SR>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kRowThreads)
 rowwise_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                const float *__restrict__ amax_ptr, int e8m0_mode, uint64_t seed,
                float *__restrict__ s_dec_out, uint8_t *__restrict__ q,
                uint8_t *__restrict__ sf, int scale_layout) {
   constexpr int BLK = MX ? 32 : 16;
+  constexpr int NV = BLK * sizeof(T) / 16;   // uint4 per block
   __shared__ float rtab[128];
   TensorScale ts{1.0f, 1.0f};
   if (!MX) {
@@ -79,142 +128,296 @@ rowwise_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
     __syncthreads();
   }
+  const PhiloxKey K(seed);
   const int64_t bpr = cols / BLK, nblk = rows * bpr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; b < nblk;
-       b += stride) {
-    const int64_t r = b / bpr, cb = b - r * bpr;
-    float v[BLK];
-    load_row_block(x + r * ld + cb * BLK, v, BLK);
-    float m = 0.0f;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kRowThreads;
+  int64_t b = static_cast<int64_t>(blockIdx.x) * kRowThreads + threadIdx.x;
+  // two independent blocks per iteration keep 2 x BLK x sizeof(T) bytes in flight
+  for (; b < nblk; b += 2 * stride) {
+    const int64_t b1 = b + stride;
+    const bool two = b1 < nblk;
+    uint4 u0[NV], u1[NV];
+    const int64_t r0 = b / bpr, cb0 = b - r0 * bpr;
+    const int64_t r1 = two ? b1 / bpr : r0, cb1 = two ? b1 - r1 * bpr : cb0;
+    load_block<T, BLK>(x + r0 * ld + cb0 * BLK, u0);
+    load_block<T, BLK>(x + r1 * ld + cb1 * BLK, u1);
 #pragma unroll
-    for (int k = 0; k < BLK; ++k) m = fmaxf(m, fabsf(v[k]));
-    uint32_t sbyte;
-    float f;
-    if (MX) {
-      int e = e8m0_exponent(m, e8m0_mode);
-      sbyte = static_cast<uint32_t>(e + 127);
-      f = exp2_neg(e);
-    } else {
-      sbyte = nvfp4_scale_code(m, ts.enc);
-      f = rtab[sbyte];
+    for (int s = 0; s < 2; ++s) {
+      if (s == 1 && !two) break;
+      const uint4(&u)[NV] = s == 0 ? u0 : u1;
+      const int64_t r = s == 0 ? r0 : r1, cb = s == 0 ? cb0 : cb1;
+      const float m = block_absmax<T, BLK>(u);
+      uint32_t sbyte;
+      float f;
+      if (MX) {
+        const int e = e8m0_exponent(m, e8m0_mode);
+        sbyte = static_cast<uint32_t>(e + 127);
+        f = exp2_neg(e);
+      } else {
+        sbyte = nvfp4_scale_code(m, ts.enc);
+        f = rtab[sbyte];
+      }
+      float v[BLK];
+      unpack_block<T, BLK>(u, v);
+      uint8_t *qp = q + r * (cols / 2) + cb * (BLK / 2);
+      if (BLK == 16) {
+        uint32_t w[2];
+        if (SR) encode_sr16(*reinterpret_cast<const float(*)[16]>(v), f, K,
+                            static_cast<uint64_t>(r * cols + cb * 16) / 8, w);
+        else encode_rne<16>(*reinterpret_cast<const float(*)[16]>(v), f,
+                            *reinterpret_cast<uint32_t(*)[2]>(w));
+        *reinterpret_cast<uint2 *>(qp) = make_uint2(w[0], w[1]);
+      } else {
+        uint32_t w[4];
+        encode_rne<32>(*reinterpret_cast<const float(*)[32]>(v), f,
+                       *reinterpret_cast<uint32_t(*)[4]>(w));
+        *reinterpret_cast<uint4 *>(qp) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      sf[scale_offset(r, cb, bpr, scale_layout)] = static_cast<uint8_t>(sbyte);
     }
-#pragma unroll
-    for (int k = 0; k < BLK; ++k) v[k] = __fmul_rn(v[k], f);
-    uint32_t words[BLK / 8];
-    if (SR) encode_sr16(v, seed, static_cast<uint64_t>(r * cols + cb * BLK), 1, words);
-    else encode_rne<BLK>(v, words);
-    uint8_t *qp = q + r * (cols / 2) + cb * (BLK / 2);
-    if (BLK == 16) *reinterpret_cast<uint2 *>(qp) = make_uint2(words[0], words[1]);
-    else *reinterpret_cast<uint4 *>(qp) = make_uint4(words[0], words[1], words[2], words[3]);
-    sf[scale_offset(r, cb, bpr, scale_layout)] = static_cast<uint8_t>(sbyte);
   }
 }
 
 // ----------------------------------------------------------------------------
-// row-wise and/or column-wise through a shared-memory tile
+// row-wise and column-wise from one read, register tiles
 // ----------------------------------------------------------------------------
-constexpr int kTile = 64;
+constexpr int kRCThreads = 128;
+
+template <typename T, bool MX>
+struct RCGeom {
+  static constexpr int CPT = 16 / sizeof(T);   // columns per thread: 8 (BF16) or 4 (FP32)
+  static constexpr int BLK = MX ? 32 : 16;
+  static constexpr int WR = 64;                // warp tile rows (4 bands of 16)
+  static constexpr int WC = 8 * CPT;           // warp tile columns
+  static constexpr int GR = BLK / CPT;         // lanes per row block
+};
+
+template <typename T>
+__device__ __forceinline__ void unpack_chunk(uint4 u, float (&v)[16 / sizeof(T)]) {
+  if (sizeof(T) == 2) {
+    v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+    v[4 % (16 / sizeof(T))] = bf16_lo(u.z); v[5 % (16 / sizeof(T))] = bf16_hi(u.z);
+    v[6 % (16 / sizeof(T))] = bf16_lo(u.w); v[7 % (16 / sizeof(T))] = bf16_hi(u.w);
+  } else {
+    v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+  }
+}
+
+// |x| maxima of the chunk: per column lane pair for BF16 (as a packed word
+// per column pair), per column for FP32
+template <typename T>
+__device__ __forceinline__ void chunk_colmax(uint4 u, uint32_t (&cm)[4]) {
+  if (sizeof(T) == 2) {
+    cm[0] = maxabs_bf16x2(cm[0], u.x); cm[1] = maxabs_bf16x2(cm[1], u.y);
+    cm[2] = maxabs_bf16x2(cm[2], u.z); cm[3] = maxabs_bf16x2(cm[3], u.w);
+  } else {
+    cm[0] = __float_as_uint(fmaxf(__uint_as_float(cm[0]), fabsf(__uint_as_float(u.x))));
+    cm[1] = __float_as_uint(fmaxf(__uint_as_float(cm[1]), fabsf(__uint_as_float(u.y))));
+    cm[2] = __float_as_uint(fmaxf(__uint_as_float(cm[2]), fabsf(__uint_as_float(u.z))));
+    cm[3] = __float_as_uint(fmaxf(__uint_as_float(cm[3]), fabsf(__uint_as_float(u.w))));
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float chunk_rowmax(uint4 u) {
+  if (sizeof(T) == 2) return absmax8(u);
+  return fmaxf(fmaxf(fabsf(__uint_as_float(u.x)), fabsf(__uint_as_float(u.y))),
+               fmaxf(fabsf(__uint_as_float(u.z)), fabsf(__uint_as_float(u.w))));
+}
 
 template <typename T, bool MX, bool SR>
-__global__ void __launch_bounds__(kThreads)
-tile_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, unsigned layouts,
-            const float *__restrict__ amax_ptr, int e8m0_mode, uint64_t seed,
-            float *__restrict__ s_dec_out, uint8_t *__restrict__ q_row,
-            uint8_t *__restrict__ sf_row, uint8_t *__restrict__ q_col,
-            uint8_t *__restrict__ sf_col, int scale_layout) {
-  constexpr int BLK = MX ? 32 : 16;
-  constexpr int PAD = 16 / sizeof(T);   // keeps 16-byte row alignment
-  __shared__ __align__(16) T tile[kTile][kTile + PAD];
+__global__ void __launch_bounds__(kRCThreads)
+rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, unsigned layouts,
+              const float *__restrict__ amax_ptr, int e8m0_mode, uint64_t seed,
+              float *__restrict__ s_dec_out, uint8_t *__restrict__ q_row,
+              uint8_t *__restrict__ sf_row, uint8_t *__restrict__ q_col,
+              uint8_t *__restrict__ sf_col, int scale_layout) {
+  using G = RCGeom<T, MX>;
+  constexpr int CPT = G::CPT, BLK = G::BLK, GR = G::GR;
   __shared__ float rtab[128];
   TensorScale ts{1.0f, 1.0f};
   if (!MX) {
     ts = tensor_scale(*amax_ptr);
     fill_factor_table(rtab, ts.enc);
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && s_dec_out)
-      *s_dec_out = ts.dec;
-  }
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kTile;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kTile;
-  const int t = threadIdx.x;
-
-  // stage: 64 rows x 8 chunks of 8 elements
-  for (int id = t; id < kTile * (kTile / 8); id += kThreads) {
-    int rr = id / (kTile / 8), cc = (id % (kTile / 8)) * 8;
-    float v[8];
-    if (r0 + rr < rows && c0 + cc < cols) {
-      Vec8<T>::load(x + (r0 + rr) * ld + c0 + cc, v);
-    } else {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = 0.0f;
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) tile[rr][cc + k] = static_cast<T>(v[k]);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
   }
   __syncthreads();
-
-  auto quantize_block = [&](float *v, uint64_t first, uint64_t step, uint32_t *words) {
-    float m = 0.0f;
+  const PhiloxKey K(seed);
+  const bool do_row = (layouts & FP4Q_ROWWISE) != 0;
+  const bool do_col = (layouts & FP4Q_COLWISE) != 0;
+  const int lane = threadIdx.x & 31, cc = lane & 7, band = lane >> 3;
+  const int64_t tiles_c = (cols + G::WC - 1) / G::WC;
+  const int64_t ntiles = tiles_c * ((rows + G::WR - 1) / G::WR);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kRCThreads / 32);
+  for (int64_t tile = static_cast<int64_t>(blockIdx.x) * (kRCThreads / 32) + (threadIdx.x >> 5);
+       tile < ntiles; tile += nwarps) {
+    const int64_t tr = tile / tiles_c, tc = tile - tr * tiles_c;
+    const int64_t r0 = tr * G::WR + band * 16, c0 = tc * G::WC + cc * CPT;
+    const bool valid = r0 < rows && c0 < cols;
+    uint4 d[16];
 #pragma unroll
-    for (int k = 0; k < BLK; ++k) m = fmaxf(m, fabsf(v[k]));
-    uint32_t sbyte;
-    float f;
-    if (MX) {
-      int e = e8m0_exponent(m, e8m0_mode);
-      sbyte = static_cast<uint32_t>(e + 127);
-      f = exp2_neg(e);
+    for (int k = 0; k < 16; ++k)
+      d[k] = valid ? __ldg(reinterpret_cast<const uint4 *>(x + (r0 + k) * ld + c0))
+                   : make_uint4(0u, 0u, 0u, 0u);
+
+    // ---- pass 1: block maxima --------------------------------------------
+    float rmax[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) rmax[k] = chunk_rowmax<T>(d[k]);
+#pragma unroll
+    for (int o = 1; o < GR; o <<= 1)
+#pragma unroll
+      for (int k = 0; k < 16; ++k) rmax[k] = fmaxf(rmax[k], __shfl_xor_sync(0xFFFFFFFFu, rmax[k], o));
+    uint32_t cm[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 16; ++k) chunk_colmax<T>(d[k], cm);
+    float cmax[CPT];
+    if (sizeof(T) == 2) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t m = cm[j] & 0x7FFF7FFFu;
+        cmax[(2 * j) % CPT] = __uint_as_float(m << 16);
+        cmax[(2 * j + 1) % CPT] = __uint_as_float(m & 0xFFFF0000u);
+      }
     } else {
-      sbyte = nvfp4_scale_code(m, ts.enc);
-      f = rtab[sbyte];
-    }
 #pragma unroll
-    for (int k = 0; k < BLK; ++k) v[k] = __fmul_rn(v[k], f);
-    if (SR) encode_sr16(v, seed, first, step, words);
-    else encode_rne<BLK>(v, words);
-    return sbyte;
-  };
+      for (int j = 0; j < CPT; ++j) cmax[j] = __uint_as_float(cm[j % 4]);
+    }
+    if (MX) {   // a 32-row column block spans two row bands
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) cmax[j] = fmaxf(cmax[j], __shfl_xor_sync(0xFFFFFFFFu, cmax[j], 8));
+    }
 
-  if (layouts & FP4Q_ROWWISE) {
-    constexpr int kBlocks = kTile * (kTile / BLK);
-    for (int id = t; id < kBlocks; id += kThreads) {
-      int rr = id / (kTile / BLK), cb = id % (kTile / BLK);
-      int64_t r = r0 + rr, c = c0 + cb * BLK;
-      if (r >= rows || c >= cols) continue;
-      float v[BLK];
+    // ---- scales --------------------------------------------------------------
+    float rf[16], cf[CPT];
+    uint32_t rbyte[16], cbyte[CPT];
 #pragma unroll
-      for (int k = 0; k < BLK; ++k) v[k] = to_f32(tile[rr][cb * BLK + k]);
-      uint32_t words[BLK / 8];
-      uint32_t sbyte = quantize_block(v, static_cast<uint64_t>(r * cols + c), 1, words);
-      uint8_t *qp = q_row + r * (cols / 2) + c / 2;
-      if (BLK == 16) *reinterpret_cast<uint2 *>(qp) = make_uint2(words[0], words[1]);
-      else *reinterpret_cast<uint4 *>(qp) = make_uint4(words[0], words[1], words[2], words[3]);
-      sf_row[scale_offset(r, c / BLK, cols / BLK, scale_layout)] = static_cast<uint8_t>(sbyte);
+    for (int k = 0; k < 16; ++k) {
+      if (MX) {
+        const int e = e8m0_exponent(rmax[k], e8m0_mode);
+        rbyte[k] = static_cast<uint32_t>(e + 127);
+        rf[k] = exp2_neg(e);
+      } else {
+        rbyte[k] = nvfp4_scale_code(rmax[k], ts.enc);
+        rf[k] = rtab[rbyte[k]];
+      }
     }
-  }
-  if (layouts & FP4Q_COLWISE) {
-    constexpr int kBlocks = kTile * (kTile / BLK);
-    for (int id = t; id < kBlocks; id += kThreads) {
-      int cc = id % kTile, rb = id / kTile;
-      int64_t c = c0 + cc, r = r0 + rb * BLK;
-      if (c >= cols || r >= rows) continue;
-      float v[BLK];
 #pragma unroll
-      for (int k = 0; k < BLK; ++k) v[k] = to_f32(tile[rb * BLK + k][cc]);
-      uint32_t words[BLK / 8];
-      uint32_t sbyte =
-          quantize_block(v, static_cast<uint64_t>(r * cols + c), static_cast<uint64_t>(cols), words);
-      uint8_t *qp = q_col + c * (rows / 2) + r / 2;
-      if (BLK == 16) *reinterpret_cast<uint2 *>(qp) = make_uint2(words[0], words[1]);
-      else *reinterpret_cast<uint4 *>(qp) = make_uint4(words[0], words[1], words[2], words[3]);
-      sf_col[scale_offset(c, r / BLK, rows / BLK, scale_layout)] = static_cast<uint8_t>(sbyte);
+    for (int j = 0; j < CPT; ++j) {
+      if (MX) {
+        const int e = e8m0_exponent(cmax[j], e8m0_mode);
+        cbyte[j] = static_cast<uint32_t>(e + 127);
+        cf[j] = exp2_neg(e);
+      } else {
+        cbyte[j] = nvfp4_scale_code(cmax[j], ts.enc);
+        cf[j] = rtab[cbyte[j]];
+      }
+    }
+    if (valid && do_row && (cc % GR) == 0) {
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        sf_row[scale_offset(r0 + k, c0 / BLK, cols / BLK, scale_layout)] =
+            static_cast<uint8_t>(rbyte[k]);
+    }
+    if (valid && do_col && (!MX || (band & 1) == 0)) {
+#pragma unroll
+      for (int j = 0; j < CPT; ++j)
+        sf_col[scale_offset(c0 + j, r0 / BLK, rows / BLK, scale_layout)] =
+            static_cast<uint8_t>(cbyte[j]);
+    }
+
+    // ---- pass 2: encode ------------------------------------------------------
+    uint32_t colw[CPT][2];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) colw[j][0] = colw[j][1] = 0u;
+#pragma unroll
+    for (int k = 0; k < 16; k += 2) {
+      float a[CPT], b[CPT];
+      unpack_chunk<T>(d[k], a);
+      unpack_chunk<T>(d[k + 1], b);
+      uint32_t ua[CPT], ub[CPT];
+      if (SR) {
+        // one Philox call covers the 8 columns of a row from a multiple of 8
+        const uint64_t ia = static_cast<uint64_t>((r0 + k) * cols + c0);
+        const uint64_t ib = ia + static_cast<uint64_t>(cols);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint64_t i = h == 0 ? ia : ib;
+          const uint64_t g = i / 8;
+          const U32x4 bits = philox(K, static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u);
+          const uint32_t words[4] = {bits.x, bits.y, bits.z, bits.w};
+#pragma unroll
+          for (int j = 0; j < CPT; ++j) {
+            const int e = static_cast<int>(i % 8) + j;
+            const uint32_t u16 = (e & 1) ? (words[(e >> 1) & 3] >> 16) : (words[(e >> 1) & 3] & 0xFFFFu);
+            if (h == 0) ua[j] = u16; else ub[j] = u16;
+          }
+        }
+      }
+      if (do_row) {
+        uint32_t wa = 0u, wb = 0u;
+        if (SR) {
+#pragma unroll
+          for (int j = 0; j < CPT; ++j) {
+            wa |= e2m1_sr_bits(__fmul_rn(a[j], rf[k]), ua[j]) << (4 * j);
+            wb |= e2m1_sr_bits(__fmul_rn(b[j], rf[k + 1]), ub[j]) << (4 * j);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < CPT; j += 2) {
+            const float2 pa = mul2(make_float2(a[j], a[j + 1]), make_float2(rf[k], rf[k]));
+            const float2 pb = mul2(make_float2(b[j], b[j + 1]), make_float2(rf[k + 1], rf[k + 1]));
+            wa |= e2m1x2(pa.x, pa.y) << (4 * j);
+            wb |= e2m1x2(pb.x, pb.y) << (4 * j);
+          }
+        }
+        if (valid) {
+          uint8_t *qa = q_row + (r0 + k) * (cols / 2) + c0 / 2;
+          if (CPT == 8) {
+            *reinterpret_cast<uint32_t *>(qa) = wa;
+            *reinterpret_cast<uint32_t *>(qa + cols / 2) = wb;
+          } else {
+            *reinterpret_cast<uint16_t *>(qa) = static_cast<uint16_t>(wa);
+            *reinterpret_cast<uint16_t *>(qa + cols / 2) = static_cast<uint16_t>(wb);
+          }
+        }
+      }
+      if (do_col) {
+#pragma unroll
+        for (int j = 0; j < CPT; j += 2) {
+          const float2 pa = mul2(make_float2(a[j], a[j + 1]), make_float2(cf[j], cf[j + 1]));
+          const float2 pb = mul2(make_float2(b[j], b[j + 1]), make_float2(cf[j], cf[j + 1]));
+          uint32_t b0, b1;
+          if (SR) {
+            b0 = e2m1_sr_bits(pa.x, ua[j]) | (e2m1_sr_bits(pb.x, ub[j]) << 4);
+            b1 = e2m1_sr_bits(pa.y, ua[j + 1]) | (e2m1_sr_bits(pb.y, ub[j + 1]) << 4);
+          } else {
+            b0 = e2m1x2(pa.x, pb.x);       // column j: rows k (low), k + 1 (high)
+            b1 = e2m1x2(pa.y, pb.y);       // column j + 1
+          }
+          colw[j][k >> 3] |= b0 << (8 * ((k >> 1) & 3));
+          colw[j + 1][k >> 3] |= b1 << (8 * ((k >> 1) & 3));
+        }
+      }
+    }
+    if (do_col && valid) {
+#pragma unroll
+      for (int j = 0; j < CPT; ++j)
+        *reinterpret_cast<uint2 *>(q_col + (c0 + j) * (rows / 2) + r0 / 2) =
+            make_uint2(colw[j][0], colw[j][1]);
     }
   }
 }
 
-int rowwise_grid(int64_t nblk, const Launch &L) {
-  int64_t want = (nblk + kThreads - 1) / kThreads;
-  int64_t cap = static_cast<int64_t>(L.num_sms) * 8;
-  return static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+int grid_cap(const void *kernel, int threads, const Launch &L) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  return per_sm * L.num_sms;
 }
 
 template <typename T, bool MX, bool SR>
@@ -224,12 +427,23 @@ cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, uns
                          int scale_layout, const Launch &L) {
   constexpr int BLK = MX ? 32 : 16;
   if (layouts == FP4Q_ROWWISE) {
-    rowwise_kernel<T, MX, SR><<<rowwise_grid(rows * (cols / BLK), L), kThreads, 0, L.stream>>>(
+    const int64_t nblk = rows * (cols / BLK);
+    static int cap = 0;
+    if (cap == 0) cap = grid_cap(reinterpret_cast<const void *>(rowwise_kernel<T, MX, SR>),
+                                 kRowThreads, L);
+    const int64_t want = (nblk + 2 * kRowThreads - 1) / (2 * kRowThreads);
+    const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+    rowwise_kernel<T, MX, SR><<<grid, kRowThreads, 0, L.stream>>>(
         x, rows, cols, ld, amax, e8m0_mode, seed, s_dec_out, q_row, sf_row, scale_layout);
   } else {
-    dim3 grid(static_cast<unsigned>((cols + kTile - 1) / kTile),
-              static_cast<unsigned>((rows + kTile - 1) / kTile));
-    tile_kernel<T, MX, SR><<<grid, kThreads, 0, L.stream>>>(
+    using G = RCGeom<T, MX>;
+    const int64_t ntiles = ((cols + G::WC - 1) / G::WC) * ((rows + G::WR - 1) / G::WR);
+    static int cap = 0;
+    if (cap == 0) cap = grid_cap(reinterpret_cast<const void *>(rowcol_kernel<T, MX, SR>),
+                                 kRCThreads, L);
+    const int64_t want = (ntiles + kRCThreads / 32 - 1) / (kRCThreads / 32);
+    const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+    rowcol_kernel<T, MX, SR><<<grid, kRCThreads, 0, L.stream>>>(
         x, rows, cols, ld, layouts, amax, e8m0_mode, seed, s_dec_out, q_row, sf_row, q_col,
         sf_col, scale_layout);
   }

@@ -3,17 +3,32 @@
 // Qiita note on NVFP4 training, "2D scaling": with 1x16 blocks q(W) differs
 // from q(W^T)^T because the scaling direction changes under transposition;
 // square 16x16 tiles give both the same scales, so W and W^T codes come out
-// of one pass.  Each 64 x 64 region is staged in shared memory; 16 threads
-// share a tile: thread i quantizes row i of the tile (W codes) and column i
-// (W^T codes) with the tile's single scale.
+// of one pass.
+//
+// Register tiles, no shared memory: a thread owns 16 rows x one 16-byte
+// column chunk (4 FP32 or 8 BF16 columns); a 16x16 tile spans 4 (FP32) or 2
+// (BF16) lanes, whose partial maxima meet by shuffle.  A warp owns 64 rows x
+// 8 chunks (lane = chunk + 8 * row band), so a warp instruction writes W^T
+// codes as whole 32-byte sectors (4 bands x 8 bytes of one column).
 #include "common.cuh"
 #include "launch.h"
 
 namespace fp4q {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kRegion = 64;
+constexpr int kThreads = 128;
+
+template <typename T>
+__device__ __forceinline__ void unpack4or8(uint4 u, float (&v)[16 / sizeof(T)]) {
+  if (sizeof(T) == 2) {
+    v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+    v[4 % (16 / sizeof(T))] = bf16_lo(u.z); v[5 % (16 / sizeof(T))] = bf16_hi(u.z);
+    v[6 % (16 / sizeof(T))] = bf16_lo(u.w); v[7 % (16 / sizeof(T))] = bf16_hi(u.w);
+  } else {
+    v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+  }
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
@@ -22,76 +37,107 @@ quant2d_kernel(const T *__restrict__ w, int64_t rows, int64_t cols, int64_t ld,
                uint8_t *__restrict__ q_w, uint8_t *__restrict__ q_wt,
                uint8_t *__restrict__ sf_tiles, uint8_t *__restrict__ sf_w_1x16,
                uint8_t *__restrict__ sf_wt_1x16, int scale_layout) {
-  // row stride of 68 floats (or 72 BF16) staggers rows across bank groups
-  constexpr int PAD = sizeof(T) == 4 ? 4 : 8;
-  __shared__ __align__(16) float tile[kRegion][kRegion + PAD];
+  constexpr int CPT = 16 / sizeof(T);       // columns per thread
+  constexpr int LPT = 16 / CPT;             // lanes per tile
+  constexpr int WC = 8 * CPT;               // warp tile columns
   __shared__ float rtab[128];
   const TensorScale ts = tensor_scale(*amax_ptr);
   fill_factor_table(rtab, ts.enc);
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
-
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kRegion;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kRegion;
-  const int t = threadIdx.x;
-  for (int id = t; id < kRegion * (kRegion / 8); id += kThreads) {
-    int rr = id / (kRegion / 8), cc = (id % (kRegion / 8)) * 8;
-    float v[8];
-    if (r0 + rr < rows && c0 + cc < cols) {
-      Vec8<T>::load(w + (r0 + rr) * ld + c0 + cc, v);
-    } else {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = 0.0f;
-    }
-    *reinterpret_cast<float4 *>(&tile[rr][cc]) = make_float4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<float4 *>(&tile[rr][cc + 4]) = make_float4(v[4], v[5], v[6], v[7]);
-  }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
   __syncthreads();
 
-  const int tid = t >> 4;            // tile within the region: 4 x 4
-  const int i = t & 15;              // row (and column) of the tile this thread owns
-  const int tr = tid >> 2, tc = tid & 3;
-  const int64_t gr = r0 + tr * 16, gc = c0 + tc * 16;   // tile origin
-  const bool valid = gr < rows && gc < cols;
+  const int lane = threadIdx.x & 31, cc = lane & 7, band = lane >> 3;
+  const int li = cc % LPT;                  // lane index within the tile
+  const int64_t tiles_c = (cols + WC - 1) / WC;
+  const int64_t ntiles = tiles_c * ((rows + 63) / 64);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  for (int64_t tile = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
+       tile < ntiles; tile += nwarps) {
+    const int64_t tr = tile / tiles_c, tcol = tile - tr * tiles_c;
+    const int64_t r0 = tr * 64 + band * 16, c0 = tcol * WC + cc * CPT;
+    const bool valid = r0 < rows && c0 < cols;   // the whole 16x16 tile shares validity
+    uint4 d[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      d[k] = valid ? __ldg(reinterpret_cast<const uint4 *>(w + (r0 + k) * ld + c0))
+                   : make_uint4(0u, 0u, 0u, 0u);
+    float m;
+    if (sizeof(T) == 2) {
+      uint32_t mm = 0u;
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        mm = maxabs_bf16x2(mm, maxabs_bf16x2(maxabs_bf16x2(d[k].x, d[k].y),
+                                             maxabs_bf16x2(d[k].z, d[k].w)));
+      m = bf16x2_hmax(mm);
+    } else {
+      m = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(__uint_as_float(d[k].x)), fabsf(__uint_as_float(d[k].y))),
+                           fmaxf(fabsf(__uint_as_float(d[k].z)), fabsf(__uint_as_float(d[k].w)))));
+    }
+#pragma unroll
+    for (int o = 1; o < LPT; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (!valid) continue;
 
-  float rowv[16], colv[16];
+    const uint32_t sbyte = nvfp4_scale_code(m, ts.enc);
+    const float f = rtab[sbyte];
+    const int64_t gr = r0, gc = c0 - li * CPT;        // tile origin
+    uint32_t colw[CPT][2];
 #pragma unroll
-  for (int k = 0; k < 16; k += 4) {
-    float4 a = *reinterpret_cast<const float4 *>(&tile[tr * 16 + i][tc * 16 + k]);
-    rowv[k] = a.x; rowv[k + 1] = a.y; rowv[k + 2] = a.z; rowv[k + 3] = a.w;
+    for (int j = 0; j < CPT; ++j) colw[j][0] = colw[j][1] = 0u;
+#pragma unroll
+    for (int k = 0; k < 16; k += 2) {
+      float a[CPT], b[CPT];
+      unpack4or8<T>(d[k], a);
+      unpack4or8<T>(d[k + 1], b);
+#pragma unroll
+      for (int j = 0; j < CPT; j += 2) {
+        const float2 pa = mul2(make_float2(a[j], a[j + 1]), make_float2(f, f));
+        const float2 pb = mul2(make_float2(b[j], b[j + 1]), make_float2(f, f));
+        a[j] = pa.x; a[j + 1] = pa.y; b[j] = pb.x; b[j + 1] = pb.y;
+      }
+      if (q_w) {
+        uint32_t wa = 0u, wb = 0u;
+#pragma unroll
+        for (int j = 0; j < CPT; j += 2) {
+          wa |= e2m1x2(a[j], a[j + 1]) << (4 * j);
+          wb |= e2m1x2(b[j], b[j + 1]) << (4 * j);
+        }
+        uint8_t *qa = q_w + (r0 + k) * (cols / 2) + c0 / 2;
+        if (CPT == 8) {
+          *reinterpret_cast<uint32_t *>(qa) = wa;
+          *reinterpret_cast<uint32_t *>(qa + cols / 2) = wb;
+        } else {
+          *reinterpret_cast<uint16_t *>(qa) = static_cast<uint16_t>(wa);
+          *reinterpret_cast<uint16_t *>(qa + cols / 2) = static_cast<uint16_t>(wb);
+        }
+      }
+      if (q_wt) {
+#pragma unroll
+        for (int j = 0; j < CPT; ++j)   // column j: rows k (low nibble), k + 1
+          colw[j][k >> 3] |= e2m1x2(a[j], b[j]) << (8 * ((k >> 1) & 3));
+      }
+    }
+    if (q_wt) {
+#pragma unroll
+      for (int j = 0; j < CPT; ++j)
+        *reinterpret_cast<uint2 *>(q_wt + (c0 + j) * (rows / 2) + r0 / 2) =
+            make_uint2(colw[j][0], colw[j][1]);
+    }
+    const uint8_t sb = static_cast<uint8_t>(sbyte);
+    if (li == 0) sf_tiles[(gr / 16) * (cols / 16) + gc / 16] = sb;
+    if (sf_w_1x16) {
+#pragma unroll
+      for (int k = 0; k < 16 / LPT; ++k)
+        sf_w_1x16[scale_offset(gr + li * (16 / LPT) + k, gc / 16, cols / 16, scale_layout)] = sb;
+    }
+    if (sf_wt_1x16) {
+#pragma unroll
+      for (int j = 0; j < CPT; ++j)
+        sf_wt_1x16[scale_offset(c0 + j, gr / 16, rows / 16, scale_layout)] = sb;
+    }
   }
-#pragma unroll
-  for (int k = 0; k < 16; ++k) colv[k] = tile[tr * 16 + k][tc * 16 + i];
-
-  float m = 0.0f;
-#pragma unroll
-  for (int k = 0; k < 16; ++k) m = fmaxf(m, fabsf(rowv[k]));
-#pragma unroll
-  for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  if (!valid) return;   // (no barrier follows)
-
-  const uint32_t sbyte = nvfp4_scale_code(m, ts.enc);
-  const float f = rtab[sbyte];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    rowv[k] = __fmul_rn(rowv[k], f);
-    colv[k] = __fmul_rn(colv[k], f);
-  }
-  uint32_t wr[2], wc[2];
-  {
-    float a[8], b[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) { a[k] = rowv[k]; b[k] = rowv[k + 8]; }
-    wr[0] = e2m1x8(a); wr[1] = e2m1x8(b);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) { a[k] = colv[k]; b[k] = colv[k + 8]; }
-    wc[0] = e2m1x8(a); wc[1] = e2m1x8(b);
-  }
-  const int64_t r = gr + i, c = gc + i;
-  if (q_w) *reinterpret_cast<uint2 *>(q_w + r * (cols / 2) + gc / 2) = make_uint2(wr[0], wr[1]);
-  if (q_wt) *reinterpret_cast<uint2 *>(q_wt + c * (rows / 2) + gr / 2) = make_uint2(wc[0], wc[1]);
-  if (i == 0) sf_tiles[(gr / 16) * (cols / 16) + gc / 16] = static_cast<uint8_t>(sbyte);
-  if (sf_w_1x16) sf_w_1x16[scale_offset(r, gc / 16, cols / 16, scale_layout)] = static_cast<uint8_t>(sbyte);
-  if (sf_wt_1x16) sf_wt_1x16[scale_offset(c, gr / 16, rows / 16, scale_layout)] = static_cast<uint8_t>(sbyte);
 }
 
 }  // namespace
@@ -100,8 +146,19 @@ cudaError_t launch_2d(const void *w, int dtype, int64_t rows, int64_t cols, int6
                       const float *amax, float *s_dec_out, uint8_t *q_w, uint8_t *q_wt,
                       uint8_t *sf_tiles, uint8_t *sf_w_1x16, uint8_t *sf_wt_1x16,
                       int scale_layout, const Launch &L) {
-  dim3 grid(static_cast<unsigned>((cols + kRegion - 1) / kRegion),
-            static_cast<unsigned>((rows + kRegion - 1) / kRegion));
+  const int cpt = dtype == FP4Q_BF16 ? 8 : 4;
+  const int64_t ntiles = ((cols + 8 * cpt - 1) / (8 * cpt)) * ((rows + 63) / 64);
+  const void *kern = dtype == FP4Q_BF16 ? reinterpret_cast<const void *>(quant2d_kernel<__nv_bfloat16>)
+                                        : reinterpret_cast<const void *>(quant2d_kernel<float>);
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
+  const int64_t want = (ntiles + kThreads / 32 - 1) / (kThreads / 32);
+  const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
   if (dtype == FP4Q_BF16)
     quant2d_kernel<__nv_bfloat16><<<grid, kThreads, 0, L.stream>>>(
         static_cast<const __nv_bfloat16 *>(w), rows, cols, ld, amax, s_dec_out, q_w, q_wt,

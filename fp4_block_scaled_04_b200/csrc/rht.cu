@@ -7,301 +7,342 @@
 // diagonal of random signs; it helps Wgrad only.  "確率的丸め": stochastic
 // rounding helps gradient quantization.
 //
-// One CTA handles 128 tokens x 64 columns, staged in shared memory as FP32:
-//   A   each thread loads 16 tokens of 2 adjacent columns, flips signs and
-//       runs the butterfly stages h = 1, 2, 4, 8 in registers;
-//   A2  (n = 128) stages h = 16, 32, 64 across the eight 16-token groups;
-//   B1  one E4M3 scale per (column, 16-token block);
-//   B2  each thread encodes 4 tokens x 8 columns -- the 8 columns of one
-//       Philox draw for stochastic rounding;
-//   C   codes and scales go out as dY^T rows.
+// Register tiles: a thread owns 4 columns x 16 consecutive tokens (one
+// 16-token group of the transform and one quantization block per column); a
+// warp owns 128 tokens x 16 columns (lane = group + 8 * column quad).
+//   * sign flip and the butterfly stages h = 1, 2, 4, 8 run in registers on
+//     f32x2 pairs of columns;
+//   * for n = 128 the stages h = 16, 32, 64 combine the eight groups: the warp
+//     swaps values through an 8 KB shared buffer (XOR-swizzled so that both
+//     the write and the transposed read hit every bank once per wavefront),
+//     runs the three stages, and swaps back;
+//   * block maxima are in-thread; stochastic rounding needs one Philox call
+//     per token per 8 columns, which two lanes share (each computes half of
+//     the tokens and passes the other lane its 64 bits by shuffle);
+//   * dY^T codes leave as 8 lanes x 8 bytes = 64 contiguous bytes per column.
 #include "common.cuh"
 #include "launch.h"
 
 namespace fp4q {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kTT = 128;  // tokens per tile
-constexpr int kTC = 64;   // columns per tile
-constexpr int kLd = kTC + 4;
+constexpr int kThreads = 128;       // 4 warps
+constexpr int kWarps = kThreads / 32;
 
-template <typename T> struct Pair;
-template <> struct Pair<__nv_bfloat16> {
-  __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float &a, float &b) {
-    uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(p));
-    a = bf16_lo(w);
-    b = bf16_hi(w);
-  }
-};
-template <> struct Pair<float> {
-  __device__ __forceinline__ static void load(const float *p, float &a, float &b) {
-    float2 v = __ldg(reinterpret_cast<const float2 *>(p));
-    a = v.x;
-    b = v.y;
-  }
-};
+template <typename T>
+__device__ __forceinline__ void load4(const T *p, float (&v)[4]);
+template <>
+__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16 *p, float (&v)[4]) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+  v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+}
+template <>
+__device__ __forceinline__ void load4<float>(const float *p, float (&v)[4]) {
+  const float4 u = __ldg(reinterpret_cast<const float4 *>(p));
+  v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+}
 
 __device__ __forceinline__ float flip(float x, uint32_t bit) {
   return __uint_as_float(__float_as_uint(x) ^ (bit << 31));
 }
 
-// butterfly stage on 2*len values held as pairs (u[i], u[i+h])
+// one butterfly stage over 16 tokens of 4 columns held as two column pairs
 template <int H>
-__device__ __forceinline__ void stage16(float (&u)[16]) {
+__device__ __forceinline__ void stage(float2 (&lo)[16], float2 (&hi)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i)
     if ((i & H) == 0) {
-      float a = u[i], b = u[i + H];
-      u[i] = __fadd_rn(a, b);
-      u[i + H] = __fsub_rn(a, b);
+      const float2 a = lo[i], b = lo[i + H];
+      lo[i] = add2(a, b);
+      lo[i + H] = sub2(a, b);
+      const float2 c = hi[i], d = hi[i + H];
+      hi[i] = add2(c, d);
+      hi[i + H] = sub2(c, d);
     }
 }
 
+// cross-group stage on 8 groups x 2 offsets: values u[g][o]
 template <int H>
-__device__ __forceinline__ void stage8(float (&u)[8]) {
+__device__ __forceinline__ void xstage(float2 (&lo)[16], float2 (&hi)[16]) {
+  // index = 2 * group + offset; stage pairs groups g and g + H
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    if ((i & H) == 0) {
-      float a = u[i], b = u[i + H];
-      u[i] = __fadd_rn(a, b);
-      u[i + H] = __fsub_rn(a, b);
-    }
+  for (int g = 0; g < 8; ++g)
+    if ((g & H) == 0)
+#pragma unroll
+      for (int o = 0; o < 2; ++o) {
+        const int i = 2 * g + o, j = 2 * (g + H) + o;
+        const float2 a = lo[i], b = lo[j];
+        lo[i] = add2(a, b);
+        lo[j] = sub2(a, b);
+        const float2 c = hi[i], d = hi[j];
+        hi[i] = add2(c, d);
+        hi[j] = sub2(c, d);
+      }
 }
 
-struct Smem {
-  float t[kTT][kLd];                 // transformed values
-  float rf[kTT / 16][kTC];           // r = RN(s_enc / S) per (block, column)
-  uint8_t sc[kTC][kTT / 16];         // E4M3 scale code per (column, block)
-  __align__(16) uint8_t cs[kTC][kTT / 2 + 16];  // packed codes per column
-  float rtab[128];
-  uint32_t red[kThreads / 32];
-};
+// 16-byte chunk (token t, column quad q) of a warp's 128 x 16 FP32 buffer,
+// XOR-swizzled within each 128-byte line
+__device__ __forceinline__ int chunk(int t, int q) {
+  const int sw = ((t >> 4) ^ (t >> 1)) & 7;
+  return (t * 4 + q) ^ sw;
+}
 
 template <typename T, int N, bool SR, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld, uint64_t seed,
            const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
            unsigned *__restrict__ amax_out, uint8_t *__restrict__ q_t,
            uint8_t *__restrict__ sf_t, int scale_layout, float *__restrict__ rht_out) {
-  __shared__ __align__(16) Smem s;
-  const int t = threadIdx.x;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kTT;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kTC;
-
+  __shared__ float rtab[128];
+  __shared__ __align__(16) float4 xbuf[N == 128 ? kWarps * 128 * 4 : 1];
   TensorScale ts{1.0f, 1.0f};
   if (!AMAX_ONLY) {
     ts = tensor_scale(*amax_ptr);
-    fill_factor_table(s.rtab, ts.enc);
-    if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0 && s_dec_out) *s_dec_out = ts.dec;
-  }
-
-  // ---- A: sign flip + in-group stages -----------------------------------
-  {
-    const int p = t & 31, g = t >> 5;
-    const int64_t col = c0 + 2 * p, tok0 = t0 + 16 * g;
-    const bool active = col < cols && tok0 < tokens;
-    // the random diagonal: bit k of Philox(counter (0,0,1,0), key seed)
-    const U32x4 sw = philox4x32_10(U32x4{0u, 0u, 1u, 0u}, static_cast<uint32_t>(seed),
-                                   static_cast<uint32_t>(seed >> 32));
-    uint32_t bits16;
-    if (N == 16) {
-      bits16 = sw.x & 0xFFFFu;
-    } else {
-      uint32_t word = (g >> 1) == 0 ? sw.x : (g >> 1) == 1 ? sw.y : (g >> 1) == 2 ? sw.z : sw.w;
-      bits16 = (word >> ((g & 1) * 16)) & 0xFFFFu;
-    }
-    float u0[16], u1[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      float a = 0.0f, b = 0.0f;
-      if (active) Pair<T>::load(dy + (tok0 + k) * ld + col, a, b);
-      uint32_t bit = (bits16 >> k) & 1u;
-      u0[k] = flip(a, bit);
-      u1[k] = flip(b, bit);
-    }
-    stage16<1>(u0); stage16<1>(u1);
-    stage16<2>(u0); stage16<2>(u1);
-    stage16<4>(u0); stage16<4>(u1);
-    stage16<8>(u0); stage16<8>(u1);
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      float a = u0[k], b = u1[k];
-      if (N == 16) {
-        a = __fmul_rn(a, 0.25f);
-        b = __fmul_rn(b, 0.25f);
-      }
-      *reinterpret_cast<float2 *>(&s.t[16 * g + k][2 * p]) = make_float2(a, b);
-    }
+    fill_factor_table(rtab, ts.enc);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
   }
   __syncthreads();
+  const int lane = threadIdx.x & 31, g = lane & 7, cq = lane >> 3;
+  float4 *buf = xbuf + (N == 128 ? (threadIdx.x >> 5) * 512 : 0);
 
-  // ---- A2: cross-group stages for n = 128 ---------------------------------
-  if (N == 128) {
-    const float c128 = __frsqrt_rn(128.0f);
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int id = t + kThreads * j;
-      const int p = id & 31, o = id >> 5;
-      float u0[8], u1[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float2 v = *reinterpret_cast<const float2 *>(&s.t[o + 16 * q][2 * p]);
-        u0[q] = v.x;
-        u1[q] = v.y;
-      }
-      stage8<1>(u0); stage8<1>(u1);   // h = 16
-      stage8<2>(u0); stage8<2>(u1);   // h = 32
-      stage8<4>(u0); stage8<4>(u1);   // h = 64
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<float2 *>(&s.t[o + 16 * q][2 * p]) =
-            make_float2(__fmul_rn(u0[q], c128), __fmul_rn(u1[q], c128));
-    }
-    __syncthreads();
+  // the random diagonal: bit k of Philox(counter (0,0,1,0), key seed)
+  const U32x4 sw = philox4x32_10(U32x4{0u, 0u, 1u, 0u}, static_cast<uint32_t>(seed),
+                                 static_cast<uint32_t>(seed >> 32));
+  uint32_t signs;   // bit k: sign of token 16 g + k of a 128-token group (bit k of a 16-group)
+  if (N == 16) {
+    signs = sw.x & 0xFFFFu;
+  } else {
+    const uint32_t word = (g >> 1) == 0 ? sw.x : (g >> 1) == 1 ? sw.y : (g >> 1) == 2 ? sw.z : sw.w;
+    signs = (word >> ((g & 1) * 16)) & 0xFFFFu;
   }
+  const float cn = N == 16 ? 0.25f : __frsqrt_rn(128.0f);
 
-  if (AMAX_ONLY) {
-    uint32_t m = 0;
-    for (int id = t; id < kTT * kTC; id += kThreads) {
-      float v = s.t[id / kTC][id % kTC];
-      m = max(m, __float_as_uint(v) & 0x7FFFFFFFu);
+  const int64_t tiles_c = (cols + 15) / 16;
+  const int64_t ntiles = tiles_c * ((tokens + 127) / 128);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+  uint32_t amax_bits = 0u;
+  for (int64_t tile = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+       tile < ntiles; tile += nwarps) {
+    const int64_t tt = tile / tiles_c, tc = tile - tt * tiles_c;
+    const int64_t t0 = tt * 128 + 16 * g, c0 = tc * 16 + 4 * cq;
+    // a column quad is all-in or all-out (cols % 8 == 0); a 16-token group
+    // likewise (tokens % 16 == 0); for n = 128 all groups of a tile are in
+    const bool valid = c0 < cols && t0 < tokens;
+
+    // ---- load, sign flip, stages h = 1..8 -----------------------------------
+    float2 lo[16], hi[16];     // columns (c0, c0+1) and (c0+2, c0+3) per token
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (valid) load4<T>(dy + (t0 + k) * ld + c0, v);
+      const uint32_t bit = (signs >> k) & 1u;
+      lo[k] = make_float2(flip(v[0], bit), flip(v[1], bit));
+      hi[k] = make_float2(flip(v[2], bit), flip(v[3], bit));
     }
-    m = __reduce_max_sync(0xFFFFFFFFu, m);
-    if ((t & 31) == 0) s.red[t >> 5] = m;
-    __syncthreads();
-    if (t < 32) {
-      uint32_t v = t < kThreads / 32 ? s.red[t] : 0u;
-      v = __reduce_max_sync(0xFFFFFFFFu, v);
-      if (t == 0) atomicMax(amax_out, v);
-    }
-    return;
-  }
+    stage<1>(lo, hi);
+    stage<2>(lo, hi);
+    stage<4>(lo, hi);
+    stage<8>(lo, hi);
 
-  if (rht_out) {
-    for (int id = t; id < kTT * (kTC / 4); id += kThreads) {
-      const int rr = id / (kTC / 4), cc = (id % (kTC / 4)) * 4;
-      if (t0 + rr < tokens && c0 + cc < cols)
-        *reinterpret_cast<float4 *>(rht_out + (t0 + rr) * cols + c0 + cc) =
-            *reinterpret_cast<const float4 *>(&s.t[rr][cc]);
-    }
-  }
-
-  // ---- B1: block scales ----------------------------------------------------
+    if (N == 128) {
+      // ---- stages h = 16, 32, 64 across the eight groups ----------------------
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int id = t + kThreads * j;
-    const int cc = id & (kTC - 1), b = id >> 6;
-    float m = 0.0f;
+      for (int k = 0; k < 16; ++k)
+        buf[chunk(16 * g + k, cq)] = make_float4(lo[k].x, lo[k].y, hi[k].x, hi[k].y);
+      __syncwarp();
+      // now this lane takes in-group offsets 2g, 2g+1 of all eight groups
 #pragma unroll
-    for (int k = 0; k < 16; ++k) m = fmaxf(m, fabsf(s.t[16 * b + k][cc]));
-    const uint32_t code = nvfp4_scale_code(m, ts.enc);
-    s.sc[cc][b] = static_cast<uint8_t>(code);
-    s.rf[b][cc] = s.rtab[code];
-  }
-  __syncthreads();
-
-  // ---- B2: encode 4 tokens x 8 columns ------------------------------------
-  {
-    const int o = t & 7, q = t >> 3;
-    const int b = q >> 2;
-    const int64_t gcol = c0 + 8 * o;
-    if (gcol < cols && t0 + 4 * q < tokens) {
-      float f[8];
-      {
-        float4 a = *reinterpret_cast<const float4 *>(&s.rf[b][8 * o]);
-        float4 c = *reinterpret_cast<const float4 *>(&s.rf[b][8 * o + 4]);
-        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-        f[4] = c.x; f[5] = c.y; f[6] = c.z; f[7] = c.w;
-      }
-      uint32_t packed[8];
+      for (int gg = 0; gg < 8; ++gg)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) packed[j] = 0u;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float v[8];
-        float4 a = *reinterpret_cast<const float4 *>(&s.t[4 * q + k][8 * o]);
-        float4 c = *reinterpret_cast<const float4 *>(&s.t[4 * q + k][8 * o + 4]);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(v[j], f[j]);
-        if (SR) {
-          const uint64_t gt = static_cast<uint64_t>(t0 + 4 * q + k);
-          const U32x4 bits = sr_bits_group(seed, (gt * static_cast<uint64_t>(cols) +
-                                                  static_cast<uint64_t>(gcol)) / 8);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) packed[j] |= e2m1_sr(v[j], half16(bits, j)) << (4 * k);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; j += 2) {
-            uint32_t pr = e2m1x2(v[j], v[j + 1]);   // columns j, j+1 of token k
-            packed[j] |= (pr & 0xFu) << (4 * k);
-            packed[j + 1] |= ((pr >> 4) & 0xFu) << (4 * k);
-          }
+        for (int o = 0; o < 2; ++o) {
+          const float4 c = buf[chunk(16 * gg + 2 * g + o, cq)];
+          lo[2 * gg + o] = make_float2(c.x, c.y);
+          hi[2 * gg + o] = make_float2(c.z, c.w);
         }
+      xstage<1>(lo, hi);   // h = 16
+      xstage<2>(lo, hi);   // h = 32
+      xstage<4>(lo, hi);   // h = 64
+#pragma unroll
+      for (int gg = 0; gg < 8; ++gg)
+#pragma unroll
+        for (int o = 0; o < 2; ++o) {
+          const int i = 2 * gg + o;
+          buf[chunk(16 * gg + 2 * g + o, cq)] = make_float4(lo[i].x, lo[i].y, hi[i].x, hi[i].y);
+        }
+      __syncwarp();
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float4 c = buf[chunk(16 * g + k, cq)];
+        lo[k] = make_float2(c.x, c.y);
+        hi[k] = make_float2(c.z, c.w);
       }
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint16_t *>(&s.cs[8 * o + j][2 * q]) = static_cast<uint16_t>(packed[j]);
+      __syncwarp();
     }
-  }
-  __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      lo[k] = mul2(lo[k], make_float2(cn, cn));
+      hi[k] = mul2(hi[k], make_float2(cn, cn));
+    }
 
-  // ---- C: store dY^T codes and scales ---------------------------------------
-  {
-    const int cc = t >> 2, ch = t & 3;
-    const int64_t col = c0 + cc;
-    if (col < cols) {
-      uint8_t *dst = q_t + col * (tokens / 2) + t0 / 2 + 16 * ch;
-      const int64_t tok = t0 + 32 * ch;
-      if (tok + 16 <= tokens)
-        *reinterpret_cast<uint2 *>(dst) = *reinterpret_cast<const uint2 *>(&s.cs[cc][16 * ch]);
-      if (tok + 32 <= tokens)
-        *reinterpret_cast<uint2 *>(dst + 8) =
-            *reinterpret_cast<const uint2 *>(&s.cs[cc][16 * ch + 8]);
+    // ---- block maxima (16 tokens of each column) ------------------------------
+    float m[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      m[0] = fmaxf(m[0], fabsf(lo[k].x));
+      m[1] = fmaxf(m[1], fabsf(lo[k].y));
+      m[2] = fmaxf(m[2], fabsf(hi[k].x));
+      m[3] = fmaxf(m[3], fabsf(hi[k].y));
+    }
+    if (AMAX_ONLY) {
+      if (valid)
+        amax_bits = max(amax_bits, __float_as_uint(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]))));
+      continue;
+    }
+    if (rht_out && valid) {
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        *reinterpret_cast<float4 *>(rht_out + (t0 + k) * cols + c0) =
+            make_float4(lo[k].x, lo[k].y, hi[k].x, hi[k].y);
+    }
+    uint32_t sbyte[4];
+    float f[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      sbyte[j] = nvfp4_scale_code(m[j], ts.enc);
+      f[j] = rtab[sbyte[j]];
+    }
+
+    // ---- encode -----------------------------------------------------------------
+    uint32_t w[4][2];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      lo[k] = mul2(lo[k], make_float2(f[0], f[1]));
+      hi[k] = mul2(hi[k], make_float2(f[2], f[3]));
+    }
+    if (SR) {
+      // element (t, c) draws from the Philox call (t * cols + c) / 8, which
+      // covers 8 columns = this lane's quad and its neighbour's (lane ^ 8):
+      // the even quad computes tokens 0..7, the odd one tokens 8..15, and each
+      // sends the other the two words of its half
+      const int half = cq & 1;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) w[j][0] = w[j][1] = 0u;
+      uint32_t chain = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int k = i + 8 * half;
+        // `chain` is zero, but opaque to the compiler: it makes each Philox call
+        // wait for the previous iteration, so only one call's state is live
+        uint32_t dep;
+        asm volatile("and.b32 %0, %1, 0;" : "=r"(dep) : "r"(chain));
+        const uint64_t gidx =
+            (static_cast<uint64_t>(t0 + k) * static_cast<uint64_t>(cols) +
+             static_cast<uint64_t>(c0 - 4 * half)) / 8 + dep;
+        // the key is re-read through an opaque move so that the ten round keys
+        // are formed per call instead of being held in twenty registers
+        uint32_t key0, key1;
+        asm volatile("mov.b32 %0, %1;" : "=r"(key0) : "r"(static_cast<uint32_t>(seed)));
+        asm volatile("mov.b32 %0, %1;" : "=r"(key1) : "r"(static_cast<uint32_t>(seed >> 32)));
+        const U32x4 b = philox4x32_10(U32x4{static_cast<uint32_t>(gidx),
+                                            static_cast<uint32_t>(gidx >> 32), 0u, 0u},
+                                      key0, key1);
+        // words 0,1 serve the even quad (columns 0-3), words 2,3 the odd quad
+        const uint32_t keep0 = half ? b.z : b.x, keep1 = half ? b.w : b.y;
+        const uint32_t send0 = half ? b.x : b.z, send1 = half ? b.y : b.w;
+        const uint32_t got0 = __shfl_xor_sync(0xFFFFFFFFu, send0, 8);
+        const uint32_t got1 = __shfl_xor_sync(0xFFFFFFFFu, send1, 8);
+        // this lane computed token i + 8 half, the partner token i + 8 (1 - half):
+        // the words of token i and of token i + 8
+        const uint32_t ti0 = half ? got0 : keep0, ti1 = half ? got1 : keep1;
+        const uint32_t tj0 = half ? keep0 : got0, tj1 = half ? keep1 : got1;
+        const float vi[4] = {lo[i].x, lo[i].y, hi[i].x, hi[i].y};
+        const float vj[4] = {lo[i + 8].x, lo[i + 8].y, hi[i + 8].x, hi[i + 8].y};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t wi = (j >> 1) ? ti1 : ti0, wj = (j >> 1) ? tj1 : tj0;
+          const uint32_t ui = (j & 1) ? (wi >> 16) : (wi & 0xFFFFu);
+          const uint32_t uj = (j & 1) ? (wj >> 16) : (wj & 0xFFFFu);
+          w[j][0] |= e2m1_sr_bits(vi[j], ui) << (4 * i);
+          w[j][1] |= e2m1_sr_bits(vj[j], uj) << (4 * i);
+        }
+        chain = b.x;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) w[j][0] = w[j][1] = 0u;
+#pragma unroll
+      for (int k = 0; k < 16; k += 2) {
+        const uint32_t sh = 8 * ((k >> 1) & 3);
+        w[0][k >> 3] |= e2m1x2(lo[k].x, lo[k + 1].x) << sh;
+        w[1][k >> 3] |= e2m1x2(lo[k].y, lo[k + 1].y) << sh;
+        w[2][k >> 3] |= e2m1x2(hi[k].x, hi[k + 1].x) << sh;
+        w[3][k >> 3] |= e2m1x2(hi[k].y, hi[k + 1].y) << sh;
+      }
+    }
+    if (valid) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        *reinterpret_cast<uint2 *>(q_t + (c0 + j) * (tokens / 2) + t0 / 2) =
+            make_uint2(w[j][0], w[j][1]);
+        sf_t[scale_offset(c0 + j, t0 / 16, tokens / 16, scale_layout)] =
+            static_cast<uint8_t>(sbyte[j]);
+      }
     }
   }
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int id = t + kThreads * j;
-    const int cc = id >> 3, b = id & 7;
-    const int64_t col = c0 + cc, blk = t0 / 16 + b;
-    if (col < cols && blk * 16 < tokens)
-      sf_t[scale_offset(col, blk, tokens / 16, scale_layout)] = s.sc[cc][b];
+  if (AMAX_ONLY) {
+    amax_bits = __reduce_max_sync(0xFFFFFFFFu, amax_bits);
+    if (lane == 0) atomicMax(amax_out, amax_bits);
   }
+}
+
+template <typename T, int N, bool SR, bool AMAX_ONLY>
+cudaError_t launch_k(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint64_t seed,
+                     const float *amax, float *s_dec_out, unsigned *amax_out, uint8_t *q_t,
+                     uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L) {
+  const void *kern = reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY>);
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess ||
+        per_sm < 1) {
+      cudaGetLastError();
+      per_sm = 1;
+    }
+  }
+  const int64_t ntiles = ((cols + 15) / 16) * ((tokens + 127) / 128);
+  const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
+  const int64_t want = (ntiles + kWarps - 1) / kWarps;
+  const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+  rht_kernel<T, N, SR, AMAX_ONLY><<<grid, kThreads, 0, L.stream>>>(
+      dy, tokens, cols, ld, seed, amax, s_dec_out, amax_out, q_t, sf_t, scale_layout, rht_out);
+  return cudaGetLastError();
 }
 
 template <typename T, int N>
 cudaError_t launch_n(const T *dy, int64_t tokens, int64_t cols, int64_t ld, int round,
                      uint64_t seed, const float *amax, float *s_dec_out, unsigned *amax_out,
                      uint8_t *q_t, uint8_t *sf_t, int scale_layout, float *rht_out,
-                     bool amax_only, cudaStream_t stream) {
-  dim3 grid(static_cast<unsigned>((cols + kTC - 1) / kTC),
-            static_cast<unsigned>((tokens + kTT - 1) / kTT));
+                     bool amax_only, const Launch &L) {
   if (amax_only)
-    rht_kernel<T, N, false, true><<<grid, kThreads, 0, stream>>>(
-        dy, tokens, cols, ld, seed, nullptr, nullptr, amax_out, nullptr, nullptr, 0, nullptr);
-  else if (round == FP4Q_SR)
-    rht_kernel<T, N, true, false><<<grid, kThreads, 0, stream>>>(
-        dy, tokens, cols, ld, seed, amax, s_dec_out, nullptr, q_t, sf_t, scale_layout, rht_out);
-  else
-    rht_kernel<T, N, false, false><<<grid, kThreads, 0, stream>>>(
-        dy, tokens, cols, ld, seed, amax, s_dec_out, nullptr, q_t, sf_t, scale_layout, rht_out);
-  return cudaGetLastError();
+    return launch_k<T, N, false, true>(dy, tokens, cols, ld, seed, nullptr, nullptr, amax_out,
+                                       nullptr, nullptr, 0, nullptr, L);
+  if (round == FP4Q_SR)
+    return launch_k<T, N, true, false>(dy, tokens, cols, ld, seed, amax, s_dec_out, nullptr, q_t,
+                                       sf_t, scale_layout, rht_out, L);
+  return launch_k<T, N, false, false>(dy, tokens, cols, ld, seed, amax, s_dec_out, nullptr, q_t,
+                                      sf_t, scale_layout, rht_out, L);
 }
 
 template <typename T>
 cudaError_t launch_t(const void *dy, int64_t tokens, int64_t cols, int64_t ld, int n, int round,
                      uint64_t seed, const float *amax, float *s_dec_out, unsigned *amax_out,
                      uint8_t *q_t, uint8_t *sf_t, int scale_layout, float *rht_out,
-                     bool amax_only, cudaStream_t stream) {
+                     bool amax_only, const Launch &L) {
   const T *p = static_cast<const T *>(dy);
   if (n == 16)
     return launch_n<T, 16>(p, tokens, cols, ld, round, seed, amax, s_dec_out, amax_out, q_t, sf_t,
-                           scale_layout, rht_out, amax_only, stream);
+                           scale_layout, rht_out, amax_only, L);
   return launch_n<T, 128>(p, tokens, cols, ld, round, seed, amax, s_dec_out, amax_out, q_t, sf_t,
-                          scale_layout, rht_out, amax_only, stream);
+                          scale_layout, rht_out, amax_only, L);
 }
 
 }  // namespace
@@ -314,9 +355,9 @@ cudaError_t launch_rht_amax(const void *dy, int dtype, int64_t tokens, int64_t c
   unsigned *out = reinterpret_cast<unsigned *>(amax_out);
   if (dtype == FP4Q_BF16)
     return launch_t<__nv_bfloat16>(dy, tokens, cols, ld, n, 0, seed, nullptr, nullptr, out,
-                                   nullptr, nullptr, 0, nullptr, true, L.stream);
+                                   nullptr, nullptr, 0, nullptr, true, L);
   return launch_t<float>(dy, tokens, cols, ld, n, 0, seed, nullptr, nullptr, out, nullptr,
-                         nullptr, 0, nullptr, true, L.stream);
+                         nullptr, 0, nullptr, true, L);
 }
 
 cudaError_t launch_rht_quant(const void *dy, int dtype, int64_t tokens, int64_t cols,
@@ -325,9 +366,9 @@ cudaError_t launch_rht_quant(const void *dy, int dtype, int64_t tokens, int64_t 
                              float *rht_out, const Launch &L) {
   if (dtype == FP4Q_BF16)
     return launch_t<__nv_bfloat16>(dy, tokens, cols, ld, n, round, seed, amax, s_dec_out,
-                                   nullptr, q_t, sf_t, scale_layout, rht_out, false, L.stream);
+                                   nullptr, q_t, sf_t, scale_layout, rht_out, false, L);
   return launch_t<float>(dy, tokens, cols, ld, n, round, seed, amax, s_dec_out, nullptr, q_t,
-                         sf_t, scale_layout, rht_out, false, L.stream);
+                         sf_t, scale_layout, rht_out, false, L);
 }
 
 }  // namespace fp4q

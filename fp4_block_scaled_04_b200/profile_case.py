@@ -1,0 +1,87 @@
+"""Run one fp4q kernel on one seeded workload, for profilers.
+
+    python -m fp4_block_scaled_04_b200.profile_case --op nvfp4_rowcol \\
+        --rows 16384 --cols 8192 --iters 3
+
+Inputs are generated on the host from the workload generators (same value
+distributions as the benchmark, any size), copied to cuda:0, the tensor amax
+is computed once, then the kernel under study runs ``--warmup`` times and
+``--iters`` times more, with a device synchronize at the end.  Each of those
+runs is exactly one launch of the kernel named by ``--op`` (the amax
+pre-pass is outside them), so a profiler can skip the warm-up launches and
+capture the rest.
+"""
+from __future__ import annotations
+
+import argparse
+import sys
+
+import torch
+
+import fp4_block_scaled_04_b200 as fq
+from fp4_block_scaled_04_b200 import workloads
+
+OPS = ["amax", "nvfp4_row", "nvfp4_rowcol", "mxfp4_rowcol", "2d", "rht16_sr", "rht128_sr",
+       "rht16_rne", "rht128_rne", "if4", "if4_dequant"]
+
+
+def make(op: str, rows: int, cols: int, dev):
+    sw = fq.SCALE_SWIZZLED if rows % 128 == 0 else fq.SCALE_LINEAR
+    if op in ("amax", "nvfp4_row", "nvfp4_rowcol", "mxfp4_rowcol"):
+        x = workloads.activation(rows=rows, cols=cols).to(dev)
+        if op == "amax":
+            out = torch.empty(1, device=dev)
+            return lambda: fq.fp4q_amax(x, out=out)
+        a = fq.fp4q_amax(x)
+        if op == "nvfp4_row":
+            o = fq.fp4q_quantize_nvfp4(x, layouts=fq.ROWWISE, amax=a, scale_layout=sw)
+            return lambda: fq.fp4q_quantize_nvfp4(x, layouts=fq.ROWWISE, amax=a, scale_layout=sw, out=o)
+        if op == "nvfp4_rowcol":
+            o = fq.fp4q_quantize_nvfp4(x, layouts=3, amax=a, scale_layout=sw)
+            return lambda: fq.fp4q_quantize_nvfp4(x, layouts=3, amax=a, scale_layout=sw, out=o)
+        o = fq.fp4q_quantize_mxfp4(x, layouts=3, scale_layout=sw)
+        return lambda: fq.fp4q_quantize_mxfp4(x, layouts=3, scale_layout=sw, out=o)
+    if op == "2d":
+        w = workloads.weight(rows=rows, cols=cols).to(dev)
+        a = fq.fp4q_amax(w)
+        o = fq.fp4q_quantize_2d(w, amax=a)
+        return lambda: fq.fp4q_quantize_2d(w, amax=a, out=o)
+    if op.startswith("rht"):
+        n = 16 if op.startswith("rht16") else 128
+        rnd = fq.SR if op.endswith("sr") else fq.RNE
+        g = workloads.gradient(tokens=rows, cols=cols).to(dev)
+        a = fq.fp4q_rht_amax(g, n)
+        o = fq.fp4q_quantize_rht_sr(g, n, round=rnd, amax_rht=a, scale_layout=sw)
+        return lambda: fq.fp4q_quantize_rht_sr(g, n, round=rnd, amax_rht=a, scale_layout=sw, out=o)
+    if op in ("if4", "if4_dequant"):
+        x = workloads.if4_blocks(rows=rows, cols=cols).to(dev)
+        a = fq.fp4q_amax(x)
+        o = fq.fp4q_quantize_if4(x, amax=a, scale_layout=sw)
+        if op == "if4":
+            return lambda: fq.fp4q_quantize_if4(x, amax=a, scale_layout=sw, out=o)
+        y = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+        return lambda: fq.fp4q_dequantize(fq.FMT_IF4, o["q"], o["sf"], rows, cols,
+                                          tensor_scale=o["s_dec"], scale_layout=sw, out=y)
+    raise ValueError(op)
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--op", choices=OPS, required=True)
+    ap.add_argument("--rows", type=int, required=True)
+    ap.add_argument("--cols", type=int, required=True)
+    ap.add_argument("--warmup", type=int, default=1)
+    ap.add_argument("--iters", type=int, default=3)
+    a = ap.parse_args(argv)
+    dev = torch.device("cuda", 0)
+    run = make(a.op, a.rows, a.cols, dev)
+    torch.cuda.synchronize(dev)
+    for _ in range(a.warmup + a.iters):
+        run()
+    torch.cuda.synchronize(dev)
+    print(f"profile_case {a.op} {a.rows}x{a.cols}: {a.warmup} warm-up + {a.iters} launches done")
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -245,7 +245,7 @@ def test_rht16_ragged_tokens(orc):
 
 @pytest.mark.parametrize("n", [16, 128])
 def test_rht_amax_and_fp32_input(orc, n):
-    dy = randmat(256, 64, torch.float32, seed=23, scale_spread=False)
+    dy = randmat(256, 128, torch.float32, seed=23, scale_spread=False)
     a = fq.fp4q_rht_amax(dy.to(DEV), n, seed=9)
     t = orc.rht(bits(dy), n, 9)
     assert_same("amax_rht", host(a), np.array([np.abs(t).max()], np.float32))

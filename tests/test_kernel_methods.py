@@ -1,0 +1,52 @@
+"""Host-side checks of arithmetic shortcuts the CUDA kernels take (CPU only).
+
+The kernels are compared with the oracle bit for bit on the GPU; these tests
+pin the shortcuts themselves over every input they can meet, which no finite
+GPU test can enumerate.
+"""
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+@pytest.fixture(scope="module")
+def div6_exe(tmp_path_factory):
+    exe = str(tmp_path_factory.mktemp("div6") / "div6_check")
+    flags = ["-O2", "-ffp-contract=off"]
+    # use the hardware FMA when the host has one (fmaf is correctly rounded either way)
+    probe = subprocess.run(["gcc", "-mfma", "-x", "c", "-", "-o", "/dev/null"],
+                           input="int main(){return 0;}", text=True, capture_output=True)
+    if probe.returncode == 0:
+        flags.append("-mfma")
+    subprocess.check_call(["gcc", *flags, os.path.join(HERE, "div6_check.c"), "-o", exe, "-lm"])
+    return exe
+
+
+def test_division_by_six_is_the_ieee_quotient(div6_exe):
+    """Markstein's corrected product equals RN(y/6) for every float y >= 2^-125
+    (checked over all finite non-negative bit patterns); below that the
+    quotient is subnormal and both round to E4M3 code 0."""
+    out = subprocess.run([div6_exe, "0", "0x7F800000"], capture_output=True, text=True,
+                         check=True).stdout.split()
+    bad, worst = int(out[0]), float(out[1])
+    assert worst < 2.0 ** -125, worst
+    assert bad < (1 << 24)                  # only the subnormal-quotient range differs
+
+
+def test_magic_number_rounding_is_round_half_even():
+    """IF4's INT4 step: RN(t + 1.5*2^23) - 1.5*2^23 == rint(t) and the low four
+    bits of the sum are rint(t) in two's complement, for |t| < 7.5."""
+    t = np.concatenate([np.linspace(-7.5, 7.5, 200_001, dtype=np.float32)[1:-1],
+                        np.arange(-7, 8, dtype=np.float32) + np.float32(0.5),
+                        np.arange(-7, 8, dtype=np.float32) - np.float32(0.5)])
+    t = t[np.abs(t) < 7.5]
+    magic = np.float32(12582912.0)
+    s = (t + magic).astype(np.float32)
+    k = (s - magic).astype(np.float32)
+    assert np.array_equal(k, np.rint(t))
+    low = s.view(np.uint32) & 0xF
+    assert np.array_equal(low, (np.rint(t).astype(np.int64) & 0xF).astype(np.uint32))
