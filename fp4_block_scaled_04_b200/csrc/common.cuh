@@ -80,6 +80,18 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
   return r;
 }
 
+// Four floats -> four nibbles in the low 16 bits, f0 in bits 0..3.
+__device__ __forceinline__ uint32_t e2m1x4(float f0, float f1, float f2, float f3) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1;\n\t.reg .b16 h;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "mov.b16 h, {b0, b1};\n\t"
+      "cvt.u32.u16 %0, h;\n\t}"
+      : "=r"(r) : "f"(f0), "f"(f1), "f"(f2), "f"(f3));
+  return r;
+}
+
 // E2M1 magnitude of a 3-bit code: 0, .5, 1, 1.5, 2, 3, 4, 6.
 __device__ __forceinline__ float e2m1_magnitude(uint32_t c3) {
   // codes 2..7 are normal: exponent (c3 >> 1) - 1, one mantissa bit (c3 & 1)
@@ -199,6 +211,24 @@ __device__ __forceinline__ int e8m0_exponent(float m, int mode) {
     }
   }
   return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// Biased E8M0 exponent (e + 127, clamped to [0, 254]) of a block with
+// maximum m, as e8m0_exponent, with the common case -- a normal quotient
+// RN(m/6) -- done by carries on the bit pattern: adding 0x3FFFFF plus the
+// exponent's parity bit rounds to the nearest power of two with ties to the
+// even exponent (RNE mode); adding 0x7FFFFF rounds up (CEIL mode).
+__device__ __forceinline__ uint32_t e8m0_biased(float m, int mode) {
+  if (mode == FP4Q_E8M0_OCP_FLOOR || !(m >= 7.1e-38f))   // OCP rule, or a subnormal quotient
+    return static_cast<uint32_t>(e8m0_exponent(m, mode) + 127);
+  const uint32_t b = __float_as_uint(div6(m));
+  const uint32_t add = mode == FP4Q_E8M0_CEIL ? 0x7FFFFFu : 0x3FFFFFu + ((b >> 23) & 1u);
+  return min((b + add) >> 23, 254u);
+}
+
+// 2^-(byte - 127) as a float for a biased E8M0 exponent byte.
+__device__ __forceinline__ float e8m0_inverse(uint32_t byte) {
+  return byte == 254u ? __uint_as_float(0x00400000u) : __uint_as_float((254u - byte) << 23);
 }
 
 // 2^-e as a float, e in [-127, 127] (2^-127 is subnormal, the rest normal).

@@ -150,9 +150,8 @@ rowwise_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
       uint32_t sbyte;
       float f;
       if (MX) {
-        const int e = e8m0_exponent(m, e8m0_mode);
-        sbyte = static_cast<uint32_t>(e + 127);
-        f = exp2_neg(e);
+        sbyte = e8m0_biased(m, e8m0_mode);
+        f = e8m0_inverse(sbyte);
       } else {
         sbyte = nvfp4_scale_code(m, ts.enc);
         f = rtab[sbyte];
@@ -226,6 +225,27 @@ __device__ __forceinline__ float chunk_rowmax(uint4 u) {
                fmaxf(fabsf(__uint_as_float(u.z)), fabsf(__uint_as_float(u.w))));
 }
 
+// packed |x| maxima of rows k and k+1 of a BF16 chunk pair -> (M_k, M_k+1)
+__device__ __forceinline__ uint32_t rowpair_max_bf16(uint4 a, uint4 b) {
+  const uint32_t ma = maxabs_bf16x2(maxabs_bf16x2(a.x, a.y), maxabs_bf16x2(a.z, a.w));
+  const uint32_t mb = maxabs_bf16x2(maxabs_bf16x2(b.x, b.y), maxabs_bf16x2(b.z, b.w));
+  // (lo_a, lo_b) and (hi_a, hi_b)
+  return maxabs_bf16x2(__byte_perm(ma, mb, 0x5410), __byte_perm(ma, mb, 0x7632));
+}
+
+template <typename T, bool MX>
+__device__ __forceinline__ uint32_t block_scale(float m, const TensorScale &ts, const float *rtab,
+                                                int mode, float &f) {
+  if (MX) {
+    const uint32_t be = e8m0_biased(m, mode);
+    f = e8m0_inverse(be);
+    return be;
+  }
+  const uint32_t code = nvfp4_scale_code(m, ts.enc);
+  f = rtab[code];
+  return code;
+}
+
 template <typename T, bool MX, bool SR>
 __global__ void __launch_bounds__(kRCThreads)
 rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, unsigned layouts,
@@ -250,6 +270,7 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
   const int64_t tiles_c = (cols + G::WC - 1) / G::WC;
   const int64_t ntiles = tiles_c * ((rows + G::WR - 1) / G::WR);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kRCThreads / 32);
+  const bool swz = scale_layout == FP4Q_SCALE_SWIZZLED_128x4;
   for (int64_t tile = static_cast<int64_t>(blockIdx.x) * (kRCThreads / 32) + (threadIdx.x >> 5);
        tile < ntiles; tile += nwarps) {
     const int64_t tr = tile / tiles_c, tc = tile - tr * tiles_c;
@@ -263,12 +284,25 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
 
     // ---- pass 1: block maxima --------------------------------------------
     float rmax[16];
+    if (sizeof(T) == 2) {
 #pragma unroll
-    for (int k = 0; k < 16; ++k) rmax[k] = chunk_rowmax<T>(d[k]);
+      for (int k = 0; k < 16; k += 2) {
+        uint32_t pm = rowpair_max_bf16(d[k], d[k + 1]);
 #pragma unroll
-    for (int o = 1; o < GR; o <<= 1)
+        for (int o = 1; o < GR; o <<= 1) pm = maxabs_bf16x2(pm, __shfl_xor_sync(0xFFFFFFFFu, pm, o));
+        pm &= 0x7FFF7FFFu;
+        rmax[k] = __uint_as_float(pm << 16);
+        rmax[k + 1] = __uint_as_float(pm & 0xFFFF0000u);
+      }
+    } else {
 #pragma unroll
-      for (int k = 0; k < 16; ++k) rmax[k] = fmaxf(rmax[k], __shfl_xor_sync(0xFFFFFFFFu, rmax[k], o));
+      for (int k = 0; k < 16; ++k) rmax[k] = chunk_rowmax<T>(d[k]);
+#pragma unroll
+      for (int o = 1; o < GR; o <<= 1)
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          rmax[k] = fmaxf(rmax[k], __shfl_xor_sync(0xFFFFFFFFu, rmax[k], o));
+    }
     uint32_t cm[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int k = 0; k < 16; ++k) chunk_colmax<T>(d[k], cm);
@@ -293,111 +327,99 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
     float rf[16], cf[CPT];
     uint32_t rbyte[16], cbyte[CPT];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      if (MX) {
-        const int e = e8m0_exponent(rmax[k], e8m0_mode);
-        rbyte[k] = static_cast<uint32_t>(e + 127);
-        rf[k] = exp2_neg(e);
-      } else {
-        rbyte[k] = nvfp4_scale_code(rmax[k], ts.enc);
-        rf[k] = rtab[rbyte[k]];
-      }
-    }
+    for (int k = 0; k < 16; ++k) rbyte[k] = block_scale<T, MX>(rmax[k], ts, rtab, e8m0_mode, rf[k]);
 #pragma unroll
-    for (int j = 0; j < CPT; ++j) {
-      if (MX) {
-        const int e = e8m0_exponent(cmax[j], e8m0_mode);
-        cbyte[j] = static_cast<uint32_t>(e + 127);
-        cf[j] = exp2_neg(e);
-      } else {
-        cbyte[j] = nvfp4_scale_code(cmax[j], ts.enc);
-        cf[j] = rtab[cbyte[j]];
-      }
-    }
+    for (int j = 0; j < CPT; ++j) cbyte[j] = block_scale<T, MX>(cmax[j], ts, rtab, e8m0_mode, cf[j]);
     if (valid && do_row && (cc % GR) == 0) {
+      // rows r0..r0+15 of one block column: in the swizzled layout they are
+      // 16 bytes apart (r0 is a multiple of 16), in the linear one cols/BLK
+      const int64_t base = scale_offset(r0, c0 / BLK, cols / BLK, scale_layout);
+      const int64_t step = swz ? 16 : cols / BLK;
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        sf_row[scale_offset(r0 + k, c0 / BLK, cols / BLK, scale_layout)] =
-            static_cast<uint8_t>(rbyte[k]);
+      for (int k = 0; k < 16; ++k) sf_row[base + k * step] = static_cast<uint8_t>(rbyte[k]);
     }
     if (valid && do_col && (!MX || (band & 1) == 0)) {
+      const int64_t base = scale_offset(c0, r0 / BLK, rows / BLK, scale_layout);
+      const int64_t step = swz ? 16 : rows / BLK;
 #pragma unroll
-      for (int j = 0; j < CPT; ++j)
-        sf_col[scale_offset(c0 + j, r0 / BLK, rows / BLK, scale_layout)] =
-            static_cast<uint8_t>(cbyte[j]);
+      for (int j = 0; j < CPT; ++j) sf_col[base + j * step] = static_cast<uint8_t>(cbyte[j]);
     }
 
-    // ---- pass 2: encode ------------------------------------------------------
+    // ---- pass 2: encode, four rows at a time ----------------------------------
     uint32_t colw[CPT][2];
 #pragma unroll
-    for (int j = 0; j < CPT; ++j) colw[j][0] = colw[j][1] = 0u;
+    for (int q4 = 0; q4 < 4; ++q4) {
+      float v[4][CPT];
 #pragma unroll
-    for (int k = 0; k < 16; k += 2) {
-      float a[CPT], b[CPT];
-      unpack_chunk<T>(d[k], a);
-      unpack_chunk<T>(d[k + 1], b);
-      uint32_t ua[CPT], ub[CPT];
+      for (int i = 0; i < 4; ++i) unpack_chunk<T>(d[4 * q4 + i], v[i]);
+      uint32_t u[4][CPT];
       if (SR) {
         // one Philox call covers the 8 columns of a row from a multiple of 8
-        const uint64_t ia = static_cast<uint64_t>((r0 + k) * cols + c0);
-        const uint64_t ib = ia + static_cast<uint64_t>(cols);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint64_t i = h == 0 ? ia : ib;
-          const uint64_t g = i / 8;
-          const U32x4 bits = philox(K, static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u);
+        for (int i = 0; i < 4; ++i) {
+          const uint64_t idx = static_cast<uint64_t>((r0 + 4 * q4 + i) * cols + c0);
+          const uint64_t gi = idx / 8;
+          const U32x4 bits = philox(K, static_cast<uint32_t>(gi), static_cast<uint32_t>(gi >> 32), 0u, 0u);
           const uint32_t words[4] = {bits.x, bits.y, bits.z, bits.w};
 #pragma unroll
           for (int j = 0; j < CPT; ++j) {
-            const int e = static_cast<int>(i % 8) + j;
-            const uint32_t u16 = (e & 1) ? (words[(e >> 1) & 3] >> 16) : (words[(e >> 1) & 3] & 0xFFFFu);
-            if (h == 0) ua[j] = u16; else ub[j] = u16;
+            const int e = static_cast<int>(idx % 8) + j;
+            const uint32_t wv = words[(e >> 1) & 3];
+            u[i][j] = (e & 1) ? (wv >> 16) : (wv & 0xFFFFu);
           }
         }
       }
       if (do_row) {
-        uint32_t wa = 0u, wb = 0u;
-        if (SR) {
 #pragma unroll
-          for (int j = 0; j < CPT; ++j) {
-            wa |= e2m1_sr_bits(__fmul_rn(a[j], rf[k]), ua[j]) << (4 * j);
-            wb |= e2m1_sr_bits(__fmul_rn(b[j], rf[k + 1]), ub[j]) << (4 * j);
-          }
-        } else {
+        for (int i = 0; i < 4; ++i) {
+          const int k = 4 * q4 + i;
+          uint32_t wr = 0u;
+          if (SR) {
 #pragma unroll
-          for (int j = 0; j < CPT; j += 2) {
-            const float2 pa = mul2(make_float2(a[j], a[j + 1]), make_float2(rf[k], rf[k]));
-            const float2 pb = mul2(make_float2(b[j], b[j + 1]), make_float2(rf[k + 1], rf[k + 1]));
-            wa |= e2m1x2(pa.x, pa.y) << (4 * j);
-            wb |= e2m1x2(pb.x, pb.y) << (4 * j);
-          }
-        }
-        if (valid) {
-          uint8_t *qa = q_row + (r0 + k) * (cols / 2) + c0 / 2;
-          if (CPT == 8) {
-            *reinterpret_cast<uint32_t *>(qa) = wa;
-            *reinterpret_cast<uint32_t *>(qa + cols / 2) = wb;
+            for (int j = 0; j < CPT; ++j) wr |= e2m1_sr_bits(__fmul_rn(v[i][j], rf[k]), u[i][j]) << (4 * j);
           } else {
-            *reinterpret_cast<uint16_t *>(qa) = static_cast<uint16_t>(wa);
-            *reinterpret_cast<uint16_t *>(qa + cols / 2) = static_cast<uint16_t>(wb);
+            float t[8];
+#pragma unroll
+            for (int j = 0; j < CPT; j += 2) {
+              const float2 p = mul2(make_float2(v[i][j], v[i][j + 1]), make_float2(rf[k], rf[k]));
+              t[j] = p.x;
+              t[j + 1] = p.y;
+            }
+            wr = CPT == 8 ? e2m1x8(t) : e2m1x4(t[0], t[1], t[2 % CPT], t[3 % CPT]);
+          }
+          if (valid) {
+            uint8_t *qa = q_row + (r0 + k) * (cols / 2) + c0 / 2;
+            if (CPT == 8) *reinterpret_cast<uint32_t *>(qa) = wr;
+            else *reinterpret_cast<uint16_t *>(qa) = static_cast<uint16_t>(wr);
           }
         }
       }
       if (do_col) {
 #pragma unroll
         for (int j = 0; j < CPT; j += 2) {
-          const float2 pa = mul2(make_float2(a[j], a[j + 1]), make_float2(cf[j], cf[j + 1]));
-          const float2 pb = mul2(make_float2(b[j], b[j + 1]), make_float2(cf[j], cf[j + 1]));
-          uint32_t b0, b1;
+          float2 p[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            p[i] = mul2(make_float2(v[i][j], v[i][j + 1]), make_float2(cf[j], cf[j + 1]));
+          uint32_t h0, h1;
           if (SR) {
-            b0 = e2m1_sr_bits(pa.x, ua[j]) | (e2m1_sr_bits(pb.x, ub[j]) << 4);
-            b1 = e2m1_sr_bits(pa.y, ua[j + 1]) | (e2m1_sr_bits(pb.y, ub[j + 1]) << 4);
+            h0 = h1 = 0u;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              h0 |= e2m1_sr_bits(p[i].x, u[i][j]) << (4 * i);
+              h1 |= e2m1_sr_bits(p[i].y, u[i][j + 1]) << (4 * i);
+            }
           } else {
-            b0 = e2m1x2(pa.x, pb.x);       // column j: rows k (low), k + 1 (high)
-            b1 = e2m1x2(pa.y, pb.y);       // column j + 1
+            h0 = e2m1x4(p[0].x, p[1].x, p[2].x, p[3].x);    // column j, rows 4q4..4q4+3
+            h1 = e2m1x4(p[0].y, p[1].y, p[2].y, p[3].y);    // column j + 1
           }
-          colw[j][k >> 3] |= b0 << (8 * ((k >> 1) & 3));
-          colw[j + 1][k >> 3] |= b1 << (8 * ((k >> 1) & 3));
+          if (q4 & 1) {
+            colw[j][q4 >> 1] |= h0 << 16;
+            colw[j + 1][q4 >> 1] |= h1 << 16;
+          } else {
+            colw[j][q4 >> 1] = h0;
+            colw[j + 1][q4 >> 1] = h1;
+          }
         }
       }
     }

@@ -10,15 +10,19 @@
 // Register tiles: a thread owns 4 columns x 16 consecutive tokens (one
 // 16-token group of the transform and one quantization block per column); a
 // warp owns 128 tokens x 16 columns (lane = group + 8 * column quad).
-//   * sign flip and the butterfly stages h = 1, 2, 4, 8 run in registers on
-//     f32x2 pairs of columns;
+//   * each warp streams its tiles through a two-stage cp.async buffer in
+//     shared memory, so the next tile is in flight while this one computes;
+//     a lane copies exactly the chunks it later reads (no cross-lane sync);
+//   * the sign flip is one LOP3 per packed word, the butterfly stages
+//     h = 1, 2, 4, 8 run in registers on f32x2 column pairs;
 //   * for n = 128 the stages h = 16, 32, 64 combine the eight groups: the warp
-//     swaps values through an 8 KB shared buffer (XOR-swizzled so that both
-//     the write and the transposed read hit every bank once per wavefront),
-//     runs the three stages, and swaps back;
+//     swaps values through an 8 KB shared buffer (XOR-swizzled so the write
+//     and the transposed read both spread over all banks), runs the three
+//     stages and swaps back;
 //   * block maxima are in-thread; stochastic rounding needs one Philox call
 //     per token per 8 columns, which two lanes share (each computes half of
-//     the tokens and passes the other lane its 64 bits by shuffle);
+//     the tokens and passes the other lane its 64 bits by shuffle).  The ten
+//     Philox round keys and the 128 signs come in as kernel parameters;
 //   * dY^T codes leave as 8 lanes x 8 bytes = 64 contiguous bytes per column.
 #include "common.cuh"
 #include "launch.h"
@@ -28,25 +32,44 @@ namespace {
 
 constexpr int kThreads = 128;       // 4 warps
 constexpr int kWarps = kThreads / 32;
+constexpr int kUnits = 128 * 4 + 32;  // input chunks per buffer (16 tokens padded by 4)
 
-template <typename T>
-__device__ __forceinline__ void load4(const T *p, float (&v)[4]);
-template <>
-__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16 *p, float (&v)[4]) {
-  const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
-  v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
-}
-template <>
-__device__ __forceinline__ void load4<float>(const float *p, float (&v)[4]) {
-  const float4 u = __ldg(reinterpret_cast<const float4 *>(p));
-  v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+struct RhtParams {
+  uint32_t k0[10], k1[10];   // Philox4x32-10 round keys of the seed
+  uint32_t signs[4];         // bit k of word k/32: sign of token k of the diagonal
+};
+
+// Philox4x32-10 of the counter (c0, c1, 0, 0) with the caller's round keys
+__device__ __forceinline__ U32x4 philox_rk(const RhtParams &P, uint32_t c0, uint32_t c1) {
+  uint32_t c2 = 0u, c3 = 0u;
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c0;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c2;
+    const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ P.k0[i];
+    const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ P.k1[i];
+    c1 = static_cast<uint32_t>(p1);
+    c3 = static_cast<uint32_t>(p0);
+    c0 = n0;
+    c2 = n2;
+  }
+  return U32x4{c0, c1, c2, c3};
 }
 
-__device__ __forceinline__ float flip(float x, uint32_t bit) {
-  return __uint_as_float(__float_as_uint(x) ^ (bit << 31));
+// Stochastic rounding onto E2M1 by fixed-point grid coordinates (the same
+// rule as round-up iff u < t * 2^16): for |v| in [1, 6] the grid coordinate
+// is G * 2^22 = bits - 0x3F000000, so one carry decides u * 64 < frac; below
+// 1 the grid is uniform and C = ceil(|v| * 2^17) comes from rounding
+// |v| * 2^17 + 2^23 up.  Checked against the oracle by tests/sr_check.c.
+__device__ __forceinline__ uint32_t e2m1_sr_fast(float v, uint32_t u16) {
+  const uint32_t raw = __float_as_uint(v);
+  const uint32_t b = raw & 0x7FFFFFFFu;
+  const uint32_t code_a = min((b - 0x3EC00001u - (u16 << 6)) >> 22, 7u);
+  const float xu = __fmaf_ru(__uint_as_float(b), 131072.0f, 8388608.0f);
+  const uint32_t code_b = (__float_as_uint(xu) - 0x4AFF0001u - u16) >> 16;
+  return (b >= 0x3F800000u ? code_a : code_b) | ((raw >> 28) & 8u);
 }
 
-// one butterfly stage over 16 tokens of 4 columns held as two column pairs
 template <int H>
 __device__ __forceinline__ void stage(float2 (&lo)[16], float2 (&hi)[16]) {
 #pragma unroll
@@ -61,10 +84,9 @@ __device__ __forceinline__ void stage(float2 (&lo)[16], float2 (&hi)[16]) {
     }
 }
 
-// cross-group stage on 8 groups x 2 offsets: values u[g][o]
+// cross-group stage on (8 groups x 2 offsets) values, index 2 * group + offset
 template <int H>
 __device__ __forceinline__ void xstage(float2 (&lo)[16], float2 (&hi)[16]) {
-  // index = 2 * group + offset; stage pairs groups g and g + H
 #pragma unroll
   for (int g = 0; g < 8; ++g)
     if ((g & H) == 0)
@@ -80,21 +102,42 @@ __device__ __forceinline__ void xstage(float2 (&lo)[16], float2 (&hi)[16]) {
       }
 }
 
-// 16-byte chunk (token t, column quad q) of a warp's 128 x 16 FP32 buffer,
-// XOR-swizzled within each 128-byte line
-__device__ __forceinline__ int chunk(int t, int q) {
-  const int sw = ((t >> 4) ^ (t >> 1)) & 7;
-  return (t * 4 + q) ^ sw;
+template <typename T>
+__device__ __forceinline__ void async_copy(uint32_t dst, const T *src) {
+  if (sizeof(T) == 2)
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+struct TileCoord {
+  int64_t t0, c0;
+  bool valid;
+  __device__ __forceinline__ TileCoord(int64_t tile, int64_t tiles_c, int g, int cq,
+                                       int64_t tokens, int64_t cols) {
+    const int64_t tt = tile / tiles_c, tc = tile - tt * tiles_c;
+    t0 = tt * 128 + 16 * g;
+    c0 = tc * 16 + 4 * cq;
+    // a column quad is all-in or all-out (cols % 8 == 0); a 16-token group
+    // likewise (tokens % 16 == 0); for n = 128 all groups of a tile are in
+    valid = c0 < cols && t0 < tokens;
+  }
+};
 
 template <typename T, int N, bool SR, bool AMAX_ONLY>
 __global__ void __launch_bounds__(kThreads, 3)
-rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld, uint64_t seed,
-           const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
+rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
+           const RhtParams P, const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
            unsigned *__restrict__ amax_out, uint8_t *__restrict__ q_t,
            uint8_t *__restrict__ sf_t, int scale_layout, float *__restrict__ rht_out) {
+  constexpr int UB = 4 * sizeof(T);                       // bytes per input chunk
+  constexpr int IN_BYTES = 2 * kUnits * UB;               // two stages
+  constexpr int WARP_BYTES = IN_BYTES + (N == 128 ? 128 * 16 * 4 : 0);
+  extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float rtab[128];
-  __shared__ __align__(16) float4 xbuf[N == 128 ? kWarps * 128 * 4 : 1];
   TensorScale ts{1.0f, 1.0f};
   if (!AMAX_ONLY) {
     ts = tensor_scale(*amax_ptr);
@@ -102,42 +145,69 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld, u
     if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, g = lane & 7, cq = lane >> 3;
-  float4 *buf = xbuf + (N == 128 ? (threadIdx.x >> 5) * 512 : 0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane & 7, cq = lane >> 3;
+  uint8_t *wbase = smem + warp * WARP_BYTES;
+  const uint32_t in_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbase));
+  float4 *xbuf = reinterpret_cast<float4 *>(wbase + IN_BYTES);
+  const int my_unit = 68 * g + cq;                        // chunk (16 g + k, cq) = my_unit + 4 k
 
-  // the random diagonal: bit k of Philox(counter (0,0,1,0), key seed)
-  const U32x4 sw = philox4x32_10(U32x4{0u, 0u, 1u, 0u}, static_cast<uint32_t>(seed),
-                                 static_cast<uint32_t>(seed >> 32));
-  uint32_t signs;   // bit k: sign of token 16 g + k of a 128-token group (bit k of a 16-group)
+  // signs of this lane's 16 tokens
+  uint32_t signs;
   if (N == 16) {
-    signs = sw.x & 0xFFFFu;
+    signs = P.signs[0] & 0xFFFFu;
   } else {
-    const uint32_t word = (g >> 1) == 0 ? sw.x : (g >> 1) == 1 ? sw.y : (g >> 1) == 2 ? sw.z : sw.w;
-    signs = (word >> ((g & 1) * 16)) & 0xFFFFu;
+    const uint32_t w = (g >> 1) == 0 ? P.signs[0] : (g >> 1) == 1 ? P.signs[1]
+                     : (g >> 1) == 2 ? P.signs[2] : P.signs[3];
+    signs = (w >> ((g & 1) * 16)) & 0xFFFFu;
   }
   const float cn = N == 16 ? 0.25f : __frsqrt_rn(128.0f);
 
   const int64_t tiles_c = (cols + 15) / 16;
   const int64_t ntiles = tiles_c * ((tokens + 127) / 128);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
-  uint32_t amax_bits = 0u;
-  for (int64_t tile = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-       tile < ntiles; tile += nwarps) {
-    const int64_t tt = tile / tiles_c, tc = tile - tt * tiles_c;
-    const int64_t t0 = tt * 128 + 16 * g, c0 = tc * 16 + 4 * cq;
-    // a column quad is all-in or all-out (cols % 8 == 0); a 16-token group
-    // likewise (tokens % 16 == 0); for n = 128 all groups of a tile are in
-    const bool valid = c0 < cols && t0 < tokens;
+  int64_t tile = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
 
-    // ---- load, sign flip, stages h = 1..8 -----------------------------------
+  auto issue = [&](int64_t t, int st) {
+    const TileCoord tl(t, tiles_c, g, cq, tokens, cols);
+    if (tl.valid) {
+      const T *src = dy + tl.t0 * ld + tl.c0;
+      const uint32_t dst = in_s + static_cast<uint32_t>((st * kUnits + my_unit) * UB);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) async_copy<T>(dst + 4 * k * UB, src + k * ld);
+    }
+  };
+
+  uint32_t amax_bits = 0u;
+  if (tile < ntiles) issue(tile, 0);
+  async_commit();
+  for (int st = 0; tile < ntiles; tile += nwarps, st ^= 1) {
+    if (tile + nwarps < ntiles) issue(tile + nwarps, st ^ 1);
+    async_commit();
+    async_wait_1();
+    const TileCoord tl(tile, tiles_c, g, cq, tokens, cols);
+    const int64_t t0 = tl.t0, c0 = tl.c0;
+    const bool valid = tl.valid;
+
+    // ---- sign flip and stages h = 1, 2, 4, 8 ----------------------------------
     float2 lo[16], hi[16];     // columns (c0, c0+1) and (c0+2, c0+3) per token
+    const uint8_t *ib = wbase + (st * kUnits + my_unit) * UB;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
-      float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (valid) load4<T>(dy + (t0 + k) * ld + c0, v);
-      const uint32_t bit = (signs >> k) & 1u;
-      lo[k] = make_float2(flip(v[0], bit), flip(v[1], bit));
-      hi[k] = make_float2(flip(v[2], bit), flip(v[3], bit));
+      // 0 or 0xFFFFFFFF: token k's sign
+      const uint32_t m = static_cast<uint32_t>(static_cast<int32_t>(signs << (31 - k)) >> 31);
+      if (sizeof(T) == 2) {
+        uint2 w = valid ? *reinterpret_cast<const uint2 *>(ib + 4 * k * UB) : make_uint2(0u, 0u);
+        w.x ^= m & 0x80008000u;
+        w.y ^= m & 0x80008000u;
+        lo[k] = make_float2(bf16_lo(w.x), bf16_hi(w.x));
+        hi[k] = make_float2(bf16_lo(w.y), bf16_hi(w.y));
+      } else {
+        uint4 w = valid ? *reinterpret_cast<const uint4 *>(ib + 4 * k * UB)
+                        : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t s = m & 0x80000000u;
+        lo[k] = make_float2(__uint_as_float(w.x ^ s), __uint_as_float(w.y ^ s));
+        hi[k] = make_float2(__uint_as_float(w.z ^ s), __uint_as_float(w.w ^ s));
+      }
     }
     stage<1>(lo, hi);
     stage<2>(lo, hi);
@@ -145,17 +215,21 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld, u
     stage<8>(lo, hi);
 
     if (N == 128) {
-      // ---- stages h = 16, 32, 64 across the eight groups ----------------------
+      // ---- stages h = 16, 32, 64 across the eight groups ------------------------
+      // the 16-byte chunk of (token t, quad q) is 4t + q with its low three
+      // bits XORed with (t/16 ^ t/2) mod 8; s = q ^ g is the lane's part of it
+      const int s = cq ^ g;
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        buf[chunk(16 * g + k, cq)] = make_float4(lo[k].x, lo[k].y, hi[k].x, hi[k].y);
+      for (int k = 0; k < 16; ++k) {
+        const int ck = (4 * (k & 1)) ^ ((k >> 1) & 7);
+        xbuf[64 * g + 8 * (k >> 1) + (s ^ ck)] = make_float4(lo[k].x, lo[k].y, hi[k].x, hi[k].y);
+      }
       __syncwarp();
-      // now this lane takes in-group offsets 2g, 2g+1 of all eight groups
 #pragma unroll
       for (int gg = 0; gg < 8; ++gg)
 #pragma unroll
         for (int o = 0; o < 2; ++o) {
-          const float4 c = buf[chunk(16 * gg + 2 * g + o, cq)];
+          const float4 c = xbuf[64 * gg + 8 * g + (s ^ ((4 * o) ^ gg))];
           lo[2 * gg + o] = make_float2(c.x, c.y);
           hi[2 * gg + o] = make_float2(c.z, c.w);
         }
@@ -167,12 +241,14 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld, u
 #pragma unroll
         for (int o = 0; o < 2; ++o) {
           const int i = 2 * gg + o;
-          buf[chunk(16 * gg + 2 * g + o, cq)] = make_float4(lo[i].x, lo[i].y, hi[i].x, hi[i].y);
+          xbuf[64 * gg + 8 * g + (s ^ ((4 * o) ^ gg))] =
+              make_float4(lo[i].x, lo[i].y, hi[i].x, hi[i].y);
         }
       __syncwarp();
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
-        const float4 c = buf[chunk(16 * g + k, cq)];
+        const int ck = (4 * (k & 1)) ^ ((k >> 1) & 7);
+        const float4 c = xbuf[64 * g + 8 * (k >> 1) + (s ^ ck)];
         lo[k] = make_float2(c.x, c.y);
         hi[k] = make_float2(c.z, c.w);
       }
@@ -211,48 +287,34 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld, u
       sbyte[j] = nvfp4_scale_code(m[j], ts.enc);
       f[j] = rtab[sbyte[j]];
     }
-
-    // ---- encode -----------------------------------------------------------------
-    uint32_t w[4][2];
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       lo[k] = mul2(lo[k], make_float2(f[0], f[1]));
       hi[k] = mul2(hi[k], make_float2(f[2], f[3]));
     }
+
+    // ---- encode -----------------------------------------------------------------
+    uint32_t w[4][2];
     if (SR) {
-      // element (t, c) draws from the Philox call (t * cols + c) / 8, which
-      // covers 8 columns = this lane's quad and its neighbour's (lane ^ 8):
-      // the even quad computes tokens 0..7, the odd one tokens 8..15, and each
-      // sends the other the two words of its half
+      // element (t, c) draws from the Philox call (t * cols + c) / 8, covering
+      // this lane's quad and its neighbour's (lane ^ 8): the even quad computes
+      // tokens 0..7, the odd one 8..15, and each sends the other its half
       const int half = cq & 1;
+      const uint64_t row0 = (static_cast<uint64_t>(t0) * static_cast<uint64_t>(cols) +
+                             static_cast<uint64_t>(c0 - 4 * half)) / 8;
+      const uint64_t rstep = static_cast<uint64_t>(cols) / 8;
 #pragma unroll
       for (int j = 0; j < 4; ++j) w[j][0] = w[j][1] = 0u;
-      uint32_t chain = 0u;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int k = i + 8 * half;
-        // `chain` is zero, but opaque to the compiler: it makes each Philox call
-        // wait for the previous iteration, so only one call's state is live
-        uint32_t dep;
-        asm volatile("and.b32 %0, %1, 0;" : "=r"(dep) : "r"(chain));
-        const uint64_t gidx =
-            (static_cast<uint64_t>(t0 + k) * static_cast<uint64_t>(cols) +
-             static_cast<uint64_t>(c0 - 4 * half)) / 8 + dep;
-        // the key is re-read through an opaque move so that the ten round keys
-        // are formed per call instead of being held in twenty registers
-        uint32_t key0, key1;
-        asm volatile("mov.b32 %0, %1;" : "=r"(key0) : "r"(static_cast<uint32_t>(seed)));
-        asm volatile("mov.b32 %0, %1;" : "=r"(key1) : "r"(static_cast<uint32_t>(seed >> 32)));
-        const U32x4 b = philox4x32_10(U32x4{static_cast<uint32_t>(gidx),
-                                            static_cast<uint32_t>(gidx >> 32), 0u, 0u},
-                                      key0, key1);
+        const uint64_t gidx = row0 + static_cast<uint64_t>(i + 8 * half) * rstep;
+        const U32x4 b = philox_rk(P, static_cast<uint32_t>(gidx), static_cast<uint32_t>(gidx >> 32));
         // words 0,1 serve the even quad (columns 0-3), words 2,3 the odd quad
         const uint32_t keep0 = half ? b.z : b.x, keep1 = half ? b.w : b.y;
         const uint32_t send0 = half ? b.x : b.z, send1 = half ? b.y : b.w;
         const uint32_t got0 = __shfl_xor_sync(0xFFFFFFFFu, send0, 8);
         const uint32_t got1 = __shfl_xor_sync(0xFFFFFFFFu, send1, 8);
-        // this lane computed token i + 8 half, the partner token i + 8 (1 - half):
-        // the words of token i and of token i + 8
+        // this lane computed token i + 8 half, the partner token i + 8 (1 - half)
         const uint32_t ti0 = half ? got0 : keep0, ti1 = half ? got1 : keep1;
         const uint32_t tj0 = half ? keep0 : got0, tj1 = half ? keep1 : got1;
         const float vi[4] = {lo[i].x, lo[i].y, hi[i].x, hi[i].y};
@@ -262,21 +324,23 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld, u
           const uint32_t wi = (j >> 1) ? ti1 : ti0, wj = (j >> 1) ? tj1 : tj0;
           const uint32_t ui = (j & 1) ? (wi >> 16) : (wi & 0xFFFFu);
           const uint32_t uj = (j & 1) ? (wj >> 16) : (wj & 0xFFFFu);
-          w[j][0] |= e2m1_sr_bits(vi[j], ui) << (4 * i);
-          w[j][1] |= e2m1_sr_bits(vj[j], uj) << (4 * i);
+          w[j][0] += e2m1_sr_fast(vi[j], ui) << (4 * i);
+          w[j][1] += e2m1_sr_fast(vj[j], uj) << (4 * i);
         }
-        chain = b.x;
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) w[j][0] = w[j][1] = 0u;
+      for (int h = 0; h < 2; ++h) {
+        float a[8], b[8], c[8], d[8];
 #pragma unroll
-      for (int k = 0; k < 16; k += 2) {
-        const uint32_t sh = 8 * ((k >> 1) & 3);
-        w[0][k >> 3] |= e2m1x2(lo[k].x, lo[k + 1].x) << sh;
-        w[1][k >> 3] |= e2m1x2(lo[k].y, lo[k + 1].y) << sh;
-        w[2][k >> 3] |= e2m1x2(hi[k].x, hi[k + 1].x) << sh;
-        w[3][k >> 3] |= e2m1x2(hi[k].y, hi[k + 1].y) << sh;
+        for (int k = 0; k < 8; ++k) {
+          a[k] = lo[8 * h + k].x; b[k] = lo[8 * h + k].y;
+          c[k] = hi[8 * h + k].x; d[k] = hi[8 * h + k].y;
+        }
+        w[0][h] = e2m1x8(a);
+        w[1][h] = e2m1x8(b);
+        w[2][h] = e2m1x8(c);
+        w[3][h] = e2m1x8(d);
       }
     }
     if (valid) {
@@ -289,20 +353,60 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld, u
       }
     }
   }
+  async_wait_0();
   if (AMAX_ONLY) {
     amax_bits = __reduce_max_sync(0xFFFFFFFFu, amax_bits);
     if (lane == 0) atomicMax(amax_out, amax_bits);
   }
 }
 
+// host side: Philox4x32-10 (Salmon et al., SC'11) for the signs, and the
+// round keys the kernel consumes
+void host_philox(uint32_t c[4], uint32_t k0, uint32_t k1) {
+  for (int i = 0; i < 10; ++i) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c[0];
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c[2];
+    const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c[1] ^ k0;
+    const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c[3] ^ k1;
+    c[1] = static_cast<uint32_t>(p1);
+    c[3] = static_cast<uint32_t>(p0);
+    c[0] = n0;
+    c[2] = n2;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+}
+
+RhtParams make_params(uint64_t seed) {
+  RhtParams P;
+  uint32_t a = static_cast<uint32_t>(seed), b = static_cast<uint32_t>(seed >> 32);
+  for (int i = 0; i < 10; ++i) {
+    P.k0[i] = a;
+    P.k1[i] = b;
+    a += 0x9E3779B9u;
+    b += 0xBB67AE85u;
+  }
+  uint32_t c[4] = {0u, 0u, 1u, 0u};
+  host_philox(c, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+  for (int i = 0; i < 4; ++i) P.signs[i] = c[i];
+  return P;
+}
+
 template <typename T, int N, bool SR, bool AMAX_ONLY>
 cudaError_t launch_k(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint64_t seed,
                      const float *amax, float *s_dec_out, unsigned *amax_out, uint8_t *q_t,
                      uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L) {
+  constexpr int UB = 4 * sizeof(T);
+  constexpr int WARP_BYTES = 2 * kUnits * UB + (N == 128 ? 128 * 16 * 4 : 0);
+  constexpr int SMEM = kWarps * WARP_BYTES;
   const void *kern = reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY>);
   static int per_sm = 0;
   if (per_sm == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess ||
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
+        cudaSuccess)
+      return cudaGetLastError();
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, SMEM) !=
+            cudaSuccess ||
         per_sm < 1) {
       cudaGetLastError();
       per_sm = 1;
@@ -312,8 +416,9 @@ cudaError_t launch_k(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint
   const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
   const int64_t want = (ntiles + kWarps - 1) / kWarps;
   const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-  rht_kernel<T, N, SR, AMAX_ONLY><<<grid, kThreads, 0, L.stream>>>(
-      dy, tokens, cols, ld, seed, amax, s_dec_out, amax_out, q_t, sf_t, scale_layout, rht_out);
+  rht_kernel<T, N, SR, AMAX_ONLY><<<grid, kThreads, SMEM, L.stream>>>(
+      dy, tokens, cols, ld, make_params(seed), amax, s_dec_out, amax_out, q_t, sf_t, scale_layout,
+      rht_out);
   return cudaGetLastError();
 }
 

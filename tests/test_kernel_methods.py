@@ -37,16 +37,29 @@ def test_division_by_six_is_the_ieee_quotient(div6_exe):
     assert bad < (1 << 24)                  # only the subnormal-quotient range differs
 
 
-def test_magic_number_rounding_is_round_half_even():
-    """IF4's INT4 step: RN(t + 1.5*2^23) - 1.5*2^23 == rint(t) and the low four
-    bits of the sum are rint(t) in two's complement, for |t| < 7.5."""
-    t = np.concatenate([np.linspace(-7.5, 7.5, 200_001, dtype=np.float32)[1:-1],
-                        np.arange(-7, 8, dtype=np.float32) + np.float32(0.5),
-                        np.arange(-7, 8, dtype=np.float32) - np.float32(0.5)])
-    t = t[np.abs(t) < 7.5]
-    magic = np.float32(12582912.0)
-    s = (t + magic).astype(np.float32)
-    k = (s - magic).astype(np.float32)
-    assert np.array_equal(k, np.rint(t))
-    low = s.view(np.uint32) & 0xF
-    assert np.array_equal(low, (np.rint(t).astype(np.int64) & 0xF).astype(np.uint32))
+def test_magic_number_low_bits_are_the_int4_nibble():
+    """IF4's INT4 nibble: for an integer-valued k in [-8, 7], RN(k + 1.5*2^23)
+    is exact and its low four bits are k in two's complement."""
+    k = np.arange(-8, 8, dtype=np.float32)
+    s = (k + np.float32(12582912.0)).astype(np.float32)
+    assert np.array_equal((s - np.float32(12582912.0)).astype(np.float32), k)
+    assert np.array_equal(s.view(np.uint32) & 0xF, (k.astype(np.int64) & 0xF).astype(np.uint32))
+
+
+def test_rint_ties_go_to_even():
+    """rint (the kernels' cvt.rni) on the INT4 ties t = j + 0.5."""
+    t = np.arange(-7, 7, dtype=np.float32) + np.float32(0.5)
+    assert np.all(np.rint(t) % 2 == 0)
+
+
+def test_stochastic_rounding_fixed_point_method(tmp_path):
+    """The kernels' integer/fixed-point stochastic rounding equals the
+    oracle's rule (round the magnitude up iff u < t * 2^16) on every u for
+    values around each E2M1 grid point and midpoint, and on 4M random pairs."""
+    exe = str(tmp_path / "sr_check")
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-frounding-math",
+                           os.path.join(HERE, "sr_check.c"),
+                           os.path.join(os.path.dirname(HERE), "oracle", "fp4q_oracle.c"),
+                           "-o", exe, "-lm"])
+    out = subprocess.run([exe, "4000000"], capture_output=True, text=True, check=True)
+    assert int(out.stdout.strip()) == 0
