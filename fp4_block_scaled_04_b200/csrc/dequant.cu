@@ -8,11 +8,14 @@
 //   IF4-INT4:         y = RN(RN(RN(k * RN(6/7)) * S) * s_dec)
 //   MXFP4:            y = g * 2^(byte - 127)
 //
-// Two blocks per thread.  E2M1 pairs decode with cvt.rn.f16x2.e2m1x2; the
-// product g * S is exact in f16 (at most 6 significant bits, within
-// [2^-10, 2688]), so it is formed as an f16x2 product and widened; the
-// multiplication by s_dec is the one FP32 rounding.  INT4 values come from a
-// 16-entry table of RN(k * RN(6/7)).
+// The codes [rows, cols/2] and the output [rows, cols] are both dense, so the
+// kernel walks the flat element range in units of E elements (one 16-byte
+// output store: E = 8 for BF16, 4 for FP32), consecutive units on
+// consecutive lanes: code loads and output stores are contiguous across the
+// warp.  E2M1 pairs decode with cvt.rn.f16x2.e2m1x2; g * S is exact in f16
+// (at most 6 significant bits, within [2^-10, 2688]) and is formed as an
+// f16x2 product; the multiplication by s_dec is the one FP32 rounding.  INT4
+// values are formed arithmetically: k = (2^23 + (nibble ^ 8)) - (2^23 + 8).
 #include "common.cuh"
 #include "launch.h"
 
@@ -42,155 +45,103 @@ __device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t h) {
   return __half22float2(v);
 }
 
-// 16 codes (two words) of one block -> 16 FP32 values
+// the two values of one code byte (element 2i in the low nibble)
 template <int FMT>
-__device__ __forceinline__ void decode16(uint32_t w0, uint32_t w1, uint32_t sbyte, float s_dec,
-                                         const float *itab, float (&y)[16]) {
-  const uint32_t w[2] = {w0, w1};
+__device__ __forceinline__ float2 decode_pair(uint32_t byte, uint32_t sbyte, float s_dec,
+                                              float c67) {
   if (FMT == FP4Q_FMT_MXFP4) {
     const float p = e8m0_value(sbyte);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float2 g = f16x2_to_f32x2(e2m1x2_to_f16x2((w[i >> 2] >> (8 * (i & 3))) & 0xFFu));
-      const float2 v = mul2(g, make_float2(p, p));
-      y[2 * i] = v.x;
-      y[2 * i + 1] = v.y;
-    }
-  } else if (FMT == FP4Q_FMT_IF4 && (sbyte & 0x80u)) {
-    const float S = e4m3_value(sbyte & 0x7Fu);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t byte = (w[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-      const float2 h = make_float2(itab[byte & 0xFu], itab[byte >> 4]);
-      const float2 v = mul2(mul2(h, make_float2(S, S)), make_float2(s_dec, s_dec));
-      y[2 * i] = v.x;
-      y[2 * i + 1] = v.y;
-    }
-  } else {
-    const float S = e4m3_value(sbyte & 0x7Fu);
-    const __half hs = __float2half_rn(S);                  // exact: S is an E4M3 value
-    const uint32_t s2 = static_cast<uint32_t>(__half_as_ushort(hs)) * 0x10001u;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t gs = hmul2_bits(e2m1x2_to_f16x2((w[i >> 2] >> (8 * (i & 3))) & 0xFFu), s2);
-      const float2 v = mul2(f16x2_to_f32x2(gs), make_float2(s_dec, s_dec));
-      y[2 * i] = v.x;
-      y[2 * i + 1] = v.y;
-    }
+    return mul2(f16x2_to_f32x2(e2m1x2_to_f16x2(byte)), make_float2(p, p));
   }
+  const float S = e4m3_value(sbyte & 0x7Fu);
+  if (FMT == FP4Q_FMT_IF4 && (sbyte & 0x80u)) {
+    // k from the two's complement nibble, exactly: (2^23 + (n ^ 8)) - (2^23 + 8)
+    const float k0 = __fsub_rn(__uint_as_float(0x4B000000u | ((byte & 0xFu) ^ 8u)), 8388616.0f);
+    const float k1 = __fsub_rn(__uint_as_float(0x4B000000u | ((byte >> 4) ^ 8u)), 8388616.0f);
+    const float2 h = mul2(make_float2(k0, k1), make_float2(c67, c67));
+    return mul2(mul2(h, make_float2(S, S)), make_float2(s_dec, s_dec));
+  }
+  const __half hs = __float2half_rn(S);                  // exact: S is an E4M3 value
+  const uint32_t s2 = static_cast<uint32_t>(__half_as_ushort(hs)) * 0x10001u;
+  const uint32_t gs = hmul2_bits(e2m1x2_to_f16x2(byte), s2);
+  return mul2(f16x2_to_f32x2(gs), make_float2(s_dec, s_dec));
 }
 
-template <bool BF16_OUT>
-__device__ __forceinline__ void store16(void *y, int64_t off, const float (&v)[16]) {
-  if (BF16_OUT) {
-    uint32_t p[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-      p[i] = *reinterpret_cast<uint32_t *>(&h2);
-    }
-    uint4 *d = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(y) + off);
-    d[0] = make_uint4(p[0], p[1], p[2], p[3]);
-    d[1] = make_uint4(p[4], p[5], p[6], p[7]);
-  } else {
-    float4 *d = reinterpret_cast<float4 *>(static_cast<float *>(y) + off);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-  }
-}
-
-// One work unit = 16 consecutive codes of a row (one NVFP4/IF4 block or half an
-// MXFP4 block) plus the next 16; a thread handles one unit pair per step.
 template <int FMT, int BROWS, bool BF16_OUT>
 __global__ void __launch_bounds__(kThreads)
 dequant_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ sf, int scale_layout,
                const float *__restrict__ s_dec_ptr, int64_t rows, int64_t cols,
                void *__restrict__ y) {
-  __shared__ float itab[16];
-  if (threadIdx.x < 16) {
-    const int k = threadIdx.x >= 8 ? static_cast<int>(threadIdx.x) - 16 : static_cast<int>(threadIdx.x);
-    itab[threadIdx.x] = __fmul_rn(static_cast<float>(k), __fdiv_rn(6.0f, 7.0f));
-  }
-  __syncthreads();
-  const float s_dec = (FMT == FP4Q_FMT_MXFP4) ? 1.0f : *s_dec_ptr;
+  constexpr int E = BF16_OUT ? 8 : 4;                  // elements per unit
   constexpr int BLK = FMT == FP4Q_FMT_MXFP4 ? 32 : 16;
-  const int64_t upr = cols / 32;                 // 32-code unit pairs per row (cols % 32 == 0)
-  const int64_t bpr = cols / BLK;
+  const float s_dec = (FMT == FP4Q_FMT_MXFP4) ? 1.0f : *s_dec_ptr;
+  const float c67 = __fdiv_rn(6.0f, 7.0f);
+  const int64_t upr = cols / E;                        // units per row
   const int64_t total = rows * upr;
+  const int64_t bpr = cols / BLK;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  for (int64_t u = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; u < total;
-       u += stride) {
-    const int64_t r = u / upr, c = (u - r * upr) * 32;
-    const uint4 cw = __ldg(reinterpret_cast<const uint4 *>(q + r * (cols / 2) + c / 2));
-    uint32_t s0, s1;
-    if (BROWS == 16) {           // 16x16 tiles: linear [rows/16, cols/16]
-      s0 = sf[(r / 16) * bpr + c / 16];
-      s1 = sf[(r / 16) * bpr + c / 16 + 1];
-    } else if (BLK == 32) {
-      s0 = s1 = sf[scale_offset(r, c / 32, bpr, scale_layout)];
+  int64_t u = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+  if (u >= total) return;
+  // (row, column) of the unit, advanced by a fixed stride each step
+  int64_t r = u / upr, c = (u - r * upr) * E;
+  const int64_t dr = stride / upr, dc = (stride - dr * upr) * E;
+  for (; u < total; u += stride) {
+    const uint32_t sbyte = (BROWS == 16) ? sf[(r / 16) * bpr + c / 16]
+                                         : sf[scale_offset(r, c / BLK, bpr, scale_layout)];
+    const int64_t e = r * cols + c;
+    float v[E];
+    if (E == 8) {
+      const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(q + e / 2));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 p = decode_pair<FMT>((w >> (8 * i)) & 0xFFu, sbyte, s_dec, c67);
+        v[2 * i] = p.x;
+        v[(2 * i + 1) % E] = p.y;
+      }
     } else {
-      s0 = sf[scale_offset(r, c / 16, bpr, scale_layout)];
-      s1 = sf[scale_offset(r, c / 16 + 1, bpr, scale_layout)];
+      const uint32_t w = __ldg(reinterpret_cast<const uint16_t *>(q + e / 2));
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float2 p = decode_pair<FMT>((w >> (8 * i)) & 0xFFu, sbyte, s_dec, c67);
+        v[2 * i] = p.x;
+        v[2 * i + 1] = p.y;
+      }
     }
-    float v0[16], v1[16];
-    decode16<FMT>(cw.x, cw.y, s0, s_dec, itab, v0);
-    decode16<FMT>(cw.z, cw.w, s1, s_dec, itab, v1);
-    store16<BF16_OUT>(y, r * cols + c, v0);
-    store16<BF16_OUT>(y, r * cols + c + 16, v1);
-  }
-}
-
-// Rows whose length is an odd number of 16-code blocks (NVFP4 / IF4 with
-// cols % 32 == 16): one block per step.
-template <int FMT, int BROWS, bool BF16_OUT>
-__global__ void __launch_bounds__(kThreads)
-dequant16_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ sf, int scale_layout,
-                 const float *__restrict__ s_dec_ptr, int64_t rows, int64_t cols,
-                 void *__restrict__ y) {
-  __shared__ float itab[16];
-  if (threadIdx.x < 16) {
-    const int k = threadIdx.x >= 8 ? static_cast<int>(threadIdx.x) - 16 : static_cast<int>(threadIdx.x);
-    itab[threadIdx.x] = __fmul_rn(static_cast<float>(k), __fdiv_rn(6.0f, 7.0f));
-  }
-  __syncthreads();
-  const float s_dec = *s_dec_ptr;
-  const int64_t bpr = cols / 16, total = rows * bpr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; b < total;
-       b += stride) {
-    const int64_t r = b / bpr, cb = b - r * bpr;
-    const uint2 cw = __ldg(reinterpret_cast<const uint2 *>(q + r * (cols / 2) + cb * 8));
-    const uint32_t s = BROWS == 16 ? sf[(r / 16) * bpr + cb] : sf[scale_offset(r, cb, bpr, scale_layout)];
-    float v[16];
-    decode16<FMT>(cw.x, cw.y, s, s_dec, itab, v);
-    store16<BF16_OUT>(y, r * cols + cb * 16, v);
+    if (BF16_OUT) {
+      uint32_t p[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[(2 * i) % E], v[(2 * i + 1) % E]);
+        p[i] = *reinterpret_cast<uint32_t *>(&h2);
+      }
+      *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(y) + e) = make_uint4(p[0], p[1], p[2], p[3]);
+    } else {
+      *reinterpret_cast<float4 *>(static_cast<float *>(y) + e) =
+          make_float4(v[0], v[1], v[2 % E], v[3 % E]);
+    }
+    r += dr;
+    c += dc;
+    if (c >= cols) {
+      c -= cols;
+      ++r;
+    }
   }
 }
 
 template <int FMT, int BROWS>
 cudaError_t launch_fmt(const uint8_t *q, const uint8_t *sf, int scale_layout, const float *s_dec,
                        int64_t rows, int64_t cols, void *y, int y_dtype, const Launch &L) {
-  const bool pairs = (cols % 32) == 0;
-  const int64_t units = pairs ? rows * (cols / 32) : rows * (cols / 16);
+  const bool bf = y_dtype == FP4Q_BF16;
+  const int64_t units = rows * (cols / (bf ? 8 : 4));
   int64_t want = (units + kThreads - 1) / kThreads;
   int64_t cap = static_cast<int64_t>(L.num_sms) * 8;
   int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-  const bool bf = y_dtype == FP4Q_BF16;
-  if (pairs) {
-    if (bf)
-      dequant_kernel<FMT, BROWS, true><<<grid, kThreads, 0, L.stream>>>(q, sf, scale_layout,
-                                                                       s_dec, rows, cols, y);
-    else
-      dequant_kernel<FMT, BROWS, false><<<grid, kThreads, 0, L.stream>>>(q, sf, scale_layout,
-                                                                        s_dec, rows, cols, y);
-  } else {
-    if (bf)
-      dequant16_kernel<FMT, BROWS, true><<<grid, kThreads, 0, L.stream>>>(q, sf, scale_layout,
-                                                                         s_dec, rows, cols, y);
-    else
-      dequant16_kernel<FMT, BROWS, false><<<grid, kThreads, 0, L.stream>>>(q, sf, scale_layout,
-                                                                          s_dec, rows, cols, y);
-  }
+  if (bf)
+    dequant_kernel<FMT, BROWS, true><<<grid, kThreads, 0, L.stream>>>(q, sf, scale_layout, s_dec,
+                                                                     rows, cols, y);
+  else
+    dequant_kernel<FMT, BROWS, false><<<grid, kThreads, 0, L.stream>>>(q, sf, scale_layout, s_dec,
+                                                                      rows, cols, y);
   return cudaGetLastError();
 }
 

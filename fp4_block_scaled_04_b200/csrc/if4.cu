@@ -12,10 +12,10 @@
 // k), so each lane still sums its own block's squared errors in order
 // k = 0..15, as the definition requires.
 //   FP4:  codes by cvt.rn.satfinite.e2m1x2, values back by cvt.f16x2.e2m1x2
-//   INT4: k = rint(t), t = RN(v * RN(7/6)); adding 1.5 * 2^23 to the
-//         integer-valued k puts its two's complement in the low bits; the
-//         clamp to [-7, 7] only matters when the block's largest |t| reaches
-//         7.5, which is tested once per block.
+//   INT4: k = rint(t), t = RN(v * RN(7/6)), as RN(t + 1.5 * 2^23) - 1.5 * 2^23
+//         (exact round-half-even for |t| < 2^22; the sum's low bits hold k in
+//         two's complement); the clamp to [-7, 7] only matters when the
+//         block's largest |t| reaches 7.5, which is tested once per block.
 #include "common.cuh"
 #include "launch.h"
 
@@ -67,16 +67,17 @@ __device__ __forceinline__ void if4_pair(const float (&xa)[16], const float (&xb
       const float2 g = s == 0 ? make_float2(ga.x, gb.x) : make_float2(ga.y, gb.y);
       // No product below feeds a packed add or subtract: ptxas may contract a
       // mul.f32x2 -> add.f32x2 pair into one fused operation even with .rn,
-      // which rounds once instead of twice.  rint is a conversion, the add of
-      // the magic number is exact (kf is an integer), and the differences
-      // with a product operand are scalar __fsub_rn, which is never fused.
-      float2 t = mul2(vk, make_float2(c76, c76));
+      // which rounds once instead of twice.  Products that are added to are
+      // scalar __fmul_rn / __fadd_rn / __fsub_rn, which are never fused.
+      // t = RN(v * RN(7/6)) and RN(t + 1.5 * 2^23) = rint(t) + 1.5 * 2^23 are
+      // scalar __fmul_rn / __fadd_rn, which are never merged into an FMA
+      float tx = __fmul_rn(vk.x, c76), ty = __fmul_rn(vk.y, c76);
       if (CLAMP) {
-        t.x = fminf(fmaxf(t.x, -7.25f), 7.25f);
-        t.y = fminf(fmaxf(t.y, -7.25f), 7.25f);
+        tx = fminf(fmaxf(tx, -7.25f), 7.25f);
+        ty = fminf(fmaxf(ty, -7.25f), 7.25f);
       }
-      const float2 kf = make_float2(rintf(t.x), rintf(t.y));     // round half to even
-      const float2 tm = add2(kf, make_float2(kMagic, kMagic));    // k in the low bits
+      const float2 tm = make_float2(__fadd_rn(tx, kMagic), __fadd_rn(ty, kMagic));
+      const float2 kf = sub2(tm, make_float2(kMagic, kMagic));    // rint(t), exact
       const float2 hv = mul2(kf, make_float2(c67, c67));
       const float2 dfp = make_float2(__fsub_rn(vk.x, g.x), __fsub_rn(vk.y, g.y));
       const float2 dint = make_float2(__fsub_rn(vk.x, hv.x), __fsub_rn(vk.y, hv.y));

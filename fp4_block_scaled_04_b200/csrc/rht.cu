@@ -11,8 +11,9 @@
 // 16-token group of the transform and one quantization block per column); a
 // warp owns 128 tokens x 16 columns (lane = group + 8 * column quad).
 //   * each warp streams its tiles through a two-stage cp.async buffer in
-//     shared memory, so the next tile is in flight while this one computes;
-//     a lane copies exactly the chunks it later reads (no cross-lane sync);
+//     shared memory, so the next tile is in flight while this one computes
+//     (16-byte copies laid out so each warp write is a contiguous 512 bytes;
+//     warp barriers order the copy, the reads and the refill);
 //   * the sign flip is one LOP3 per packed word, the butterfly stages
 //     h = 1, 2, 4, 8 run in registers on f32x2 column pairs;
 //   * for n = 128 the stages h = 16, 32, 64 combine the eight groups: the warp
@@ -32,7 +33,12 @@ namespace {
 
 constexpr int kThreads = 128;       // 4 warps
 constexpr int kWarps = kThreads / 32;
-constexpr int kUnits = 128 * 4 + 32;  // input chunks per buffer (16 tokens padded by 4)
+// input buffer of one warp tile: 128 tokens x 4 column quads ("units" of 4
+// elements); every 16 tokens are padded by 2 units, which makes the lanes'
+// 8-byte reads (lane = group + 8 * quad, token 16 group + k) fall on 16
+// distinct bank pairs per half-warp
+constexpr int kUnits = 128 * 4 + 16;
+__device__ __forceinline__ int unit_of(int t, int q) { return 4 * t + 2 * (t >> 4) + q; }
 
 struct RhtParams {
   uint32_t k0[10], k1[10];   // Philox4x32-10 round keys of the seed
@@ -102,12 +108,8 @@ __device__ __forceinline__ void xstage(float2 (&lo)[16], float2 (&hi)[16]) {
       }
 }
 
-template <typename T>
-__device__ __forceinline__ void async_copy(uint32_t dst, const T *src) {
-  if (sizeof(T) == 2)
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-  else
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+__device__ __forceinline__ void async_copy16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
@@ -149,7 +151,7 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   uint8_t *wbase = smem + warp * WARP_BYTES;
   const uint32_t in_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbase));
   float4 *xbuf = reinterpret_cast<float4 *>(wbase + IN_BYTES);
-  const int my_unit = 68 * g + cq;                        // chunk (16 g + k, cq) = my_unit + 4 k
+  const int my_unit = unit_of(16 * g, cq);                // unit (16 g + k, cq) = my_unit + 4 k
 
   // signs of this lane's 16 tokens
   uint32_t signs;
@@ -167,13 +169,25 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
   int64_t tile = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
 
+  // the copy of a tile is spread differently from the reads: lane L moves the
+  // 16-byte pieces L + 32 i (token (L + 32 i) / PPT, piece (L + 32 i) % PPT,
+  // PPT = 16 columns * sizeof(T) / 16), so a warp writes whole
+  // 512-byte stretches of shared memory; a __syncwarp after the wait hands
+  // the data to the lanes that read it (PPT = pieces per token row)
+  constexpr int PPT = sizeof(T);                          // 16-byte pieces per token row
+  constexpr int UPP = 16 / UB;                            // units per piece
   auto issue = [&](int64_t t, int st) {
-    const TileCoord tl(t, tiles_c, g, cq, tokens, cols);
-    if (tl.valid) {
-      const T *src = dy + tl.t0 * ld + tl.c0;
-      const uint32_t dst = in_s + static_cast<uint32_t>((st * kUnits + my_unit) * UB);
+    const int64_t tt = t / tiles_c, tc = t - tt * tiles_c;
+    const int64_t tbase = tt * 128, cbase = tc * 16;
+    const uint32_t dst0 = in_s + static_cast<uint32_t>(st * kUnits * UB);
 #pragma unroll
-      for (int k = 0; k < 16; ++k) async_copy<T>(dst + 4 * k * UB, src + k * ld);
+    for (int i = 0; i < 4 * PPT; ++i) {
+      const int piece = lane + 32 * i;
+      const int tok = piece / PPT, pc = piece % PPT;
+      const int64_t col = cbase + pc * (16 / static_cast<int>(sizeof(T)));
+      if (tbase + tok < tokens && col < cols)
+        async_copy16(dst0 + static_cast<uint32_t>(unit_of(tok, pc * UPP) * UB),
+                     dy + (tbase + tok) * ld + col);
     }
   };
 
@@ -181,9 +195,11 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   if (tile < ntiles) issue(tile, 0);
   async_commit();
   for (int st = 0; tile < ntiles; tile += nwarps, st ^= 1) {
+    __syncwarp();   // every lane is done with stage st ^ 1 (last tile) before it is refilled
     if (tile + nwarps < ntiles) issue(tile + nwarps, st ^ 1);
     async_commit();
     async_wait_1();
+    __syncwarp();
     const TileCoord tl(tile, tiles_c, g, cq, tokens, cols);
     const int64_t t0 = tl.t0, c0 = tl.c0;
     const bool valid = tl.valid;

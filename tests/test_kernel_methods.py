@@ -37,6 +37,19 @@ def test_division_by_six_is_the_ieee_quotient(div6_exe):
     assert bad < (1 << 24)                  # only the subnormal-quotient range differs
 
 
+def test_magic_number_rounding_is_round_half_even():
+    """IF4's INT4 step: RN(t + 1.5*2^23) - 1.5*2^23 == rint(t) for |t| < 7.5,
+    including every tie j + 1/2."""
+    t = np.concatenate([np.linspace(-7.5, 7.5, 200_001, dtype=np.float32)[1:-1],
+                        np.arange(-7, 7, dtype=np.float32) + np.float32(0.5)])
+    t = t[np.abs(t) < 7.5]
+    magic = np.float32(12582912.0)
+    s = (t + magic).astype(np.float32)
+    assert np.array_equal((s - magic).astype(np.float32), np.rint(t))
+    assert np.array_equal(s.view(np.uint32) & 0xF,
+                          (np.rint(t).astype(np.int64) & 0xF).astype(np.uint32))
+
+
 def test_magic_number_low_bits_are_the_int4_nibble():
     """IF4's INT4 nibble: for an integer-valued k in [-8, 7], RN(k + 1.5*2^23)
     is exact and its low four bits are k in two's complement."""
