@@ -411,6 +411,7 @@ def main():
     import torch
     import torch.distributed as dist
     import fp4_block_scaled_04_b200 as fq
+    from fp4_block_scaled_04_b200 import dist as fdist
 
     ws, rank, local = dist_env()
     if ws != args.gpus and ws > 1:
@@ -462,15 +463,10 @@ def main():
     per_job_ms = [sum(events[s][j][0].elapsed_time(events[s][j][1]) for s in range(args.steps))
                   for j in range(len(jobs))]
     total_ms = sum(per_job_ms)
-    if ws > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms_max = float(t.item())
-    else:
-        total_ms_max = total_ms
+    total_ms_max = fdist.max_over_ranks(total_ms, device=device)
 
     step_bytes = sum(j.bytes for j in jobs)
-    value = ws * step_bytes * args.steps / (total_ms_max * 1e-3) / 1e9
+    value = fdist.aggregate_gbs(step_bytes, ws, args.steps, total_ms_max)
     peak, peak_kind = hbm_peak()
 
     per_config = []
@@ -509,12 +505,8 @@ def main():
                 d2h += b
         e1.record(stream)
         torch.cuda.synchronize(device)
-        e_ms = e0.elapsed_time(e1)
-        if ws > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": round(ws * step_bytes * k / (e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+        e_ms = fdist.max_over_ranks(e0.elapsed_time(e1), device=device)
+        e2e = {"value": round(fdist.aggregate_gbs(step_bytes, ws, k, e_ms), 3), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k,
                "path": "pinned host -> device copy, C-ABI call (tensor amax computed inside), "
                        "device -> pinned host copy of every output"}
