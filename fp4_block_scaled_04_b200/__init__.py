@@ -29,6 +29,7 @@ __all__ = [
     "fp4q_status_string", "fp4q_version", "fp4q_workspace_bytes", "fp4q_scale_bytes",
     "fp4q_amax", "fp4q_quantize_nvfp4", "fp4q_quantize_mxfp4", "fp4q_quantize_2d",
     "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
+    "fp4q_quantize_nvfp4_noalloc",
 ]
 
 ROWWISE, COLWISE = 1, 2
@@ -80,6 +81,8 @@ _SIGNATURES = {
                                   _P, _P, _SZ, _P]),
     "fp4q_quantize_if4": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "fp4q_dequantize": (_I, [_I, _P, _P, _I, _I, _I, _P, _I64, _I64, _P, _I, _P]),
+    "fp4q_quantize_nvfp4_noalloc": (_I, [_P, _I, _I64, _I64, _I64, _U, _I, _U64, _P, _P, _P,
+                                         _P, _P, _P, _I, _P]),
 }
 
 
@@ -204,6 +207,22 @@ def fp4q_quantize_nvfp4(x: torch.Tensor, layouts: int = ROWWISE, round: int = RN
         _ptr(out.get("s_dec")), _ptr(out.get("q_row")), _ptr(out.get("sf_row")),
         _ptr(out.get("q_col")), _ptr(out.get("sf_col")), scale_layout, _ptr(ws),
         0 if ws is None else ws.numel(), _stream(dev)))
+    return out
+
+
+def fp4q_quantize_nvfp4_noalloc(x: torch.Tensor, out: dict, layouts: int = ROWWISE,
+                                round: int = RNE, seed: int = 0,
+                                amax: torch.Tensor | None = None,
+                                scale_layout: int = SCALE_LINEAR) -> dict:
+    """``fp4q_quantize_nvfp4`` for callers that cannot allocate: the outputs in
+    ``out`` are the caller's buffers and, when ``amax`` is None, the library's
+    own 256-byte device array holds the amax instead of a workspace.  Calls
+    on one device that overlap on the GPU race on that array."""
+    rows, cols, ld = _matrix(x)
+    _check("fp4q_quantize_nvfp4_noalloc", lib().fp4q_quantize_nvfp4_noalloc(
+        _ptr(x), _dtype(x), rows, cols, ld, layouts, round, seed, _ptr(amax),
+        _ptr(out.get("s_dec")), _ptr(out.get("q_row")), _ptr(out.get("sf_row")),
+        _ptr(out.get("q_col")), _ptr(out.get("sf_col")), scale_layout, _stream(x.device)))
     return out
 
 

@@ -220,6 +220,34 @@ fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int
                             int block_rows, int block_cols, const float *tensor_scale,
                             int64_t rows, int64_t cols, void *y, int y_dtype, void *stream);
 
+/* fp4q_quantize_nvfp4 without a workspace argument, for callers that cannot
+ * allocate device memory: code inside a host application or framework that
+ * owns every device buffer, or that must not call cudaMalloc once set-up is
+ * over.  The pages have no counterpart; this is a library convenience.
+ * The arguments, outputs and error codes are those of fp4q_quantize_nvfp4.
+ * The one difference is where the amax goes when amax == NULL. It is
+ * computed into a 256-byte array that the library keeps in device memory:
+ *   - Every GPU that loads the library holds that array until the process
+ *     exits. The array's size is the most workspace this call can use.
+ *     The call returns FP4Q_ERR_WORKSPACE_TOO_SMALL if
+ *     fp4q_workspace_bytes() ever exceeded it.
+ *     The amax needs 4 bytes at any tensor size, so no shape is refused for
+ *     scratch.
+ *   - The first call on a device with amax == NULL looks the array's device
+ *     address up (cudaGetSymbolAddress, with that device made current).
+ *     Make that first call before any stream capture begins.
+ *   - All calls on one device share the array. The amax pre-pass clears it
+ *     before use, and the array keeps the last call's amax afterwards.
+ *     Calls with amax == NULL that can overlap on the GPU (different streams,
+ *     no ordering between them) race on it. Order them, or pass amax.
+ * This call allocates nothing: no cudaMalloc, no cudaFree, no library
+ * allocator. */
+fp4q_status fp4q_quantize_nvfp4_noalloc(const void *x, int dtype, int64_t rows, int64_t cols,
+                                        int64_t ld, unsigned layouts, int round, uint64_t seed,
+                                        const float *amax, float *tensor_scale_out,
+                                        uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col,
+                                        uint8_t *sf_col, int scale_layout, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
