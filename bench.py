@@ -13,7 +13,14 @@ device, as with delayed scaling or a fused producer):
   if4       16384x8192 BF16   IF4 quantize, and IF4 -> BF16 dequantize
 
 Each kernel is timed with CUDA events on the launching stream; the L2 is
-flushed (256 MiB write) before every kernel, outside the timed events.
+flushed before every kernel, outside the timed events: a 256 MiB buffer is
+written and then read back, so the kernel starts with none of its own data
+in L2 and without the flush's dirty lines still waiting to be written back
+(which would charge the flush's DRAM writes to the kernel).  A short
+device-side sleep before each flush keeps the GPU busy while the host
+enqueues the flush, the start event and the kernel, so the events bracket the
+kernel itself rather than the host's launch latency (which the e2e figure
+includes).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -41,6 +48,7 @@ if ROOT not in sys.path:
 METRIC = "quantize throughput GB/s (bytes in+out) and % of B200 HBM peak per config"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
+LEAD_SLEEP_CYCLES = 200_000  # ~0.1 ms at 1.965 GHz, untimed
 
 
 def hbm_peak():
@@ -434,11 +442,14 @@ def main():
     inputs = suite_inputs()
     jobs = build_jobs(device, fq, inputs)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    flush_sum = torch.empty((), dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
     def step(record):
         for j, job in enumerate(jobs):
+            torch.cuda._sleep(LEAD_SLEEP_CYCLES)
             flush.fill_(float(j))
+            torch.sum(flush, dim=0, out=flush_sum)
             if record is not None:
                 record[j][0].record(stream)
             job.run()
@@ -527,7 +538,8 @@ def main():
                                    "and mxfp4 row+col; weight 14336x4096 fp32 2d16x16; gradient "
                                    "8192x5120 rht16/rht128 x sr/rne; if4 16384x8192 quant + "
                                    "bf16 dequant",
-                       "l2": "flushed before every kernel (256 MiB write, untimed)",
+                       "l2": "flushed before every kernel (256 MiB written then read, untimed)",
+                       "launch": "device sleep before each flush hides host launch latency",
                        "amax": "precomputed on the device (headline); e2e computes it",
                        "parallelism": f"replicas x{ws}" if ws > 1 else "single gpu"},
             "pct_of_peak": round(100 * value / (ws * peak), 2),

@@ -9,13 +9,21 @@
 //   MXFP4:            y = g * 2^(byte - 127)
 //
 // The codes [rows, cols/2] and the output [rows, cols] are both dense, so the
-// kernel walks the flat element range in units of E elements (one 16-byte
-// output store: E = 8 for BF16, 4 for FP32), consecutive units on
-// consecutive lanes: code loads and output stores are contiguous across the
-// warp.  E2M1 pairs decode with cvt.rn.f16x2.e2m1x2; g * S is exact in f16
-// (at most 6 significant bits, within [2^-10, 2688]) and is formed as an
-// f16x2 product; the multiplication by s_dec is the one FP32 rounding.  INT4
-// values are formed arithmetically: k = (2^23 + (nibble ^ 8)) - (2^23 + 8).
+// kernel walks the flat element range in units of 8 elements (4 code bytes,
+// one 16-byte BF16 store), consecutive units on consecutive lanes, four
+// units per lane per step so that four loads are in flight.  With a linear
+// 1x16 or 1x32 scale matrix the scale index is the flat element index / 16
+// (or / 32), so the walk needs no row and column; the swizzled and
+// 16x16-tile layouts carry (row, column) along with a fixed stride.
+//
+// Arithmetic: E2M1 pairs decode with cvt.rn.f16x2.e2m1x2 and E4M3 scales
+// with cvt.rn.f16x2.e4m3x2.  g * S is exact in f16 (at most 6 significant
+// bits, within [2^-10, 2688]).  IF4 blocks are decoded without branching on
+// the per-block flag (neighbouring threads hold blocks of either kind): the
+// f16 pair is the E2M1 pair or the INT4 pair k = (1024 + (n ^ 8)) - 1032 (exact
+// in f16), then RN(pair * m) with m = 1 (FP4) or RN(6/7) (INT4), RN(* S),
+// RN(* s_dec), all in FP32 -- for FP4 blocks the first two products are exact
+// and the result equals RN(RN(g * S) * s_dec).
 #include "common.cuh"
 #include "launch.h"
 
@@ -34,9 +42,23 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
   return h2;
 }
 
+// (S, S) in f16 from a 7-bit E4M3 code
+__device__ __forceinline__ uint32_t e4m3_to_f16x2_dup(uint32_t code7) {
+  uint32_t h2;
+  const uint16_t w = static_cast<uint16_t>(code7 * 0x0101u);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(w));
+  return h2;
+}
+
 __device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hsub2_bits(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
 
@@ -45,104 +67,159 @@ __device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t h) {
   return __half22float2(v);
 }
 
-// the two values of one code byte (element 2i in the low nibble)
+// (k0, k1) in f16 for the two two's-complement nibbles of `byte`
+__device__ __forceinline__ uint32_t int4x2_to_f16x2(uint32_t byte) {
+  const uint32_t t = ((byte * 0x1001u) & 0x000F000Fu) ^ 0x64086408u;  // 1024 + (n ^ 8)
+  return hsub2_bits(t, 0x64086408u);                                   // - 1032
+}
+
+struct Store {
+  __device__ __forceinline__ static void put(float *y, const float2 (&v)[4]) {
+    float4 *p = reinterpret_cast<float4 *>(y);
+    p[0] = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+    p[1] = make_float4(v[2].x, v[2].y, v[3].x, v[3].y);
+  }
+  __device__ __forceinline__ static void put(__nv_bfloat16 *y, const float2 (&v)[4]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[i].x, v[i].y);
+      w[i] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    *reinterpret_cast<uint4 *>(y) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+// 8 values of one unit: 4 code bytes (element 2i in the low nibble)
 template <int FMT>
-__device__ __forceinline__ float2 decode_pair(uint32_t byte, uint32_t sbyte, float s_dec,
-                                              float c67) {
+__device__ __forceinline__ void decode8(uint32_t codes, uint32_t sbyte, float s_dec, float c67,
+                                        float2 (&v)[4]) {
+  const float2 sd = make_float2(s_dec, s_dec);
   if (FMT == FP4Q_FMT_MXFP4) {
     const float p = e8m0_value(sbyte);
-    return mul2(f16x2_to_f32x2(e2m1x2_to_f16x2(byte)), make_float2(p, p));
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      v[i] = mul2(f16x2_to_f32x2(e2m1x2_to_f16x2((codes >> (8 * i)) & 0xFFu)), make_float2(p, p));
+  } else if (FMT == FP4Q_FMT_NVFP4) {
+    const uint32_t s2 = e4m3_to_f16x2_dup(sbyte & 0x7Fu);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      v[i] = mul2(f16x2_to_f32x2(hmul2_bits(e2m1x2_to_f16x2((codes >> (8 * i)) & 0xFFu), s2)), sd);
+  } else {  // IF4
+    const bool int4 = (sbyte & 0x80u) != 0;
+    const uint32_t s2 = e4m3_to_f16x2_dup(sbyte & 0x7Fu);
+    const float S = __half2float(__ushort_as_half(static_cast<unsigned short>(s2 & 0xFFFFu)));
+    const float m = int4 ? c67 : 1.0f;
+    const uint32_t pick = int4 ? 0xFFFFFFFFu : 0u;   // select, not branch, per pair
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t byte = (codes >> (8 * i)) & 0xFFu;
+      const uint32_t h = (int4x2_to_f16x2(byte) & pick) | (e2m1x2_to_f16x2(byte) & ~pick);
+      v[i] = mul2(mul2(mul2(f16x2_to_f32x2(h), make_float2(m, m)), make_float2(S, S)), sd);
+    }
   }
-  const float S = e4m3_value(sbyte & 0x7Fu);
-  if (FMT == FP4Q_FMT_IF4 && (sbyte & 0x80u)) {
-    // k from the two's complement nibble, exactly: (2^23 + (n ^ 8)) - (2^23 + 8)
-    const float k0 = __fsub_rn(__uint_as_float(0x4B000000u | ((byte & 0xFu) ^ 8u)), 8388616.0f);
-    const float k1 = __fsub_rn(__uint_as_float(0x4B000000u | ((byte >> 4) ^ 8u)), 8388616.0f);
-    const float2 h = mul2(make_float2(k0, k1), make_float2(c67, c67));
-    return mul2(mul2(h, make_float2(S, S)), make_float2(s_dec, s_dec));
-  }
-  const __half hs = __float2half_rn(S);                  // exact: S is an E4M3 value
-  const uint32_t s2 = static_cast<uint32_t>(__half_as_ushort(hs)) * 0x10001u;
-  const uint32_t gs = hmul2_bits(e2m1x2_to_f16x2(byte), s2);
-  return mul2(f16x2_to_f32x2(gs), make_float2(s_dec, s_dec));
 }
 
-template <int FMT, int BROWS, bool BF16_OUT>
+// Byte offset of the scale of the 8-element unit starting at (r, c) (SWZ:
+// the 128x4 tile layout; BROWS == 16: the linear [rows/16, cols/16] tile
+// matrix).
+template <int BLK, int BROWS, bool SWZ>
+__device__ __forceinline__ int64_t unit_scale(int64_t r, int64_t c, int64_t cols) {
+  const int64_t sc = BLK == 32 ? (c >> 5) : (c >> 4);   // c, cols >= 0
+  const int64_t scols = BLK == 32 ? (cols >> 5) : (cols >> 4);
+  if (BROWS == 16) return (r >> 4) * scols + sc;
+  if (!SWZ) return r * scols + sc;
+  const int64_t tile = (r >> 7) * (scols >> 2) + (sc >> 2);
+  return tile * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (sc & 3);
+}
+
+// A warp takes NU x 32 consecutive 8-element units per step, lane l the units
+// l, l + 32, ...: every code load and output store of the warp is then one
+// contiguous stretch, and a thread has NU independent loads in flight.
+template <int FMT, int BROWS, bool SWZ, typename OutT>
 __global__ void __launch_bounds__(kThreads)
-dequant_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ sf, int scale_layout,
+dequant_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ sf,
                const float *__restrict__ s_dec_ptr, int64_t rows, int64_t cols,
-               void *__restrict__ y) {
-  constexpr int E = BF16_OUT ? 8 : 4;                  // elements per unit
+               OutT *__restrict__ y) {
+  constexpr int NU = 4;
   constexpr int BLK = FMT == FP4Q_FMT_MXFP4 ? 32 : 16;
+  constexpr bool FLAT = !SWZ && BROWS == 1;          // scale index from the unit index
   const float s_dec = (FMT == FP4Q_FMT_MXFP4) ? 1.0f : *s_dec_ptr;
   const float c67 = __fdiv_rn(6.0f, 7.0f);
-  const int64_t upr = cols / E;                        // units per row
-  const int64_t total = rows * upr;
-  const int64_t bpr = cols / BLK;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  int64_t u = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-  if (u >= total) return;
-  // (row, column) of the unit, advanced by a fixed stride each step
-  int64_t r = u / upr, c = (u - r * upr) * E;
-  const int64_t dr = stride / upr, dc = (stride - dr * upr) * E;
-  for (; u < total; u += stride) {
-    const uint32_t sbyte = (BROWS == 16) ? sf[(r / 16) * bpr + c / 16]
-                                         : sf[scale_offset(r, c / BLK, bpr, scale_layout)];
-    const int64_t e = r * cols + c;
-    float v[E];
-    if (E == 8) {
-      const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(q + e / 2));
+  const int64_t total = rows * (cols / 8);           // units
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  const uint32_t *qw = reinterpret_cast<const uint32_t *>(q);
+  // (row, column) of each of the lane's NU units, advanced by a fixed stride
+  int64_t r[NU], c[NU];
+  int64_t dr = 0, dc = 0;
+  if (!FLAT) {
+    const int64_t estride = wstride * NU * 32 * 8;   // elements per step
+    dr = estride / cols;
+    dc = estride - dr * cols;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 p = decode_pair<FMT>((w >> (8 * i)) & 0xFFu, sbyte, s_dec, c67);
-        v[2 * i] = p.x;
-        v[(2 * i + 1) % E] = p.y;
-      }
-    } else {
-      const uint32_t w = __ldg(reinterpret_cast<const uint16_t *>(q + e / 2));
+    for (int j = 0; j < NU; ++j) {
+      const int64_t e = (warp0 * NU * 32 + 32 * j + lane) * 8;
+      r[j] = e / cols;
+      c[j] = e - r[j] * cols;
+    }
+  }
+  for (int64_t base = warp0 * NU * 32 + lane; base < total; base += wstride * NU * 32) {
+    uint32_t cw[NU], sb[NU];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const float2 p = decode_pair<FMT>((w >> (8 * i)) & 0xFFu, sbyte, s_dec, c67);
-        v[2 * i] = p.x;
-        v[2 * i + 1] = p.y;
+    for (int j = 0; j < NU; ++j) {
+      const int64_t u = base + 32 * j;
+      if (u < total) {
+        const int64_t si = FLAT ? (BLK == 32 ? (u >> 2) : (u >> 1))
+                                : unit_scale<BLK, BROWS, SWZ>(r[j], c[j], cols);
+        cw[j] = __ldg(qw + u);
+        sb[j] = __ldg(sf + si);
       }
     }
-    if (BF16_OUT) {
-      uint32_t p[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[(2 * i) % E], v[(2 * i + 1) % E]);
-        p[i] = *reinterpret_cast<uint32_t *>(&h2);
+    for (int j = 0; j < NU; ++j) {
+      const int64_t u = base + 32 * j;
+      if (u < total) {
+        float2 v[4];
+        decode8<FMT>(cw[j], sb[j], s_dec, c67, v);
+        Store::put(y + u * 8, v);
       }
-      *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(y) + e) = make_uint4(p[0], p[1], p[2], p[3]);
-    } else {
-      *reinterpret_cast<float4 *>(static_cast<float *>(y) + e) =
-          make_float4(v[0], v[1], v[2 % E], v[3 % E]);
-    }
-    r += dr;
-    c += dc;
-    if (c >= cols) {
-      c -= cols;
-      ++r;
+      if (!FLAT) {
+        r[j] += dr;
+        c[j] += dc;
+        if (c[j] >= cols) {
+          c[j] -= cols;
+          ++r[j];
+        }
+      }
     }
   }
 }
 
-template <int FMT, int BROWS>
-cudaError_t launch_fmt(const uint8_t *q, const uint8_t *sf, int scale_layout, const float *s_dec,
-                       int64_t rows, int64_t cols, void *y, int y_dtype, const Launch &L) {
-  const bool bf = y_dtype == FP4Q_BF16;
-  const int64_t units = rows * (cols / (bf ? 8 : 4));
-  int64_t want = (units + kThreads - 1) / kThreads;
-  int64_t cap = static_cast<int64_t>(L.num_sms) * 8;
-  int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-  if (bf)
-    dequant_kernel<FMT, BROWS, true><<<grid, kThreads, 0, L.stream>>>(q, sf, scale_layout, s_dec,
-                                                                     rows, cols, y);
+template <int FMT, int BROWS, bool SWZ>
+cudaError_t launch_fmt(const uint8_t *q, const uint8_t *sf, const float *s_dec, int64_t rows,
+                       int64_t cols, void *y, int y_dtype, const Launch &L) {
+  const int64_t steps = (rows * (cols / 8) + 4 * kThreads - 1) / (4 * kThreads);
+  const int64_t want = steps;
+  const int64_t cap = static_cast<int64_t>(L.num_sms) * 8;
+  const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+  if (y_dtype == FP4Q_BF16)
+    dequant_kernel<FMT, BROWS, SWZ><<<grid, kThreads, 0, L.stream>>>(
+        q, sf, s_dec, rows, cols, static_cast<__nv_bfloat16 *>(y));
   else
-    dequant_kernel<FMT, BROWS, false><<<grid, kThreads, 0, L.stream>>>(q, sf, scale_layout, s_dec,
-                                                                      rows, cols, y);
+    dequant_kernel<FMT, BROWS, SWZ><<<grid, kThreads, 0, L.stream>>>(
+        q, sf, s_dec, rows, cols, static_cast<float *>(y));
   return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t launch_layout(const uint8_t *q, const uint8_t *sf, int scale_layout,
+                          const float *s_dec, int64_t rows, int64_t cols, void *y, int y_dtype,
+                          const Launch &L) {
+  if (scale_layout == FP4Q_SCALE_SWIZZLED_128x4)
+    return launch_fmt<FMT, 1, true>(q, sf, s_dec, rows, cols, y, y_dtype, L);
+  return launch_fmt<FMT, 1, false>(q, sf, s_dec, rows, cols, y, y_dtype, L);
 }
 
 }  // namespace
@@ -152,12 +229,12 @@ cudaError_t launch_dequant(int format, const uint8_t *q, const uint8_t *sf, int 
                            int64_t cols, void *y, int y_dtype, const Launch &L) {
   (void)block_cols;
   if (format == FP4Q_FMT_MXFP4)
-    return launch_fmt<FP4Q_FMT_MXFP4, 1>(q, sf, scale_layout, s_dec, rows, cols, y, y_dtype, L);
+    return launch_layout<FP4Q_FMT_MXFP4>(q, sf, scale_layout, s_dec, rows, cols, y, y_dtype, L);
   if (format == FP4Q_FMT_IF4)
-    return launch_fmt<FP4Q_FMT_IF4, 1>(q, sf, scale_layout, s_dec, rows, cols, y, y_dtype, L);
+    return launch_layout<FP4Q_FMT_IF4>(q, sf, scale_layout, s_dec, rows, cols, y, y_dtype, L);
   if (block_rows == 16)
-    return launch_fmt<FP4Q_FMT_NVFP4, 16>(q, sf, scale_layout, s_dec, rows, cols, y, y_dtype, L);
-  return launch_fmt<FP4Q_FMT_NVFP4, 1>(q, sf, scale_layout, s_dec, rows, cols, y, y_dtype, L);
+    return launch_fmt<FP4Q_FMT_NVFP4, 16, false>(q, sf, s_dec, rows, cols, y, y_dtype, L);
+  return launch_layout<FP4Q_FMT_NVFP4>(q, sf, scale_layout, s_dec, rows, cols, y, y_dtype, L);
 }
 
 }  // namespace fp4q

@@ -7,85 +7,120 @@
 // maps INT4's range 0..7 onto FP4's 0..6: values are multiplied by 7/6
 // before rounding to an integer and by 6/7 when decoded.
 //
-// A thread quantizes two adjacent blocks at once: every elementwise step is
-// one f32x2 instruction whose lanes are (block A element k, block B element
-// k), so each lane still sums its own block's squared errors in order
-// k = 0..15, as the definition requires.
-//   FP4:  codes by cvt.rn.satfinite.e2m1x2, values back by cvt.f16x2.e2m1x2
+// A lane quantizes two adjacent blocks at once: every elementwise step is one
+// f32x2 instruction whose lanes are (block A element k, block B element k),
+// so each lane still sums its own block's squared errors in order k = 0..15,
+// as the definition requires.
+//   FP4:  codes by cvt.rn.satfinite.e2m1x2, values back by cvt.f16x2.e2m1x2,
+//         errors RN(g - v) by the mixed-precision sub.f32.f16 (g is exact in
+//         f16; the sign of the difference does not change its square)
 //   INT4: k = rint(t), t = RN(v * RN(7/6)), as RN(t + 1.5 * 2^23) - 1.5 * 2^23
 //         (exact round-half-even for |t| < 2^22; the sum's low bits hold k in
 //         two's complement); the clamp to [-7, 7] only matters when the
 //         block's largest |t| reaches 7.5, which is tested once per block.
+//         Eight nibbles are packed by multiply-adds: the sum of
+//         bits(t + 1.5 * 2^23) * 16^i minus a constant leaves k_i + 8 in
+//         nibble i, and XOR 0x88888888 turns that into k_i mod 16.
+//
+// Memory: each warp streams tiles of 32 block pairs through a three-stage
+// cp.async buffer in shared memory (each lane copies and later reads only
+// its own pair, so no barrier is needed), so two tiles are in flight while
+// one computes.  The lane's 16-byte pieces are XOR-swizzled so that both the
+// copies and the reads of eight consecutive lanes hit distinct bank groups.
 #include "common.cuh"
 #include "launch.h"
 
 namespace fp4q {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
+constexpr int kWarps = kThreads / 32;
+constexpr int kStages = 3;
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+// sum over i < 8 of (bits(1.5 * 2^23) - 8) * 16^i, modulo 2^32
+constexpr uint32_t kPackBias = 0x4B3FFFF8u * 0x11111111u;
 
-// E2M1 values of the two nibbles of a byte, via the sm_100a conversion to f16x2
-__device__ __forceinline__ float2 e2m1_byte_values(uint32_t byte) {
-  uint32_t h2;
-  asm("{\n\t.reg .b8 q;\n\t.reg .b16 w;\n\t"
-      "cvt.u16.u32 w, %1;\n\t"
-      "cvt.u8.u16 q, w;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, q;\n\t}"
-      : "=r"(h2) : "r"(byte));
-  const __half2 h = *reinterpret_cast<const __half2 *>(&h2);
-  return __half22float2(h);
+// FP4 candidate of eight values: the packed codes (v[0] in bits 0..3) and
+// the eight rounding differences d[k] = RN(g_k - v_k).
+__device__ __forceinline__ uint32_t fp4_codes_diffs(const float (&v)[8], float (&d)[8]) {
+  uint32_t w;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
+      ".reg .f16 g0, g1, g2, g3, g4, g5, g6, g7;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %10, %9;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %12, %11;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %14, %13;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %16, %15;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t"
+      "cvt.rn.f16x2.e2m1x2 h0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
+      "mov.b32 {g0, g1}, h0;\n\t"
+      "mov.b32 {g2, g3}, h1;\n\t"
+      "mov.b32 {g4, g5}, h2;\n\t"
+      "mov.b32 {g6, g7}, h3;\n\t"
+      "sub.rn.f32.f16 %1, g0, %9;\n\t"
+      "sub.rn.f32.f16 %2, g1, %10;\n\t"
+      "sub.rn.f32.f16 %3, g2, %11;\n\t"
+      "sub.rn.f32.f16 %4, g3, %12;\n\t"
+      "sub.rn.f32.f16 %5, g4, %13;\n\t"
+      "sub.rn.f32.f16 %6, g5, %14;\n\t"
+      "sub.rn.f32.f16 %7, g6, %15;\n\t"
+      "sub.rn.f32.f16 %8, g7, %16;\n\t}"
+      : "=r"(w), "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3]), "=f"(d[4]), "=f"(d[5]),
+        "=f"(d[6]), "=f"(d[7])
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+        "f"(v[7]));
+  return w;
 }
 
-template <typename T, bool CLAMP>
-__device__ __forceinline__ void if4_pair(const float (&xa)[16], const float (&xb)[16], float fa,
-                                         float fb, float c76, float c67, uint32_t (&wa)[2],
-                                         uint32_t (&wb)[2], bool &int_a, bool &int_b) {
-  float2 v[16];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) v[k] = mul2(make_float2(xa[k], xb[k]), make_float2(fa, fb));
-  // FP4 candidate codes (row order within each block)
+// Both candidates of blocks A and B (lanes .x / .y of the pairs); picks the
+// smaller error per block.
+template <bool CLAMP>
+__device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float c67,
+                                         uint32_t (&wa)[2], uint32_t (&wb)[2], bool &int_a,
+                                         bool &int_b) {
+  // FP4 candidates and their differences, in element order
   uint32_t fpa[2], fpb[2];
+  float da[16], db[16];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    float ta[8], tb[8];
+    float ta[8], tb[8], ea[8], eb[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) { ta[k] = v[8 * h + k].x; tb[k] = v[8 * h + k].y; }
-    fpa[h] = e2m1x8(ta);
-    fpb[h] = e2m1x8(tb);
+    fpa[h] = fp4_codes_diffs(ta, ea);
+    fpb[h] = fp4_codes_diffs(tb, eb);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) { da[8 * h + k] = ea[k]; db[8 * h + k] = eb[k]; }
   }
   float2 efp = make_float2(0.0f, 0.0f), eint = make_float2(0.0f, 0.0f);
   uint32_t ia[2] = {0u, 0u}, ib[2] = {0u, 0u};
 #pragma unroll
-  for (int k = 0; k < 16; k += 2) {
-    const int h = k >> 3, sh = 4 * (k & 7);
-    const float2 ga = e2m1_byte_values((fpa[h] >> sh) & 0xFFu);   // block A, k and k+1
-    const float2 gb = e2m1_byte_values((fpb[h] >> sh) & 0xFFu);
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      const float2 vk = v[k + s];
-      const float2 g = s == 0 ? make_float2(ga.x, gb.x) : make_float2(ga.y, gb.y);
-      // No product below feeds a packed add or subtract: ptxas may contract a
-      // mul.f32x2 -> add.f32x2 pair into one fused operation even with .rn,
-      // which rounds once instead of twice.  Products that are added to are
-      // scalar __fmul_rn / __fadd_rn / __fsub_rn, which are never fused.
-      // t = RN(v * RN(7/6)) and RN(t + 1.5 * 2^23) = rint(t) + 1.5 * 2^23 are
-      // scalar __fmul_rn / __fadd_rn, which are never merged into an FMA
-      float tx = __fmul_rn(vk.x, c76), ty = __fmul_rn(vk.y, c76);
-      if (CLAMP) {
-        tx = fminf(fmaxf(tx, -7.25f), 7.25f);
-        ty = fminf(fmaxf(ty, -7.25f), 7.25f);
-      }
-      const float2 tm = make_float2(__fadd_rn(tx, kMagic), __fadd_rn(ty, kMagic));
-      const float2 kf = sub2(tm, make_float2(kMagic, kMagic));    // rint(t), exact
-      const float2 hv = mul2(kf, make_float2(c67, c67));
-      const float2 dfp = make_float2(__fsub_rn(vk.x, g.x), __fsub_rn(vk.y, g.y));
-      const float2 dint = make_float2(__fsub_rn(vk.x, hv.x), __fsub_rn(vk.y, hv.y));
-      efp = fma2(dfp, dfp, efp);
-      eint = fma2(dint, dint, eint);
-      ia[h] |= (__float_as_uint(tm.x) & 0xFu) << (sh + 4 * s);
-      ib[h] |= (__float_as_uint(tm.y) & 0xFu) << (sh + 4 * s);
+  for (int k = 0; k < 16; ++k) {
+    const int h = k >> 3, i = k & 7;
+    const float2 vk = v[k];
+    // No product below feeds a packed add or subtract: ptxas may contract a
+    // mul.f32x2 -> add.f32x2 pair into one fused operation even with .rn,
+    // which rounds once instead of twice.  Products that are added to are
+    // scalar __fmul_rn / __fadd_rn / __fsub_rn, which are never fused.
+    float tx = __fmul_rn(vk.x, c76), ty = __fmul_rn(vk.y, c76);
+    if (CLAMP) {
+      tx = fminf(fmaxf(tx, -7.25f), 7.25f);
+      ty = fminf(fmaxf(ty, -7.25f), 7.25f);
     }
+    const float2 tm = make_float2(__fadd_rn(tx, kMagic), __fadd_rn(ty, kMagic));
+    const float2 kf = sub2(tm, make_float2(kMagic, kMagic));    // rint(t), exact
+    const float2 hv = mul2(kf, make_float2(c67, c67));
+    const float2 dint = make_float2(__fsub_rn(vk.x, hv.x), __fsub_rn(vk.y, hv.y));
+    efp = fma2(make_float2(da[k], db[k]), make_float2(da[k], db[k]), efp);
+    eint = fma2(dint, dint, eint);
+    ia[h] += __float_as_uint(tm.x) << (4 * i);
+    ib[h] += __float_as_uint(tm.y) << (4 * i);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    ia[h] = (ia[h] - kPackBias) ^ 0x88888888u;
+    ib[h] = (ib[h] - kPackBias) ^ 0x88888888u;
   }
   int_a = eint.x < efp.x;
   int_b = eint.y < efp.y;
@@ -95,45 +130,43 @@ __device__ __forceinline__ void if4_pair(const float (&xa)[16], const float (&xb
   wb[1] = int_b ? ib[1] : fpb[1];
 }
 
-template <typename T>
-__device__ __forceinline__ void load_pair(const T *p, float (&xa)[16], float (&xb)[16],
-                                          float &ma, float &mb) {
-  if (sizeof(T) == 2) {
-    const uint4 *q = reinterpret_cast<const uint4 *>(p);
-    const uint4 u0 = __ldg(q), u1 = __ldg(q + 1), u2 = __ldg(q + 2), u3 = __ldg(q + 3);
-    ma = bf16x2_hmax(maxabs_bf16x2(maxabs_bf16x2(maxabs_bf16x2(u0.x, u0.y), maxabs_bf16x2(u0.z, u0.w)),
-                                   maxabs_bf16x2(maxabs_bf16x2(u1.x, u1.y), maxabs_bf16x2(u1.z, u1.w))));
-    mb = bf16x2_hmax(maxabs_bf16x2(maxabs_bf16x2(maxabs_bf16x2(u2.x, u2.y), maxabs_bf16x2(u2.z, u2.w)),
-                                   maxabs_bf16x2(maxabs_bf16x2(u3.x, u3.y), maxabs_bf16x2(u3.z, u3.w))));
-    const uint32_t wa[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-    const uint32_t wb[8] = {u2.x, u2.y, u2.z, u2.w, u3.x, u3.y, u3.z, u3.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      xa[2 * i] = bf16_lo(wa[i]); xa[2 * i + 1] = bf16_hi(wa[i]);
-      xb[2 * i] = bf16_lo(wb[i]); xb[2 * i + 1] = bf16_hi(wb[i]);
-    }
-  } else {
-    const float4 *q = reinterpret_cast<const float4 *>(p);
-    ma = mb = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 a = __ldg(q + i), b = __ldg(q + 4 + i);
-      xa[4 * i] = a.x; xa[4 * i + 1] = a.y; xa[4 * i + 2] = a.z; xa[4 * i + 3] = a.w;
-      xb[4 * i] = b.x; xb[4 * i + 1] = b.y; xb[4 * i + 2] = b.z; xb[4 * i + 3] = b.w;
-    }
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      ma = fmaxf(ma, fabsf(xa[k]));
-      mb = fmaxf(mb, fabsf(xb[k]));
+__device__ __forceinline__ void async_copy16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Position of a lane's pair: row r and first block cb = 2 * pc, advanced by
+// a fixed stride of pairs.
+struct Cursor {
+  int64_t p, r, pc;
+  __device__ __forceinline__ void init(int64_t p0, int64_t ppr) {
+    p = p0;
+    r = p0 / ppr;
+    pc = p0 - r * ppr;
+  }
+  __device__ __forceinline__ void advance(int64_t stride, int64_t dr, int64_t dpc, int64_t ppr) {
+    p += stride;
+    r += dr;
+    pc += dpc;
+    if (pc >= ppr) {
+      pc -= ppr;
+      ++r;
     }
   }
-}
+};
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads, 2)
+template <typename T, bool SWZ>
+__global__ void __launch_bounds__(kThreads, 4)
 if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
            const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
-           uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int scale_layout) {
+           uint8_t *__restrict__ q, uint8_t *__restrict__ sf) {
+  constexpr int LB = 32 * sizeof(T);          // bytes of a lane's pair
+  constexpr int PPL = LB / 16;                // 16-byte pieces per lane
+  constexpr int PPB = PPL / 2;                // pieces per block
+  constexpr int STAGE = 32 * LB;              // bytes of a warp's stage
+  extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float rtab[128];
   const TensorScale ts = tensor_scale(*amax_ptr);
   fill_factor_table(rtab, ts.enc);
@@ -142,53 +175,107 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
   const float c76 = __fdiv_rn(7.0f, 6.0f);   // RN(7/6)
   const float c67 = __fdiv_rn(6.0f, 7.0f);   // RN(6/7)
 
-  // work unit: a pair of adjacent blocks (b, b+1) of one row; an odd last
-  // block of a row pairs with itself
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // piece i of this lane sits in slot i ^ swz: eight consecutive lanes then
+  // cover eight distinct 16-byte bank groups
+  const int swz = PPL == 4 ? ((lane >> 1) & 3) : (lane & 7);
+  const uint32_t my_s = static_cast<uint32_t>(__cvta_generic_to_shared(smem)) +
+                        static_cast<uint32_t>(warp * kStages * STAGE + lane * LB);
+  const uint8_t *my_g = smem + warp * kStages * STAGE + lane * LB;
+
+  // work unit: a pair of adjacent blocks (cb, cb + 1) of one row; an odd
+  // last block of a row pairs with itself
   const int64_t bpr = cols / 16, ppr = (bpr + 1) / 2, npairs = rows * ppr;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  for (int64_t p = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; p < npairs;
-       p += stride) {
-    const int64_t r = p / ppr, cb = 2 * (p - r * ppr);
+  const int64_t p0 = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+  const int64_t dr = stride / ppr, dpc = stride - dr * ppr;
+
+  auto issue = [&](const Cursor &c, int st) {
+    if (c.p >= npairs) return;
+    const int64_t cb = 2 * c.pc;
+    const uint8_t *src = reinterpret_cast<const uint8_t *>(x + c.r * ld + cb * 16);
+    const int n = (cb + 1 < bpr) ? PPL : PPB;
+    const uint32_t dst = my_s + static_cast<uint32_t>(st * STAGE);
+#pragma unroll
+    for (int i = 0; i < PPL; ++i)
+      if (i < n) async_copy16(dst + static_cast<uint32_t>((i ^ swz) * 16), src + 16 * i);
+  };
+
+  Cursor ci, cc;
+  ci.init(p0, ppr);
+  cc = ci;
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    issue(ci, s);
+    async_commit();
+    ci.advance(stride, dr, dpc, ppr);
+  }
+  for (int st = 0; cc.p < npairs; st = (st + 1 == kStages ? 0 : st + 1)) {
+    issue(ci, st == 0 ? kStages - 1 : st - 1);
+    async_commit();
+    ci.advance(stride, dr, dpc, ppr);
+    async_wait<kStages - 1>();
+
+    const int64_t r = cc.r, cb = 2 * cc.pc;
     const bool has_b = cb + 1 < bpr;
-    float xa[16], xb[16], ma, mb;
-    if (has_b) {
-      load_pair<T>(x + r * ld + cb * 16, xa, xb, ma, mb);
+    const uint8_t *buf = my_g + st * STAGE;
+    float2 v[16];
+    float ma, mb;
+    if (sizeof(T) == 2) {
+      uint4 u[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) u[i] = *reinterpret_cast<const uint4 *>(buf + 16 * (i ^ swz));
+      if (!has_b) { u[2] = u[0]; u[3] = u[1]; }   // a single trailing block: its copy is discarded
+      ma = bf16x2_hmax(maxabs_bf16x2(maxabs_bf16x2(maxabs_bf16x2(u[0].x, u[0].y), maxabs_bf16x2(u[0].z, u[0].w)),
+                                     maxabs_bf16x2(maxabs_bf16x2(u[1].x, u[1].y), maxabs_bf16x2(u[1].z, u[1].w))));
+      mb = bf16x2_hmax(maxabs_bf16x2(maxabs_bf16x2(maxabs_bf16x2(u[2].x, u[2].y), maxabs_bf16x2(u[2].z, u[2].w)),
+                                     maxabs_bf16x2(maxabs_bf16x2(u[3].x, u[3].y), maxabs_bf16x2(u[3].z, u[3].w))));
+      const uint32_t wa[8] = {u[0].x, u[0].y, u[0].z, u[0].w, u[1].x, u[1].y, u[1].z, u[1].w};
+      const uint32_t wb[8] = {u[2].x, u[2].y, u[2].z, u[2].w, u[3].x, u[3].y, u[3].z, u[3].w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = make_float2(bf16_lo(wa[i]), bf16_lo(wb[i]));
+        v[2 * i + 1] = make_float2(bf16_hi(wa[i]), bf16_hi(wb[i]));
+      }
     } else {
-      // a single trailing block: load it into both lanes (the copy is discarded)
-      if (sizeof(T) == 2) {
-        const uint4 *qq = reinterpret_cast<const uint4 *>(x + r * ld + cb * 16);
-        const uint4 u0 = __ldg(qq), u1 = __ldg(qq + 1);
-        ma = bf16x2_hmax(maxabs_bf16x2(maxabs_bf16x2(maxabs_bf16x2(u0.x, u0.y), maxabs_bf16x2(u0.z, u0.w)),
-                                       maxabs_bf16x2(maxabs_bf16x2(u1.x, u1.y), maxabs_bf16x2(u1.z, u1.w))));
-        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      float4 a[4], b[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) { xa[2 * i] = bf16_lo(w[i]); xa[2 * i + 1] = bf16_hi(w[i]); }
-      } else {
-        const float4 *qq = reinterpret_cast<const float4 *>(x + r * ld + cb * 16);
-        ma = 0.0f;
+      for (int i = 0; i < 4; ++i) {
+        a[i] = *reinterpret_cast<const float4 *>(buf + 16 * (i ^ swz));
+        b[i] = *reinterpret_cast<const float4 *>(buf + 16 * ((i + 4) ^ swz));
+      }
+      if (!has_b) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 a = __ldg(qq + i);
-          xa[4 * i] = a.x; xa[4 * i + 1] = a.y; xa[4 * i + 2] = a.z; xa[4 * i + 3] = a.w;
-        }
+        for (int i = 0; i < 4; ++i) b[i] = a[i];
+      }
+      ma = mb = 0.0f;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) ma = fmaxf(ma, fabsf(xa[k]));
+      for (int i = 0; i < 4; ++i) {
+        v[4 * i] = make_float2(a[i].x, b[i].x);
+        v[4 * i + 1] = make_float2(a[i].y, b[i].y);
+        v[4 * i + 2] = make_float2(a[i].z, b[i].z);
+        v[4 * i + 3] = make_float2(a[i].w, b[i].w);
       }
 #pragma unroll
-      for (int k = 0; k < 16; ++k) xb[k] = xa[k];
-      mb = ma;
+      for (int k = 0; k < 16; ++k) {
+        ma = fmaxf(ma, fabsf(v[k].x));
+        mb = fmaxf(mb, fabsf(v[k].y));
+      }
     }
     const uint32_t sa = nvfp4_scale_code(ma, ts.enc), sb = nvfp4_scale_code(mb, ts.enc);
     const float fa = rtab[sa], fb = rtab[sb];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = mul2(v[k], make_float2(fa, fb));
     // |t| of the block maximum: the clamp can only bind when it reaches 7.5
     const float ta = __fmul_rn(__fmul_rn(ma, fa), c76), tb = __fmul_rn(__fmul_rn(mb, fb), c76);
     uint32_t wa[2], wb[2];
     bool ia, ib;
     if (ta < 7.5f && tb < 7.5f)
-      if4_pair<T, false>(xa, xb, fa, fb, c76, c67, wa, wb, ia, ib);
+      if4_pair<false>(v, c76, c67, wa, wb, ia, ib);
     else
-      if4_pair<T, true>(xa, xb, fa, fb, c76, c67, wa, wb, ia, ib);
+      if4_pair<true>(v, c76, c67, wa, wb, ia, ib);
     uint8_t *qp = q + r * (cols / 2) + cb * 8;
+    const uint32_t ba = sa | (ia ? 0x80u : 0u), bb = sb | (ib ? 0x80u : 0u);
     if (has_b) {
       if ((cols & 31) == 0) {
         *reinterpret_cast<uint4 *>(qp) = make_uint4(wa[0], wa[1], wb[0], wb[1]);
@@ -196,12 +283,59 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
         *reinterpret_cast<uint2 *>(qp) = make_uint2(wa[0], wa[1]);
         *reinterpret_cast<uint2 *>(qp + 8) = make_uint2(wb[0], wb[1]);
       }
-      sf[scale_offset(r, cb + 1, bpr, scale_layout)] = static_cast<uint8_t>(sb | (ib ? 0x80u : 0u));
     } else {
       *reinterpret_cast<uint2 *>(qp) = make_uint2(wa[0], wa[1]);
     }
-    sf[scale_offset(r, cb, bpr, scale_layout)] = static_cast<uint8_t>(sa | (ia ? 0x80u : 0u));
+    if (SWZ) {
+      // (cb, cb + 1) are adjacent bytes of one 4-column group (cb even, and
+      // bpr % 4 == 0 gives every block a partner)
+      const int64_t tile = (r >> 7) * (bpr >> 2) + (cb >> 2);
+      const int64_t o = tile * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (cb & 3);
+      sf[o] = static_cast<uint8_t>(ba);
+      sf[o + 1] = static_cast<uint8_t>(bb);
+    } else {
+      sf[r * bpr + cb] = static_cast<uint8_t>(ba);
+      if (has_b) sf[r * bpr + cb + 1] = static_cast<uint8_t>(bb);
+    }
+    cc.advance(stride, dr, dpc, ppr);
   }
+  async_wait<0>();
+}
+
+template <typename T, bool SWZ>
+cudaError_t launch_t(const T *x, int64_t rows, int64_t cols, int64_t ld, const float *amax,
+                     float *s_dec_out, uint8_t *q, uint8_t *sf, const Launch &L) {
+  constexpr int SMEM = kWarps * kStages * 32 * 32 * static_cast<int>(sizeof(T));
+  const void *kern = reinterpret_cast<const void *>(if4_kernel<T, SWZ>);
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
+        cudaSuccess)
+      return cudaGetLastError();
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, SMEM) !=
+            cudaSuccess ||
+        per_sm < 1) {
+      cudaGetLastError();
+      per_sm = 1;
+    }
+  }
+  const int64_t npairs = rows * ((cols / 16 + 1) / 2);
+  const int64_t want = (npairs + kThreads - 1) / kThreads;
+  const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
+  const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+  if4_kernel<T, SWZ><<<grid, kThreads, SMEM, L.stream>>>(x, rows, cols, ld, amax, s_dec_out, q,
+                                                         sf);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_layout(const void *x, int64_t rows, int64_t cols, int64_t ld,
+                          const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,
+                          int scale_layout, const Launch &L) {
+  const T *p = static_cast<const T *>(x);
+  if (scale_layout == FP4Q_SCALE_SWIZZLED_128x4)
+    return launch_t<T, true>(p, rows, cols, ld, amax, s_dec_out, q, sf, L);
+  return launch_t<T, false>(p, rows, cols, ld, amax, s_dec_out, q, sf, L);
 }
 
 }  // namespace
@@ -209,18 +343,10 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
 cudaError_t launch_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                        const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,
                        int scale_layout, const Launch &L) {
-  const int64_t npairs = rows * ((cols / 16 + 1) / 2);
-  int64_t want = (npairs + kThreads - 1) / kThreads;
-  int64_t cap = static_cast<int64_t>(L.num_sms) * 8;
-  int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
   if (dtype == FP4Q_BF16)
-    if4_kernel<__nv_bfloat16><<<grid, kThreads, 0, L.stream>>>(
-        static_cast<const __nv_bfloat16 *>(x), rows, cols, ld, amax, s_dec_out, q, sf,
-        scale_layout);
-  else
-    if4_kernel<float><<<grid, kThreads, 0, L.stream>>>(static_cast<const float *>(x), rows, cols,
-                                                       ld, amax, s_dec_out, q, sf, scale_layout);
-  return cudaGetLastError();
+    return launch_layout<__nv_bfloat16>(x, rows, cols, ld, amax, s_dec_out, q, sf, scale_layout,
+                                        L);
+  return launch_layout<float>(x, rows, cols, ld, amax, s_dec_out, q, sf, scale_layout, L);
 }
 
 }  // namespace fp4q

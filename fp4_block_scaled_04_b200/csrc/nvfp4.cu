@@ -9,14 +9,18 @@
 //
 // rowwise_kernel  one thread per block of 16 (NVFP4) or 32 (MXFP4) values of
 //                 a row, two blocks per iteration; 128-bit loads.
-// rowcol_kernel   register-tiled, no shared memory.  A thread owns 16 rows x
-//                 one 16-byte column chunk (8 BF16 or 4 FP32 columns); a warp
-//                 owns 64 rows x 8 chunks (lane = chunk + 8 * row band).
-//                 Pass 1 takes row and column block maxima on the packed
-//                 data (row blocks span 2..8 lanes: shuffle), pass 2 scales
-//                 and encodes every element twice.  Row codes of a warp
-//                 instruction are 8 lanes x 4 bytes of one row, column codes
-//                 4 lanes x 8 bytes of one column: whole 32-byte sectors.
+// rowcol_kernel   register tiles fed by a two-stage cp.async buffer.  A
+//                 warp owns 64 rows x 128 bytes (8 16-byte chunks of 8 BF16
+//                 or 4 FP32 columns) and copies the next such tile into
+//                 shared memory while it computes this one; each warp copy
+//                 instruction moves four whole 128-byte row segments.  A
+//                 thread works on 16 rows x one chunk (lane = chunk + 8 * row
+//                 band).  Pass 1 takes row and column block maxima on the
+//                 packed data (row blocks span 2..8 lanes: shuffle), pass 2
+//                 reads the rows again and scales and encodes every element
+//                 twice.  Row codes of a warp instruction are 8 lanes x 4
+//                 bytes of one row, column codes 4 lanes x 8 bytes of one
+//                 column: whole 32-byte sectors.
 #include "common.cuh"
 #include "launch.h"
 
@@ -246,8 +250,18 @@ __device__ __forceinline__ uint32_t block_scale(float m, const TensorScale &ts, 
   return code;
 }
 
+__device__ __forceinline__ void rc_copy16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void rc_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void rc_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void rc_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+constexpr int kRCTileBytes = 64 * 128;            // one warp tile: 64 rows x 128 bytes
+constexpr int kRCSmem = (kRCThreads / 32) * 2 * kRCTileBytes;
+
 template <typename T, bool MX, bool SR>
-__global__ void __launch_bounds__(kRCThreads)
+__global__ void __launch_bounds__(kRCThreads, SR ? 2 : 3)
 rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, unsigned layouts,
               const float *__restrict__ amax_ptr, int e8m0_mode, uint64_t seed,
               float *__restrict__ s_dec_out, uint8_t *__restrict__ q_row,
@@ -271,16 +285,42 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
   const int64_t ntiles = tiles_c * ((rows + G::WR - 1) / G::WR);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kRCThreads / 32);
   const bool swz = scale_layout == FP4Q_SCALE_SWIZZLED_128x4;
-  for (int64_t tile = static_cast<int64_t>(blockIdx.x) * (kRCThreads / 32) + (threadIdx.x >> 5);
-       tile < ntiles; tile += nwarps) {
+  extern __shared__ __align__(16) uint8_t rc_smem[];
+  const int warp = threadIdx.x >> 5;
+  const uint32_t stage_s = static_cast<uint32_t>(__cvta_generic_to_shared(rc_smem)) +
+                           static_cast<uint32_t>(warp * 2 * kRCTileBytes);
+  const uint4 *stage_g = reinterpret_cast<const uint4 *>(rc_smem + warp * 2 * kRCTileBytes);
+  // lane L copies the 16-byte pieces L + 32 i: row (L + 32 i) / 8, chunk L % 8
+  auto issue = [&](int64_t t, int st) {
+    const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+    const int64_t col = tc * G::WC + cc * CPT;
+    if (col >= cols) return;
+    const uint32_t dst = stage_s + static_cast<uint32_t>(st * kRCTileBytes + cc * 16);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int row = (lane >> 3) + 4 * i;
+      if (tr * G::WR + row < rows)
+        rc_copy16(dst + static_cast<uint32_t>(row * 128), x + (tr * G::WR + row) * ld + col);
+    }
+  };
+  int64_t tile = static_cast<int64_t>(blockIdx.x) * (kRCThreads / 32) + warp;
+  if (tile < ntiles) issue(tile, 0);
+  rc_commit();
+  for (int st = 0; tile < ntiles; tile += nwarps, st ^= 1) {
+    __syncwarp();   // every lane is done with stage st ^ 1 before it is refilled
+    if (tile + nwarps < ntiles) issue(tile + nwarps, st ^ 1);
+    rc_commit();
+    rc_wait_1();
+    __syncwarp();
     const int64_t tr = tile / tiles_c, tc = tile - tr * tiles_c;
     const int64_t r0 = tr * G::WR + band * 16, c0 = tc * G::WC + cc * CPT;
     const bool valid = r0 < rows && c0 < cols;
+    // row k of this thread's 16: tb[8 * k] (rows outside the matrix are never
+    // copied; their lanes' values only meet other outside lanes and are not stored)
+    const uint4 *tb = stage_g + st * (kRCTileBytes / 16) + band * 16 * 8 + cc;
     uint4 d[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k)
-      d[k] = valid ? __ldg(reinterpret_cast<const uint4 *>(x + (r0 + k) * ld + c0))
-                   : make_uint4(0u, 0u, 0u, 0u);
+    for (int k = 0; k < 16; ++k) d[k] = tb[8 * k];
 
     // ---- pass 1: block maxima --------------------------------------------
     float rmax[16];
@@ -346,12 +386,14 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
     }
 
     // ---- pass 2: encode, four rows at a time ----------------------------------
+    // read the rows from shared memory again rather than keeping all 16 live
+    asm volatile("" ::: "memory");
     uint32_t colw[CPT][2];
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
       float v[4][CPT];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) unpack_chunk<T>(d[4 * q4 + i], v[i]);
+      for (int i = 0; i < 4; ++i) unpack_chunk<T>(tb[8 * (4 * q4 + i)], v[i]);
       uint32_t u[4][CPT];
       if (SR) {
         // one Philox call covers the 8 columns of a row from a multiple of 8
@@ -430,6 +472,7 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
             make_uint2(colw[j][0], colw[j][1]);
     }
   }
+  rc_wait_0();
 }
 
 int grid_cap(const void *kernel, int threads, const Launch &L) {
@@ -460,12 +503,23 @@ cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, uns
   } else {
     using G = RCGeom<T, MX>;
     const int64_t ntiles = ((cols + G::WC - 1) / G::WC) * ((rows + G::WR - 1) / G::WR);
-    static int cap = 0;
-    if (cap == 0) cap = grid_cap(reinterpret_cast<const void *>(rowcol_kernel<T, MX, SR>),
-                                 kRCThreads, L);
+    const void *kern = reinterpret_cast<const void *>(rowcol_kernel<T, MX, SR>);
+    static int per_sm = 0;
+    if (per_sm == 0) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRCSmem) !=
+          cudaSuccess)
+        return cudaGetLastError();
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRCThreads, kRCSmem) !=
+              cudaSuccess ||
+          per_sm < 1) {
+        cudaGetLastError();
+        per_sm = 1;
+      }
+    }
+    const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
     const int64_t want = (ntiles + kRCThreads / 32 - 1) / (kRCThreads / 32);
     const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-    rowcol_kernel<T, MX, SR><<<grid, kRCThreads, 0, L.stream>>>(
+    rowcol_kernel<T, MX, SR><<<grid, kRCThreads, kRCSmem, L.stream>>>(
         x, rows, cols, ld, layouts, amax, e8m0_mode, seed, s_dec_out, q_row, sf_row, q_col,
         sf_col, scale_layout);
   }
