@@ -47,9 +47,6 @@ template <> struct Vec8<float> {
   }
 };
 
-__device__ __forceinline__ float to_f32(__nv_bfloat16 h) { return __bfloat162float(h); }
-__device__ __forceinline__ float to_f32(float f) { return f; }
-
 // ---------------------------------------------------------------------------
 // E2M1 encode / decode
 // ---------------------------------------------------------------------------
@@ -90,19 +87,6 @@ __device__ __forceinline__ uint32_t e2m1x4(float f0, float f1, float f2, float f
       "cvt.u32.u16 %0, h;\n\t}"
       : "=r"(r) : "f"(f0), "f"(f1), "f"(f2), "f"(f3));
   return r;
-}
-
-// E2M1 magnitude of a 3-bit code: 0, .5, 1, 1.5, 2, 3, 4, 6.
-__device__ __forceinline__ float e2m1_magnitude(uint32_t c3) {
-  // codes 2..7 are normal: exponent (c3 >> 1) - 1, one mantissa bit (c3 & 1)
-  uint32_t normal = ((((c3 >> 1) + 126u) << 23) | ((c3 & 1u) << 22));
-  float v = __uint_as_float(normal);
-  return c3 >= 2 ? v : (c3 == 1 ? 0.5f : 0.0f);
-}
-
-__device__ __forceinline__ float e2m1_value(uint32_t code) {
-  float m = e2m1_magnitude(code & 7u);
-  return (code & 8u) ? -m : m;
 }
 
 // ---------------------------------------------------------------------------
@@ -231,13 +215,6 @@ __device__ __forceinline__ float e8m0_inverse(uint32_t byte) {
   return byte == 254u ? __uint_as_float(0x00400000u) : __uint_as_float((254u - byte) << 23);
 }
 
-// 2^-e as a float, e in [-127, 127] (2^-127 is subnormal, the rest normal).
-__device__ __forceinline__ float exp2_neg(int e) {
-  int k = -e;
-  if (k >= -126) return __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
-  return __uint_as_float(0x00400000u);  // 2^-127
-}
-
 // 2^e as a float for a stored E8M0 byte (e = byte - 127, e <= 127).
 __device__ __forceinline__ float e8m0_value(uint32_t byte) {
   if (byte == 0) return __uint_as_float(0x00400000u);
@@ -249,52 +226,6 @@ __device__ __forceinline__ float e8m0_value(uint32_t byte) {
 // ---------------------------------------------------------------------------
 
 struct U32x4 { uint32_t x, y, z, w; };
-
-__device__ __forceinline__ U32x4 philox4x32_10(U32x4 c, uint32_t k0, uint32_t k1) {
-#pragma unroll
-  for (int i = 0; i < 10; ++i) {
-    uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
-    uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
-    U32x4 n = {hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0};
-    c = n;
-    k0 += 0x9E3779B9u;
-    k1 += 0xBB67AE85u;
-  }
-  return c;
-}
-
-// 16 random bits for elements 8g .. 8g+7 (flat input index) of a seed.
-__device__ __forceinline__ U32x4 sr_bits_group(uint64_t seed, uint64_t g) {
-  U32x4 c = {static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u};
-  return philox4x32_10(c, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
-}
-
-__device__ __forceinline__ uint32_t half16(const U32x4 &w, int j) {
-  uint32_t word = (j >> 1) == 0 ? w.x : (j >> 1) == 1 ? w.y : (j >> 1) == 2 ? w.z : w.w;
-  return (j & 1) ? (word >> 16) : (word & 0xFFFFu);
-}
-
-// Stochastic rounding of v onto E2M1: between adjacent magnitudes
-// lo <= |v| < hi round up iff u < (|v| - lo) / (hi - lo) * 2^16; |v| >= 6 -> 6;
-// the sign is copied.  Returns the 4-bit code.
-__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t u16) {
-  float a = fabsf(v);
-  uint32_t sign = (__float_as_uint(v) >> 28) & 8u;
-  uint32_t code;
-  if (a >= 6.0f) {
-    code = 7u;
-  } else {
-    // lower neighbour: codes 0..7 at 0, .5, 1, 1.5, 2, 3, 4, 6
-    uint32_t lo = (a >= 0.5f) + (a >= 1.0f) + (a >= 1.5f) + (a >= 2.0f) + (a >= 3.0f) +
-                  (a >= 4.0f);
-    float lo_v = e2m1_magnitude(lo);
-    // spacing to the next value: .5 below 2, 1 in [2, 4), 2 in [4, 6)
-    float inv_gap_2p16 = lo >= 6 ? 32768.0f : (lo >= 4 ? 65536.0f : 131072.0f);
-    float t16 = __fmul_rn(__fsub_rn(a, lo_v), inv_gap_2p16);  // exact
-    code = lo + (static_cast<float>(u16) < t16 ? 1u : 0u);
-  }
-  return code | sign;
-}
 
 // ---------------------------------------------------------------------------
 // scale-factor layouts
@@ -372,28 +303,27 @@ __device__ __forceinline__ float absmax8(uint4 u) {
   return bf16x2_hmax(maxabs_bf16x2(maxabs_bf16x2(u.x, u.y), maxabs_bf16x2(u.z, u.w)));
 }
 
-// E2M1 codes of two floats as the low byte of a 32-bit register
-__device__ __forceinline__ uint32_t e2m1_byte(float lo, float hi) { return e2m1x2(lo, hi); }
-
-// Stochastic rounding onto E2M1 by integer comparisons (same rule as
-// e2m1_sr): for |v| in [1, 6) the grid has one mantissa bit and t * 2^16 is
-// the low 22 mantissa bits / 64; in [0.5, 1) the spacing is 0.5 and t * 2^16
-// is the 23 mantissa bits / 128; below 0.5, t * 2^16 = |v| * 2^17.
-__device__ __forceinline__ uint32_t e2m1_sr_bits(float v, uint32_t u16) {
-  const uint32_t raw = __float_as_uint(v);
-  const uint32_t sign = (raw >> 28) & 8u;
-  const uint32_t b = raw & 0x7FFFFFFFu;
-  const bool ge1 = b >= 0x3F800000u;
-  const uint32_t shifted = ge1 ? (u16 << 6) : (u16 << 7);
-  const uint32_t frac = ge1 ? (b & 0x3FFFFFu) : (b & 0x7FFFFFu);
-  const uint32_t base = ge1 ? (b >> 22) - 252u : 1u;
-  uint32_t code = base + (shifted < frac ? 1u : 0u);
-  const uint32_t small =
-      (static_cast<float>(u16) < __fmul_rn(__uint_as_float(b), 131072.0f)) ? 1u : 0u;
-  code = b >= 0x3F000000u ? code : small;
-  code = b >= 0x40C00000u ? 7u : code;
-  return code | sign;
+// Stochastic rounding of v onto the E2M1 grid, returned as a float that the
+// round-to-nearest conversion (cvt.rn.satfinite.e2m1x2) then encodes exactly
+// (the oracle's rule: the magnitude goes up iff u < t * 2^16).  On
+// [1, 8) E2M1 is a float with one mantissa bit, so adding 0x3FFFFF - 64 u to
+// the bits and clearing the low 22 rounds up exactly when 64 u < frac; below
+// 1 the spacing 0.5 equals that of [1, 2), so w = RU(|v| + 1) is rounded the
+// same way and 1 subtracted again (rounding the sum up keeps the comparison
+// with the integer 64 u exact).  Values rounded to 8 saturate to 6 in the
+// conversion; the sign is copied.  Checked against the oracle by
+// tests/sr_check.c (method 1).  z = 0x3FFFFF - 64 u.
+__device__ __forceinline__ float e2m1_sr_value(float v, uint32_t z) {
+  const float av = fabsf(v);
+  const float a = av < 1.0f ? 1.0f : 0.0f;
+  const float w = __fadd_ru(av, a);
+  const float r = __fsub_rn(__uint_as_float((__float_as_uint(w) + z) & 0xFFC00000u), a);
+  return __uint_as_float(__float_as_uint(r) | (__float_as_uint(v) & 0x80000000u));
 }
+// z of a 16-bit uniform, and of the low / high 16-bit uniform of a 32-bit word
+__device__ __forceinline__ uint32_t sr_z(uint32_t u16) { return 0x3FFFFFu ^ (u16 << 6); }
+__device__ __forceinline__ uint32_t sr_z_lo(uint32_t w) { return 0x3FFFFFu ^ ((w << 6) & 0x3FFFC0u); }
+__device__ __forceinline__ uint32_t sr_z_hi(uint32_t w) { return 0x3FFFFFu ^ ((w >> 10) & 0x3FFFC0u); }
 
 // Philox4x32-10 with the round keys held by the caller (they depend only on
 // the seed).
@@ -425,12 +355,6 @@ __device__ __forceinline__ U32x4 philox(const PhiloxKey &K, uint32_t c0, uint32_
     c2 = n2;
   }
   return U32x4{c0, c1, c2, c3};
-}
-
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
 }
 
 }  // namespace fp4q

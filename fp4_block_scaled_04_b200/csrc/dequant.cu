@@ -32,16 +32,6 @@ namespace {
 
 constexpr int kThreads = 256;
 
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
-  uint32_t h2;
-  asm("{\n\t.reg .b8 q;\n\t.reg .b16 w;\n\t"
-      "cvt.u16.u32 w, %1;\n\t"
-      "cvt.u8.u16 q, w;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, q;\n\t}"
-      : "=r"(h2) : "r"(byte));
-  return h2;
-}
-
 // (S, S) in f16 from a 7-bit E4M3 code
 __device__ __forceinline__ uint32_t e4m3_to_f16x2_dup(uint32_t code7) {
   uint32_t h2;
@@ -67,12 +57,6 @@ __device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t h) {
   return __half22float2(v);
 }
 
-// (k0, k1) in f16 for the two two's-complement nibbles of `byte`
-__device__ __forceinline__ uint32_t int4x2_to_f16x2(uint32_t byte) {
-  const uint32_t t = ((byte * 0x1001u) & 0x000F000Fu) ^ 0x64086408u;  // 1024 + (n ^ 8)
-  return hsub2_bits(t, 0x64086408u);                                   // - 1032
-}
-
 struct Store {
   __device__ __forceinline__ static void put(float *y, const float2 (&v)[4]) {
     float4 *p = reinterpret_cast<float4 *>(y);
@@ -90,31 +74,55 @@ struct Store {
   }
 };
 
+// The four E2M1 pairs of a code word as f16x2 (byte i -> element pair i).
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t codes, uint32_t (&h)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(codes));
+}
+
+// The four INT4 pairs of a code word as f16x2 k values: for byte i the
+// permute puts its low nibble in bits 0..3 and (from codes >> 4) its high
+// nibble in bits 16..19; then 1024 + (n ^ 8) - 1032 = k exactly in f16.
+__device__ __forceinline__ void int4x8_to_f16x2(uint32_t codes, uint32_t (&h)[4]) {
+  const uint32_t hi = codes >> 4;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t t = (__byte_perm(codes, hi, 0x0400u | (0x0101u * i)) & 0x000F000Fu) ^ 0x64086408u;
+    h[i] = hsub2_bits(t, 0x64086408u);
+  }
+}
+
 // 8 values of one unit: 4 code bytes (element 2i in the low nibble)
 template <int FMT>
 __device__ __forceinline__ void decode8(uint32_t codes, uint32_t sbyte, float s_dec, float c67,
                                         float2 (&v)[4]) {
   const float2 sd = make_float2(s_dec, s_dec);
+  uint32_t g[4];
+  e2m1x8_to_f16x2(codes, g);
   if (FMT == FP4Q_FMT_MXFP4) {
     const float p = e8m0_value(sbyte);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      v[i] = mul2(f16x2_to_f32x2(e2m1x2_to_f16x2((codes >> (8 * i)) & 0xFFu)), make_float2(p, p));
+    for (int i = 0; i < 4; ++i) v[i] = mul2(f16x2_to_f32x2(g[i]), make_float2(p, p));
   } else if (FMT == FP4Q_FMT_NVFP4) {
     const uint32_t s2 = e4m3_to_f16x2_dup(sbyte & 0x7Fu);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      v[i] = mul2(f16x2_to_f32x2(hmul2_bits(e2m1x2_to_f16x2((codes >> (8 * i)) & 0xFFu), s2)), sd);
+    for (int i = 0; i < 4; ++i) v[i] = mul2(f16x2_to_f32x2(hmul2_bits(g[i], s2)), sd);
   } else {  // IF4
     const bool int4 = (sbyte & 0x80u) != 0;
     const uint32_t s2 = e4m3_to_f16x2_dup(sbyte & 0x7Fu);
     const float S = __half2float(__ushort_as_half(static_cast<unsigned short>(s2 & 0xFFFFu)));
     const float m = int4 ? c67 : 1.0f;
     const uint32_t pick = int4 ? 0xFFFFFFFFu : 0u;   // select, not branch, per pair
+    uint32_t k[4];
+    int4x8_to_f16x2(codes, k);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t byte = (codes >> (8 * i)) & 0xFFu;
-      const uint32_t h = (int4x2_to_f16x2(byte) & pick) | (e2m1x2_to_f16x2(byte) & ~pick);
+      const uint32_t h = (k[i] & pick) | (g[i] & ~pick);
       v[i] = mul2(mul2(mul2(f16x2_to_f32x2(h), make_float2(m, m)), make_float2(S, S)), sd);
     }
   }
@@ -122,68 +130,67 @@ __device__ __forceinline__ void decode8(uint32_t codes, uint32_t sbyte, float s_
 
 // Byte offset of the scale of the 8-element unit starting at (r, c) (SWZ:
 // the 128x4 tile layout; BROWS == 16: the linear [rows/16, cols/16] tile
-// matrix).
-template <int BLK, int BROWS, bool SWZ>
-__device__ __forceinline__ int64_t unit_scale(int64_t r, int64_t c, int64_t cols) {
-  const int64_t sc = BLK == 32 ? (c >> 5) : (c >> 4);   // c, cols >= 0
-  const int64_t scols = BLK == 32 ? (cols >> 5) : (cols >> 4);
+// matrix).  I is the index type: 32-bit when every index fits.
+template <int BLK, int BROWS, bool SWZ, typename I>
+__device__ __forceinline__ I unit_scale(I r, I c, I cols) {
+  const I sc = BLK == 32 ? (c >> 5) : (c >> 4);   // c, cols >= 0
+  const I scols = BLK == 32 ? (cols >> 5) : (cols >> 4);
   if (BROWS == 16) return (r >> 4) * scols + sc;
   if (!SWZ) return r * scols + sc;
-  const int64_t tile = (r >> 7) * (scols >> 2) + (sc >> 2);
+  const I tile = (r >> 7) * (scols >> 2) + (sc >> 2);
   return tile * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (sc & 3);
 }
 
 // A warp takes NU x 32 consecutive 8-element units per step, lane l the units
 // l, l + 32, ...: every code load and output store of the warp is then one
 // contiguous stretch, and a thread has NU independent loads in flight.
-template <int FMT, int BROWS, bool SWZ, typename OutT>
+template <int FMT, int BROWS, bool SWZ, typename I, typename OutT>
 __global__ void __launch_bounds__(kThreads)
 dequant_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ sf,
-               const float *__restrict__ s_dec_ptr, int64_t rows, int64_t cols,
-               OutT *__restrict__ y) {
+               const float *__restrict__ s_dec_ptr, I rows, I cols, OutT *__restrict__ y) {
   constexpr int NU = 4;
   constexpr int BLK = FMT == FP4Q_FMT_MXFP4 ? 32 : 16;
   constexpr bool FLAT = !SWZ && BROWS == 1;          // scale index from the unit index
   const float s_dec = (FMT == FP4Q_FMT_MXFP4) ? 1.0f : *s_dec_ptr;
   const float c67 = __fdiv_rn(6.0f, 7.0f);
-  const int64_t total = rows * (cols / 8);           // units
-  const int lane = threadIdx.x & 31;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-  const int64_t wstride = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  const I total = rows * (cols / 8);                 // units
+  const I lane = threadIdx.x & 31;
+  const I warp0 = (static_cast<I>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+  const I wstride = static_cast<I>(gridDim.x) * (kThreads / 32);
   const uint32_t *qw = reinterpret_cast<const uint32_t *>(q);
   // (row, column) of each of the lane's NU units, advanced by a fixed stride
-  int64_t r[NU], c[NU];
-  int64_t dr = 0, dc = 0;
+  I r[NU], c[NU];
+  I dr = 0, dc = 0;
   if (!FLAT) {
-    const int64_t estride = wstride * NU * 32 * 8;   // elements per step
+    const I estride = wstride * NU * 32 * 8;         // elements per step
     dr = estride / cols;
     dc = estride - dr * cols;
 #pragma unroll
     for (int j = 0; j < NU; ++j) {
-      const int64_t e = (warp0 * NU * 32 + 32 * j + lane) * 8;
+      const I e = (warp0 * NU * 32 + 32 * j + lane) * 8;
       r[j] = e / cols;
       c[j] = e - r[j] * cols;
     }
   }
-  for (int64_t base = warp0 * NU * 32 + lane; base < total; base += wstride * NU * 32) {
+  for (I base = warp0 * NU * 32 + lane; base < total; base += wstride * NU * 32) {
     uint32_t cw[NU], sb[NU];
 #pragma unroll
     for (int j = 0; j < NU; ++j) {
-      const int64_t u = base + 32 * j;
+      const I u = base + 32 * j;
       if (u < total) {
-        const int64_t si = FLAT ? (BLK == 32 ? (u >> 2) : (u >> 1))
-                                : unit_scale<BLK, BROWS, SWZ>(r[j], c[j], cols);
+        const I si = FLAT ? (BLK == 32 ? (u >> 2) : (u >> 1))
+                          : unit_scale<BLK, BROWS, SWZ, I>(r[j], c[j], cols);
         cw[j] = __ldg(qw + u);
         sb[j] = __ldg(sf + si);
       }
     }
 #pragma unroll
     for (int j = 0; j < NU; ++j) {
-      const int64_t u = base + 32 * j;
+      const I u = base + 32 * j;
       if (u < total) {
         float2 v[4];
         decode8<FMT>(cw[j], sb[j], s_dec, c67, v);
-        Store::put(y + u * 8, v);
+        Store::put(y + static_cast<size_t>(u) * 8, v);
       }
       if (!FLAT) {
         r[j] += dr;
@@ -200,16 +207,31 @@ dequant_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ sf,
 template <int FMT, int BROWS, bool SWZ>
 cudaError_t launch_fmt(const uint8_t *q, const uint8_t *sf, const float *s_dec, int64_t rows,
                        int64_t cols, void *y, int y_dtype, const Launch &L) {
-  const int64_t steps = (rows * (cols / 8) + 4 * kThreads - 1) / (4 * kThreads);
-  const int64_t want = steps;
+  const int64_t units = rows * (cols / 8);
+  const int64_t want = (units + 4 * kThreads - 1) / (4 * kThreads);
   const int64_t cap = static_cast<int64_t>(L.num_sms) * 8;
   const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-  if (y_dtype == FP4Q_BF16)
-    dequant_kernel<FMT, BROWS, SWZ><<<grid, kThreads, 0, L.stream>>>(
-        q, sf, s_dec, rows, cols, static_cast<__nv_bfloat16 *>(y));
-  else
-    dequant_kernel<FMT, BROWS, SWZ><<<grid, kThreads, 0, L.stream>>>(
-        q, sf, s_dec, rows, cols, static_cast<float *>(y));
+  // 32-bit indices when the unit index, stepped once past the end, the
+  // element index of a row start and the scale offsets all stay below 2^31
+  const bool narrow = units + static_cast<int64_t>(grid) * 4 * kThreads < (int64_t(1) << 31) &&
+                      rows * cols < (int64_t(1) << 31);
+  if (y_dtype == FP4Q_BF16) {
+    auto *yp = static_cast<__nv_bfloat16 *>(y);
+    if (narrow)
+      dequant_kernel<FMT, BROWS, SWZ, uint32_t><<<grid, kThreads, 0, L.stream>>>(
+          q, sf, s_dec, static_cast<uint32_t>(rows), static_cast<uint32_t>(cols), yp);
+    else
+      dequant_kernel<FMT, BROWS, SWZ, int64_t><<<grid, kThreads, 0, L.stream>>>(q, sf, s_dec, rows,
+                                                                               cols, yp);
+  } else {
+    auto *yp = static_cast<float *>(y);
+    if (narrow)
+      dequant_kernel<FMT, BROWS, SWZ, uint32_t><<<grid, kThreads, 0, L.stream>>>(
+          q, sf, s_dec, static_cast<uint32_t>(rows), static_cast<uint32_t>(cols), yp);
+    else
+      dequant_kernel<FMT, BROWS, SWZ, int64_t><<<grid, kThreads, 0, L.stream>>>(q, sf, s_dec, rows,
+                                                                               cols, yp);
+  }
   return cudaGetLastError();
 }
 

@@ -90,13 +90,13 @@ __device__ __forceinline__ void encode_sr16(const float (&v)[16], float f, const
     const uint64_t g = g0 + h;
     const U32x4 bits = philox(K, static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u);
     const uint32_t words[4] = {bits.x, bits.y, bits.z, bits.w};
-    uint32_t acc = 0;
+    float t[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const uint32_t u16 = (k & 1) ? (words[k >> 1] >> 16) : (words[k >> 1] & 0xFFFFu);
-      acc |= e2m1_sr_bits(__fmul_rn(v[8 * h + k], f), u16) << (4 * k);
+      const uint32_t z = (k & 1) ? sr_z_hi(words[k >> 1]) : sr_z_lo(words[k >> 1]);
+      t[k] = e2m1_sr_value(__fmul_rn(v[8 * h + k], f), z);
     }
-    w[h] = acc;
+    w[h] = e2m1x8(t);
   }
 }
 
@@ -318,16 +318,16 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
     // row k of this thread's 16: tb[8 * k] (rows outside the matrix are never
     // copied; their lanes' values only meet other outside lanes and are not stored)
     const uint4 *tb = stage_g + st * (kRCTileBytes / 16) + band * 16 * 8 + cc;
-    uint4 d[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) d[k] = tb[8 * k];
-
     // ---- pass 1: block maxima --------------------------------------------
     float rmax[16];
+    uint32_t cm[4] = {0u, 0u, 0u, 0u};
     if (sizeof(T) == 2) {
 #pragma unroll
       for (int k = 0; k < 16; k += 2) {
-        uint32_t pm = rowpair_max_bf16(d[k], d[k + 1]);
+        const uint4 a = tb[8 * k], b = tb[8 * k + 8];
+        chunk_colmax<T>(a, cm);
+        chunk_colmax<T>(b, cm);
+        uint32_t pm = rowpair_max_bf16(a, b);
 #pragma unroll
         for (int o = 1; o < GR; o <<= 1) pm = maxabs_bf16x2(pm, __shfl_xor_sync(0xFFFFFFFFu, pm, o));
         pm &= 0x7FFF7FFFu;
@@ -336,16 +336,17 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
       }
     } else {
 #pragma unroll
-      for (int k = 0; k < 16; ++k) rmax[k] = chunk_rowmax<T>(d[k]);
+      for (int k = 0; k < 16; ++k) {
+        const uint4 a = tb[8 * k];
+        chunk_colmax<T>(a, cm);
+        rmax[k] = chunk_rowmax<T>(a);
+      }
 #pragma unroll
       for (int o = 1; o < GR; o <<= 1)
 #pragma unroll
         for (int k = 0; k < 16; ++k)
           rmax[k] = fmaxf(rmax[k], __shfl_xor_sync(0xFFFFFFFFu, rmax[k], o));
     }
-    uint32_t cm[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-    for (int k = 0; k < 16; ++k) chunk_colmax<T>(d[k], cm);
     float cmax[CPT];
     if (sizeof(T) == 2) {
 #pragma unroll
@@ -364,20 +365,33 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
     }
 
     // ---- scales --------------------------------------------------------------
-    float rf[16], cf[CPT];
-    uint32_t rbyte[16], cbyte[CPT];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) rbyte[k] = block_scale<T, MX>(rmax[k], ts, rtab, e8m0_mode, rf[k]);
-#pragma unroll
-    for (int j = 0; j < CPT; ++j) cbyte[j] = block_scale<T, MX>(cmax[j], ts, rtab, e8m0_mode, cf[j]);
-    if (valid && do_row && (cc % GR) == 0) {
+    // the GR lanes of a row block share its 16 row maxima: lane gi of the
+    // group computes the scales of rows gi, gi + GR, ... and the factors are
+    // gathered back by shuffles
+    constexpr int RPL = 16 / GR;                      // rows per lane
+    const int gi = cc % GR;
+    float rf[16], cf[CPT], own_f[RPL];
+    uint32_t cbyte[CPT];
+    {
       // rows r0..r0+15 of one block column: in the swizzled layout they are
       // 16 bytes apart (r0 is a multiple of 16), in the linear one cols/BLK
-      const int64_t base = scale_offset(r0, c0 / BLK, cols / BLK, scale_layout);
       const int64_t step = swz ? 16 : cols / BLK;
+      uint8_t *srow = sf_row + scale_offset(r0, c0 / BLK, cols / BLK, scale_layout) + gi * step;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) sf_row[base + k * step] = static_cast<uint8_t>(rbyte[k]);
+      for (int i = 0; i < RPL; ++i) {
+        float m = rmax[i * GR];
+#pragma unroll
+        for (int g = 1; g < GR; ++g)
+          if (g == gi) m = rmax[i * GR + g];
+        const uint32_t b = block_scale<T, MX>(m, ts, rtab, e8m0_mode, own_f[i]);
+        if (valid && do_row) srow[i * GR * step] = static_cast<uint8_t>(b);
+      }
     }
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      rf[k] = GR == 1 ? own_f[k] : __shfl_sync(0xFFFFFFFFu, own_f[k / GR], lane - gi + k % GR);
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) cbyte[j] = block_scale<T, MX>(cmax[j], ts, rtab, e8m0_mode, cf[j]);
     if (valid && do_col && (!MX || (band & 1) == 0)) {
       const int64_t base = scale_offset(c0, r0 / BLK, rows / BLK, scale_layout);
       const int64_t step = swz ? 16 : rows / BLK;
@@ -387,7 +401,8 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
 
     // ---- pass 2: encode, four rows at a time ----------------------------------
     // read the rows from shared memory again rather than keeping all 16 live
-    asm volatile("" ::: "memory");
+    // (the warp barrier keeps the second reads from being hoisted into pass 1)
+    __syncwarp();
     uint32_t colw[CPT][2];
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
@@ -407,7 +422,7 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
           for (int j = 0; j < CPT; ++j) {
             const int e = static_cast<int>(idx % 8) + j;
             const uint32_t wv = words[(e >> 1) & 3];
-            u[i][j] = (e & 1) ? (wv >> 16) : (wv & 0xFFFFu);
+            u[i][j] = (e & 1) ? sr_z_hi(wv) : sr_z_lo(wv);   // z of the 16-bit uniform
           }
         }
       }
@@ -416,19 +431,14 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
         for (int i = 0; i < 4; ++i) {
           const int k = 4 * q4 + i;
           uint32_t wr = 0u;
-          if (SR) {
+          float t[8];
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) wr |= e2m1_sr_bits(__fmul_rn(v[i][j], rf[k]), u[i][j]) << (4 * j);
-          } else {
-            float t[8];
-#pragma unroll
-            for (int j = 0; j < CPT; j += 2) {
-              const float2 p = mul2(make_float2(v[i][j], v[i][j + 1]), make_float2(rf[k], rf[k]));
-              t[j] = p.x;
-              t[j + 1] = p.y;
-            }
-            wr = CPT == 8 ? e2m1x8(t) : e2m1x4(t[0], t[1], t[2 % CPT], t[3 % CPT]);
+          for (int j = 0; j < CPT; j += 2) {
+            const float2 p = mul2(make_float2(v[i][j], v[i][j + 1]), make_float2(rf[k], rf[k]));
+            t[j] = SR ? e2m1_sr_value(p.x, u[i][j]) : p.x;
+            t[j + 1] = SR ? e2m1_sr_value(p.y, u[i][j + 1]) : p.y;
           }
+          wr = CPT == 8 ? e2m1x8(t) : e2m1x4(t[0], t[1], t[2 % CPT], t[3 % CPT]);
           if (valid) {
             uint8_t *qa = q_row + (r0 + k) * (cols / 2) + c0 / 2;
             if (CPT == 8) *reinterpret_cast<uint32_t *>(qa) = wr;
@@ -443,18 +453,13 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             p[i] = mul2(make_float2(v[i][j], v[i][j + 1]), make_float2(cf[j], cf[j + 1]));
-          uint32_t h0, h1;
           if (SR) {
-            h0 = h1 = 0u;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              h0 |= e2m1_sr_bits(p[i].x, u[i][j]) << (4 * i);
-              h1 |= e2m1_sr_bits(p[i].y, u[i][j + 1]) << (4 * i);
-            }
-          } else {
-            h0 = e2m1x4(p[0].x, p[1].x, p[2].x, p[3].x);    // column j, rows 4q4..4q4+3
-            h1 = e2m1x4(p[0].y, p[1].y, p[2].y, p[3].y);    // column j + 1
+            for (int i = 0; i < 4; ++i)
+              p[i] = make_float2(e2m1_sr_value(p[i].x, u[i][j]), e2m1_sr_value(p[i].y, u[i][j + 1]));
           }
+          const uint32_t h0 = e2m1x4(p[0].x, p[1].x, p[2].x, p[3].x);  // column j, rows 4q4..4q4+3
+          const uint32_t h1 = e2m1x4(p[0].y, p[1].y, p[2].y, p[3].y);  // column j + 1
           if (q4 & 1) {
             colw[j][q4 >> 1] |= h0 << 16;
             colw[j + 1][q4 >> 1] |= h1 << 16;

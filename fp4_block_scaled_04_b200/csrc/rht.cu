@@ -23,7 +23,9 @@
 //   * block maxima are in-thread; stochastic rounding needs one Philox call
 //     per token per 8 columns, which two lanes share (each computes half of
 //     the tokens and passes the other lane its 64 bits by shuffle).  The ten
-//     Philox round keys and the 128 signs come in as kernel parameters;
+//     Philox round keys and the 128 signs come in as kernel parameters.  The
+//     values are rounded stochastically in place (e2m1_sr_value) and then
+//     packed by the same round-to-nearest conversion as the RNE path;
 //   * dY^T codes leave as 8 lanes x 8 bytes = 64 contiguous bytes per column.
 #include "common.cuh"
 #include "launch.h"
@@ -60,20 +62,6 @@ __device__ __forceinline__ U32x4 philox_rk(const RhtParams &P, uint32_t c0, uint
     c2 = n2;
   }
   return U32x4{c0, c1, c2, c3};
-}
-
-// Stochastic rounding onto E2M1 by fixed-point grid coordinates (the same
-// rule as round-up iff u < t * 2^16): for |v| in [1, 6] the grid coordinate
-// is G * 2^22 = bits - 0x3F000000, so one carry decides u * 64 < frac; below
-// 1 the grid is uniform and C = ceil(|v| * 2^17) comes from rounding
-// |v| * 2^17 + 2^23 up.  Checked against the oracle by tests/sr_check.c.
-__device__ __forceinline__ uint32_t e2m1_sr_fast(float v, uint32_t u16) {
-  const uint32_t raw = __float_as_uint(v);
-  const uint32_t b = raw & 0x7FFFFFFFu;
-  const uint32_t code_a = min((b - 0x3EC00001u - (u16 << 6)) >> 22, 7u);
-  const float xu = __fmaf_ru(__uint_as_float(b), 131072.0f, 8388608.0f);
-  const uint32_t code_b = (__float_as_uint(xu) - 0x4AFF0001u - u16) >> 16;
-  return (b >= 0x3F800000u ? code_a : code_b) | ((raw >> 28) & 8u);
 }
 
 template <int H>
@@ -314,13 +302,12 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
     if (SR) {
       // element (t, c) draws from the Philox call (t * cols + c) / 8, covering
       // this lane's quad and its neighbour's (lane ^ 8): the even quad computes
-      // tokens 0..7, the odd one 8..15, and each sends the other its half
+      // tokens 0..7, the odd one 8..15, and each sends the other its half.
+      // The values are rounded in place; the RNE packing below encodes them.
       const int half = cq & 1;
       const uint64_t row0 = (static_cast<uint64_t>(t0) * static_cast<uint64_t>(cols) +
                              static_cast<uint64_t>(c0 - 4 * half)) / 8;
       const uint64_t rstep = static_cast<uint64_t>(cols) / 8;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) w[j][0] = w[j][1] = 0u;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint64_t gidx = row0 + static_cast<uint64_t>(i + 8 * half) * rstep;
@@ -333,18 +320,17 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
         // this lane computed token i + 8 half, the partner token i + 8 (1 - half)
         const uint32_t ti0 = half ? got0 : keep0, ti1 = half ? got1 : keep1;
         const uint32_t tj0 = half ? keep0 : got0, tj1 = half ? keep1 : got1;
-        const float vi[4] = {lo[i].x, lo[i].y, hi[i].x, hi[i].y};
-        const float vj[4] = {lo[i + 8].x, lo[i + 8].y, hi[i + 8].x, hi[i + 8].y};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t wi = (j >> 1) ? ti1 : ti0, wj = (j >> 1) ? tj1 : tj0;
-          const uint32_t ui = (j & 1) ? (wi >> 16) : (wi & 0xFFFFu);
-          const uint32_t uj = (j & 1) ? (wj >> 16) : (wj & 0xFFFFu);
-          w[j][0] += e2m1_sr_fast(vi[j], ui) << (4 * i);
-          w[j][1] += e2m1_sr_fast(vj[j], uj) << (4 * i);
-        }
+        lo[i].x = e2m1_sr_value(lo[i].x, sr_z_lo(ti0));
+        lo[i].y = e2m1_sr_value(lo[i].y, sr_z_hi(ti0));
+        hi[i].x = e2m1_sr_value(hi[i].x, sr_z_lo(ti1));
+        hi[i].y = e2m1_sr_value(hi[i].y, sr_z_hi(ti1));
+        lo[i + 8].x = e2m1_sr_value(lo[i + 8].x, sr_z_lo(tj0));
+        lo[i + 8].y = e2m1_sr_value(lo[i + 8].y, sr_z_hi(tj0));
+        hi[i + 8].x = e2m1_sr_value(hi[i + 8].x, sr_z_lo(tj1));
+        hi[i + 8].y = e2m1_sr_value(hi[i + 8].y, sr_z_hi(tj1));
       }
-    } else {
+    }
+    {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float a[8], b[8], c[8], d[8];

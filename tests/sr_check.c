@@ -1,10 +1,21 @@
-/* Check of the stochastic-rounding method the CUDA kernels use, against the
- * oracle's definition (linked from oracle/fp4q_oracle.c): for |v| in [1, 6]
- * the E2M1 grid coordinate is G * 2^22 = bits(|v|) - 0x3F000000 and the code
- * is (bits - 0x3EC00001 - (u << 6)) >> 22 (one carry decides "u * 64 < frac");
+/* Check of the stochastic-rounding methods the CUDA kernels use, against the
+ * oracle's definition (linked from oracle/fp4q_oracle.c).
+ *
+ * Method 0 (codes): for |v| in [1, 6] the E2M1 grid coordinate is
+ * G * 2^22 = bits(|v|) - 0x3F000000 and the code is
+ * (bits - 0x3EC00001 - (u << 6)) >> 22 (one carry decides "u * 64 < frac");
  * below 1 the grid is uniform, C = ceil(|v| * 2^17) is read from
  * RU(|v| * 2^17 + 2^23) and the code is (C + 0xFFFF - u) >> 16.
- * Usage: sr_check <n_random> -- prints the number of mismatches. */
+ *
+ * Method 1 (values): on [1, 8) E2M1 is a float with one mantissa bit, so the
+ * stochastically rounded magnitude is (bits(w) + 0x3FFFFF - 64 u) with the
+ * low 22 bits cleared; below 1 the spacing 0.5 is that of [1, 2), so
+ * w = RU(|v| + 1) is rounded the same way and 1 subtracted again (rounding
+ * the sum up keeps "64 u < frac" exact, as frac is compared with an integer).
+ * The sign is copied and the value converted by round-to-nearest-even with
+ * saturation (the hardware conversion; the oracle's RNE stands in for it
+ * here), which also maps 8 to 6.
+ * Usage: sr_check <n_random> [method] -- prints the number of mismatches. */
 #include <fenv.h>
 #include <math.h>
 #include <stdint.h>
@@ -30,11 +41,29 @@ static uint32_t method(float v, uint32_t u16) {
   return code | ((raw >> 28) & 8u);
 }
 
+uint8_t orc_e2m1_rne(float v);
+
+static uint32_t method1(float v, uint32_t u16) {
+  uint32_t raw = bits(v);
+  float av = fabsf(v);
+  float a = av < 1.0f ? 1.0f : 0.0f;
+  fesetround(FE_UPWARD);
+  volatile float w = av + a;
+  fesetround(FE_TONEAREST);
+  uint32_t R = (bits(w) + (0x3FFFFFu - (u16 << 6))) & 0xFFC00000u;
+  volatile float r = flt(R) - a;
+  return orc_e2m1_rne(flt(bits(r) | (raw & 0x80000000u)));
+}
+
+static int which = 0;
+static uint32_t pick(float v, uint32_t u16) { return which ? method1(v, u16) : method(v, u16); }
+
 static uint64_t s = 0x9E3779B97F4A7C15ull;
 static uint64_t rnd(void) { s ^= s << 13; s ^= s >> 7; s ^= s << 17; return s; }
 
 int main(int argc, char **argv) {
   long n = atol(argv[1]);
+  if (argc > 2) which = atoi(argv[2]);
   long bad = 0;
   /* every E2M1 boundary region: values near grid points and midpoints,
      with all 2^16 u for each, then random (v, u) pairs */
@@ -46,8 +75,8 @@ int main(int argc, char **argv) {
       if ((int64_t)b + d < 0) continue;
       float v = flt(b + d);
       for (uint32_t u = 0; u < 65536; ++u) {
-        if (method(v, u) != orc_e2m1_sr(v, u)) ++bad;
-        if (method(-v, u) != orc_e2m1_sr(-v, u)) ++bad;
+        if (pick(v, u) != orc_e2m1_sr(v, u)) ++bad;
+        if (pick(-v, u) != orc_e2m1_sr(-v, u)) ++bad;
       }
     }
   for (long i = 0; i < n; ++i) {
@@ -56,7 +85,7 @@ int main(int argc, char **argv) {
     float v = flt((uint32_t)(0x30800000u + (r % (0x41800000u - 0x30800000u))));
     if (r >> 63) v = -v;
     uint32_t u = (uint32_t)(r >> 40) & 0xFFFFu;
-    if (method(v, u) != orc_e2m1_sr(v, u)) ++bad;
+    if (pick(v, u) != orc_e2m1_sr(v, u)) ++bad;
   }
   printf("%ld\n", bad);
   return 0;

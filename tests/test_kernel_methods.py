@@ -65,14 +65,17 @@ def test_rint_ties_go_to_even():
     assert np.all(np.rint(t) % 2 == 0)
 
 
-def test_stochastic_rounding_fixed_point_method(tmp_path):
-    """The kernels' integer/fixed-point stochastic rounding equals the
-    oracle's rule (round the magnitude up iff u < t * 2^16) on every u for
-    values around each E2M1 grid point and midpoint, and on 4M random pairs."""
+@pytest.mark.parametrize("method", [0, 1])
+def test_stochastic_rounding_fixed_point_method(tmp_path, method):
+    """The kernels' stochastic rounding methods (0: integer codes, 1: rounded
+    values then the round-to-nearest conversion) equal the oracle's rule
+    (round the magnitude up iff u < t * 2^16) on every u for values around
+    each E2M1 grid point and midpoint, and on 4M random pairs."""
     exe = str(tmp_path / "sr_check")
     subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-frounding-math",
                            os.path.join(HERE, "sr_check.c"),
                            os.path.join(os.path.dirname(HERE), "oracle", "fp4q_oracle.c"),
                            "-o", exe, "-lm"])
-    out = subprocess.run([exe, "4000000"], capture_output=True, text=True, check=True)
+    out = subprocess.run([exe, "4000000", str(method)], capture_output=True, text=True,
+                         check=True)
     assert int(out.stdout.strip()) == 0
