@@ -357,4 +357,39 @@ __device__ __forceinline__ U32x4 philox(const PhiloxKey &K, uint32_t c0, uint32_
   return U32x4{c0, c1, c2, c3};
 }
 
+// ---------------------------------------------------------------------------
+// cp.async staging (16-byte global -> shared copies, grouped per thread)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Coordinates (tile row tt, tile column tc) of a linear tile index over a
+// grid of tiles_c tile columns, stepped by a fixed number of tiles without
+// dividing.
+struct TileCursor {
+  int64_t tile, tt, tc;
+  __device__ __forceinline__ void init(int64_t t, int64_t tiles_c) {
+    tile = t;
+    tt = t / tiles_c;
+    tc = t - tt * tiles_c;
+  }
+  __device__ __forceinline__ void advance(int64_t step, int64_t dtt, int64_t dtc,
+                                          int64_t tiles_c) {
+    tile += step;
+    tt += dtt;
+    tc += dtc;
+    if (tc >= tiles_c) {
+      tc -= tiles_c;
+      ++tt;
+    }
+  }
+};
+
 }  // namespace fp4q

@@ -130,12 +130,6 @@ __device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float
   wb[1] = int_b ? ib[1] : fpb[1];
 }
 
-__device__ __forceinline__ void async_copy16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Position of a lane's pair: row r and first block cb = 2 * pc, advanced by
 // a fixed stride of pairs.
@@ -198,7 +192,7 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     const uint32_t dst = my_s + static_cast<uint32_t>(st * STAGE);
 #pragma unroll
     for (int i = 0; i < PPL; ++i)
-      if (i < n) async_copy16(dst + static_cast<uint32_t>((i ^ swz) * 16), src + 16 * i);
+      if (i < n) cp_async16(dst + static_cast<uint32_t>((i ^ swz) * 16), src + 16 * i);
   };
 
   Cursor ci, cc;
@@ -207,14 +201,14 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
 #pragma unroll
   for (int s = 0; s < kStages - 1; ++s) {
     issue(ci, s);
-    async_commit();
+    cp_async_commit();
     ci.advance(stride, dr, dpc, ppr);
   }
   for (int st = 0; cc.p < npairs; st = (st + 1 == kStages ? 0 : st + 1)) {
     issue(ci, st == 0 ? kStages - 1 : st - 1);
-    async_commit();
+    cp_async_commit();
     ci.advance(stride, dr, dpc, ppr);
-    async_wait<kStages - 1>();
+    cp_async_wait<kStages - 1>();
 
     const int64_t r = cc.r, cb = 2 * cc.pc;
     const bool has_b = cb + 1 < bpr;
@@ -299,7 +293,7 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     }
     cc.advance(stride, dr, dpc, ppr);
   }
-  async_wait<0>();
+  cp_async_wait<0>();
 }
 
 template <typename T, bool SWZ>

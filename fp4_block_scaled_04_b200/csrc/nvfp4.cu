@@ -250,12 +250,6 @@ __device__ __forceinline__ uint32_t block_scale(float m, const TensorScale &ts, 
   return code;
 }
 
-__device__ __forceinline__ void rc_copy16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void rc_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void rc_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void rc_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 constexpr int kRCTileBytes = 64 * 128;            // one warp tile: 64 rows x 128 bytes
 constexpr int kRCSmem = (kRCThreads / 32) * 2 * kRCTileBytes;
@@ -291,8 +285,8 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
                            static_cast<uint32_t>(warp * 2 * kRCTileBytes);
   const uint4 *stage_g = reinterpret_cast<const uint4 *>(rc_smem + warp * 2 * kRCTileBytes);
   // lane L copies the 16-byte pieces L + 32 i: row (L + 32 i) / 8, chunk L % 8
-  auto issue = [&](int64_t t, int st) {
-    const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+  auto issue = [&](const TileCursor &t, int st) {
+    const int64_t tr = t.tt, tc = t.tc;
     const int64_t col = tc * G::WC + cc * CPT;
     if (col >= cols) return;
     const uint32_t dst = stage_s + static_cast<uint32_t>(st * kRCTileBytes + cc * 16);
@@ -300,19 +294,24 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
     for (int i = 0; i < 16; ++i) {
       const int row = (lane >> 3) + 4 * i;
       if (tr * G::WR + row < rows)
-        rc_copy16(dst + static_cast<uint32_t>(row * 128), x + (tr * G::WR + row) * ld + col);
+        cp_async16(dst + static_cast<uint32_t>(row * 128), x + (tr * G::WR + row) * ld + col);
     }
   };
-  int64_t tile = static_cast<int64_t>(blockIdx.x) * (kRCThreads / 32) + warp;
-  if (tile < ntiles) issue(tile, 0);
-  rc_commit();
-  for (int st = 0; tile < ntiles; tile += nwarps, st ^= 1) {
+  const int64_t dtr = nwarps / tiles_c, dtc = nwarps - dtr * tiles_c;
+  TileCursor cur, nxt;                                    // this tile, the one being copied
+  cur.init(static_cast<int64_t>(blockIdx.x) * (kRCThreads / 32) + warp, tiles_c);
+  nxt = cur;
+  if (nxt.tile < ntiles) issue(nxt, 0);
+  cp_async_commit();
+  nxt.advance(nwarps, dtr, dtc, tiles_c);
+  for (int st = 0; cur.tile < ntiles; cur.advance(nwarps, dtr, dtc, tiles_c), st ^= 1) {
     __syncwarp();   // every lane is done with stage st ^ 1 before it is refilled
-    if (tile + nwarps < ntiles) issue(tile + nwarps, st ^ 1);
-    rc_commit();
-    rc_wait_1();
+    if (nxt.tile < ntiles) issue(nxt, st ^ 1);
+    cp_async_commit();
+    nxt.advance(nwarps, dtr, dtc, tiles_c);
+    cp_async_wait<1>();
     __syncwarp();
-    const int64_t tr = tile / tiles_c, tc = tile - tr * tiles_c;
+    const int64_t tr = cur.tt, tc = cur.tc;
     const int64_t r0 = tr * G::WR + band * 16, c0 = tc * G::WC + cc * CPT;
     const bool valid = r0 < rows && c0 < cols;
     // row k of this thread's 16: tb[8 * k] (rows outside the matrix are never
@@ -477,7 +476,7 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
             make_uint2(colw[j][0], colw[j][1]);
     }
   }
-  rc_wait_0();
+  cp_async_wait<0>();
 }
 
 int grid_cap(const void *kernel, int threads, const Launch &L) {

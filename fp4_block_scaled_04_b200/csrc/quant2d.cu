@@ -5,11 +5,13 @@
 // square 16x16 tiles give both the same scales, so W and W^T codes come out
 // of one pass.
 //
-// Register tiles, no shared memory: a thread owns 16 rows x one 16-byte
-// column chunk (4 FP32 or 8 BF16 columns); a 16x16 tile spans 4 (FP32) or 2
-// (BF16) lanes, whose partial maxima meet by shuffle.  A warp owns 64 rows x
-// 8 chunks (lane = chunk + 8 * row band), so a warp instruction writes W^T
-// codes as whole 32-byte sectors (4 bands x 8 bytes of one column).
+// Register tiles fed by a two-stage cp.async buffer: a warp owns 64 rows x
+// 128 bytes (8 16-byte chunks of 4 FP32 or 8 BF16 columns) and copies the
+// next such tile into shared memory while it encodes this one.  A thread
+// owns 16 rows x one chunk; a 16x16 tile spans 4 (FP32) or 2 (BF16) lanes,
+// whose partial maxima meet by shuffle (lane = chunk + 8 * row band), so a
+// warp instruction writes W^T codes as whole 32-byte sectors (4 bands x 8
+// bytes of one column).
 #include "common.cuh"
 #include "launch.h"
 
@@ -17,6 +19,8 @@ namespace fp4q {
 namespace {
 
 constexpr int kThreads = 128;
+constexpr int kTileBytes = 64 * 128;               // one warp tile: 64 rows x 128 bytes
+constexpr int kSmem = (kThreads / 32) * 2 * kTileBytes;
 
 template <typename T>
 __device__ __forceinline__ void unpack4or8(uint4 u, float (&v)[16 / sizeof(T)]) {
@@ -46,21 +50,50 @@ quant2d_kernel(const T *__restrict__ w, int64_t rows, int64_t cols, int64_t ld,
   if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
   __syncthreads();
 
-  const int lane = threadIdx.x & 31, cc = lane & 7, band = lane >> 3;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int lane = threadIdx.x & 31, cc = lane & 7, band = lane >> 3, warp = threadIdx.x >> 5;
   const int li = cc % LPT;                  // lane index within the tile
   const int64_t tiles_c = (cols + WC - 1) / WC;
   const int64_t ntiles = tiles_c * ((rows + 63) / 64);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
-  for (int64_t tile = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
-       tile < ntiles; tile += nwarps) {
-    const int64_t tr = tile / tiles_c, tcol = tile - tr * tiles_c;
-    const int64_t r0 = tr * 64 + band * 16, c0 = tcol * WC + cc * CPT;
+  const int64_t dtr = nwarps / tiles_c, dtc = nwarps - dtr * tiles_c;
+  const uint32_t stage_s = static_cast<uint32_t>(__cvta_generic_to_shared(smem)) +
+                           static_cast<uint32_t>(warp * 2 * kTileBytes);
+  const uint4 *stage_g = reinterpret_cast<const uint4 *>(smem + warp * 2 * kTileBytes);
+  // lane L copies the 16-byte pieces L + 32 i: row (L + 32 i) / 8, chunk L % 8;
+  // each warp copy instruction moves four whole 128-byte row segments
+  auto issue = [&](const TileCursor &t, int st) {
+    const int64_t col = t.tc * WC + cc * CPT;
+    if (col >= cols) return;
+    const uint32_t dst = stage_s + static_cast<uint32_t>(st * kTileBytes + cc * 16);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int row = (lane >> 3) + 4 * i;
+      if (t.tt * 64 + row < rows)
+        cp_async16(dst + static_cast<uint32_t>(row * 128), w + (t.tt * 64 + row) * ld + col);
+    }
+  };
+  TileCursor cur, nxt;                                    // this tile, the one being copied
+  cur.init(static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + warp, tiles_c);
+  nxt = cur;
+  if (nxt.tile < ntiles) issue(nxt, 0);
+  cp_async_commit();
+  nxt.advance(nwarps, dtr, dtc, tiles_c);
+  for (int st = 0; cur.tile < ntiles; cur.advance(nwarps, dtr, dtc, tiles_c), st ^= 1) {
+    __syncwarp();   // every lane is done with stage st ^ 1 before it is refilled
+    if (nxt.tile < ntiles) issue(nxt, st ^ 1);
+    cp_async_commit();
+    nxt.advance(nwarps, dtr, dtc, tiles_c);
+    cp_async_wait<1>();
+    __syncwarp();
+    const int64_t r0 = cur.tt * 64 + band * 16, c0 = cur.tc * WC + cc * CPT;
     const bool valid = r0 < rows && c0 < cols;   // the whole 16x16 tile shares validity
+    // rows outside the matrix are never copied; their lanes' values only meet
+    // other outside lanes and are not stored
+    const uint4 *tb = stage_g + st * (kTileBytes / 16) + band * 16 * 8 + cc;
     uint4 d[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k)
-      d[k] = valid ? __ldg(reinterpret_cast<const uint4 *>(w + (r0 + k) * ld + c0))
-                   : make_uint4(0u, 0u, 0u, 0u);
+    for (int k = 0; k < 16; ++k) d[k] = tb[8 * k];
     float m;
     if (sizeof(T) == 2) {
       uint32_t mm = 0u;
@@ -138,6 +171,7 @@ quant2d_kernel(const T *__restrict__ w, int64_t rows, int64_t cols, int64_t ld,
         sf_wt_1x16[scale_offset(c0 + j, gr / 16, rows / 16, scale_layout)] = sb;
     }
   }
+  cp_async_wait<0>();
 }
 
 }  // namespace
@@ -148,23 +182,31 @@ cudaError_t launch_2d(const void *w, int dtype, int64_t rows, int64_t cols, int6
                       int scale_layout, const Launch &L) {
   const int cpt = dtype == FP4Q_BF16 ? 8 : 4;
   const int64_t ntiles = ((cols + 8 * cpt - 1) / (8 * cpt)) * ((rows + 63) / 64);
-  const void *kern = dtype == FP4Q_BF16 ? reinterpret_cast<const void *>(quant2d_kernel<__nv_bfloat16>)
-                                        : reinterpret_cast<const void *>(quant2d_kernel<float>);
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess ||
-      per_sm < 1) {
-    cudaGetLastError();
-    per_sm = 1;
+  const bool bf = dtype == FP4Q_BF16;
+  const void *kern = bf ? reinterpret_cast<const void *>(quant2d_kernel<__nv_bfloat16>)
+                        : reinterpret_cast<const void *>(quant2d_kernel<float>);
+  static int per_sm_t[2] = {0, 0};
+  int &per_sm = per_sm_t[bf ? 1 : 0];
+  if (per_sm == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
+        cudaSuccess)
+      return cudaGetLastError();
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, kSmem) !=
+            cudaSuccess ||
+        per_sm < 1) {
+      cudaGetLastError();
+      per_sm = 1;
+    }
   }
   const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
   const int64_t want = (ntiles + kThreads / 32 - 1) / (kThreads / 32);
   const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
   if (dtype == FP4Q_BF16)
-    quant2d_kernel<__nv_bfloat16><<<grid, kThreads, 0, L.stream>>>(
+    quant2d_kernel<__nv_bfloat16><<<grid, kThreads, kSmem, L.stream>>>(
         static_cast<const __nv_bfloat16 *>(w), rows, cols, ld, amax, s_dec_out, q_w, q_wt,
         sf_tiles, sf_w_1x16, sf_wt_1x16, scale_layout);
   else
-    quant2d_kernel<float><<<grid, kThreads, 0, L.stream>>>(
+    quant2d_kernel<float><<<grid, kThreads, kSmem, L.stream>>>(
         static_cast<const float *>(w), rows, cols, ld, amax, s_dec_out, q_w, q_wt, sf_tiles,
         sf_w_1x16, sf_wt_1x16, scale_layout);
   return cudaGetLastError();

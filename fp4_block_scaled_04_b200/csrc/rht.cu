@@ -96,29 +96,9 @@ __device__ __forceinline__ void xstage(float2 (&lo)[16], float2 (&hi)[16]) {
       }
 }
 
-__device__ __forceinline__ void async_copy16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-struct TileCoord {
-  int64_t t0, c0;
-  bool valid;
-  __device__ __forceinline__ TileCoord(int64_t tile, int64_t tiles_c, int g, int cq,
-                                       int64_t tokens, int64_t cols) {
-    const int64_t tt = tile / tiles_c, tc = tile - tt * tiles_c;
-    t0 = tt * 128 + 16 * g;
-    c0 = tc * 16 + 4 * cq;
-    // a column quad is all-in or all-out (cols % 8 == 0); a 16-token group
-    // likewise (tokens % 16 == 0); for n = 128 all groups of a tile are in
-    valid = c0 < cols && t0 < tokens;
-  }
-};
 
 template <typename T, int N, bool SR, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, N == 16 ? 4 : 3)
 rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
            const RhtParams P, const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
            unsigned *__restrict__ amax_out, uint8_t *__restrict__ q_t,
@@ -155,7 +135,10 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   const int64_t tiles_c = (cols + 15) / 16;
   const int64_t ntiles = tiles_c * ((tokens + 127) / 128);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
-  int64_t tile = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+  const int64_t dtt = nwarps / tiles_c, dtc = nwarps - dtt * tiles_c;
+  TileCursor cur, nxt;                                    // this tile, the one being copied
+  cur.init(static_cast<int64_t>(blockIdx.x) * kWarps + warp, tiles_c);
+  nxt = cur;
 
   // the copy of a tile is spread differently from the reads: lane L moves the
   // 16-byte pieces L + 32 i (token (L + 32 i) / PPT, piece (L + 32 i) % PPT,
@@ -164,9 +147,8 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   // the data to the lanes that read it (PPT = pieces per token row)
   constexpr int PPT = sizeof(T);                          // 16-byte pieces per token row
   constexpr int UPP = 16 / UB;                            // units per piece
-  auto issue = [&](int64_t t, int st) {
-    const int64_t tt = t / tiles_c, tc = t - tt * tiles_c;
-    const int64_t tbase = tt * 128, cbase = tc * 16;
+  auto issue = [&](const TileCursor &t, int st) {
+    const int64_t tbase = t.tt * 128, cbase = t.tc * 16;
     const uint32_t dst0 = in_s + static_cast<uint32_t>(st * kUnits * UB);
 #pragma unroll
     for (int i = 0; i < 4 * PPT; ++i) {
@@ -174,23 +156,26 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
       const int tok = piece / PPT, pc = piece % PPT;
       const int64_t col = cbase + pc * (16 / static_cast<int>(sizeof(T)));
       if (tbase + tok < tokens && col < cols)
-        async_copy16(dst0 + static_cast<uint32_t>(unit_of(tok, pc * UPP) * UB),
+        cp_async16(dst0 + static_cast<uint32_t>(unit_of(tok, pc * UPP) * UB),
                      dy + (tbase + tok) * ld + col);
     }
   };
 
   uint32_t amax_bits = 0u;
-  if (tile < ntiles) issue(tile, 0);
-  async_commit();
-  for (int st = 0; tile < ntiles; tile += nwarps, st ^= 1) {
+  if (nxt.tile < ntiles) issue(nxt, 0);
+  cp_async_commit();
+  nxt.advance(nwarps, dtt, dtc, tiles_c);
+  for (int st = 0; cur.tile < ntiles; cur.advance(nwarps, dtt, dtc, tiles_c), st ^= 1) {
     __syncwarp();   // every lane is done with stage st ^ 1 (last tile) before it is refilled
-    if (tile + nwarps < ntiles) issue(tile + nwarps, st ^ 1);
-    async_commit();
-    async_wait_1();
+    if (nxt.tile < ntiles) issue(nxt, st ^ 1);
+    cp_async_commit();
+    nxt.advance(nwarps, dtt, dtc, tiles_c);
+    cp_async_wait<1>();
     __syncwarp();
-    const TileCoord tl(tile, tiles_c, g, cq, tokens, cols);
-    const int64_t t0 = tl.t0, c0 = tl.c0;
-    const bool valid = tl.valid;
+    // a column quad is all-in or all-out (cols % 8 == 0); a 16-token group
+    // likewise (tokens % 16 == 0); for n = 128 all groups of a tile are in
+    const int64_t t0 = cur.tt * 128 + 16 * g, c0 = cur.tc * 16 + 4 * cq;
+    const bool valid = c0 < cols && t0 < tokens;
 
     // ---- sign flip and stages h = 1, 2, 4, 8 ----------------------------------
     float2 lo[16], hi[16];     // columns (c0, c0+1) and (c0+2, c0+3) per token
@@ -346,16 +331,19 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
       }
     }
     if (valid) {
+      // columns c0..c0+3 (c0 % 4 == 0): code rows tokens/2 bytes apart, scale
+      // rows 16 bytes apart in the swizzled layout, tokens/16 in the linear one
+      uint8_t *qp = q_t + c0 * (tokens / 2) + t0 / 2;
+      uint8_t *sp = sf_t + scale_offset(c0, t0 / 16, tokens / 16, scale_layout);
+      const int64_t sstep = scale_layout == FP4Q_SCALE_SWIZZLED_128x4 ? 16 : tokens / 16;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        *reinterpret_cast<uint2 *>(q_t + (c0 + j) * (tokens / 2) + t0 / 2) =
-            make_uint2(w[j][0], w[j][1]);
-        sf_t[scale_offset(c0 + j, t0 / 16, tokens / 16, scale_layout)] =
-            static_cast<uint8_t>(sbyte[j]);
+        *reinterpret_cast<uint2 *>(qp + j * (tokens / 2)) = make_uint2(w[j][0], w[j][1]);
+        sp[j * sstep] = static_cast<uint8_t>(sbyte[j]);
       }
     }
   }
-  async_wait_0();
+  cp_async_wait<0>();
   if (AMAX_ONLY) {
     amax_bits = __reduce_max_sync(0xFFFFFFFFu, amax_bits);
     if (lane == 0) atomicMax(amax_out, amax_bits);
