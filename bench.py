@@ -70,8 +70,51 @@ class Job:
         self.bytes = bytes_moved    # algorithmic bytes (input once + outputs)
         self.launches = launches    # our kernels per call
         self.run = run              # device call (inputs resident)
-        self.e2e = e2e              # host-buffer call: returns (h2d_bytes, d2h_bytes)
+        self.e2e = e2e              # E2E: host inputs -> public API -> host outputs
         self.oracle = oracle        # CPU oracle on a row fraction: returns bytes done
+
+
+class E2E:
+    """One job end to end: pinned host inputs are copied into the job's own
+    device buffers, the public API call runs on them (computing the tensor
+    amax itself), and every output is copied back to pinned host memory.
+    The three steps run on three streams so that the copies of neighbouring
+    jobs overlap (host-to-device and device-to-host run at the same time);
+    events order each job's steps and keep a buffer from being refilled
+    while an earlier step still uses it."""
+
+    def __init__(self, host_in, dev_in, compute, dev_out):
+        import torch
+        self.host_in, self.dev_in, self.compute_fn = host_in, dev_in, compute
+        self.dev_out = dev_out
+        self.host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                         for k, v in dev_out.items()}
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in host_in)
+        self.d2h_bytes = sum(t.numel() * t.element_size() for t in dev_out.values())
+        self.ev_in = torch.cuda.Event()      # inputs on the device
+        self.ev_comp = torch.cuda.Event()    # outputs written, inputs free
+        self.ev_out = torch.cuda.Event()     # outputs copied out
+
+    def step(self, s_in, s_comp, s_out, first):
+        import torch
+        with torch.cuda.stream(s_in):
+            if not first:
+                s_in.wait_event(self.ev_comp)          # the last call has read the inputs
+            for h, d in zip(self.host_in, self.dev_in):
+                d.copy_(h, non_blocking=True)
+            self.ev_in.record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(self.ev_in)
+            if not first:
+                s_comp.wait_event(self.ev_out)         # the last outputs are out
+            self.compute_fn()
+            self.ev_comp.record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(self.ev_comp)
+            for k, v in self.dev_out.items():
+                self.host_out[k].copy_(v, non_blocking=True)
+            self.ev_out.record(s_out)
+        return self.h2d_bytes, self.d2h_bytes
 
 
 def build_jobs(device, fq, inputs):
@@ -84,12 +127,8 @@ def build_jobs(device, fq, inputs):
     def pinned_like(t):
         return torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
 
-    def to_host(outs, hosts):
-        n = 0
-        for k, v in outs.items():
-            hosts[k].copy_(v, non_blocking=True)
-            n += v.numel() * v.element_size()
-        return n
+    def dev_like(t):
+        return torch.empty(t.shape, dtype=t.dtype, device=device)
 
     # ---- activation: NVFP4 row + col, MXFP4 row + col -------------------
     xa_cpu = inputs["activation"]
@@ -101,18 +140,13 @@ def build_jobs(device, fq, inputs):
     nb_nv = R * C * 2 + 2 * (R * C // 2) + 2 * (R * C // 16) + 4
     nb_mx = R * C * 2 + 2 * (R * C // 2) + 2 * (R * C // 32)
     xa_h = pinned_like(xa_cpu).copy_(xa_cpu)
-    hn = {k: pinned_like(v.cpu()) for k, v in out_nv.items()}
-    hm = {k: pinned_like(v.cpu()) for k, v in out_mx.items()}
-
-    def e2e_nv():
-        x = xa_h.to(device, non_blocking=True)
-        o = fq.fp4q_quantize_nvfp4(x, layouts=3, scale_layout=SW, out=out_nv)
-        return xa_h.numel() * 2, to_host(o, hn)
-
-    def e2e_mx():
-        x = xa_h.to(device, non_blocking=True)
-        o = fq.fp4q_quantize_mxfp4(x, layouts=3, scale_layout=SW, out=out_mx)
-        return xa_h.numel() * 2, to_host(o, hm)
+    xe_nv, xe_mx = dev_like(xa), dev_like(xa)
+    oe_nv = {k: dev_like(v) for k, v in out_nv.items()}
+    oe_mx = {k: dev_like(v) for k, v in out_mx.items()}
+    e2e_nv = E2E([xa_h], [xe_nv], lambda: fq.fp4q_quantize_nvfp4(
+        xe_nv, layouts=3, scale_layout=SW, out=oe_nv), oe_nv)
+    e2e_mx = E2E([xa_h], [xe_mx], lambda: fq.fp4q_quantize_mxfp4(
+        xe_mx, layouts=3, scale_layout=SW, out=oe_mx), oe_mx)
 
     jobs.append(Job("activation 8192x4096 bf16 nvfp4 row+col", "nvfp4.cu", nb_nv, 1,
                     lambda: fq.fp4q_quantize_nvfp4(xa, layouts=3, amax=amax_a, scale_layout=SW,
@@ -129,12 +163,9 @@ def build_jobs(device, fq, inputs):
     R, C = w.shape
     nb_w = R * C * 4 + 2 * (R * C // 2) + (R // 16) * (C // 16) + 4
     w_h = pinned_like(w_cpu).copy_(w_cpu)
-    hw = {k: pinned_like(v.cpu()) for k, v in out_w.items()}
-
-    def e2e_w():
-        x = w_h.to(device, non_blocking=True)
-        o = fq.fp4q_quantize_2d(x, out=out_w)
-        return w_h.numel() * 4, to_host(o, hw)
+    we = dev_like(w)
+    oe_w = {k: dev_like(v) for k, v in out_w.items()}
+    e2e_w = E2E([w_h], [we], lambda: fq.fp4q_quantize_2d(we, out=oe_w), oe_w)
 
     jobs.append(Job("weight 14336x4096 fp32 2d16x16 w+wt", "quant2d.cu", nb_w, 1,
                     lambda: fq.fp4q_quantize_2d(w, amax=amax_w, out=out_w), e2e_w))
@@ -150,12 +181,10 @@ def build_jobs(device, fq, inputs):
         for rnd, rname in ((fq.SR, "sr"), (fq.RNE, "rne")):
             out_g = fq.fp4q_quantize_rht_sr(g, n, round=rnd, seed=0, amax_rht=amax_g,
                                             scale_layout=SW)
-            hg = {k: pinned_like(v.cpu()) for k, v in out_g.items()}
-
-            def e2e_g(n=n, rnd=rnd, out_g=out_g, hg=hg):
-                x = g_h.to(device, non_blocking=True)
-                o = fq.fp4q_quantize_rht_sr(x, n, round=rnd, seed=0, scale_layout=SW, out=out_g)
-                return g_h.numel() * 2, to_host(o, hg)
+            ge = dev_like(g)
+            oe_g = {k: dev_like(v) for k, v in out_g.items()}
+            e2e_g = E2E([g_h], [ge], lambda n=n, rnd=rnd, ge=ge, oe_g=oe_g: fq.fp4q_quantize_rht_sr(
+                ge, n, round=rnd, seed=0, scale_layout=SW, out=oe_g), oe_g)
 
             jobs.append(Job(f"gradient 8192x5120 bf16 rht{n}+{rname}", "rht.cu", nb_g, 1,
                             lambda n=n, rnd=rnd, a=amax_g, o=out_g: fq.fp4q_quantize_rht_sr(
@@ -176,22 +205,13 @@ def build_jobs(device, fq, inputs):
     y5 = torch.empty((R, C), dtype=torch.bfloat16, device=device)
     nb_d5 = R * C // 2 + R * C // 16 + 4 + R * C * 2
     x5_h = pinned_like(x5_cpu).copy_(x5_cpu)
-    h5 = {k: pinned_like(v.cpu()) for k, v in out5.items()}
+    x5e = dev_like(x5)
+    oe5 = {k: dev_like(v) for k, v in out5.items()}
+    e2e_q5 = E2E([x5_h], [x5e], lambda: fq.fp4q_quantize_if4(x5e, scale_layout=SW, out=oe5), oe5)
     q5_h, sf5_h, s5_h = q5.cpu().pin_memory(), sf5.cpu().pin_memory(), s5.cpu().pin_memory()
-    y5_h = torch.empty((R, C), dtype=torch.bfloat16, pin_memory=True)
-
-    def e2e_q5():
-        x = x5_h.to(device, non_blocking=True)
-        o = fq.fp4q_quantize_if4(x, scale_layout=SW, out=out5)
-        return x5_h.numel() * 2, to_host(o, h5)
-
-    def e2e_d5():
-        q = q5_h.to(device, non_blocking=True)
-        sf = sf5_h.to(device, non_blocking=True)
-        s = s5_h.to(device, non_blocking=True)
-        fq.fp4q_dequantize(fq.FMT_IF4, q, sf, R, C, tensor_scale=s, scale_layout=SW, out=y5)
-        y5_h.copy_(y5, non_blocking=True)
-        return q5_h.numel() + sf5_h.numel() + 4, y5_h.numel() * 2
+    q5e, sf5e, s5e, y5e = dev_like(q5), dev_like(sf5), dev_like(s5), dev_like(y5)
+    e2e_d5 = E2E([q5_h, sf5_h, s5_h], [q5e, sf5e, s5e], lambda: fq.fp4q_dequantize(
+        fq.FMT_IF4, q5e, sf5e, R, C, tensor_scale=s5e, scale_layout=SW, out=y5e), {"y": y5e})
 
     jobs.append(Job("if4 16384x8192 bf16 quantize", "if4.cu", nb_q5, 1,
                     lambda: fq.fp4q_quantize_if4(x5, amax=amax5, scale_layout=SW, out=out5),
@@ -500,27 +520,35 @@ def main():
     e2e = None
     if not args.no_e2e:
         k = args.e2e_steps or max(1, min(args.steps, 10))
-        for job in jobs:
-            job.e2e()
+        s_in, s_comp, s_out = (torch.cuda.Stream(device) for _ in range(3))
+        for i, job in enumerate(jobs):
+            job.e2e.step(s_in, s_comp, s_out, first=True)
         torch.cuda.synchronize(device)
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         h2d = d2h = 0
         e0.record(stream)
+        for st in (s_in, s_comp, s_out):
+            st.wait_event(e0)
         for _ in range(k):
             h2d = d2h = 0
             for job in jobs:
-                a, b = job.e2e()
+                a, b = job.e2e.step(s_in, s_comp, s_out, first=False)
                 h2d += a
                 d2h += b
+        for st in (s_in, s_comp, s_out):
+            ev = torch.cuda.Event()
+            ev.record(st)
+            stream.wait_event(ev)
         e1.record(stream)
         torch.cuda.synchronize(device)
         e_ms = fdist.max_over_ranks(e0.elapsed_time(e1), device=device)
         e2e = {"value": round(fdist.aggregate_gbs(step_bytes, ws, k, e_ms), 3), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k,
                "path": "pinned host -> device copy, C-ABI call (tensor amax computed inside), "
-                       "device -> pinned host copy of every output"}
+                       "device -> pinned host copy of every output; copies, calls and copies "
+                       "back on three streams, so neighbouring jobs' transfers overlap"}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

@@ -285,16 +285,20 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
                            static_cast<uint32_t>(warp * 2 * kRCTileBytes);
   const uint4 *stage_g = reinterpret_cast<const uint4 *>(rc_smem + warp * 2 * kRCTileBytes);
   // lane L copies the 16-byte pieces L + 32 i: row (L + 32 i) / 8, chunk L % 8
+  // row (L >> 3) + 4 i lies in the 16-row band i / 4 for every lane, and rows
+  // is a multiple of 16, so the row bound is one test per band
   auto issue = [&](const TileCursor &t, int st) {
-    const int64_t tr = t.tt, tc = t.tc;
-    const int64_t col = tc * G::WC + cc * CPT;
+    const int64_t col = t.tc * G::WC + cc * CPT;
     if (col >= cols) return;
-    const uint32_t dst = stage_s + static_cast<uint32_t>(st * kRCTileBytes + cc * 16);
+    const int64_t row0 = t.tt * G::WR;
+    const T *src = x + (row0 + (lane >> 3)) * ld + col;
+    const uint32_t dst =
+        stage_s + static_cast<uint32_t>(st * kRCTileBytes + (lane >> 3) * 128 + cc * 16);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int row = (lane >> 3) + 4 * i;
-      if (tr * G::WR + row < rows)
-        cp_async16(dst + static_cast<uint32_t>(row * 128), x + (tr * G::WR + row) * ld + col);
+      if (row0 + 16 * (i / 4) >= rows) break;
+      cp_async16(dst + static_cast<uint32_t>(i * 512), src);
+      src += 4 * ld;
     }
   };
   const int64_t dtr = nwarps / tiles_c, dtc = nwarps - dtr * tiles_c;

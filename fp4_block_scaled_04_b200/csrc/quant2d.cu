@@ -62,15 +62,20 @@ quant2d_kernel(const T *__restrict__ w, int64_t rows, int64_t cols, int64_t ld,
   const uint4 *stage_g = reinterpret_cast<const uint4 *>(smem + warp * 2 * kTileBytes);
   // lane L copies the 16-byte pieces L + 32 i: row (L + 32 i) / 8, chunk L % 8;
   // each warp copy instruction moves four whole 128-byte row segments
+  // row (L >> 3) + 4 i lies in the 16-row band i / 4 for every lane, and rows
+  // is a multiple of 16, so the row bound is one test per band
   auto issue = [&](const TileCursor &t, int st) {
     const int64_t col = t.tc * WC + cc * CPT;
     if (col >= cols) return;
-    const uint32_t dst = stage_s + static_cast<uint32_t>(st * kTileBytes + cc * 16);
+    const int64_t row0 = t.tt * 64;
+    const T *src = w + (row0 + (lane >> 3)) * ld + col;
+    const uint32_t dst =
+        stage_s + static_cast<uint32_t>(st * kTileBytes + (lane >> 3) * 128 + cc * 16);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int row = (lane >> 3) + 4 * i;
-      if (t.tt * 64 + row < rows)
-        cp_async16(dst + static_cast<uint32_t>(row * 128), w + (t.tt * 64 + row) * ld + col);
+      if (row0 + 16 * (i / 4) >= rows) break;
+      cp_async16(dst + static_cast<uint32_t>(i * 512), src);
+      src += 4 * ld;
     }
   };
   TileCursor cur, nxt;                                    // this tile, the one being copied

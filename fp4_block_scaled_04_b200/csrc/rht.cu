@@ -98,7 +98,7 @@ __device__ __forceinline__ void xstage(float2 (&lo)[16], float2 (&hi)[16]) {
 
 
 template <typename T, int N, bool SR, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kThreads, N == 16 ? 4 : 3)
+__global__ void __launch_bounds__(kThreads, (N == 16 && !SR) ? 4 : 3)
 rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
            const RhtParams P, const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
            unsigned *__restrict__ amax_out, uint8_t *__restrict__ q_t,
@@ -147,17 +147,25 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   // the data to the lanes that read it (PPT = pieces per token row)
   constexpr int PPT = sizeof(T);                          // 16-byte pieces per token row
   constexpr int UPP = 16 / UB;                            // units per piece
+  // token (L + 32 i) / PPT = tok0 + TPI i and piece pc = L % PPT; the 16-token
+  // group of copy i is TPI i / 16 for every lane, so the token bound (tokens
+  // is a multiple of 16) is one test per i, and a piece is all-in or all-out
+  // (cols % 8 == 0)
+  constexpr int TPI = 32 / PPT;                           // tokens per copy step
+  const int tok0 = lane / PPT, pc = lane % PPT;
+  const uint32_t lane_dst = in_s + static_cast<uint32_t>(unit_of(tok0, pc * UPP) * UB);
   auto issue = [&](const TileCursor &t, int st) {
-    const int64_t tbase = t.tt * 128, cbase = t.tc * 16;
-    const uint32_t dst0 = in_s + static_cast<uint32_t>(st * kUnits * UB);
+    const int64_t tbase = t.tt * 128;
+    const int64_t col = t.tc * 16 + pc * (16 / static_cast<int>(sizeof(T)));
+    if (col >= cols) return;
+    const T *src = dy + (tbase + tok0) * ld + col;
+    const uint32_t dst = lane_dst + static_cast<uint32_t>(st * kUnits * UB);
 #pragma unroll
     for (int i = 0; i < 4 * PPT; ++i) {
-      const int piece = lane + 32 * i;
-      const int tok = piece / PPT, pc = piece % PPT;
-      const int64_t col = cbase + pc * (16 / static_cast<int>(sizeof(T)));
-      if (tbase + tok < tokens && col < cols)
-        cp_async16(dst0 + static_cast<uint32_t>(unit_of(tok, pc * UPP) * UB),
-                     dy + (tbase + tok) * ld + col);
+      if (tbase + 16 * ((TPI * i) / 16) >= tokens) break;
+      // unit_of(tok0 + TPI i, .) - unit_of(tok0, .) = 4 TPI i + 2 ((TPI i) / 16)
+      cp_async16(dst + static_cast<uint32_t>((4 * TPI * i + 2 * ((TPI * i) / 16)) * UB), src);
+      src += TPI * ld;
     }
   };
 
