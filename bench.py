@@ -307,6 +307,20 @@ def suite_inputs():
             "gradient": workloads.gradient(), "if4": workloads.if4_blocks()}
 
 
+def input_digests(inputs):
+    """First 16 hex digits of the SHA-256 of each input's bytes, for the log."""
+    out = {}
+    for k, t in inputs.items():
+        b = t.contiguous().view(-1).view(torch_uint8()).numpy().tobytes()
+        out[k] = hashlib.sha256(b).hexdigest()[:16]
+    return out
+
+
+def torch_uint8():
+    import torch
+    return torch.uint8
+
+
 def oracle_sample(rows_fraction: float, inputs=None):
     """Run the oracle over the first rows_fraction of every workload of the
     suite; returns (algorithmic bytes of the sample, seconds, description)."""
@@ -569,7 +583,8 @@ def main():
                        "l2": "flushed before every kernel (256 MiB written then read, untimed)",
                        "launch": "device sleep before each flush hides host launch latency",
                        "amax": "precomputed on the device (headline); e2e computes it",
-                       "parallelism": f"replicas x{ws}" if ws > 1 else "single gpu"},
+                       "parallelism": f"replicas x{ws}" if ws > 1 else "single gpu",
+                       "input_sha256_16": input_digests(inputs)},
             "pct_of_peak": round(100 * value / (ws * peak), 2),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": sum(j.launches for j in jobs) * args.steps,
