@@ -162,12 +162,6 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
   constexpr int STAGE = 32 * LB;              // bytes of a warp's stage
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float rtab[128];
-  const TensorScale ts = tensor_scale(*amax_ptr);
-  fill_factor_table(rtab, ts.enc);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
-  __syncthreads();
-  const float c76 = __fdiv_rn(7.0f, 6.0f);   // RN(7/6)
-  const float c67 = __fdiv_rn(6.0f, 7.0f);   // RN(6/7)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // piece i of this lane sits in slot i ^ swz: eight consecutive lanes then
@@ -204,6 +198,14 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     cp_async_commit();
     ci.advance(stride, dr, dpc, ppr);
   }
+  // the tensor scale and the factor table are set up while the first tiles
+  // are already in flight
+  const TensorScale ts = tensor_scale(*amax_ptr);
+  fill_factor_table(rtab, ts.enc);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
+  __syncthreads();
+  const float c76 = __fdiv_rn(7.0f, 6.0f);   // RN(7/6)
+  const float c67 = __fdiv_rn(6.0f, 7.0f);   // RN(6/7)
   for (int st = 0; cc.p < npairs; st = (st + 1 == kStages ? 0 : st + 1)) {
     issue(ci, st == 0 ? kStages - 1 : st - 1);
     cp_async_commit();

@@ -264,13 +264,6 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
   using G = RCGeom<T, MX>;
   constexpr int CPT = G::CPT, BLK = G::BLK, GR = G::GR;
   __shared__ float rtab[128];
-  TensorScale ts{1.0f, 1.0f};
-  if (!MX) {
-    ts = tensor_scale(*amax_ptr);
-    fill_factor_table(rtab, ts.enc);
-    if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
-  }
-  __syncthreads();
   const PhiloxKey K(seed);
   const bool do_row = (layouts & FP4Q_ROWWISE) != 0;
   const bool do_col = (layouts & FP4Q_COLWISE) != 0;
@@ -308,6 +301,15 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
   if (nxt.tile < ntiles) issue(nxt, 0);
   cp_async_commit();
   nxt.advance(nwarps, dtr, dtc, tiles_c);
+  // the tensor scale and the factor table are set up while the first tile
+  // is already in flight
+  TensorScale ts{1.0f, 1.0f};
+  if (!MX) {
+    ts = tensor_scale(*amax_ptr);
+    fill_factor_table(rtab, ts.enc);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
+  }
+  __syncthreads();
   for (int st = 0; cur.tile < ntiles; cur.advance(nwarps, dtr, dtc, tiles_c), st ^= 1) {
     __syncwarp();   // every lane is done with stage st ^ 1 before it is refilled
     if (nxt.tile < ntiles) issue(nxt, st ^ 1);

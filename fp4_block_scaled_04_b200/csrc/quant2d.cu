@@ -45,10 +45,6 @@ quant2d_kernel(const T *__restrict__ w, int64_t rows, int64_t cols, int64_t ld,
   constexpr int LPT = 16 / CPT;             // lanes per tile
   constexpr int WC = 8 * CPT;               // warp tile columns
   __shared__ float rtab[128];
-  const TensorScale ts = tensor_scale(*amax_ptr);
-  fill_factor_table(rtab, ts.enc);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
-  __syncthreads();
 
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, cc = lane & 7, band = lane >> 3, warp = threadIdx.x >> 5;
@@ -84,6 +80,12 @@ quant2d_kernel(const T *__restrict__ w, int64_t rows, int64_t cols, int64_t ld,
   if (nxt.tile < ntiles) issue(nxt, 0);
   cp_async_commit();
   nxt.advance(nwarps, dtr, dtc, tiles_c);
+  // the tensor scale and the factor table are set up while the first tile
+  // is already in flight
+  const TensorScale ts = tensor_scale(*amax_ptr);
+  fill_factor_table(rtab, ts.enc);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
+  __syncthreads();
   for (int st = 0; cur.tile < ntiles; cur.advance(nwarps, dtr, dtc, tiles_c), st ^= 1) {
     __syncwarp();   // every lane is done with stage st ^ 1 before it is refilled
     if (nxt.tile < ntiles) issue(nxt, st ^ 1);

@@ -108,13 +108,6 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   constexpr int WARP_BYTES = IN_BYTES + (N == 128 ? 128 * 16 * 4 : 0);
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float rtab[128];
-  TensorScale ts{1.0f, 1.0f};
-  if (!AMAX_ONLY) {
-    ts = tensor_scale(*amax_ptr);
-    fill_factor_table(rtab, ts.enc);
-    if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
-  }
-  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane & 7, cq = lane >> 3;
   uint8_t *wbase = smem + warp * WARP_BYTES;
   const uint32_t in_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbase));
@@ -173,6 +166,15 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   if (nxt.tile < ntiles) issue(nxt, 0);
   cp_async_commit();
   nxt.advance(nwarps, dtt, dtc, tiles_c);
+  // the tensor scale and the factor table are set up while the first tile
+  // is already in flight
+  TensorScale ts{1.0f, 1.0f};
+  if (!AMAX_ONLY) {
+    ts = tensor_scale(*amax_ptr);
+    fill_factor_table(rtab, ts.enc);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
+  }
+  __syncthreads();
   for (int st = 0; cur.tile < ntiles; cur.advance(nwarps, dtt, dtc, tiles_c), st ^= 1) {
     __syncwarp();   // every lane is done with stage st ^ 1 (last tile) before it is refilled
     if (nxt.tile < ntiles) issue(nxt, st ^ 1);
