@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "orc_if4_c76": (F, []),
             "orc_if4_c67": (F, []),
             "orc_quantize_if4": (I, [P, I, I64, I64, I64, P, P, P, P, I, I]),
+            "orc_quantize_four_over_six": (I, [P, I, I64, I64, I64, U, P, P, P, P, P, P, I]),
             "orc_dequantize": (I, [I, P, P, I, I, I, P, I64, I64, P, I]),
             "orc_glossary_mae": (ctypes.c_double, [P, I64, I64]),
             "orc_e2m1_rne_n": (None, [P, P, I64]),
@@ -260,6 +261,28 @@ def quantize_nvfp4(x: np.ndarray, layouts: int = ROWWISE, round: int = RNE, seed
     return out
 
 
+def quantize_four_over_six(x: np.ndarray, layouts: int = ROWWISE, amax: float | None = None,
+                           scale_layout: int = SCALE_LINEAR) -> dict:
+    """NVFP4 1x16 layout with every block maximum mapped to 4 (the 4/6 method)."""
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    out = {"s_dec": np.zeros(1, np.float32)}
+    if layouts & ROWWISE:
+        out["q_row"] = np.zeros((rows, cols // 2), np.uint8)
+        out["sf_row"] = np.zeros(scale_bytes(rows, cols // 16, scale_layout), np.uint8)
+    if layouts & COLWISE:
+        out["q_col"] = np.zeros((cols, rows // 2), np.uint8)
+        out["sf_col"] = np.zeros(scale_bytes(cols, rows // 16, scale_layout), np.uint8)
+    keep, ap = _amax_arg(amax)
+    rc = lib().orc_quantize_four_over_six(_ptr(x), _dtype_code(x), rows, cols, cols, layouts,
+                                          ap, _ptr(out["s_dec"]), _ptr(out.get("q_row")),
+                                          _ptr(out.get("sf_row")), _ptr(out.get("q_col")),
+                                          _ptr(out.get("sf_col")), scale_layout)
+    if rc != 0:
+        raise ValueError(f"oracle rejected shape {x.shape}")
+    return out
+
+
 def quantize_mxfp4(x: np.ndarray, layouts: int = ROWWISE, e8m0_mode: int = E8M0_RNE,
                    scale_layout: int = SCALE_LINEAR) -> dict:
     x = np.ascontiguousarray(x)
@@ -334,7 +357,9 @@ def if4_constants():
 
 
 def quantize_if4(x: np.ndarray, amax: float | None = None, scale_layout: int = SCALE_LINEAR,
-                 allow_int4: bool = True) -> dict:
+                 allow_int4: bool = True, int4_only: bool = False) -> dict:
+    """IF4 (default); allow_int4=False: FP4 in every block (NVFP4);
+    int4_only=True: INT4 in every block (NVINT4)."""
     x = np.ascontiguousarray(x)
     rows, cols = x.shape
     out = {"s_dec": np.zeros(1, np.float32),
@@ -343,7 +368,7 @@ def quantize_if4(x: np.ndarray, amax: float | None = None, scale_layout: int = S
     keep, ap = _amax_arg(amax)
     rc = lib().orc_quantize_if4(_ptr(x), _dtype_code(x), rows, cols, cols, ap,
                                 _ptr(out["s_dec"]), _ptr(out["q"]), _ptr(out["sf"]),
-                                scale_layout, 1 if allow_int4 else 0)
+                                scale_layout, 2 if int4_only else (1 if allow_int4 else 0))
     if rc != 0:
         raise ValueError(f"oracle rejected shape {x.shape}")
     return out

@@ -284,21 +284,32 @@ float orc_amax(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld)
 /* global (encode) scale s_enc = RN(2688 / amax), clamped to FLT_MAX, and
  * the stored (decode) scale s_dec = RN(amax / 2688).  amax == 0 gives 1, 1.
  * 2688 = 6 * 448 is the largest NVFP4 magnitude ([Q] "NVFP4の表現できる最大値"). */
-void orc_tensor_scales(float amax, float *s_enc, float *s_dec) {
+/* The same with the largest scaled magnitude as a parameter: top = qmax *
+ * 448 for a block grid whose maximum is qmax (6 for NVFP4, 4 for 4/6). */
+static void tensor_scales_top(float amax, float top, float *s_enc, float *s_dec) {
   if (amax == 0.0f) { *s_enc = 1.0f; *s_dec = 1.0f; return; }
-  float e = 2688.0f / amax;
+  float e = top / amax;
   if (e > FLT_MAX) e = FLT_MAX;
   *s_enc = e;
-  *s_dec = amax / 2688.0f;
+  *s_dec = amax / top;
 }
 
-/* One NVFP4 block scale  [Q] "scaleの導出": x2 = x * global_scale, the
- * block's local scale is max|x2| / 6 cast to E4M3.  Because RN is monotone,
- * max|RN(x * s)| = RN(max|x| * s), so the block maximum is taken on x. */
-static uint8_t nvfp4_block_scale(float block_amax, float s_enc) {
+void orc_tensor_scales(float amax, float *s_enc, float *s_dec) {
+  tensor_scales_top(amax, 2688.0f, s_enc, s_dec);
+}
+
+/* One block scale  [Q] "scaleの導出": x2 = x * global_scale, the block's
+ * local scale is max|x2| / qmax cast to E4M3 (qmax = 6 for NVFP4).  Because
+ * RN is monotone, max|RN(x * s)| = RN(max|x| * s), so the block maximum is
+ * taken on x. */
+static uint8_t block_scale_q(float block_amax, float s_enc, float qmax) {
   float x2_max = block_amax * s_enc;
-  float local = x2_max / 6.0f;
+  float local = x2_max / qmax;
   return orc_e4m3_rne_sat(local);
+}
+
+static uint8_t nvfp4_block_scale(float block_amax, float s_enc) {
+  return block_scale_q(block_amax, s_enc, 6.0f);
 }
 
 /* READING: the element step divides by the block scale once per block:
@@ -334,15 +345,16 @@ static void put_nibble(uint8_t *q, int64_t byte_index, int high, uint8_t code) {
   else q[byte_index] = (uint8_t)((q[byte_index] & 0xF0) | (code & 0xF));
 }
 
-int orc_quantize_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
-                       unsigned layouts, int round, uint64_t seed, const float *amax_in,
-                       float *s_dec_out, uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col,
-                       uint8_t *sf_col, int scale_layout) {
+/* 1x16 quantization with block grid maximum qmax (6: NVFP4, 4: 4/6). */
+static int quantize_1x16(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                         unsigned layouts, int round, uint64_t seed, const float *amax_in,
+                         float *s_dec_out, uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col,
+                         uint8_t *sf_col, int scale_layout, float qmax) {
   if ((layouts & ORC_ROWWISE) && cols % 16 != 0) return 1;
   if ((layouts & ORC_COLWISE) && rows % 16 != 0) return 1;
   float amax = amax_in ? *amax_in : orc_amax(x, dtype, rows, cols, ld);
   float s_enc, s_dec;
-  orc_tensor_scales(amax, &s_enc, &s_dec);
+  tensor_scales_top(amax, qmax * 448.0f, &s_enc, &s_dec);
   if (s_dec_out) *s_dec_out = s_dec;
 
   if (layouts & ORC_ROWWISE) {
@@ -353,7 +365,7 @@ int orc_quantize_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols, int
           float a = fabsf(load_elem(x, dtype, ld, r, b * 16 + k));
           if (a > m) m = a;
         }
-        uint8_t sf = nvfp4_block_scale(m, s_enc);
+        uint8_t sf = block_scale_q(m, s_enc, qmax);
         float rf = nvfp4_block_factor(sf, s_enc);
         sf_row[orc_scale_offset(r, b, rows, cols / 16, scale_layout)] = sf;
         for (int k = 0; k < 16; ++k) {
@@ -372,7 +384,7 @@ int orc_quantize_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols, int
           float a = fabsf(load_elem(x, dtype, ld, b * 16 + k, c));
           if (a > m) m = a;
         }
-        uint8_t sf = nvfp4_block_scale(m, s_enc);
+        uint8_t sf = block_scale_q(m, s_enc, qmax);
         float rf = nvfp4_block_factor(sf, s_enc);
         sf_col[orc_scale_offset(c, b, cols, rows / 16, scale_layout)] = sf;
         for (int k = 0; k < 16; ++k) {
@@ -384,6 +396,34 @@ int orc_quantize_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols, int
       }
   }
   return 0;
+}
+
+int orc_quantize_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                       unsigned layouts, int round, uint64_t seed, const float *amax_in,
+                       float *s_dec_out, uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col,
+                       uint8_t *sf_col, int scale_layout) {
+  return quantize_1x16(x, dtype, rows, cols, ld, layouts, round, seed, amax_in, s_dec_out,
+                       q_row, sf_row, q_col, sf_col, scale_layout, 6.0f);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Four over six ("4/6"), the remedy [I] section 1 contrasts IF4 with: the   */
+/* block maximum is mapped to 4 instead of 6, which makes the grid finer     */
+/* relative to the block at the cost of the codes +-6.                       */
+/* READING: everything else is NVFP4 1x16 with 4 in place of 6: tensor       */
+/* scales s_enc = RN(1792 / amax), s_dec = RN(amax / 1792) (1792 = 4 * 448,  */
+/* so the block scales use the E4M3 range as NVFP4's do), block scale        */
+/* S = E4M3_rne_sat(RN(RN(m * s_enc) / 4)), r = RN(s_enc / S),               */
+/* v = RN(x * r), E2M1 round to nearest even.  |v| <= 4 (1 + 2^-4) < 5, so    */
+/* no code reaches 6.  Dequantization is NVFP4's, y = RN(RN(g * S) * s_dec). */
+/* ------------------------------------------------------------------------ */
+
+int orc_quantize_four_over_six(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                               unsigned layouts, const float *amax_in, float *s_dec_out,
+                               uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col, uint8_t *sf_col,
+                               int scale_layout) {
+  return quantize_1x16(x, dtype, rows, cols, ld, layouts, ORC_RNE, 0, amax_in, s_dec_out,
+                       q_row, sf_row, q_col, sf_col, scale_layout, 4.0f);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -578,7 +618,10 @@ int orc_quantize_rht(const void *dy, int dtype, int64_t tokens, int64_t cols, in
 /*         order i = 0..15 as e = fma(d, d, e) with d = RN(v_i - q_i)         */
 /*   INT4 iff e_int < e_fp (ties keep FP4).                                   */
 /* READING: INT4 nibbles hold k_i in two's complement; scale bit 7 set means  */
-/* INT4.  With allow_int4 = 0 the result is NVFP4 row-wise byte for byte.    */
+/* INT4.  int4_mode 1 is IF4; 0 keeps FP4 everywhere (NVFP4 row-wise byte for */
+/* byte); 2 keeps INT4 everywhere: NVINT4, the INT4 comparison format of [I] */
+/* section 4, read as IF4's INT4 candidate (same scale S, 6/7 method) in     */
+/* every block, flagged so that the IF4 dequantization decodes it.           */
 /* ------------------------------------------------------------------------ */
 
 float orc_if4_c76(void) { return 7.0f / 6.0f; }
@@ -586,7 +629,7 @@ float orc_if4_c67(void) { return 6.0f / 7.0f; }
 
 int orc_quantize_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                      const float *amax_in, float *s_dec_out, uint8_t *q, uint8_t *sf_out,
-                     int scale_layout, int allow_int4) {
+                     int scale_layout, int int4_mode) {
   if (cols % 16 != 0) return 1;
   float amax = amax_in ? *amax_in : orc_amax(x, dtype, rows, cols, ld);
   float s_enc, s_dec;
@@ -620,7 +663,7 @@ int orc_quantize_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64
         e_fp = fmaf(d_fp, d_fp, e_fp);
         e_int = fmaf(d_int, d_int, e_int);
       }
-      int use_int = allow_int4 && (e_int < e_fp);
+      int use_int = int4_mode == 2 || (int4_mode == 1 && e_int < e_fp);
       sf_out[orc_scale_offset(r, b, rows, cols / 16, scale_layout)] =
           (uint8_t)(sf | (use_int ? 0x80 : 0x00));
       for (int k = 0; k < 16; ++k) {
