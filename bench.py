@@ -223,6 +223,32 @@ def build_jobs(device, fq, inputs):
     return jobs
 
 
+def build_extra_jobs(device, fq, inputs):
+    """The comparison formats of the IF4 explainer, timed like the suite but
+    reported apart from its value: four-over-six on the activation workload
+    (row + col, swizzled) and NVINT4 on the IF4 workload (swizzled)."""
+    import torch
+    SW = fq.SCALE_SWIZZLED
+    xa = inputs["activation"].to(device)
+    amax_a = fq.fp4q_amax(xa)
+    o46 = fq.fp4q_quantize_four_over_six(xa, layouts=3, amax=amax_a, scale_layout=SW)
+    R, C = xa.shape
+    nb46 = R * C * 2 + 2 * (R * C // 2) + 2 * (R * C // 16) + 4
+    x5 = inputs["if4"].to(device)
+    amax5 = fq.fp4q_amax(x5)
+    oi4 = fq.fp4q_quantize_nvint4(x5, amax=amax5, scale_layout=SW)
+    R5, C5 = x5.shape
+    nbi4 = R5 * C5 * 2 + R5 * C5 // 2 + R5 * C5 // 16 + 4
+    torch.cuda.synchronize(device)
+    return [
+        Job("activation 8192x4096 bf16 four-over-six row+col", "nvfp4.cu", nb46, 1,
+            lambda: fq.fp4q_quantize_four_over_six(xa, layouts=3, amax=amax_a, scale_layout=SW,
+                                                   out=o46)),
+        Job("if4 16384x8192 bf16 nvint4", "if4.cu", nbi4, 1,
+            lambda: fq.fp4q_quantize_nvint4(x5, amax=amax5, scale_layout=SW, out=oi4)),
+    ]
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region (NVML, read only)
 # ---------------------------------------------------------------------------
@@ -443,6 +469,8 @@ def main():
     ap.add_argument("--cpu-baseline-fraction", type=float, default=1.0 / 8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip timing the comparison formats (four-over-six, NVINT4)")
     ap.add_argument("--e2e-steps", type=int, default=None)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -513,6 +541,33 @@ def main():
     step_bytes = sum(j.bytes for j in jobs)
     value = fdist.aggregate_gbs(step_bytes, ws, args.steps, total_ms_max)
     peak, peak_kind = hbm_peak()
+
+    # ---- comparison formats, timed the same way, outside the headline -------
+    extra = []
+    if not args.no_extra:
+        xjobs = build_extra_jobs(device, fq, inputs)
+        for job in xjobs:
+            for _ in range(args.warmup):
+                torch.cuda._sleep(LEAD_SLEEP_CYCLES)
+                flush.fill_(1.0)
+                torch.sum(flush, dim=0, out=flush_sum)
+                job.run()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for a, b in ev:
+                torch.cuda._sleep(LEAD_SLEEP_CYCLES)
+                flush.fill_(2.0)
+                torch.sum(flush, dim=0, out=flush_sum)
+                a.record(stream)
+                job.run()
+                b.record(stream)
+            torch.cuda.synchronize(device)
+            avg_s = sum(a.elapsed_time(b) for a, b in ev) * 1e-3 / args.steps
+            gbs = job.bytes / avg_s / 1e9
+            extra.append({"workload": job.name, "bytes": job.bytes, "us": round(avg_s * 1e6, 2),
+                          "GB/s": round(gbs, 1), "pct_of_peak": round(100 * gbs / peak, 1)})
+        del xjobs
+        torch.cuda.synchronize(device)
 
     per_config = []
     for job, ms in zip(jobs, per_job_ms):
@@ -590,6 +645,7 @@ def main():
             "gpu_launches": sum(j.launches for j in jobs) * args.steps,
             "clocks": clocks.summary(), "wall_s_timed_region": round(wall, 4),
             "per_config": per_config,
+            "extra_configs": extra,
         }
         print(json.dumps(line), flush=True)
     if ws > 1:

@@ -29,7 +29,7 @@ __all__ = [
     "fp4q_status_string", "fp4q_version", "fp4q_workspace_bytes", "fp4q_scale_bytes",
     "fp4q_amax", "fp4q_quantize_nvfp4", "fp4q_quantize_mxfp4", "fp4q_quantize_2d",
     "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
-    "fp4q_quantize_nvfp4_noalloc",
+    "fp4q_quantize_nvfp4_noalloc", "fp4q_quantize_nvint4", "fp4q_quantize_four_over_six",
 ]
 
 ROWWISE, COLWISE = 1, 2
@@ -83,6 +83,9 @@ _SIGNATURES = {
     "fp4q_dequantize": (_I, [_I, _P, _P, _I, _I, _I, _P, _I64, _I64, _P, _I, _P]),
     "fp4q_quantize_nvfp4_noalloc": (_I, [_P, _I, _I64, _I64, _I64, _U, _I, _U64, _P, _P, _P,
                                          _P, _P, _P, _I, _P]),
+    "fp4q_quantize_nvint4": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _SZ, _P]),
+    "fp4q_quantize_four_over_six": (_I, [_P, _I, _I64, _I64, _I64, _U, _P, _P, _P, _P, _P, _P,
+                                         _I, _P, _SZ, _P]),
 }
 
 
@@ -315,6 +318,49 @@ def fp4q_quantize_if4(x: torch.Tensor, amax: torch.Tensor | None = None,
         _ptr(x), _dtype(x), rows, cols, ld, _ptr(amax), _ptr(out.get("s_dec")),
         _ptr(out.get("q")), _ptr(out.get("sf")), scale_layout, _ptr(ws),
         0 if ws is None else ws.numel(), _stream(dev)))
+    return out
+
+
+def fp4q_quantize_nvint4(x: torch.Tensor, amax: torch.Tensor | None = None,
+                         scale_layout: int = SCALE_LINEAR, out: dict | None = None) -> dict:
+    """NVINT4 row-wise 1x16 (IF4's INT4 candidate in every block, flagged);
+    returns {'s_dec', 'q', 'sf'}; decode with FMT_IF4."""
+    rows, cols, ld = _matrix(x)
+    dev = x.device
+    if out is None:
+        out = {"s_dec": torch.empty(1, dtype=torch.float32, device=dev),
+               "q": _u8((rows, cols // 2), dev),
+               "sf": _u8(fp4q_scale_bytes(rows, cols, 16, scale_layout), dev)}
+    ws = _workspace(dev) if amax is None else None
+    _check("fp4q_quantize_nvint4", lib().fp4q_quantize_nvint4(
+        _ptr(x), _dtype(x), rows, cols, ld, _ptr(amax), _ptr(out.get("s_dec")),
+        _ptr(out.get("q")), _ptr(out.get("sf")), scale_layout, _ptr(ws),
+        0 if ws is None else ws.numel(), _stream(dev)))
+    return out
+
+
+def fp4q_quantize_four_over_six(x: torch.Tensor, layouts: int = ROWWISE,
+                                amax: torch.Tensor | None = None,
+                                scale_layout: int = SCALE_LINEAR, out: dict | None = None) -> dict:
+    """NVFP4 1x16 layout with every block maximum mapped to 4 (the 4/6 method);
+    returns {'s_dec', 'q_row', 'sf_row', 'q_col', 'sf_col'} (requested ones);
+    decode with FMT_NVFP4."""
+    rows, cols, ld = _matrix(x)
+    dev = x.device
+    if out is None:
+        out = {"s_dec": torch.empty(1, dtype=torch.float32, device=dev)}
+        if layouts & ROWWISE:
+            out["q_row"] = _u8((rows, cols // 2), dev)
+            out["sf_row"] = _u8(fp4q_scale_bytes(rows, cols, 16, scale_layout), dev)
+        if layouts & COLWISE:
+            out["q_col"] = _u8((cols, rows // 2), dev)
+            out["sf_col"] = _u8(fp4q_scale_bytes(cols, rows, 16, scale_layout), dev)
+    ws = _workspace(dev) if amax is None else None
+    _check("fp4q_quantize_four_over_six", lib().fp4q_quantize_four_over_six(
+        _ptr(x), _dtype(x), rows, cols, ld, layouts, _ptr(amax), _ptr(out.get("s_dec")),
+        _ptr(out.get("q_row")), _ptr(out.get("sf_row")), _ptr(out.get("q_col")),
+        _ptr(out.get("sf_col")), scale_layout, _ptr(ws), 0 if ws is None else ws.numel(),
+        _stream(dev)))
     return out
 
 

@@ -90,8 +90,9 @@ fp4q_status check_swizzle(int layout, int64_t srows, int64_t scols) {
 
 fp4q_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA; }
 
+template <int QMAX = 6>
 __global__ void write_s_dec_kernel(const float *amax, float *out) {
-  if (threadIdx.x == 0) *out = tensor_scale(*amax).dec;
+  if (threadIdx.x == 0) *out = tensor_scale_q<QMAX>(*amax).dec;
 }
 
 // Resolve the tensor amax: the caller's pointer, or one computed into the
@@ -121,6 +122,43 @@ fp4q_status resolve_amax(const void *x, int dtype, int64_t rows, int64_t cols, i
 }  // namespace fp4q
 
 using namespace fp4q;
+
+namespace fp4q {
+namespace {
+
+fp4q_status quantize_if4_mode(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                              const float *amax, float *tensor_scale_out, uint8_t *q,
+                              uint8_t *sf, int scale_layout, void *workspace, size_t ws_bytes,
+                              void *stream, int int4_mode) {
+  FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
+  if (!valid_layout(scale_layout)) return FP4Q_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
+  if ((!q || !sf) && rows > 0 && cols > 0) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned16(q)) return FP4Q_ERR_MISALIGNED;
+  FP4Q_TRY(check_swizzle(scale_layout, rows, cols / 16));
+  Launch L;
+  bool none = false;
+  FP4Q_TRY(bind_first({x, tensor_scale_out, amax}, stream, &L, &none));
+  if (none) return FP4Q_OK;
+  if (rows > 0 && cols > 0) {
+    FP4Q_TRY(check_dev(q, false));
+    FP4Q_TRY(check_dev(sf, false));
+  }
+  FP4Q_TRY(check_dev(amax, true));
+  FP4Q_TRY(check_dev(tensor_scale_out, true));
+  const float *a = nullptr;
+  FP4Q_TRY(resolve_amax(x, dtype, rows, cols, ld, amax, workspace, ws_bytes, L, &a));
+  if (rows == 0 || cols == 0) {
+    if (tensor_scale_out) write_s_dec_kernel<<<1, 1, 0, L.stream>>>(a, tensor_scale_out);
+    return cuda_status(cudaGetLastError());
+  }
+  return cuda_status(
+      launch_if4(x, dtype, rows, cols, ld, a, tensor_scale_out, q, sf, scale_layout, int4_mode,
+                 L));
+}
+
+}  // namespace
+}  // namespace fp4q
 
 extern "C" {
 
@@ -326,30 +364,55 @@ fp4q_status fp4q_quantize_if4(const void *x, int dtype, int64_t rows, int64_t co
                               const float *amax, float *tensor_scale_out, uint8_t *q,
                               uint8_t *sf, int scale_layout, void *workspace, size_t ws_bytes,
                               void *stream) {
+  return quantize_if4_mode(x, dtype, rows, cols, ld, amax, tensor_scale_out, q, sf, scale_layout,
+                           workspace, ws_bytes, stream, 1);
+}
+
+fp4q_status fp4q_quantize_nvint4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                                 const float *amax, float *tensor_scale_out, uint8_t *q,
+                                 uint8_t *sf, int scale_layout, void *workspace,
+                                 size_t ws_bytes, void *stream) {
+  return quantize_if4_mode(x, dtype, rows, cols, ld, amax, tensor_scale_out, q, sf, scale_layout,
+                           workspace, ws_bytes, stream, 2);
+}
+
+fp4q_status fp4q_quantize_four_over_six(const void *x, int dtype, int64_t rows, int64_t cols,
+                                        int64_t ld, unsigned layouts, const float *amax,
+                                        float *tensor_scale_out, uint8_t *q_row, uint8_t *sf_row,
+                                        uint8_t *q_col, uint8_t *sf_col, int scale_layout,
+                                        void *workspace, size_t ws_bytes, void *stream) {
   FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
+  if (layouts == 0 || (layouts & ~(FP4Q_ROWWISE | FP4Q_COLWISE)) != 0) return FP4Q_ERR_INVALID_ARG;
   if (!valid_layout(scale_layout)) return FP4Q_ERR_INVALID_ARG;
   if (cols % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
-  if ((!q || !sf) && rows > 0 && cols > 0) return FP4Q_ERR_INVALID_ARG;
-  if (!aligned16(q)) return FP4Q_ERR_MISALIGNED;
-  FP4Q_TRY(check_swizzle(scale_layout, rows, cols / 16));
+  if ((layouts & FP4Q_COLWISE) && rows % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
+  const bool nonempty = rows > 0 && cols > 0;
+  if (layouts & FP4Q_ROWWISE) {
+    if ((!q_row || !sf_row) && nonempty) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned16(q_row)) return FP4Q_ERR_MISALIGNED;
+    FP4Q_TRY(check_swizzle(scale_layout, rows, cols / 16));
+  }
+  if (layouts & FP4Q_COLWISE) {
+    if ((!q_col || !sf_col) && nonempty) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned16(q_col)) return FP4Q_ERR_MISALIGNED;
+    FP4Q_TRY(check_swizzle(scale_layout, cols, rows / 16));
+  }
   Launch L;
   bool none = false;
   FP4Q_TRY(bind_first({x, tensor_scale_out, amax}, stream, &L, &none));
   if (none) return FP4Q_OK;
-  if (rows > 0 && cols > 0) {
-    FP4Q_TRY(check_dev(q, false));
-    FP4Q_TRY(check_dev(sf, false));
-  }
   FP4Q_TRY(check_dev(amax, true));
   FP4Q_TRY(check_dev(tensor_scale_out, true));
+  FP4Q_TRY(check_dev((layouts & FP4Q_ROWWISE) ? q_row : nullptr, true));
+  FP4Q_TRY(check_dev((layouts & FP4Q_COLWISE) ? q_col : nullptr, true));
   const float *a = nullptr;
   FP4Q_TRY(resolve_amax(x, dtype, rows, cols, ld, amax, workspace, ws_bytes, L, &a));
-  if (rows == 0 || cols == 0) {
-    if (tensor_scale_out) write_s_dec_kernel<<<1, 1, 0, L.stream>>>(a, tensor_scale_out);
+  if (!nonempty) {
+    if (tensor_scale_out) write_s_dec_kernel<4><<<1, 1, 0, L.stream>>>(a, tensor_scale_out);
     return cuda_status(cudaGetLastError());
   }
-  return cuda_status(
-      launch_if4(x, dtype, rows, cols, ld, a, tensor_scale_out, q, sf, scale_layout, L));
+  return cuda_status(launch_four_over_six(x, dtype, rows, cols, ld, layouts, a, tensor_scale_out,
+                                          q_row, sf_row, q_col, sf_col, scale_layout, L));
 }
 
 fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,

@@ -19,7 +19,6 @@
 
 namespace fp4q {
 
-constexpr float kNvfp4Max = 2688.0f;   // 6 (E2M1 max) * 448 (E4M3 max)
 
 // ---------------------------------------------------------------------------
 // element loads
@@ -116,16 +115,25 @@ struct TensorScale {
   float dec;  // RN(amax / 2688); 1 if amax == 0
 };
 
-__device__ __forceinline__ TensorScale tensor_scale(float amax) {
+// Tensor scales for a block grid whose largest magnitude is QMAX: the top
+// value is QMAX * 448 (E4M3 max), 2688 for NVFP4 (QMAX 6) and 1792 for the
+// four-over-six variant (QMAX 4).
+template <int QMAX>
+__device__ __forceinline__ TensorScale tensor_scale_q(float amax) {
+  constexpr float top = static_cast<float>(QMAX) * 448.0f;
   TensorScale t;
   if (amax == 0.0f) {
     t.enc = 1.0f;
     t.dec = 1.0f;
   } else {
-    t.enc = fminf(__fdiv_rn(kNvfp4Max, amax), 3.402823466e+38f);
-    t.dec = __fdiv_rn(amax, kNvfp4Max);
+    t.enc = fminf(__fdiv_rn(top, amax), 3.402823466e+38f);
+    t.dec = __fdiv_rn(amax, top);
   }
   return t;
+}
+
+__device__ __forceinline__ TensorScale tensor_scale(float amax) {
+  return tensor_scale_q<6>(amax);
 }
 
 // RN(y / 6) in three instructions: Markstein's correction of RN(y * RN(1/6))
@@ -146,6 +154,15 @@ __device__ __forceinline__ float div6(float y) {
 // below the smallest E4M3 subnormal and give code 0.
 __device__ __forceinline__ uint32_t nvfp4_scale_code(float block_amax, float s_enc) {
   return e4m3_code(div6(__fmul_rn(block_amax, s_enc)));
+}
+
+// The same for a grid maximum QMAX: RN(RN(m * s_enc) / QMAX); dividing by 4
+// is the exact product with 0.25.
+template <int QMAX>
+__device__ __forceinline__ uint32_t scale_code_q(float block_amax, float s_enc) {
+  static_assert(QMAX == 6 || QMAX == 4, "grid maximum 6 or 4");
+  if (QMAX == 6) return nvfp4_scale_code(block_amax, s_enc);
+  return e4m3_code(__fmul_rn(__fmul_rn(block_amax, s_enc), 0.25f));
 }
 
 // Per-CTA table of r = RN(s_enc / S) for the 128 non-negative E4M3 codes

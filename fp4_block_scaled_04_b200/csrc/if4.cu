@@ -75,23 +75,26 @@ __device__ __forceinline__ uint32_t fp4_codes_diffs(const float (&v)[8], float (
 }
 
 // Both candidates of blocks A and B (lanes .x / .y of the pairs); picks the
-// smaller error per block.
-template <bool CLAMP>
+// smaller error per block (MODE 1, IF4) or keeps INT4 (MODE 2, NVINT4, which
+// needs neither the FP4 candidate nor the errors).
+template <bool CLAMP, int MODE>
 __device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float c67,
                                          uint32_t (&wa)[2], uint32_t (&wb)[2], bool &int_a,
                                          bool &int_b) {
   // FP4 candidates and their differences, in element order
-  uint32_t fpa[2], fpb[2];
+  uint32_t fpa[2] = {0u, 0u}, fpb[2] = {0u, 0u};
   float da[16], db[16];
+  if (MODE == 1) {
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    float ta[8], tb[8], ea[8], eb[8];
+    for (int h = 0; h < 2; ++h) {
+      float ta[8], tb[8], ea[8], eb[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) { ta[k] = v[8 * h + k].x; tb[k] = v[8 * h + k].y; }
-    fpa[h] = fp4_codes_diffs(ta, ea);
-    fpb[h] = fp4_codes_diffs(tb, eb);
+      for (int k = 0; k < 8; ++k) { ta[k] = v[8 * h + k].x; tb[k] = v[8 * h + k].y; }
+      fpa[h] = fp4_codes_diffs(ta, ea);
+      fpb[h] = fp4_codes_diffs(tb, eb);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) { da[8 * h + k] = ea[k]; db[8 * h + k] = eb[k]; }
+      for (int k = 0; k < 8; ++k) { da[8 * h + k] = ea[k]; db[8 * h + k] = eb[k]; }
+    }
   }
   float2 efp = make_float2(0.0f, 0.0f), eint = make_float2(0.0f, 0.0f);
   uint32_t ia[2] = {0u, 0u}, ib[2] = {0u, 0u};
@@ -109,11 +112,13 @@ __device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float
       ty = fminf(fmaxf(ty, -7.25f), 7.25f);
     }
     const float2 tm = make_float2(__fadd_rn(tx, kMagic), __fadd_rn(ty, kMagic));
-    const float2 kf = sub2(tm, make_float2(kMagic, kMagic));    // rint(t), exact
-    const float2 hv = mul2(kf, make_float2(c67, c67));
-    const float2 dint = make_float2(__fsub_rn(vk.x, hv.x), __fsub_rn(vk.y, hv.y));
-    efp = fma2(make_float2(da[k], db[k]), make_float2(da[k], db[k]), efp);
-    eint = fma2(dint, dint, eint);
+    if (MODE == 1) {
+      const float2 kf = sub2(tm, make_float2(kMagic, kMagic));    // rint(t), exact
+      const float2 hv = mul2(kf, make_float2(c67, c67));
+      const float2 dint = make_float2(__fsub_rn(vk.x, hv.x), __fsub_rn(vk.y, hv.y));
+      efp = fma2(make_float2(da[k], db[k]), make_float2(da[k], db[k]), efp);
+      eint = fma2(dint, dint, eint);
+    }
     ia[h] += __float_as_uint(tm.x) << (4 * i);
     ib[h] += __float_as_uint(tm.y) << (4 * i);
   }
@@ -122,8 +127,8 @@ __device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float
     ia[h] = (ia[h] - kPackBias) ^ 0x88888888u;
     ib[h] = (ib[h] - kPackBias) ^ 0x88888888u;
   }
-  int_a = eint.x < efp.x;
-  int_b = eint.y < efp.y;
+  int_a = MODE == 2 || eint.x < efp.x;
+  int_b = MODE == 2 || eint.y < efp.y;
   wa[0] = int_a ? ia[0] : fpa[0];
   wa[1] = int_a ? ia[1] : fpa[1];
   wb[0] = int_b ? ib[0] : fpb[0];
@@ -151,7 +156,7 @@ struct Cursor {
   }
 };
 
-template <typename T, bool SWZ>
+template <typename T, bool SWZ, int MODE>
 __global__ void __launch_bounds__(kThreads, 4)
 if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
            const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
@@ -267,9 +272,9 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     uint32_t wa[2], wb[2];
     bool ia, ib;
     if (ta < 7.5f && tb < 7.5f)
-      if4_pair<false>(v, c76, c67, wa, wb, ia, ib);
+      if4_pair<false, MODE>(v, c76, c67, wa, wb, ia, ib);
     else
-      if4_pair<true>(v, c76, c67, wa, wb, ia, ib);
+      if4_pair<true, MODE>(v, c76, c67, wa, wb, ia, ib);
     uint8_t *qp = q + r * (cols / 2) + cb * 8;
     const uint32_t ba = sa | (ia ? 0x80u : 0u), bb = sb | (ib ? 0x80u : 0u);
     if (has_b) {
@@ -298,11 +303,11 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
   cp_async_wait<0>();
 }
 
-template <typename T, bool SWZ>
+template <typename T, bool SWZ, int MODE>
 cudaError_t launch_t(const T *x, int64_t rows, int64_t cols, int64_t ld, const float *amax,
                      float *s_dec_out, uint8_t *q, uint8_t *sf, const Launch &L) {
   constexpr int SMEM = kWarps * kStages * 32 * 32 * static_cast<int>(sizeof(T));
-  const void *kern = reinterpret_cast<const void *>(if4_kernel<T, SWZ>);
+  const void *kern = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE>);
   static int per_sm = 0;
   if (per_sm == 0) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
@@ -319,30 +324,40 @@ cudaError_t launch_t(const T *x, int64_t rows, int64_t cols, int64_t ld, const f
   const int64_t want = (npairs + kThreads - 1) / kThreads;
   const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
   const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-  if4_kernel<T, SWZ><<<grid, kThreads, SMEM, L.stream>>>(x, rows, cols, ld, amax, s_dec_out, q,
+  if4_kernel<T, SWZ, MODE><<<grid, kThreads, SMEM, L.stream>>>(x, rows, cols, ld, amax, s_dec_out, q,
                                                          sf);
   return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, int MODE>
 cudaError_t launch_layout(const void *x, int64_t rows, int64_t cols, int64_t ld,
                           const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,
                           int scale_layout, const Launch &L) {
   const T *p = static_cast<const T *>(x);
   if (scale_layout == FP4Q_SCALE_SWIZZLED_128x4)
-    return launch_t<T, true>(p, rows, cols, ld, amax, s_dec_out, q, sf, L);
-  return launch_t<T, false>(p, rows, cols, ld, amax, s_dec_out, q, sf, L);
+    return launch_t<T, true, MODE>(p, rows, cols, ld, amax, s_dec_out, q, sf, L);
+  return launch_t<T, false, MODE>(p, rows, cols, ld, amax, s_dec_out, q, sf, L);
+}
+
+template <typename T>
+cudaError_t launch_mode(const void *x, int64_t rows, int64_t cols, int64_t ld,
+                        const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,
+                        int scale_layout, int int4_mode, const Launch &L) {
+  if (int4_mode == 2)
+    return launch_layout<T, 2>(x, rows, cols, ld, amax, s_dec_out, q, sf, scale_layout, L);
+  return launch_layout<T, 1>(x, rows, cols, ld, amax, s_dec_out, q, sf, scale_layout, L);
 }
 
 }  // namespace
 
 cudaError_t launch_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                        const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,
-                       int scale_layout, const Launch &L) {
+                       int scale_layout, int int4_mode, const Launch &L) {
   if (dtype == FP4Q_BF16)
-    return launch_layout<__nv_bfloat16>(x, rows, cols, ld, amax, s_dec_out, q, sf, scale_layout,
-                                        L);
-  return launch_layout<float>(x, rows, cols, ld, amax, s_dec_out, q, sf, scale_layout, L);
+    return launch_mode<__nv_bfloat16>(x, rows, cols, ld, amax, s_dec_out, q, sf, scale_layout,
+                                      int4_mode, L);
+  return launch_mode<float>(x, rows, cols, ld, amax, s_dec_out, q, sf, scale_layout, int4_mode,
+                            L);
 }
 
 }  // namespace fp4q

@@ -21,6 +21,13 @@ cudaError_t launch_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols, i
                          float *s_dec_out, uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col,
                          uint8_t *sf_col, int scale_layout, const Launch &L);
 
+// NVFP4 1x16 layout with every block maximum mapped to 4 (round to nearest)
+cudaError_t launch_four_over_six(const void *x, int dtype, int64_t rows, int64_t cols,
+                                 int64_t ld, unsigned layouts, const float *amax,
+                                 float *s_dec_out, uint8_t *q_row, uint8_t *sf_row,
+                                 uint8_t *q_col, uint8_t *sf_col, int scale_layout,
+                                 const Launch &L);
+
 cudaError_t launch_mxfp4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                          unsigned layouts, int e8m0_mode, uint8_t *q_row, uint8_t *sf_row,
                          uint8_t *q_col, uint8_t *sf_col, int scale_layout, const Launch &L);
@@ -39,9 +46,10 @@ cudaError_t launch_rht_quant(const void *dy, int dtype, int64_t tokens, int64_t 
                              float *s_dec_out, uint8_t *q_t, uint8_t *sf_t, int scale_layout,
                              float *rht_out, const Launch &L);
 
+// int4_mode 1: IF4 (per-block choice); 2: NVINT4 (the INT4 candidate everywhere)
 cudaError_t launch_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                        const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,
-                       int scale_layout, const Launch &L);
+                       int scale_layout, int int4_mode, const Launch &L);
 
 cudaError_t launch_dequant(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,
                            int block_rows, int block_cols, const float *s_dec, int64_t rows,

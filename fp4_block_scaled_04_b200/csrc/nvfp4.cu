@@ -116,7 +116,7 @@ __device__ __forceinline__ void encode_rne(const float (&v)[BLK], float f,
   }
 }
 
-template <typename T, bool MX, bool SR>
+template <typename T, bool MX, bool SR, int QMAX>
 __global__ void __launch_bounds__(kRowThreads)
 rowwise_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                const float *__restrict__ amax_ptr, int e8m0_mode, uint64_t seed,
@@ -127,7 +127,7 @@ rowwise_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
   __shared__ float rtab[128];
   TensorScale ts{1.0f, 1.0f};
   if (!MX) {
-    ts = tensor_scale(*amax_ptr);
+    ts = tensor_scale_q<QMAX>(*amax_ptr);
     fill_factor_table(rtab, ts.enc);
     if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
     __syncthreads();
@@ -157,7 +157,7 @@ rowwise_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
         sbyte = e8m0_biased(m, e8m0_mode);
         f = e8m0_inverse(sbyte);
       } else {
-        sbyte = nvfp4_scale_code(m, ts.enc);
+        sbyte = scale_code_q<QMAX>(m, ts.enc);
         f = rtab[sbyte];
       }
       float v[BLK];
@@ -237,7 +237,7 @@ __device__ __forceinline__ uint32_t rowpair_max_bf16(uint4 a, uint4 b) {
   return maxabs_bf16x2(__byte_perm(ma, mb, 0x5410), __byte_perm(ma, mb, 0x7632));
 }
 
-template <typename T, bool MX>
+template <typename T, bool MX, int QMAX>
 __device__ __forceinline__ uint32_t block_scale(float m, const TensorScale &ts, const float *rtab,
                                                 int mode, float &f) {
   if (MX) {
@@ -245,7 +245,7 @@ __device__ __forceinline__ uint32_t block_scale(float m, const TensorScale &ts, 
     f = e8m0_inverse(be);
     return be;
   }
-  const uint32_t code = nvfp4_scale_code(m, ts.enc);
+  const uint32_t code = scale_code_q<QMAX>(m, ts.enc);
   f = rtab[code];
   return code;
 }
@@ -254,7 +254,7 @@ __device__ __forceinline__ uint32_t block_scale(float m, const TensorScale &ts, 
 constexpr int kRCTileBytes = 64 * 128;            // one warp tile: 64 rows x 128 bytes
 constexpr int kRCSmem = (kRCThreads / 32) * 2 * kRCTileBytes;
 
-template <typename T, bool MX, bool SR>
+template <typename T, bool MX, bool SR, int QMAX>
 __global__ void __launch_bounds__(kRCThreads, SR ? 2 : 3)
 rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, unsigned layouts,
               const float *__restrict__ amax_ptr, int e8m0_mode, uint64_t seed,
@@ -305,7 +305,7 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
   // is already in flight
   TensorScale ts{1.0f, 1.0f};
   if (!MX) {
-    ts = tensor_scale(*amax_ptr);
+    ts = tensor_scale_q<QMAX>(*amax_ptr);
     fill_factor_table(rtab, ts.enc);
     if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
   }
@@ -388,7 +388,7 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
 #pragma unroll
         for (int g = 1; g < GR; ++g)
           if (g == gi) m = rmax[i * GR + g];
-        const uint32_t b = block_scale<T, MX>(m, ts, rtab, e8m0_mode, own_f[i]);
+        const uint32_t b = block_scale<T, MX, QMAX>(m, ts, rtab, e8m0_mode, own_f[i]);
         if (valid && do_row) srow[i * GR * step] = static_cast<uint8_t>(b);
       }
     }
@@ -396,7 +396,7 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
     for (int k = 0; k < 16; ++k)
       rf[k] = GR == 1 ? own_f[k] : __shfl_sync(0xFFFFFFFFu, own_f[k / GR], lane - gi + k % GR);
 #pragma unroll
-    for (int j = 0; j < CPT; ++j) cbyte[j] = block_scale<T, MX>(cmax[j], ts, rtab, e8m0_mode, cf[j]);
+    for (int j = 0; j < CPT; ++j) cbyte[j] = block_scale<T, MX, QMAX>(cmax[j], ts, rtab, e8m0_mode, cf[j]);
     if (valid && do_col && (!MX || (band & 1) == 0)) {
       const int64_t base = scale_offset(c0, r0 / BLK, rows / BLK, scale_layout);
       const int64_t step = swz ? 16 : rows / BLK;
@@ -495,7 +495,7 @@ int grid_cap(const void *kernel, int threads, const Launch &L) {
   return per_sm * L.num_sms;
 }
 
-template <typename T, bool MX, bool SR>
+template <typename T, bool MX, bool SR, int QMAX = 6>
 cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, unsigned layouts,
                          const float *amax, int e8m0_mode, uint64_t seed, float *s_dec_out,
                          uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col, uint8_t *sf_col,
@@ -504,16 +504,16 @@ cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, uns
   if (layouts == FP4Q_ROWWISE) {
     const int64_t nblk = rows * (cols / BLK);
     static int cap = 0;
-    if (cap == 0) cap = grid_cap(reinterpret_cast<const void *>(rowwise_kernel<T, MX, SR>),
+    if (cap == 0) cap = grid_cap(reinterpret_cast<const void *>(rowwise_kernel<T, MX, SR, QMAX>),
                                  kRowThreads, L);
     const int64_t want = (nblk + 2 * kRowThreads - 1) / (2 * kRowThreads);
     const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-    rowwise_kernel<T, MX, SR><<<grid, kRowThreads, 0, L.stream>>>(
+    rowwise_kernel<T, MX, SR, QMAX><<<grid, kRowThreads, 0, L.stream>>>(
         x, rows, cols, ld, amax, e8m0_mode, seed, s_dec_out, q_row, sf_row, scale_layout);
   } else {
     using G = RCGeom<T, MX>;
     const int64_t ntiles = ((cols + G::WC - 1) / G::WC) * ((rows + G::WR - 1) / G::WR);
-    const void *kern = reinterpret_cast<const void *>(rowcol_kernel<T, MX, SR>);
+    const void *kern = reinterpret_cast<const void *>(rowcol_kernel<T, MX, SR, QMAX>);
     static int per_sm = 0;
     if (per_sm == 0) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRCSmem) !=
@@ -529,7 +529,7 @@ cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, uns
     const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
     const int64_t want = (ntiles + kRCThreads / 32 - 1) / (kRCThreads / 32);
     const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-    rowcol_kernel<T, MX, SR><<<grid, kRCThreads, kRCSmem, L.stream>>>(
+    rowcol_kernel<T, MX, SR, QMAX><<<grid, kRCThreads, kRCSmem, L.stream>>>(
         x, rows, cols, ld, layouts, amax, e8m0_mode, seed, s_dec_out, q_row, sf_row, q_col,
         sf_col, scale_layout);
   }
@@ -558,6 +558,20 @@ cudaError_t launch_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols, i
             : launch_typed<float, false, false>(p, rows, cols, ld, layouts, amax, 0, seed,
                                                 s_dec_out, q_row, sf_row, q_col, sf_col,
                                                 scale_layout, L);
+}
+
+cudaError_t launch_four_over_six(const void *x, int dtype, int64_t rows, int64_t cols,
+                                 int64_t ld, unsigned layouts, const float *amax,
+                                 float *s_dec_out, uint8_t *q_row, uint8_t *sf_row,
+                                 uint8_t *q_col, uint8_t *sf_col, int scale_layout,
+                                 const Launch &L) {
+  if (dtype == FP4Q_BF16)
+    return launch_typed<__nv_bfloat16, false, false, 4>(
+        static_cast<const __nv_bfloat16 *>(x), rows, cols, ld, layouts, amax, 0, 0, s_dec_out,
+        q_row, sf_row, q_col, sf_col, scale_layout, L);
+  return launch_typed<float, false, false, 4>(static_cast<const float *>(x), rows, cols, ld,
+                                              layouts, amax, 0, 0, s_dec_out, q_row, sf_row,
+                                              q_col, sf_col, scale_layout, L);
 }
 
 cudaError_t launch_mxfp4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,

@@ -22,11 +22,22 @@ import fp4_block_scaled_04_b200 as fq
 from fp4_block_scaled_04_b200 import workloads
 
 OPS = ["amax", "nvfp4_row", "nvfp4_rowcol", "mxfp4_rowcol", "2d", "rht16_sr", "rht128_sr",
-       "rht16_rne", "rht128_rne", "if4", "if4_dequant"]
+       "rht16_rne", "rht128_rne", "if4", "if4_dequant", "four_over_six_rowcol", "nvint4"]
 
 
 def make(op: str, rows: int, cols: int, dev):
     sw = fq.SCALE_SWIZZLED if rows % 128 == 0 else fq.SCALE_LINEAR
+    if op == "four_over_six_rowcol":
+        x = workloads.activation(rows=rows, cols=cols).to(dev)
+        a = fq.fp4q_amax(x)
+        o = fq.fp4q_quantize_four_over_six(x, layouts=3, amax=a, scale_layout=sw)
+        return lambda: fq.fp4q_quantize_four_over_six(x, layouts=3, amax=a, scale_layout=sw,
+                                                      out=o)
+    if op == "nvint4":
+        x = workloads.if4_blocks(rows=rows, cols=cols).to(dev)
+        a = fq.fp4q_amax(x)
+        o = fq.fp4q_quantize_nvint4(x, amax=a, scale_layout=sw)
+        return lambda: fq.fp4q_quantize_nvint4(x, amax=a, scale_layout=sw, out=o)
     if op in ("amax", "nvfp4_row", "nvfp4_rowcol", "mxfp4_rowcol"):
         x = workloads.activation(rows=rows, cols=cols).to(dev)
         if op == "amax":

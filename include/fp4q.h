@@ -205,6 +205,31 @@ fp4q_status fp4q_quantize_if4(const void *x, int dtype, int64_t rows, int64_t co
                               uint8_t *sf, int scale_layout, void *workspace, size_t ws_bytes,
                               void *stream);
 
+/* NVINT4, the INT4 comparison format of the "Adaptive Block-Scaled Data
+ * Types" explainer (section 4), read as IF4's INT4 candidate in every block:
+ * the NVFP4 scale S and factor r, v = RN(x*r), k = clamp(rint(RN(v * RN(7/6))),
+ * -7, 7) in two's complement, and bit 7 of every scale byte set, so that
+ * fp4q_dequantize(FP4Q_FMT_IF4, ...) decodes it (k * RN(6/7) * S * s_dec).
+ * Arguments, layouts and errors as for fp4q_quantize_if4. */
+fp4q_status fp4q_quantize_nvint4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                                 const float *amax, float *tensor_scale_out, uint8_t *q,
+                                 uint8_t *sf, int scale_layout, void *workspace,
+                                 size_t ws_bytes, void *stream);
+
+/* Four over six ("4/6"), the remedy the IF4 explainer (section 1) contrasts
+ * IF4 with: every block maximum is mapped to 4 instead of 6, giving a finer
+ * grid relative to the block at the cost of the codes +-6.  Read as NVFP4
+ * 1x16 with 4 in place of 6: s_enc = RN(1792/amax), s_dec = RN(amax/1792)
+ * (1792 = 4 * 448), S = E4M3_rne_sat(RN(RN(m * s_enc) / 4)), r = RN(s_enc/S),
+ * v = RN(x * r), E2M1 round to nearest even (|v| < 5, so no code reaches 6).
+ * Outputs, layouts and errors as for fp4q_quantize_nvfp4 with FP4Q_RNE;
+ * fp4q_dequantize(FP4Q_FMT_NVFP4, ...) with this call's s_dec decodes it. */
+fp4q_status fp4q_quantize_four_over_six(const void *x, int dtype, int64_t rows, int64_t cols,
+                                        int64_t ld, unsigned layouts, const float *amax,
+                                        float *tensor_scale_out, uint8_t *q_row, uint8_t *sf_row,
+                                        uint8_t *q_col, uint8_t *sf_col, int scale_layout,
+                                        void *workspace, size_t ws_bytes, void *stream);
+
 /* Dequantization of packed codes [rows, cols/2] back to y [rows, cols]
  * (FP32 or BF16 = RNE of the FP32 value), Ultralytics glossary "FP4の仕組み"
  * (grid value * sign * scale):
