@@ -224,9 +224,10 @@ def build_jobs(device, fq, inputs):
 
 
 def build_extra_jobs(device, fq, inputs):
-    """The comparison formats of the IF4 explainer, timed like the suite but
-    reported apart from its value: four-over-six on the activation workload
-    (row + col, swizzled) and NVINT4 on the IF4 workload (swizzled)."""
+    """Calls outside the headline suite, timed like it but reported apart from
+    its value: the fused backward call and the row-wise operand alone on the
+    gradient workload, and the IF4 explainer's comparison formats
+    (four-over-six on the activation workload, NVINT4 on the IF4 workload)."""
     import torch
     SW = fq.SCALE_SWIZZLED
     xa = inputs["activation"].to(device)
@@ -239,8 +240,37 @@ def build_extra_jobs(device, fq, inputs):
     oi4 = fq.fp4q_quantize_nvint4(x5, amax=amax5, scale_layout=SW)
     R5, C5 = x5.shape
     nbi4 = R5 * C5 * 2 + R5 * C5 // 2 + R5 * C5 // 16 + 4
+    # the fused backward call on the gradient workload, and the row-wise
+    # operand alone (the column-wise operand alone is in the suite)
+    g = inputs["gradient"].to(device)
+    T, Cg = g.shape
+    amax_g = fq.fp4q_amax(g)
+    amax_r16 = fq.fp4q_rht_amax(g, 16, seed=0)
+    obw = fq.fp4q_quantize_backward(g, 16, round=fq.SR, seed_row=1, seed_col=0, amax_row=amax_g,
+                                    amax_rht=amax_r16, scale_layout=SW)
+    orow = fq.fp4q_quantize_nvfp4(g, layouts=fq.ROWWISE, round=fq.SR, seed=1, amax=amax_g,
+                                  scale_layout=SW)
+    obw_n = fq.fp4q_quantize_backward(g, 16, round=fq.RNE, amax_row=amax_g, amax_rht=amax_r16,
+                                      scale_layout=SW)
+    orow_n = fq.fp4q_quantize_nvfp4(g, layouts=fq.ROWWISE, amax=amax_g, scale_layout=SW)
+    nb_row = T * Cg * 2 + T * Cg // 2 + T * Cg // 16 + 4
+    nb_bw = T * Cg * 2 + 2 * (T * Cg // 2 + T * Cg // 16 + 4)
     torch.cuda.synchronize(device)
     return [
+        Job("gradient 8192x5120 bf16 backward: row-wise sr + rht16+sr from one read", "rht.cu",
+            nb_bw, 1, lambda: fq.fp4q_quantize_backward(
+                g, 16, round=fq.SR, seed_row=1, seed_col=0, amax_row=amax_g, amax_rht=amax_r16,
+                scale_layout=SW, out=obw)),
+        Job("gradient 8192x5120 bf16 row-wise nvfp4 sr", "nvfp4.cu", nb_row, 1,
+            lambda: fq.fp4q_quantize_nvfp4(g, layouts=fq.ROWWISE, round=fq.SR, seed=1,
+                                           amax=amax_g, scale_layout=SW, out=orow)),
+        Job("gradient 8192x5120 bf16 backward: row-wise rne + rht16+rne from one read", "rht.cu",
+            nb_bw, 1, lambda: fq.fp4q_quantize_backward(
+                g, 16, round=fq.RNE, amax_row=amax_g, amax_rht=amax_r16, scale_layout=SW,
+                out=obw_n)),
+        Job("gradient 8192x5120 bf16 row-wise nvfp4 rne", "nvfp4.cu", nb_row, 1,
+            lambda: fq.fp4q_quantize_nvfp4(g, layouts=fq.ROWWISE, amax=amax_g, scale_layout=SW,
+                                           out=orow_n)),
         Job("activation 8192x4096 bf16 four-over-six row+col", "nvfp4.cu", nb46, 1,
             lambda: fq.fp4q_quantize_four_over_six(xa, layouts=3, amax=amax_a, scale_layout=SW,
                                                    out=o46)),
@@ -542,7 +572,7 @@ def main():
     value = fdist.aggregate_gbs(step_bytes, ws, args.steps, total_ms_max)
     peak, peak_kind = hbm_peak()
 
-    # ---- comparison formats, timed the same way, outside the headline -------
+    # ---- further calls, timed the same way, outside the headline ----------
     extra = []
     if not args.no_extra:
         xjobs = build_extra_jobs(device, fq, inputs)

@@ -30,6 +30,7 @@ __all__ = [
     "fp4q_amax", "fp4q_quantize_nvfp4", "fp4q_quantize_mxfp4", "fp4q_quantize_2d",
     "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
     "fp4q_quantize_nvfp4_noalloc", "fp4q_quantize_nvint4", "fp4q_quantize_four_over_six",
+    "fp4q_quantize_backward",
 ]
 
 ROWWISE, COLWISE = 1, 2
@@ -84,6 +85,8 @@ _SIGNATURES = {
     "fp4q_quantize_nvfp4_noalloc": (_I, [_P, _I, _I64, _I64, _I64, _U, _I, _U64, _P, _P, _P,
                                          _P, _P, _P, _I, _P]),
     "fp4q_quantize_nvint4": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _SZ, _P]),
+    "fp4q_quantize_backward": (_I, [_P, _I, _I64, _I64, _I64, _I, _I, _U64, _U64, _P, _P, _P,
+                                    _P, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "fp4q_quantize_four_over_six": (_I, [_P, _I, _I64, _I64, _I64, _U, _P, _P, _P, _P, _P, _P,
                                          _I, _P, _SZ, _P]),
 }
@@ -318,6 +321,33 @@ def fp4q_quantize_if4(x: torch.Tensor, amax: torch.Tensor | None = None,
         _ptr(x), _dtype(x), rows, cols, ld, _ptr(amax), _ptr(out.get("s_dec")),
         _ptr(out.get("q")), _ptr(out.get("sf")), scale_layout, _ptr(ws),
         0 if ws is None else ws.numel(), _stream(dev)))
+    return out
+
+
+def fp4q_quantize_backward(dy: torch.Tensor, hadamard_n: int = 16, round: int = SR,
+                           seed_row: int = 0, seed_col: int = 1,
+                           amax_row: torch.Tensor | None = None,
+                           amax_rht: torch.Tensor | None = None,
+                           scale_layout: int = SCALE_LINEAR, out: dict | None = None) -> dict:
+    """Both backward operands of dY from one read: {'s_dec_row', 'q_row', 'sf_row'}
+    (row-wise NVFP4, the Dgrad operand) and {'s_dec_col', 'q_t', 'sf_t'} (RHT +
+    column-wise NVFP4 of dY^T, the Wgrad operand)."""
+    tokens, cols, ld = _matrix(dy, "dy")
+    dev = dy.device
+    if out is None:
+        out = {"s_dec_row": torch.empty(1, dtype=torch.float32, device=dev),
+               "q_row": _u8((tokens, cols // 2), dev),
+               "sf_row": _u8(fp4q_scale_bytes(tokens, cols, 16, scale_layout), dev),
+               "s_dec_col": torch.empty(1, dtype=torch.float32, device=dev),
+               "q_t": _u8((cols, tokens // 2), dev),
+               "sf_t": _u8(fp4q_scale_bytes(cols, tokens, 16, scale_layout), dev)}
+    ws = _workspace(dev) if (amax_row is None or amax_rht is None) else None
+    _check("fp4q_quantize_backward", lib().fp4q_quantize_backward(
+        _ptr(dy), _dtype(dy), tokens, cols, ld, hadamard_n, round, seed_row, seed_col,
+        _ptr(amax_row), _ptr(amax_rht), _ptr(out.get("s_dec_row")), _ptr(out.get("s_dec_col")),
+        _ptr(out.get("q_row")), _ptr(out.get("sf_row")), _ptr(out.get("q_t")),
+        _ptr(out.get("sf_t")), scale_layout, _ptr(ws), 0 if ws is None else ws.numel(),
+        _stream(dev)))
     return out
 
 

@@ -360,6 +360,70 @@ fp4q_status fp4q_quantize_rht_sr(const void *dy, int dtype, int64_t tokens, int6
                                       L));
 }
 
+fp4q_status fp4q_quantize_backward(const void *dy, int dtype, int64_t tokens, int64_t cols,
+                                   int64_t ld, int hadamard_n, int round, uint64_t seed_row,
+                                   uint64_t seed_col, const float *amax_row,
+                                   const float *amax_rht, float *s_dec_row_out,
+                                   float *s_dec_col_out, uint8_t *q_row, uint8_t *sf_row,
+                                   uint8_t *q_t, uint8_t *sf_t, int scale_layout, void *workspace,
+                                   size_t ws_bytes, void *stream) {
+  FP4Q_TRY(check_matrix(dy, dtype, tokens, cols, ld));
+  if (hadamard_n != 16 && hadamard_n != 128) return FP4Q_ERR_INVALID_ARG;
+  if (round != FP4Q_RNE && round != FP4Q_SR) return FP4Q_ERR_INVALID_ARG;
+  if (!valid_layout(scale_layout)) return FP4Q_ERR_INVALID_ARG;
+  if (tokens % hadamard_n != 0 || cols % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
+  const bool nonempty = tokens > 0 && cols > 0;
+  if ((!q_row || !sf_row || !q_t || !sf_t) && nonempty) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned16(q_row) || !aligned16(q_t)) return FP4Q_ERR_MISALIGNED;
+  FP4Q_TRY(check_swizzle(scale_layout, tokens, cols / 16));
+  FP4Q_TRY(check_swizzle(scale_layout, cols, tokens / 16));
+  Launch L;
+  bool none = false;
+  FP4Q_TRY(bind_first({dy, s_dec_row_out, s_dec_col_out, amax_row, amax_rht}, stream, &L, &none));
+  if (none) return FP4Q_OK;
+  if (nonempty) {
+    FP4Q_TRY(check_dev(q_row, false));
+    FP4Q_TRY(check_dev(sf_row, false));
+    FP4Q_TRY(check_dev(q_t, false));
+    FP4Q_TRY(check_dev(sf_t, false));
+  }
+  FP4Q_TRY(check_dev(amax_row, true));
+  FP4Q_TRY(check_dev(amax_rht, true));
+  FP4Q_TRY(check_dev(s_dec_row_out, true));
+  FP4Q_TRY(check_dev(s_dec_col_out, true));
+  // missing amaxes are computed into the workspace: the row amax at byte 0,
+  // the amax of the transform at byte 128
+  const float *ar = amax_row, *ac = amax_rht;
+  if (ar == nullptr || ac == nullptr) {
+    if (workspace == nullptr || ws_bytes < kWorkspaceBytes) return FP4Q_ERR_WORKSPACE_TOO_SMALL;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 3u) != 0) return FP4Q_ERR_MISALIGNED;
+  }
+  if (ar == nullptr) {
+    float *w = static_cast<float *>(workspace);
+    if (nonempty)
+      FP4Q_TRY(cuda_status(launch_amax(dy, dtype, tokens, cols, ld, w, L)));
+    else
+      FP4Q_TRY(cuda_status(cudaMemsetAsync(w, 0, sizeof(float), L.stream)));
+    ar = w;
+  }
+  if (ac == nullptr) {
+    float *w = static_cast<float *>(workspace) + 32;
+    if (nonempty)
+      FP4Q_TRY(cuda_status(launch_rht_amax(dy, dtype, tokens, cols, ld, hadamard_n, seed_col, w, L)));
+    else
+      FP4Q_TRY(cuda_status(cudaMemsetAsync(w, 0, sizeof(float), L.stream)));
+    ac = w;
+  }
+  if (!nonempty) {
+    if (s_dec_row_out) write_s_dec_kernel<<<1, 1, 0, L.stream>>>(ar, s_dec_row_out);
+    if (s_dec_col_out) write_s_dec_kernel<<<1, 1, 0, L.stream>>>(ac, s_dec_col_out);
+    return cuda_status(cudaGetLastError());
+  }
+  return cuda_status(launch_rht_backward(dy, dtype, tokens, cols, ld, hadamard_n, round, seed_row,
+                                         seed_col, ar, ac, s_dec_row_out, s_dec_col_out, q_row,
+                                         sf_row, q_t, sf_t, scale_layout, L));
+}
+
 fp4q_status fp4q_quantize_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                               const float *amax, float *tensor_scale_out, uint8_t *q,
                               uint8_t *sf, int scale_layout, void *workspace, size_t ws_bytes,

@@ -46,6 +46,15 @@ cudaError_t launch_rht_quant(const void *dy, int dtype, int64_t tokens, int64_t 
                              float *s_dec_out, uint8_t *q_t, uint8_t *sf_t, int scale_layout,
                              float *rht_out, const Launch &L);
 
+// One read of dY: row-wise NVFP4 (the Dgrad operand, seed_row, amax_row) and
+// the RHT + column-wise NVFP4 of dY^T (the Wgrad operand, seed_col, amax_rht)
+cudaError_t launch_rht_backward(const void *dy, int dtype, int64_t tokens, int64_t cols,
+                                int64_t ld, int n, int round, uint64_t seed_row,
+                                uint64_t seed_col, const float *amax_row, const float *amax_rht,
+                                float *s_dec_row, float *s_dec_col, uint8_t *q_row,
+                                uint8_t *sf_row, uint8_t *q_t, uint8_t *sf_t, int scale_layout,
+                                const Launch &L);
+
 // int4_mode 1: IF4 (per-block choice); 2: NVINT4 (the INT4 candidate everywhere)
 cudaError_t launch_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                        const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,

@@ -47,8 +47,19 @@ struct RhtParams {
   uint32_t signs[4];         // bit k of word k/32: sign of token k of the diagonal
 };
 
+// The row-wise (Dgrad) output of the fused backward call: NVFP4 1x16 of dY
+// itself, with its own tensor amax and its own stochastic-rounding seed.
+struct RowArgs {
+  const float *amax;         // tensor amax of dY
+  float *s_dec_out;          // <- RN(amax / 2688) (may be NULL)
+  uint8_t *q;                // codes [tokens, cols/2]
+  uint8_t *sf;               // scales [tokens, cols/16]
+  uint32_t k0[10], k1[10];   // Philox4x32-10 round keys of the row seed
+};
+
 // Philox4x32-10 of the counter (c0, c1, 0, 0) with the caller's round keys
-__device__ __forceinline__ U32x4 philox_rk(const RhtParams &P, uint32_t c0, uint32_t c1) {
+template <typename K>
+__device__ __forceinline__ U32x4 philox_rk(const K &P, uint32_t c0, uint32_t c1) {
   uint32_t c2 = 0u, c3 = 0u;
 #pragma unroll
   for (int i = 0; i < 10; ++i) {
@@ -97,17 +108,19 @@ __device__ __forceinline__ void xstage(float2 (&lo)[16], float2 (&hi)[16]) {
 }
 
 
-template <typename T, int N, bool SR, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kThreads, (N == 16 && !SR) ? 4 : 3)
+template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW>
+__global__ void __launch_bounds__(kThreads, (N == 16 && !SR && !ROW) ? 4 : 3)
 rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
            const RhtParams P, const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
            unsigned *__restrict__ amax_out, uint8_t *__restrict__ q_t,
-           uint8_t *__restrict__ sf_t, int scale_layout, float *__restrict__ rht_out) {
+           uint8_t *__restrict__ sf_t, int scale_layout, float *__restrict__ rht_out,
+           const RowArgs R) {
   constexpr int UB = 4 * sizeof(T);                       // bytes per input chunk
   constexpr int IN_BYTES = 2 * kUnits * UB;               // two stages
   constexpr int WARP_BYTES = IN_BYTES + (N == 128 ? 128 * 16 * 4 : 0);
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float rtab[128];
+  __shared__ float rtab_row[ROW ? 128 : 1];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane & 7, cq = lane >> 3;
   uint8_t *wbase = smem + warp * WARP_BYTES;
   const uint32_t in_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbase));
@@ -168,11 +181,16 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   nxt.advance(nwarps, dtt, dtc, tiles_c);
   // the tensor scale and the factor table are set up while the first tile
   // is already in flight
-  TensorScale ts{1.0f, 1.0f};
+  TensorScale ts{1.0f, 1.0f}, tsr{1.0f, 1.0f};
   if (!AMAX_ONLY) {
     ts = tensor_scale(*amax_ptr);
     fill_factor_table(rtab, ts.enc);
     if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
+  }
+  if (ROW) {
+    tsr = tensor_scale(*R.amax);
+    fill_factor_table(rtab_row, tsr.enc);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && R.s_dec_out) *R.s_dec_out = tsr.dec;
   }
   __syncthreads();
   for (int st = 0; cur.tile < ntiles; cur.advance(nwarps, dtt, dtc, tiles_c), st ^= 1) {
@@ -352,6 +370,106 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
         sp[j * sstep] = static_cast<uint8_t>(sbyte[j]);
       }
     }
+    if (ROW) {
+      // ---- row-wise NVFP4 of dY itself (the Dgrad operand) ----------------------
+      // The stage buffer still holds this tile's raw values (it is refilled
+      // only after the next tile), so they are read again here rather than
+      // kept in registers through the transform.  A 1x16 row block is one
+      // token's 16 columns: the column quads of lanes g, g + 8, g + 16, g + 24.
+      float2 xl[16], xh[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        if (sizeof(T) == 2) {
+          const uint2 w = valid ? *reinterpret_cast<const uint2 *>(ib + 4 * k * UB) : make_uint2(0u, 0u);
+          xl[k] = make_float2(bf16_lo(w.x), bf16_hi(w.x));
+          xh[k] = make_float2(bf16_lo(w.y), bf16_hi(w.y));
+        } else {
+          const uint4 w = valid ? *reinterpret_cast<const uint4 *>(ib + 4 * k * UB)
+                                : make_uint4(0u, 0u, 0u, 0u);
+          xl[k] = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
+          xh[k] = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
+        }
+      }
+      float mk[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        mk[k] = fmaxf(fmaxf(fabsf(xl[k].x), fabsf(xl[k].y)), fmaxf(fabsf(xh[k].x), fabsf(xh[k].y)));
+      // reduce-scatter the maxima over the quads (xor 16, then xor 8): this
+      // lane ends with the tokens 8 b1 + 4 b0 + j, j = 0..3
+      const int b1 = cq >> 1, b0 = cq & 1;
+      float m8[8], m4[4], f4[4];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float send = b1 ? mk[j] : mk[8 + j], keep = b1 ? mk[8 + j] : mk[j];
+        m8[j] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 16));
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float send = b0 ? m8[j] : m8[4 + j], keep = b0 ? m8[4 + j] : m8[j];
+        m4[j] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 8));
+      }
+      const int tb = 8 * b1 + 4 * b0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t sb = nvfp4_scale_code(m4[j], tsr.enc);
+        f4[j] = rtab_row[sb];
+        if (valid)
+          R.sf[scale_offset(t0 + tb + j, cur.tc, cols / 16, scale_layout)] = static_cast<uint8_t>(sb);
+      }
+      // gather the 16 factors back (xor 8, then xor 16)
+      float f8[8], F[16];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float o = __shfl_xor_sync(0xFFFFFFFFu, f4[j], 8);
+        f8[j] = b0 ? o : f4[j];
+        f8[4 + j] = b0 ? f4[j] : o;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float o = __shfl_xor_sync(0xFFFFFFFFu, f8[j], 16);
+        F[j] = b1 ? o : f8[j];
+        F[8 + j] = b1 ? f8[j] : o;
+      }
+      // token k's four codes are 16 bits of its code row
+      auto put_row = [&](int k, float x0, float x1, float x2, float x3) {
+        if (valid)
+          *reinterpret_cast<uint16_t *>(R.q + (t0 + k) * (cols / 2) + c0 / 2) =
+              static_cast<uint16_t>(e2m1x4(x0, x1, x2, x3));
+      };
+      if (SR) {
+        // the same Philox counters as the column path, keyed on the row seed
+        const int half = cq & 1;
+        const uint64_t row0 = (static_cast<uint64_t>(t0) * static_cast<uint64_t>(cols) +
+                               static_cast<uint64_t>(c0 - 4 * half)) / 8;
+        const uint64_t rstep = static_cast<uint64_t>(cols) / 8;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint64_t gidx = row0 + static_cast<uint64_t>(i + 8 * half) * rstep;
+          const U32x4 b = philox_rk(R, static_cast<uint32_t>(gidx), static_cast<uint32_t>(gidx >> 32));
+          const uint32_t keep0 = half ? b.z : b.x, keep1 = half ? b.w : b.y;
+          const uint32_t send0 = half ? b.x : b.z, send1 = half ? b.y : b.w;
+          const uint32_t got0 = __shfl_xor_sync(0xFFFFFFFFu, send0, 8);
+          const uint32_t got1 = __shfl_xor_sync(0xFFFFFFFFu, send1, 8);
+          const uint32_t ti0 = half ? got0 : keep0, ti1 = half ? got1 : keep1;
+          const uint32_t tj0 = half ? keep0 : got0, tj1 = half ? keep1 : got1;
+          const float2 a0 = mul2(xl[i], make_float2(F[i], F[i]));
+          const float2 a1 = mul2(xh[i], make_float2(F[i], F[i]));
+          put_row(i, e2m1_sr_value(a0.x, sr_z_lo(ti0)), e2m1_sr_value(a0.y, sr_z_hi(ti0)),
+                  e2m1_sr_value(a1.x, sr_z_lo(ti1)), e2m1_sr_value(a1.y, sr_z_hi(ti1)));
+          const float2 b0v = mul2(xl[i + 8], make_float2(F[i + 8], F[i + 8]));
+          const float2 b1v = mul2(xh[i + 8], make_float2(F[i + 8], F[i + 8]));
+          put_row(i + 8, e2m1_sr_value(b0v.x, sr_z_lo(tj0)), e2m1_sr_value(b0v.y, sr_z_hi(tj0)),
+                  e2m1_sr_value(b1v.x, sr_z_lo(tj1)), e2m1_sr_value(b1v.y, sr_z_hi(tj1)));
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float2 a0 = mul2(xl[k], make_float2(F[k], F[k]));
+          const float2 a1 = mul2(xh[k], make_float2(F[k], F[k]));
+          put_row(k, a0.x, a0.y, a1.x, a1.y);
+        }
+      }
+    }
   }
   cp_async_wait<0>();
   if (AMAX_ONLY) {
@@ -392,14 +510,32 @@ RhtParams make_params(uint64_t seed) {
   return P;
 }
 
-template <typename T, int N, bool SR, bool AMAX_ONLY>
+RowArgs make_row_args(const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,
+                      uint64_t seed) {
+  RowArgs R;
+  R.amax = amax;
+  R.s_dec_out = s_dec_out;
+  R.q = q;
+  R.sf = sf;
+  uint32_t a = static_cast<uint32_t>(seed), b = static_cast<uint32_t>(seed >> 32);
+  for (int i = 0; i < 10; ++i) {
+    R.k0[i] = a;
+    R.k1[i] = b;
+    a += 0x9E3779B9u;
+    b += 0xBB67AE85u;
+  }
+  return R;
+}
+
+template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW = false>
 cudaError_t launch_k(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint64_t seed,
                      const float *amax, float *s_dec_out, unsigned *amax_out, uint8_t *q_t,
-                     uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L) {
+                     uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L,
+                     const RowArgs &R = RowArgs{}) {
   constexpr int UB = 4 * sizeof(T);
   constexpr int WARP_BYTES = 2 * kUnits * UB + (N == 128 ? 128 * 16 * 4 : 0);
   constexpr int SMEM = kWarps * WARP_BYTES;
-  const void *kern = reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY>);
+  const void *kern = reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY, ROW>);
   static int per_sm = 0;
   if (per_sm == 0) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
@@ -416,9 +552,9 @@ cudaError_t launch_k(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint
   const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
   const int64_t want = (ntiles + kWarps - 1) / kWarps;
   const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-  rht_kernel<T, N, SR, AMAX_ONLY><<<grid, kThreads, SMEM, L.stream>>>(
+  rht_kernel<T, N, SR, AMAX_ONLY, ROW><<<grid, kThreads, SMEM, L.stream>>>(
       dy, tokens, cols, ld, make_params(seed), amax, s_dec_out, amax_out, q_t, sf_t, scale_layout,
-      rht_out);
+      rht_out, R);
   return cudaGetLastError();
 }
 
@@ -450,7 +586,46 @@ cudaError_t launch_t(const void *dy, int64_t tokens, int64_t cols, int64_t ld, i
                           scale_layout, rht_out, amax_only, L);
 }
 
+template <typename T, int N>
+cudaError_t launch_bwd_n(const T *dy, int64_t tokens, int64_t cols, int64_t ld, int round,
+                         uint64_t seed_col, const float *amax_rht, float *s_dec_col,
+                         uint8_t *q_t, uint8_t *sf_t, int scale_layout, const RowArgs &R,
+                         const Launch &L) {
+  if (round == FP4Q_SR)
+    return launch_k<T, N, true, false, true>(dy, tokens, cols, ld, seed_col, amax_rht, s_dec_col,
+                                             nullptr, q_t, sf_t, scale_layout, nullptr, L, R);
+  return launch_k<T, N, false, false, true>(dy, tokens, cols, ld, seed_col, amax_rht, s_dec_col,
+                                            nullptr, q_t, sf_t, scale_layout, nullptr, L, R);
+}
+
+template <typename T>
+cudaError_t launch_bwd_t(const void *dy, int64_t tokens, int64_t cols, int64_t ld, int n,
+                         int round, uint64_t seed_col, const float *amax_rht, float *s_dec_col,
+                         uint8_t *q_t, uint8_t *sf_t, int scale_layout, const RowArgs &R,
+                         const Launch &L) {
+  const T *p = static_cast<const T *>(dy);
+  if (n == 16)
+    return launch_bwd_n<T, 16>(p, tokens, cols, ld, round, seed_col, amax_rht, s_dec_col, q_t,
+                               sf_t, scale_layout, R, L);
+  return launch_bwd_n<T, 128>(p, tokens, cols, ld, round, seed_col, amax_rht, s_dec_col, q_t,
+                              sf_t, scale_layout, R, L);
+}
+
 }  // namespace
+
+cudaError_t launch_rht_backward(const void *dy, int dtype, int64_t tokens, int64_t cols,
+                                int64_t ld, int n, int round, uint64_t seed_row,
+                                uint64_t seed_col, const float *amax_row, const float *amax_rht,
+                                float *s_dec_row, float *s_dec_col, uint8_t *q_row,
+                                uint8_t *sf_row, uint8_t *q_t, uint8_t *sf_t, int scale_layout,
+                                const Launch &L) {
+  const RowArgs R = make_row_args(amax_row, s_dec_row, q_row, sf_row, seed_row);
+  if (dtype == FP4Q_BF16)
+    return launch_bwd_t<__nv_bfloat16>(dy, tokens, cols, ld, n, round, seed_col, amax_rht,
+                                       s_dec_col, q_t, sf_t, scale_layout, R, L);
+  return launch_bwd_t<float>(dy, tokens, cols, ld, n, round, seed_col, amax_rht, s_dec_col, q_t,
+                             sf_t, scale_layout, R, L);
+}
 
 cudaError_t launch_rht_amax(const void *dy, int dtype, int64_t tokens, int64_t cols,
                             int64_t ld, int n, uint64_t seed, float *amax_out,

@@ -22,11 +22,24 @@ import fp4_block_scaled_04_b200 as fq
 from fp4_block_scaled_04_b200 import workloads
 
 OPS = ["amax", "nvfp4_row", "nvfp4_rowcol", "mxfp4_rowcol", "2d", "rht16_sr", "rht128_sr",
-       "rht16_rne", "rht128_rne", "if4", "if4_dequant", "four_over_six_rowcol", "nvint4"]
+       "rht16_rne", "rht128_rne", "if4", "if4_dequant", "four_over_six_rowcol", "nvint4",
+       "bwd16_sr", "bwd16_rne", "row_sr"]
 
 
 def make(op: str, rows: int, cols: int, dev):
     sw = fq.SCALE_SWIZZLED if rows % 128 == 0 else fq.SCALE_LINEAR
+    if op in ("bwd16_sr", "bwd16_rne", "row_sr"):
+        g = workloads.gradient(tokens=rows, cols=cols).to(dev)
+        a = fq.fp4q_amax(g)
+        ar = fq.fp4q_rht_amax(g, 16)
+        rnd = fq.RNE if op == "bwd16_rne" else fq.SR
+        if op == "row_sr":
+            o = fq.fp4q_quantize_nvfp4(g, layouts=fq.ROWWISE, round=fq.SR, amax=a, scale_layout=sw)
+            return lambda: fq.fp4q_quantize_nvfp4(g, layouts=fq.ROWWISE, round=fq.SR, amax=a,
+                                                  scale_layout=sw, out=o)
+        o = fq.fp4q_quantize_backward(g, 16, round=rnd, amax_row=a, amax_rht=ar, scale_layout=sw)
+        return lambda: fq.fp4q_quantize_backward(g, 16, round=rnd, amax_row=a, amax_rht=ar,
+                                                 scale_layout=sw, out=o)
     if op == "four_over_six_rowcol":
         x = workloads.activation(rows=rows, cols=cols).to(dev)
         a = fq.fp4q_amax(x)

@@ -191,7 +191,32 @@ fp4q_status fp4q_quantize_rht_sr(const void *dy, int dtype, int64_t tokens, int6
                                  uint8_t *sf_t, int scale_layout, float *rht_debug_out,
                                  void *workspace, size_t ws_bytes, void *stream);
 
-/* IF4 adaptive quantization, row-wise 1x16 ("Adaptive Block-Scaled Data
+/* Both quantized operands of dY for the backward pass from ONE read of dY.
+ * Qiita note, "誤差逆伝播と転置": Dgrad uses dY as is, Wgrad the transposed
+ * dY^T; "ランダムアダマール変換": the transform is applied to the Wgrad
+ * operands only.  The outputs are byte for byte those of
+ *   fp4q_quantize_nvfp4(dy, FP4Q_ROWWISE, round, seed_row, amax_row)
+ *       -> s_dec_row_out, q_row [tokens, cols/2], sf_row [tokens, cols/16]
+ *   fp4q_quantize_rht_sr(dy, hadamard_n, round, seed_col, amax_rht)
+ *       -> s_dec_col_out, q_t [cols, tokens/2], sf_t [cols, tokens/16]
+ * with separate seeds, so the two operands draw independent random bits.
+ * The random signs S depend only on seed_col: quantizing the activation X
+ * with fp4q_quantize_rht_sr and the same seed applies the same H diag(S) to
+ * the other Wgrad operand.
+ *   amax_row, amax_rht  device floats (the tensor amax of dY, and that of
+ *          its transform), or NULL: then computed first into the workspace
+ *          (each NULL costs one extra read of dY)
+ * Shape: tokens % hadamard_n == 0, cols % 16 == 0.  Both scale matrices use
+ * scale_layout. */
+fp4q_status fp4q_quantize_backward(const void *dy, int dtype, int64_t tokens, int64_t cols,
+                                   int64_t ld, int hadamard_n, int round, uint64_t seed_row,
+                                   uint64_t seed_col, const float *amax_row,
+                                   const float *amax_rht, float *s_dec_row_out,
+                                   float *s_dec_col_out, uint8_t *q_row, uint8_t *sf_row,
+                                   uint8_t *q_t, uint8_t *sf_t, int scale_layout, void *workspace,
+                                   size_t ws_bytes, void *stream);
+
+/* IF4 adaptive quantization, row-wise 1x16/* IF4 adaptive quantization, row-wise 1x16 ("Adaptive Block-Scaled Data
  * Types" explainer, section 2): per block the NVFP4 scale S and factor r,
  * v = RN(x*r); FP4 candidate E2M1_rne(v); INT4 candidate
  * k = clamp(rint(RN(v * RN(7/6))), -7, 7) decoded as RN(k * RN(6/7)) (the 6/7

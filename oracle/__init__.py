@@ -283,6 +283,20 @@ def quantize_four_over_six(x: np.ndarray, layouts: int = ROWWISE, amax: float | 
     return out
 
 
+def quantize_backward(dy: np.ndarray, n: int, round: int = SR, seed_row: int = 0,
+                      seed_col: int = 1, amax_row: float | None = None,
+                      amax_rht: float | None = None, scale_layout: int = SCALE_LINEAR) -> dict:
+    """Both backward operands of dY: the row-wise NVFP4 of dY (Dgrad operand,
+    seed_row) and the RHT + column-wise NVFP4 of dY^T (Wgrad operand,
+    seed_col) -- by definition the two oracle calls, composed."""
+    r = quantize_nvfp4(dy, layouts=ROWWISE, round=round, seed=seed_row, amax=amax_row,
+                       scale_layout=scale_layout)
+    c = quantize_rht(dy, n, round=round, seed=seed_col, amax_rht=amax_rht,
+                     scale_layout=scale_layout)
+    return {"s_dec_row": r["s_dec"], "q_row": r["q_row"], "sf_row": r["sf_row"],
+            "s_dec_col": c["s_dec"], "q_t": c["q_t"], "sf_t": c["sf_t"]}
+
+
 def quantize_mxfp4(x: np.ndarray, layouts: int = ROWWISE, e8m0_mode: int = E8M0_RNE,
                    scale_layout: int = SCALE_LINEAR) -> dict:
     x = np.ascontiguousarray(x)
