@@ -373,100 +373,73 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
     if (ROW) {
       // ---- row-wise NVFP4 of dY itself (the Dgrad operand) ----------------------
       // The stage buffer still holds this tile's raw values (it is refilled
-      // only after the next tile), so they are read again here rather than
-      // kept in registers through the transform.  A 1x16 row block is one
-      // token's 16 columns: the column quads of lanes g, g + 8, g + 16, g + 24.
-      float2 xl[16], xh[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
+      // only after the next tile), so the row blocks are read from it again
+      // with a row-friendly split: lane L takes tokens L, L + 32, L + 64,
+      // L + 96, each a whole 16-column block (32 bytes, BF16) held by one
+      // lane -- the block maximum needs no shuffles and each code row leaves
+      // as one 8-byte store.  With BF16 input, lanes L and L ^ 4 read the two
+      // 16-byte halves of their tokens in opposite order, so eight consecutive
+      // lanes hit eight distinct bank groups.
+      const uint8_t *sb0 = wbase + st * kUnits * UB;
+      const int64_t tile_t0 = cur.tt * 128, col0 = cur.tc * 16;
+      const bool cvalid = col0 < cols;
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        const int tok = lane + 32 * j;
+        const int64_t t = tile_t0 + tok;
+        const bool tv = cvalid && t < tokens;
+        const uint8_t *src = sb0 + unit_of(tok, 0) * UB;    // 16 values, 16 * sizeof(T) bytes
+        float x[16];
         if (sizeof(T) == 2) {
-          const uint2 w = valid ? *reinterpret_cast<const uint2 *>(ib + 4 * k * UB) : make_uint2(0u, 0u);
-          xl[k] = make_float2(bf16_lo(w.x), bf16_hi(w.x));
-          xh[k] = make_float2(bf16_lo(w.y), bf16_hi(w.y));
+          // two 16-byte pieces, read in lane-dependent order and put back by select
+          const int sw = (lane >> 2) & 1;
+          uint4 w0 = tv ? *reinterpret_cast<const uint4 *>(src + 16 * sw) : make_uint4(0u, 0u, 0u, 0u);
+          uint4 w1 = tv ? *reinterpret_cast<const uint4 *>(src + 16 * (sw ^ 1)) : make_uint4(0u, 0u, 0u, 0u);
+          const uint4 p0 = sw ? w1 : w0, p1 = sw ? w0 : w1;
+          const uint32_t ws[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            x[2 * i] = bf16_lo(ws[i]);
+            x[2 * i + 1] = bf16_hi(ws[i]);
+          }
         } else {
-          const uint4 w = valid ? *reinterpret_cast<const uint4 *>(ib + 4 * k * UB)
-                                : make_uint4(0u, 0u, 0u, 0u);
-          xl[k] = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
-          xh[k] = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const uint4 w = tv ? *reinterpret_cast<const uint4 *>(src + 16 * p) : make_uint4(0u, 0u, 0u, 0u);
+            x[4 * p + 0] = __uint_as_float(w.x); x[4 * p + 1] = __uint_as_float(w.y);
+            x[4 * p + 2] = __uint_as_float(w.z); x[4 * p + 3] = __uint_as_float(w.w);
+          }
         }
-      }
-      float mk[16];
+        float m = 0.0f;
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        mk[k] = fmaxf(fmaxf(fabsf(xl[k].x), fabsf(xl[k].y)), fmaxf(fabsf(xh[k].x), fabsf(xh[k].y)));
-      // reduce-scatter the maxima over the quads (xor 16, then xor 8): this
-      // lane ends with the tokens 8 b1 + 4 b0 + j, j = 0..3
-      const int b1 = cq >> 1, b0 = cq & 1;
-      float m8[8], m4[4], f4[4];
+        for (int k = 0; k < 16; ++k) m = fmaxf(m, fabsf(x[k]));
+        const uint32_t sbr = nvfp4_scale_code(m, tsr.enc);
+        const float f = rtab_row[sbr];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float send = b1 ? mk[j] : mk[8 + j], keep = b1 ? mk[8 + j] : mk[j];
-        m8[j] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 16));
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float send = b0 ? m8[j] : m8[4 + j], keep = b0 ? m8[4 + j] : m8[j];
-        m4[j] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 8));
-      }
-      const int tb = 8 * b1 + 4 * b0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t sb = nvfp4_scale_code(m4[j], tsr.enc);
-        f4[j] = rtab_row[sb];
-        if (valid)
-          R.sf[scale_offset(t0 + tb + j, cur.tc, cols / 16, scale_layout)] = static_cast<uint8_t>(sb);
-      }
-      // gather the 16 factors back (xor 8, then xor 16)
-      float f8[8], F[16];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float o = __shfl_xor_sync(0xFFFFFFFFu, f4[j], 8);
-        f8[j] = b0 ? o : f4[j];
-        f8[4 + j] = b0 ? f4[j] : o;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float o = __shfl_xor_sync(0xFFFFFFFFu, f8[j], 16);
-        F[j] = b1 ? o : f8[j];
-        F[8 + j] = b1 ? f8[j] : o;
-      }
-      // token k's four codes are 16 bits of its code row
-      auto put_row = [&](int k, float x0, float x1, float x2, float x3) {
-        if (valid)
-          *reinterpret_cast<uint16_t *>(R.q + (t0 + k) * (cols / 2) + c0 / 2) =
-              static_cast<uint16_t>(e2m1x4(x0, x1, x2, x3));
-      };
-      if (SR) {
-        // the same Philox counters as the column path, keyed on the row seed
-        const int half = cq & 1;
-        const uint64_t row0 = (static_cast<uint64_t>(t0) * static_cast<uint64_t>(cols) +
-                               static_cast<uint64_t>(c0 - 4 * half)) / 8;
-        const uint64_t rstep = static_cast<uint64_t>(cols) / 8;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint64_t gidx = row0 + static_cast<uint64_t>(i + 8 * half) * rstep;
-          const U32x4 b = philox_rk(R, static_cast<uint32_t>(gidx), static_cast<uint32_t>(gidx >> 32));
-          const uint32_t keep0 = half ? b.z : b.x, keep1 = half ? b.w : b.y;
-          const uint32_t send0 = half ? b.x : b.z, send1 = half ? b.y : b.w;
-          const uint32_t got0 = __shfl_xor_sync(0xFFFFFFFFu, send0, 8);
-          const uint32_t got1 = __shfl_xor_sync(0xFFFFFFFFu, send1, 8);
-          const uint32_t ti0 = half ? got0 : keep0, ti1 = half ? got1 : keep1;
-          const uint32_t tj0 = half ? keep0 : got0, tj1 = half ? keep1 : got1;
-          const float2 a0 = mul2(xl[i], make_float2(F[i], F[i]));
-          const float2 a1 = mul2(xh[i], make_float2(F[i], F[i]));
-          put_row(i, e2m1_sr_value(a0.x, sr_z_lo(ti0)), e2m1_sr_value(a0.y, sr_z_hi(ti0)),
-                  e2m1_sr_value(a1.x, sr_z_lo(ti1)), e2m1_sr_value(a1.y, sr_z_hi(ti1)));
-          const float2 b0v = mul2(xl[i + 8], make_float2(F[i + 8], F[i + 8]));
-          const float2 b1v = mul2(xh[i + 8], make_float2(F[i + 8], F[i + 8]));
-          put_row(i + 8, e2m1_sr_value(b0v.x, sr_z_lo(tj0)), e2m1_sr_value(b0v.y, sr_z_hi(tj0)),
-                  e2m1_sr_value(b1v.x, sr_z_lo(tj1)), e2m1_sr_value(b1v.y, sr_z_hi(tj1)));
+        for (int k = 0; k < 16; k += 2) {
+          const float2 v = mul2(make_float2(x[k], x[k + 1]), make_float2(f, f));
+          x[k] = v.x;
+          x[k + 1] = v.y;
         }
-      } else {
+        if (SR) {
+          // element (t, c) draws 16 bits from Philox call (t * cols + c) / 8
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float2 a0 = mul2(xl[k], make_float2(F[k], F[k]));
-          const float2 a1 = mul2(xh[k], make_float2(F[k], F[k]));
-          put_row(k, a0.x, a0.y, a1.x, a1.y);
+          for (int h = 0; h < 2; ++h) {
+            const uint64_t gidx = (static_cast<uint64_t>(t) * static_cast<uint64_t>(cols) +
+                                   static_cast<uint64_t>(col0 + 8 * h)) / 8;
+            const U32x4 b = philox_rk(R, static_cast<uint32_t>(gidx), static_cast<uint32_t>(gidx >> 32));
+            const uint32_t wd[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              x[8 * h + k] = e2m1_sr_value(x[8 * h + k], (k & 1) ? sr_z_hi(wd[k >> 1]) : sr_z_lo(wd[k >> 1]));
+          }
+        }
+        float lo8[8], hi8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) { lo8[k] = x[k]; hi8[k] = x[8 + k]; }
+        if (tv) {
+          *reinterpret_cast<uint2 *>(R.q + t * (cols / 2) + col0 / 2) = make_uint2(e2m1x8(lo8), e2m1x8(hi8));
+          R.sf[scale_offset(t, cur.tc, cols / 16, scale_layout)] = static_cast<uint8_t>(sbr);
         }
       }
     }
