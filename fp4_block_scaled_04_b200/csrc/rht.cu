@@ -16,10 +16,13 @@
 //     warp barriers order the copy, the reads and the refill);
 //   * the sign flip is one LOP3 per packed word, the butterfly stages
 //     h = 1, 2, 4, 8 run in registers on f32x2 column pairs;
-//   * for n = 128 the stages h = 16, 32, 64 combine the eight groups: the warp
-//     swaps values through an 8 KB shared buffer (XOR-swizzled so the write
-//     and the transposed read both spread over all banks), runs the three
-//     stages and swaps back;
+//   * for n = 128 the stages h = 16, 32, 64 combine the eight groups of a
+//     column quad: butterflies between lanes g and g ^ 1, g ^ 2, g ^ 4 by
+//     shuffle, each output fma(own, +-1, partner) (an exact product, so one
+//     rounding of the sum or difference).  With stochastic rounding, where
+//     registers are short, the warp instead swaps values through an 8 KB
+//     shared buffer (XOR-swizzled so the write and the transposed read both
+//     spread over all banks), runs the three stages and swaps back;
 //   * block maxima are in-thread; stochastic rounding needs one Philox call
 //     per token per 8 columns, which two lanes share (each computes half of
 //     the tokens and passes the other lane its 64 bits by shuffle).  The ten
@@ -107,7 +110,6 @@ __device__ __forceinline__ void xstage(float2 (&lo)[16], float2 (&hi)[16]) {
       }
 }
 
-
 template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW>
 __global__ void __launch_bounds__(kThreads, (N == 16 && !SR && !ROW) ? 4 : 3)
 rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
@@ -117,7 +119,10 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
            const RowArgs R) {
   constexpr int UB = 4 * sizeof(T);                       // bytes per input chunk
   constexpr int IN_BYTES = 2 * kUnits * UB;               // two stages
-  constexpr int WARP_BYTES = IN_BYTES + (N == 128 ? 128 * 16 * 4 : 0);
+  // with stochastic rounding the 128-point cross-group stages go through a
+  // shared exchange buffer (registers are short); otherwise through shuffles
+  constexpr bool XSMEM = N == 128 && SR;
+  constexpr int WARP_BYTES = IN_BYTES + (XSMEM ? 128 * 16 * 4 : 0);
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float rtab[128];
   __shared__ float rtab_row[ROW ? 128 : 1];
@@ -231,7 +236,28 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
     stage<4>(lo, hi);
     stage<8>(lo, hi);
 
-    if (N == 128) {
+    if (N == 128 && !XSMEM) {
+      // ---- stages h = 16, 32, 64 across the eight groups ------------------------
+      // token 16 g + k meets token 16 (g ^ m) + k, m = 1, 2, 4: the lane with
+      // bit m of g clear keeps RN(a + b), its partner RN(a - b); both are
+      // fma(own, +-1, partner), whose product is exact
+#pragma unroll
+      for (int sgi = 0; sgi < 3; ++sgi) {
+        const int m = 1 << sgi;
+        const float sg = (g & m) ? -1.0f : 1.0f;
+        const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float2 pl = make_float2(__shfl_xor_sync(0xFFFFFFFFu, lo[k].x, m),
+                                        __shfl_xor_sync(0xFFFFFFFFu, lo[k].y, m));
+          const float2 ph = make_float2(__shfl_xor_sync(0xFFFFFFFFu, hi[k].x, m),
+                                        __shfl_xor_sync(0xFFFFFFFFu, hi[k].y, m));
+          lo[k] = fma2(lo[k], sg2, pl);
+          hi[k] = fma2(hi[k], sg2, ph);
+        }
+      }
+    }
+    if (N == 128 && XSMEM) {
       // ---- stages h = 16, 32, 64 across the eight groups ------------------------
       // the 16-byte chunk of (token t, quad q) is 4t + q with its low three
       // bits XORed with (t/16 ^ t/2) mod 8; s = q ^ g is the lane's part of it
@@ -506,7 +532,7 @@ cudaError_t launch_k(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint
                      uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L,
                      const RowArgs &R = RowArgs{}) {
   constexpr int UB = 4 * sizeof(T);
-  constexpr int WARP_BYTES = 2 * kUnits * UB + (N == 128 ? 128 * 16 * 4 : 0);
+  constexpr int WARP_BYTES = 2 * kUnits * UB + ((N == 128 && SR) ? 128 * 16 * 4 : 0);
   constexpr int SMEM = kWarps * WARP_BYTES;
   const void *kern = reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY, ROW>);
   static int per_sm = 0;
