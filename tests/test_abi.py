@@ -99,6 +99,41 @@ def test_host_side_argument_checks(L):
     assert L.fp4q_dequantize(0, FAKE, FAKE, 0, 1, 16, None, 16, 64, FAKE, 1, None) == 1
 
 
+def test_host_side_argument_checks_of_the_added_calls(L):
+    # four-over-six: the NVFP4 rules
+    f46 = lambda **kw: L.fp4q_quantize_four_over_six(
+        kw.get("x", FAKE), 0, kw.get("rows", 32), kw.get("cols", 64), kw.get("ld", 64),
+        kw.get("layouts", 1), FAKE, FAKE, kw.get("q_row", FAKE), FAKE, FAKE, FAKE,
+        kw.get("layout", 0), None, 0, None)
+    assert f46(layouts=0) == 1
+    assert f46(cols=24, ld=24) == 2
+    assert f46(rows=24, layouts=2) == 2
+    assert f46(layout=1) == 2
+    assert f46(q_row=ctypes.c_void_p(0x7F0000000008)) == 3
+    assert f46(q_row=None) == 1
+    # NVINT4: the IF4 rules
+    assert L.fp4q_quantize_nvint4(FAKE, 0, 16, 40, 40, FAKE, FAKE, FAKE, FAKE, 0, None, 0,
+                                  None) == 2
+    assert L.fp4q_quantize_nvint4(FAKE, 0, 16, 48, 52, FAKE, FAKE, FAKE, FAKE, 0, None, 0,
+                                  None) == 3
+    assert L.fp4q_quantize_nvint4(FAKE, 0, 16, 48, 48, FAKE, FAKE, FAKE, FAKE, 5, None, 0,
+                                  None) == 1
+    # backward: RHT rules plus cols % 16 and both outputs
+    bw = lambda **kw: L.fp4q_quantize_backward(
+        FAKE, 0, kw.get("tokens", 128), kw.get("cols", 64), kw.get("ld", 64), kw.get("n", 16),
+        kw.get("round", 1), 0, 1, FAKE, FAKE, FAKE, FAKE, kw.get("q_row", FAKE), FAKE,
+        kw.get("q_t", FAKE), FAKE, kw.get("layout", 0), None, 0, None)
+    assert bw(n=32) == 1
+    assert bw(round=3) == 1
+    assert bw(tokens=120) == 2
+    assert bw(cols=72, ld=72) == 2                  # the row-wise output needs cols % 16
+    assert bw(q_row=None) == 1 and bw(q_t=None) == 1
+    assert bw(q_t=ctypes.c_void_p(0x7F0000000004)) == 3
+    assert bw(layout=1, tokens=128, cols=64) == 2   # swizzled dY^T scales need cols % 128
+    assert L.fp4q_quantize_nvfp4_noalloc(FAKE, 0, 32, 24, 24, 1, 0, 0, FAKE, FAKE, FAKE, FAKE,
+                                         None, None, 0, None) == 2
+
+
 def test_python_binding_refuses_cpu_tensors(L):
     import torch
     with pytest.raises(ValueError):
