@@ -30,7 +30,8 @@ ROWWISE, COLWISE = 1, 2
 RNE, SR = 0, 1
 SCALE_LINEAR, SCALE_SWIZZLED = 0, 1
 E8M0_RNE, E8M0_CEIL, E8M0_OCP_FLOOR = 0, 1, 2
-FMT_NVFP4, FMT_MXFP4, FMT_IF4 = 0, 1, 2
+FMT_NVFP4, FMT_MXFP4, FMT_IF4, FMT_MXFP6_E2M3, FMT_MXFP6_E3M2 = 0, 1, 2, 3, 4
+FP6_E2M3, FP6_E3M2 = 0, 1
 
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
 
@@ -72,6 +73,9 @@ def lib() -> ctypes.CDLL:
             "orc_tensor_scales": (None, [F, P, P]),
             "orc_quantize_nvfp4": (I, [P, I, I64, I64, I64, U, I, U64, P, P, P, P, P, P, I]),
             "orc_quantize_mxfp4": (I, [P, I, I64, I64, I64, U, I, P, P, P, P, I]),
+            "orc_quantize_mxfp6": (I, [P, I, I64, I64, I64, I, I, P, P, I]),
+            "orc_fp6_value": (F, [ctypes.c_uint8, I]),
+            "orc_fp6_rne": (ctypes.c_uint8, [F, I]),
             "orc_quantize_2d": (I, [P, I, I64, I64, I64, P, P, P, P, P, P, P, I]),
             "orc_rht_norm": (F, [I]),
             "orc_rht": (I, [P, I, I64, I64, I64, I, U64, P]),
@@ -295,6 +299,28 @@ def quantize_backward(dy: np.ndarray, n: int, round: int = SR, seed_row: int = 0
                      scale_layout=scale_layout)
     return {"s_dec_row": r["s_dec"], "q_row": r["q_row"], "sf_row": r["sf_row"],
             "s_dec_col": c["s_dec"], "q_t": c["q_t"], "sf_t": c["sf_t"]}
+
+
+def fp6_value(code: int, fmt: int) -> float:
+    return float(lib().orc_fp6_value(code, fmt))
+
+
+def fp6_rne(v: float, fmt: int) -> int:
+    return int(lib().orc_fp6_rne(float(np.float32(v)), fmt))
+
+
+def quantize_mxfp6(x: np.ndarray, fmt: int = FP6_E2M3, e8m0_mode: int = E8M0_RNE,
+                   scale_layout: int = SCALE_LINEAR) -> dict:
+    """MXFP6 row-wise 1x32 (E2M3 or E3M2 codes packed four per three bytes)."""
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    out = {"q": np.zeros((rows, cols * 3 // 4), np.uint8),
+           "sf": np.zeros(scale_bytes(rows, cols // 32, scale_layout), np.uint8)}
+    rc = lib().orc_quantize_mxfp6(_ptr(x), _dtype_code(x), rows, cols, cols, fmt, e8m0_mode,
+                                  _ptr(out["q"]), _ptr(out["sf"]), scale_layout)
+    if rc != 0:
+        raise ValueError(f"oracle rejected shape {x.shape}")
+    return out
 
 
 def quantize_mxfp4(x: np.ndarray, layouts: int = ROWWISE, e8m0_mode: int = E8M0_RNE,

@@ -47,6 +47,10 @@
 #define ORC_FMT_NVFP4 0
 #define ORC_FMT_MXFP4 1
 #define ORC_FMT_IF4 2
+#define ORC_FMT_MXFP6_E2M3 3
+#define ORC_FMT_MXFP6_E3M2 4
+#define ORC_FP6_E2M3 0
+#define ORC_FP6_E3M2 1
 
 /* ------------------------------------------------------------------------ */
 /* Scalar helpers                                                            */
@@ -165,17 +169,20 @@ static void split_pow2(float a, double *f, int *E) {
   *E = e2 - 1;
 }
 
-int orc_e8m0_exponent(float block_amax, int mode) {
+/* The exponent for an element format whose largest magnitude is qmax =
+ * 1.x * 2^emax (E2M1: 6 = 1.5 * 2^2; FP6 E2M3: 7.5 = 1.875 * 2^2; E3M2:
+ * 28 = 1.75 * 2^4). */
+static int e8m0_exponent_q(float block_amax, int mode, float qmax, int emax) {
   int e;
   if (!(block_amax > 0.0f)) return -127;
   if (mode == ORC_E8M0_OCP_FLOOR) {
-    /* floor(log2(amax)) - 2: the largest E2M1 magnitude is 1.5 * 2^2 */
+    /* floor(log2(amax)) - emax */
     double f; int E;
     split_pow2(block_amax, &f, &E);
-    e = E - 2;
+    e = E - emax;
   } else {
-    /* map the block maximum to 6: the scale before rounding is RN(amax/6) */
-    float target = block_amax / 6.0f;
+    /* map the block maximum to qmax: the scale before rounding is RN(amax/qmax) */
+    float target = block_amax / qmax;
     if (!(target > 0.0f)) return -127;
     double f; int E;
     split_pow2(target, &f, &E);
@@ -193,6 +200,10 @@ int orc_e8m0_exponent(float block_amax, int mode) {
   if (e < -127) e = -127;
   if (e > 127) e = 127;
   return e;
+}
+
+int orc_e8m0_exponent(float block_amax, int mode) {
+  return e8m0_exponent_q(block_amax, mode, 6.0f, 2);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -675,10 +686,82 @@ int orc_quantize_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64
 }
 
 /* ------------------------------------------------------------------------ */
+/* FP6 (OCP MX element formats)  [F] "FP6で隣り合う値の間隔を見てみる":       */
+/* E2M3 = sign, 2 exponent bits (bias 1), 3 mantissa bits, largest 7.5;      */
+/* E3M2 = sign, 3 exponent bits (bias 3), 2 mantissa bits, largest 28 (8, 10,*/
+/* 12, 14, then 16, 20, 24, 28; spacing 0.0625 near 0); subnormals, no Inf or*/
+/* NaN.  Codes are 6 bits, sign in bit 5.                                     */
+/* ------------------------------------------------------------------------ */
+
+float orc_fp6_value(uint8_t code, int fmt) {
+  int m = code & 0x1F;
+  int mb = (fmt == ORC_FP6_E2M3) ? 3 : 2;                /* mantissa bits */
+  int bias = (fmt == ORC_FP6_E2M3) ? 1 : 3;
+  int e = m >> mb, f = m & ((1 << mb) - 1);
+  double v = (e == 0) ? ldexp((double)f, 1 - bias - mb)
+                      : ldexp(1.0 + (double)f / (double)(1 << mb), e - bias);
+  return (float)((code & 0x20) ? -v : v);
+}
+
+/* nearest FP6 magnitude (ties to the even code), saturating at the largest,
+ * sign copied; v finite */
+uint8_t orc_fp6_rne(float v, int fmt) {
+  uint8_t sign = signbit(v) ? 0x20 : 0x00;
+  double a = fabs((double)v);
+  int best = 0;
+  double best_d = INFINITY;
+  for (int c = 0; c < 32; ++c) {
+    double d = fabs(a - (double)orc_fp6_value((uint8_t)c, fmt));
+    if (d < best_d || (d == best_d && (c % 2) == 0)) { best = c; best_d = d; }
+  }
+  if (a >= (double)orc_fp6_value(31, fmt)) best = 31;
+  return (uint8_t)(best | sign);
+}
+
+/* MXFP6: 32 values share one E8M0 scale chosen as for MXFP4 with the FP6
+ * format's largest magnitude (7.5 = 1.875 * 2^2 for E2M3, 28 = 1.75 * 2^4 for
+ * E3M2); elements v = RN(x * 2^-e), FP6 round to nearest even with
+ * saturation.  READING ([F] notes that values cross byte boundaries but fixes
+ * no order): four 6-bit codes go into three bytes, code j of the group in bits
+ * 6j..6j+5 of the little-endian 24-bit word.  Codes [rows, cols * 3/4] bytes,
+ * scales [rows, cols/32].  Row-wise only. */
+int orc_quantize_mxfp6(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld, int fmt,
+                       int e8m0_mode, uint8_t *q, uint8_t *sf, int scale_layout) {
+  if (cols % 32 != 0) return 1;
+  float qmax = orc_fp6_value(31, fmt);
+  int emax = (fmt == ORC_FP6_E2M3) ? 2 : 4;
+  int64_t rb = cols * 3 / 4;                              /* code bytes per row */
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < cols / 32; ++b) {
+      float m = 0.0f;
+      for (int k = 0; k < 32; ++k) {
+        float a = fabsf(load_elem(x, dtype, ld, r, b * 32 + k));
+        if (a > m) m = a;
+      }
+      int e = e8m0_exponent_q(m, e8m0_mode, qmax, emax);
+      sf[orc_scale_offset(r, b, rows, cols / 32, scale_layout)] = (uint8_t)(e + 127);
+      float inv = pow2f_exact(-e);
+      for (int g = 0; g < 8; ++g) {
+        uint32_t w = 0;
+        for (int j = 0; j < 4; ++j) {
+          int64_t c = b * 32 + g * 4 + j;
+          w |= (uint32_t)orc_fp6_rne(load_elem(x, dtype, ld, r, c) * inv, fmt) << (6 * j);
+        }
+        uint8_t *dst = q + r * rb + (b * 8 + g) * 3;
+        dst[0] = (uint8_t)(w & 0xFF);
+        dst[1] = (uint8_t)((w >> 8) & 0xFF);
+        dst[2] = (uint8_t)((w >> 16) & 0xFF);
+      }
+    }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Dequantization  [G] "FP4の仕組み" (reconstruct = grid value * sign * scale)*/
 /* NVFP4:  y = RN(RN(g * S) * s_dec)   (g * S is exact)                       */
 /* IF4 INT4 blocks: h = RN(k * C67), y = RN(RN(h * S) * s_dec)                */
 /* MXFP4:  y = RN(g * 2^e)                                                    */
+/* MXFP6 (E2M3 / E3M2, codes packed 4 per 3 bytes): y = RN(value * 2^e)      */
 /* Block shape: block_rows x block_cols (1x16, 1x32, or 16x16 for 2D tiles,  */
 /* whose scales are [rows/16, cols/16] linear).  Output FP32 or BF16 (RNE of */
 /* the FP32 result).                                                         */
@@ -691,10 +774,18 @@ int orc_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_la
   float s_dec = s_dec_in ? *s_dec_in : 1.0f;
   int64_t srows = rows / block_rows, scols = cols / block_cols;
   const float C67 = orc_if4_c67();
+  const int fp6 = (format == ORC_FMT_MXFP6_E2M3 || format == ORC_FMT_MXFP6_E3M2);
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t c = 0; c < cols; ++c) {
-      uint8_t byte = q[r * (cols / 2) + c / 2];
-      uint8_t code = (c & 1) ? (byte >> 4) : (byte & 0xF);
+      uint8_t code;
+      if (fp6) {
+        const uint8_t *g3 = q + r * (cols * 3 / 4) + (c / 4) * 3;
+        uint32_t w = (uint32_t)g3[0] | ((uint32_t)g3[1] << 8) | ((uint32_t)g3[2] << 16);
+        code = (uint8_t)((w >> (6 * (c % 4))) & 0x3F);
+      } else {
+        uint8_t byte = q[r * (cols / 2) + c / 2];
+        code = (c & 1) ? (byte >> 4) : (byte & 0xF);
+      }
       int64_t sr = r / block_rows, sc = c / block_cols;
       int64_t off = (block_rows == 1) ? orc_scale_offset(sr, sc, srows, scols, scale_layout)
                                       : sr * scols + sc;
@@ -702,6 +793,9 @@ int orc_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_la
       float out;
       if (format == ORC_FMT_MXFP4) {
         out = orc_e2m1_value(code) * pow2f_exact((int)s - 127);
+      } else if (fp6) {
+        out = orc_fp6_value(code, format == ORC_FMT_MXFP6_E2M3 ? ORC_FP6_E2M3 : ORC_FP6_E3M2) *
+              pow2f_exact((int)s - 127);
       } else {
         float S = orc_e4m3_value((uint8_t)(s & 0x7F));
         if (format == ORC_FMT_IF4 && (s & 0x80)) {
