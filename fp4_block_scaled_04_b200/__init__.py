@@ -13,6 +13,7 @@ Formats and layouts (see the header for the arithmetic):
   2D     NVFP4 with one scale per 16x16 tile (W and W^T codes)
   RHT    random Hadamard transform along tokens + NVFP4 (SR or RNE) of dY^T
   IF4    per-block FP4 / INT4 choice, flag in bit 7 of the scale byte
+  MXFP6  FP6 (E2M3 or E3M2) codes, four per three bytes + E8M0 scale per 32
 """
 from __future__ import annotations
 
@@ -30,14 +31,16 @@ __all__ = [
     "fp4q_amax", "fp4q_quantize_nvfp4", "fp4q_quantize_mxfp4", "fp4q_quantize_2d",
     "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
     "fp4q_quantize_nvfp4_noalloc", "fp4q_quantize_nvint4", "fp4q_quantize_four_over_six",
-    "fp4q_quantize_backward",
+    "fp4q_quantize_backward", "fp4q_quantize_mxfp6", "FMT_MXFP6_E2M3", "FMT_MXFP6_E3M2",
+    "FP6_E2M3", "FP6_E3M2",
 ]
 
 ROWWISE, COLWISE = 1, 2
 RNE, SR = 0, 1
 SCALE_LINEAR, SCALE_SWIZZLED = 0, 1
 E8M0_RNE, E8M0_CEIL, E8M0_OCP_FLOOR = 0, 1, 2
-FMT_NVFP4, FMT_MXFP4, FMT_IF4 = 0, 1, 2
+FMT_NVFP4, FMT_MXFP4, FMT_IF4, FMT_MXFP6_E2M3, FMT_MXFP6_E3M2 = 0, 1, 2, 3, 4
+FP6_E2M3, FP6_E3M2 = 0, 1
 _BF16, _FP32 = 0, 1
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -89,6 +92,7 @@ _SIGNATURES = {
                                     _P, _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "fp4q_quantize_four_over_six": (_I, [_P, _I, _I64, _I64, _I64, _U, _P, _P, _P, _P, _P, _P,
                                          _I, _P, _SZ, _P]),
+    "fp4q_quantize_mxfp6": (_I, [_P, _I, _I64, _I64, _I64, _I, _I, _P, _P, _I, _P]),
 }
 
 
@@ -252,6 +256,20 @@ def fp4q_quantize_mxfp4(x: torch.Tensor, layouts: int = ROWWISE, e8m0_mode: int 
     return out
 
 
+def fp4q_quantize_mxfp6(x: torch.Tensor, fp6_format: int = FP6_E2M3, e8m0_mode: int = E8M0_RNE,
+                        scale_layout: int = SCALE_LINEAR, out: dict | None = None) -> dict:
+    """MXFP6 1x32 row-wise; returns {'q': [rows, cols*3/4] bytes, 'sf'}."""
+    rows, cols, ld = _matrix(x)
+    dev = x.device
+    if out is None:
+        out = {"q": _u8((rows, cols * 3 // 4), dev),
+               "sf": _u8(fp4q_scale_bytes(rows, cols, 32, scale_layout), dev)}
+    _check("fp4q_quantize_mxfp6", lib().fp4q_quantize_mxfp6(
+        _ptr(x), _dtype(x), rows, cols, ld, fp6_format, e8m0_mode, _ptr(out["q"]),
+        _ptr(out["sf"]), scale_layout, _stream(dev)))
+    return out
+
+
 def fp4q_quantize_2d(w: torch.Tensor, amax: torch.Tensor | None = None, with_1x16: bool = False,
                      scale_layout: int = SCALE_LINEAR, emit_w: bool = True,
                      emit_wt: bool = True, out: dict | None = None) -> dict:
@@ -399,7 +417,8 @@ def fp4q_dequantize(fmt: int, q: torch.Tensor, sf: torch.Tensor, rows: int, cols
                     tensor_scale: torch.Tensor | None = None, scale_layout: int = SCALE_LINEAR,
                     out_dtype: torch.dtype = torch.float32,
                     out: torch.Tensor | None = None) -> torch.Tensor:
-    """Packed codes [rows, cols/2] + scales -> [rows, cols] in out_dtype (fp32 or bf16)."""
+    """Packed codes ([rows, cols/2], or [rows, cols*3/4] for MXFP6) + scales ->
+    [rows, cols] in out_dtype (fp32 or bf16)."""
     if not q.is_cuda:
         raise ValueError("q must be a CUDA tensor")
     y = torch.empty((rows, cols), dtype=out_dtype, device=q.device) if out is None else out

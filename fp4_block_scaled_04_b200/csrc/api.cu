@@ -479,28 +479,54 @@ fp4q_status fp4q_quantize_four_over_six(const void *x, int dtype, int64_t rows, 
                                           q_row, sf_row, q_col, sf_col, scale_layout, L));
 }
 
+fp4q_status fp4q_quantize_mxfp6(const void *x, int dtype, int64_t rows, int64_t cols,
+                                int64_t ld, int fp6_format, int e8m0_mode, uint8_t *q,
+                                uint8_t *sf, int scale_layout, void *stream) {
+  FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
+  if (fp6_format != FP4Q_FP6_E2M3 && fp6_format != FP4Q_FP6_E3M2) return FP4Q_ERR_INVALID_ARG;
+  if (e8m0_mode < FP4Q_E8M0_RNE || e8m0_mode > FP4Q_E8M0_OCP_FLOOR) return FP4Q_ERR_INVALID_ARG;
+  if (!valid_layout(scale_layout)) return FP4Q_ERR_INVALID_ARG;
+  if (cols % 32 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
+  FP4Q_TRY(check_swizzle(scale_layout, rows, cols / 32));
+  if (rows == 0 || cols == 0) return FP4Q_OK;
+  if (!q || !sf) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned16(q)) return FP4Q_ERR_MISALIGNED;
+  Launch L;
+  FP4Q_TRY(bind_device(x, stream, &L));
+  FP4Q_TRY(check_dev(q, false));
+  FP4Q_TRY(check_dev(sf, false));
+  return cuda_status(
+      launch_mxfp6(x, dtype, rows, cols, ld, fp6_format, e8m0_mode, q, sf, scale_layout, L));
+}
+
 fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,
                             int block_rows, int block_cols, const float *tensor_scale,
                             int64_t rows, int64_t cols, void *y, int y_dtype, void *stream) {
-  if (format < FP4Q_FMT_NVFP4 || format > FP4Q_FMT_IF4) return FP4Q_ERR_INVALID_ARG;
+  if (format < FP4Q_FMT_NVFP4 || format > FP4Q_FMT_MXFP6_E3M2) return FP4Q_ERR_INVALID_ARG;
+  const bool fp6 = format == FP4Q_FMT_MXFP6_E2M3 || format == FP4Q_FMT_MXFP6_E3M2;
+  const bool pow2 = fp6 || format == FP4Q_FMT_MXFP4;   // E8M0 scales, no tensor scale
   if (!valid_layout(scale_layout) || !valid_dtype(y_dtype)) return FP4Q_ERR_INVALID_ARG;
   if (rows < 0 || cols < 0) return FP4Q_ERR_INVALID_ARG;
   const bool shape_ok =
-      (format == FP4Q_FMT_MXFP4 && block_rows == 1 && block_cols == 32) ||
+      (pow2 && block_rows == 1 && block_cols == 32) ||
       (format == FP4Q_FMT_IF4 && block_rows == 1 && block_cols == 16) ||
       (format == FP4Q_FMT_NVFP4 && block_cols == 16 && (block_rows == 1 || block_rows == 16));
   if (!shape_ok) return FP4Q_ERR_INVALID_ARG;
   if (cols % block_cols != 0 || rows % block_rows != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
   if (rows == 0 || cols == 0) return FP4Q_OK;
   if (!q || !sf || !y) return FP4Q_ERR_INVALID_ARG;
-  if (format != FP4Q_FMT_MXFP4 && !tensor_scale) return FP4Q_ERR_INVALID_ARG;
+  if (!pow2 && !tensor_scale) return FP4Q_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(y)) return FP4Q_ERR_MISALIGNED;
   if (block_rows == 1) FP4Q_TRY(check_swizzle(scale_layout, rows, cols / block_cols));
   Launch L;
   FP4Q_TRY(bind_device(q, stream, &L));
   FP4Q_TRY(check_dev(sf, false));
   FP4Q_TRY(check_dev(y, false));
-  FP4Q_TRY(check_dev(format != FP4Q_FMT_MXFP4 ? tensor_scale : nullptr, true));
+  FP4Q_TRY(check_dev(pow2 ? nullptr : tensor_scale, true));
+  if (fp6)
+    return cuda_status(launch_mxfp6_dequant(
+        q, sf, scale_layout, rows, cols,
+        format == FP4Q_FMT_MXFP6_E2M3 ? FP4Q_FP6_E2M3 : FP4Q_FP6_E3M2, y, y_dtype, L));
   return cuda_status(launch_dequant(format, q, sf, scale_layout, block_rows, block_cols,
                                     tensor_scale, rows, cols, y, y_dtype, L));
 }

@@ -214,6 +214,43 @@ __device__ __forceinline__ int e8m0_exponent(float m, int mode) {
   return e < -127 ? -127 : (e > 127 ? 127 : e);
 }
 
+// The exponent for an element format whose largest magnitude is qmax =
+// 1.x * 2^emax (MXFP6: 7.5 = 1.875 * 2^2 for E2M3, 28 = 1.75 * 2^4 for E3M2):
+// OCP floor(log2 m) - emax, or RN(m / qmax) rounded up (CEIL) or to the
+// nearest power of two with ties to the even biased exponent (RNE).
+__device__ __forceinline__ int e8m0_exponent_q(float m, int mode, float qmax, int emax) {
+  if (!(m > 0.0f)) return -127;
+  int e;
+  if (mode == FP4Q_E8M0_OCP_FLOOR) {
+    uint32_t b = __float_as_uint(m);
+    int E = static_cast<int>(b >> 23) - 127;
+    if ((b >> 23) == 0) E = -127 - (__clz(static_cast<int>(b)) - 9);  // subnormal
+    e = E - emax;
+  } else {
+    const float t = __fdiv_rn(m, qmax);
+    if (!(t > 0.0f)) return -127;
+    uint32_t b = __float_as_uint(t);
+    int E;
+    uint32_t frac;
+    if ((b >> 23) != 0) {
+      E = static_cast<int>(b >> 23) - 127;
+      frac = b & 0x7FFFFFu;
+    } else {
+      int p = 31 - __clz(static_cast<int>(b));
+      E = p - 149;
+      frac = (b << (23 - p)) & 0x7FFFFFu;
+    }
+    if (mode == FP4Q_E8M0_CEIL) {
+      e = (frac != 0) ? E + 1 : E;
+    } else {
+      if (frac > 0x400000u) e = E + 1;
+      else if (frac < 0x400000u) e = E;
+      else e = (((E + 127) & 1) == 0) ? E : E + 1;
+    }
+  }
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
 // Biased E8M0 exponent (e + 127, clamped to [0, 254]) of a block with
 // maximum m, as e8m0_exponent, with the common case -- a normal quotient
 // RN(m/6) -- done by carries on the bit pattern: adding 0x3FFFFF plus the

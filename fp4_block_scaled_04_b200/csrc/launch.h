@@ -55,6 +55,15 @@ cudaError_t launch_rht_backward(const void *dy, int dtype, int64_t tokens, int64
                                 uint8_t *sf_row, uint8_t *q_t, uint8_t *sf_t, int scale_layout,
                                 const Launch &L);
 
+// MXFP6 row-wise (fp6_format FP4Q_FP6_E2M3 / FP4Q_FP6_E3M2), codes packed
+// four per three bytes, and its decode
+cudaError_t launch_mxfp6(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                         int fp6_format, int e8m0_mode, uint8_t *q, uint8_t *sf,
+                         int scale_layout, const Launch &L);
+cudaError_t launch_mxfp6_dequant(const uint8_t *q, const uint8_t *sf, int scale_layout,
+                                 int64_t rows, int64_t cols, int fp6_format, void *y,
+                                 int y_dtype, const Launch &L);
+
 // int4_mode 1: IF4 (per-block choice); 2: NVINT4 (the INT4 candidate everywhere)
 cudaError_t launch_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                        const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,

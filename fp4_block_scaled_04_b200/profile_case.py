@@ -23,7 +23,7 @@ from fp4_block_scaled_04_b200 import workloads
 
 OPS = ["amax", "nvfp4_row", "nvfp4_rowcol", "mxfp4_rowcol", "2d", "rht16_sr", "rht128_sr",
        "rht16_rne", "rht128_rne", "if4", "if4_dequant", "four_over_six_rowcol", "nvint4",
-       "bwd16_sr", "bwd16_rne", "row_sr"]
+       "bwd16_sr", "bwd16_rne", "row_sr", "mxfp6_e2m3", "mxfp6_dequant"]
 
 
 def make(op: str, rows: int, cols: int, dev):
@@ -46,6 +46,14 @@ def make(op: str, rows: int, cols: int, dev):
         o = fq.fp4q_quantize_four_over_six(x, layouts=3, amax=a, scale_layout=sw)
         return lambda: fq.fp4q_quantize_four_over_six(x, layouts=3, amax=a, scale_layout=sw,
                                                       out=o)
+    if op in ("mxfp6_e2m3", "mxfp6_dequant"):
+        x = workloads.activation(rows=rows, cols=cols).to(dev)
+        o = fq.fp4q_quantize_mxfp6(x, fq.FP6_E2M3, scale_layout=sw)
+        if op == "mxfp6_e2m3":
+            return lambda: fq.fp4q_quantize_mxfp6(x, fq.FP6_E2M3, scale_layout=sw, out=o)
+        y = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+        return lambda: fq.fp4q_dequantize(fq.FMT_MXFP6_E2M3, o["q"], o["sf"], rows, cols, 1, 32,
+                                          scale_layout=sw, out=y)
     if op == "nvint4":
         x = workloads.if4_blocks(rows=rows, cols=cols).to(dev)
         a = fq.fp4q_amax(x)

@@ -78,7 +78,14 @@ typedef enum { FP4Q_BF16 = 0, FP4Q_FP32 = 1 } fp4q_dtype;
 typedef enum { FP4Q_RNE = 0, FP4Q_SR = 1 } fp4q_round;
 typedef enum { FP4Q_SCALE_LINEAR = 0, FP4Q_SCALE_SWIZZLED_128x4 = 1 } fp4q_scale_layout;
 typedef enum { FP4Q_E8M0_RNE = 0, FP4Q_E8M0_CEIL = 1, FP4Q_E8M0_OCP_FLOOR = 2 } fp4q_e8m0_mode;
-typedef enum { FP4Q_FMT_NVFP4 = 0, FP4Q_FMT_MXFP4 = 1, FP4Q_FMT_IF4 = 2 } fp4q_format;
+typedef enum {
+  FP4Q_FMT_NVFP4 = 0,
+  FP4Q_FMT_MXFP4 = 1,
+  FP4Q_FMT_IF4 = 2,
+  FP4Q_FMT_MXFP6_E2M3 = 3,   /* codes packed four per three bytes */
+  FP4Q_FMT_MXFP6_E3M2 = 4
+} fp4q_format;
+typedef enum { FP4Q_FP6_E2M3 = 0, FP4Q_FP6_E3M2 = 1 } fp4q_fp6_format;
 
 #define FP4Q_ROWWISE 1u
 #define FP4Q_COLWISE 2u
@@ -255,15 +262,45 @@ fp4q_status fp4q_quantize_four_over_six(const void *x, int dtype, int64_t rows, 
                                         uint8_t *q_col, uint8_t *sf_col, int scale_layout,
                                         void *workspace, size_t ws_bytes, void *stream);
 
+/* MXFP6 1x32, row-wise: the OCP FP6 element formats with E8M0 block scales.
+ * "FP6から考えるLLM量子化" (blog.ast.moe), "FP6で隣り合う値の間隔を見てみる":
+ * E2M3 (sign, 2 exponent bits with bias 1, 3 mantissa bits; largest 7.5)
+ * spends its bits on spacing, E3M2 (3 exponent bits with bias 3, 2 mantissa
+ * bits; largest 28) on range; both have subnormals and no Inf/NaN.  32
+ * values share one power-of-two scale as in fp4q_quantize_mxfp4, with the
+ * format's largest magnitude qmax = 1.x * 2^emax in place of 6:
+ *   FP4Q_E8M0_RNE        RN(m / qmax) to the nearest power of two (exact
+ *                        midpoints to the even biased exponent)
+ *   FP4Q_E8M0_CEIL       smallest power of two >= RN(m / qmax)
+ *   FP4Q_E8M0_OCP_FLOOR  2^(floor(log2 m) - emax), emax 2 (E2M3) or 4 (E3M2)
+ * Elements v = RN(x * 2^-e), FP6 round to nearest even with saturation, the
+ * sign copied (a negative value that rounds to zero keeps its sign bit).
+ *   fp6_format   FP4Q_FP6_E2M3 or FP4Q_FP6_E3M2
+ *   q            [rows, cols * 3/4] bytes: each group of four codes c0..c3
+ *                (consecutive columns) is the little-endian 24-bit word
+ *                c0 | c1 << 6 | c2 << 12 | c3 << 18 (the page notes that FP6
+ *                values straddle byte boundaries; this order is the
+ *                library's reading)
+ *   sf           [rows, cols/32] biased exponents e + 127, in scale_layout
+ * Shape: cols % 32 == 0; swizzled scales need rows % 128 == 0 and
+ * (cols/32) % 4 == 0.  x, q 16-byte aligned; ld * element size % 16 == 0.
+ * fp4q_dequantize(FP4Q_FMT_MXFP6_E2M3 / _E3M2, ..., 1, 32, NULL, ...) decodes
+ * it.  All buffers are the caller's; nothing is allocated. */
+fp4q_status fp4q_quantize_mxfp6(const void *x, int dtype, int64_t rows, int64_t cols,
+                                int64_t ld, int fp6_format, int e8m0_mode, uint8_t *q,
+                                uint8_t *sf, int scale_layout, void *stream);
+
 /* Dequantization of packed codes [rows, cols/2] back to y [rows, cols]
  * (FP32 or BF16 = RNE of the FP32 value), Ultralytics glossary "FP4の仕組み"
  * (grid value * sign * scale):
  *   NVFP4  y = RN(RN(g * S) * s_dec)           block 1x16 or 16x16
  *   IF4    INT4 blocks (scale bit 7): y = RN(RN(RN(k * RN(6/7)) * S) * s_dec)
  *   MXFP4  y = g * 2^(scale - 127)             block 1x32
+ *   MXFP6  y = RN(g * 2^(scale - 127))         block 1x32; q is [rows,
+ *          cols * 3/4] bytes packed as fp4q_quantize_mxfp6 writes them
  *   block_rows x block_cols: 1x16 (NVFP4, IF4), 16x16 (NVFP4 2D tiles; then
- *   sf is the linear [rows/16, cols/16] tile matrix), 1x32 (MXFP4).
- *   tensor_scale: device float s_dec (NVFP4 / IF4), ignored for MXFP4.
+ *   sf is the linear [rows/16, cols/16] tile matrix), 1x32 (MXFP4, MXFP6).
+ *   tensor_scale: device float s_dec (NVFP4 / IF4), ignored for MXFP4/6.
  *   Column-wise outputs are dequantized as the [cols, rows] matrices they are.
  * Shape: cols % block_cols == 0, rows % block_rows == 0. */
 fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,

@@ -30,7 +30,8 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["fp4q_amax", "fp4q_quantize_nvfp4", "fp4q_quantize_mxfp4", "fp4q_quantize_2d",
               "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
-              "fp4q_scale_bytes", "fp4q_workspace_bytes", "fp4q_status_string", "fp4q_version"]:
+              "fp4q_scale_bytes", "fp4q_workspace_bytes", "fp4q_status_string", "fp4q_version",
+              "fp4q_quantize_mxfp6"]:
         assert n in names
 
 
@@ -132,6 +133,26 @@ def test_host_side_argument_checks_of_the_added_calls(L):
     assert bw(layout=1, tokens=128, cols=64) == 2   # swizzled dY^T scales need cols % 128
     assert L.fp4q_quantize_nvfp4_noalloc(FAKE, 0, 32, 24, 24, 1, 0, 0, FAKE, FAKE, FAKE, FAKE,
                                          None, None, 0, None) == 2
+    # MXFP6: cols % 32, the FP6 format and E8M0 mode, 16-byte aligned codes
+    m6 = lambda **kw: L.fp4q_quantize_mxfp6(
+        kw.get("x", FAKE), kw.get("dtype", 0), kw.get("rows", 32), kw.get("cols", 64),
+        kw.get("ld", 64), kw.get("fmt", 0), kw.get("mode", 0), kw.get("q", FAKE), FAKE,
+        kw.get("layout", 0), None)
+    assert m6(fmt=2) == 1 and m6(fmt=-1) == 1
+    assert m6(mode=3) == 1
+    assert m6(layout=2) == 1
+    assert m6(cols=48, ld=48) == 2
+    assert m6(layout=1) == 2                        # swizzle needs rows % 128
+    assert m6(rows=128, cols=96, ld=96, layout=1) == 2   # and (cols/32) % 4
+    assert m6(ld=60) == 1                           # ld < cols
+    assert m6(x=ctypes.c_void_p(0x7F0000000008)) == 3
+    assert m6(q=ctypes.c_void_p(0x7F0000000008)) == 3
+    assert m6(q=None) == 1
+    assert m6(rows=0) == 0                          # nothing to do, nothing touched
+    # dequantize: MXFP6 formats take 1x32 blocks and no tensor scale
+    assert L.fp4q_dequantize(3, FAKE, FAKE, 0, 1, 16, None, 16, 64, FAKE, 1, None) == 1
+    assert L.fp4q_dequantize(4, FAKE, FAKE, 0, 1, 32, None, 16, 48, FAKE, 1, None) == 2
+    assert L.fp4q_dequantize(5, FAKE, FAKE, 0, 1, 32, None, 16, 64, FAKE, 1, None) == 1
 
 
 def test_python_binding_refuses_cpu_tensors(L):
