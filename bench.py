@@ -554,7 +554,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
-                    help="skip timing the comparison formats (four-over-six, NVINT4)")
+                    help="skip the calls outside the suite (fused backward, row-wise alone, "
+                         "four-over-six, NVINT4, MXFP6) and the consumer GEMM")
     ap.add_argument("--e2e-steps", type=int, default=None)
     args = ap.parse_args()
     if args.warmup < 3:

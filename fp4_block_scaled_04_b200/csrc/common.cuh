@@ -139,7 +139,7 @@ __device__ __forceinline__ TensorScale tensor_scale(float amax) {
 // RN(y / 6) in three instructions: Markstein's correction of RN(y * RN(1/6))
 // with an exact FMA remainder (P. Markstein, IBM J. Res. Dev. 34(1), 1990).
 // Equal to the IEEE quotient for every float y in [2^-125, 4096] (checked
-// exhaustively on the host by tests/div6_check.c); below that the quotient
+// exhaustively on the host by tests/div_check.c); below that the quotient
 // is subnormal, where callers either do not care (E4M3 rounds it to 0) or
 // use the IEEE division.
 __device__ __forceinline__ float div6(float y) {
@@ -147,6 +147,16 @@ __device__ __forceinline__ float div6(float y) {
   const float q0 = __fmul_rn(y, kInv6);
   const float r = __fmaf_rn(-q0, 6.0f, y);
   return __fmaf_rn(r, kInv6, q0);
+}
+
+// RN(y / d) by the same correction for the FP6 grid maxima d = 7.5 and 28
+// (inv_d = RN(1/d)); equal to the IEEE quotient for every float y >= 2^-122
+// (tests/div_check.c, exhaustively), the IEEE division below that.
+__device__ __forceinline__ float div_qmax(float y, float d, float inv_d) {
+  if (!(y >= 0x1p-122f)) return __fdiv_rn(y, d);
+  const float q0 = __fmul_rn(y, inv_d);
+  const float r = __fmaf_rn(-q0, d, y);
+  return __fmaf_rn(r, inv_d, q0);
 }
 
 // E4M3 code of the block scale: RN(RN(m * s_enc) / 6).  RN(m * s_enc) is at
@@ -218,7 +228,8 @@ __device__ __forceinline__ int e8m0_exponent(float m, int mode) {
 // 1.x * 2^emax (MXFP6: 7.5 = 1.875 * 2^2 for E2M3, 28 = 1.75 * 2^4 for E3M2):
 // OCP floor(log2 m) - emax, or RN(m / qmax) rounded up (CEIL) or to the
 // nearest power of two with ties to the even biased exponent (RNE).
-__device__ __forceinline__ int e8m0_exponent_q(float m, int mode, float qmax, int emax) {
+__device__ __forceinline__ int e8m0_exponent_q(float m, int mode, float qmax, float inv_qmax,
+                                               int emax) {
   if (!(m > 0.0f)) return -127;
   int e;
   if (mode == FP4Q_E8M0_OCP_FLOOR) {
@@ -227,7 +238,7 @@ __device__ __forceinline__ int e8m0_exponent_q(float m, int mode, float qmax, in
     if ((b >> 23) == 0) E = -127 - (__clz(static_cast<int>(b)) - 9);  // subnormal
     e = E - emax;
   } else {
-    const float t = __fdiv_rn(m, qmax);
+    const float t = div_qmax(m, qmax, inv_qmax);
     if (!(t > 0.0f)) return -127;
     uint32_t b = __float_as_uint(t);
     int E;

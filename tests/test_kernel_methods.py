@@ -14,26 +14,29 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 
 
 @pytest.fixture(scope="module")
-def div6_exe(tmp_path_factory):
-    exe = str(tmp_path_factory.mktemp("div6") / "div6_check")
+def div_exe(tmp_path_factory):
+    exe = str(tmp_path_factory.mktemp("div") / "div_check")
     flags = ["-O2", "-ffp-contract=off"]
     # use the hardware FMA when the host has one (fmaf is correctly rounded either way)
     probe = subprocess.run(["gcc", "-mfma", "-x", "c", "-", "-o", "/dev/null"],
                            input="int main(){return 0;}", text=True, capture_output=True)
     if probe.returncode == 0:
         flags.append("-mfma")
-    subprocess.check_call(["gcc", *flags, os.path.join(HERE, "div6_check.c"), "-o", exe, "-lm"])
+    subprocess.check_call(["gcc", *flags, os.path.join(HERE, "div_check.c"), "-o", exe, "-lm"])
     return exe
 
 
-def test_division_by_six_is_the_ieee_quotient(div6_exe):
-    """Markstein's corrected product equals RN(y/6) for every float y >= 2^-125
-    (checked over all finite non-negative bit patterns); below that the
-    quotient is subnormal and both round to E4M3 code 0."""
-    out = subprocess.run([div6_exe, "0", "0x7F800000"], capture_output=True, text=True,
+@pytest.mark.parametrize("d,floor", [("6", -125), ("7.5", -122), ("28", -122)])
+def test_division_by_the_grid_maximum_is_the_ieee_quotient(div_exe, d, floor):
+    """Markstein's corrected product equals RN(y/d) for every float y >= 2^floor
+    (checked over all finite non-negative bit patterns), for the FP4 maximum 6
+    and the FP6 maxima 7.5 (E2M3) and 28 (E3M2).  Below 2^-125 the quotient
+    by 6 is subnormal and rounds to E4M3 code 0; the FP6 kernels divide with
+    IEEE division below 2^-122."""
+    out = subprocess.run([div_exe, "0", "0x7F800000", d], capture_output=True, text=True,
                          check=True).stdout.split()
     bad, worst = int(out[0]), float(out[1])
-    assert worst < 2.0 ** -125, worst
+    assert worst < 2.0 ** floor, worst
     assert bad < (1 << 24)                  # only the subnormal-quotient range differs
 
 
