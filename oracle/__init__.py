@@ -431,3 +431,25 @@ def dequantize(fmt: int, q: np.ndarray, sf: np.ndarray, rows: int, cols: int,
 def glossary_mae(x: np.ndarray, block: int) -> float:
     x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1)
     return float(lib().orc_glossary_mae(_ptr(x), x.size, block))
+
+
+def gemm_block_scaled(qa: np.ndarray, sfa: np.ndarray, qb: np.ndarray, sfb: np.ndarray,
+                      M: int, N: int, K: int, alpha: float = 1.0, fmt: int = FMT_NVFP4,
+                      scale_layout: int = SCALE_SWIZZLED) -> np.ndarray:
+    """The product a block-scaled FP4 GEMM computes from quantized operands.
+
+    Qiita note on NVFP4 training: the quantized operands feed FP4 GEMMs (Fprop
+    X W^T; Wgrad dY^T X from the column-wise copies), each block's codes
+    multiplied by its block scale, the two tensor scales applied to the result.
+    Here: A = dequantize(qa, sfa) [M, K] and B = dequantize(qb, sfb) [N, K]
+    with the block scales only (tensor scale 1, which makes every element the
+    exact product g * S), then C = alpha * (A B^T), the contraction and the
+    final product taken in float64 (a library matmul).  alpha carries the
+    product of the two tensor scales.  Returns float64 [M, N].
+    """
+    blk = 16 if fmt == FMT_NVFP4 else 32
+    a = dequantize(fmt, qa, sfa, M, K, 1, blk, s_dec=1.0 if fmt != FMT_MXFP4 else None,
+                   scale_layout=scale_layout)
+    b = dequantize(fmt, qb, sfb, N, K, 1, blk, s_dec=1.0 if fmt != FMT_MXFP4 else None,
+                   scale_layout=scale_layout)
+    return (a.astype(np.float64) @ b.astype(np.float64).T) * float(alpha)
