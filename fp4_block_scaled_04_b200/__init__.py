@@ -14,6 +14,7 @@ Formats and layouts (see the header for the arithmetic):
   RHT    random Hadamard transform along tokens + NVFP4 (SR or RNE) of dY^T
   IF4    per-block FP4 / INT4 choice, flag in bit 7 of the scale byte
   MXFP6  FP6 (E2M3 or E3M2) codes, four per three bytes + E8M0 scale per 32
+  GEMM   C = s_a s_b (A B^T) from NVFP4 operands on the tensor cores
 """
 from __future__ import annotations
 
@@ -32,7 +33,7 @@ __all__ = [
     "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
     "fp4q_quantize_nvfp4_noalloc", "fp4q_quantize_nvint4", "fp4q_quantize_four_over_six",
     "fp4q_quantize_backward", "fp4q_quantize_mxfp6", "FMT_MXFP6_E2M3", "FMT_MXFP6_E3M2",
-    "FP6_E2M3", "FP6_E3M2",
+    "FP6_E2M3", "FP6_E3M2", "fp4q_gemm_nvfp4",
 ]
 
 ROWWISE, COLWISE = 1, 2
@@ -93,6 +94,7 @@ _SIGNATURES = {
     "fp4q_quantize_four_over_six": (_I, [_P, _I, _I64, _I64, _I64, _U, _P, _P, _P, _P, _P, _P,
                                          _I, _P, _SZ, _P]),
     "fp4q_quantize_mxfp6": (_I, [_P, _I, _I64, _I64, _I64, _I, _I, _P, _P, _I, _P]),
+    "fp4q_gemm_nvfp4": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P, _P]),
 }
 
 
@@ -268,6 +270,24 @@ def fp4q_quantize_mxfp6(x: torch.Tensor, fp6_format: int = FP6_E2M3, e8m0_mode: 
         _ptr(x), _dtype(x), rows, cols, ld, fp6_format, e8m0_mode, _ptr(out["q"]),
         _ptr(out["sf"]), scale_layout, _stream(dev)))
     return out
+
+
+def fp4q_gemm_nvfp4(qa: torch.Tensor, sfa: torch.Tensor, qb: torch.Tensor, sfb: torch.Tensor,
+                    K: int, tensor_scale_a: torch.Tensor | None = None,
+                    tensor_scale_b: torch.Tensor | None = None,
+                    out_dtype: torch.dtype = torch.float32, out: torch.Tensor | None = None,
+                    status: torch.Tensor | None = None) -> torch.Tensor:
+    """C [M, N] = s_a s_b (A B^T) from NVFP4 operands: codes qa [M, K/2], qb
+    [N, K/2] and their swizzled 1x16 scales (as fp4q_quantize_nvfp4 writes them)."""
+    if not qa.is_cuda:
+        raise ValueError("qa must be a CUDA tensor")
+    M, N = qa.shape[0], qb.shape[0]
+    c = torch.empty((M, N), dtype=out_dtype, device=qa.device) if out is None else out
+    cdt = _BF16 if c.dtype == torch.bfloat16 else _FP32
+    _check("fp4q_gemm_nvfp4", lib().fp4q_gemm_nvfp4(
+        _ptr(qa), _ptr(sfa), _ptr(tensor_scale_a), _ptr(qb), _ptr(sfb), _ptr(tensor_scale_b),
+        M, N, K, _ptr(c), cdt, c.stride(0) if M > 1 else N, _ptr(status), _stream(qa.device)))
+    return c
 
 
 def fp4q_quantize_2d(w: torch.Tensor, amax: torch.Tensor | None = None, with_1x16: bool = False,

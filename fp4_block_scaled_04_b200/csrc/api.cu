@@ -499,6 +499,41 @@ fp4q_status fp4q_quantize_mxfp6(const void *x, int dtype, int64_t rows, int64_t 
       launch_mxfp6(x, dtype, rows, cols, ld, fp6_format, e8m0_mode, q, sf, scale_layout, L));
 }
 
+fp4q_status fp4q_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *tensor_scale_a,
+                            const uint8_t *qb, const uint8_t *sfb, const float *tensor_scale_b,
+                            int64_t M, int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
+                            int *status, void *stream) {
+  if (!valid_dtype(c_dtype)) return FP4Q_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4Q_ERR_INVALID_ARG;
+  if (M % 128 != 0 || N % 128 != 0 || K % 256 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
+  if (K > (int64_t{1} << 30) || M / 128 > 65535 || N / 128 > (int64_t{1} << 30))
+    return FP4Q_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return FP4Q_OK;
+  if (!c) return FP4Q_ERR_INVALID_ARG;
+  const int64_t esz = elem_size(c_dtype);
+  if (!aligned16(c) || (ldc * esz) % 16 != 0) return FP4Q_ERR_MISALIGNED;
+  if (K > 0) {
+    if (!qa || !sfa || !qb || !sfb) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned16(qa) || !aligned16(qb) || !aligned16(sfa) || !aligned16(sfb))
+      return FP4Q_ERR_MISALIGNED;
+  }
+  Launch L;
+  FP4Q_TRY(bind_device(c, stream, &L));
+  if (K == 0)   // an empty sum
+    return cuda_status(cudaMemset2DAsync(c, static_cast<size_t>(ldc * esz), 0,
+                                         static_cast<size_t>(N * esz), static_cast<size_t>(M),
+                                         L.stream));
+  FP4Q_TRY(check_dev(qa, false));
+  FP4Q_TRY(check_dev(sfa, false));
+  FP4Q_TRY(check_dev(qb, false));
+  FP4Q_TRY(check_dev(sfb, false));
+  FP4Q_TRY(check_dev(tensor_scale_a, true));
+  FP4Q_TRY(check_dev(tensor_scale_b, true));
+  FP4Q_TRY(check_dev(status, true));
+  return cuda_status(launch_gemm_nvfp4(qa, sfa, tensor_scale_a, qb, sfb, tensor_scale_b, M, N, K,
+                                       c, c_dtype, ldc, status, L));
+}
+
 fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,
                             int block_rows, int block_cols, const float *tensor_scale,
                             int64_t rows, int64_t cols, void *y, int y_dtype, void *stream) {

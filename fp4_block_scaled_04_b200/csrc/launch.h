@@ -64,6 +64,13 @@ cudaError_t launch_mxfp6_dequant(const uint8_t *q, const uint8_t *sf, int scale_
                                  int64_t rows, int64_t cols, int fp6_format, void *y,
                                  int y_dtype, const Launch &L);
 
+// C[M, N] = s_a s_b (A B^T) from NVFP4 operands (codes [rows, K/2], swizzled
+// 1x16 scales) on the tensor cores; status (may be NULL) <- 1 if a wait ran out
+cudaError_t launch_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *s_a,
+                              const uint8_t *qb, const uint8_t *sfb, const float *s_b, int64_t M,
+                              int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
+                              int *status, const Launch &L);
+
 // int4_mode 1: IF4 (per-block choice); 2: NVINT4 (the INT4 candidate everywhere)
 cudaError_t launch_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                        const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,

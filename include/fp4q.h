@@ -290,6 +290,37 @@ fp4q_status fp4q_quantize_mxfp6(const void *x, int dtype, int64_t rows, int64_t 
                                 int64_t ld, int fp6_format, int e8m0_mode, uint8_t *q,
                                 uint8_t *sf, int scale_layout, void *stream);
 
+/* Block-scaled NVFP4 GEMM on the tensor cores: the consumer of the
+ * quantized operands.  Qiita note on NVFP4 training ("Blockwise", "誤差逆伝播と
+ * 転置"): Fprop multiplies X by W^T with both in NVFP4, Wgrad multiplies dY^T
+ * by X^T from the column-wise copies; every 16-value block's E2M1 codes are
+ * multiplied by its E4M3 block scale and the FP32 tensor scales multiply the
+ * product.  With A = dequantize(qa, sfa) and B = dequantize(qb, sfb) taken
+ * with the block scales only:
+ *   C[m, n] = RN(acc[m, n] * RN(s_a * s_b)),  acc = A B^T accumulated in FP32
+ * by tcgen05.mma kind::mxf4nvf4 (the order of the FP32 additions is the
+ * hardware's; the result is within FP32 accumulation error of the exact
+ * product, not bit-reproducible against a CPU sum).
+ *   qa, sfa      A codes [M, K/2] (row-wise, K-major) and its 1x16 scales in
+ *                FP4Q_SCALE_SWIZZLED_128x4, as fp4q_quantize_nvfp4 writes them
+ *                (a column-wise output is the row-wise layout of the transpose)
+ *   qb, sfb      B codes [N, K/2] and scales, the same way
+ *   tensor_scale_a, tensor_scale_b  device floats s_dec of A and B, or NULL
+ *                for 1
+ *   c, c_dtype, ldc  output [M, ldc] row-major, FP32 or BF16 (RNE of the FP32
+ *                value); ldc >= N
+ *   status       device int or NULL: set to 1 if a wait inside the kernel ran
+ *                out (about a second; the tile is then not written).  The
+ *                library never clears it
+ * Shape: M % 128 == 0, N % 128 == 0, K % 256 == 0 (one 128x128 output tile
+ * per CTA, 256 values of K per pipeline stage).  All pointers 16-byte
+ * aligned, ldc * element size % 16 == 0.  K == 0 writes zeros.  Device memory
+ * is the caller's; nothing is allocated. */
+fp4q_status fp4q_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *tensor_scale_a,
+                            const uint8_t *qb, const uint8_t *sfb, const float *tensor_scale_b,
+                            int64_t M, int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
+                            int *status, void *stream);
+
 /* Dequantization of packed codes [rows, cols/2] back to y [rows, cols]
  * (FP32 or BF16 = RNE of the FP32 value), Ultralytics glossary "FP4の仕組み"
  * (grid value * sign * scale):

@@ -31,7 +31,7 @@ def test_header_declares_the_entry_points():
     for n in ["fp4q_amax", "fp4q_quantize_nvfp4", "fp4q_quantize_mxfp4", "fp4q_quantize_2d",
               "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
               "fp4q_scale_bytes", "fp4q_workspace_bytes", "fp4q_status_string", "fp4q_version",
-              "fp4q_quantize_mxfp6"]:
+              "fp4q_quantize_mxfp6", "fp4q_gemm_nvfp4"]:
         assert n in names
 
 
@@ -149,6 +149,18 @@ def test_host_side_argument_checks_of_the_added_calls(L):
     assert m6(q=ctypes.c_void_p(0x7F0000000008)) == 3
     assert m6(q=None) == 1
     assert m6(rows=0) == 0                          # nothing to do, nothing touched
+    # GEMM: 128x128 output tiles, K % 256, aligned operands
+    gm = lambda **kw: L.fp4q_gemm_nvfp4(
+        kw.get("qa", FAKE), FAKE, None, FAKE, FAKE, None, kw.get("M", 128), kw.get("N", 128),
+        kw.get("K", 256), kw.get("c", FAKE), kw.get("dt", 1), kw.get("ldc", 128), None, None)
+    assert gm(dt=3) == 1
+    assert gm(ldc=64) == 1
+    assert gm(M=96) == 2 and gm(N=200, ldc=200) == 2 and gm(K=128) == 2
+    assert gm(c=ctypes.c_void_p(0x7F0000000008)) == 3
+    assert gm(ldc=130) == 3                         # row stride not 16-byte aligned (FP32)
+    assert gm(qa=None) == 1
+    assert gm(qa=ctypes.c_void_p(0x7F0000000004)) == 3
+    assert gm(M=0) == 0
     # dequantize: MXFP6 formats take 1x32 blocks and no tensor scale
     assert L.fp4q_dequantize(3, FAKE, FAKE, 0, 1, 16, None, 16, 64, FAKE, 1, None) == 1
     assert L.fp4q_dequantize(4, FAKE, FAKE, 0, 1, 32, None, 16, 48, FAKE, 1, None) == 2

@@ -1,0 +1,143 @@
+"""GPU parity of the tensor-core NVFP4 GEMM (fp4q_gemm_nvfp4) against the
+oracle's gemm_block_scaled, through the C ABI.
+
+Qiita note on NVFP4 training: the quantized operands feed the FP4 GEMMs
+(Fprop X W^T from the row-wise copies, Wgrad dY^T X from the column-wise
+ones).  The GEMM accumulates in FP32 in the tensor core's own order, so the
+comparison is against the exact product of the dequantized operands with
+the FP32 accumulation bound: every product of two dequantized values is
+exact, only the K additions round, |C - exact| <= (K + 2) 2^-22 (|A| |B|^T)
+(four times the textbook bound, leaving room for the hardware's order),
+plus one rounding for the tensor-scale product and one for the output type.
+A misplaced code nibble, scale byte or tile is off by the size of the values.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fp4_block_scaled_04_b200 as fq
+
+from test_gpu_parity import DEV, host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    fq.lib()
+
+
+def random_operand(rows, K, seed):
+    rng = np.random.default_rng(seed)
+    q = rng.integers(0, 256, (rows, K // 2), dtype=np.uint8)
+    sf = rng.integers(0x20, 0x50, rows * K // 16, dtype=np.uint8)   # E4M3 2^-4 .. 2^3
+    return q, sf
+
+
+def check(orc, qa, sfa, qb, sfb, M, N, K, c, alpha=1.0, out_bits=24):
+    exact = orc.gemm_block_scaled(qa, sfa, qb, sfb, M, N, K)
+    a = orc.dequantize(orc.FMT_NVFP4, qa, sfa, M, K, 1, 16, s_dec=1.0,
+                       scale_layout=orc.SCALE_SWIZZLED).astype(np.float64)
+    b = orc.dequantize(orc.FMT_NVFP4, qb, sfb, N, K, 1, 16, s_dec=1.0,
+                       scale_layout=orc.SCALE_SWIZZLED).astype(np.float64)
+    mag = np.abs(a) @ np.abs(b).T
+    bound = alpha * (K + 2) * 2.0 ** -22 * mag + abs(alpha * exact) * (2.0 ** -23 + 2.0 ** -out_bits)
+    bound += 1e-30
+    err = np.abs(c.astype(np.float64) - alpha * exact)
+    worst = float(np.max(err / bound))
+    assert worst <= 1.0, f"GEMM differs from the exact product by {worst:.3g} x the bound"
+    assert np.linalg.norm(exact) > 0
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 128, 512), (128, 384, 1024),
+                                   (384, 256, 768), (256, 256, 4096)])
+def test_gemm_random_codes_and_scales(orc, M, N, K):
+    qa, sfa = random_operand(M, K, 1)
+    qb, sfb = random_operand(N, K, 2)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    c = fq.fp4q_gemm_nvfp4(torch.from_numpy(qa).to(DEV), torch.from_numpy(sfa).to(DEV),
+                           torch.from_numpy(qb).to(DEV), torch.from_numpy(sfb).to(DEV), K,
+                           status=status)
+    assert int(status.item()) == 0
+    check(orc, qa, sfa, qb, sfb, M, N, K, host(c))
+
+
+def test_gemm_one_hot_selects_columns(orc):
+    """B rows one-hot at 1.0: C is a column selection of dequantized A, which
+    every FP32 order computes exactly."""
+    M, N, K = 256, 128, 512
+    qa, sfa = random_operand(M, K, 3)
+    rng = np.random.default_rng(4)
+    kn = rng.permutation(K)[:N]
+    cb = np.zeros((N, K), np.uint8)
+    cb[np.arange(N), kn] = 0x2
+    qb = (cb[:, 0::2] | (cb[:, 1::2] << 4)).astype(np.uint8)
+    sfb = np.full(N * K // 16, 0x38, np.uint8)
+    c = fq.fp4q_gemm_nvfp4(torch.from_numpy(qa).to(DEV), torch.from_numpy(sfa).to(DEV),
+                           torch.from_numpy(qb).to(DEV), torch.from_numpy(sfb).to(DEV), K)
+    want = orc.gemm_block_scaled(qa, sfa, qb, sfb, M, N, K)
+    np.testing.assert_array_equal(host(c).astype(np.float64), want)
+
+
+def quantized(x):
+    o = fq.fp4q_quantize_nvfp4(x, layouts=fq.ROWWISE | fq.COLWISE, scale_layout=fq.SCALE_SWIZZLED)
+    return o
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_fprop_from_quantized_activations_and_weights(orc, out_dtype):
+    """Fprop: X [M, K] and W [N, K] through fp4q_quantize_nvfp4 (row-wise,
+    swizzled scales), then C = s_x s_w (X_q W_q^T)."""
+    M, N, K = 256, 384, 1024
+    g = torch.Generator().manual_seed(11)
+    x = (torch.randn(M, K, generator=g) * 3).to(torch.bfloat16).to(DEV)
+    w = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16).to(DEV)
+    ox, ow = quantized(x), quantized(w)
+    c = fq.fp4q_gemm_nvfp4(ox["q_row"], ox["sf_row"], ow["q_row"], ow["sf_row"], K,
+                           tensor_scale_a=ox["s_dec"], tensor_scale_b=ow["s_dec"],
+                           out_dtype=out_dtype)
+    alpha = float(np.float32(ox["s_dec"].item()) * np.float32(ow["s_dec"].item()))
+    check(orc, host(ox["q_row"]), host(ox["sf_row"]), host(ow["q_row"]), host(ow["sf_row"]),
+          M, N, K, host(c.float()), alpha=alpha, out_bits=24 if out_dtype == torch.float32 else 8)
+
+
+def test_wgrad_from_column_wise_copies(orc):
+    """Wgrad = dY^T X: both operands are the column-wise outputs (rows run
+    along tokens, the contraction dimension)."""
+    T, Co, Ci = 512, 128, 256
+    g = torch.Generator().manual_seed(12)
+    dy = (torch.randn(T, Co, generator=g) * 1e-3).to(torch.bfloat16).to(DEV)
+    x = torch.randn(T, Ci, generator=g).to(torch.bfloat16).to(DEV)
+    od, ox = quantized(dy), quantized(x)
+    c = fq.fp4q_gemm_nvfp4(od["q_col"], od["sf_col"], ox["q_col"], ox["sf_col"], T,
+                           tensor_scale_a=od["s_dec"], tensor_scale_b=ox["s_dec"])
+    alpha = float(np.float32(od["s_dec"].item()) * np.float32(ox["s_dec"].item()))
+    check(orc, host(od["q_col"]), host(od["sf_col"]), host(ox["q_col"]), host(ox["sf_col"]),
+          Co, Ci, T, host(c), alpha=alpha)
+
+
+def test_gemm_strided_output_and_empty_k():
+    M, N, K = 128, 128, 256
+    qa, sfa = random_operand(M, K, 5)
+    qb, sfb = random_operand(N, K, 6)
+    big = torch.full((M, N + 64), 7.0, device=DEV)
+    view = big[:, :N]
+    fq.fp4q_gemm_nvfp4(torch.from_numpy(qa).to(DEV), torch.from_numpy(sfa).to(DEV),
+                       torch.from_numpy(qb).to(DEV), torch.from_numpy(sfb).to(DEV), K, out=view)
+    assert torch.all(big[:, N:] == 7.0)                 # nothing written past ldc's row
+    z = torch.full((M, N), 5.0, device=DEV)
+    e = torch.empty((M, 0), dtype=torch.uint8, device=DEV)
+    fq.fp4q_gemm_nvfp4(e, e, torch.empty((N, 0), dtype=torch.uint8, device=DEV), e, 0, out=z)
+    assert torch.all(z == 0)
+
+
+def test_gemm_rejects_ragged_shapes():
+    q = torch.zeros((128, 64), dtype=torch.uint8, device=DEV)
+    s = torch.zeros(128 * 8, dtype=torch.uint8, device=DEV)
+    with pytest.raises(fq.Fp4qError):
+        fq.fp4q_gemm_nvfp4(q, s, q, s, 128)             # K % 256
+    q2 = torch.zeros((96, 128), dtype=torch.uint8, device=DEV)
+    with pytest.raises(fq.Fp4qError):
+        fq.fp4q_gemm_nvfp4(q2, s, q, s, 256)            # M % 128
