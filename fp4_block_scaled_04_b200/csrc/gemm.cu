@@ -12,50 +12,69 @@
 //   C[m, n] = RN(acc[m, n] * RN(s_a * s_b)),
 //   acc[m, n] = sum_k (g_a[m,k] S_a[m,k/16]) (g_b[n,k] S_b[n,k/16])   (FP32)
 //
-// One CTA computes a 128x128 tile of C with 4 warps:
-//  - all threads stage K-tiles of 256 values (128 code bytes per row) of A
-//    and B into shared memory with cp.async, in the 128-byte-swizzled
-//    K-major layout, plus the 4 scale tiles (512 bytes each) of A and B;
-//    four stages, loads running two K-tiles ahead of the tensor core;
-//  - one thread copies the scale tiles into tensor memory (tcgen05.cp
-//    32x128b.warpx4: one 512-byte tile per 64-value K step) and issues four
-//    tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=128, K=64), accumulating
-//    in tensor memory, then tcgen05.commit to the stage's mbarrier, which
-//    tells the loaders that the stage may be refilled;
-//  - at the end every warp reads its 32 accumulator rows with tcgen05.ld
-//    and writes C (FP32 or BF16).
-// Every wait on an mbarrier is bounded (about a second of clock cycles);
-// a wait that runs out sets *status and the CTA leaves the K loop, waits
-// (bounded) for its tensor-core work, frees its tensor memory and returns.
+// One CTA computes a 128 x BN tile of C (BN = 256, or 128 when N is not a
+// multiple of 256) with 4 warps in three roles:
+//  - one thread of warp 0 is the producer: per K-tile of 256 values it
+//    loads the A and B code tiles with TMA (cp.async.bulk.tensor, 128-byte
+//    swizzle, which is the K-major layout the MMA descriptors describe) and
+//    the 2 KiB scale blocks with plain bulk copies (the 128x4 tiles of one
+//    K-tile are contiguous in the swizzled layout), all completing on the
+//    stage's "full" mbarrier; four stages;
+//  - one thread of warp 1 issues the tensor-core work: tcgen05.cp
+//    32x128b.warpx4 of each 512-byte scale tile into tensor memory (4
+//    columns per 64-value K step and 128 rows), then four tcgen05.mma
+//    kind::mxf4nvf4 block16 (M = 128, N = BN, K = 64) accumulating in
+//    tensor memory, then tcgen05.commit to the stage's "empty" mbarrier;
+//  - at the end all four warps read their 32 accumulator rows with
+//    tcgen05.ld and write C (FP32 or BF16).
+// No load uses cluster multicast.  Every mbarrier wait is bounded (about a
+// second of clock cycles); a wait that runs out sets *status, the roles stop
+// issuing, and the CTA waits (bounded) for its tensor-core work, frees its
+// tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
 namespace fp4q {
 namespace {
 
-constexpr int BM = 128, BN = 128;
+constexpr int BM = 128;
 constexpr int KTILE = 256;                       // K values per stage
 constexpr int KTB = KTILE / 2;                   // 128 code bytes per row per stage
 constexpr int STAGES = 4;
 constexpr int kThreads = 128;
-constexpr int A_BYTES = BM * KTB;                // 16384
-constexpr int B_BYTES = BN * KTB;                // 16384
 constexpr int SF_TILE = 512;                     // 128 rows x 4 scales
-constexpr int SF_BYTES = (KTILE / 64) * SF_TILE; // 2048 per operand per stage
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;   // 36864 = 36 KiB
-constexpr int BAR_BYTES = 128;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
-constexpr uint32_t TMEM_COLS = 256;              // 128 accumulator + 4 x 32 scale columns
-constexpr uint32_t SF_COL0 = 128;
+constexpr int SF_BYTES = (KTILE / 64) * SF_TILE; // 2048: one operand row tile, one K-tile
 constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at the B200's clock
 
-static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
-
-// Instruction descriptor of tcgen05.mma kind::mxf4nvf4 (block-scaled):
-// A and B E2M1 (format 1), K-major, E4M3 scales (bit 23 = 0), N = 128
-// (bits 17-22 = N/8), M = 128 (bits 24-28 = M/16), dense, K = 64.
-constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
-                            (uint32_t(BM >> 4) << 24);
+template <int BN>
+struct Tile {
+  static constexpr int A_BYTES = BM * KTB;                      // 16384
+  static constexpr int B_BYTES = BN * KTB;                      // 16384 or 32768
+  static constexpr int SFB_BYTES = (BN / 128) * SF_BYTES;       // [row tile][K step][512]
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES + SFB_BYTES;
+  static constexpr int BAR_BYTES = 128;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  // tensor memory: accumulator columns [0, BN), then per stage 16 columns of
+  // A scales and 4 * BN / 32 columns of B scales
+  static constexpr uint32_t SF_COL0 = BN;
+  static constexpr uint32_t SFB_COLS = 4 * (BN / 32);
+  static constexpr uint32_t STAGE_COLS = 16 + SFB_COLS;
+  static constexpr uint32_t COLS_USED = BN + STAGES * STAGE_COLS;
+  static constexpr uint32_t TMEM_COLS = COLS_USED <= 256 ? 256 : 512;
+  // Instruction descriptor of tcgen05.mma kind::mxf4nvf4 (block-scaled): A and
+  // B E2M1 (format 1), K-major, E4M3 scales (bit 23 = 0), N (bits 17-22 =
+  // N/8), M = 128 (bits 24-28 = M/16), dense, K = 64.
+  static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
+                                    (uint32_t(BM >> 4) << 24);
+  static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+  static_assert(COLS_USED <= 512, "tensor memory");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -116,14 +135,14 @@ __device__ __forceinline__ void tc_copy_sf(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
                : "memory");
 }
-__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t sfa,
-                                       uint32_t sfb, uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
       "[%6], p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
 }
 
@@ -145,115 +164,139 @@ __device__ __forceinline__ void tc_load32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Stage K-tile kt of this CTA's A rows, B rows and their scale tiles.
-__device__ __forceinline__ void load_stage(uint32_t st, const uint8_t *qa, const uint8_t *qb,
-                                           const uint8_t *sfa, const uint8_t *sfb, int64_t ldk,
-                                           int kt) {
-  const int tid = threadIdx.x;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {                  // 1024 16-byte pieces per operand
-    const int i = tid + kThreads * j;
-    const int r = i >> 3, c = i & 7;
-    const uint32_t so = static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
-    const int64_t go = r * ldk + static_cast<int64_t>(kt) * KTB + c * 16;
-    cp_async16(st + so, qa + go);
-    cp_async16(st + A_BYTES + so, qb + go);
-  }
-  // the four 512-byte scale tiles of this K-tile are contiguous
-  cp_async16(st + A_BYTES + B_BYTES + tid * 16, sfa + static_cast<int64_t>(kt) * SF_BYTES + tid * 16);
-  cp_async16(st + A_BYTES + B_BYTES + SF_BYTES + tid * 16,
-             sfb + static_cast<int64_t>(kt) * SF_BYTES + tid * 16);
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
 }
 
-template <typename OutT>
+// TMA tile load of a 2-D box (x in bytes along the row, y rows), completing
+// on an mbarrier; no multicast
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// contiguous bulk copy (16-byte aligned, size a multiple of 16) completing
+// on an mbarrier; no multicast
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+template <typename OutT, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_nvfp4_kernel(const uint8_t *__restrict__ qa, const uint8_t *__restrict__ sfa,
-                  const float *__restrict__ s_a, const uint8_t *__restrict__ qb,
-                  const uint8_t *__restrict__ sfb, const float *__restrict__ s_b, int K,
-                  OutT *__restrict__ c, int64_t ldc, int *__restrict__ status) {
+gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
+                  const __grid_constant__ CUtensorMap map_b, const uint8_t *__restrict__ sfa,
+                  const float *__restrict__ s_a, const uint8_t *__restrict__ sfb,
+                  const float *__restrict__ s_b, int K, OutT *__restrict__ c, int64_t ldc,
+                  int *__restrict__ status) {
+  using T = Tile<BN>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t bars = base + STAGES * STAGE_BYTES;   // STAGES empty barriers, then done
-  const uint32_t done_bar = bars + 8 * STAGES;
+  const uint32_t full = base + STAGES * T::STAGE_BYTES;   // STAGES "full" barriers
+  const uint32_t empty = full + 8 * STAGES;               // STAGES "empty" barriers
+  const uint32_t done_bar = empty + 8 * STAGES;
   const uint32_t tmem_slot = done_bar + 8;
-  uint8_t *const slot_ptr = smem_raw + (tmem_slot - raw);
+  const uint32_t err_slot = tmem_slot + 4;
+  volatile uint32_t *slot_ptr = reinterpret_cast<volatile uint32_t *>(smem_raw + (tmem_slot - raw));
+  volatile int *err_ptr = reinterpret_cast<volatile int *>(smem_raw + (err_slot - raw));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * BM;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BN;
-  const int64_t ldk = K / 2;                           // code bytes per row
+  const int m0 = static_cast<int>(blockIdx.y) * BM;
+  const int n0 = static_cast<int>(blockIdx.x) * BN;
   const int KT = K / KTILE;
-  const int64_t sf_per_rowtile = static_cast<int64_t>(K / 64) * SF_TILE;
-  const uint8_t *a_rows = qa + m0 * ldk, *b_rows = qb + n0 * ldk;
-  const uint8_t *a_sf = sfa + (m0 / BM) * sf_per_rowtile, *b_sf = sfb + (n0 / BN) * sf_per_rowtile;
+  const int64_t sf_rowtile = static_cast<int64_t>(K / 64) * SF_TILE;   // bytes per 128-row tile
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      tmem_slot),
-                 "r"(TMEM_COLS)
+                 "r"(T::TMEM_COLS)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) mbar_init(bars + 8 * s, 1);
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(full + 8 * i, 1);
+      mbar_init(empty + 8 * i, 1);
+    }
     mbar_init(done_bar, 1);
+    *err_ptr = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(slot_ptr);
+  const uint32_t tmem = *slot_ptr;
 
-  // prologue: K-tiles 0 .. STAGES-3
-#pragma unroll
-  for (int t = 0; t < STAGES - 2; ++t) {
-    if (t < KT) load_stage(base + t * STAGE_BYTES, a_rows, b_rows, a_sf, b_sf, ldk, t);
-    cp_async_commit();
-  }
-  int err = 0;
-  for (int kt = 0; kt < KT; ++kt) {
-    const int t = kt + STAGES - 2;                     // the K-tile loaded now
-    if (t < KT) {
-      const int s = t % STAGES;
-      // its stage last held K-tile kt - 2: wait until the MMAs reading it are done
-      if (kt >= 2 && !mbar_wait(bars + 8 * s, static_cast<uint32_t>(((kt - 2) / STAGES) & 1)))
-        err = 1;
-      if (!err) load_stage(base + s * STAGE_BYTES, a_rows, b_rows, a_sf, b_sf, ldk, t);
-    }
-    cp_async_commit();
-    cp_async_wait<STAGES - 2>();                        // K-tile kt has landed
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    if (__syncthreads_or(err)) {
-      err = 1;
-      break;
-    }
-    if (tid == 0) {
-      tc_fence_after();
+  if (warp == 0 && lane == 0) {
+    // ---- producer ----
+    const uint8_t *sfa_tile = sfa + static_cast<int64_t>(m0 / BM) * sf_rowtile;
+    const uint8_t *sfb_tile = sfb + static_cast<int64_t>(n0 / 128) * sf_rowtile;
+    for (int kt = 0; kt < KT; ++kt) {
       const int s = kt % STAGES;
-      const uint32_t st = base + s * STAGE_BYTES;
-      const uint32_t sfa_col = tmem + SF_COL0 + 32u * s, sfb_col = sfa_col + 16u;
+      if (kt >= STAGES &&
+          !mbar_wait(empty + 8 * s, static_cast<uint32_t>((kt / STAGES - 1) & 1))) {
+        *err_ptr = 1;
+        break;
+      }
+      const uint32_t st = base + s * T::STAGE_BYTES;
+      const uint32_t bar = full + 8 * s;
+      mbar_expect_tx(bar, T::STAGE_BYTES);
+      tma_load_2d(st, &map_a, kt * KTB, m0, bar);
+      tma_load_2d(st + T::A_BYTES, &map_b, kt * KTB, n0, bar);
+      bulk_load(st + T::A_BYTES + T::B_BYTES, sfa_tile + static_cast<int64_t>(kt) * SF_BYTES,
+                SF_BYTES, bar);
+#pragma unroll
+      for (int h = 0; h < BN / 128; ++h)
+        bulk_load(st + T::A_BYTES + T::B_BYTES + SF_BYTES + h * SF_BYTES,
+                  sfb_tile + h * sf_rowtile + static_cast<int64_t>(kt) * SF_BYTES, SF_BYTES, bar);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---- tensor-core issue ----
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % STAGES;
+      if (!mbar_wait(full + 8 * s, static_cast<uint32_t>((kt / STAGES) & 1))) {
+        *err_ptr = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t st = base + s * T::STAGE_BYTES;
+      const uint32_t sfa_col = tmem + T::SF_COL0 + T::STAGE_COLS * s;
+      const uint32_t sfb_col = sfa_col + 16u;
 #pragma unroll
       for (int kb = 0; kb < KTILE / 64; ++kb) {
-        tc_copy_sf(sfa_col + 4u * kb, desc_sf(st + A_BYTES + B_BYTES + kb * SF_TILE));
-        tc_copy_sf(sfb_col + 4u * kb, desc_sf(st + A_BYTES + B_BYTES + SF_BYTES + kb * SF_TILE));
+        tc_copy_sf(sfa_col + 4u * kb, desc_sf(st + T::A_BYTES + T::B_BYTES + kb * SF_TILE));
+#pragma unroll
+        for (int h = 0; h < BN / 128; ++h)    // B rows 128h .. 128h + 127: columns 4h .. 4h + 3
+          tc_copy_sf(sfb_col + (T::SFB_COLS / 4) * kb + 4u * h,
+                     desc_sf(st + T::A_BYTES + T::B_BYTES + SF_BYTES + h * SF_BYTES +
+                             kb * SF_TILE));
       }
-      const uint64_t da = desc_sw128(st), db = desc_sw128(st + A_BYTES);
+      const uint64_t da = desc_sw128(st), db = desc_sw128(st + T::A_BYTES);
 #pragma unroll
       for (int kb = 0; kb < KTILE / 64; ++kb)          // 64 values = 32 bytes = 2 descriptor units
-        tc_mma(tmem, da + 2u * kb, db + 2u * kb, sfa_col + 4u * kb, sfb_col + 4u * kb,
-               (kt | kb) != 0);
-      tc_commit(bars + 8 * s);
+        tc_mma(tmem, da + 2u * kb, db + 2u * kb, T::IDESC, sfa_col + 4u * kb,
+               sfb_col + (T::SFB_COLS / 4) * kb, (kt | kb) != 0);
+      tc_commit(empty + 8 * s);
     }
+    tc_commit(done_bar);                                // everything issued above
   }
-  cp_async_wait<0>();
-  if (tid == 0) tc_commit(done_bar);                    // all MMAs issued so far
+  __syncwarp();
   const int late = mbar_wait(done_bar, 0) ? 0 : 1;
-  err = __syncthreads_or(err | late);
+  const int err = __syncthreads_or(late | *err_ptr);
   tc_fence_after();
-  if (!err && KT > 0) {
+  if (!err) {
     const float alpha = __fmul_rn(s_a ? *s_a : 1.0f, s_b ? *s_b : 1.0f);
-    OutT *row = c + (m0 + warp * 32 + lane) * ldc + n0;
+    OutT *row = c + (static_cast<int64_t>(m0) + warp * 32 + lane) * ldc + n0;
 #pragma unroll 1
     for (int j = 0; j < BN / 32; ++j) {
       uint32_t r[32];
@@ -288,27 +331,72 @@ gemm_nvfp4_kernel(const uint8_t *__restrict__ qa, const uint8_t *__restrict__ sf
   __syncthreads();
   if (warp == 0)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(TMEM_COLS)
+                 "r"(T::TMEM_COLS)
                  : "memory");
 }
 
-template <typename OutT>
+// cuTensorMapEncodeTiled, reached through the runtime (no link to the driver
+// library)
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// A [rows, row_bytes] byte matrix read as boxes of 128 bytes x box_rows rows
+// into 128-byte-swizzled shared memory.
+bool make_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t row_bytes,
+              int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(KTB), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename OutT, int BN>
 cudaError_t launch_t(const uint8_t *qa, const uint8_t *sfa, const float *s_a, const uint8_t *qb,
                      const uint8_t *sfb, const float *s_b, int64_t M, int64_t N, int64_t K,
                      void *c, int64_t ldc, int *status, const Launch &L) {
+  using T = Tile<BN>;
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
     const cudaError_t e = cudaFuncSetAttribute(
-        gemm_nvfp4_kernel<OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        gemm_nvfp4_kernel<OutT, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
+  CUtensorMap map_a, map_b;
+  if (!make_map(&map_a, qa, M, K / 2, BM) || !make_map(&map_b, qb, N, K / 2, BN))
+    return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(N / BN), static_cast<unsigned>(M / BM));
-  gemm_nvfp4_kernel<OutT><<<grid, kThreads, SMEM_BYTES, L.stream>>>(
-      qa, sfa, s_a, qb, sfb, s_b, static_cast<int>(K), static_cast<OutT *>(c), ldc, status);
+  gemm_nvfp4_kernel<OutT, BN><<<grid, kThreads, T::SMEM_BYTES, L.stream>>>(
+      map_a, map_b, sfa, s_a, sfb, s_b, static_cast<int>(K), static_cast<OutT *>(c), ldc, status);
   return cudaGetLastError();
+}
+
+template <typename OutT>
+cudaError_t launch_o(const uint8_t *qa, const uint8_t *sfa, const float *s_a, const uint8_t *qb,
+                     const uint8_t *sfb, const float *s_b, int64_t M, int64_t N, int64_t K,
+                     void *c, int64_t ldc, int *status, const Launch &L) {
+  if (N % 256 == 0)
+    return launch_t<OutT, 256>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, L);
+  return launch_t<OutT, 128>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, L);
 }
 
 }  // namespace
@@ -318,8 +406,8 @@ cudaError_t launch_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float
                               int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
                               int *status, const Launch &L) {
   if (c_dtype == FP4Q_BF16)
-    return launch_t<__nv_bfloat16>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, L);
-  return launch_t<float>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, L);
+    return launch_o<__nv_bfloat16>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, L);
+  return launch_o<float>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, L);
 }
 
 }  // namespace fp4q

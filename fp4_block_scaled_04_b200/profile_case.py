@@ -23,7 +23,7 @@ from fp4_block_scaled_04_b200 import workloads
 
 OPS = ["amax", "nvfp4_row", "nvfp4_rowcol", "mxfp4_rowcol", "2d", "rht16_sr", "rht128_sr",
        "rht16_rne", "rht128_rne", "if4", "if4_dequant", "four_over_six_rowcol", "nvint4",
-       "bwd16_sr", "bwd16_rne", "row_sr", "mxfp6_e2m3", "mxfp6_dequant"]
+       "bwd16_sr", "bwd16_rne", "row_sr", "mxfp6_e2m3", "mxfp6_dequant", "gemm_nvfp4"]
 
 
 def make(op: str, rows: int, cols: int, dev):
@@ -46,6 +46,16 @@ def make(op: str, rows: int, cols: int, dev):
         o = fq.fp4q_quantize_four_over_six(x, layouts=3, amax=a, scale_layout=sw)
         return lambda: fq.fp4q_quantize_four_over_six(x, layouts=3, amax=a, scale_layout=sw,
                                                       out=o)
+    if op == "gemm_nvfp4":              # M = N = rows, K = cols
+        g = torch.Generator().manual_seed(5)
+        x = torch.randn(rows, cols, generator=g).to(torch.bfloat16).to(dev)
+        w = (torch.randn(rows, cols, generator=g) * 0.05).to(torch.bfloat16).to(dev)
+        ox = fq.fp4q_quantize_nvfp4(x, scale_layout=fq.SCALE_SWIZZLED)
+        ow = fq.fp4q_quantize_nvfp4(w, scale_layout=fq.SCALE_SWIZZLED)
+        c = torch.empty((rows, rows), dtype=torch.bfloat16, device=dev)
+        return lambda: fq.fp4q_gemm_nvfp4(ox["q_row"], ox["sf_row"], ow["q_row"], ow["sf_row"],
+                                          cols, tensor_scale_a=ox["s_dec"],
+                                          tensor_scale_b=ow["s_dec"], out=c)
     if op in ("mxfp6_e2m3", "mxfp6_dequant"):
         x = workloads.activation(rows=rows, cols=cols).to(dev)
         o = fq.fp4q_quantize_mxfp6(x, fq.FP6_E2M3, scale_layout=sw)
