@@ -12,21 +12,27 @@
 //   C[m, n] = RN(acc[m, n] * RN(s_a * s_b)),
 //   acc[m, n] = sum_k (g_a[m,k] S_a[m,k/16]) (g_b[n,k] S_b[n,k/16])   (FP32)
 //
-// One CTA computes a 128 x BN tile of C (BN = 256, or 128 when N is not a
-// multiple of 256) with 4 warps in three roles:
-//  - one thread of warp 0 is the producer: per K-tile of 256 values it
-//    loads the A and B code tiles with TMA (cp.async.bulk.tensor, 128-byte
-//    swizzle, which is the K-major layout the MMA descriptors describe) and
-//    the 2 KiB scale blocks with plain bulk copies (the 128x4 tiles of one
-//    K-tile are contiguous in the swizzled layout), all completing on the
-//    stage's "full" mbarrier; four stages;
+// The kernel is persistent: one CTA per SM walks the 128 x BN output tiles
+// (BN = 256, or 128 when N is not a multiple of 256) in row-major order,
+// taking every gridDim-th tile, with six warps in three roles:
+//  - one thread of warp 0 is the producer: for every K-tile of 256 values of
+//    every tile it loads the A and B code tiles with TMA (cp.async.bulk.tensor,
+//    128-byte swizzle, which is the K-major layout the MMA descriptors
+//    describe) and the 2 KiB scale blocks with plain bulk copies (the 128x4
+//    tiles of one K-tile are contiguous in the swizzled layout), completing on
+//    the stage's "full" mbarrier; four stages, one stream across tiles, so the
+//    next tile's first K-tiles load while the current one finishes;
 //  - one thread of warp 1 issues the tensor-core work: tcgen05.cp
 //    32x128b.warpx4 of each 512-byte scale tile into tensor memory (4
 //    columns per 64-value K step and 128 rows), then four tcgen05.mma
-//    kind::mxf4nvf4 block16 (M = 128, N = BN, K = 64) accumulating in
-//    tensor memory, then tcgen05.commit to the stage's "empty" mbarrier;
-//  - at the end all four warps read their 32 accumulator rows with
-//    tcgen05.ld and write C (FP32 or BF16).
+//    kind::mxf4nvf4 block16 (M = 128, N = BN, K = 64) accumulating in tensor
+//    memory, then tcgen05.commit to the stage's "empty" mbarrier; after the
+//    last K-tile it commits to "acc_full", and it starts the next tile only
+//    once the epilogue has signalled "acc_empty";
+//  - warps 2-5 are the epilogue: each reads its 32 accumulator rows with
+//    tcgen05.ld (warp w reaches lanes 32 (w % 4) .. + 31), scales by
+//    RN(s_a s_b), hands tensor memory back (for BF16 output as soon as the
+//    row is in registers) and writes C.
 // No load uses cluster multicast.  Every mbarrier wait is bounded (about a
 // second of clock cycles); a wait that runs out sets *status, the roles stop
 // issuing, and the CTA waits (bounded) for its tensor-core work, frees its
@@ -46,7 +52,7 @@ constexpr int BM = 128;
 constexpr int KTILE = 256;                       // K values per stage
 constexpr int KTB = KTILE / 2;                   // 128 code bytes per row per stage
 constexpr int STAGES = 4;
-constexpr int kThreads = 128;
+constexpr int kThreads = 192;                    // producer warp, MMA warp, 4 epilogue warps
 constexpr int SF_TILE = 512;                     // 128 rows x 4 scales
 constexpr int SF_BYTES = (KTILE / 64) * SF_TILE; // 2048: one operand row tile, one K-tile
 constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at the B200's clock
@@ -146,21 +152,19 @@ __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint3
       : "memory");
 }
 
-// 32 consecutive FP32 accumulator columns of this thread's row (warp w reads
-// lanes 32w .. 32w + 31)
-__device__ __forceinline__ void tc_load32(uint32_t taddr, uint32_t (&r)[32]) {
+// 16 consecutive FP32 accumulator columns of this thread's row (warp w reads
+// lanes 32 (w % 4) .. + 31); the wait is separate so that loads can overlap
+__device__ __forceinline__ void tc_load16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
       : "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
@@ -196,23 +200,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
                   const __grid_constant__ CUtensorMap map_b, const uint8_t *__restrict__ sfa,
                   const float *__restrict__ s_a, const uint8_t *__restrict__ sfb,
-                  const float *__restrict__ s_b, int K, OutT *__restrict__ c, int64_t ldc,
-                  int *__restrict__ status) {
+                  const float *__restrict__ s_b, int K, int n_tiles_n, int n_tiles,
+                  OutT *__restrict__ c, int64_t ldc, int *__restrict__ status) {
   using T = Tile<BN>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const uint32_t full = base + STAGES * T::STAGE_BYTES;   // STAGES "full" barriers
   const uint32_t empty = full + 8 * STAGES;               // STAGES "empty" barriers
-  const uint32_t done_bar = empty + 8 * STAGES;
-  const uint32_t tmem_slot = done_bar + 8;
+  const uint32_t acc_full = empty + 8 * STAGES;           // accumulator written
+  const uint32_t acc_empty = acc_full + 8;                // accumulator read out
+  const uint32_t tmem_slot = acc_empty + 8;
   const uint32_t err_slot = tmem_slot + 4;
   volatile uint32_t *slot_ptr = reinterpret_cast<volatile uint32_t *>(smem_raw + (tmem_slot - raw));
   volatile int *err_ptr = reinterpret_cast<volatile int *>(smem_raw + (err_slot - raw));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m0 = static_cast<int>(blockIdx.y) * BM;
-  const int n0 = static_cast<int>(blockIdx.x) * BN;
   const int KT = K / KTILE;
   const int64_t sf_rowtile = static_cast<int64_t>(K / 64) * SF_TILE;   // bytes per 128-row tile
 
@@ -228,7 +231,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
       mbar_init(full + 8 * i, 1);
       mbar_init(empty + 8 * i, 1);
     }
-    mbar_init(done_bar, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);                              // one arrival per epilogue warp
     *err_ptr = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -237,98 +241,142 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
   tc_fence_after();
   const uint32_t tmem = *slot_ptr;
 
-  if (warp == 0 && lane == 0) {
-    // ---- producer ----
-    const uint8_t *sfa_tile = sfa + static_cast<int64_t>(m0 / BM) * sf_rowtile;
-    const uint8_t *sfb_tile = sfb + static_cast<int64_t>(n0 / 128) * sf_rowtile;
-    for (int kt = 0; kt < KT; ++kt) {
-      const int s = kt % STAGES;
-      if (kt >= STAGES &&
-          !mbar_wait(empty + 8 * s, static_cast<uint32_t>((kt / STAGES - 1) & 1))) {
-        *err_ptr = 1;
-        break;
-      }
-      const uint32_t st = base + s * T::STAGE_BYTES;
-      const uint32_t bar = full + 8 * s;
-      mbar_expect_tx(bar, T::STAGE_BYTES);
-      tma_load_2d(st, &map_a, kt * KTB, m0, bar);
-      tma_load_2d(st + T::A_BYTES, &map_b, kt * KTB, n0, bar);
-      bulk_load(st + T::A_BYTES + T::B_BYTES, sfa_tile + static_cast<int64_t>(kt) * SF_BYTES,
-                SF_BYTES, bar);
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- producer: the K-tiles of this CTA's output tiles, one stream ----
+      int g = 0;                                          // K-tiles issued so far
+      for (int tile = blockIdx.x; tile < n_tiles && !*err_ptr; tile += gridDim.x) {
+        const int m0 = (tile / n_tiles_n) * BM, n0 = (tile % n_tiles_n) * BN;
+        const uint8_t *sfa_tile = sfa + static_cast<int64_t>(m0 / BM) * sf_rowtile;
+        const uint8_t *sfb_tile = sfb + static_cast<int64_t>(n0 / 128) * sf_rowtile;
+        for (int kt = 0; kt < KT; ++kt, ++g) {
+          const int s = g % STAGES;
+          if (g >= STAGES &&
+              !mbar_wait(empty + 8 * s, static_cast<uint32_t>((g / STAGES - 1) & 1))) {
+            *err_ptr = 1;
+            break;
+          }
+          const uint32_t st = base + s * T::STAGE_BYTES;
+          const uint32_t bar = full + 8 * s;
+          mbar_expect_tx(bar, T::STAGE_BYTES);
+          tma_load_2d(st, &map_a, kt * KTB, m0, bar);
+          tma_load_2d(st + T::A_BYTES, &map_b, kt * KTB, n0, bar);
+          bulk_load(st + T::A_BYTES + T::B_BYTES, sfa_tile + static_cast<int64_t>(kt) * SF_BYTES,
+                    SF_BYTES, bar);
 #pragma unroll
-      for (int h = 0; h < BN / 128; ++h)
-        bulk_load(st + T::A_BYTES + T::B_BYTES + SF_BYTES + h * SF_BYTES,
-                  sfb_tile + h * sf_rowtile + static_cast<int64_t>(kt) * SF_BYTES, SF_BYTES, bar);
+          for (int h = 0; h < BN / 128; ++h)
+            bulk_load(st + T::A_BYTES + T::B_BYTES + SF_BYTES + h * SF_BYTES,
+                      sfb_tile + h * sf_rowtile + static_cast<int64_t>(kt) * SF_BYTES, SF_BYTES,
+                      bar);
+        }
+      }
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---- tensor-core issue ----
-    for (int kt = 0; kt < KT; ++kt) {
-      const int s = kt % STAGES;
-      if (!mbar_wait(full + 8 * s, static_cast<uint32_t>((kt / STAGES) & 1))) {
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- tensor-core issue ----
+      int g = 0, i = 0;                                   // K-tiles consumed, tiles done
+      for (int tile = blockIdx.x; tile < n_tiles && !*err_ptr; tile += gridDim.x, ++i) {
+        // the epilogue must have read the previous tile's accumulator
+        if (i > 0 && !mbar_wait(acc_empty, static_cast<uint32_t>((i - 1) & 1))) {
+          *err_ptr = 1;
+          break;
+        }
+        tc_fence_after();
+        for (int kt = 0; kt < KT; ++kt, ++g) {
+          const int s = g % STAGES;
+          if (!mbar_wait(full + 8 * s, static_cast<uint32_t>((g / STAGES) & 1))) {
+            *err_ptr = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = base + s * T::STAGE_BYTES;
+          const uint32_t sfa_col = tmem + T::SF_COL0 + T::STAGE_COLS * s;
+          const uint32_t sfb_col = sfa_col + 16u;
+#pragma unroll
+          for (int kb = 0; kb < KTILE / 64; ++kb) {
+            tc_copy_sf(sfa_col + 4u * kb, desc_sf(st + T::A_BYTES + T::B_BYTES + kb * SF_TILE));
+#pragma unroll
+            for (int h = 0; h < BN / 128; ++h)   // B rows 128h .. 128h + 127: columns 4h .. 4h + 3
+              tc_copy_sf(sfb_col + (T::SFB_COLS / 4) * kb + 4u * h,
+                         desc_sf(st + T::A_BYTES + T::B_BYTES + SF_BYTES + h * SF_BYTES +
+                                 kb * SF_TILE));
+          }
+          const uint64_t da = desc_sw128(st), db = desc_sw128(st + T::A_BYTES);
+#pragma unroll
+          for (int kb = 0; kb < KTILE / 64; ++kb)       // 64 values = 32 bytes = 2 descriptor units
+            tc_mma(tmem, da + 2u * kb, db + 2u * kb, T::IDESC, sfa_col + 4u * kb,
+                   sfb_col + (T::SFB_COLS / 4) * kb, (kt | kb) != 0);
+          tc_commit(empty + 8 * s);
+        }
+        tc_commit(acc_full);                            // this tile's accumulator is complete
+      }
+    }
+  } else {
+    // ---- epilogue: warp w reads accumulator lanes 32 (w % 4) .. + 31 ----
+    const int quarter = warp & 3;
+    const float alpha = __fmul_rn(s_a ? *s_a : 1.0f, s_b ? *s_b : 1.0f);
+    int i = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+      const int ok = mbar_wait(acc_full, static_cast<uint32_t>(i & 1)) ? 1 : 0;
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
         *err_ptr = 1;
         break;
       }
       tc_fence_after();
-      const uint32_t st = base + s * T::STAGE_BYTES;
-      const uint32_t sfa_col = tmem + T::SF_COL0 + T::STAGE_COLS * s;
-      const uint32_t sfb_col = sfa_col + 16u;
+      const int m0 = (tile / n_tiles_n) * BM, n0 = (tile % n_tiles_n) * BN;
+      OutT *row = c + (static_cast<int64_t>(m0) + quarter * 32 + lane) * ldc + n0;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+      if (sizeof(OutT) == 2) {
+        // BF16: the whole converted row (BN / 2 words) stays in registers, so
+        // tensor memory is handed back before the stores
+        uint32_t w[BN / 2];
 #pragma unroll
-      for (int kb = 0; kb < KTILE / 64; ++kb) {
-        tc_copy_sf(sfa_col + 4u * kb, desc_sf(st + T::A_BYTES + T::B_BYTES + kb * SF_TILE));
+        for (int j = 0; j < BN / 16; ++j) {
+          uint32_t r[16];
+          tc_load16(taddr + 16u * j, r);
+          tc_wait_ld();
 #pragma unroll
-        for (int h = 0; h < BN / 128; ++h)    // B rows 128h .. 128h + 127: columns 4h .. 4h + 3
-          tc_copy_sf(sfb_col + (T::SFB_COLS / 4) * kb + 4u * h,
-                     desc_sf(st + T::A_BYTES + T::B_BYTES + SF_BYTES + h * SF_BYTES +
-                             kb * SF_TILE));
-      }
-      const uint64_t da = desc_sw128(st), db = desc_sw128(st + T::A_BYTES);
-#pragma unroll
-      for (int kb = 0; kb < KTILE / 64; ++kb)          // 64 values = 32 bytes = 2 descriptor units
-        tc_mma(tmem, da + 2u * kb, db + 2u * kb, T::IDESC, sfa_col + 4u * kb,
-               sfb_col + (T::SFB_COLS / 4) * kb, (kt | kb) != 0);
-      tc_commit(empty + 8 * s);
-    }
-    tc_commit(done_bar);                                // everything issued above
-  }
-  __syncwarp();
-  const int late = mbar_wait(done_bar, 0) ? 0 : 1;
-  const int err = __syncthreads_or(late | *err_ptr);
-  tc_fence_after();
-  if (!err) {
-    const float alpha = __fmul_rn(s_a ? *s_a : 1.0f, s_b ? *s_b : 1.0f);
-    OutT *row = c + (static_cast<int64_t>(m0) + warp * 32 + lane) * ldc + n0;
-#pragma unroll 1
-    for (int j = 0; j < BN / 32; ++j) {
-      uint32_t r[32];
-      tc_load32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + 32u * j, r);
-      if (sizeof(OutT) == 4) {
-        float4 *d = reinterpret_cast<float4 *>(row + 32 * j);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          d[q] = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), alpha),
-                             __fmul_rn(__uint_as_float(r[4 * q + 1]), alpha),
-                             __fmul_rn(__uint_as_float(r[4 * q + 2]), alpha),
-                             __fmul_rn(__uint_as_float(r[4 * q + 3]), alpha));
-      } else {
-        uint4 *d = reinterpret_cast<uint4 *>(row + 32 * j);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t w[4];
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                __fmul_rn(__uint_as_float(r[8 * q + 2 * h]), alpha),
-                __fmul_rn(__uint_as_float(r[8 * q + 2 * h + 1]), alpha));
-            memcpy(&w[h], &b2, sizeof(uint32_t));
+          for (int q = 0; q < 8; ++q) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * q]), alpha),
+                                                      __fmul_rn(__uint_as_float(r[2 * q + 1]), alpha));
+            memcpy(&w[8 * j + q], &b2, sizeof(uint32_t));
           }
-          d[q] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty) : "memory");
+        uint4 *d = reinterpret_cast<uint4 *>(row);
+#pragma unroll
+        for (int q = 0; q < BN / 8; ++q) d[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+      } else {
+        // FP32: chunk by chunk; tensor memory is handed back after the last load
+        float4 *d = reinterpret_cast<float4 *>(row);
+#pragma unroll
+        for (int j = 0; j < BN / 16; ++j) {
+          uint32_t r[16];
+          tc_load16(taddr + 16u * j, r);
+          tc_wait_ld();
+          if (j == BN / 16 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+              asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty) : "memory");
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            d[4 * j + q] = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), alpha),
+                                       __fmul_rn(__uint_as_float(r[4 * q + 1]), alpha),
+                                       __fmul_rn(__uint_as_float(r[4 * q + 2]), alpha),
+                                       __fmul_rn(__uint_as_float(r[4 * q + 3]), alpha));
         }
       }
     }
   }
-  if (err && tid == 0 && status) atomicExch(status, 1);
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
+  if (tid == 0 && status && *err_ptr) atomicExch(status, 1);
   if (warp == 0)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(T::TMEM_COLS)
@@ -384,9 +432,13 @@ cudaError_t launch_t(const uint8_t *qa, const uint8_t *sfa, const float *s_a, co
   CUtensorMap map_a, map_b;
   if (!make_map(&map_a, qa, M, K / 2, BM) || !make_map(&map_b, qb, N, K / 2, BN))
     return cudaErrorInvalidValue;
-  const dim3 grid(static_cast<unsigned>(N / BN), static_cast<unsigned>(M / BM));
+  // persistent: one CTA per SM (the stages fill its shared memory), output
+  // tiles in row-major order, each CTA taking every gridDim-th tile
+  const int64_t n_tiles_n = N / BN, n_tiles = (M / BM) * n_tiles_n;
+  const int grid = static_cast<int>(n_tiles < L.num_sms ? n_tiles : L.num_sms);
   gemm_nvfp4_kernel<OutT, BN><<<grid, kThreads, T::SMEM_BYTES, L.stream>>>(
-      map_a, map_b, sfa, s_a, sfb, s_b, static_cast<int>(K), static_cast<OutT *>(c), ldc, status);
+      map_a, map_b, sfa, s_a, sfb, s_b, static_cast<int>(K), static_cast<int>(n_tiles_n),
+      static_cast<int>(n_tiles), static_cast<OutT *>(c), ldc, status);
   return cudaGetLastError();
 }
 
