@@ -267,7 +267,8 @@ def time_consumer_gemm(fq, device, stream, args, M=8192, N=8192, K=8192):
     out["fp4q"] = timed(lambda: fq.fp4q_gemm_nvfp4(
         ox["q_row"], ox["sf_row"], ow["q_row"], ow["sf_row"], K, tensor_scale_a=ox["s_dec"],
         tensor_scale_b=ow["s_dec"], out=c))
-    out["fp4q"]["kernel"] = "gemm_nvfp4_kernel (tcgen05.mma kind::mxf4nvf4, 128x128 tiles)"
+    out["fp4q"]["kernel"] = ("gemm_nvfp4_kernel (tcgen05.mma kind::mxf4nvf4, persistent, "
+                             "128x256 tiles)")
     A = ox["q_row"].view(torch.float4_e2m1fn_x2)
     B = ow["q_row"].view(torch.float4_e2m1fn_x2).t()
     sa, sb = ox["sf_row"].view(torch.float8_e4m3fn), ow["sf_row"].view(torch.float8_e4m3fn)
