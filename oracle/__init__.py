@@ -30,7 +30,7 @@ ROWWISE, COLWISE = 1, 2
 RNE, SR = 0, 1
 SCALE_LINEAR, SCALE_SWIZZLED = 0, 1
 E8M0_RNE, E8M0_CEIL, E8M0_OCP_FLOOR = 0, 1, 2
-FMT_NVFP4, FMT_MXFP4, FMT_IF4, FMT_MXFP6_E2M3, FMT_MXFP6_E3M2 = 0, 1, 2, 3, 4
+FMT_NVFP4, FMT_MXFP4, FMT_IF4, FMT_MXFP6_E2M3, FMT_MXFP6_E3M2, FMT_IF6 = 0, 1, 2, 3, 4, 5
 FP6_E2M3, FP6_E3M2 = 0, 1
 
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
@@ -83,6 +83,9 @@ def lib() -> ctypes.CDLL:
             "orc_if4_c76": (F, []),
             "orc_if4_c67": (F, []),
             "orc_quantize_if4": (I, [P, I, I64, I64, I64, P, P, P, P, I, I]),
+            "orc_if6_cu": (F, []),
+            "orc_if6_cd": (F, []),
+            "orc_quantize_if6": (I, [P, I, I64, I64, I64, P, P, P, P, I, I]),
             "orc_quantize_four_over_six": (I, [P, I, I64, I64, I64, U, P, P, P, P, P, P, I]),
             "orc_dequantize": (I, [I, P, P, I, I, I, P, I64, I64, P, I]),
             "orc_glossary_mae": (ctypes.c_double, [P, I64, I64]),
@@ -409,6 +412,29 @@ def quantize_if4(x: np.ndarray, amax: float | None = None, scale_layout: int = S
     rc = lib().orc_quantize_if4(_ptr(x), _dtype_code(x), rows, cols, cols, ap,
                                 _ptr(out["s_dec"]), _ptr(out["q"]), _ptr(out["sf"]),
                                 scale_layout, 2 if int4_only else (1 if allow_int4 else 0))
+    if rc != 0:
+        raise ValueError(f"oracle rejected shape {x.shape}")
+    return out
+
+
+def if6_constants():
+    return float(lib().orc_if6_cu()), float(lib().orc_if6_cd())
+
+
+def quantize_if6(x: np.ndarray, amax: float | None = None, scale_layout: int = SCALE_LINEAR,
+                 mode: int = 1) -> dict:
+    """IF6 (mode 1): per 16-block FP6 E2M3 or INT6 (the 6/7 method with 31 and
+    7.5); mode 0 keeps FP6 everywhere, mode 2 INT6 everywhere.  Codes
+    [rows, cols * 3/4] (four 6-bit codes per three bytes)."""
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    out = {"s_dec": np.zeros(1, np.float32),
+           "q": np.zeros((rows, cols * 3 // 4), np.uint8),
+           "sf": np.zeros(scale_bytes(rows, cols // 16, scale_layout), np.uint8)}
+    keep, ap = _amax_arg(amax)
+    rc = lib().orc_quantize_if6(_ptr(x), _dtype_code(x), rows, cols, cols, ap,
+                                _ptr(out["s_dec"]), _ptr(out["q"]), _ptr(out["sf"]),
+                                scale_layout, mode)
     if rc != 0:
         raise ValueError(f"oracle rejected shape {x.shape}")
     return out

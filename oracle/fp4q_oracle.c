@@ -49,6 +49,7 @@
 #define ORC_FMT_IF4 2
 #define ORC_FMT_MXFP6_E2M3 3
 #define ORC_FMT_MXFP6_E3M2 4
+#define ORC_FMT_IF6 5
 #define ORC_FP6_E2M3 0
 #define ORC_FP6_E3M2 1
 
@@ -757,6 +758,84 @@ int orc_quantize_mxfp6(const void *x, int dtype, int64_t rows, int64_t cols, int
 }
 
 /* ------------------------------------------------------------------------ */
+/* IF6: the IF idea at 6 bits.  [I] section 2 says the per-block FP/INT      */
+/* choice applies to 6-bit (IF6) formats as well, without details.           */
+/* READING (the plainest one the IF4 description supports):                 */
+/*   the FP candidate is FP6 E2M3 (the finer FP6 grid, largest 7.5, [F]);    */
+/*   the block scale maps the block maximum to 7.5 as NVFP4 maps it to 6:    */
+/*     s_enc = RN(3360/amax), s_dec = RN(amax/3360) with 3360 = 7.5 * 448,  */
+/*     S = E4M3_rne_sat(RN(RN(m * s_enc) / 7.5)), r = RN(s_enc / S),         */
+/*     v_i = RN(x_i * r);                                                    */
+/*   FP6:  g_i = E2M3 value of fp6_rne(v_i)                                  */
+/*   INT6 (the 6/7 method with 31 and 7.5): k_i = clamp(rint(RN(v_i * CU)),  */
+/*         -31, 31), h_i = RN(k_i * CD), CU = RN(31/7.5), CD = RN(7.5/31);   */
+/*   errors, their order and the choice exactly as IF4 (INT6 iff strictly    */
+/*   smaller); scale bit 7 set = INT6.                                       */
+/* Codes are 6 bits (FP6 code with the sign in bit 5, or k_i in 6-bit two's */
+/* complement), packed four per three bytes like MXFP6: codes [rows,         */
+/* cols * 3/4], scales [rows, cols/16].  int6_mode 0 keeps FP6 everywhere,   */
+/* 1 is IF6, 2 keeps INT6 everywhere.                                        */
+/* ------------------------------------------------------------------------ */
+
+float orc_if6_cu(void) { return 31.0f / 7.5f; }
+float orc_if6_cd(void) { return 7.5f / 31.0f; }
+
+int orc_quantize_if6(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                     const float *amax_in, float *s_dec_out, uint8_t *q, uint8_t *sf_out,
+                     int scale_layout, int int6_mode) {
+  if (cols % 16 != 0) return 1;
+  float amax = amax_in ? *amax_in : orc_amax(x, dtype, rows, cols, ld);
+  float s_enc, s_dec;
+  tensor_scales_top(amax, 7.5f * 448.0f, &s_enc, &s_dec);
+  if (s_dec_out) *s_dec_out = s_dec;
+  const float CU = orc_if6_cu(), CD = orc_if6_cd();
+  const int64_t rb = cols * 3 / 4;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < cols / 16; ++b) {
+      float xv[16];
+      float m = 0.0f;
+      for (int k = 0; k < 16; ++k) {
+        xv[k] = load_elem(x, dtype, ld, r, b * 16 + k);
+        if (fabsf(xv[k]) > m) m = fabsf(xv[k]);
+      }
+      uint8_t sf = block_scale_q(m, s_enc, 7.5f);
+      float rf = nvfp4_block_factor(sf, s_enc);
+      uint8_t fp_code[16], int_code[16];
+      float e_fp = 0.0f, e_int = 0.0f;
+      for (int k = 0; k < 16; ++k) {
+        float v = xv[k] * rf;
+        fp_code[k] = orc_fp6_rne(v, ORC_FP6_E2M3);
+        float g = orc_fp6_value(fp_code[k], ORC_FP6_E2M3);
+        float kk = rintf(v * CU);
+        if (kk > 31.0f) kk = 31.0f;
+        if (kk < -31.0f) kk = -31.0f;
+        int ki = (int)kk;
+        int_code[k] = (uint8_t)(ki & 0x3F);
+        float h = (float)ki * CD;
+        float d_fp = v - g;
+        float d_int = v - h;
+        e_fp = fmaf(d_fp, d_fp, e_fp);
+        e_int = fmaf(d_int, d_int, e_int);
+      }
+      int use_int = int6_mode == 2 || (int6_mode == 1 && e_int < e_fp);
+      sf_out[orc_scale_offset(r, b, rows, cols / 16, scale_layout)] =
+          (uint8_t)(sf | (use_int ? 0x80 : 0x00));
+      for (int g4 = 0; g4 < 4; ++g4) {
+        uint32_t w = 0;
+        for (int j = 0; j < 4; ++j) {
+          int k = g4 * 4 + j;
+          w |= (uint32_t)(use_int ? int_code[k] : fp_code[k]) << (6 * j);
+        }
+        uint8_t *dst = q + r * rb + (b * 4 + g4) * 3;
+        dst[0] = (uint8_t)(w & 0xFF);
+        dst[1] = (uint8_t)((w >> 8) & 0xFF);
+        dst[2] = (uint8_t)((w >> 16) & 0xFF);
+      }
+    }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Dequantization  [G] "FP4の仕組み" (reconstruct = grid value * sign * scale)*/
 /* NVFP4:  y = RN(RN(g * S) * s_dec)   (g * S is exact)                       */
 /* IF4 INT4 blocks: h = RN(k * C67), y = RN(RN(h * S) * s_dec)                */
@@ -773,12 +852,13 @@ int orc_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_la
   if (cols % block_cols != 0 || rows % block_rows != 0) return 1;
   float s_dec = s_dec_in ? *s_dec_in : 1.0f;
   int64_t srows = rows / block_rows, scols = cols / block_cols;
-  const float C67 = orc_if4_c67();
+  const float C67 = orc_if4_c67(), CD6 = orc_if6_cd();
   const int fp6 = (format == ORC_FMT_MXFP6_E2M3 || format == ORC_FMT_MXFP6_E3M2);
+  const int six = fp6 || format == ORC_FMT_IF6;             /* 6-bit codes, 4 per 3 bytes */
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t c = 0; c < cols; ++c) {
       uint8_t code;
-      if (fp6) {
+      if (six) {
         const uint8_t *g3 = q + r * (cols * 3 / 4) + (c / 4) * 3;
         uint32_t w = (uint32_t)g3[0] | ((uint32_t)g3[1] << 8) | ((uint32_t)g3[2] << 16);
         code = (uint8_t)((w >> (6 * (c % 4))) & 0x3F);
@@ -802,6 +882,12 @@ int orc_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_la
           int k = (code & 0x8) ? (int)code - 16 : (int)code;
           float h = (float)k * C67;
           out = (h * S) * s_dec;
+        } else if (format == ORC_FMT_IF6 && (s & 0x80)) {
+          int k = (code & 0x20) ? (int)code - 64 : (int)code;
+          float h = (float)k * CD6;
+          out = (h * S) * s_dec;
+        } else if (format == ORC_FMT_IF6) {
+          out = (orc_fp6_value(code, ORC_FP6_E2M3) * S) * s_dec;
         } else {
           out = (orc_e2m1_value(code) * S) * s_dec;
         }
