@@ -286,8 +286,8 @@ def build_extra_jobs(device, fq, inputs):
     """Calls outside the headline suite, timed like it but reported apart from
     its value: the fused backward call and the row-wise operand alone on the
     gradient workload, and the IF4 explainer's comparison formats
-    (four-over-six on the activation workload, NVINT4 on the IF4 workload) and
-    MXFP6 E2M3 on the activation workload."""
+    (four-over-six on the activation workload, NVINT4 on the IF4 workload),
+    IF6 on the IF4 workload and MXFP6 E2M3 on the activation workload."""
     import torch
     SW = fq.SCALE_SWIZZLED
     xa = inputs["activation"].to(device)
@@ -315,6 +315,9 @@ def build_extra_jobs(device, fq, inputs):
     orow_n = fq.fp4q_quantize_nvfp4(g, layouts=fq.ROWWISE, amax=amax_g, scale_layout=SW)
     nb_row = T * Cg * 2 + T * Cg // 2 + T * Cg // 16 + 4
     nb_bw = T * Cg * 2 + 2 * (T * Cg // 2 + T * Cg // 16 + 4)
+    # IF6 of the IF4 workload: 2 bytes in, 0.75 + 1/16 out
+    oi6 = fq.fp4q_quantize_if6(x5, amax=amax5, scale_layout=SW)
+    nbi6 = R5 * C5 * 2 + R5 * C5 * 3 // 4 + R5 * C5 // 16 + 4
     # MXFP6 (E2M3) of the activation workload: 2 bytes in, 0.75 + 1/32 out
     o6 = fq.fp4q_quantize_mxfp6(xa, fq.FP6_E2M3, scale_layout=SW)
     nb6 = R * C * 2 + R * C * 3 // 4 + R * C // 32
@@ -339,6 +342,8 @@ def build_extra_jobs(device, fq, inputs):
                                                    out=o46)),
         Job("if4 16384x8192 bf16 nvint4", "if4.cu", nbi4, 1,
             lambda: fq.fp4q_quantize_nvint4(x5, amax=amax5, scale_layout=SW, out=oi4)),
+        Job("if4 16384x8192 bf16 if6", "if6.cu", nbi6, 1,
+            lambda: fq.fp4q_quantize_if6(x5, amax=amax5, scale_layout=SW, out=oi6)),
         Job("activation 8192x4096 bf16 mxfp6 e2m3 row-wise", "mxfp6.cu", nb6, 1,
             lambda: fq.fp4q_quantize_mxfp6(xa, fq.FP6_E2M3, scale_layout=SW, out=o6)),
     ]
@@ -566,7 +571,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the calls outside the suite (fused backward, row-wise alone, "
-                         "four-over-six, NVINT4, MXFP6) and the consumer GEMM")
+                         "four-over-six, NVINT4, IF6, MXFP6) and the consumer GEMM")
     ap.add_argument("--e2e-steps", type=int, default=None)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -15,6 +15,7 @@ Formats and layouts (see the header for the arithmetic):
   IF4    per-block FP4 / INT4 choice, flag in bit 7 of the scale byte
   MXFP6  FP6 (E2M3 or E3M2) codes, four per three bytes + E8M0 scale per 32
   GEMM   C = s_a s_b (A B^T) from NVFP4 operands on the tensor cores
+  IF6    per-block FP6 E2M3 / INT6 choice, six-bit codes, flag in bit 7 of the scale
 """
 from __future__ import annotations
 
@@ -33,14 +34,14 @@ __all__ = [
     "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
     "fp4q_quantize_nvfp4_noalloc", "fp4q_quantize_nvint4", "fp4q_quantize_four_over_six",
     "fp4q_quantize_backward", "fp4q_quantize_mxfp6", "FMT_MXFP6_E2M3", "FMT_MXFP6_E3M2",
-    "FP6_E2M3", "FP6_E3M2", "fp4q_gemm_nvfp4",
+    "FP6_E2M3", "FP6_E3M2", "fp4q_gemm_nvfp4", "fp4q_quantize_if6", "FMT_IF6",
 ]
 
 ROWWISE, COLWISE = 1, 2
 RNE, SR = 0, 1
 SCALE_LINEAR, SCALE_SWIZZLED = 0, 1
 E8M0_RNE, E8M0_CEIL, E8M0_OCP_FLOOR = 0, 1, 2
-FMT_NVFP4, FMT_MXFP4, FMT_IF4, FMT_MXFP6_E2M3, FMT_MXFP6_E3M2 = 0, 1, 2, 3, 4
+FMT_NVFP4, FMT_MXFP4, FMT_IF4, FMT_MXFP6_E2M3, FMT_MXFP6_E3M2, FMT_IF6 = 0, 1, 2, 3, 4, 5
 FP6_E2M3, FP6_E3M2 = 0, 1
 _BF16, _FP32 = 0, 1
 
@@ -95,6 +96,7 @@ _SIGNATURES = {
                                          _I, _P, _SZ, _P]),
     "fp4q_quantize_mxfp6": (_I, [_P, _I, _I64, _I64, _I64, _I, _I, _P, _P, _I, _P]),
     "fp4q_gemm_nvfp4": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P, _P]),
+    "fp4q_quantize_if6": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _SZ, _P]),
 }
 
 
@@ -269,6 +271,22 @@ def fp4q_quantize_mxfp6(x: torch.Tensor, fp6_format: int = FP6_E2M3, e8m0_mode: 
     _check("fp4q_quantize_mxfp6", lib().fp4q_quantize_mxfp6(
         _ptr(x), _dtype(x), rows, cols, ld, fp6_format, e8m0_mode, _ptr(out["q"]),
         _ptr(out["sf"]), scale_layout, _stream(dev)))
+    return out
+
+
+def fp4q_quantize_if6(x: torch.Tensor, amax: torch.Tensor | None = None,
+                      scale_layout: int = SCALE_LINEAR, out: dict | None = None) -> dict:
+    """IF6 (FP6 E2M3 or INT6 per 16-block); returns {'s_dec', 'q' [rows, cols*3/4], 'sf'}."""
+    rows, cols, ld = _matrix(x)
+    dev = x.device
+    if out is None:
+        out = {"s_dec": torch.empty(1, dtype=torch.float32, device=dev),
+               "q": _u8((rows, cols * 3 // 4), dev),
+               "sf": _u8(fp4q_scale_bytes(rows, cols, 16, scale_layout), dev)}
+    ws = _workspace(dev) if amax is None else None
+    _check("fp4q_quantize_if6", lib().fp4q_quantize_if6(
+        _ptr(x), _dtype(x), rows, cols, ld, _ptr(amax), _ptr(out.get("s_dec")), _ptr(out["q"]),
+        _ptr(out["sf"]), scale_layout, _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
     return out
 
 

@@ -71,6 +71,15 @@ cudaError_t launch_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float
                               int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
                               int *status, const Launch &L);
 
+// IF6: per 16-value block FP6 E2M3 or INT6 (rescaled by 7.5/31), codes four
+// per three bytes; and its decode
+cudaError_t launch_if6(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                       const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,
+                       int scale_layout, const Launch &L);
+cudaError_t launch_if6_dequant(const uint8_t *q, const uint8_t *sf, int scale_layout,
+                               const float *s_dec, int64_t rows, int64_t cols, void *y,
+                               int y_dtype, const Launch &L);
+
 // int4_mode 1: IF4 (per-block choice); 2: NVINT4 (the INT4 candidate everywhere)
 cudaError_t launch_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                        const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,

@@ -23,7 +23,7 @@ from fp4_block_scaled_04_b200 import workloads
 
 OPS = ["amax", "nvfp4_row", "nvfp4_rowcol", "mxfp4_rowcol", "2d", "rht16_sr", "rht128_sr",
        "rht16_rne", "rht128_rne", "if4", "if4_dequant", "four_over_six_rowcol", "nvint4",
-       "bwd16_sr", "bwd16_rne", "row_sr", "mxfp6_e2m3", "mxfp6_dequant", "gemm_nvfp4"]
+       "bwd16_sr", "bwd16_rne", "row_sr", "mxfp6_e2m3", "mxfp6_dequant", "gemm_nvfp4", "if6"]
 
 
 def make(op: str, rows: int, cols: int, dev):
@@ -64,6 +64,11 @@ def make(op: str, rows: int, cols: int, dev):
         y = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
         return lambda: fq.fp4q_dequantize(fq.FMT_MXFP6_E2M3, o["q"], o["sf"], rows, cols, 1, 32,
                                           scale_layout=sw, out=y)
+    if op == "if6":
+        x = workloads.if4_blocks(rows=rows, cols=cols).to(dev)
+        a = fq.fp4q_amax(x)
+        o = fq.fp4q_quantize_if6(x, amax=a, scale_layout=sw)
+        return lambda: fq.fp4q_quantize_if6(x, amax=a, scale_layout=sw, out=o)
     if op == "nvint4":
         x = workloads.if4_blocks(rows=rows, cols=cols).to(dev)
         a = fq.fp4q_amax(x)

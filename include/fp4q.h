@@ -83,7 +83,8 @@ typedef enum {
   FP4Q_FMT_MXFP4 = 1,
   FP4Q_FMT_IF4 = 2,
   FP4Q_FMT_MXFP6_E2M3 = 3,   /* codes packed four per three bytes */
-  FP4Q_FMT_MXFP6_E3M2 = 4
+  FP4Q_FMT_MXFP6_E3M2 = 4,
+  FP4Q_FMT_IF6 = 5           /* 6-bit codes, four per three bytes */
 } fp4q_format;
 typedef enum { FP4Q_FP6_E2M3 = 0, FP4Q_FP6_E3M2 = 1 } fp4q_fp6_format;
 
@@ -262,6 +263,28 @@ fp4q_status fp4q_quantize_four_over_six(const void *x, int dtype, int64_t rows, 
                                         uint8_t *q_col, uint8_t *sf_col, int scale_layout,
                                         void *workspace, size_t ws_bytes, void *stream);
 
+/* IF6: the IF per-block choice at 6 bits.  "Adaptive Block-Scaled Data
+ * Types" explainer, section 2: each block is quantized to a float grid and to
+ * a scaled integer grid, the smaller squared error wins, the scale's sign bit
+ * records the choice, and the idea extends to 6 bits.  The library's reading:
+ * FP6 E2M3 (largest 7.5; "FP6で隣り合う値の間隔を見てみる") against INT6
+ * (-31..31) rescaled by 7.5/31, with NVFP4's scaling at 7.5 in place of 6:
+ *   s_enc = RN(3360/amax), s_dec = RN(amax/3360)       (3360 = 7.5 * 448)
+ *   S = E4M3_rne_sat(RN(RN(m * s_enc) / 7.5)), r = RN(s_enc / S), v = RN(x*r)
+ *   FP6:  E2M3 round to nearest even with saturation, sign copied
+ *   INT6: k = clamp(rint(RN(v * RN(31/7.5))), -31, 31), value RN(k * RN(7.5/31))
+ *   errors sum fma(d, d, e) over the block in order, d = RN(v - value);
+ *   INT6 iff its error is strictly smaller; scale bit 7 set = INT6.
+ *   q   [rows, cols * 3/4] bytes: four 6-bit codes per three bytes as in
+ *       fp4q_quantize_mxfp6 (the E2M3 code, or k in 6-bit two's complement)
+ *   sf  [rows, cols/16] flagged E4M3 scales in scale_layout
+ * amax, tensor_scale_out, workspace and errors as for fp4q_quantize_if4;
+ * shape cols % 16 == 0.  fp4q_dequantize(FP4Q_FMT_IF6, ..., 1, 16, s_dec, ...)
+ * decodes it: y = RN(RN(value * S) * s_dec). */
+fp4q_status fp4q_quantize_if6(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                              const float *amax, float *tensor_scale_out, uint8_t *q, uint8_t *sf,
+                              int scale_layout, void *workspace, size_t ws_bytes, void *stream);
+
 /* MXFP6 1x32, row-wise: the OCP FP6 element formats with E8M0 block scales.
  * "FP6から考えるLLM量子化" (blog.ast.moe), "FP6で隣り合う値の間隔を見てみる":
  * E2M3 (sign, 2 exponent bits with bias 1, 3 mantissa bits; largest 7.5)
@@ -329,9 +352,11 @@ fp4q_status fp4q_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *
  *   MXFP4  y = g * 2^(scale - 127)             block 1x32
  *   MXFP6  y = RN(g * 2^(scale - 127))         block 1x32; q is [rows,
  *          cols * 3/4] bytes packed as fp4q_quantize_mxfp6 writes them
- *   block_rows x block_cols: 1x16 (NVFP4, IF4), 16x16 (NVFP4 2D tiles; then
+ *   IF6    y = RN(RN(value * S) * s_dec)        block 1x16, 6-bit codes as
+ *          fp4q_quantize_if6 writes them (INT6 blocks: value = RN(k * RN(7.5/31)))
+ *   block_rows x block_cols: 1x16 (NVFP4, IF4, IF6), 16x16 (NVFP4 2D tiles; then
  *   sf is the linear [rows/16, cols/16] tile matrix), 1x32 (MXFP4, MXFP6).
- *   tensor_scale: device float s_dec (NVFP4 / IF4), ignored for MXFP4/6.
+ *   tensor_scale: device float s_dec (NVFP4 / IF4 / IF6), ignored for MXFP4/6.
  *   Column-wise outputs are dequantized as the [cols, rows] matrices they are.
  * Shape: cols % block_cols == 0, rows % block_rows == 0. */
 fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,
