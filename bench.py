@@ -287,6 +287,7 @@ def build_extra_jobs(device, fq, inputs):
     its value: the fused backward call and the row-wise operand alone on the
     gradient workload, and the IF4 explainer's comparison formats
     (four-over-six on the activation workload, NVINT4 on the IF4 workload),
+    the tensor amax of the activation workload (which the suite takes as given),
     IF6 on the IF4 workload and MXFP6 E2M3 on the activation workload."""
     import torch
     SW = fq.SCALE_SWIZZLED
@@ -342,6 +343,8 @@ def build_extra_jobs(device, fq, inputs):
                                                    out=o46)),
         Job("if4 16384x8192 bf16 nvint4", "if4.cu", nbi4, 1,
             lambda: fq.fp4q_quantize_nvint4(x5, amax=amax5, scale_layout=SW, out=oi4)),
+        Job("activation 8192x4096 bf16 tensor amax", "amax.cu", R * C * 2 + 4, 1,
+            lambda: fq.fp4q_amax(xa, out=amax_a)),
         Job("if4 16384x8192 bf16 if6", "if6.cu", nbi6, 1,
             lambda: fq.fp4q_quantize_if6(x5, amax=amax5, scale_layout=SW, out=oi6)),
         Job("activation 8192x4096 bf16 mxfp6 e2m3 row-wise", "mxfp6.cu", nb6, 1,

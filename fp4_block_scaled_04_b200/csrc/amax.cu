@@ -22,54 +22,60 @@ __device__ __forceinline__ void block_max_to_global(uint32_t m, unsigned *out) {
   }
 }
 
-// BF16: 8 elements per 16-byte chunk; the max of the 16-bit |x| patterns,
-// shifted into FP32 position, is the FP32 bit pattern of the amax.
+// The 16-byte chunk idx of a [rows, cols] matrix with row stride ld: a flat
+// offset when the rows are contiguous (FLAT, no division), else row idx / cpr.
+template <int PER, bool FLAT, typename I>
+__device__ __forceinline__ const uint4 *chunk_ptr(const void *x, I idx, I cpr, I ld) {
+  const I off = FLAT ? idx * PER : (idx / cpr) * ld + (idx % cpr) * PER;
+  return reinterpret_cast<const uint4 *>(static_cast<const char *>(x) +
+                                         static_cast<int64_t>(off) * (16 / PER));
+}
+
+constexpr int kUnroll = 4;                         // 16-byte loads in flight per thread
+
+// BF16 (PER = 8 elements per chunk): the max of the 16-bit |x| patterns in
+// two lanes, shifted into FP32 position, is the FP32 bit pattern of the amax.
+// FP32 (PER = 4): the max of the 32-bit |x| patterns.
+template <int PER, bool FLAT, typename I>
 __global__ void __launch_bounds__(kThreads)
-amax_bf16_kernel(const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-                 unsigned *__restrict__ out) {
-  const int64_t cpr = cols / 8, total = rows * cpr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  uint32_t acc = 0;  // two 16-bit lanes
-  int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-  for (; i + stride < total; i += 2 * stride) {
-    int64_t r0 = i / cpr, r1 = (i + stride) / cpr;
-    uint4 a = __ldg(reinterpret_cast<const uint4 *>(x + r0 * ld + (i - r0 * cpr) * 8));
-    uint4 b = __ldg(reinterpret_cast<const uint4 *>(x + r1 * ld + (i + stride - r1 * cpr) * 8));
-    acc = __vmaxu2(acc, a.x & 0x7FFF7FFFu); acc = __vmaxu2(acc, a.y & 0x7FFF7FFFu);
-    acc = __vmaxu2(acc, a.z & 0x7FFF7FFFu); acc = __vmaxu2(acc, a.w & 0x7FFF7FFFu);
-    acc = __vmaxu2(acc, b.x & 0x7FFF7FFFu); acc = __vmaxu2(acc, b.y & 0x7FFF7FFFu);
-    acc = __vmaxu2(acc, b.z & 0x7FFF7FFFu); acc = __vmaxu2(acc, b.w & 0x7FFF7FFFu);
+amax_kernel(const void *__restrict__ x, I rows, I cols, I ld, unsigned *__restrict__ out) {
+  const I cpr = cols / PER, total = rows * cpr;
+  const I stride = static_cast<I>(gridDim.x) * kThreads;
+  uint32_t acc = 0;
+  for (I i = static_cast<I>(blockIdx.x) * kThreads + threadIdx.x; i < total;
+       i += kUnroll * stride) {
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int j = 0; j < kUnroll; ++j) {
+      const I idx = i + j * stride;
+      v[j] = idx < total ? __ldg(chunk_ptr<PER, FLAT, I>(x, idx, cpr, ld)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < kUnroll; ++j) {
+      if (PER == 8) {
+        acc = __vmaxu2(acc, v[j].x & 0x7FFF7FFFu); acc = __vmaxu2(acc, v[j].y & 0x7FFF7FFFu);
+        acc = __vmaxu2(acc, v[j].z & 0x7FFF7FFFu); acc = __vmaxu2(acc, v[j].w & 0x7FFF7FFFu);
+      } else {
+        acc = max(acc, max(max(v[j].x & 0x7FFFFFFFu, v[j].y & 0x7FFFFFFFu),
+                           max(v[j].z & 0x7FFFFFFFu, v[j].w & 0x7FFFFFFFu)));
+      }
+    }
   }
-  if (i < total) {
-    int64_t r0 = i / cpr;
-    uint4 a = __ldg(reinterpret_cast<const uint4 *>(x + r0 * ld + (i - r0 * cpr) * 8));
-    acc = __vmaxu2(acc, a.x & 0x7FFF7FFFu); acc = __vmaxu2(acc, a.y & 0x7FFF7FFFu);
-    acc = __vmaxu2(acc, a.z & 0x7FFF7FFFu); acc = __vmaxu2(acc, a.w & 0x7FFF7FFFu);
-  }
-  uint32_t m = max(acc & 0xFFFFu, acc >> 16) << 16;
+  const uint32_t m = PER == 8 ? max(acc & 0xFFFFu, acc >> 16) << 16 : acc;
   block_max_to_global(m, out);
 }
 
-__global__ void __launch_bounds__(kThreads)
-amax_f32_kernel(const uint32_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-                unsigned *__restrict__ out) {
-  const int64_t cpr = cols / 4, total = rows * cpr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  uint32_t m = 0;
-  int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-  for (; i + stride < total; i += 2 * stride) {
-    int64_t r0 = i / cpr, r1 = (i + stride) / cpr;
-    uint4 a = __ldg(reinterpret_cast<const uint4 *>(x + r0 * ld + (i - r0 * cpr) * 4));
-    uint4 b = __ldg(reinterpret_cast<const uint4 *>(x + r1 * ld + (i + stride - r1 * cpr) * 4));
-    m = max(m, max(max(a.x & 0x7FFFFFFFu, a.y & 0x7FFFFFFFu), max(a.z & 0x7FFFFFFFu, a.w & 0x7FFFFFFFu)));
-    m = max(m, max(max(b.x & 0x7FFFFFFFu, b.y & 0x7FFFFFFFu), max(b.z & 0x7FFFFFFFu, b.w & 0x7FFFFFFFu)));
-  }
-  if (i < total) {
-    int64_t r0 = i / cpr;
-    uint4 a = __ldg(reinterpret_cast<const uint4 *>(x + r0 * ld + (i - r0 * cpr) * 4));
-    m = max(m, max(max(a.x & 0x7FFFFFFFu, a.y & 0x7FFFFFFFu), max(a.z & 0x7FFFFFFFu, a.w & 0x7FFFFFFFu)));
-  }
-  block_max_to_global(m, out);
+template <int PER, bool FLAT>
+void launch_k(const void *x, int64_t rows, int64_t cols, int64_t ld, unsigned *out, int grid,
+              const Launch &L) {
+  // 32-bit indices when every chunk index and offset a step can reach fits
+  const int64_t reach = rows * (ld > cols ? ld : cols) + int64_t{kUnroll} * grid * kThreads * PER;
+  if (reach < (int64_t{1} << 31))
+    amax_kernel<PER, FLAT, uint32_t><<<grid, kThreads, 0, L.stream>>>(
+        x, static_cast<uint32_t>(rows), static_cast<uint32_t>(cols), static_cast<uint32_t>(ld),
+        out);
+  else
+    amax_kernel<PER, FLAT, int64_t><<<grid, kThreads, 0, L.stream>>>(x, rows, cols, ld, out);
 }
 
 }  // namespace
@@ -78,18 +84,20 @@ cudaError_t launch_amax(const void *x, int dtype, int64_t rows, int64_t cols, in
                         float *amax_out, const Launch &L) {
   cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), L.stream);
   if (e != cudaSuccess) return e;
-  const int64_t chunks = rows * cols / (dtype == FP4Q_BF16 ? 8 : 4);
-  int64_t want = (chunks + 2 * kThreads - 1) / (2 * kThreads);
-  int64_t cap = static_cast<int64_t>(L.num_sms) * 8;
-  int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-  if (dtype == FP4Q_BF16)
-    amax_bf16_kernel<<<grid, kThreads, 0, L.stream>>>(static_cast<const uint16_t *>(x), rows,
-                                                      cols, ld,
-                                                      reinterpret_cast<unsigned *>(amax_out));
-  else
-    amax_f32_kernel<<<grid, kThreads, 0, L.stream>>>(static_cast<const uint32_t *>(x), rows,
-                                                     cols, ld,
-                                                     reinterpret_cast<unsigned *>(amax_out));
+  const int per = dtype == FP4Q_BF16 ? 8 : 4;
+  const int64_t chunks = rows * cols / per;
+  const int64_t want = (chunks + kUnroll * kThreads - 1) / (kUnroll * kThreads);
+  const int64_t cap = static_cast<int64_t>(L.num_sms) * 8;
+  const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+  unsigned *out = reinterpret_cast<unsigned *>(amax_out);
+  const bool flat = ld == cols || rows == 1;
+  if (dtype == FP4Q_BF16) {
+    if (flat) launch_k<8, true>(x, rows, cols, ld, out, grid, L);
+    else launch_k<8, false>(x, rows, cols, ld, out, grid, L);
+  } else {
+    if (flat) launch_k<4, true>(x, rows, cols, ld, out, grid, L);
+    else launch_k<4, false>(x, rows, cols, ld, out, grid, L);
+  }
   return cudaGetLastError();
 }
 

@@ -89,6 +89,19 @@ def test_amax_strided_input(orc):
     assert_same("amax", host(got), np.array([orc.amax(bits(x))], np.float32))
 
 
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("where", ["first", "last", "middle"])
+def test_amax_position_and_stride(orc, dtype, where):
+    """The maximum in the first, last or a middle chunk, for a contiguous
+    tensor spanning several grid-stride steps and for a strided view."""
+    base = randmat(2304, 640, dtype, seed=3, scale_spread=False)
+    pos = {"first": (0, 0), "last": (2303, 639), "middle": (1151, 333)}[where]
+    base[pos] = -1000.0
+    for x in (base, base[:, 64:576]):
+        got = fq.fp4q_amax(x.to(DEV) if x is base else base.to(DEV)[:, 64:576])
+        assert_same("amax", host(got), np.array([orc.amax(bits(x))], np.float32))
+
+
 # ------------------------------------------------------------------ NVFP4
 
 @pytest.mark.parametrize("dtype", DTYPES)
