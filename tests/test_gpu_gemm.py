@@ -52,7 +52,10 @@ def check(orc, qa, sfa, qb, sfb, M, N, K, c, alpha=1.0, out_bits=24):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 128, 512), (128, 384, 1024),
-                                   (384, 256, 768), (256, 256, 4096)])
+                                   (384, 256, 768), (256, 256, 4096),
+                                   # M and N multiples of 256: the two-SM (cluster) kernel
+                                   (256, 512, 512), (512, 256, 1024), (768, 768, 256),
+                                   (1024, 1024, 2048)])
 def test_gemm_random_codes_and_scales(orc, M, N, K):
     qa, sfa = random_operand(M, K, 1)
     qb, sfb = random_operand(N, K, 2)
@@ -64,10 +67,12 @@ def test_gemm_random_codes_and_scales(orc, M, N, K):
     check(orc, qa, sfa, qb, sfb, M, N, K, host(c))
 
 
-def test_gemm_one_hot_selects_columns(orc):
+@pytest.mark.parametrize("M,N", [(256, 128), (512, 256)])
+def test_gemm_one_hot_selects_columns(orc, M, N):
     """B rows one-hot at 1.0: C is a column selection of dequantized A, which
-    every FP32 order computes exactly."""
-    M, N, K = 256, 128, 512
+    every FP32 order computes exactly (both kernels: N = 128 and the two-SM
+    form)."""
+    K = 512
     qa, sfa = random_operand(M, K, 3)
     rng = np.random.default_rng(4)
     kn = rng.permutation(K)[:N]
@@ -90,7 +95,7 @@ def quantized(x):
 def test_fprop_from_quantized_activations_and_weights(orc, out_dtype):
     """Fprop: X [M, K] and W [N, K] through fp4q_quantize_nvfp4 (row-wise,
     swizzled scales), then C = s_x s_w (X_q W_q^T)."""
-    M, N, K = 256, 384, 1024
+    M, N, K = (256, 384, 1024) if out_dtype == torch.bfloat16 else (512, 512, 1024)
     g = torch.Generator().manual_seed(11)
     x = (torch.randn(M, K, generator=g) * 3).to(torch.bfloat16).to(DEV)
     w = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16).to(DEV)
