@@ -383,301 +383,6 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
                  : "memory");
 }
 
-// ---------------------------------------------------------------------------
-// The pair form: two CTAs of a cluster (two SMs) share one 256 x 256 output
-// tile through tcgen05.mma.cta_group::2 (M = 256: each CTA holds 128 rows of A
-// and, in its tensor memory, the accumulator of those rows; N = 256: each CTA
-// holds 128 rows of B, and the MMA reads both halves).  Each SM then moves a
-// third fewer bytes per FLOP than with 128 x 256 tiles.
-//  - both CTAs' producers load their own A and B halves, the scales of their
-//    A rows and the scales of all 256 B rows (the MMA reads B scales for the
-//    whole N = 256 from each CTA's tensor memory) with TMA (.cta_group::2, no
-//    multicast), completing on the leader CTA's "full" barrier, which only the
-//    leader's producer arms with both CTAs' bytes;
-//  - the leader's MMA thread copies both CTAs' scale tiles into their tensor
-//    memory (tcgen05.cp.cta_group::2) and issues the MMAs; its commits are
-//    multicast to the "empty" and "acc_full" barriers of both CTAs;
-//  - the epilogue warps of both CTAs read their own accumulator rows and
-//    arrive on the leader's "acc_empty" barrier (8 arrivals per tile).
-// Both CTAs allocate tensor memory together (tcgen05.alloc.cta_group::2) and
-// free it after a cluster barrier.
-// ---------------------------------------------------------------------------
-namespace pair {
-
-constexpr int BM = 256, BN = 256;                 // per cluster
-constexpr int HALF = 128;                         // rows of A and of B per CTA
-constexpr int STAGES = 5;
-constexpr int A_BYTES = HALF * KTB;               // 16384
-constexpr int B_BYTES = HALF * KTB;               // 16384
-constexpr int SFB_BYTES = 2 * SF_BYTES;           // both 128-row halves of B
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES + SFB_BYTES;   // 38912
-constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-constexpr uint32_t SF_COL0 = BN;                  // accumulator columns [0, 256)
-constexpr uint32_t STAGE_COLS = 48;               // 16 A-scale + 32 B-scale columns
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
-                           (uint32_t(BM >> 4) << 24);
-static_assert(BN + STAGES * STAGE_COLS <= TMEM_COLS, "tensor memory");
-static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
-static_assert(SMEM_BYTES <= 232448, "shared memory");
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// the shared::cluster address of the same variable in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-__device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_test_cluster(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return false;
-  return true;
-}
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                                 uint32_t leader_bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(leader_bar)
-      : "memory");
-}
-__device__ __forceinline__ void tc_copy_sf_pair(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
-__device__ __forceinline__ void tc_mma_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t sfa,
-                                            uint32_t sfb, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
-      "[%6], p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(IDESC), "r"(accumulate), "r"(sfa), "r"(sfb)
-      : "memory");
-}
-// arrive on the barrier at this offset in both CTAs of the pair
-__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
-      "[%0], %1;" ::"r"(bar),
-      "h"(static_cast<uint16_t>(3))
-      : "memory");
-}
-
-template <typename OutT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap map_a,
-                       const __grid_constant__ CUtensorMap map_b,
-                       const __grid_constant__ CUtensorMap map_sfa,
-                       const __grid_constant__ CUtensorMap map_sfb, const float *__restrict__ s_a,
-                       const float *__restrict__ s_b, int K, int n_tiles_n, int n_tiles,
-                       OutT *__restrict__ c, int64_t ldc, int *__restrict__ status) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t full = base + STAGES * STAGE_BYTES;
-  const uint32_t empty = full + 8 * STAGES;
-  const uint32_t acc_full = empty + 8 * STAGES;
-  const uint32_t acc_empty = acc_full + 8;
-  const uint32_t tmem_slot = acc_empty + 8;
-  const uint32_t err_slot = tmem_slot + 4;
-  volatile uint32_t *slot_ptr = reinterpret_cast<volatile uint32_t *>(smem_raw + (tmem_slot - raw));
-  volatile int *err_ptr = reinterpret_cast<volatile int *>(smem_raw + (err_slot - raw));
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = cluster_rank();
-  const int cluster = blockIdx.x / 2, n_clusters = gridDim.x / 2;
-  const int KT = K / KTILE;
-  const int sf_rows_per_tile = (K / 64) * SF_TILE / 256;   // 256-byte rows of one 128-row tile
-
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     tmem_slot),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-  }
-  if (tid == 0) {
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(full + 8 * i, 1);
-      mbar_init(empty + 8 * i, 1);
-    }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 8);                    // 4 epilogue warps in each CTA
-    *err_ptr = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();                               // the leader's barriers exist before use
-  tc_fence_after();
-  const uint32_t tmem = *slot_ptr;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---- producer (both CTAs): this CTA's halves of A and B ----
-      int g = 0;
-      for (int tile = cluster; tile < n_tiles && !*err_ptr; tile += n_clusters) {
-        const int m0 = (tile / n_tiles_n) * BM + HALF * rank;
-        const int n0 = (tile % n_tiles_n) * BN + HALF * rank;
-        for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int s = g % STAGES;
-          if (g >= STAGES &&
-              !mbar_wait(empty + 8 * s, static_cast<uint32_t>((g / STAGES - 1) & 1))) {
-            *err_ptr = 1;
-            break;
-          }
-          const uint32_t st = base + s * STAGE_BYTES;
-          const uint32_t bar = peer_addr(full + 8 * s, 0);
-          if (rank == 0) mbar_expect_tx(full + 8 * s, 2 * STAGE_BYTES);
-          tma_load_2d_pair(st, &map_a, kt * KTB, m0, bar);
-          tma_load_2d_pair(st + A_BYTES, &map_b, kt * KTB, n0, bar);
-          tma_load_2d_pair(st + A_BYTES + B_BYTES, &map_sfa, 0,
-                           (m0 / 128) * sf_rows_per_tile + kt * (SF_BYTES / 256), bar);
-          const int nb = (tile % n_tiles_n) * (BN / 128);     // first 128-row tile of B
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            tma_load_2d_pair(st + A_BYTES + B_BYTES + SF_BYTES + h * SF_BYTES, &map_sfb, 0,
-                             (nb + h) * sf_rows_per_tile + kt * (SF_BYTES / 256), bar);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
-      // ---- tensor-core issue (leader only) ----
-      int g = 0, i = 0;
-      for (int tile = cluster; tile < n_tiles && !*err_ptr; tile += n_clusters, ++i) {
-        if (i > 0 && !mbar_wait_cluster(acc_empty, static_cast<uint32_t>((i - 1) & 1))) {
-          *err_ptr = 1;
-          break;
-        }
-        tc_fence_after();
-        for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int s = g % STAGES;
-          if (!mbar_wait(full + 8 * s, static_cast<uint32_t>((g / STAGES) & 1))) {
-            *err_ptr = 1;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t st = base + s * STAGE_BYTES;
-          const uint32_t sfa_col = tmem + SF_COL0 + STAGE_COLS * s, sfb_col = sfa_col + 16u;
-#pragma unroll
-          for (int kb = 0; kb < KTILE / 64; ++kb) {
-            tc_copy_sf_pair(sfa_col + 4u * kb, desc_sf(st + A_BYTES + B_BYTES + kb * SF_TILE));
-#pragma unroll
-            for (int h = 0; h < 2; ++h)        // B rows 128h .. 128h + 127: columns 4h .. 4h + 3
-              tc_copy_sf_pair(sfb_col + 8u * kb + 4u * h,
-                              desc_sf(st + A_BYTES + B_BYTES + SF_BYTES + h * SF_BYTES +
-                                      kb * SF_TILE));
-          }
-          const uint64_t da = desc_sw128(st), db = desc_sw128(st + A_BYTES);
-#pragma unroll
-          for (int kb = 0; kb < KTILE / 64; ++kb)
-            tc_mma_pair(tmem, da + 2u * kb, db + 2u * kb, sfa_col + 4u * kb, sfb_col + 8u * kb,
-                        (kt | kb) != 0);
-          tc_commit_pair(empty + 8 * s);
-        }
-        tc_commit_pair(acc_full);
-      }
-    }
-  } else {
-    // ---- epilogue (both CTAs): this CTA's 128 accumulator rows ----
-    const int quarter = warp & 3;
-    const float alpha = __fmul_rn(s_a ? *s_a : 1.0f, s_b ? *s_b : 1.0f);
-    const uint32_t leader_acc_empty = peer_addr(acc_empty, 0);
-    int i = 0;
-    for (int tile = cluster; tile < n_tiles; tile += n_clusters, ++i) {
-      const int ok = mbar_wait_cluster(acc_full, static_cast<uint32_t>(i & 1)) ? 1 : 0;
-      if (!__all_sync(0xFFFFFFFFu, ok)) {
-        *err_ptr = 1;
-        break;
-      }
-      tc_fence_after();
-      const int m0 = (tile / n_tiles_n) * BM + HALF * rank, n0 = (tile % n_tiles_n) * BN;
-      OutT *row = c + (static_cast<int64_t>(m0) + quarter * 32 + lane) * ldc + n0;
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-      if (sizeof(OutT) == 2) {
-        uint32_t w[BN / 2];
-#pragma unroll
-        for (int j = 0; j < BN / 16; ++j) {
-          uint32_t r[16];
-          tc_load16(taddr + 16u * j, r);
-          tc_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * q]), alpha),
-                                                      __fmul_rn(__uint_as_float(r[2 * q + 1]), alpha));
-            memcpy(&w[8 * j + q], &b2, sizeof(uint32_t));
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0)
-          asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                           leader_acc_empty)
-                       : "memory");
-        uint4 *d = reinterpret_cast<uint4 *>(row);
-#pragma unroll
-        for (int q = 0; q < BN / 8; ++q) d[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-      } else {
-        float4 *d = reinterpret_cast<float4 *>(row);
-#pragma unroll
-        for (int j = 0; j < BN / 16; ++j) {
-          uint32_t r[16];
-          tc_load16(taddr + 16u * j, r);
-          tc_wait_ld();
-          if (j == BN / 16 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-              asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                               leader_acc_empty)
-                           : "memory");
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            d[4 * j + q] = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), alpha),
-                                       __fmul_rn(__uint_as_float(r[4 * q + 1]), alpha),
-                                       __fmul_rn(__uint_as_float(r[4 * q + 2]), alpha),
-                                       __fmul_rn(__uint_as_float(r[4 * q + 3]), alpha));
-        }
-      }
-    }
-  }
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();                               // the pair's MMAs and reads are over
-  if (tid == 0 && status && *err_ptr) atomicExch(status, 1);
-  if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(TMEM_COLS)
-                 : "memory");
-}
-
-}  // namespace pair
-
 // cuTensorMapEncodeTiled, reached through the runtime (no link to the driver
 // library)
 PFN_cuTensorMapEncodeTiled_v12000 encoder() {
@@ -708,69 +413,6 @@ bool make_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t row_b
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(base), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// The scale bytes of a [rows, K/16] swizzled scale matrix seen as rows of 256
-// bytes; one K-tile of one 128-row tile is a box of 8 such rows (2 KiB).
-bool make_sf_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t K) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
-  if (!enc) return false;
-  const int64_t bytes = rows * (K / 16);
-  const cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(bytes / 256)};
-  const cuuint64_t strides[1] = {256};
-  const cuuint32_t box[2] = {256, static_cast<cuuint32_t>(SF_BYTES / 256)};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(base), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <typename OutT>
-cudaError_t launch_pair(const uint8_t *qa, const uint8_t *sfa, const float *s_a,
-                        const uint8_t *qb, const uint8_t *sfb, const float *s_b, int64_t M,
-                        int64_t N, int64_t K, void *c, int64_t ldc, int *status, const Launch &L) {
-  static bool configured[64] = {};
-  static int max_clusters[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(pair::gemm_nvfp4_pair_kernel<OutT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         pair::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    // how many pairs fit at once (a persistent grid must not exceed it)
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (L.num_sms / 2));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = pair::SMEM_BYTES;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 2;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, pair::gemm_nvfp4_pair_kernel<OutT>, &cfg);
-    if (e != cudaSuccess || n < 1) {
-      cudaGetLastError();
-      n = L.num_sms / 2 > 1 ? L.num_sms / 2 - 4 : 1;
-    }
-    max_clusters[dev] = n;
-    configured[dev] = true;
-  }
-  CUtensorMap map_a, map_b, map_sfa, map_sfb;
-  if (!make_map(&map_a, qa, M, K / 2, pair::HALF) || !make_map(&map_b, qb, N, K / 2, pair::HALF) ||
-      !make_sf_map(&map_sfa, sfa, M, K) || !make_sf_map(&map_sfb, sfb, N, K))
-    return cudaErrorInvalidValue;
-  const int64_t n_tiles_n = N / pair::BN, n_tiles = (M / pair::BM) * n_tiles_n;
-  const int64_t clusters = n_tiles < max_clusters[dev] ? n_tiles : max_clusters[dev];
-  pair::gemm_nvfp4_pair_kernel<OutT><<<static_cast<unsigned>(2 * clusters), kThreads,
-                                       pair::SMEM_BYTES, L.stream>>>(
-      map_a, map_b, map_sfa, map_sfb, s_a, s_b, static_cast<int>(K), static_cast<int>(n_tiles_n),
-      static_cast<int>(n_tiles), static_cast<OutT *>(c), ldc, status);
-  return cudaGetLastError();
 }
 
 template <typename OutT, int BN>
@@ -804,8 +446,6 @@ template <typename OutT>
 cudaError_t launch_o(const uint8_t *qa, const uint8_t *sfa, const float *s_a, const uint8_t *qb,
                      const uint8_t *sfb, const float *s_b, int64_t M, int64_t N, int64_t K,
                      void *c, int64_t ldc, int *status, const Launch &L) {
-  if (M % 256 == 0 && N % 256 == 0)
-    return launch_pair<OutT>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, L);
   if (N % 256 == 0)
     return launch_t<OutT, 256>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, L);
   return launch_t<OutT, 128>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, L);
