@@ -146,3 +146,54 @@ def test_gemm_rejects_ragged_shapes():
     q2 = torch.zeros((96, 128), dtype=torch.uint8, device=DEV)
     with pytest.raises(fq.Fp4qError):
         fq.fp4q_gemm_nvfp4(q2, s, q, s, 256)            # M % 128
+
+
+def test_dgrad_from_the_backward_call(orc):
+    """Dgrad = dY W: A is the row-wise dY from fp4q_quantize_backward (the
+    contraction runs over the output features), B is the column-wise copy of
+    W [N_out, K_in], i.e. W^T [K_in, N_out] row-wise."""
+    T, Nout, Kin = 256, 512, 384
+    g = torch.Generator().manual_seed(13)
+    dy = (torch.randn(T, Nout, generator=g) * 1e-3).to(torch.bfloat16).to(DEV)
+    w = (torch.randn(Nout, Kin, generator=g) * 0.02).to(torch.bfloat16).to(DEV)
+    sw = fq.SCALE_SWIZZLED
+    ob = fq.fp4q_quantize_backward(dy, 16, round=fq.SR, seed_row=5, seed_col=6, scale_layout=sw)
+    ow = fq.fp4q_quantize_nvfp4(w, layouts=fq.COLWISE, scale_layout=sw)
+    c = fq.fp4q_gemm_nvfp4(ob["q_row"], ob["sf_row"], ow["q_col"], ow["sf_col"], Nout,
+                           tensor_scale_a=ob["s_dec_row"], tensor_scale_b=ow["s_dec"])
+    alpha = float(np.float32(ob["s_dec_row"].item()) * np.float32(ow["s_dec"].item()))
+    check(orc, host(ob["q_row"]), host(ob["sf_row"]), host(ow["q_col"]), host(ow["sf_col"]),
+          T, Kin, Nout, host(c), alpha=alpha)
+    # and it estimates the unquantized product
+    ref = (dy.float() @ w.float()).cpu().numpy().astype(np.float64)
+    rel = np.linalg.norm(host(c) - ref) / np.linalg.norm(ref)
+    assert rel < 0.3, rel                # about 0.17 from NVFP4 and SR noise
+
+
+@pytest.mark.parametrize("n", [16, 128])
+def test_wgrad_from_rht_operands_with_the_same_signs(orc, n):
+    """Qiita note, "ランダムアダマール変換": Wgrad multiplies the transformed
+    dY^T and X^T; with the same random signs the transform cancels
+    ((H S dY)^T (H S X) c^2 = dY^T X), so the GEMM of the two RHT outputs
+    estimates dY^T X."""
+    T, Co, Ci = 512, 128, 256
+    g = torch.Generator().manual_seed(14)
+    dy = (torch.randn(T, Co, generator=g) * 1e-3).to(torch.bfloat16).to(DEV)
+    x = torch.randn(T, Ci, generator=g).to(torch.bfloat16).to(DEV)
+    sw = fq.SCALE_SWIZZLED
+    od = fq.fp4q_quantize_rht_sr(dy, n, round=fq.SR, seed=21, scale_layout=sw)
+    ox = fq.fp4q_quantize_rht_sr(x, n, round=fq.SR, seed=21, scale_layout=sw)
+    c = fq.fp4q_gemm_nvfp4(od["q_t"], od["sf_t"], ox["q_t"], ox["sf_t"], T,
+                           tensor_scale_a=od["s_dec"], tensor_scale_b=ox["s_dec"])
+    alpha = float(np.float32(od["s_dec"].item()) * np.float32(ox["s_dec"].item()))
+    check(orc, host(od["q_t"]), host(od["sf_t"]), host(ox["q_t"]), host(ox["sf_t"]),
+          Co, Ci, T, host(c), alpha=alpha)
+    ref = (dy.float().t() @ x.float()).cpu().numpy().astype(np.float64)
+    rel = np.linalg.norm(host(c) - ref) / np.linalg.norm(ref)
+    assert rel < 0.3, rel                # about 0.2 from NVFP4 and SR noise
+    # with different signs the transform does not cancel
+    ox2 = fq.fp4q_quantize_rht_sr(x, n, round=fq.SR, seed=22, scale_layout=sw)
+    c2 = fq.fp4q_gemm_nvfp4(od["q_t"], od["sf_t"], ox2["q_t"], ox2["sf_t"], T,
+                            tensor_scale_a=od["s_dec"], tensor_scale_b=ox2["s_dec"])
+    rel2 = np.linalg.norm(host(c2) - ref) / np.linalg.norm(ref)
+    assert rel2 > 1.0, rel2              # about 1.5: uncorrelated with dY^T X
