@@ -385,8 +385,7 @@ __device__ __forceinline__ float e2m1_sr_value(float v, uint32_t z) {
   const float r = __fsub_rn(__uint_as_float((__float_as_uint(w) + z) & 0xFFC00000u), a);
   return __uint_as_float(__float_as_uint(r) | (__float_as_uint(v) & 0x80000000u));
 }
-// z of a 16-bit uniform, and of the low / high 16-bit uniform of a 32-bit word
-__device__ __forceinline__ uint32_t sr_z(uint32_t u16) { return 0x3FFFFFu ^ (u16 << 6); }
+// z of the low / high 16-bit uniform of a 32-bit word
 __device__ __forceinline__ uint32_t sr_z_lo(uint32_t w) { return 0x3FFFFFu ^ ((w << 6) & 0x3FFFC0u); }
 __device__ __forceinline__ uint32_t sr_z_hi(uint32_t w) { return 0x3FFFFFu ^ ((w >> 10) & 0x3FFFC0u); }
 
