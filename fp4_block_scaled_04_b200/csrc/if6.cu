@@ -18,6 +18,9 @@
 // bytes (code j of a group in bits 6j..6j+5), so a block is 12 bytes.
 // Quantize: one thread per block, 32 or 64 bytes in, three 4-byte code stores
 // and a scale byte out; r comes from a per-CTA table over the 128 scale codes.
+// Exact shortcuts (as in IF4): rint by adding and subtracting 1.5 * 2^23, whose
+// bits also carry the INT6 code, packed by multiply-add; FP6 errors by a
+// mixed-precision subtract from the decoded f16 grid values.
 // Dequantize: one thread per block, y = RN(RN(q * S) * s_dec) with q the E2M3
 // value or h.
 #include <cuda_fp16.h>
@@ -46,6 +49,35 @@ __device__ __forceinline__ float2 e2m3x2_value(uint32_t two_codes) {
   __half2 v;
   memcpy(&v, &h, sizeof(v));
   return __half22float2(v);
+}
+
+constexpr float kMagic = 12582912.0f;             // 1.5 * 2^23: RN(t + kMagic) - kMagic = rint(t)
+// bits(RN(t + kMagic)) = 0x4B400000 + rint(t); four such words summed with
+// weights 64^i, minus this, give sum of (rint(t_i) + 32) 64^i
+constexpr uint32_t kGroupBias = (0x4B400000u - 32u) * (1u + 64u + 4096u + 262144u);
+
+// Four values to FP6 E2M3 codes (one per byte, value order) and the
+// differences d = RN(g - v) from their grid values g (exact in f16; the
+// square equals that of RN(v - g)), subtracted in mixed precision.
+__device__ __forceinline__ uint32_t e2m3x4_codes_diffs(const float (&v)[4], float (&d)[4]) {
+  uint32_t w;
+  asm("{\n\t.reg .b16 p0, p1;\n\t.reg .b32 h0, h1;\n\t.reg .f16 g0, g1, g2, g3;\n\t"
+      "cvt.rn.satfinite.e2m3x2.f32 p0, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m3x2.f32 p1, %8, %7;\n\t"
+      "and.b16 p0, p0, 0x3F3F;\n\t"
+      "and.b16 p1, p1, 0x3F3F;\n\t"
+      "mov.b32 %0, {p0, p1};\n\t"
+      "cvt.rn.f16x2.e2m3x2 h0, p0;\n\t"
+      "cvt.rn.f16x2.e2m3x2 h1, p1;\n\t"
+      "mov.b32 {g0, g1}, h0;\n\t"
+      "mov.b32 {g2, g3}, h1;\n\t"
+      "sub.rn.f32.f16 %1, g0, %5;\n\t"
+      "sub.rn.f32.f16 %2, g1, %6;\n\t"
+      "sub.rn.f32.f16 %3, g2, %7;\n\t"
+      "sub.rn.f32.f16 %4, g3, %8;\n\t}"
+      : "=r"(w), "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]));
+  return w;
 }
 
 template <typename T>
@@ -93,39 +125,42 @@ if6_kernel(const T *__restrict__ x, I rows, I cols, I ld, const float *__restric
     for (int k = 0; k < 16; ++k) m = fmaxf(m, fabsf(v[k]));
     const uint32_t code = e4m3_code(div_qmax(__fmul_rn(m, s_enc), 7.5f, 1.0f / 7.5f));
     const float rf = tab[code];
+    // |t| <= RN(RN(m * r) * RN(31/7.5)) by monotonicity; only a block reaching
+    // 31.25 needs the clamp (which then makes rint land on +-31, as clamping
+    // rint(t) to +-31 does)
+    const bool clamp = __fmul_rn(__fmul_rn(m, rf), kUp) > 31.25f;
     float e_fp = 0.0f, e_int = 0.0f;
-    uint32_t fp_pair[8];
-    int kk[16];
+    uint32_t fp_group[4], int_group[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float v0 = __fmul_rn(v[2 * j], rf), v1 = __fmul_rn(v[2 * j + 1], rf);
-      fp_pair[j] = e2m3x2(v0, v1);
-      const float2 g = e2m3x2_value(fp_pair[j] & 0x3F3Fu);
-      const float vv[2] = {v0, v1}, gg[2] = {g.x, g.y};
+    for (int q4 = 0; q4 < 4; ++q4) {                   // groups of four elements
+      float vv[4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float d_fp = __fsub_rn(vv[h], gg[h]);
-        e_fp = __fmaf_rn(d_fp, d_fp, e_fp);
-        int k = __float2int_rn(__fmul_rn(vv[h], kUp));
-        k = k > 31 ? 31 : (k < -31 ? -31 : k);
-        kk[2 * j + h] = k;
-        const float d_int = __fsub_rn(vv[h], __fmul_rn(static_cast<float>(k), kDown));
-        e_int = __fmaf_rn(d_int, d_int, e_int);
+      for (int h = 0; h < 4; ++h) vv[h] = __fmul_rn(v[4 * q4 + h], rf);
+      float d[4];
+      const uint32_t w = e2m3x4_codes_diffs(vv, d);     // codes as bytes; d = RN(g - v)
+#pragma unroll
+      for (int h = 0; h < 4; ++h) e_fp = __fmaf_rn(d[h], d[h], e_fp);
+      fp_group[q4] = (w & 0x3Fu) | ((w >> 2) & 0xFC0u) | ((w >> 4) & 0x3F000u) |
+                     ((w >> 6) & 0xFC0000u);
+      uint32_t tb[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {                    // element order, as the errors sum
+        float t = __fmul_rn(vv[h], kUp);
+        if (clamp) t = fminf(fmaxf(t, -31.25f), 31.25f);
+        const float tm = __fadd_rn(t, kMagic);         // rint(t) in the low bits
+        const float kf = __fsub_rn(tm, kMagic);        // exact
+        const float dint = __fsub_rn(vv[h], __fmul_rn(kf, kDown));
+        e_int = __fmaf_rn(dint, dint, e_int);
+        tb[h] = __float_as_uint(tm);
       }
+      const uint32_t acc = ((tb[3] * 64u + tb[2]) * 64u + tb[1]) * 64u + tb[0];
+      // sum of (k + 32) 64^i, then bit 5 of each field flipped: k in two's complement
+      int_group[q4] = (acc - kGroupBias) ^ 0x820820u;
     }
     const bool use_int = e_int < e_fp;
-    uint32_t g[4];                                      // 24-bit groups of four codes
+    uint32_t g[4];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      uint32_t c[4];
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const int k = 4 * t + h;
-        const uint32_t fpc = (fp_pair[k >> 1] >> (8 * (k & 1))) & 0x3Fu;
-        c[h] = use_int ? (static_cast<uint32_t>(kk[k]) & 0x3Fu) : fpc;
-      }
-      g[t] = c[0] | c[1] << 6 | c[2] << 12 | c[3] << 18;
-    }
+    for (int t = 0; t < 4; ++t) g[t] = use_int ? int_group[t] : fp_group[t];
     uint32_t *dst = reinterpret_cast<uint32_t *>(q + b * 12);   // codes are dense, 12 B per block
     dst[0] = g[0] | g[1] << 24;
     dst[1] = g[1] >> 8 | g[2] << 16;

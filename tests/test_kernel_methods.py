@@ -62,6 +62,27 @@ def test_magic_number_low_bits_are_the_int4_nibble():
     assert np.array_equal(s.view(np.uint32) & 0xF, (k.astype(np.int64) & 0xF).astype(np.uint32))
 
 
+def test_magic_number_rint_and_int6_group_packing():
+    """IF6's INT6 step: RN(t + 1.5*2^23) - 1.5*2^23 == rint(t) for |t| <= 31.25
+    (every tie j + 1/2 included), and four such words summed with weights 64^i,
+    minus (0x4B400000 - 32) * (1 + 64 + 64^2 + 64^3), XOR 0x820820, is the
+    24-bit group of the four 6-bit two's-complement codes."""
+    magic = np.float32(12582912.0)
+    t = np.concatenate([np.linspace(-31.25, 31.25, 400_001, dtype=np.float32),
+                        np.arange(-31, 31, dtype=np.float32) + np.float32(0.5)])
+    s_ = (t + magic).astype(np.float32)
+    assert np.array_equal((s_ - magic).astype(np.float32), np.rint(t))
+    rng = np.random.default_rng(0)
+    k = np.concatenate([rng.integers(-31, 32, (20000, 4)),
+                        np.array([[-31, -31, -31, -31], [31, 31, 31, 31], [0, -1, 1, -31]])])
+    bits = (k.astype(np.float32) + magic).astype(np.float32).view(np.uint32).astype(np.uint64)
+    acc = (((bits[:, 3] * 64 + bits[:, 2]) * 64 + bits[:, 1]) * 64 + bits[:, 0]) % 2**32
+    bias = ((0x4B400000 - 32) * (1 + 64 + 4096 + 262144)) % 2**32
+    got = ((acc - bias) % 2**32) ^ 0x820820
+    want = sum((k[:, i] & 0x3F).astype(np.uint64) << (6 * i) for i in range(4))
+    assert np.array_equal(got, want)
+
+
 def test_rint_ties_go_to_even():
     """rint (the kernels' cvt.rni) on the INT4 ties t = j + 0.5."""
     t = np.arange(-7, 7, dtype=np.float32) + np.float32(0.5)
