@@ -96,6 +96,8 @@ _SIGNATURES = {
                                          _I, _P, _SZ, _P]),
     "fp4q_quantize_mxfp6": (_I, [_P, _I, _I64, _I64, _I64, _I, _I, _P, _P, _I, _P]),
     "fp4q_gemm_nvfp4": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P, _P]),
+    "fp4q_gemm_nvfp4_withhold_loads": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I,
+                                            _I64, _P, _P]),
     "fp4q_quantize_if6": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _SZ, _P]),
 }
 

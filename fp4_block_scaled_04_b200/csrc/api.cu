@@ -534,10 +534,41 @@ fp4q_status fp4q_quantize_mxfp6(const void *x, int dtype, int64_t rows, int64_t 
       launch_mxfp6(x, dtype, rows, cols, ld, fp6_format, e8m0_mode, q, sf, scale_layout, L));
 }
 
+namespace fp4q {
+namespace {
+fp4q_status gemm_checked(const uint8_t *qa, const uint8_t *sfa, const float *tensor_scale_a,
+                         const uint8_t *qb, const uint8_t *sfb, const float *tensor_scale_b,
+                         int64_t M, int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
+                         int *status, void *stream, int withhold);
+}  // namespace
+}  // namespace fp4q
+
 fp4q_status fp4q_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *tensor_scale_a,
                             const uint8_t *qb, const uint8_t *sfb, const float *tensor_scale_b,
                             int64_t M, int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
                             int *status, void *stream) {
+  return gemm_checked(qa, sfa, tensor_scale_a, qb, sfb, tensor_scale_b, M, N, K, c, c_dtype, ldc,
+                      status, stream, 0);
+}
+
+fp4q_status fp4q_gemm_nvfp4_withhold_loads(const uint8_t *qa, const uint8_t *sfa,
+                                           const float *tensor_scale_a, const uint8_t *qb,
+                                           const uint8_t *sfb, const float *tensor_scale_b,
+                                           int64_t M, int64_t N, int64_t K, void *c, int c_dtype,
+                                           int64_t ldc, int *status, void *stream) {
+  if (!status || K == 0) return FP4Q_ERR_INVALID_ARG;   // the hook exists to set *status
+  return gemm_checked(qa, sfa, tensor_scale_a, qb, sfb, tensor_scale_b, M, N, K, c, c_dtype, ldc,
+                      status, stream, 1);
+}
+
+}  // extern "C"
+
+namespace fp4q {
+namespace {
+fp4q_status gemm_checked(const uint8_t *qa, const uint8_t *sfa, const float *tensor_scale_a,
+                         const uint8_t *qb, const uint8_t *sfb, const float *tensor_scale_b,
+                         int64_t M, int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
+                         int *status, void *stream, int withhold) {
   if (!valid_dtype(c_dtype)) return FP4Q_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4Q_ERR_INVALID_ARG;
   if (M % 128 != 0 || N % 128 != 0 || K % 256 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
@@ -566,8 +597,12 @@ fp4q_status fp4q_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *
   FP4Q_TRY(check_dev(tensor_scale_b, true));
   FP4Q_TRY(check_dev(status, true));
   return cuda_status(launch_gemm_nvfp4(qa, sfa, tensor_scale_a, qb, sfb, tensor_scale_b, M, N, K,
-                                       c, c_dtype, ldc, status, L));
+                                       c, c_dtype, ldc, status, withhold, L));
 }
+}  // namespace
+}  // namespace fp4q
+
+extern "C" {
 
 fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,
                             int block_rows, int block_cols, const float *tensor_scale,

@@ -65,11 +65,12 @@ cudaError_t launch_mxfp6_dequant(const uint8_t *q, const uint8_t *sf, int scale_
                                  int y_dtype, const Launch &L);
 
 // C[M, N] = s_a s_b (A B^T) from NVFP4 operands (codes [rows, K/2], swizzled
-// 1x16 scales) on the tensor cores; status (may be NULL) <- 1 if a wait ran out
+// 1x16 scales) on the tensor cores; status (may be NULL) <- 1 if a wait ran out;
+// withhold != 0 (a failure-detection test hook) issues no operand loads
 cudaError_t launch_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *s_a,
                               const uint8_t *qb, const uint8_t *sfb, const float *s_b, int64_t M,
                               int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
-                              int *status, const Launch &L);
+                              int *status, int withhold, const Launch &L);
 
 // IF6: per 16-value block FP6 E2M3 or INT6 (rescaled by 7.5/31), codes four
 // per three bytes; and its decode

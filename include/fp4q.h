@@ -344,6 +344,19 @@ fp4q_status fp4q_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *
                             int64_t M, int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
                             int *status, void *stream);
 
+/* Failure-detection test hook for fp4q_gemm_nvfp4: the same call, but the
+ * kernel's loader issues no operand loads, so that the tensor-core thread's
+ * bounded wait runs out (after about a second).  No tensor-core work is ever
+ * issued; the kernel sets *status to 1, writes unspecified values to C, frees
+ * its tensor memory and returns, and the CUDA context stays usable.
+ * Arguments as for fp4q_gemm_nvfp4; status must be non-NULL and K > 0.  For
+ * tests only. */
+fp4q_status fp4q_gemm_nvfp4_withhold_loads(const uint8_t *qa, const uint8_t *sfa,
+                                           const float *tensor_scale_a, const uint8_t *qb,
+                                           const uint8_t *sfb, const float *tensor_scale_b,
+                                           int64_t M, int64_t N, int64_t K, void *c, int c_dtype,
+                                           int64_t ldc, int *status, void *stream);
+
 /* Dequantization of packed codes [rows, cols/2] back to y [rows, cols]
  * (FP32 or BF16 = RNE of the FP32 value), Ultralytics glossary "FP4の仕組み"
  * (grid value * sign * scale):

@@ -161,6 +161,9 @@ def test_host_side_argument_checks_of_the_added_calls(L):
     assert gm(qa=None) == 1
     assert gm(qa=ctypes.c_void_p(0x7F0000000004)) == 3
     assert gm(M=0) == 0
+    # the test hook wants a status pointer and some K
+    assert L.fp4q_gemm_nvfp4_withhold_loads(FAKE, FAKE, None, FAKE, FAKE, None, 128, 128, 256,
+                                            FAKE, 1, 128, None, None) == 1
     # IF6: the IF4 rules
     assert L.fp4q_quantize_if6(FAKE, 0, 16, 40, 40, FAKE, FAKE, FAKE, FAKE, 0, None, 0,
                                None) == 2

@@ -197,3 +197,26 @@ def test_wgrad_from_rht_operands_with_the_same_signs(orc, n):
                             tensor_scale_a=od["s_dec"], tensor_scale_b=ox2["s_dec"])
     rel2 = np.linalg.norm(host(c2) - ref) / np.linalg.norm(ref)
     assert rel2 > 1.0, rel2              # about 1.5: uncorrelated with dY^T X
+
+
+def test_gemm_wait_that_runs_out_sets_status_and_leaves_the_context_usable(orc):
+    """Failure detection without a GPU fault: the test hook withholds the
+    operand loads, so the tensor-core thread's bounded wait (about a second)
+    runs out; the kernel must report it through status and return, and the
+    next GEMM must be correct."""
+    M, N, K = 128, 128, 256
+    qa, sfa = random_operand(M, K, 7)
+    qb, sfb = random_operand(N, K, 8)
+    ta, tsa, tb, tsb = (torch.from_numpy(a).to(DEV) for a in (qa, sfa, qb, sfb))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    c = torch.empty((M, N), device=DEV)
+    rc = fq.lib().fp4q_gemm_nvfp4_withhold_loads(
+        fq._ptr(ta), fq._ptr(tsa), None, fq._ptr(tb), fq._ptr(tsb), None, M, N, K, fq._ptr(c),
+        1, N, fq._ptr(status), fq._stream(ta.device))
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1
+    status.zero_()
+    c = fq.fp4q_gemm_nvfp4(ta, tsa, tb, tsb, K, status=status)
+    assert int(status.item()) == 0
+    check(orc, qa, sfa, qb, sfb, M, N, K, host(c))
