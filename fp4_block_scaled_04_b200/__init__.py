@@ -35,6 +35,7 @@ __all__ = [
     "fp4q_quantize_nvfp4_noalloc", "fp4q_quantize_nvint4", "fp4q_quantize_four_over_six",
     "fp4q_quantize_backward", "fp4q_quantize_mxfp6", "FMT_MXFP6_E2M3", "FMT_MXFP6_E3M2",
     "FP6_E2M3", "FP6_E3M2", "fp4q_gemm_nvfp4", "fp4q_quantize_if6", "FMT_IF6",
+    "fp4q_gemm_if4_nvfp4",
 ]
 
 ROWWISE, COLWISE = 1, 2
@@ -98,6 +99,9 @@ _SIGNATURES = {
     "fp4q_gemm_nvfp4": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P, _P]),
     "fp4q_gemm_nvfp4_withhold_loads": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I,
                                             _I64, _P, _P]),
+    "fp4q_gemm_if4_workspace_bytes": (_SZ, [_I64, _I64]),
+    "fp4q_gemm_if4_nvfp4": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _SZ,
+                                 _P, _P]),
     "fp4q_quantize_if6": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _SZ, _P]),
 }
 
@@ -307,6 +311,26 @@ def fp4q_gemm_nvfp4(qa: torch.Tensor, sfa: torch.Tensor, qb: torch.Tensor, sfb: 
     _check("fp4q_gemm_nvfp4", lib().fp4q_gemm_nvfp4(
         _ptr(qa), _ptr(sfa), _ptr(tensor_scale_a), _ptr(qb), _ptr(sfb), _ptr(tensor_scale_b),
         M, N, K, _ptr(c), cdt, c.stride(0) if M > 1 else N, _ptr(status), _stream(qa.device)))
+    return c
+
+
+def fp4q_gemm_if4_nvfp4(qa: torch.Tensor, sfa: torch.Tensor, qb: torch.Tensor, sfb: torch.Tensor,
+                        K: int, tensor_scale_a: torch.Tensor | None = None,
+                        tensor_scale_b: torch.Tensor | None = None,
+                        out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                        status: torch.Tensor | None = None) -> torch.Tensor:
+    """C [M, N] FP32 = s_a s_b (A B^T) with A in IF4 (codes [M, K/2], flagged
+    swizzled scales as fp4q_quantize_if4 writes them) and B in NVFP4."""
+    if not qa.is_cuda:
+        raise ValueError("qa must be a CUDA tensor")
+    M, N = qa.shape[0], qb.shape[0]
+    c = torch.empty((M, N), dtype=torch.float32, device=qa.device) if out is None else out
+    need = int(lib().fp4q_gemm_if4_workspace_bytes(M, K))
+    ws = _u8(max(need, 16), qa.device) if workspace is None else workspace
+    _check("fp4q_gemm_if4_nvfp4", lib().fp4q_gemm_if4_nvfp4(
+        _ptr(qa), _ptr(sfa), _ptr(tensor_scale_a), _ptr(qb), _ptr(sfb), _ptr(tensor_scale_b),
+        M, N, K, _ptr(c), c.stride(0) if M > 1 else N, _ptr(ws), ws.numel(), _ptr(status),
+        _stream(qa.device)))
     return c
 
 

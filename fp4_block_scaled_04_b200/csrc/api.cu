@@ -551,6 +551,60 @@ fp4q_status fp4q_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *
                       status, stream, 0);
 }
 
+size_t fp4q_gemm_if4_workspace_bytes(int64_t M, int64_t K) {
+  if (M < 0 || K < 0) return 0;
+  return static_cast<size_t>(3 * (M * K / 2) + M * K / 16);
+}
+
+fp4q_status fp4q_gemm_if4_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *tensor_scale_a,
+                                const uint8_t *qb, const uint8_t *sfb,
+                                const float *tensor_scale_b, int64_t M, int64_t N, int64_t K,
+                                float *c, int64_t ldc, void *workspace, size_t ws_bytes,
+                                int *status, void *stream) {
+  if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4Q_ERR_INVALID_ARG;
+  if (M % 128 != 0 || N % 128 != 0 || K % 256 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
+  if (K > (int64_t{1} << 30) || M / 128 > 65535) return FP4Q_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return FP4Q_OK;
+  if (!c) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned16(c) || (ldc * 4) % 16 != 0) return FP4Q_ERR_MISALIGNED;
+  if (K > 0) {
+    if (!qa || !sfa || !qb || !sfb) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned16(qa) || !aligned16(qb) || !aligned16(sfa) || !aligned16(sfb))
+      return FP4Q_ERR_MISALIGNED;
+    if (!workspace || ws_bytes < fp4q_gemm_if4_workspace_bytes(M, K))
+      return FP4Q_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace)) return FP4Q_ERR_MISALIGNED;
+  }
+  Launch L;
+  FP4Q_TRY(bind_device(c, stream, &L));
+  if (K == 0)
+    return cuda_status(cudaMemset2DAsync(c, static_cast<size_t>(ldc * 4), 0,
+                                         static_cast<size_t>(N * 4), static_cast<size_t>(M),
+                                         L.stream));
+  FP4Q_TRY(check_dev(qa, false));
+  FP4Q_TRY(check_dev(sfa, false));
+  FP4Q_TRY(check_dev(qb, false));
+  FP4Q_TRY(check_dev(sfb, false));
+  FP4Q_TRY(check_dev(workspace, false));
+  FP4Q_TRY(check_dev(tensor_scale_a, true));
+  FP4Q_TRY(check_dev(tensor_scale_b, true));
+  FP4Q_TRY(check_dev(status, true));
+  uint8_t *w = static_cast<uint8_t *>(workspace);
+  const int64_t codes = M * K / 2;
+  uint8_t *q_fp = w, *q_k1 = w + codes, *q_k2 = w + 2 * codes, *sf_plain = w + 3 * codes;
+  FP4Q_TRY(cuda_status(launch_if4_split(qa, sfa, M, K, FP4Q_SCALE_SWIZZLED_128x4, q_fp, q_k1,
+                                        q_k2, sf_plain, L)));
+  GemmOptions opt;                                     // C = RN(acc_fp * alpha)
+  FP4Q_TRY(cuda_status(launch_gemm_nvfp4(q_fp, sf_plain, tensor_scale_a, qb, sfb, tensor_scale_b,
+                                         M, N, K, c, FP4Q_FP32, ldc, status, opt, L)));
+  opt.alpha_mul = 6.0f / 7.0f;                         // C += RN(acc_k * RN(alpha * RN(6/7)))
+  opt.accumulate = 1;
+  FP4Q_TRY(cuda_status(launch_gemm_nvfp4(q_k1, sf_plain, tensor_scale_a, qb, sfb, tensor_scale_b,
+                                         M, N, K, c, FP4Q_FP32, ldc, status, opt, L)));
+  return cuda_status(launch_gemm_nvfp4(q_k2, sf_plain, tensor_scale_a, qb, sfb, tensor_scale_b,
+                                       M, N, K, c, FP4Q_FP32, ldc, status, opt, L));
+}
+
 fp4q_status fp4q_gemm_nvfp4_withhold_loads(const uint8_t *qa, const uint8_t *sfa,
                                            const float *tensor_scale_a, const uint8_t *qb,
                                            const uint8_t *sfb, const float *tensor_scale_b,
@@ -596,8 +650,10 @@ fp4q_status gemm_checked(const uint8_t *qa, const uint8_t *sfa, const float *ten
   FP4Q_TRY(check_dev(tensor_scale_a, true));
   FP4Q_TRY(check_dev(tensor_scale_b, true));
   FP4Q_TRY(check_dev(status, true));
+  GemmOptions opt;
+  opt.withhold = withhold;
   return cuda_status(launch_gemm_nvfp4(qa, sfa, tensor_scale_a, qb, sfb, tensor_scale_b, M, N, K,
-                                       c, c_dtype, ldc, status, withhold, L));
+                                       c, c_dtype, ldc, status, opt, L));
 }
 }  // namespace
 }  // namespace fp4q

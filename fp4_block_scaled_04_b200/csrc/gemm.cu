@@ -201,7 +201,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
                   const __grid_constant__ CUtensorMap map_b, const uint8_t *__restrict__ sfa,
                   const float *__restrict__ s_a, const uint8_t *__restrict__ sfb,
                   const float *__restrict__ s_b, int K, int n_tiles_n, int n_tiles,
-                  OutT *__restrict__ c, int64_t ldc, int *__restrict__ status, int withhold) {
+                  OutT *__restrict__ c, int64_t ldc, int *__restrict__ status,
+                  GemmOptions opt) {
   using T = Tile<BN>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -247,7 +248,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
       int g = 0;                                          // K-tiles issued so far
       // withhold (a failure-detection test hook): issue nothing, so that the
       // MMA thread's first wait runs out
-      for (int tile = blockIdx.x; tile < n_tiles && !*err_ptr && !withhold; tile += gridDim.x) {
+      for (int tile = blockIdx.x; tile < n_tiles && !*err_ptr && !opt.withhold;
+           tile += gridDim.x) {
         const int m0 = (tile / n_tiles_n) * BM, n0 = (tile % n_tiles_n) * BN;
         const uint8_t *sfa_tile = sfa + static_cast<int64_t>(m0 / BM) * sf_rowtile;
         const uint8_t *sfb_tile = sfb + static_cast<int64_t>(n0 / 128) * sf_rowtile;
@@ -316,7 +318,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
   } else {
     // ---- epilogue: warp w reads accumulator lanes 32 (w % 4) .. + 31 ----
     const int quarter = warp & 3;
-    const float alpha = __fmul_rn(s_a ? *s_a : 1.0f, s_b ? *s_b : 1.0f);
+    const float alpha =
+        __fmul_rn(__fmul_rn(s_a ? *s_a : 1.0f, s_b ? *s_b : 1.0f), opt.alpha_mul);
     int i = 0;
     for (int tile = blockIdx.x; tile < n_tiles && !*err_ptr; tile += gridDim.x, ++i) {
       const int ok = mbar_wait(acc_full, static_cast<uint32_t>(i & 1)) ? 1 : 0;
@@ -366,11 +369,18 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
               asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty) : "memory");
           }
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            d[4 * j + q] = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), alpha),
-                                       __fmul_rn(__uint_as_float(r[4 * q + 1]), alpha),
-                                       __fmul_rn(__uint_as_float(r[4 * q + 2]), alpha),
-                                       __fmul_rn(__uint_as_float(r[4 * q + 3]), alpha));
+          for (int q = 0; q < 4; ++q) {
+            float4 o = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), alpha),
+                                   __fmul_rn(__uint_as_float(r[4 * q + 1]), alpha),
+                                   __fmul_rn(__uint_as_float(r[4 * q + 2]), alpha),
+                                   __fmul_rn(__uint_as_float(r[4 * q + 3]), alpha));
+            if (opt.accumulate) {                       // C += RN(acc * alpha)
+              const float4 p = d[4 * j + q];
+              o = make_float4(__fadd_rn(p.x, o.x), __fadd_rn(p.y, o.y), __fadd_rn(p.z, o.z),
+                              __fadd_rn(p.w, o.w));
+            }
+            d[4 * j + q] = o;
+          }
         }
       }
     }
@@ -420,7 +430,7 @@ bool make_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t row_b
 template <typename OutT, int BN>
 cudaError_t launch_t(const uint8_t *qa, const uint8_t *sfa, const float *s_a, const uint8_t *qb,
                      const uint8_t *sfb, const float *s_b, int64_t M, int64_t N, int64_t K,
-                     void *c, int64_t ldc, int *status, int withhold, const Launch &L) {
+                     void *c, int64_t ldc, int *status, GemmOptions opt, const Launch &L) {
   using T = Tile<BN>;
   static bool configured[64] = {};
   int dev = 0;
@@ -440,17 +450,17 @@ cudaError_t launch_t(const uint8_t *qa, const uint8_t *sfa, const float *s_a, co
   const int grid = static_cast<int>(n_tiles < L.num_sms ? n_tiles : L.num_sms);
   gemm_nvfp4_kernel<OutT, BN><<<grid, kThreads, T::SMEM_BYTES, L.stream>>>(
       map_a, map_b, sfa, s_a, sfb, s_b, static_cast<int>(K), static_cast<int>(n_tiles_n),
-      static_cast<int>(n_tiles), static_cast<OutT *>(c), ldc, status, withhold);
+      static_cast<int>(n_tiles), static_cast<OutT *>(c), ldc, status, opt);
   return cudaGetLastError();
 }
 
 template <typename OutT>
 cudaError_t launch_o(const uint8_t *qa, const uint8_t *sfa, const float *s_a, const uint8_t *qb,
                      const uint8_t *sfb, const float *s_b, int64_t M, int64_t N, int64_t K,
-                     void *c, int64_t ldc, int *status, int withhold, const Launch &L) {
+                     void *c, int64_t ldc, int *status, GemmOptions opt, const Launch &L) {
   if (N % 256 == 0)
-    return launch_t<OutT, 256>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, withhold, L);
-  return launch_t<OutT, 128>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, withhold, L);
+    return launch_t<OutT, 256>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
+  return launch_t<OutT, 128>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
 }
 
 }  // namespace
@@ -458,10 +468,10 @@ cudaError_t launch_o(const uint8_t *qa, const uint8_t *sfa, const float *s_a, co
 cudaError_t launch_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *s_a,
                               const uint8_t *qb, const uint8_t *sfb, const float *s_b, int64_t M,
                               int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
-                              int *status, int withhold, const Launch &L) {
+                              int *status, GemmOptions opt, const Launch &L) {
   if (c_dtype == FP4Q_BF16)
-    return launch_o<__nv_bfloat16>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, withhold, L);
-  return launch_o<float>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, withhold, L);
+    return launch_o<__nv_bfloat16>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
+  return launch_o<float>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
 }
 
 }  // namespace fp4q

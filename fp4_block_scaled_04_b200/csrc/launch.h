@@ -64,13 +64,29 @@ cudaError_t launch_mxfp6_dequant(const uint8_t *q, const uint8_t *sf, int scale_
                                  int64_t rows, int64_t cols, int fp6_format, void *y,
                                  int y_dtype, const Launch &L);
 
+// Options of the tensor-core GEMM: the product is scaled by RN(RN(s_a s_b) *
+// alpha_mul); accumulate != 0 adds it to the FP32 C already there (C =
+// RN(C + RN(acc * alpha))); withhold != 0 (a failure-detection test hook)
+// issues no operand loads.
+struct GemmOptions {
+  float alpha_mul = 1.0f;
+  int accumulate = 0;
+  int withhold = 0;
+};
+
 // C[M, N] = s_a s_b (A B^T) from NVFP4 operands (codes [rows, K/2], swizzled
-// 1x16 scales) on the tensor cores; status (may be NULL) <- 1 if a wait ran out;
-// withhold != 0 (a failure-detection test hook) issues no operand loads
+// 1x16 scales) on the tensor cores; status (may be NULL) <- 1 if a wait ran out
 cudaError_t launch_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *s_a,
                               const uint8_t *qb, const uint8_t *sfb, const float *s_b, int64_t M,
                               int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
-                              int *status, int withhold, const Launch &L);
+                              int *status, GemmOptions opt, const Launch &L);
+
+// Split IF4 codes [rows, K/2] with flagged scales into three NVFP4 code
+// matrices sharing the unflagged scales: FP4 blocks (INT4 blocks zero) and the
+// two E2M1 parts g1 + g2 = k of the INT4 blocks (FP4 blocks zero)
+cudaError_t launch_if4_split(const uint8_t *q, const uint8_t *sf, int64_t rows, int64_t K,
+                             int scale_layout, uint8_t *q_fp, uint8_t *q_k1, uint8_t *q_k2,
+                             uint8_t *sf_plain, const Launch &L);
 
 // IF6: per 16-value block FP6 E2M3 or INT6 (rescaled by 7.5/31), codes four
 // per three bytes; and its decode

@@ -344,6 +344,33 @@ fp4q_status fp4q_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *
                             int64_t M, int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
                             int *status, void *stream);
 
+/* IF4 x NVFP4 GEMM on the tensor cores: the IF4 operand of the consumer GEMM.
+ * "Adaptive Block-Scaled Data Types" explainer, section 2: an IF4 block is
+ * FP4 (E2M1 code * S) or INT4 (k * RN(6/7) * S), flagged by the scale's sign
+ * bit.  The block-scaled MMA multiplies E2M1 codes by E4M3 scales only, and
+ * RN(6/7) * S is not an E4M3 value; every k in -7..7 is the sum of at most two
+ * E2M1 values (5 = 4 + 1, 7 = 6 + 1), so A is split into three NVFP4 operands
+ * sharing the unflagged scales (the FP4 blocks, and the two E2M1 parts of the
+ * INT4 blocks) and
+ *   C = RN(acc_fp * a) + RN(acc_1 * a67) + RN(acc_2 * a67) (added in that
+ *   order, each sum rounded), a = RN(s_a * s_b), a67 = RN(a * RN(6/7)),
+ * each acc accumulated in FP32 by tcgen05.mma.  The result is within FP32
+ * accumulation and rounding error of the exact product of the dequantized IF4
+ * and NVFP4 operands.
+ *   qa, sfa      IF4 codes [M, K/2] and flagged scales in the 128x4 layout, as
+ *                fp4q_quantize_if4 writes them with FP4Q_SCALE_SWIZZLED_128x4
+ *   qb, sfb      NVFP4 codes [N, K/2] and swizzled scales
+ *   c, ldc       FP32 output [M, ldc]
+ *   workspace    device memory of fp4q_gemm_if4_workspace_bytes(M, K) bytes,
+ *                16-byte aligned (the split operands; the caller's)
+ *   tensor scales, status and shapes as for fp4q_gemm_nvfp4. */
+size_t fp4q_gemm_if4_workspace_bytes(int64_t M, int64_t K);
+fp4q_status fp4q_gemm_if4_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *tensor_scale_a,
+                                const uint8_t *qb, const uint8_t *sfb,
+                                const float *tensor_scale_b, int64_t M, int64_t N, int64_t K,
+                                float *c, int64_t ldc, void *workspace, size_t ws_bytes,
+                                int *status, void *stream);
+
 /* Failure-detection test hook for fp4q_gemm_nvfp4: the same call, but the
  * kernel's loader issues no operand loads, so that the tensor-core thread's
  * bounded wait runs out (after about a second).  No tensor-core work is ever

@@ -471,11 +471,14 @@ def gemm_block_scaled(qa: np.ndarray, sfa: np.ndarray, qb: np.ndarray, sfb: np.n
     with the block scales only (tensor scale 1, which makes every element the
     exact product g * S), then C = alpha * (A B^T), the contraction and the
     final product taken in float64 (a library matmul).  alpha carries the
-    product of the two tensor scales.  Returns float64 [M, N].
+    product of the two tensor scales.  fmt FMT_IF4 dequantizes A as IF4 (INT4
+    blocks RN(RN(k * RN(6/7)) * S)); B is always NVFP4 then.  Returns float64
+    [M, N].
     """
-    blk = 16 if fmt == FMT_NVFP4 else 32
+    blk = 32 if fmt == FMT_MXFP4 else 16       # NVFP4 and IF4 use 16-value blocks
     a = dequantize(fmt, qa, sfa, M, K, 1, blk, s_dec=1.0 if fmt != FMT_MXFP4 else None,
                    scale_layout=scale_layout)
-    b = dequantize(fmt, qb, sfb, N, K, 1, blk, s_dec=1.0 if fmt != FMT_MXFP4 else None,
+    fb = FMT_NVFP4 if fmt == FMT_IF4 else fmt
+    b = dequantize(fb, qb, sfb, N, K, 1, blk, s_dec=1.0 if fb != FMT_MXFP4 else None,
                    scale_layout=scale_layout)
     return (a.astype(np.float64) @ b.astype(np.float64).T) * float(alpha)

@@ -31,7 +31,8 @@ def test_header_declares_the_entry_points():
     for n in ["fp4q_amax", "fp4q_quantize_nvfp4", "fp4q_quantize_mxfp4", "fp4q_quantize_2d",
               "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
               "fp4q_scale_bytes", "fp4q_workspace_bytes", "fp4q_status_string", "fp4q_version",
-              "fp4q_quantize_mxfp6", "fp4q_gemm_nvfp4", "fp4q_quantize_if6"]:
+              "fp4q_quantize_mxfp6", "fp4q_gemm_nvfp4", "fp4q_quantize_if6",
+              "fp4q_gemm_if4_nvfp4"]:
         assert n in names
 
 
@@ -161,6 +162,14 @@ def test_host_side_argument_checks_of_the_added_calls(L):
     assert gm(qa=None) == 1
     assert gm(qa=ctypes.c_void_p(0x7F0000000004)) == 3
     assert gm(M=0) == 0
+    # the IF4 GEMM: GEMM shapes plus a workspace of the stated size
+    assert L.fp4q_gemm_if4_workspace_bytes(128, 256) == 3 * 128 * 128 + 128 * 16
+    g4 = lambda **kw: L.fp4q_gemm_if4_nvfp4(
+        FAKE, FAKE, None, FAKE, FAKE, None, kw.get("M", 128), 128, kw.get("K", 256), FAKE, 128,
+        kw.get("ws", FAKE), kw.get("wsb", 1 << 20), None, None)
+    assert g4(K=128) == 2 and g4(M=96) == 2
+    assert g4(wsb=100) == 4 and g4(ws=None) == 4
+    assert g4(ws=ctypes.c_void_p(0x7F0000000008)) == 3
     # the test hook wants a status pointer and some K
     assert L.fp4q_gemm_nvfp4_withhold_loads(FAKE, FAKE, None, FAKE, FAKE, None, 128, 128, 256,
                                             FAKE, 1, 128, None, None) == 1

@@ -16,6 +16,7 @@ import pytest
 import torch
 
 import fp4_block_scaled_04_b200 as fq
+from fp4_block_scaled_04_b200 import workloads
 
 from test_gpu_parity import DEV, host
 
@@ -220,3 +221,34 @@ def test_gemm_wait_that_runs_out_sets_status_and_leaves_the_context_usable(orc):
     c = fq.fp4q_gemm_nvfp4(ta, tsa, tb, tsb, K, status=status)
     assert int(status.item()) == 0
     check(orc, qa, sfa, qb, sfb, M, N, K, host(c))
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 384, 1024), (512, 256, 2048)])
+def test_if4_operand_in_the_tensor_core_gemm(orc, M, N, K):
+    """IF4 x NVFP4: the IF4 operand split into FP4 blocks and the two E2M1
+    parts of its INT4 blocks, three accumulating GEMMs.  Compared with the
+    exact product of the dequantized IF4 and NVFP4 operands, with room for
+    three FP32 accumulations, the RN(6/7) factor and two output additions."""
+    x = workloads.if4_blocks(rows=M, cols=K).to(DEV)
+    g = torch.Generator().manual_seed(15)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16).to(DEV)
+    sw = fq.SCALE_SWIZZLED
+    ox = fq.fp4q_quantize_if4(x, scale_layout=sw)
+    ow = fq.fp4q_quantize_nvfp4(w, scale_layout=sw)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    c = fq.fp4q_gemm_if4_nvfp4(ox["q"], ox["sf"], ow["q_row"], ow["sf_row"], K,
+                               tensor_scale_a=ox["s_dec"], tensor_scale_b=ow["s_dec"],
+                               status=status)
+    assert int(status.item()) == 0
+    qa, sa, qb, sb = host(ox["q"]), host(ox["sf"]), host(ow["q_row"]), host(ow["sf_row"])
+    assert 0.05 < np.mean(sa >= 0x80) < 0.95          # both kinds of block present
+    alpha = float(np.float32(ox["s_dec"].item()) * np.float32(ow["s_dec"].item()))
+    exact = orc.gemm_block_scaled(qa, sa, qb, sb, M, N, K, fmt=orc.FMT_IF4)
+    a = orc.dequantize(orc.FMT_IF4, qa, sa, M, K, 1, 16, s_dec=1.0,
+                       scale_layout=orc.SCALE_SWIZZLED).astype(np.float64)
+    b = orc.dequantize(orc.FMT_NVFP4, qb, sb, N, K, 1, 16, s_dec=1.0,
+                       scale_layout=orc.SCALE_SWIZZLED).astype(np.float64)
+    bound = alpha * (3 * K + 16) * 2.0 ** -22 * (np.abs(a) @ np.abs(b).T) \
+        + abs(alpha * exact) * 2.0 ** -21 + 1e-30
+    worst = float(np.max(np.abs(host(c).astype(np.float64) - alpha * exact) / bound))
+    assert worst <= 1.0, f"IF4 GEMM differs from the exact product by {worst:.3g} x the bound"

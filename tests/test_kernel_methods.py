@@ -83,6 +83,21 @@ def test_magic_number_rint_and_int6_group_packing():
     assert np.array_equal(got, want)
 
 
+def test_if4_split_tables_sum_to_k():
+    """The IF4 GEMM's split: for every INT4 nibble n (k in two's complement)
+    the two E2M1 codes of the tables the split kernel uses add up to k."""
+    part1, part2 = 0xACDEEFFF77665420, 0x0000A0AC20200000
+    e2m1 = [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+
+    def value(code):
+        return -e2m1[code & 7] if code & 8 else e2m1[code & 7]
+
+    for n in range(16):
+        k = n - 16 if n & 8 else n
+        c1, c2 = (part1 >> (4 * n)) & 0xF, (part2 >> (4 * n)) & 0xF
+        assert value(c1) + value(c2) == k, (n, c1, c2)
+
+
 def test_rint_ties_go_to_even():
     """rint (the kernels' cvt.rni) on the INT4 ties t = j + 0.5."""
     t = np.arange(-7, 7, dtype=np.float32) + np.float32(0.5)
