@@ -269,7 +269,7 @@ def time_consumer_gemm(fq, device, stream, args, M=8192, N=8192, K=8192):
         tensor_scale_b=ow["s_dec"], out=c))
     out["fp4q"]["kernel"] = ("gemm_nvfp4_kernel (tcgen05.mma kind::mxf4nvf4, persistent, "
                              "128x256 tiles)")
-    # the same product with an IF4 activation operand (split pass + three GEMM passes)
+    # the same product with an IF4 activation operand (split pass + one two-accumulator GEMM)
     g5 = torch.Generator().manual_seed(6)
     xi = torch.randn(M, K, generator=g5).to(torch.bfloat16).to(device)
     oi = fq.fp4q_quantize_if4(xi, scale_layout=sw)
@@ -280,8 +280,8 @@ def time_consumer_gemm(fq, device, stream, args, M=8192, N=8192, K=8192):
     out["fp4q_if4"] = timed(lambda: fq.fp4q_gemm_if4_nvfp4(
         oi["q"], oi["sf"], ow["q_row"], ow["sf_row"], K, tensor_scale_a=oi["s_dec"],
         tensor_scale_b=ow["s_dec"], out=ci, workspace=wsi))
-    out["fp4q_if4"]["kernel"] = ("if4_split_kernel + 3 x gemm_nvfp4_kernel (IF4 x NVFP4, "
-                                 "FP32 out)")
+    out["fp4q_if4"]["kernel"] = ("if4_split_kernel + gemm_nvfp4_kernel with three A operands "
+                                 "and two accumulators (IF4 x NVFP4, FP32 out)")
     del wsi, ci
     A = ox["q_row"].view(torch.float4_e2m1fn_x2)
     B = ow["q_row"].view(torch.float4_e2m1fn_x2).t()

@@ -594,15 +594,9 @@ fp4q_status fp4q_gemm_if4_nvfp4(const uint8_t *qa, const uint8_t *sfa, const flo
   uint8_t *q_fp = w, *q_k1 = w + codes, *q_k2 = w + 2 * codes, *sf_plain = w + 3 * codes;
   FP4Q_TRY(cuda_status(launch_if4_split(qa, sfa, M, K, FP4Q_SCALE_SWIZZLED_128x4, q_fp, q_k1,
                                         q_k2, sf_plain, L)));
-  GemmOptions opt;                                     // C = RN(acc_fp * alpha)
-  FP4Q_TRY(cuda_status(launch_gemm_nvfp4(q_fp, sf_plain, tensor_scale_a, qb, sfb, tensor_scale_b,
-                                         M, N, K, c, FP4Q_FP32, ldc, status, opt, L)));
-  opt.alpha_mul = 6.0f / 7.0f;                         // C += RN(acc_k * RN(alpha * RN(6/7)))
-  opt.accumulate = 1;
-  FP4Q_TRY(cuda_status(launch_gemm_nvfp4(q_k1, sf_plain, tensor_scale_a, qb, sfb, tensor_scale_b,
-                                         M, N, K, c, FP4Q_FP32, ldc, status, opt, L)));
-  return cuda_status(launch_gemm_nvfp4(q_k2, sf_plain, tensor_scale_a, qb, sfb, tensor_scale_b,
-                                       M, N, K, c, FP4Q_FP32, ldc, status, opt, L));
+  return cuda_status(launch_gemm_if4_split(q_fp, q_k1, q_k2, sf_plain, tensor_scale_a, qb, sfb,
+                                           tensor_scale_b, M, N, K, c, FP4Q_FP32, ldc, status,
+                                           L));
 }
 
 fp4q_status fp4q_gemm_nvfp4_withhold_loads(const uint8_t *qa, const uint8_t *sfa,

@@ -51,26 +51,31 @@ namespace {
 constexpr int BM = 128;
 constexpr int KTILE = 256;                       // K values per stage
 constexpr int KTB = KTILE / 2;                   // 128 code bytes per row per stage
-constexpr int STAGES = 4;
 constexpr int kThreads = 192;                    // producer warp, MMA warp, 4 epilogue warps
 constexpr int SF_TILE = 512;                     // 128 rows x 4 scales
 constexpr int SF_BYTES = (KTILE / 64) * SF_TILE; // 2048: one operand row tile, one K-tile
 constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at the B200's clock
 
-template <int BN>
+// NA A operands per output tile: 1 (NVFP4), or 3 (the IF4 split: the FP4
+// blocks accumulate into one accumulator, the two E2M1 parts of the INT4
+// blocks into a second; all three share the A scales).
+template <int BN, int NA = 1>
 struct Tile {
-  static constexpr int A_BYTES = BM * KTB;                      // 16384
+  static constexpr int STAGES = NA == 1 ? 4 : 3;
+  static constexpr int NACC = NA == 1 ? 1 : 2;
+  static constexpr int A_BYTES = BM * KTB;                      // 16384 per A operand
   static constexpr int B_BYTES = BN * KTB;                      // 16384 or 32768
+  static constexpr int B_OFF = NA * A_BYTES;
   static constexpr int SFB_BYTES = (BN / 128) * SF_BYTES;       // [row tile][K step][512]
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES + SFB_BYTES;
+  static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES + SF_BYTES + SFB_BYTES;
   static constexpr int BAR_BYTES = 128;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-  // tensor memory: accumulator columns [0, BN), then per stage 16 columns of
-  // A scales and 4 * BN / 32 columns of B scales
-  static constexpr uint32_t SF_COL0 = BN;
+  // tensor memory: NACC accumulators of BN columns, then per stage 16 columns
+  // of A scales and 4 * BN / 32 columns of B scales
+  static constexpr uint32_t SF_COL0 = NACC * BN;
   static constexpr uint32_t SFB_COLS = 4 * (BN / 32);
   static constexpr uint32_t STAGE_COLS = 16 + SFB_COLS;
-  static constexpr uint32_t COLS_USED = BN + STAGES * STAGE_COLS;
+  static constexpr uint32_t COLS_USED = NACC * BN + STAGES * STAGE_COLS;
   static constexpr uint32_t TMEM_COLS = COLS_USED <= 256 ? 256 : 512;
   // Instruction descriptor of tcgen05.mma kind::mxf4nvf4 (block-scaled): A and
   // B E2M1 (format 1), K-major, E4M3 scales (bit 23 = 0), N (bits 17-22 =
@@ -195,15 +200,18 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
       : "memory");
 }
 
-template <typename OutT, int BN>
+template <typename OutT, int BN, int NA>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
+                  const __grid_constant__ CUtensorMap map_a1,
+                  const __grid_constant__ CUtensorMap map_a2,
                   const __grid_constant__ CUtensorMap map_b, const uint8_t *__restrict__ sfa,
                   const float *__restrict__ s_a, const uint8_t *__restrict__ sfb,
                   const float *__restrict__ s_b, int K, int n_tiles_n, int n_tiles,
                   OutT *__restrict__ c, int64_t ldc, int *__restrict__ status,
                   GemmOptions opt) {
-  using T = Tile<BN>;
+  using T = Tile<BN, NA>;
+  constexpr int STAGES = T::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -264,12 +272,16 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
           const uint32_t bar = full + 8 * s;
           mbar_expect_tx(bar, T::STAGE_BYTES);
           tma_load_2d(st, &map_a, kt * KTB, m0, bar);
-          tma_load_2d(st + T::A_BYTES, &map_b, kt * KTB, n0, bar);
-          bulk_load(st + T::A_BYTES + T::B_BYTES, sfa_tile + static_cast<int64_t>(kt) * SF_BYTES,
+          if (NA == 3) {
+            tma_load_2d(st + T::A_BYTES, &map_a1, kt * KTB, m0, bar);
+            tma_load_2d(st + 2 * T::A_BYTES, &map_a2, kt * KTB, m0, bar);
+          }
+          tma_load_2d(st + T::B_OFF, &map_b, kt * KTB, n0, bar);
+          bulk_load(st + T::B_OFF + T::B_BYTES, sfa_tile + static_cast<int64_t>(kt) * SF_BYTES,
                     SF_BYTES, bar);
 #pragma unroll
           for (int h = 0; h < BN / 128; ++h)
-            bulk_load(st + T::A_BYTES + T::B_BYTES + SF_BYTES + h * SF_BYTES,
+            bulk_load(st + T::B_OFF + T::B_BYTES + SF_BYTES + h * SF_BYTES,
                       sfb_tile + h * sf_rowtile + static_cast<int64_t>(kt) * SF_BYTES, SF_BYTES,
                       bar);
         }
@@ -298,18 +310,24 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
           const uint32_t sfb_col = sfa_col + 16u;
 #pragma unroll
           for (int kb = 0; kb < KTILE / 64; ++kb) {
-            tc_copy_sf(sfa_col + 4u * kb, desc_sf(st + T::A_BYTES + T::B_BYTES + kb * SF_TILE));
+            tc_copy_sf(sfa_col + 4u * kb, desc_sf(st + T::B_OFF + T::B_BYTES + kb * SF_TILE));
 #pragma unroll
             for (int h = 0; h < BN / 128; ++h)   // B rows 128h .. 128h + 127: columns 4h .. 4h + 3
               tc_copy_sf(sfb_col + (T::SFB_COLS / 4) * kb + 4u * h,
-                         desc_sf(st + T::A_BYTES + T::B_BYTES + SF_BYTES + h * SF_BYTES +
+                         desc_sf(st + T::B_OFF + T::B_BYTES + SF_BYTES + h * SF_BYTES +
                                  kb * SF_TILE));
           }
-          const uint64_t da = desc_sw128(st), db = desc_sw128(st + T::A_BYTES);
+          const uint64_t da = desc_sw128(st), db = desc_sw128(st + T::B_OFF);
 #pragma unroll
-          for (int kb = 0; kb < KTILE / 64; ++kb)       // 64 values = 32 bytes = 2 descriptor units
-            tc_mma(tmem, da + 2u * kb, db + 2u * kb, T::IDESC, sfa_col + 4u * kb,
-                   sfb_col + (T::SFB_COLS / 4) * kb, (kt | kb) != 0);
+          for (int kb = 0; kb < KTILE / 64; ++kb) {     // 64 values = 32 bytes = 2 descriptor units
+            const uint32_t sa = sfa_col + 4u * kb, sb = sfb_col + (T::SFB_COLS / 4) * kb;
+            tc_mma(tmem, da + 2u * kb, db + 2u * kb, T::IDESC, sa, sb, (kt | kb) != 0);
+            if (NA == 3) {                              // both INT4 parts into accumulator 1
+              const uint64_t da1 = desc_sw128(st + T::A_BYTES), da2 = desc_sw128(st + 2 * T::A_BYTES);
+              tc_mma(tmem + BN, da1 + 2u * kb, db + 2u * kb, T::IDESC, sa, sb, (kt | kb) != 0);
+              tc_mma(tmem + BN, da2 + 2u * kb, db + 2u * kb, T::IDESC, sa, sb, 1u);
+            }
+          }
           tc_commit(empty + 8 * s);
         }
         tc_commit(acc_full);                            // this tile's accumulator is complete
@@ -318,8 +336,27 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
   } else {
     // ---- epilogue: warp w reads accumulator lanes 32 (w % 4) .. + 31 ----
     const int quarter = warp & 3;
-    const float alpha =
+    const float a0 =
         __fmul_rn(__fmul_rn(s_a ? *s_a : 1.0f, s_b ? *s_b : 1.0f), opt.alpha_mul);
+    const float a1 = __fmul_rn(a0, opt.alpha_int);     // the second accumulator's factor
+    // with two accumulators the combined value is formed first and then
+    // multiplied by 1 (exact) in the conversions below
+    const float alpha = NA == 3 ? 1.0f : a0;
+    // 16 columns of this thread's row, combined from both accumulators (NA 3)
+    auto load_chunk = [&](uint32_t taddr, int j, uint32_t (&r)[16]) {
+      tc_load16(taddr + 16u * j, r);
+      if (NA == 3) {
+        uint32_t r1[16];
+        tc_load16(taddr + BN + 16u * j, r1);
+        tc_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          r[q] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(r[q]), a0),
+                                           __fmul_rn(__uint_as_float(r1[q]), a1)));
+      } else {
+        tc_wait_ld();
+      }
+    };
     int i = 0;
     for (int tile = blockIdx.x; tile < n_tiles && !*err_ptr; tile += gridDim.x, ++i) {
       const int ok = mbar_wait(acc_full, static_cast<uint32_t>(i & 1)) ? 1 : 0;
@@ -338,8 +375,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
 #pragma unroll
         for (int j = 0; j < BN / 16; ++j) {
           uint32_t r[16];
-          tc_load16(taddr + 16u * j, r);
-          tc_wait_ld();
+          load_chunk(taddr, j, r);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * q]), alpha),
@@ -360,8 +396,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
 #pragma unroll
         for (int j = 0; j < BN / 16; ++j) {
           uint32_t r[16];
-          tc_load16(taddr + 16u * j, r);
-          tc_wait_ld();
+          load_chunk(taddr, j, r);
           if (j == BN / 16 - 1) {
             tc_fence_before();
             __syncwarp();
@@ -369,18 +404,11 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
               asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty) : "memory");
           }
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float4 o = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), alpha),
-                                   __fmul_rn(__uint_as_float(r[4 * q + 1]), alpha),
-                                   __fmul_rn(__uint_as_float(r[4 * q + 2]), alpha),
-                                   __fmul_rn(__uint_as_float(r[4 * q + 3]), alpha));
-            if (opt.accumulate) {                       // C += RN(acc * alpha)
-              const float4 p = d[4 * j + q];
-              o = make_float4(__fadd_rn(p.x, o.x), __fadd_rn(p.y, o.y), __fadd_rn(p.z, o.z),
-                              __fadd_rn(p.w, o.w));
-            }
-            d[4 * j + q] = o;
-          }
+          for (int q = 0; q < 4; ++q)
+            d[4 * j + q] = make_float4(__fmul_rn(__uint_as_float(r[4 * q]), alpha),
+                                       __fmul_rn(__uint_as_float(r[4 * q + 1]), alpha),
+                                       __fmul_rn(__uint_as_float(r[4 * q + 2]), alpha),
+                                       __fmul_rn(__uint_as_float(r[4 * q + 3]), alpha));
         }
       }
     }
@@ -427,30 +455,34 @@ bool make_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t row_b
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename OutT, int BN>
-cudaError_t launch_t(const uint8_t *qa, const uint8_t *sfa, const float *s_a, const uint8_t *qb,
-                     const uint8_t *sfb, const float *s_b, int64_t M, int64_t N, int64_t K,
-                     void *c, int64_t ldc, int *status, GemmOptions opt, const Launch &L) {
-  using T = Tile<BN>;
+template <typename OutT, int BN, int NA>
+cudaError_t launch_t(const uint8_t *const (&qa)[3], const uint8_t *sfa, const float *s_a,
+                     const uint8_t *qb, const uint8_t *sfb, const float *s_b, int64_t M,
+                     int64_t N, int64_t K, void *c, int64_t ldc, int *status, GemmOptions opt,
+                     const Launch &L) {
+  using T = Tile<BN, NA>;
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        gemm_nvfp4_kernel<OutT, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM_BYTES);
+    const cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<OutT, BN, NA>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               T::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  CUtensorMap map_a, map_b;
-  if (!make_map(&map_a, qa, M, K / 2, BM) || !make_map(&map_b, qb, N, K / 2, BN))
-    return cudaErrorInvalidValue;
+  CUtensorMap map_a[3], map_b;
+  for (int i = 0; i < 3; ++i)
+    if (!make_map(&map_a[i], qa[NA == 3 ? i : 0], M, K / 2, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&map_b, qb, N, K / 2, BN)) return cudaErrorInvalidValue;
   // persistent: one CTA per SM (the stages fill its shared memory), output
   // tiles in row-major order, each CTA taking every gridDim-th tile
   const int64_t n_tiles_n = N / BN, n_tiles = (M / BM) * n_tiles_n;
   const int grid = static_cast<int>(n_tiles < L.num_sms ? n_tiles : L.num_sms);
-  gemm_nvfp4_kernel<OutT, BN><<<grid, kThreads, T::SMEM_BYTES, L.stream>>>(
-      map_a, map_b, sfa, s_a, sfb, s_b, static_cast<int>(K), static_cast<int>(n_tiles_n),
-      static_cast<int>(n_tiles), static_cast<OutT *>(c), ldc, status, opt);
+  gemm_nvfp4_kernel<OutT, BN, NA><<<grid, kThreads, T::SMEM_BYTES, L.stream>>>(
+      map_a[0], map_a[1], map_a[2], map_b, sfa, s_a, sfb, s_b, static_cast<int>(K),
+      static_cast<int>(n_tiles_n), static_cast<int>(n_tiles), static_cast<OutT *>(c), ldc,
+      status, opt);
   return cudaGetLastError();
 }
 
@@ -458,12 +490,27 @@ template <typename OutT>
 cudaError_t launch_o(const uint8_t *qa, const uint8_t *sfa, const float *s_a, const uint8_t *qb,
                      const uint8_t *sfb, const float *s_b, int64_t M, int64_t N, int64_t K,
                      void *c, int64_t ldc, int *status, GemmOptions opt, const Launch &L) {
+  const uint8_t *const a[3] = {qa, qa, qa};
   if (N % 256 == 0)
-    return launch_t<OutT, 256>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
-  return launch_t<OutT, 128>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
+    return launch_t<OutT, 256, 1>(a, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
+  return launch_t<OutT, 128, 1>(a, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
 }
 
 }  // namespace
+
+cudaError_t launch_gemm_if4_split(const uint8_t *q_fp, const uint8_t *q_k1, const uint8_t *q_k2,
+                                  const uint8_t *sfa, const float *s_a, const uint8_t *qb,
+                                  const uint8_t *sfb, const float *s_b, int64_t M, int64_t N,
+                                  int64_t K, void *c, int c_dtype, int64_t ldc, int *status,
+                                  const Launch &L) {
+  const uint8_t *const a[3] = {q_fp, q_k1, q_k2};
+  GemmOptions opt;
+  opt.alpha_int = 6.0f / 7.0f;                         // RN(6/7)
+  if (c_dtype == FP4Q_BF16)
+    return launch_t<__nv_bfloat16, 128, 3>(a, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status,
+                                           opt, L);
+  return launch_t<float, 128, 3>(a, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
+}
 
 cudaError_t launch_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *s_a,
                               const uint8_t *qb, const uint8_t *sfb, const float *s_b, int64_t M,

@@ -10,7 +10,8 @@
 // split into three NVFP4 operands that share the unflagged scales:
 //   A_fp: the FP4 blocks (INT4 blocks zero),
 //   A_1, A_2: the two E2M1 parts of each INT4 block (FP4 blocks zero),
-// and A B^T = A_fp B^T + RN(6/7) (A_1 B^T + A_2 B^T) up to rounding.  One
+// and A B^T = A_fp B^T + RN(6/7) (A_1 B^T + A_2 B^T) up to rounding (one GEMM
+// pass with two accumulators, in gemm.cu).  One
 // thread per 16-value block: 8 code bytes and a scale byte in, three times 8
 // code bytes and a scale byte out.
 #include "common.cuh"

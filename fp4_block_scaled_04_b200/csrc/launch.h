@@ -64,13 +64,13 @@ cudaError_t launch_mxfp6_dequant(const uint8_t *q, const uint8_t *sf, int scale_
                                  int64_t rows, int64_t cols, int fp6_format, void *y,
                                  int y_dtype, const Launch &L);
 
-// Options of the tensor-core GEMM: the product is scaled by RN(RN(s_a s_b) *
-// alpha_mul); accumulate != 0 adds it to the FP32 C already there (C =
-// RN(C + RN(acc * alpha))); withhold != 0 (a failure-detection test hook)
-// issues no operand loads.
+// Options of the tensor-core GEMM: the product is scaled by a = RN(RN(s_a s_b)
+// * alpha_mul); with a second accumulator (the IF4 GEMM) that one is scaled by
+// RN(a * alpha_int); withhold != 0 (a failure-detection test hook) issues no
+// operand loads.
 struct GemmOptions {
   float alpha_mul = 1.0f;
-  int accumulate = 0;
+  float alpha_int = 1.0f;
   int withhold = 0;
 };
 
@@ -80,6 +80,15 @@ cudaError_t launch_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float
                               const uint8_t *qb, const uint8_t *sfb, const float *s_b, int64_t M,
                               int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
                               int *status, GemmOptions opt, const Launch &L);
+
+// IF4 x NVFP4 in one pass over the split operands: C = RN(RN(acc_fp * a) +
+// RN(acc_int * RN(a * RN(6/7)))), acc_int accumulating both INT4 parts; FP32
+// or BF16 output, N % 128 == 0
+cudaError_t launch_gemm_if4_split(const uint8_t *q_fp, const uint8_t *q_k1, const uint8_t *q_k2,
+                                  const uint8_t *sfa, const float *s_a, const uint8_t *qb,
+                                  const uint8_t *sfb, const float *s_b, int64_t M, int64_t N,
+                                  int64_t K, void *c, int c_dtype, int64_t ldc, int *status,
+                                  const Launch &L);
 
 // Split IF4 codes [rows, K/2] with flagged scales into three NVFP4 code
 // matrices sharing the unflagged scales: FP4 blocks (INT4 blocks zero) and the

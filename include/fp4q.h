@@ -351,12 +351,13 @@ fp4q_status fp4q_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *
  * RN(6/7) * S is not an E4M3 value; every k in -7..7 is the sum of at most two
  * E2M1 values (5 = 4 + 1, 7 = 6 + 1), so A is split into three NVFP4 operands
  * sharing the unflagged scales (the FP4 blocks, and the two E2M1 parts of the
- * INT4 blocks) and
- *   C = RN(acc_fp * a) + RN(acc_1 * a67) + RN(acc_2 * a67) (added in that
- *   order, each sum rounded), a = RN(s_a * s_b), a67 = RN(a * RN(6/7)),
- * each acc accumulated in FP32 by tcgen05.mma.  The result is within FP32
- * accumulation and rounding error of the exact product of the dequantized IF4
- * and NVFP4 operands.
+ * INT4 blocks), and one GEMM pass accumulates the FP4 part and both INT4
+ * parts in two tensor-memory accumulators (FP32, by tcgen05.mma; B is read
+ * once):
+ *   C = RN(RN(acc_fp * a) + RN(acc_int * a67)),  a = RN(s_a * s_b),
+ *   a67 = RN(a * RN(6/7)).
+ * The result is within FP32 accumulation and rounding error of the exact
+ * product of the dequantized IF4 and NVFP4 operands.
  *   qa, sfa      IF4 codes [M, K/2] and flagged scales in the 128x4 layout, as
  *                fp4q_quantize_if4 writes them with FP4Q_SCALE_SWIZZLED_128x4
  *   qb, sfb      NVFP4 codes [N, K/2] and swizzled scales

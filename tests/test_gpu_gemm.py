@@ -226,9 +226,10 @@ def test_gemm_wait_that_runs_out_sets_status_and_leaves_the_context_usable(orc):
 @pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 384, 1024), (512, 256, 2048)])
 def test_if4_operand_in_the_tensor_core_gemm(orc, M, N, K):
     """IF4 x NVFP4: the IF4 operand split into FP4 blocks and the two E2M1
-    parts of its INT4 blocks, three accumulating GEMMs.  Compared with the
-    exact product of the dequantized IF4 and NVFP4 operands, with room for
-    three FP32 accumulations, the RN(6/7) factor and two output additions."""
+    parts of its INT4 blocks, one GEMM pass with an FP4 and an INT4
+    accumulator.  Compared with the exact product of the dequantized IF4 and
+    NVFP4 operands, with room for three FP32 accumulation chains, the RN(6/7)
+    factor and the output addition."""
     x = workloads.if4_blocks(rows=M, cols=K).to(DEV)
     g = torch.Generator().manual_seed(15)
     w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16).to(DEV)
