@@ -8,8 +8,8 @@ distributions as the benchmark, any size), copied to cuda:0, the tensor amax
 is computed once, then the kernel under study runs ``--warmup`` times and
 ``--iters`` times more, with a device synchronize at the end.  Each of those
 runs is exactly one launch of the kernel named by ``--op`` (the amax
-pre-pass is outside them), so a profiler can skip the warm-up launches and
-capture the rest.
+pre-pass is outside them; ``gemm_if4`` launches the IF4 split pass before
+its GEMM), so a profiler can skip the warm-up launches and capture the rest.
 """
 from __future__ import annotations
 
@@ -23,7 +23,7 @@ from fp4_block_scaled_04_b200 import workloads
 
 OPS = ["amax", "nvfp4_row", "nvfp4_rowcol", "mxfp4_rowcol", "2d", "rht16_sr", "rht128_sr",
        "rht16_rne", "rht128_rne", "if4", "if4_dequant", "four_over_six_rowcol", "nvint4",
-       "bwd16_sr", "bwd16_rne", "row_sr", "mxfp6_e2m3", "mxfp6_dequant", "gemm_nvfp4", "if6"]
+       "bwd16_sr", "bwd16_rne", "row_sr", "mxfp6_e2m3", "mxfp6_dequant", "gemm_nvfp4", "gemm_if4", "if6"]
 
 
 def make(op: str, rows: int, cols: int, dev):
@@ -56,6 +56,18 @@ def make(op: str, rows: int, cols: int, dev):
         return lambda: fq.fp4q_gemm_nvfp4(ox["q_row"], ox["sf_row"], ow["q_row"], ow["sf_row"],
                                           cols, tensor_scale_a=ox["s_dec"],
                                           tensor_scale_b=ow["s_dec"], out=c)
+    if op == "gemm_if4":                # IF4 x NVFP4, M = N = rows, K = cols, FP32 out
+        g = torch.Generator().manual_seed(6)
+        x = torch.randn(rows, cols, generator=g).to(torch.bfloat16).to(dev)
+        w = (torch.randn(rows, cols, generator=g) * 0.05).to(torch.bfloat16).to(dev)
+        ox = fq.fp4q_quantize_if4(x, scale_layout=fq.SCALE_SWIZZLED)
+        ow = fq.fp4q_quantize_nvfp4(w, scale_layout=fq.SCALE_SWIZZLED)
+        c = torch.empty((rows, rows), dtype=torch.float32, device=dev)
+        ws = torch.empty(int(fq.lib().fp4q_gemm_if4_workspace_bytes(rows, cols)),
+                         dtype=torch.uint8, device=dev)
+        return lambda: fq.fp4q_gemm_if4_nvfp4(ox["q"], ox["sf"], ow["q_row"], ow["sf_row"], cols,
+                                              tensor_scale_a=ox["s_dec"],
+                                              tensor_scale_b=ow["s_dec"], out=c, workspace=ws)
     if op in ("mxfp6_e2m3", "mxfp6_dequant"):
         x = workloads.activation(rows=rows, cols=cols).to(dev)
         o = fq.fp4q_quantize_mxfp6(x, fq.FP6_E2M3, scale_layout=sw)
