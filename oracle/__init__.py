@@ -30,7 +30,8 @@ ROWWISE, COLWISE = 1, 2
 RNE, SR = 0, 1
 SCALE_LINEAR, SCALE_SWIZZLED = 0, 1
 E8M0_RNE, E8M0_CEIL, E8M0_OCP_FLOOR = 0, 1, 2
-FMT_NVFP4, FMT_MXFP4, FMT_IF4, FMT_MXFP6_E2M3, FMT_MXFP6_E3M2, FMT_IF6 = 0, 1, 2, 3, 4, 5
+FMT_NVFP4, FMT_MXFP4, FMT_IF4, FMT_MXFP6_E2M3, FMT_MXFP6_E3M2, FMT_IF6, FMT_IF3 = (
+    0, 1, 2, 3, 4, 5, 6)
 FP6_E2M3, FP6_E3M2 = 0, 1
 
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
@@ -86,6 +87,11 @@ def lib() -> ctypes.CDLL:
             "orc_if6_cu": (F, []),
             "orc_if6_cd": (F, []),
             "orc_quantize_if6": (I, [P, I, I64, I64, I64, P, P, P, P, I, I]),
+            "orc_fp3_value": (F, [ctypes.c_uint8]),
+            "orc_fp3_rne": (ctypes.c_uint8, [F]),
+            "orc_if3_cu": (F, []),
+            "orc_if3_cd": (F, []),
+            "orc_quantize_if3": (I, [P, I, I64, I64, I64, P, P, P, P, I, I]),
             "orc_quantize_four_over_six": (I, [P, I, I64, I64, I64, U, P, P, P, P, P, P, I]),
             "orc_dequantize": (I, [I, P, P, I, I, I, P, I64, I64, P, I]),
             "orc_glossary_mae": (ctypes.c_double, [P, I64, I64]),
@@ -433,6 +439,37 @@ def quantize_if6(x: np.ndarray, amax: float | None = None, scale_layout: int = S
            "sf": np.zeros(scale_bytes(rows, cols // 16, scale_layout), np.uint8)}
     keep, ap = _amax_arg(amax)
     rc = lib().orc_quantize_if6(_ptr(x), _dtype_code(x), rows, cols, cols, ap,
+                                _ptr(out["s_dec"]), _ptr(out["q"]), _ptr(out["sf"]),
+                                scale_layout, mode)
+    if rc != 0:
+        raise ValueError(f"oracle rejected shape {x.shape}")
+    return out
+
+
+def fp3_value(code: int) -> float:
+    return float(lib().orc_fp3_value(code))
+
+
+def fp3_rne(v: float) -> int:
+    return int(lib().orc_fp3_rne(float(np.float32(v))))
+
+
+def if3_constants():
+    return float(lib().orc_if3_cu()), float(lib().orc_if3_cd())
+
+
+def quantize_if3(x: np.ndarray, amax: float | None = None, scale_layout: int = SCALE_LINEAR,
+                 mode: int = 1) -> dict:
+    """IF3 (mode 1): per 16-block FP3 E2M0 or INT3 (the 6/7 method with 3 and
+    4); mode 0 keeps FP3 everywhere, mode 2 INT3 everywhere.  Codes
+    [rows, cols * 3/8] (eight 3-bit codes per three bytes)."""
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    out = {"s_dec": np.zeros(1, np.float32),
+           "q": np.zeros((rows, cols * 3 // 8), np.uint8),
+           "sf": np.zeros(scale_bytes(rows, cols // 16, scale_layout), np.uint8)}
+    keep, ap = _amax_arg(amax)
+    rc = lib().orc_quantize_if3(_ptr(x), _dtype_code(x), rows, cols, cols, ap,
                                 _ptr(out["s_dec"]), _ptr(out["q"]), _ptr(out["sf"]),
                                 scale_layout, mode)
     if rc != 0:

@@ -50,6 +50,7 @@
 #define ORC_FMT_MXFP6_E2M3 3
 #define ORC_FMT_MXFP6_E3M2 4
 #define ORC_FMT_IF6 5
+#define ORC_FMT_IF3 6
 #define ORC_FP6_E2M3 0
 #define ORC_FP6_E3M2 1
 
@@ -836,11 +837,117 @@ int orc_quantize_if6(const void *x, int dtype, int64_t rows, int64_t cols, int64
 }
 
 /* ------------------------------------------------------------------------ */
+/* IF3: the IF idea at 3 bits.  [I] section 2 names IF3 beside IF6 and gives */
+/* no details.  READING:                                                      */
+/*   a 3-bit code is a sign and two magnitude bits.  Of the two float splits */
+/*   of two bits, E1M1 has the uniform magnitudes 0, 0.5, 1, 1.5, which are  */
+/*   INT3's 0..3 times 0.5: with it the FP/INT choice would have nothing to  */
+/*   choose between.  So the FP candidate is FP3 E2M0 (two exponent bits,    */
+/*   bias 1, no mantissa; exponent field 0 is zero, as in E2M1 with a zero   */
+/*   mantissa): magnitudes 0, 1, 2, 4;                                       */
+/*   the block scale maps the block maximum to 4 (as 4/6 does):             */
+/*     s_enc = RN(1792/amax), s_dec = RN(amax/1792) with 1792 = 4 * 448,    */
+/*     S = E4M3_rne_sat(RN(RN(m * s_enc) / 4)), r = RN(s_enc / S),           */
+/*     v_i = RN(x_i * r);                                                    */
+/*   FP3:  g_i = E2M0 value of the nearest magnitude (ties to the even code, */
+/*         saturating at 4), sign copied;                                    */
+/*   INT3 (the 6/7 method with 3 and 4): k_i = clamp(rint(RN(v_i * CU)),     */
+/*         -3, 3), h_i = RN(k_i * CD), CU = RN(3/4), CD = RN(4/3);           */
+/*   errors, their order and the choice exactly as IF4 (INT3 iff strictly    */
+/*   smaller); scale bit 7 set = INT3.                                       */
+/* Codes are 3 bits (FP3: sign in bit 2, magnitude code in bits 0-1; INT3:  */
+/* k_i in 3-bit two's complement), packed eight per three bytes, code j of  */
+/* the group in bits 3j..3j+2 of the little-endian 24-bit word: codes       */
+/* [rows, cols * 3/8], scales [rows, cols/16].  int3_mode 0 keeps FP3       */
+/* everywhere, 1 is IF3, 2 keeps INT3 everywhere.                           */
+/* ------------------------------------------------------------------------ */
+
+float orc_fp3_value(uint8_t code) {
+  static const float mag[4] = {0.0f, 1.0f, 2.0f, 4.0f};
+  float v = mag[code & 0x3];
+  return (code & 0x4) ? -v : v;
+}
+
+/* nearest E2M0 magnitude (ties to the even code), saturating at 4, sign
+ * copied; v finite */
+uint8_t orc_fp3_rne(float v) {
+  uint8_t sign = signbit(v) ? 0x4 : 0x0;
+  double a = fabs((double)v);
+  int best = 0;
+  double best_d = INFINITY;
+  for (int c = 0; c < 4; ++c) {
+    double d = fabs(a - (double)orc_fp3_value((uint8_t)c));
+    if (d < best_d || (d == best_d && (c % 2) == 0)) { best = c; best_d = d; }
+  }
+  return (uint8_t)(best | sign);
+}
+
+float orc_if3_cu(void) { return 3.0f / 4.0f; }
+float orc_if3_cd(void) { return 4.0f / 3.0f; }
+
+int orc_quantize_if3(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                     const float *amax_in, float *s_dec_out, uint8_t *q, uint8_t *sf_out,
+                     int scale_layout, int int3_mode) {
+  if (cols % 16 != 0) return 1;
+  float amax = amax_in ? *amax_in : orc_amax(x, dtype, rows, cols, ld);
+  float s_enc, s_dec;
+  tensor_scales_top(amax, 4.0f * 448.0f, &s_enc, &s_dec);
+  if (s_dec_out) *s_dec_out = s_dec;
+  const float CU = orc_if3_cu(), CD = orc_if3_cd();
+  const int64_t rb = cols * 3 / 8;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < cols / 16; ++b) {
+      float xv[16];
+      float m = 0.0f;
+      for (int k = 0; k < 16; ++k) {
+        xv[k] = load_elem(x, dtype, ld, r, b * 16 + k);
+        if (fabsf(xv[k]) > m) m = fabsf(xv[k]);
+      }
+      uint8_t sf = block_scale_q(m, s_enc, 4.0f);
+      float rf = nvfp4_block_factor(sf, s_enc);
+      uint8_t fp_code[16], int_code[16];
+      float e_fp = 0.0f, e_int = 0.0f;
+      for (int k = 0; k < 16; ++k) {
+        float v = xv[k] * rf;
+        fp_code[k] = orc_fp3_rne(v);
+        float g = orc_fp3_value(fp_code[k]);
+        float kk = rintf(v * CU);
+        if (kk > 3.0f) kk = 3.0f;
+        if (kk < -3.0f) kk = -3.0f;
+        int ki = (int)kk;
+        int_code[k] = (uint8_t)(ki & 0x7);
+        float h = (float)ki * CD;
+        float d_fp = v - g;
+        float d_int = v - h;
+        e_fp = fmaf(d_fp, d_fp, e_fp);
+        e_int = fmaf(d_int, d_int, e_int);
+      }
+      int use_int = int3_mode == 2 || (int3_mode == 1 && e_int < e_fp);
+      sf_out[orc_scale_offset(r, b, rows, cols / 16, scale_layout)] =
+          (uint8_t)(sf | (use_int ? 0x80 : 0x00));
+      for (int g8 = 0; g8 < 2; ++g8) {
+        uint32_t w = 0;
+        for (int j = 0; j < 8; ++j) {
+          int k = g8 * 8 + j;
+          w |= (uint32_t)(use_int ? int_code[k] : fp_code[k]) << (3 * j);
+        }
+        uint8_t *dst = q + r * rb + (b * 2 + g8) * 3;
+        dst[0] = (uint8_t)(w & 0xFF);
+        dst[1] = (uint8_t)((w >> 8) & 0xFF);
+        dst[2] = (uint8_t)((w >> 16) & 0xFF);
+      }
+    }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Dequantization  [G] "FP4の仕組み" (reconstruct = grid value * sign * scale)*/
 /* NVFP4:  y = RN(RN(g * S) * s_dec)   (g * S is exact)                       */
 /* IF4 INT4 blocks: h = RN(k * C67), y = RN(RN(h * S) * s_dec)                */
 /* MXFP4:  y = RN(g * 2^e)                                                    */
 /* MXFP6 (E2M3 / E3M2, codes packed 4 per 3 bytes): y = RN(value * 2^e)      */
+/* IF6 / IF3: FP blocks as NVFP4 with the FP6 E2M3 / FP3 E2M0 value, INT      */
+/* blocks as IF4 with CD6 = RN(7.5/31) / CD3 = RN(4/3); codes 4 / 8 per 3 B   */
 /* Block shape: block_rows x block_cols (1x16, 1x32, or 16x16 for 2D tiles,  */
 /* whose scales are [rows/16, cols/16] linear).  Output FP32 or BF16 (RNE of */
 /* the FP32 result).                                                         */
@@ -852,13 +959,18 @@ int orc_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_la
   if (cols % block_cols != 0 || rows % block_rows != 0) return 1;
   float s_dec = s_dec_in ? *s_dec_in : 1.0f;
   int64_t srows = rows / block_rows, scols = cols / block_cols;
-  const float C67 = orc_if4_c67(), CD6 = orc_if6_cd();
+  const float C67 = orc_if4_c67(), CD6 = orc_if6_cd(), CD3 = orc_if3_cd();
   const int fp6 = (format == ORC_FMT_MXFP6_E2M3 || format == ORC_FMT_MXFP6_E3M2);
   const int six = fp6 || format == ORC_FMT_IF6;             /* 6-bit codes, 4 per 3 bytes */
+  const int three = format == ORC_FMT_IF3;                  /* 3-bit codes, 8 per 3 bytes */
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t c = 0; c < cols; ++c) {
       uint8_t code;
-      if (six) {
+      if (three) {
+        const uint8_t *g3 = q + r * (cols * 3 / 8) + (c / 8) * 3;
+        uint32_t w = (uint32_t)g3[0] | ((uint32_t)g3[1] << 8) | ((uint32_t)g3[2] << 16);
+        code = (uint8_t)((w >> (3 * (c % 8))) & 0x7);
+      } else if (six) {
         const uint8_t *g3 = q + r * (cols * 3 / 4) + (c / 4) * 3;
         uint32_t w = (uint32_t)g3[0] | ((uint32_t)g3[1] << 8) | ((uint32_t)g3[2] << 16);
         code = (uint8_t)((w >> (6 * (c % 4))) & 0x3F);
@@ -888,6 +1000,12 @@ int orc_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_la
           out = (h * S) * s_dec;
         } else if (format == ORC_FMT_IF6) {
           out = (orc_fp6_value(code, ORC_FP6_E2M3) * S) * s_dec;
+        } else if (format == ORC_FMT_IF3 && (s & 0x80)) {
+          int k = (code & 0x4) ? (int)code - 8 : (int)code;
+          float h = (float)k * CD3;
+          out = (h * S) * s_dec;
+        } else if (format == ORC_FMT_IF3) {
+          out = (orc_fp3_value(code) * S) * s_dec;
         } else {
           out = (orc_e2m1_value(code) * S) * s_dec;
         }
