@@ -302,7 +302,7 @@ def build_extra_jobs(device, fq, inputs):
     gradient workload, and the IF4 explainer's comparison formats
     (four-over-six on the activation workload, NVINT4 on the IF4 workload),
     the tensor amax of the activation workload (which the suite takes as given),
-    IF6 on the IF4 workload and MXFP6 E2M3 on the activation workload."""
+    IF6 and IF3 on the IF4 workload and MXFP6 E2M3 on the activation workload."""
     import torch
     SW = fq.SCALE_SWIZZLED
     xa = inputs["activation"].to(device)
@@ -333,6 +333,9 @@ def build_extra_jobs(device, fq, inputs):
     # IF6 of the IF4 workload: 2 bytes in, 0.75 + 1/16 out
     oi6 = fq.fp4q_quantize_if6(x5, amax=amax5, scale_layout=SW)
     nbi6 = R5 * C5 * 2 + R5 * C5 * 3 // 4 + R5 * C5 // 16 + 4
+    # IF3 of the IF4 workload: 2 bytes in, 0.375 + 1/16 out
+    oi3 = fq.fp4q_quantize_if3(x5, amax=amax5, scale_layout=SW)
+    nbi3 = R5 * C5 * 2 + R5 * C5 * 3 // 8 + R5 * C5 // 16 + 4
     # MXFP6 (E2M3) of the activation workload: 2 bytes in, 0.75 + 1/32 out
     o6 = fq.fp4q_quantize_mxfp6(xa, fq.FP6_E2M3, scale_layout=SW)
     nb6 = R * C * 2 + R * C * 3 // 4 + R * C // 32
@@ -361,6 +364,8 @@ def build_extra_jobs(device, fq, inputs):
             lambda: fq.fp4q_amax(xa, out=amax_a)),
         Job("if4 16384x8192 bf16 if6", "if6.cu", nbi6, 1,
             lambda: fq.fp4q_quantize_if6(x5, amax=amax5, scale_layout=SW, out=oi6)),
+        Job("if4 16384x8192 bf16 if3", "if3.cu", nbi3, 1,
+            lambda: fq.fp4q_quantize_if3(x5, amax=amax5, scale_layout=SW, out=oi3)),
         Job("activation 8192x4096 bf16 mxfp6 e2m3 row-wise", "mxfp6.cu", nb6, 1,
             lambda: fq.fp4q_quantize_mxfp6(xa, fq.FP6_E2M3, scale_layout=SW, out=o6)),
     ]

@@ -35,14 +35,15 @@ __all__ = [
     "fp4q_quantize_nvfp4_noalloc", "fp4q_quantize_nvint4", "fp4q_quantize_four_over_six",
     "fp4q_quantize_backward", "fp4q_quantize_mxfp6", "FMT_MXFP6_E2M3", "FMT_MXFP6_E3M2",
     "FP6_E2M3", "FP6_E3M2", "fp4q_gemm_nvfp4", "fp4q_quantize_if6", "FMT_IF6",
-    "fp4q_gemm_if4_nvfp4",
+    "fp4q_gemm_if4_nvfp4", "fp4q_quantize_if3", "FMT_IF3",
 ]
 
 ROWWISE, COLWISE = 1, 2
 RNE, SR = 0, 1
 SCALE_LINEAR, SCALE_SWIZZLED = 0, 1
 E8M0_RNE, E8M0_CEIL, E8M0_OCP_FLOOR = 0, 1, 2
-FMT_NVFP4, FMT_MXFP4, FMT_IF4, FMT_MXFP6_E2M3, FMT_MXFP6_E3M2, FMT_IF6 = 0, 1, 2, 3, 4, 5
+FMT_NVFP4, FMT_MXFP4, FMT_IF4, FMT_MXFP6_E2M3, FMT_MXFP6_E3M2, FMT_IF6, FMT_IF3 = (
+    0, 1, 2, 3, 4, 5, 6)
 FP6_E2M3, FP6_E3M2 = 0, 1
 _BF16, _FP32 = 0, 1
 
@@ -103,6 +104,7 @@ _SIGNATURES = {
     "fp4q_gemm_if4_nvfp4": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _SZ,
                                  _P, _P]),
     "fp4q_quantize_if6": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _SZ, _P]),
+    "fp4q_quantize_if3": (_I, [_P, _I, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _SZ, _P]),
 }
 
 
@@ -296,6 +298,22 @@ def fp4q_quantize_if6(x: torch.Tensor, amax: torch.Tensor | None = None,
     return out
 
 
+def fp4q_quantize_if3(x: torch.Tensor, amax: torch.Tensor | None = None,
+                      scale_layout: int = SCALE_LINEAR, out: dict | None = None) -> dict:
+    """IF3 (FP3 E2M0 or INT3 per 16-block); returns {'s_dec', 'q' [rows, cols*3/8], 'sf'}."""
+    rows, cols, ld = _matrix(x)
+    dev = x.device
+    if out is None:
+        out = {"s_dec": torch.empty(1, dtype=torch.float32, device=dev),
+               "q": _u8((rows, cols * 3 // 8), dev),
+               "sf": _u8(fp4q_scale_bytes(rows, cols, 16, scale_layout), dev)}
+    ws = _workspace(dev) if amax is None else None
+    _check("fp4q_quantize_if3", lib().fp4q_quantize_if3(
+        _ptr(x), _dtype(x), rows, cols, ld, _ptr(amax), _ptr(out.get("s_dec")), _ptr(out["q"]),
+        _ptr(out["sf"]), scale_layout, _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
+    return out
+
+
 def fp4q_gemm_nvfp4(qa: torch.Tensor, sfa: torch.Tensor, qb: torch.Tensor, sfb: torch.Tensor,
                     K: int, tensor_scale_a: torch.Tensor | None = None,
                     tensor_scale_b: torch.Tensor | None = None,
@@ -481,8 +499,8 @@ def fp4q_dequantize(fmt: int, q: torch.Tensor, sf: torch.Tensor, rows: int, cols
                     tensor_scale: torch.Tensor | None = None, scale_layout: int = SCALE_LINEAR,
                     out_dtype: torch.dtype = torch.float32,
                     out: torch.Tensor | None = None) -> torch.Tensor:
-    """Packed codes ([rows, cols/2], or [rows, cols*3/4] for MXFP6) + scales ->
-    [rows, cols] in out_dtype (fp32 or bf16)."""
+    """Packed codes ([rows, cols/2]; [rows, cols*3/4] for MXFP6 and IF6; [rows,
+    cols*3/8] for IF3) + scales -> [rows, cols] in out_dtype (fp32 or bf16)."""
     if not q.is_cuda:
         raise ValueError("q must be a CUDA tensor")
     y = torch.empty((rows, cols), dtype=out_dtype, device=q.device) if out is None else out

@@ -514,6 +514,35 @@ fp4q_status fp4q_quantize_if6(const void *x, int dtype, int64_t rows, int64_t co
       launch_if6(x, dtype, rows, cols, ld, a, tensor_scale_out, q, sf, scale_layout, L));
 }
 
+fp4q_status fp4q_quantize_if3(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                              const float *amax, float *tensor_scale_out, uint8_t *q, uint8_t *sf,
+                              int scale_layout, void *workspace, size_t ws_bytes, void *stream) {
+  FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
+  if (!valid_layout(scale_layout)) return FP4Q_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
+  if ((!q || !sf) && rows > 0 && cols > 0) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned16(q)) return FP4Q_ERR_MISALIGNED;
+  FP4Q_TRY(check_swizzle(scale_layout, rows, cols / 16));
+  Launch L;
+  bool none = false;
+  FP4Q_TRY(bind_first({x, tensor_scale_out, amax}, stream, &L, &none));
+  if (none) return FP4Q_OK;
+  if (rows > 0 && cols > 0) {
+    FP4Q_TRY(check_dev(q, false));
+    FP4Q_TRY(check_dev(sf, false));
+  }
+  FP4Q_TRY(check_dev(amax, true));
+  FP4Q_TRY(check_dev(tensor_scale_out, true));
+  const float *a = nullptr;
+  FP4Q_TRY(resolve_amax(x, dtype, rows, cols, ld, amax, workspace, ws_bytes, L, &a));
+  if (rows == 0 || cols == 0) {
+    if (tensor_scale_out) write_s_dec_top_kernel<<<1, 1, 0, L.stream>>>(a, 1792.0f, tensor_scale_out);
+    return cuda_status(cudaGetLastError());
+  }
+  return cuda_status(
+      launch_if3(x, dtype, rows, cols, ld, a, tensor_scale_out, q, sf, scale_layout, L));
+}
+
 fp4q_status fp4q_quantize_mxfp6(const void *x, int dtype, int64_t rows, int64_t cols,
                                 int64_t ld, int fp6_format, int e8m0_mode, uint8_t *q,
                                 uint8_t *sf, int scale_layout, void *stream) {
@@ -657,15 +686,15 @@ extern "C" {
 fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,
                             int block_rows, int block_cols, const float *tensor_scale,
                             int64_t rows, int64_t cols, void *y, int y_dtype, void *stream) {
-  if (format < FP4Q_FMT_NVFP4 || format > FP4Q_FMT_IF6) return FP4Q_ERR_INVALID_ARG;
+  if (format < FP4Q_FMT_NVFP4 || format > FP4Q_FMT_IF3) return FP4Q_ERR_INVALID_ARG;
   const bool fp6 = format == FP4Q_FMT_MXFP6_E2M3 || format == FP4Q_FMT_MXFP6_E3M2;
   const bool pow2 = fp6 || format == FP4Q_FMT_MXFP4;   // E8M0 scales, no tensor scale
   if (!valid_layout(scale_layout) || !valid_dtype(y_dtype)) return FP4Q_ERR_INVALID_ARG;
   if (rows < 0 || cols < 0) return FP4Q_ERR_INVALID_ARG;
   const bool shape_ok =
       (pow2 && block_rows == 1 && block_cols == 32) ||
-      ((format == FP4Q_FMT_IF4 || format == FP4Q_FMT_IF6) && block_rows == 1 &&
-       block_cols == 16) ||
+      ((format == FP4Q_FMT_IF4 || format == FP4Q_FMT_IF6 || format == FP4Q_FMT_IF3) &&
+       block_rows == 1 && block_cols == 16) ||
       (format == FP4Q_FMT_NVFP4 && block_cols == 16 && (block_rows == 1 || block_rows == 16));
   if (!shape_ok) return FP4Q_ERR_INVALID_ARG;
   if (cols % block_cols != 0 || rows % block_rows != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
@@ -682,6 +711,9 @@ fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int
   if (format == FP4Q_FMT_IF6)
     return cuda_status(
         launch_if6_dequant(q, sf, scale_layout, tensor_scale, rows, cols, y, y_dtype, L));
+  if (format == FP4Q_FMT_IF3)
+    return cuda_status(
+        launch_if3_dequant(q, sf, scale_layout, tensor_scale, rows, cols, y, y_dtype, L));
   if (fp6)
     return cuda_status(launch_mxfp6_dequant(
         q, sf, scale_layout, rows, cols,

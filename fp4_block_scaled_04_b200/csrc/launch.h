@@ -106,6 +106,15 @@ cudaError_t launch_if6_dequant(const uint8_t *q, const uint8_t *sf, int scale_la
                                const float *s_dec, int64_t rows, int64_t cols, void *y,
                                int y_dtype, const Launch &L);
 
+// IF3: per 16-value block FP3 E2M0 or INT3 (rescaled by 4/3), codes eight
+// per three bytes; and its decode
+cudaError_t launch_if3(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                       const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,
+                       int scale_layout, const Launch &L);
+cudaError_t launch_if3_dequant(const uint8_t *q, const uint8_t *sf, int scale_layout,
+                               const float *s_dec, int64_t rows, int64_t cols, void *y,
+                               int y_dtype, const Launch &L);
+
 // int4_mode 1: IF4 (per-block choice); 2: NVINT4 (the INT4 candidate everywhere)
 cudaError_t launch_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                        const float *amax, float *s_dec_out, uint8_t *q, uint8_t *sf,

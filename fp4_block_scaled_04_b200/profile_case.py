@@ -23,7 +23,8 @@ from fp4_block_scaled_04_b200 import workloads
 
 OPS = ["amax", "nvfp4_row", "nvfp4_rowcol", "mxfp4_rowcol", "2d", "rht16_sr", "rht128_sr",
        "rht16_rne", "rht128_rne", "if4", "if4_dequant", "four_over_six_rowcol", "nvint4",
-       "bwd16_sr", "bwd16_rne", "row_sr", "mxfp6_e2m3", "mxfp6_dequant", "gemm_nvfp4", "gemm_if4", "if6"]
+       "bwd16_sr", "bwd16_rne", "row_sr", "mxfp6_e2m3", "mxfp6_dequant", "gemm_nvfp4", "gemm_if4", "if6", "if3",
+       "if3_dequant"]
 
 
 def make(op: str, rows: int, cols: int, dev):
@@ -81,6 +82,15 @@ def make(op: str, rows: int, cols: int, dev):
         a = fq.fp4q_amax(x)
         o = fq.fp4q_quantize_if6(x, amax=a, scale_layout=sw)
         return lambda: fq.fp4q_quantize_if6(x, amax=a, scale_layout=sw, out=o)
+    if op in ("if3", "if3_dequant"):
+        x = workloads.if4_blocks(rows=rows, cols=cols).to(dev)
+        a = fq.fp4q_amax(x)
+        o = fq.fp4q_quantize_if3(x, amax=a, scale_layout=sw)
+        if op == "if3":
+            return lambda: fq.fp4q_quantize_if3(x, amax=a, scale_layout=sw, out=o)
+        y = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+        return lambda: fq.fp4q_dequantize(fq.FMT_IF3, o["q"], o["sf"], rows, cols, 1, 16,
+                                          tensor_scale=o["s_dec"], scale_layout=sw, out=y)
     if op == "nvint4":
         x = workloads.if4_blocks(rows=rows, cols=cols).to(dev)
         a = fq.fp4q_amax(x)

@@ -84,7 +84,8 @@ typedef enum {
   FP4Q_FMT_IF4 = 2,
   FP4Q_FMT_MXFP6_E2M3 = 3,   /* codes packed four per three bytes */
   FP4Q_FMT_MXFP6_E3M2 = 4,
-  FP4Q_FMT_IF6 = 5           /* 6-bit codes, four per three bytes */
+  FP4Q_FMT_IF6 = 5,          /* 6-bit codes, four per three bytes */
+  FP4Q_FMT_IF3 = 6           /* 3-bit codes, eight per three bytes */
 } fp4q_format;
 typedef enum { FP4Q_FP6_E2M3 = 0, FP4Q_FP6_E3M2 = 1 } fp4q_fp6_format;
 
@@ -285,6 +286,32 @@ fp4q_status fp4q_quantize_if6(const void *x, int dtype, int64_t rows, int64_t co
                               const float *amax, float *tensor_scale_out, uint8_t *q, uint8_t *sf,
                               int scale_layout, void *workspace, size_t ws_bytes, void *stream);
 
+/* IF3: the IF per-block choice at 3 bits ("Adaptive Block-Scaled Data Types"
+ * explainer, section 2, names IF3 beside IF6).  The library's reading: a
+ * 3-bit code is a sign and two magnitude bits; the float split E1M1 would
+ * give the uniform magnitudes 0, 0.5, 1, 1.5, which are INT3 times 0.5 and
+ * leave nothing to choose, so the float grid is FP3 E2M0 (two exponent bits,
+ * bias 1, no mantissa; field 0 is zero): magnitudes 0, 1, 2, 4.  Against it
+ * INT3 (-3..3) rescaled by 4/3, with NVFP4's scaling at 4 in place of 6:
+ *   s_enc = RN(1792/amax), s_dec = RN(amax/1792)       (1792 = 4 * 448)
+ *   S = E4M3_rne_sat(RN(RN(m * s_enc) / 4)), r = RN(s_enc / S), v = RN(x*r)
+ *   FP3:  nearest of 0, 1, 2, 4 to |v|, ties to the even code (0.5 -> 0,
+ *         1.5 -> 2, 3 -> 2), saturating at 4, sign copied
+ *   INT3: k = clamp(rint(RN(v * 0.75)), -3, 3), value RN(k * RN(4/3))
+ *   errors sum fma(d, d, e) over the block in order, d = RN(v - value);
+ *   INT3 iff its error is strictly smaller; scale bit 7 set = INT3.
+ *   q   [rows, cols * 3/8] bytes: eight 3-bit codes per three bytes, code j
+ *       of a group in bits 3j..3j+2 of the little-endian 24-bit word (FP3:
+ *       sign in bit 2, the magnitude's index 0..3 in bits 0-1; INT3: k in
+ *       3-bit two's complement)
+ *   sf  [rows, cols/16] flagged E4M3 scales in scale_layout
+ * amax, tensor_scale_out, workspace and errors as for fp4q_quantize_if4;
+ * shape cols % 16 == 0.  fp4q_dequantize(FP4Q_FMT_IF3, ..., 1, 16, s_dec, ...)
+ * decodes it: y = RN(RN(value * S) * s_dec). */
+fp4q_status fp4q_quantize_if3(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                              const float *amax, float *tensor_scale_out, uint8_t *q, uint8_t *sf,
+                              int scale_layout, void *workspace, size_t ws_bytes, void *stream);
+
 /* MXFP6 1x32, row-wise: the OCP FP6 element formats with E8M0 block scales.
  * "FP6から考えるLLM量子化" (blog.ast.moe), "FP6で隣り合う値の間隔を見てみる":
  * E2M3 (sign, 2 exponent bits with bias 1, 3 mantissa bits; largest 7.5)
@@ -395,9 +422,12 @@ fp4q_status fp4q_gemm_nvfp4_withhold_loads(const uint8_t *qa, const uint8_t *sfa
  *          cols * 3/4] bytes packed as fp4q_quantize_mxfp6 writes them
  *   IF6    y = RN(RN(value * S) * s_dec)        block 1x16, 6-bit codes as
  *          fp4q_quantize_if6 writes them (INT6 blocks: value = RN(k * RN(7.5/31)))
- *   block_rows x block_cols: 1x16 (NVFP4, IF4, IF6), 16x16 (NVFP4 2D tiles; then
+ *   IF3    y = RN(RN(value * S) * s_dec)        block 1x16, 3-bit codes as
+ *          fp4q_quantize_if3 writes them (INT3 blocks: value = RN(k * RN(4/3)))
+ *   block_rows x block_cols: 1x16 (NVFP4, IF4, IF6, IF3), 16x16 (NVFP4 2D tiles; then
  *   sf is the linear [rows/16, cols/16] tile matrix), 1x32 (MXFP4, MXFP6).
- *   tensor_scale: device float s_dec (NVFP4 / IF4 / IF6), ignored for MXFP4/6.
+ *   tensor_scale: device float s_dec (NVFP4 / IF4 / IF6 / IF3), ignored for
+ *   MXFP4/6.
  *   Column-wise outputs are dequantized as the [cols, rows] matrices they are.
  * Shape: cols % block_cols == 0, rows % block_rows == 0. */
 fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,

@@ -32,7 +32,7 @@ def test_header_declares_the_entry_points():
               "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
               "fp4q_scale_bytes", "fp4q_workspace_bytes", "fp4q_status_string", "fp4q_version",
               "fp4q_quantize_mxfp6", "fp4q_gemm_nvfp4", "fp4q_quantize_if6",
-              "fp4q_gemm_if4_nvfp4"]:
+              "fp4q_gemm_if4_nvfp4", "fp4q_quantize_if3"]:
         assert n in names
 
 
@@ -187,7 +187,21 @@ def test_host_side_argument_checks_of_the_added_calls(L):
     # dequantize: MXFP6 formats take 1x32 blocks and no tensor scale
     assert L.fp4q_dequantize(3, FAKE, FAKE, 0, 1, 16, None, 16, 64, FAKE, 1, None) == 1
     assert L.fp4q_dequantize(4, FAKE, FAKE, 0, 1, 32, None, 16, 48, FAKE, 1, None) == 2
-    assert L.fp4q_dequantize(6, FAKE, FAKE, 0, 1, 32, None, 16, 64, FAKE, 1, None) == 1
+    assert L.fp4q_dequantize(7, FAKE, FAKE, 0, 1, 16, FAKE, 16, 64, FAKE, 1, None) == 1
+    # IF3: the IF4 rules, 1x16 blocks with a tensor scale
+    assert L.fp4q_quantize_if3(FAKE, 0, 16, 40, 40, FAKE, FAKE, FAKE, FAKE, 0, None, 0,
+                               None) == 2
+    assert L.fp4q_quantize_if3(FAKE, 0, 16, 48, 52, FAKE, FAKE, FAKE, FAKE, 0, None, 0,
+                               None) == 3
+    assert L.fp4q_quantize_if3(FAKE, 0, 16, 48, 48, FAKE, FAKE, FAKE, FAKE, 4, None, 0,
+                               None) == 1
+    assert L.fp4q_quantize_if3(FAKE, 0, 16, 48, 48, FAKE, FAKE, None, FAKE, 0, None, 0,
+                               None) == 1
+    assert L.fp4q_quantize_if3(FAKE, 0, 16, 48, 48, FAKE, FAKE,
+                               ctypes.c_void_p(0x7F0000000008), FAKE, 0, None, 0, None) == 3
+    assert L.fp4q_dequantize(6, FAKE, FAKE, 0, 1, 32, FAKE, 16, 64, FAKE, 1, None) == 1
+    assert L.fp4q_dequantize(6, FAKE, FAKE, 0, 1, 16, None, 16, 64, FAKE, 1, None) == 1
+    assert L.fp4q_dequantize(6, FAKE, FAKE, 0, 1, 16, FAKE, 16, 40, FAKE, 1, None) == 2
 
 
 def test_python_binding_refuses_cpu_tensors(L):

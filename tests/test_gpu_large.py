@@ -75,15 +75,18 @@ def test_large_mxfp6(orc, big):
     assert_same("sf", sample(out["sf"].view(R, C // 32)), want["sf"])
 
 
-@pytest.mark.parametrize("fmt", ["if4", "if6"])
+@pytest.mark.parametrize("fmt", ["if4", "if6", "if3"])
 def test_large_if(orc, big, fmt):
     x, amax = big
     if fmt == "if4":
         out = fq.fp4q_quantize_if4(x, amax=amax)
         want = orc.quantize_if4(bits(x[ROWS]), amax=PEAK)
-    else:
+    elif fmt == "if6":
         out = fq.fp4q_quantize_if6(x, amax=amax)
         want = orc.quantize_if6(bits(x[ROWS]), amax=PEAK)
+    else:
+        out = fq.fp4q_quantize_if3(x, amax=amax)
+        want = orc.quantize_if3(bits(x[ROWS]), amax=PEAK)
     assert_same("s_dec", host(out["s_dec"]), want["s_dec"])
     assert_same("q", sample(out["q"]), want["q"])
     assert_same("sf", sample(out["sf"].view(R, C // 16)), want["sf"])
