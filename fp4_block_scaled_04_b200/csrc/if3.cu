@@ -20,9 +20,10 @@
 // Codes are 3 bits (sign in bit 2 and the magnitude's index, or k in two's
 // complement), eight per three bytes (code j of a group in bits 3j..3j+2),
 // so a block is 6 bytes.
-// Quantize: one thread per block, 32 or 64 bytes in, three 2-byte code
-// stores and a scale byte out; r comes from a per-CTA table over the 128
-// scale codes.  The FP3 rounding is three comparisons: with s1 = [|v| > 0.5],
+// Quantize: one thread per pair of blocks, whose elements go through the
+// arithmetic as the two lanes of f32x2 instructions; 64 or 128 bytes in,
+// three 4-byte code stores and two scale bytes out; r comes from a per-CTA
+// table over the 128 scale codes.  The FP3 rounding is three comparisons: with s1 = [|v| > 0.5],
 // s2 = [|v| >= 1.5], s3 = [|v| > 3] the magnitude's index is s1 + s2 + s3 and
 // its value s1 + s2 + 2 s3.  As in IF4, rint adds and subtracts 1.5 * 2^23;
 // the low bits of that sum (and of the index plus 1.5 * 2^23) are packed by
@@ -80,8 +81,83 @@ __device__ __forceinline__ void load16(const T *p, float (&v)[16]) {
   }
 }
 
+// Both candidates of blocks A and B (lanes .x / .y): the packed codes of each
+// (two 24-bit groups) and whether INT3 wins.  Each lane sums its own block's
+// errors in element order.  No packed add or subtract consumes a product
+// (ptxas may contract a mul.f32x2 -> add.f32x2 pair even with .rn); the
+// additions that follow a product are scalar __fadd_rn / __fsub_rn.
+template <bool CLAMP>
+__device__ __forceinline__ void if3_pair(const float (&va)[16], const float (&vb)[16], float2 rf,
+                                         uint32_t (&ga)[2], uint32_t (&gb)[2], bool &int_a,
+                                         bool &int_b) {
+  float2 e_fp = make_float2(0.0f, 0.0f), e_int = make_float2(0.0f, 0.0f);
+  uint32_t fa[2] = {0u, 0u}, fb[2] = {0u, 0u}, ia[2] = {0u, 0u}, ib[2] = {0u, 0u};
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {                       // element order, as the errors sum
+    const int h = k >> 3;
+    const uint32_t w8 = 1u << (3 * (k & 7));           // code k's weight in its group
+    const float2 vv = mul2(make_float2(va[k], vb[k]), rf);
+    const float ax = fabsf(vv.x), ay = fabsf(vv.y);
+    const float2 s1 = make_float2(set_gt(ax, 0.5f), set_gt(ay, 0.5f));
+    const float2 s2 = make_float2(set_ge(ax, 1.5f), set_ge(ay, 1.5f));
+    const float2 s3 = make_float2(set_gt(ax, 3.0f), set_gt(ay, 3.0f));
+    const float2 s12 = add2(s1, s2);
+    const float2 g = fma2(s3, make_float2(2.0f, 2.0f), s12);   // 0, 1, 2 or 4 (exact)
+    const float2 dfp = make_float2(__fsub_rn(ax, g.x), __fsub_rn(ay, g.y));
+    e_fp = fma2(dfp, dfp, e_fp);
+    const float2 idx = add2(add2(s12, make_float2(kMagic, kMagic)), s3);
+    const uint32_t bx = __float_as_uint(vv.x), by = __float_as_uint(vv.y);
+    fa[h] += (__float_as_uint(idx.x) + ((bx >> 31) << 2)) * w8;
+    fb[h] += (__float_as_uint(idx.y) + ((by >> 31) << 2)) * w8;
+    float2 t = mul2(vv, make_float2(0.75f, 0.75f));
+    if (CLAMP) {
+      t.x = fminf(fmaxf(t.x, -3.25f), 3.25f);
+      t.y = fminf(fmaxf(t.y, -3.25f), 3.25f);
+    }
+    const float2 tm = make_float2(__fadd_rn(t.x, kMagic), __fadd_rn(t.y, kMagic));
+    const float2 kf = sub2(tm, make_float2(kMagic, kMagic));   // rint(t), exact
+    const float2 hv = mul2(kf, make_float2(kDown, kDown));
+    const float2 dint = make_float2(__fsub_rn(vv.x, hv.x), __fsub_rn(vv.y, hv.y));
+    e_int = fma2(dint, dint, e_int);
+    ia[h] += __float_as_uint(tm.x) * w8;
+    ib[h] += __float_as_uint(tm.y) * w8;
+  }
+  int_a = e_int.x < e_fp.x;
+  int_b = e_int.y < e_fp.y;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    ga[h] = int_a ? (ia[h] - kBiasInt) ^ kSignBits : fa[h] - kBiasFp;
+    gb[h] = int_b ? (ib[h] - kBiasInt) ^ kSignBits : fb[h] - kBiasFp;
+  }
+}
+
+// Scale code, factor and clamp flag of one block.
+struct BlockScale3 {
+  uint32_t code;
+  float rf;
+  bool clamp;
+};
+
+__device__ __forceinline__ BlockScale3 block_scale3(const float (&v)[16], float s_enc,
+                                                    const float *tab) {
+  float m = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) m = fmaxf(m, fabsf(v[k]));
+  BlockScale3 b;
+  b.code = scale_code_q<4>(m, s_enc);
+  b.rf = tab[b.code];
+  // |t| <= RN(RN(m * r) * 0.75) by monotonicity; only a block reaching 3.25
+  // needs the clamp (which then makes rint land on +-3, as clamping rint(t)
+  // to +-3 does).  A block whose scale is an E4M3 subnormal can get there.
+  b.clamp = __fmul_rn(__fmul_rn(m, b.rf), 0.75f) > 3.25f;
+  return b;
+}
+
+// One thread per pair of consecutive blocks (2p, 2p + 1) in row-major block
+// order; the pair's 12 code bytes are contiguous.  With an odd block count
+// the last thread's second block is a copy of its first and is not stored.
 template <typename T, typename I>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, sizeof(I) == 4 ? 4 : 2)   // 64 registers with 32-bit indices
 if3_kernel(const T *__restrict__ x, I rows, I cols, I ld, const float *__restrict__ amax,
            float *__restrict__ s_dec_out, uint8_t *__restrict__ q, uint8_t *__restrict__ sf,
            int scale_layout) {
@@ -90,59 +166,41 @@ if3_kernel(const T *__restrict__ x, I rows, I cols, I ld, const float *__restric
   if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out) *s_dec_out = ts.dec;
   fill_factor_table(tab, ts.enc);
   __syncthreads();
-  const I bpr = cols / 16, nblk = rows * bpr;
+  const I bpr = cols / 16, nblk = rows * bpr, npairs = (nblk + 1) / 2;
   const I stride = static_cast<I>(gridDim.x) * kThreads;
-  for (I b = static_cast<I>(blockIdx.x) * kThreads + threadIdx.x; b < nblk; b += stride) {
-    const I r = b / bpr, cb = b - r * bpr;
-    float v[16];
-    load16<T>(x + r * ld + cb * 16, v);
-    float m = 0.0f;
+  for (I p = static_cast<I>(blockIdx.x) * kThreads + threadIdx.x; p < npairs; p += stride) {
+    const I b0 = 2 * p;
+    const bool has_b = b0 + 1 < nblk;
+    const I r0 = b0 / bpr, c0 = b0 - r0 * bpr;
+    const I r1 = (c0 + 1 == bpr) ? r0 + 1 : r0, c1 = (c0 + 1 == bpr) ? 0 : c0 + 1;
+    float va[16], vb[16];
+    load16<T>(x + r0 * ld + c0 * 16, va);
+    if (has_b) {
+      load16<T>(x + r1 * ld + c1 * 16, vb);
+    } else {
 #pragma unroll
-    for (int k = 0; k < 16; ++k) m = fmaxf(m, fabsf(v[k]));
-    const uint32_t code = scale_code_q<4>(m, ts.enc);
-    const float rf = tab[code];
-    // |t| <= RN(RN(m * r) * 0.75) by monotonicity; only a block reaching 3.25
-    // needs the clamp (which then makes rint land on +-3, as clamping rint(t)
-    // to +-3 does).  A block whose scale is an E4M3 subnormal can get there.
-    const bool clamp = __fmul_rn(__fmul_rn(m, rf), 0.75f) > 3.25f;
-    float e_fp = 0.0f, e_int = 0.0f;
-    uint32_t acc_fp[2] = {0u, 0u}, acc_sign[2] = {0u, 0u}, acc_int[2] = {0u, 0u};
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {                     // element order, as the errors sum
-      const int h = k >> 3;
-      const uint32_t w8 = 1u << (3 * (k & 7));         // code k's weight in its group
-      const float vv = __fmul_rn(v[k], rf);
-      const float a = fabsf(vv);
-      const float s1 = set_gt(a, 0.5f), s2 = set_ge(a, 1.5f), s3 = set_gt(a, 3.0f);
-      const float s12 = __fadd_rn(s1, s2);
-      const float g = __fmaf_rn(s3, 2.0f, s12);        // 0, 1, 2 or 4 (exact)
-      const float dfp = __fsub_rn(a, g);               // |v - sign(v) g|: the same square
-      e_fp = __fmaf_rn(dfp, dfp, e_fp);
-      const float idx = __fadd_rn(__fadd_rn(s12, kMagic), s3);   // magnitude index, low bits
-      acc_fp[h] += __float_as_uint(idx) * w8;
-      acc_sign[h] += (__float_as_uint(vv) >> 31) * w8;
-      float t = __fmul_rn(vv, 0.75f);
-      if (clamp) t = fminf(fmaxf(t, -3.25f), 3.25f);
-      const float tm = __fadd_rn(t, kMagic);           // rint(t) in the low bits
-      const float kf = __fsub_rn(tm, kMagic);          // exact
-      const float dint = __fsub_rn(vv, __fmul_rn(kf, kDown));
-      e_int = __fmaf_rn(dint, dint, e_int);
-      acc_int[h] += __float_as_uint(tm) * w8;
+      for (int k = 0; k < 16; ++k) vb[k] = va[k];
     }
-    uint32_t fp_group[2], int_group[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      fp_group[h] = (acc_fp[h] - kBiasFp) | (acc_sign[h] << 2);
-      int_group[h] = (acc_int[h] - kBiasInt) ^ kSignBits;
+    const BlockScale3 sa = block_scale3(va, ts.enc, tab), sb = block_scale3(vb, ts.enc, tab);
+    uint32_t ga[2], gb[2];
+    bool int_a, int_b;
+    if (sa.clamp || sb.clamp)
+      if3_pair<true>(va, vb, make_float2(sa.rf, sb.rf), ga, gb, int_a, int_b);
+    else
+      if3_pair<false>(va, vb, make_float2(sa.rf, sb.rf), ga, gb, int_a, int_b);
+    sf[scale_offset(r0, c0, bpr, scale_layout)] = static_cast<uint8_t>(sa.code | (int_a ? 0x80u : 0u));
+    if (has_b) {
+      uint32_t *dst = reinterpret_cast<uint32_t *>(q + b0 * 6);   // 12 B, 4-byte aligned
+      dst[0] = ga[0] | ga[1] << 24;
+      dst[1] = ga[1] >> 8 | gb[0] << 16;
+      dst[2] = gb[0] >> 16 | gb[1] << 8;
+      sf[scale_offset(r1, c1, bpr, scale_layout)] = static_cast<uint8_t>(sb.code | (int_b ? 0x80u : 0u));
+    } else {
+      uint16_t *dst = reinterpret_cast<uint16_t *>(q + b0 * 6);
+      dst[0] = static_cast<uint16_t>(ga[0]);
+      dst[1] = static_cast<uint16_t>((ga[0] >> 16) | (ga[1] << 8));
+      dst[2] = static_cast<uint16_t>(ga[1] >> 8);
     }
-    const bool use_int = e_int < e_fp;
-    const uint32_t g0 = use_int ? int_group[0] : fp_group[0];
-    const uint32_t g1 = use_int ? int_group[1] : fp_group[1];
-    uint16_t *dst = reinterpret_cast<uint16_t *>(q + b * 6);   // codes are dense, 6 B per block
-    dst[0] = static_cast<uint16_t>(g0);
-    dst[1] = static_cast<uint16_t>((g0 >> 16) | (g1 << 8));
-    dst[2] = static_cast<uint16_t>(g1 >> 8);
-    sf[scale_offset(r, cb, bpr, scale_layout)] = static_cast<uint8_t>(code | (use_int ? 0x80u : 0u));
   }
 }
 
@@ -218,9 +276,9 @@ template <typename T>
 cudaError_t launch_q(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *amax,
                      float *s_dec_out, uint8_t *q, uint8_t *sf, int scale_layout,
                      const Launch &L) {
-  const int grid = grid_for(rows * (cols / 16), L);
+  const int grid = grid_for((rows * (cols / 16) + 1) / 2, L);      // one thread per block pair
   const T *p = static_cast<const T *>(x);
-  if (narrow(rows, cols, ld, grid))
+  if (narrow(rows, cols, ld, 2 * grid))           // a pair step spans two blocks
     if3_kernel<T, uint32_t><<<grid, kThreads, 0, L.stream>>>(
         p, static_cast<uint32_t>(rows), static_cast<uint32_t>(cols), static_cast<uint32_t>(ld),
         amax, s_dec_out, q, sf, scale_layout);
