@@ -879,6 +879,7 @@ uint8_t orc_fp3_rne(float v) {
     double d = fabs(a - (double)orc_fp3_value((uint8_t)c));
     if (d < best_d || (d == best_d && (c % 2) == 0)) { best = c; best_d = d; }
   }
+  if (a >= 4.0) best = 3;                  /* saturate: huge a ties every distance */
   return (uint8_t)(best | sign);
 }
 

@@ -83,6 +83,64 @@ def test_magic_number_rint_and_int6_group_packing():
     assert np.array_equal(got, want)
 
 
+def test_if3_fp3_by_three_comparisons():
+    """IF3's FP3 step: with s1 = [a > 0.5], s2 = [a >= 1.5], s3 = [a > 3] the
+    index s1 + s2 + s3 and value s1 + s2 + 2 s3 are the nearest E2M0 magnitude
+    (0, 1, 2, 4; ties to the even index; saturating) by exhaustive search."""
+    grid = np.array([0.0, 1.0, 2.0, 4.0])
+    a = np.concatenate([np.linspace(0, 8, 400_001, dtype=np.float32),
+                        np.float32([0.5, 1.5, 3.0, np.nextafter(np.float32(0.5), 1),
+                                    np.nextafter(np.float32(1.5), 0),
+                                    np.nextafter(np.float32(3.0), 4), 1e30])])
+    d = np.abs(a.astype(np.float64)[:, None] - grid[None, :])
+    # among the nearest magnitudes (two only at a tie) take the even index
+    best = np.argmin(np.where(d == d.min(1, keepdims=True), np.arange(4) % 2, 9), axis=1)
+    best[a >= 4] = 3                                # saturation (float64 distances tie at 1e30)
+    s1, s2, s3 = (a > 0.5), (a >= 1.5), (a > 3.0)
+    idx = s1.astype(int) + s2 + s3
+    assert np.array_equal(idx, best)
+    assert np.array_equal(s1 + s2.astype(float) + 2 * s3, grid[best])
+
+
+def test_if3_group_packing_and_pair_store():
+    """IF3's packing: eight words RN(n + 1.5*2^23) (n the FP3 index, or k in
+    -3..3) summed with weights 8^j, minus 0x4B400000 (or 0x4B400000 - 4) times
+    0x249249, give the 24-bit group (FP3: plus the sign bits shifted into bit
+    2; INT3: XOR 0x924924 for two's complement); a pair of blocks' groups go
+    out as three little-endian words holding 12 consecutive code bytes, and
+    three 16-bit loads give a block's two groups back."""
+    magic = np.float32(12582912.0)
+    w = np.array([8 ** j for j in range(8)], dtype=np.uint64)
+    kocts = 0x249249
+    rng = np.random.default_rng(1)
+    n = rng.integers(0, 4, (5000, 8))
+    sg = rng.integers(0, 2, (5000, 8))
+    bits = (n.astype(np.float32) + magic).astype(np.float32).view(np.uint32).astype(np.uint64)
+    acc = ((bits + 4 * sg.astype(np.uint64)) * w).sum(axis=1) % 2**32
+    got_fp = (acc - (0x4B400000 * kocts) % 2**32) % 2**32
+    assert np.array_equal(got_fp, ((n + 4 * sg).astype(np.uint64) * w).sum(axis=1))
+    t = np.concatenate([np.linspace(-3.25, 3.25, 100_001, dtype=np.float32),
+                        np.float32([-2.5, -1.5, -0.5, 0.5, 1.5, 2.5])])
+    assert np.array_equal(((t + magic).astype(np.float32) - magic).astype(np.float32), np.rint(t))
+    k = np.concatenate([rng.integers(-3, 4, (5000, 8)), np.full((1, 8), -3), np.full((1, 8), 3)])
+    bits = (k.astype(np.float32) + magic).astype(np.float32).view(np.uint32).astype(np.uint64)
+    acc = (bits * w).sum(axis=1) % 2**32
+    got_int = ((acc - ((0x4B400000 - 4) * kocts) % 2**32) % 2**32) ^ 0x924924
+    assert np.array_equal(got_int, ((k & 7).astype(np.uint64) * w).sum(axis=1))
+    # the pair store and the dequantizer's reassembly
+    for ga0, ga1, gb0, gb1 in rng.integers(0, 1 << 24, (200, 4)).tolist():
+        w0 = (ga0 | ga1 << 24) & 0xFFFFFFFF
+        w1 = (ga1 >> 8 | gb0 << 16) & 0xFFFFFFFF
+        w2 = (gb0 >> 16 | gb1 << 8) & 0xFFFFFFFF
+        out = b"".join(v.to_bytes(4, "little") for v in (w0, w1, w2))
+        want = b"".join(g.to_bytes(3, "little") for g in (ga0, ga1, gb0, gb1))
+        assert out == want
+        for blk in (out[:6], out[6:]):
+            h0, h1, h2 = (int.from_bytes(blk[2 * i:2 * i + 2], "little") for i in range(3))
+            g0, g1 = (h0 | h1 << 16) & 0xFFFFFF, (h1 >> 8) | (h2 << 8)
+            assert blk == g0.to_bytes(3, "little") + g1.to_bytes(3, "little")
+
+
 def test_if4_split_tables_sum_to_k():
     """The IF4 GEMM's split: for every INT4 nibble n (k in two's complement)
     the two E2M1 codes of the tables the split kernel uses add up to k."""

@@ -60,6 +60,8 @@ def test_fp3_rounding_against_brute_force(orc):
         assert orc.fp3_rne(v) == brute_fp3(v), v
     # the ties: 0.5 -> 0, 1.5 -> 2, 3 -> 2 (even codes 0 and 2)
     assert [orc.fp3_rne(v) for v in (0.5, 1.5, 3.0)] == [0, 2, 2]
+    # saturation holds for every magnitude, also where float64 distances tie
+    assert [orc.fp3_rne(v) for v in (1e30, -3e38, 4.0)] == [3, 7, 3]
 
 
 def test_block_on_the_fp3_grid_keeps_fp3(orc):
