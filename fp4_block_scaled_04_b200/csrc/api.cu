@@ -624,8 +624,7 @@ fp4q_status fp4q_gemm_if4_nvfp4(const uint8_t *qa, const uint8_t *sfa, const flo
   FP4Q_TRY(cuda_status(launch_if4_split(qa, sfa, M, K, FP4Q_SCALE_SWIZZLED_128x4, q_fp, q_k1,
                                         q_k2, sf_plain, L)));
   return cuda_status(launch_gemm_if4_split(q_fp, q_k1, q_k2, sf_plain, tensor_scale_a, qb, sfb,
-                                           tensor_scale_b, M, N, K, c, FP4Q_FP32, ldc, status,
-                                           L));
+                                           tensor_scale_b, M, N, K, c, ldc, status, L));
 }
 
 fp4q_status fp4q_gemm_nvfp4_withhold_loads(const uint8_t *qa, const uint8_t *sfa,

@@ -501,14 +501,11 @@ cudaError_t launch_o(const uint8_t *qa, const uint8_t *sfa, const float *s_a, co
 cudaError_t launch_gemm_if4_split(const uint8_t *q_fp, const uint8_t *q_k1, const uint8_t *q_k2,
                                   const uint8_t *sfa, const float *s_a, const uint8_t *qb,
                                   const uint8_t *sfb, const float *s_b, int64_t M, int64_t N,
-                                  int64_t K, void *c, int c_dtype, int64_t ldc, int *status,
+                                  int64_t K, float *c, int64_t ldc, int *status,
                                   const Launch &L) {
   const uint8_t *const a[3] = {q_fp, q_k1, q_k2};
   GemmOptions opt;
   opt.alpha_int = 6.0f / 7.0f;                         // RN(6/7)
-  if (c_dtype == FP4Q_BF16)
-    return launch_t<__nv_bfloat16, 128, 3>(a, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status,
-                                           opt, L);
   return launch_t<float, 128, 3>(a, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
 }
 

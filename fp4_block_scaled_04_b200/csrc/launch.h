@@ -83,11 +83,11 @@ cudaError_t launch_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float
 
 // IF4 x NVFP4 in one pass over the split operands: C = RN(RN(acc_fp * a) +
 // RN(acc_int * RN(a * RN(6/7)))), acc_int accumulating both INT4 parts; FP32
-// or BF16 output, N % 128 == 0
+// output, N % 128 == 0
 cudaError_t launch_gemm_if4_split(const uint8_t *q_fp, const uint8_t *q_k1, const uint8_t *q_k2,
                                   const uint8_t *sfa, const float *s_a, const uint8_t *qb,
                                   const uint8_t *sfb, const float *s_b, int64_t M, int64_t N,
-                                  int64_t K, void *c, int c_dtype, int64_t ldc, int *status,
+                                  int64_t K, float *c, int64_t ldc, int *status,
                                   const Launch &L);
 
 // Split IF4 codes [rows, K/2] with flagged scales into three NVFP4 code
