@@ -95,3 +95,57 @@ def test_layouts_agree_and_alpha_scales(orc):
     c_q = orc.gemm_block_scaled(qa, la.ravel(), qb, lb.ravel(), M, N, K, alpha=0.25,
                                 scale_layout=orc.SCALE_LINEAR)
     np.testing.assert_array_equal(c_q, c_lin * 0.25)
+
+
+def test_mxfp4_operands_by_brute_force(orc):
+    """MXFP4 operands: 32-value blocks with E8M0 scales 2^(s - 127); the exact
+    product from the E2M1 table and powers of two."""
+    M, N, K = 2, 3, 64
+    rng = np.random.default_rng(4)
+    ca = rng.integers(0, 16, (M, K), dtype=np.uint8)
+    cb = rng.integers(0, 16, (N, K), dtype=np.uint8)
+    sa = rng.integers(120, 134, (M, K // 32), dtype=np.uint8)
+    sb = rng.integers(120, 134, (N, K // 32), dtype=np.uint8)
+    got = orc.gemm_block_scaled(pack(ca), sa.ravel(), pack(cb), sb.ravel(), M, N, K,
+                                fmt=orc.FMT_MXFP4, scale_layout=orc.SCALE_LINEAR)
+    for m in range(M):
+        for n in range(N):
+            want = sum(e2m1(int(ca[m, k])) * Fraction(2) ** (int(sa[m, k // 32]) - 127) *
+                       e2m1(int(cb[n, k])) * Fraction(2) ** (int(sb[n, k // 32]) - 127)
+                       for k in range(K))
+            assert Fraction(got[m, n]) == want, (m, n)
+
+
+def test_if4_operand_by_brute_force(orc):
+    """An IF4 A operand (scale bit 7 set: INT4 block, k in two's complement,
+    value RN(RN(k * RN(6/7)) * S)) against an NVFP4 B operand, 16-value
+    blocks: the exact sum of the products of those binary32 values."""
+    M, N, K = 2, 3, 64
+    rng = np.random.default_rng(5)
+    ca = rng.integers(0, 16, (M, K), dtype=np.uint8)
+    ca[ca == 8] = 9                                   # -8 is not an INT4 code
+    cb = rng.integers(0, 16, (N, K), dtype=np.uint8)
+    keys = np.array(list(E4M3))
+    sa = rng.choice(keys, (M, K // 16)).astype(np.uint8)
+    sa[:, ::2] |= 0x80                                # every other A block is INT4
+    sb = rng.choice(keys, (N, K // 16)).astype(np.uint8)
+    got = orc.gemm_block_scaled(pack(ca), sa.ravel(), pack(cb), sb.ravel(), M, N, K,
+                                fmt=orc.FMT_IF4, scale_layout=orc.SCALE_LINEAR)
+    c67 = np.float32(6.0) / np.float32(7.0)
+
+    def a_value(m, k):
+        s = int(sa[m, k // 16])
+        S = np.float32(E4M3[s & 0x7F])
+        c = int(ca[m, k])
+        if s & 0x80:
+            kk = c - 16 if c & 8 else c
+            return Fraction(float(np.float32(np.float32(kk) * c67) * S))
+        return e2m1(c) * Fraction(float(S))
+
+    for m in range(M):
+        for n in range(N):
+            terms = [a_value(m, k) * e2m1(int(cb[n, k])) * Fraction(E4M3[int(sb[n, k // 16])])
+                     for k in range(K)]
+            # each product is exact in float64; only the K - 1 additions round
+            bound = sum(abs(t) for t in terms) * K * Fraction(1, 2 ** 53)
+            assert abs(Fraction(got[m, n]) - sum(terms)) <= bound, (m, n)
