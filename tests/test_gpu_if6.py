@@ -4,7 +4,6 @@
 to 6 bits).  Codes, flagged scale bytes, the tensor scale and the dequantized
 values must match the oracle bit for bit.
 """
-import numpy as np
 import pytest
 import torch
 

@@ -9,7 +9,6 @@ row-independent once the tensor amax is given, so that comparison is exact.
 Round to nearest throughout (the stochastic-rounding bits depend on the
 global element index).
 """
-import numpy as np
 import pytest
 import torch
 

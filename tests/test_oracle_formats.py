@@ -5,13 +5,11 @@ pages print, an independent library (ml_dtypes, torch's float8 cast, scipy),
 published test vectors, or exact rational arithmetic.
 """
 import decimal
-import json
 import os
 from fractions import Fraction
 
 import ml_dtypes
 import numpy as np
-import pytest
 import torch
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")

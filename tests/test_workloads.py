@@ -1,6 +1,5 @@
 """The seeded generators: shapes, dtypes, determinism, finiteness and the
 value structure each workload is specified with."""
-import numpy as np
 import torch
 
 from fp4_block_scaled_04_b200 import workloads as w
