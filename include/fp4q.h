@@ -225,7 +225,7 @@ fp4q_status fp4q_quantize_backward(const void *dy, int dtype, int64_t tokens, in
                                    uint8_t *q_t, uint8_t *sf_t, int scale_layout, void *workspace,
                                    size_t ws_bytes, void *stream);
 
-/* IF4 adaptive quantization, row-wise 1x16/* IF4 adaptive quantization, row-wise 1x16 ("Adaptive Block-Scaled Data
+/* IF4 adaptive quantization, row-wise 1x16 ("Adaptive Block-Scaled Data
  * Types" explainer, section 2): per block the NVFP4 scale S and factor r,
  * v = RN(x*r); FP4 candidate E2M1_rne(v); INT4 candidate
  * k = clamp(rint(RN(v * RN(7/6))), -7, 7) decoded as RN(k * RN(6/7)) (the 6/7

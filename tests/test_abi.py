@@ -208,3 +208,37 @@ def test_python_binding_refuses_cpu_tensors(L):
     import torch
     with pytest.raises(ValueError):
         fq.fp4q_quantize_nvfp4(torch.zeros(16, 16, dtype=torch.bfloat16))
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "fp4q.h"
+int main(void) {
+  if (strstr(fp4q_version(), "sm_100a") == NULL) return 2;
+  if (fp4q_scale_bytes(130, 80, 16, FP4Q_SCALE_SWIZZLED_128x4) != 256 * 8) return 3;
+  if (strcmp(fp4q_status_string(FP4Q_ERR_MISALIGNED), "FP4Q_ERR_MISALIGNED") != 0) return 4;
+  /* an argument error is returned before anything touches a device */
+  if (fp4q_quantize_if3(NULL, FP4Q_BF16, 16, 48, 48, NULL, NULL, NULL, NULL,
+                        FP4Q_SCALE_LINEAR, NULL, 0, NULL) != FP4Q_ERR_INVALID_ARG) return 5;
+  puts("ok");
+  return 0;
+}
+"""
+
+
+@pytest.mark.parametrize("compiler", [["gcc", "-std=c99", "-x", "c"],
+                                      ["g++", "-std=c++17", "-x", "c++"]])
+def test_header_is_plain_c_and_links(L, tmp_path, compiler):
+    """The public header compiles as strict C99 and as C++ (extern "C"), and a
+    program linked against the library runs its host-side calls."""
+    import subprocess
+    src = tmp_path / "use_fp4q.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "use_fp4q"
+    libdir = os.path.dirname(fq.library_path)
+    subprocess.check_call([*compiler, "-Wall", "-Wextra", "-pedantic", "-Werror",
+                           "-I", os.path.join(ROOT, "include"), str(src), "-x", "none",
+                           "-L", libdir, "-lfp4q", f"-Wl,-rpath,{libdir}", "-o", str(exe)])
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stderr)
