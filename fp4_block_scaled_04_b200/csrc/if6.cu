@@ -36,12 +36,6 @@ constexpr float kTop = 7.5f * 448.0f;             // 3360
 constexpr float kUp = 31.0f / 7.5f;               // RN(31/7.5)
 constexpr float kDown = 7.5f / 31.0f;             // RN(7.5/31)
 
-__device__ __forceinline__ uint32_t e2m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
 __device__ __forceinline__ float2 e2m3x2_value(uint32_t two_codes) {
   uint32_t h;
   const uint16_t w = static_cast<uint16_t>(two_codes);
