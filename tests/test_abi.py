@@ -242,3 +242,11 @@ def test_header_is_plain_c_and_links(L, tmp_path, compiler):
                            "-L", libdir, "-lfp4q", f"-Wl,-rpath,{libdir}", "-o", str(exe)])
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stderr)
+
+
+def test_binding_declares_every_header_function():
+    """The Python binding gives every entry point of the header a ctypes
+    signature, and none that the header lacks."""
+    src = open(os.path.join(ROOT, "fp4_block_scaled_04_b200", "__init__.py")).read()
+    bound = set(re.findall(r'"(fp4q_\w+)":\s*\(', src))
+    assert bound == set(declared_functions())
