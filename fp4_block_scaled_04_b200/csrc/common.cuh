@@ -309,6 +309,32 @@ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t c, int64_t co
 // ---------------------------------------------------------------------------
 
 // ---------------------------------------------------------------------------
+// one block of N contiguous BF16 or FP32 values (16-byte aligned) to FP32
+// ---------------------------------------------------------------------------
+
+template <int N, typename T>
+__device__ __forceinline__ void load_values(const T *p, float (&v)[N]) {
+  const uint4 *q = reinterpret_cast<const uint4 *>(p);
+  if (sizeof(T) == 2) {
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i) {
+      const uint4 u = __ldg(q + i);
+      v[8 * i + 0] = bf16_lo(u.x); v[8 * i + 1] = bf16_hi(u.x);
+      v[8 * i + 2] = bf16_lo(u.y); v[8 * i + 3] = bf16_hi(u.y);
+      v[8 * i + 4] = bf16_lo(u.z); v[8 * i + 5] = bf16_hi(u.z);
+      v[8 * i + 6] = bf16_lo(u.w); v[8 * i + 7] = bf16_hi(u.w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const uint4 u = __ldg(q + i);
+      v[4 * i + 0] = __uint_as_float(u.x); v[4 * i + 1] = __uint_as_float(u.y);
+      v[4 * i + 2] = __uint_as_float(u.z); v[4 * i + 3] = __uint_as_float(u.w);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // packed arithmetic (sm_100a f32x2 and bf16x2)
 // ---------------------------------------------------------------------------
 

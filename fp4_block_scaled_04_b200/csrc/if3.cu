@@ -59,28 +59,6 @@ __device__ __forceinline__ float set_ge(float a, float b) {
   return r;
 }
 
-template <typename T>
-__device__ __forceinline__ void load16(const T *p, float (&v)[16]) {
-  const uint4 *q = reinterpret_cast<const uint4 *>(p);
-  if (sizeof(T) == 2) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const uint4 u = __ldg(q + i);
-      v[8 * i + 0] = bf16_lo(u.x); v[8 * i + 1] = bf16_hi(u.x);
-      v[8 * i + 2] = bf16_lo(u.y); v[8 * i + 3] = bf16_hi(u.y);
-      v[8 * i + 4] = bf16_lo(u.z); v[8 * i + 5] = bf16_hi(u.z);
-      v[8 * i + 6] = bf16_lo(u.w); v[8 * i + 7] = bf16_hi(u.w);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 u = __ldg(q + i);
-      v[4 * i + 0] = __uint_as_float(u.x); v[4 * i + 1] = __uint_as_float(u.y);
-      v[4 * i + 2] = __uint_as_float(u.z); v[4 * i + 3] = __uint_as_float(u.w);
-    }
-  }
-}
-
 // Both candidates of blocks A and B (lanes .x / .y): the packed codes of each
 // (two 24-bit groups) and whether INT3 wins.  Each lane sums its own block's
 // errors in element order.  No packed add or subtract consumes a product
@@ -174,9 +152,9 @@ if3_kernel(const T *__restrict__ x, I rows, I cols, I ld, const float *__restric
     const I r0 = b0 / bpr, c0 = b0 - r0 * bpr;
     const I r1 = (c0 + 1 == bpr) ? r0 + 1 : r0, c1 = (c0 + 1 == bpr) ? 0 : c0 + 1;
     float va[16], vb[16];
-    load16<T>(x + r0 * ld + c0 * 16, va);
+    load_values<16, T>(x + r0 * ld + c0 * 16, va);
     if (has_b) {
-      load16<T>(x + r1 * ld + c1 * 16, vb);
+      load_values<16, T>(x + r1 * ld + c1 * 16, vb);
     } else {
 #pragma unroll
       for (int k = 0; k < 16; ++k) vb[k] = va[k];

@@ -74,28 +74,6 @@ __device__ __forceinline__ uint32_t e2m3x4_codes_diffs(const float (&v)[4], floa
   return w;
 }
 
-template <typename T>
-__device__ __forceinline__ void load16(const T *p, float (&v)[16]) {
-  const uint4 *q = reinterpret_cast<const uint4 *>(p);
-  if (sizeof(T) == 2) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const uint4 u = __ldg(q + i);
-      v[8 * i + 0] = bf16_lo(u.x); v[8 * i + 1] = bf16_hi(u.x);
-      v[8 * i + 2] = bf16_lo(u.y); v[8 * i + 3] = bf16_hi(u.y);
-      v[8 * i + 4] = bf16_lo(u.z); v[8 * i + 5] = bf16_hi(u.z);
-      v[8 * i + 6] = bf16_lo(u.w); v[8 * i + 7] = bf16_hi(u.w);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 u = __ldg(q + i);
-      v[4 * i + 0] = __uint_as_float(u.x); v[4 * i + 1] = __uint_as_float(u.y);
-      v[4 * i + 2] = __uint_as_float(u.z); v[4 * i + 3] = __uint_as_float(u.w);
-    }
-  }
-}
-
 template <typename T, typename I>
 __global__ void __launch_bounds__(kThreads)
 if6_kernel(const T *__restrict__ x, I rows, I cols, I ld, const float *__restrict__ amax,
@@ -113,7 +91,7 @@ if6_kernel(const T *__restrict__ x, I rows, I cols, I ld, const float *__restric
   for (I b = static_cast<I>(blockIdx.x) * kThreads + threadIdx.x; b < nblk; b += stride) {
     const I r = b / bpr, cb = b - r * bpr;
     float v[16];
-    load16<T>(x + r * ld + cb * 16, v);
+    load_values<16, T>(x + r * ld + cb * 16, v);
     float m = 0.0f;
 #pragma unroll
     for (int k = 0; k < 16; ++k) m = fmaxf(m, fabsf(v[k]));

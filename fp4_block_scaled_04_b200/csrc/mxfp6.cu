@@ -52,28 +52,6 @@ __device__ __forceinline__ float2 half2_bits_to_f32x2(uint32_t h) {
   return __half22float2(v);
 }
 
-template <typename T>
-__device__ __forceinline__ void load32(const T *p, float (&v)[32]) {
-  const uint4 *q = reinterpret_cast<const uint4 *>(p);
-  if (sizeof(T) == 2) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 u = __ldg(q + i);
-      v[8 * i + 0] = bf16_lo(u.x); v[8 * i + 1] = bf16_hi(u.x);
-      v[8 * i + 2] = bf16_lo(u.y); v[8 * i + 3] = bf16_hi(u.y);
-      v[8 * i + 4] = bf16_lo(u.z); v[8 * i + 5] = bf16_hi(u.z);
-      v[8 * i + 6] = bf16_lo(u.w); v[8 * i + 7] = bf16_hi(u.w);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint4 u = __ldg(q + i);
-      v[4 * i + 0] = __uint_as_float(u.x); v[4 * i + 1] = __uint_as_float(u.y);
-      v[4 * i + 2] = __uint_as_float(u.z); v[4 * i + 3] = __uint_as_float(u.w);
-    }
-  }
-}
-
 // Quantize: one thread per 32-value block (64 or 128 bytes in, 24 code
 // bytes and a scale byte out).  Four lanes per block with a shuffled block
 // maximum moved the same bytes more slowly on B200: the shuffles and the
@@ -91,7 +69,7 @@ mxfp6_kernel(const T *__restrict__ x, I rows, I cols, I ld, int mode, uint8_t *_
   for (I b = static_cast<I>(blockIdx.x) * kThreads + threadIdx.x; b < nblk; b += stride) {
     const I r = b / bpr, cb = b - r * bpr;
     float v[32];
-    load32<T>(x + r * ld + cb * 32, v);
+    load_values<32, T>(x + r * ld + cb * 32, v);
     float m = 0.0f;
 #pragma unroll
     for (int k = 0; k < 32; ++k) m = fmaxf(m, fabsf(v[k]));
