@@ -76,7 +76,7 @@ _SZ = ctypes.c_size_t
 _SIGNATURES = {
     "fp4q_status_string": (ctypes.c_char_p, [_I]),
     "fp4q_version": (ctypes.c_char_p, []),
-    "fp4q_workspace_bytes": (_SZ, []),
+    "fp4q_workspace_bytes": (_SZ, [_I64, _I64]),
     "fp4q_scale_bytes": (_SZ, [_I64, _I64, _I, _I]),
     "fp4q_amax": (_I, [_P, _I, _I64, _I64, _I64, _P, _P]),
     "fp4q_quantize_nvfp4": (_I, [_P, _I, _I64, _I64, _I64, _U, _I, _U64, _P, _P, _P, _P, _P,
@@ -193,8 +193,8 @@ def fp4q_version() -> str:
     return lib().fp4q_version().decode()
 
 
-def fp4q_workspace_bytes() -> int:
-    return int(lib().fp4q_workspace_bytes())
+def fp4q_workspace_bytes(rows: int = 0, cols: int = 0) -> int:
+    return int(lib().fp4q_workspace_bytes(int(rows), int(cols)))
 
 
 def fp4q_scale_bytes(rows: int, cols: int, block: int, scale_layout: int = SCALE_LINEAR) -> int:

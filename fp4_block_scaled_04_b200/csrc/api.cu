@@ -164,6 +164,30 @@ fp4q_status quantize_if4_mode(const void *x, int dtype, int64_t rows, int64_t co
 }
 
 }  // namespace
+
+int check_nvfp4_args(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                     unsigned layouts, int round, const uint8_t *q_row, const uint8_t *sf_row,
+                     const uint8_t *q_col, const uint8_t *sf_col, int scale_layout) {
+  FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
+  if (layouts == 0 || (layouts & ~(FP4Q_ROWWISE | FP4Q_COLWISE)) != 0) return FP4Q_ERR_INVALID_ARG;
+  if (round != FP4Q_RNE && round != FP4Q_SR) return FP4Q_ERR_INVALID_ARG;
+  if (!valid_layout(scale_layout)) return FP4Q_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
+  if ((layouts & FP4Q_COLWISE) && rows % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
+  const bool nonempty = rows > 0 && cols > 0;
+  if (layouts & FP4Q_ROWWISE) {
+    if ((!q_row || !sf_row) && nonempty) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned16(q_row)) return FP4Q_ERR_MISALIGNED;
+    FP4Q_TRY(check_swizzle(scale_layout, rows, cols / 16));
+  }
+  if (layouts & FP4Q_COLWISE) {
+    if ((!q_col || !sf_col) && nonempty) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned16(q_col)) return FP4Q_ERR_MISALIGNED;
+    FP4Q_TRY(check_swizzle(scale_layout, cols, rows / 16));
+  }
+  return FP4Q_OK;
+}
+
 }  // namespace fp4q
 
 extern "C" {
@@ -182,7 +206,9 @@ const char *fp4q_status_string(int status) {
 
 const char *fp4q_version(void) { return "fp4q 0.1 (sm_100a)"; }
 
-size_t fp4q_workspace_bytes(void) { return kWorkspaceBytes; }
+size_t fp4q_workspace_bytes(int64_t rows, int64_t cols) {
+  return (rows < 0 || cols < 0) ? 0 : kWorkspaceBytes;
+}
 
 size_t fp4q_scale_bytes(int64_t rows, int64_t cols, int block, int scale_layout) {
   if (rows < 0 || cols < 0 || block <= 0 || cols % block != 0 || !valid_layout(scale_layout))
@@ -194,6 +220,7 @@ size_t fp4q_scale_bytes(int64_t rows, int64_t cols, int block, int scale_layout)
 
 fp4q_status fp4q_amax(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                       float *amax_out, void *stream) {
+  DeviceGuard guard;
   FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
   if (cols % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
   Launch L;
@@ -211,23 +238,10 @@ fp4q_status fp4q_quantize_nvfp4(const void *x, int dtype, int64_t rows, int64_t 
                                 uint8_t *sf_row, uint8_t *q_col, uint8_t *sf_col,
                                 int scale_layout, void *workspace, size_t ws_bytes,
                                 void *stream) {
-  FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
-  if (layouts == 0 || (layouts & ~(FP4Q_ROWWISE | FP4Q_COLWISE)) != 0) return FP4Q_ERR_INVALID_ARG;
-  if (round != FP4Q_RNE && round != FP4Q_SR) return FP4Q_ERR_INVALID_ARG;
-  if (!valid_layout(scale_layout)) return FP4Q_ERR_INVALID_ARG;
-  if (cols % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
-  if ((layouts & FP4Q_COLWISE) && rows % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
-  const bool nonempty = rows > 0 && cols > 0;
-  if (layouts & FP4Q_ROWWISE) {
-    if ((!q_row || !sf_row) && nonempty) return FP4Q_ERR_INVALID_ARG;
-    if (!aligned16(q_row)) return FP4Q_ERR_MISALIGNED;
-    FP4Q_TRY(check_swizzle(scale_layout, rows, cols / 16));
-  }
-  if (layouts & FP4Q_COLWISE) {
-    if ((!q_col || !sf_col) && nonempty) return FP4Q_ERR_INVALID_ARG;
-    if (!aligned16(q_col)) return FP4Q_ERR_MISALIGNED;
-    FP4Q_TRY(check_swizzle(scale_layout, cols, rows / 16));
-  }
+  DeviceGuard guard;
+  FP4Q_TRY(static_cast<fp4q_status>(check_nvfp4_args(x, dtype, rows, cols, ld, layouts, round,
+                                                     q_row, sf_row, q_col, sf_col,
+                                                     scale_layout)));
   Launch L;
   bool none = false;
   FP4Q_TRY(bind_first({x, tensor_scale_out, amax}, stream, &L, &none));
@@ -251,6 +265,7 @@ fp4q_status fp4q_quantize_mxfp4(const void *x, int dtype, int64_t rows, int64_t 
                                 int64_t ld, unsigned layouts, int e8m0_mode, uint8_t *q_row,
                                 uint8_t *sf_row, uint8_t *q_col, uint8_t *sf_col,
                                 int scale_layout, void *stream) {
+  DeviceGuard guard;
   FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
   if (layouts == 0 || (layouts & ~(FP4Q_ROWWISE | FP4Q_COLWISE)) != 0) return FP4Q_ERR_INVALID_ARG;
   if (e8m0_mode < FP4Q_E8M0_RNE || e8m0_mode > FP4Q_E8M0_OCP_FLOOR) return FP4Q_ERR_INVALID_ARG;
@@ -281,6 +296,7 @@ fp4q_status fp4q_quantize_2d(const void *w, int dtype, int64_t rows, int64_t col
                              uint8_t *q_wt, uint8_t *sf_tiles, uint8_t *sf_w_1x16,
                              uint8_t *sf_wt_1x16, int scale_layout, void *workspace,
                              size_t ws_bytes, void *stream) {
+  DeviceGuard guard;
   FP4Q_TRY(check_matrix(w, dtype, rows, cols, ld));
   if (!valid_layout(scale_layout)) return FP4Q_ERR_INVALID_ARG;
   if (rows % 16 != 0 || cols % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
@@ -309,6 +325,7 @@ fp4q_status fp4q_quantize_2d(const void *w, int dtype, int64_t rows, int64_t col
 
 fp4q_status fp4q_rht_amax(const void *dy, int dtype, int64_t tokens, int64_t cols, int64_t ld,
                           int hadamard_n, uint64_t seed, float *amax_out, void *stream) {
+  DeviceGuard guard;
   FP4Q_TRY(check_matrix(dy, dtype, tokens, cols, ld));
   if (hadamard_n != 16 && hadamard_n != 128) return FP4Q_ERR_INVALID_ARG;
   if (tokens % hadamard_n != 0 || cols % 8 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
@@ -326,6 +343,7 @@ fp4q_status fp4q_quantize_rht_sr(const void *dy, int dtype, int64_t tokens, int6
                                  const float *amax_rht, float *tensor_scale_out, uint8_t *q_t,
                                  uint8_t *sf_t, int scale_layout, float *rht_debug_out,
                                  void *workspace, size_t ws_bytes, void *stream) {
+  DeviceGuard guard;
   FP4Q_TRY(check_matrix(dy, dtype, tokens, cols, ld));
   if (hadamard_n != 16 && hadamard_n != 128) return FP4Q_ERR_INVALID_ARG;
   if (round != FP4Q_RNE && round != FP4Q_SR) return FP4Q_ERR_INVALID_ARG;
@@ -373,6 +391,7 @@ fp4q_status fp4q_quantize_backward(const void *dy, int dtype, int64_t tokens, in
                                    float *s_dec_col_out, uint8_t *q_row, uint8_t *sf_row,
                                    uint8_t *q_t, uint8_t *sf_t, int scale_layout, void *workspace,
                                    size_t ws_bytes, void *stream) {
+  DeviceGuard guard;
   FP4Q_TRY(check_matrix(dy, dtype, tokens, cols, ld));
   if (hadamard_n != 16 && hadamard_n != 128) return FP4Q_ERR_INVALID_ARG;
   if (round != FP4Q_RNE && round != FP4Q_SR) return FP4Q_ERR_INVALID_ARG;
@@ -434,6 +453,7 @@ fp4q_status fp4q_quantize_if4(const void *x, int dtype, int64_t rows, int64_t co
                               const float *amax, float *tensor_scale_out, uint8_t *q,
                               uint8_t *sf, int scale_layout, void *workspace, size_t ws_bytes,
                               void *stream) {
+  DeviceGuard guard;
   return quantize_if4_mode(x, dtype, rows, cols, ld, amax, tensor_scale_out, q, sf, scale_layout,
                            workspace, ws_bytes, stream, 1);
 }
@@ -442,6 +462,7 @@ fp4q_status fp4q_quantize_nvint4(const void *x, int dtype, int64_t rows, int64_t
                                  const float *amax, float *tensor_scale_out, uint8_t *q,
                                  uint8_t *sf, int scale_layout, void *workspace,
                                  size_t ws_bytes, void *stream) {
+  DeviceGuard guard;
   return quantize_if4_mode(x, dtype, rows, cols, ld, amax, tensor_scale_out, q, sf, scale_layout,
                            workspace, ws_bytes, stream, 2);
 }
@@ -451,6 +472,7 @@ fp4q_status fp4q_quantize_four_over_six(const void *x, int dtype, int64_t rows, 
                                         float *tensor_scale_out, uint8_t *q_row, uint8_t *sf_row,
                                         uint8_t *q_col, uint8_t *sf_col, int scale_layout,
                                         void *workspace, size_t ws_bytes, void *stream) {
+  DeviceGuard guard;
   FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
   if (layouts == 0 || (layouts & ~(FP4Q_ROWWISE | FP4Q_COLWISE)) != 0) return FP4Q_ERR_INVALID_ARG;
   if (!valid_layout(scale_layout)) return FP4Q_ERR_INVALID_ARG;
@@ -488,6 +510,7 @@ fp4q_status fp4q_quantize_four_over_six(const void *x, int dtype, int64_t rows, 
 fp4q_status fp4q_quantize_if6(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                               const float *amax, float *tensor_scale_out, uint8_t *q, uint8_t *sf,
                               int scale_layout, void *workspace, size_t ws_bytes, void *stream) {
+  DeviceGuard guard;
   FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
   if (!valid_layout(scale_layout)) return FP4Q_ERR_INVALID_ARG;
   if (cols % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
@@ -517,6 +540,7 @@ fp4q_status fp4q_quantize_if6(const void *x, int dtype, int64_t rows, int64_t co
 fp4q_status fp4q_quantize_if3(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                               const float *amax, float *tensor_scale_out, uint8_t *q, uint8_t *sf,
                               int scale_layout, void *workspace, size_t ws_bytes, void *stream) {
+  DeviceGuard guard;
   FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
   if (!valid_layout(scale_layout)) return FP4Q_ERR_INVALID_ARG;
   if (cols % 16 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
@@ -546,6 +570,7 @@ fp4q_status fp4q_quantize_if3(const void *x, int dtype, int64_t rows, int64_t co
 fp4q_status fp4q_quantize_mxfp6(const void *x, int dtype, int64_t rows, int64_t cols,
                                 int64_t ld, int fp6_format, int e8m0_mode, uint8_t *q,
                                 uint8_t *sf, int scale_layout, void *stream) {
+  DeviceGuard guard;
   FP4Q_TRY(check_matrix(x, dtype, rows, cols, ld));
   if (fp6_format != FP4Q_FP6_E2M3 && fp6_format != FP4Q_FP6_E3M2) return FP4Q_ERR_INVALID_ARG;
   if (e8m0_mode < FP4Q_E8M0_RNE || e8m0_mode > FP4Q_E8M0_OCP_FLOOR) return FP4Q_ERR_INVALID_ARG;
@@ -576,6 +601,7 @@ fp4q_status fp4q_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float *
                             const uint8_t *qb, const uint8_t *sfb, const float *tensor_scale_b,
                             int64_t M, int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
                             int *status, void *stream) {
+  DeviceGuard guard;
   return gemm_checked(qa, sfa, tensor_scale_a, qb, sfb, tensor_scale_b, M, N, K, c, c_dtype, ldc,
                       status, stream, 0);
 }
@@ -590,6 +616,7 @@ fp4q_status fp4q_gemm_if4_nvfp4(const uint8_t *qa, const uint8_t *sfa, const flo
                                 const float *tensor_scale_b, int64_t M, int64_t N, int64_t K,
                                 float *c, int64_t ldc, void *workspace, size_t ws_bytes,
                                 int *status, void *stream) {
+  DeviceGuard guard;
   if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4Q_ERR_INVALID_ARG;
   if (M % 128 != 0 || N % 128 != 0 || K % 256 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
   if (K > (int64_t{1} << 30) || M / 128 > 65535) return FP4Q_ERR_UNSUPPORTED_SHAPE;
@@ -632,6 +659,7 @@ fp4q_status fp4q_gemm_nvfp4_withhold_loads(const uint8_t *qa, const uint8_t *sfa
                                            const uint8_t *sfb, const float *tensor_scale_b,
                                            int64_t M, int64_t N, int64_t K, void *c, int c_dtype,
                                            int64_t ldc, int *status, void *stream) {
+  DeviceGuard guard;
   if (!status || K == 0) return FP4Q_ERR_INVALID_ARG;   // the hook exists to set *status
   return gemm_checked(qa, sfa, tensor_scale_a, qb, sfb, tensor_scale_b, M, N, K, c, c_dtype, ldc,
                       status, stream, 1);
@@ -685,6 +713,7 @@ extern "C" {
 fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_layout,
                             int block_rows, int block_cols, const float *tensor_scale,
                             int64_t rows, int64_t cols, void *y, int y_dtype, void *stream) {
+  DeviceGuard guard;
   if (format < FP4Q_FMT_NVFP4 || format > FP4Q_FMT_IF3) return FP4Q_ERR_INVALID_ARG;
   const bool fp6 = format == FP4Q_FMT_MXFP6_E2M3 || format == FP4Q_FMT_MXFP6_E3M2;
   const bool pow2 = fp6 || format == FP4Q_FMT_MXFP4;   // E8M0 scales, no tensor scale

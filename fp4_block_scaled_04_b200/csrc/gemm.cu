@@ -461,16 +461,12 @@ cudaError_t launch_t(const uint8_t *const (&qa)[3], const uint8_t *sfa, const fl
                      int64_t N, int64_t K, void *c, int64_t ldc, int *status, GemmOptions opt,
                      const Launch &L) {
   using T = Tile<BN, NA>;
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<OutT, BN, NA>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               T::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static KernelSetup setup;
+  int per_sm = 0;
+  const cudaError_t e =
+      kernel_setup(setup, reinterpret_cast<const void *>(gemm_nvfp4_kernel<OutT, BN, NA>),
+                   kThreads, T::SMEM_BYTES, &per_sm);
+  if (e != cudaSuccess) return e;
   CUtensorMap map_a[3], map_b;
   for (int i = 0; i < 3; ++i)
     if (!make_map(&map_a[i], qa[NA == 3 ? i : 0], M, K / 2, BM)) return cudaErrorInvalidValue;

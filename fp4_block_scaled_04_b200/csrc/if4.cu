@@ -308,18 +308,10 @@ cudaError_t launch_t(const T *x, int64_t rows, int64_t cols, int64_t ld, const f
                      float *s_dec_out, uint8_t *q, uint8_t *sf, const Launch &L) {
   constexpr int SMEM = kWarps * kStages * 32 * 32 * static_cast<int>(sizeof(T));
   const void *kern = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE>);
-  static int per_sm = 0;
-  if (per_sm == 0) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
-        cudaSuccess)
-      return cudaGetLastError();
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, SMEM) !=
-            cudaSuccess ||
-        per_sm < 1) {
-      cudaGetLastError();
-      per_sm = 1;
-    }
-  }
+  static KernelSetup setup;
+  int per_sm = 0;
+  const cudaError_t e = kernel_setup(setup, kern, kThreads, SMEM, &per_sm);
+  if (e != cudaSuccess) return e;
   const int64_t npairs = rows * ((cols / 16 + 1) / 2);
   const int64_t want = (npairs + kThreads - 1) / kThreads;
   const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;

@@ -4,6 +4,8 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
+
 #include <cuda_runtime.h>
 
 namespace fp4q {
@@ -12,6 +14,72 @@ struct Launch {
   cudaStream_t stream;
   int num_sms;
 };
+
+// Puts the caller's current device back when an entry point returns: the
+// entry points make the device that owns their data current before they
+// enqueue work, and the caller's thread state is not theirs to keep.
+class DeviceGuard {
+ public:
+  DeviceGuard() {
+    if (cudaGetDevice(&prev_) != cudaSuccess) {
+      cudaGetLastError();
+      prev_ = -1;
+    }
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev_ >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev_) cudaSetDevice(prev_);
+  }
+  DeviceGuard(const DeviceGuard &) = delete;
+  DeviceGuard &operator=(const DeviceGuard &) = delete;
+
+ private:
+  int prev_ = -1;
+};
+
+// One-time set-up of a kernel on the current device: its dynamic shared
+// memory limit (when it needs more than the default 48 KB) and how many of
+// its CTAs fit on one SM.  Function attributes belong to a device, so each
+// device is set up once; std::call_once makes concurrent first calls from
+// several host threads safe.  Devices beyond the first 64 are not cached.
+struct KernelSetup {
+  std::once_flag once[64];
+  cudaError_t err[64] = {};
+  int per_sm[64] = {};
+};
+
+inline cudaError_t kernel_setup(KernelSetup &ks, const void *kern, int threads, int smem,
+                                int *per_sm) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return cudaGetLastError();
+  auto run = [&](cudaError_t *err, int *n) {
+    *err = cudaSuccess;
+    if (smem > 48 * 1024) {
+      *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (*err != cudaSuccess) return;
+    }
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, kern, threads, smem) != cudaSuccess ||
+        *n < 1) {
+      cudaGetLastError();
+      *n = 1;
+    }
+  };
+  if (dev >= 64) {
+    cudaError_t e;
+    run(&e, per_sm);
+    return e;
+  }
+  std::call_once(ks.once[dev], [&] { run(&ks.err[dev], &ks.per_sm[dev]); });
+  *per_sm = ks.per_sm[dev];
+  return ks.err[dev];
+}
+
+// The host-side argument checks of fp4q_quantize_nvfp4 that need no device
+// (enums, shape, alignment, required pointers); FP4Q_OK or the status that
+// call would return.
+int check_nvfp4_args(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                     unsigned layouts, int round, const uint8_t *q_row, const uint8_t *sf_row,
+                     const uint8_t *q_col, const uint8_t *sf_col, int scale_layout);
 
 cudaError_t launch_amax(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                         float *amax_out, const Launch &L);

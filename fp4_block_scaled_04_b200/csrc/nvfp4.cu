@@ -485,15 +485,6 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
   cp_async_wait<0>();
 }
 
-int grid_cap(const void *kernel, int threads, const Launch &L) {
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess ||
-      per_sm < 1) {
-    cudaGetLastError();
-    per_sm = 1;
-  }
-  return per_sm * L.num_sms;
-}
 
 template <typename T, bool MX, bool SR, int QMAX = 6>
 cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, unsigned layouts,
@@ -503,9 +494,13 @@ cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, uns
   constexpr int BLK = MX ? 32 : 16;
   if (layouts == FP4Q_ROWWISE) {
     const int64_t nblk = rows * (cols / BLK);
-    static int cap = 0;
-    if (cap == 0) cap = grid_cap(reinterpret_cast<const void *>(rowwise_kernel<T, MX, SR, QMAX>),
-                                 kRowThreads, L);
+    static KernelSetup setup;
+    int per_sm = 0;
+    const cudaError_t e = kernel_setup(
+        setup, reinterpret_cast<const void *>(rowwise_kernel<T, MX, SR, QMAX>), kRowThreads, 0,
+        &per_sm);
+    if (e != cudaSuccess) return e;
+    const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
     const int64_t want = (nblk + 2 * kRowThreads - 1) / (2 * kRowThreads);
     const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
     rowwise_kernel<T, MX, SR, QMAX><<<grid, kRowThreads, 0, L.stream>>>(
@@ -514,18 +509,10 @@ cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, uns
     using G = RCGeom<T, MX>;
     const int64_t ntiles = ((cols + G::WC - 1) / G::WC) * ((rows + G::WR - 1) / G::WR);
     const void *kern = reinterpret_cast<const void *>(rowcol_kernel<T, MX, SR, QMAX>);
-    static int per_sm = 0;
-    if (per_sm == 0) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRCSmem) !=
-          cudaSuccess)
-        return cudaGetLastError();
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRCThreads, kRCSmem) !=
-              cudaSuccess ||
-          per_sm < 1) {
-        cudaGetLastError();
-        per_sm = 1;
-      }
-    }
+    static KernelSetup setup;
+    int per_sm = 0;
+    const cudaError_t e = kernel_setup(setup, kern, kRCThreads, kRCSmem, &per_sm);
+    if (e != cudaSuccess) return e;
     const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
     const int64_t want = (ntiles + kRCThreads / 32 - 1) / (kRCThreads / 32);
     const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));

@@ -192,19 +192,10 @@ cudaError_t launch_2d(const void *w, int dtype, int64_t rows, int64_t cols, int6
   const bool bf = dtype == FP4Q_BF16;
   const void *kern = bf ? reinterpret_cast<const void *>(quant2d_kernel<__nv_bfloat16>)
                         : reinterpret_cast<const void *>(quant2d_kernel<float>);
-  static int per_sm_t[2] = {0, 0};
-  int &per_sm = per_sm_t[bf ? 1 : 0];
-  if (per_sm == 0) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
-        cudaSuccess)
-      return cudaGetLastError();
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, kSmem) !=
-            cudaSuccess ||
-        per_sm < 1) {
-      cudaGetLastError();
-      per_sm = 1;
-    }
-  }
+  static KernelSetup setup_t[2];
+  int per_sm = 0;
+  const cudaError_t e = kernel_setup(setup_t[bf ? 1 : 0], kern, kThreads, kSmem, &per_sm);
+  if (e != cudaSuccess) return e;
   const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
   const int64_t want = (ntiles + kThreads / 32 - 1) / (kThreads / 32);
   const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));

@@ -535,18 +535,10 @@ cudaError_t launch_k(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint
   constexpr int WARP_BYTES = 2 * kUnits * UB + ((N == 128 && SR) ? 128 * 16 * 4 : 0);
   constexpr int SMEM = kWarps * WARP_BYTES;
   const void *kern = reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY, ROW>);
-  static int per_sm = 0;
-  if (per_sm == 0) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
-        cudaSuccess)
-      return cudaGetLastError();
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, SMEM) !=
-            cudaSuccess ||
-        per_sm < 1) {
-      cudaGetLastError();
-      per_sm = 1;
-    }
-  }
+  static KernelSetup setup;
+  int per_sm = 0;
+  const cudaError_t e = kernel_setup(setup, kern, kThreads, SMEM, &per_sm);
+  if (e != cudaSuccess) return e;
   const int64_t ntiles = ((cols + 15) / 16) * ((tokens + 127) / 128);
   const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
   const int64_t want = (ntiles + kWarps - 1) / kWarps;

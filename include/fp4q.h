@@ -34,7 +34,9 @@
  *   - Every pointer argument is a DEVICE pointer owned by the caller, unless
  *     stated otherwise.  The library allocates nothing and keeps no state
  *     between calls.  Inputs, outputs and workspace of one call must be on
- *     the same device; the call runs on that device.
+ *     the same device; the call runs on that device, making it current while
+ *     it enqueues work, and puts the caller's current device back before it
+ *     returns.
  *   - Matrices are row-major.  `ld` is the input's leading dimension in
  *     elements (ld >= cols); ld * element size must be a multiple of 16 bytes
  *     and every pointer must be 16-byte aligned.
@@ -98,9 +100,11 @@ const char *fp4q_status_string(int status);
 /* Library version string (static). */
 const char *fp4q_version(void);
 
-/* Bytes of device workspace the quantize calls need when they compute the
- * tensor amax themselves (amax argument NULL).  Constant. */
-size_t fp4q_workspace_bytes(void);
+/* Bytes of device workspace the quantize calls need for a [rows, cols]
+ * input when they compute the tensor amax themselves (amax argument NULL).
+ * The amax takes 4 bytes at any size, so this is the same 256 bytes for
+ * every valid shape; 0 for negative sizes. */
+size_t fp4q_workspace_bytes(int64_t rows, int64_t cols);
 
 /* Bytes of a scale matrix for a [rows, cols] tensor quantized in blocks of
  * `block` values along cols: [rows, cols/block] in the given layout (the
@@ -129,7 +133,7 @@ fp4q_status fp4q_amax(const void *x, int dtype, int64_t rows, int64_t cols, int6
  *   q_row, sf_row     row-wise codes [rows, cols/2], scales [rows, cols/16]
  *   q_col, sf_col     column-wise codes [cols, rows/2], scales [cols, rows/16]
  *                (pointers of a layout not requested may be NULL)
- *   workspace, ws_bytes  >= fp4q_workspace_bytes() when amax == NULL
+ *   workspace, ws_bytes  >= fp4q_workspace_bytes(rows, cols) when amax == NULL
  * Shape: cols % 16 == 0; COLWISE also needs rows % 16 == 0. */
 fp4q_status fp4q_quantize_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols,
                                 int64_t ld, unsigned layouts, int round, uint64_t seed,
@@ -399,7 +403,11 @@ fp4q_status fp4q_gemm_if4_nvfp4(const uint8_t *qa, const uint8_t *sfa, const flo
                                 float *c, int64_t ldc, void *workspace, size_t ws_bytes,
                                 int *status, void *stream);
 
-/* Failure-detection test hook for fp4q_gemm_nvfp4: the same call, but the
+/* ---- TEST-ONLY ENTRY POINT: not part of the supported interface ----------
+ * Exported so that the failure-detection test can reach it through the C
+ * ABI; production code has no reason to call it.
+ *
+ * Failure-detection test hook for fp4q_gemm_nvfp4: the same call, but the
  * kernel's loader issues no operand loads, so that the tensor-core thread's
  * bounded wait runs out (after about a second).  No tensor-core work is ever
  * issued; the kernel sets *status to 1, writes unspecified values to C, frees
@@ -444,12 +452,16 @@ fp4q_status fp4q_dequantize(int format, const uint8_t *q, const uint8_t *sf, int
  *   - Every GPU that loads the library holds that array until the process
  *     exits. The array's size is the most workspace this call can use.
  *     The call returns FP4Q_ERR_WORKSPACE_TOO_SMALL if
- *     fp4q_workspace_bytes() ever exceeded it.
+ *     fp4q_workspace_bytes(rows, cols) ever exceeded it.
  *     The amax needs 4 bytes at any tensor size, so no shape is refused for
  *     scratch.
  *   - The first call on a device with amax == NULL looks the array's device
  *     address up (cudaGetSymbolAddress, with that device made current).
- *     Make that first call before any stream capture begins.
+ *     Make that first call before any stream capture begins.  The address
+ *     is kept per device and per context: after a cudaDeviceReset the next
+ *     call looks it up again, so make that call outside capture too.
+ *   - Arguments are checked exactly as fp4q_quantize_nvfp4 checks them, and
+ *     a rejected call returns that status before touching any device.
  *   - All calls on one device share the array. The amax pre-pass clears it
  *     before use, and the array keeps the last call's amax afterwards.
  *     Calls with amax == NULL that can overlap on the GPU (different streams,

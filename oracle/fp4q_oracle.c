@@ -91,19 +91,27 @@ float orc_e2m1_value(uint8_t code) {
   return (float)(s ? -mag : mag);
 }
 
+/* Code (0..7) of the E2M1 magnitude nearest to a >= 0, found by trying all
+ * eight magnitudes.  An exact tie between two magnitudes goes to the even
+ * code when ties_to_even is set, else to the smaller magnitude.  a must be
+ * below 6 or saturation is the caller's business (a NaN gives code 0). */
+static int e2m1_nearest_magnitude(double a, int ties_to_even) {
+  int best = 0;
+  double best_d = INFINITY;
+  for (int c = 0; c < 8; ++c) {
+    double d = fabs(a - (double)orc_e2m1_value((uint8_t)c));
+    if (d < best_d || (ties_to_even && d == best_d && (c % 2) == 0)) { best = c; best_d = d; }
+  }
+  return best;
+}
+
 /* Nearest E2M1 value to v; a tie goes to the even code (round to nearest
  * even); magnitudes beyond 6 saturate to 6.  READING: the sign bit copies the
  * sign of v, so a negative value that rounds to zero gives code 0x8. */
 uint8_t orc_e2m1_rne(float v) {
   double a = fabs((double)v);
-  int best = 0;
-  double best_d = INFINITY;
-  if (a >= 6.0) /* saturate: 6 is the nearest value to anything above it */
-    return (uint8_t)(7 | (signbit(v) ? 8 : 0));
-  for (int c = 0; c < 8; ++c) {
-    double d = fabs(a - (double)orc_e2m1_value((uint8_t)c));
-    if (d < best_d || (d == best_d && (c % 2) == 0)) { best = c; best_d = d; }
-  }
+  int best = (a >= 6.0) ? 7 /* 6 is the nearest value to anything above it */
+                        : e2m1_nearest_magnitude(a, 1);
   return (uint8_t)(best | (signbit(v) ? 8 : 0));
 }
 
@@ -1026,25 +1034,23 @@ int orc_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_la
 /* ------------------------------------------------------------------------ */
 
 double orc_glossary_mae(const float *x, int64_t n, int64_t block) {
-  static const float grid[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  /* [G] "FP4の仕組み": the worked example scales each block so that its
+   * largest magnitude becomes 6 (an FP32 scale, not rounded to E4M3),
+   * rounds every scaled magnitude to the nearest E2M1 value -- an exact tie
+   * going to the smaller magnitude -- restores the sign, scales back and
+   * reports the mean absolute error over the tensor. */
   double err = 0.0;
   for (int64_t b = 0; b < n / block; ++b) {
+    const float *xb = x + b * block;
     float m = 0.0f;
     for (int64_t k = 0; k < block; ++k)
-      if (fabsf(x[b * block + k]) > m) m = fabsf(x[b * block + k]);
-    float scale = m / 6.0f;
+      if (fabsf(xb[k]) > m) m = fabsf(xb[k]);
+    const float scale = m / 6.0f;
     for (int64_t k = 0; k < block; ++k) {
-      float xv = x[b * block + k];
-      float v = fabsf(xv) / scale;
-      int best = 0;
-      float best_d = fabsf(v - grid[0]);
-      for (int c = 1; c < 8; ++c) {
-        float d = fabsf(v - grid[c]);
-        if (d < best_d) { best = c; best_d = d; }
-      }
-      float sgn = (xv > 0.0f) ? 1.0f : (xv < 0.0f ? -1.0f : 0.0f);
-      float deq = (grid[best] * sgn) * scale;
-      err += fabs((double)deq - (double)xv);
+      int code = e2m1_nearest_magnitude((double)(fabsf(xb[k]) / scale), 0);
+      if (xb[k] < 0.0f) code |= 8;
+      const float back = orc_e2m1_value((uint8_t)code) * scale;
+      err += fabs((double)back - (double)xb[k]);
     }
   }
   return err / (double)n;

@@ -47,6 +47,8 @@ def test_status_strings_and_constants(L):
     assert fq.fp4q_status_string(99) == "FP4Q_ERR_UNKNOWN"
     assert "sm_100a" in fq.fp4q_version()
     assert fq.fp4q_workspace_bytes() >= 4
+    assert fq.fp4q_workspace_bytes(8192, 4096) == fq.fp4q_workspace_bytes(16, 16) >= 4
+    assert fq.fp4q_workspace_bytes(-1, 16) == 0
 
 
 def test_scale_bytes(L):
@@ -250,3 +252,25 @@ def test_binding_declares_every_header_function():
     src = open(os.path.join(ROOT, "fp4_block_scaled_04_b200", "__init__.py")).read()
     bound = set(re.findall(r'"(fp4q_\w+)":\s*\(', src))
     assert bound == set(declared_functions())
+
+
+def test_noalloc_rejects_what_the_workspace_call_rejects(L):
+    """The no-allocation call checks its arguments exactly as
+    fp4q_quantize_nvfp4 does, before it looks at any device: with amax NULL
+    (the path that would otherwise look up its scratch array first) every
+    rejected call returns the workspace call's status.  No GPU is needed,
+    because nothing past the checks runs."""
+    def both(**kw):
+        a = (kw.get("x", FAKE), kw.get("dtype", 0), kw.get("rows", 32), kw.get("cols", 64),
+             kw.get("ld", 64), kw.get("layouts", 3), kw.get("round", 0), 0, None, FAKE,
+             kw.get("q_row", FAKE), FAKE, kw.get("q_col", FAKE), FAKE, kw.get("layout", 0))
+        return (L.fp4q_quantize_nvfp4_noalloc(*a, None),
+                L.fp4q_quantize_nvfp4(*a, FAKE, 256, None))
+    cases = [dict(dtype=7), dict(layouts=0), dict(layouts=4), dict(round=2), dict(layout=5),
+             dict(cols=24, ld=24), dict(rows=24), dict(ld=60), dict(layout=1),
+             dict(q_row=ctypes.c_void_p(0x7F0000000008)), dict(q_col=None),
+             dict(x=ctypes.c_void_p(0x7F0000000004))]
+    for kw in cases:
+        got, want = both(**kw)
+        assert want != 0, kw
+        assert got == want, (kw, got, want)

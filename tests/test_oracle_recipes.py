@@ -398,3 +398,44 @@ def test_dequant_single_rounding(orc):
     assert np.array_equal(y, want)
     yb = orc.dequantize(orc.FMT_NVFP4, q, sf, rows, cols, s_dec=s_dec, out_dtype=orc.BF16)
     assert np.array_equal(yb, bf16_bits(torch.from_numpy(want)))
+
+
+# ------------------------------------------------ overflow of the block factor
+
+def test_tiny_tensor_clamps_encode_scale_and_block_factor(orc):
+    """A tensor whose amax is 2^-127, worked by hand.
+
+    Reading (the pages never consider overflow): s_enc = RN(2688 / amax) and
+    the block factor r = RN(s_enc / S) are both clamped to FLT_MAX.
+      s_enc: 2688 * 2^127 > FLT_MAX, so s_enc = FLT_MAX = (2 - 2^-23) 2^127.
+      block 0 (max 2^-127): RN(2^-127 * s_enc) = 2 - 2^-23 exactly; divided by
+        6 it is 0.33333331, whose nearest E4M3 values are 0.3125 and 0.34375
+        (midpoint 0.328125), so S = 0.34375 = 11/32, code 0x2B.
+      r = FLT_MAX / (11/32) overflows, so r = FLT_MAX and v = x * FLT_MAX:
+        2^-127 -> 2 - 2^-23 -> E2M1 2 (code 4); -2^-127 -> code 0xC;
+        2^-128 -> 1 - 2^-24 -> 1 (code 2); 3 * 2^-129 -> 1.5 (code 3);
+        2^-129 -> 0.5 - 2^-24 -> 0.5 (code 1); 2^-130 -> 0.25 - 2^-26, just
+        below the tie with 0, -> 0 (code 0); +0 -> +0 (code 0); -0 -> -0
+        (code 8).
+      block 1 is all zeros (and one -0): S = 0, r = 0, codes 0 and 8.
+      s_dec = RN(2^-127 / 2688) = 1560 * 2^-149 (2048 / 1.3125 = 1560.38).
+    Without the clamp on r, r = inf: the non-zero values saturate to +-6 and
+    0 * inf is NaN, so these codes would differ."""
+    p = np.ldexp(1.0, -127)
+    x = np.zeros((1, 32), np.float32)
+    x[0, :8] = [p, -p, p / 2, 3 * p / 4, p / 4, p / 8, 0.0, -0.0]
+    x[0, 17] = -0.0
+    assert x[0, 0] == np.float32(p) and x[0, 3] == np.float32(0.75 * p)   # all exact
+    o = orc.quantize_nvfp4(x, layouts=orc.ROWWISE)
+    assert o["s_dec"].view(np.uint32)[0] == 1560
+    assert list(o["sf_row"].reshape(-1)) == [0x2B, 0x00]
+    codes = unpack(o["q_row"].reshape(1, 16))[0]
+    want = np.zeros(32, np.uint8)
+    want[:8] = [4, 0xC, 2, 3, 1, 0, 0, 8]
+    want[17] = 8
+    assert list(codes) == list(want)
+    # the same tensor through the transposed layout: one column block each
+    oc = orc.quantize_nvfp4(np.ascontiguousarray(x.reshape(32, 1).repeat(16, axis=1)),
+                            layouts=orc.COLWISE)
+    ccodes = unpack(oc["q_col"].reshape(16, 16))[0]
+    assert list(ccodes) == list(want)
