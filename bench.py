@@ -64,14 +64,16 @@ def hbm_peak():
 # ---------------------------------------------------------------------------
 
 class Job:
-    def __init__(self, name, src, bytes_moved, launches, run, e2e=None, oracle=None):
+    def __init__(self, name, src, bytes_moved, launches, run, e2e=None, oracle=None,
+                 run_amax=None):
         self.name = name            # workload / variant
         self.src = src              # CUDA source file of the kernel
         self.bytes = bytes_moved    # algorithmic bytes (input once + outputs)
         self.launches = launches    # our kernels per call
-        self.run = run              # device call (inputs resident)
+        self.run = run              # device call (inputs resident, tensor amax given)
         self.e2e = e2e              # E2E: host inputs -> public API -> host outputs
         self.oracle = oracle        # CPU oracle on a row fraction: returns bytes done
+        self.run_amax = run_amax    # the same call computing the tensor amax first
 
 
 class E2E:
@@ -150,7 +152,9 @@ def build_jobs(device, fq, inputs):
 
     jobs.append(Job("activation 8192x4096 bf16 nvfp4 row+col", "nvfp4.cu", nb_nv, 1,
                     lambda: fq.fp4q_quantize_nvfp4(xa, layouts=3, amax=amax_a, scale_layout=SW,
-                                                   out=out_nv), e2e_nv))
+                                                   out=out_nv), e2e_nv,
+                    run_amax=lambda: fq.fp4q_quantize_nvfp4(xa, layouts=3, scale_layout=SW,
+                                                            out=out_nv)))
     jobs.append(Job("activation 8192x4096 bf16 mxfp4 row+col", "nvfp4.cu", nb_mx, 1,
                     lambda: fq.fp4q_quantize_mxfp4(xa, layouts=3, scale_layout=SW, out=out_mx),
                     e2e_mx))
@@ -168,7 +172,8 @@ def build_jobs(device, fq, inputs):
     e2e_w = E2E([w_h], [we], lambda: fq.fp4q_quantize_2d(we, out=oe_w), oe_w)
 
     jobs.append(Job("weight 14336x4096 fp32 2d16x16 w+wt", "quant2d.cu", nb_w, 1,
-                    lambda: fq.fp4q_quantize_2d(w, amax=amax_w, out=out_w), e2e_w))
+                    lambda: fq.fp4q_quantize_2d(w, amax=amax_w, out=out_w), e2e_w,
+                    run_amax=lambda: fq.fp4q_quantize_2d(w, out=out_w)))
 
     # ---- gradient: RHT + NVFP4 of dY^T ----------------------------------
     g_cpu = inputs["gradient"]
@@ -189,7 +194,9 @@ def build_jobs(device, fq, inputs):
             jobs.append(Job(f"gradient 8192x5120 bf16 rht{n}+{rname}", "rht.cu", nb_g, 1,
                             lambda n=n, rnd=rnd, a=amax_g, o=out_g: fq.fp4q_quantize_rht_sr(
                                 g, n, round=rnd, seed=0, amax_rht=a, scale_layout=SW, out=o),
-                            e2e_g))
+                            e2e_g,
+                            run_amax=lambda n=n, rnd=rnd, o=out_g: fq.fp4q_quantize_rht_sr(
+                                g, n, round=rnd, seed=0, scale_layout=SW, out=o)))
 
     # ---- IF4: quantize and dequantize -----------------------------------
     x5_cpu = inputs["if4"]
@@ -215,7 +222,8 @@ def build_jobs(device, fq, inputs):
 
     jobs.append(Job("if4 16384x8192 bf16 quantize", "if4.cu", nb_q5, 1,
                     lambda: fq.fp4q_quantize_if4(x5, amax=amax5, scale_layout=SW, out=out5),
-                    e2e_q5))
+                    e2e_q5,
+                    run_amax=lambda: fq.fp4q_quantize_if4(x5, scale_layout=SW, out=out5)))
     jobs.append(Job("if4 16384x8192 dequantize to bf16", "dequant.cu", nb_d5, 1,
                     lambda: fq.fp4q_dequantize(fq.FMT_IF4, q5, sf5, R, C, tensor_scale=s5,
                                                scale_layout=SW, out=y5), e2e_d5))
@@ -339,8 +347,22 @@ def build_extra_jobs(device, fq, inputs):
     # MXFP6 (E2M3) of the activation workload: 2 bytes in, 0.75 + 1/32 out
     o6 = fq.fp4q_quantize_mxfp6(xa, fq.FP6_E2M3, scale_layout=SW)
     nb6 = R * C * 2 + R * C * 3 // 4 + R * C // 32
+    # the small parity workload: NVFP4 1x16 of a 256x256 BF16 matrix (codes,
+    # scales, s_dec) and its FP32 dequantization; launch-latency bound
+    xs = inputs["small"].to(device)
+    amax_s = fq.fp4q_amax(xs)
+    osm = fq.fp4q_quantize_nvfp4(xs, layouts=fq.ROWWISE, amax=amax_s)
+    ysm = torch.empty((256, 256), dtype=torch.float32, device=device)
+    nb_sq = 256 * 256 * 2 + 256 * 128 + 256 * 16 + 4
+    nb_sd = 256 * 128 + 256 * 16 + 4 + 256 * 256 * 4
     torch.cuda.synchronize(device)
     return [
+        Job("small 256x256 bf16 nvfp4 quantize (row-wise, rne)", "nvfp4.cu", nb_sq, 1,
+            lambda: fq.fp4q_quantize_nvfp4(xs, layouts=fq.ROWWISE, amax=amax_s, out=osm),
+            run_amax=lambda: fq.fp4q_quantize_nvfp4(xs, layouts=fq.ROWWISE, out=osm)),
+        Job("small 256x256 nvfp4 dequantize to fp32", "dequant.cu", nb_sd, 1,
+            lambda: fq.fp4q_dequantize(fq.FMT_NVFP4, osm["q_row"], osm["sf_row"], 256, 256,
+                                       tensor_scale=osm["s_dec"], out=ysm)),
         Job("gradient 8192x5120 bf16 backward: row-wise sr + rht16+sr from one read", "rht.cu",
             nb_bw, 1, lambda: fq.fp4q_quantize_backward(
                 g, 16, round=fq.SR, seed_row=1, seed_col=0, amax_row=amax_g, amax_rht=amax_r16,
@@ -449,10 +471,12 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 def suite_inputs():
-    """CPU copies of the suite's inputs (activation, weight, gradient, if4)."""
+    """CPU copies of the suite's inputs (activation, weight, gradient, if4)
+    and of the small parity workload."""
     from fp4_block_scaled_04_b200 import workloads
     return {"activation": workloads.activation(), "weight": workloads.weight(),
-            "gradient": workloads.gradient(), "if4": workloads.if4_blocks()}
+            "gradient": workloads.gradient(), "if4": workloads.if4_blocks(),
+            "small": workloads.small_matrix()}
 
 
 def input_digests(inputs):
@@ -522,10 +546,57 @@ def oracle_sample(rows_fraction: float, inputs=None):
                    out_dtype=orc.BF16)
     total_s += time.perf_counter() - t0
     total_b += 2 * (r5 * C * 2 + r5 * C // 2 + r5 * C // 16 + 4)
-    desc = (f"oracle (plain C, 1 thread) on the first {rows_fraction:.4g} of the rows of every "
+    desc = (f"oracle (plain C) on the first {rows_fraction:.4g} of the rows of every "
             f"workload of the suite: activation {ra} rows, weight {rw}, gradient {rg}, "
             f"if4 {r5}")
     return total_b, total_s, desc
+
+
+def host_info():
+    """(usable host cores, CPU model name) of this machine."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:
+        cores = os.cpu_count() or 1
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except Exception:
+        pass
+    return cores, model
+
+
+def oracle_baseline(fraction: float, inputs, runs: int = 3):
+    """The oracle on the same bounded sample, single-threaded and on all host
+    cores (its OpenMP build, which splits only independent rows, columns and
+    tile rows and gives the same bytes); the median of `runs` runs each."""
+    import oracle as orc
+    cores, model = host_info()
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    out = {}
+    try:
+        for mode in ("single", "all"):
+            orc.use_openmp(mode == "all")
+            times, b, desc = [], 0, ""
+            for _ in range(runs):
+                b, sec, desc = oracle_sample(fraction, inputs)
+                times.append(sec)
+            out[mode] = (b, statistics.median(times), desc)
+    finally:
+        orc.use_openmp(False)
+    b1, s1, desc = out["single"]
+    ba, sa, _ = out["all"]
+    return {"value": round(ba / sa / 1e9, 5), "unit": "GB/s",
+            "cores": int(os.environ.get("OMP_NUM_THREADS", cores)), "kind": "oracle",
+            "sample": desc + "; all host cores (OpenMP build, same bytes)",
+            "seconds": round(sa, 3), "runs": runs, "statistic": "median",
+            "host_cores": cores, "cpu_model": model,
+            "single_thread": {"value": round(b1 / s1 / 1e9, 5), "unit": "GB/s", "cores": 1,
+                              "seconds": round(s1, 3)}}
 
 
 # ---------------------------------------------------------------------------
@@ -554,9 +625,13 @@ def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
+    import oracle as orc
     frac = args.reference_fraction
     times, nbytes, desc = [], 0, ""
     inputs = suite_inputs()
+    cores, model = host_info()
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    orc.use_openmp(True)
     for i in range(args.warmup + args.steps):
         b, s, desc = oracle_sample(frac, inputs)
         if i >= args.warmup:
@@ -572,8 +647,10 @@ def run_reference(args):
         "impl": "reference",
         "config": {"workload": "fp4 quantization suite (bounded row sample per step)",
                    "rows_fraction": frac, "l2": "n/a (CPU)", "parallelism": "rank 0 only"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": desc},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s",
+                         "cores": int(os.environ["OMP_NUM_THREADS"]), "kind": "oracle",
+                         "sample": desc + "; all host cores (OpenMP build, same bytes)",
+                         "cpu_model": model},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -588,7 +665,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--reference-fraction", type=float, default=1.0 / 32)
-    ap.add_argument("--cpu-baseline-fraction", type=float, default=1.0 / 8)
+    ap.add_argument("--cpu-baseline-fraction", type=float, default=1.0 / 16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
@@ -665,30 +742,44 @@ def main():
     value = fdist.aggregate_gbs(step_bytes, ws, args.steps, total_ms_max)
     peak, peak_kind = hbm_peak()
 
+    def time_call(run, tag):
+        """Average device time (s) of one call, timed like the suite."""
+        for _ in range(args.warmup):
+            torch.cuda._sleep(LEAD_SLEEP_CYCLES)
+            flush.fill_(tag)
+            torch.sum(flush, dim=0, out=flush_sum)
+            run()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ev:
+            torch.cuda._sleep(LEAD_SLEEP_CYCLES)
+            flush.fill_(tag + 1.0)
+            torch.sum(flush, dim=0, out=flush_sum)
+            a.record(stream)
+            run()
+            b.record(stream)
+        torch.cuda.synchronize(device)
+        return sum(a.elapsed_time(b) for a, b in ev) * 1e-3 / args.steps
+
+    # ---- the same calls with the tensor amax computed first (a pre-pass that
+    # reads the input once more; for the gradient it is the transform's amax)
+    incl_amax = {}
+    for job in jobs:
+        if job.run_amax is not None:
+            incl_amax[job.name] = time_call(job.run_amax, 3.0)
+
     # ---- further calls, timed the same way, outside the headline ----------
     extra = []
     if not args.no_extra:
         xjobs = build_extra_jobs(device, fq, inputs)
         for job in xjobs:
-            for _ in range(args.warmup):
-                torch.cuda._sleep(LEAD_SLEEP_CYCLES)
-                flush.fill_(1.0)
-                torch.sum(flush, dim=0, out=flush_sum)
-                job.run()
-            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
-            for a, b in ev:
-                torch.cuda._sleep(LEAD_SLEEP_CYCLES)
-                flush.fill_(2.0)
-                torch.sum(flush, dim=0, out=flush_sum)
-                a.record(stream)
-                job.run()
-                b.record(stream)
-            torch.cuda.synchronize(device)
-            avg_s = sum(a.elapsed_time(b) for a, b in ev) * 1e-3 / args.steps
+            avg_s = time_call(job.run, 1.0)
             gbs = job.bytes / avg_s / 1e9
-            extra.append({"workload": job.name, "bytes": job.bytes, "us": round(avg_s * 1e6, 2),
-                          "GB/s": round(gbs, 1), "pct_of_peak": round(100 * gbs / peak, 1)})
+            entry = {"workload": job.name, "bytes": job.bytes, "us": round(avg_s * 1e6, 2),
+                     "GB/s": round(gbs, 1), "pct_of_peak": round(100 * gbs / peak, 1)}
+            if job.run_amax is not None:
+                entry["us_incl_amax"] = round(time_call(job.run_amax, 5.0) * 1e6, 2)
+            extra.append(entry)
         del xjobs
         torch.cuda.synchronize(device)
 
@@ -701,10 +792,17 @@ def main():
     for job, ms in zip(jobs, per_job_ms):
         avg_s = ms * 1e-3 / args.steps
         gbs = job.bytes / avg_s / 1e9
-        per_config.append({"workload": job.name, "bytes": job.bytes,
-                           "us": round(avg_s * 1e6, 2), "GB/s": round(gbs, 1),
-                           "pct_of_peak": round(100 * gbs / peak, 1),
-                           "share": round(ms / total_ms, 4)})
+        entry = {"workload": job.name, "bytes": job.bytes,
+                 "us": round(avg_s * 1e6, 2), "GB/s": round(gbs, 1),
+                 "pct_of_peak": round(100 * gbs / peak, 1),
+                 "share": round(ms / total_ms, 4)}
+        if job.name in incl_amax:
+            # the algorithmic bytes stay those of the call itself; the amax
+            # pre-pass's re-read of the input is overhead, not work
+            t = incl_amax[job.name]
+            entry["us_incl_amax"] = round(t * 1e6, 2)
+            entry["GB/s_incl_amax"] = round(job.bytes / t / 1e9, 1)
+        per_config.append(entry)
     dom = max(range(len(jobs)), key=lambda j: per_job_ms[j])
     dom_avg_s = per_job_ms[dom] * 1e-3 / args.steps
     dom_achieved = jobs[dom].bytes / dom_avg_s / 1e9
@@ -749,9 +847,7 @@ def main():
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        b, s, desc = oracle_sample(args.cpu_baseline_fraction, inputs)
-        cpu = {"value": round(b / s / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": desc, "seconds": round(s, 2)}
+        cpu = oracle_baseline(args.cpu_baseline_fraction, inputs)
 
     if rank == 0:
         line = {
@@ -765,7 +861,8 @@ def main():
                                    "bf16 dequant",
                        "l2": "flushed before every kernel (256 MiB written then read, untimed)",
                        "launch": "device sleep before each flush hides host launch latency",
-                       "amax": "precomputed on the device (headline); e2e computes it",
+                       "amax": "precomputed on the device (headline); per_config "
+                               "us_incl_amax and e2e compute it first",
                        "parallelism": f"replicas x{ws}" if ws > 1 else "single gpu",
                        "input_sha256_16": input_digests(inputs)},
             "pct_of_peak": round(100 * value / (ws * peak), 2),

@@ -22,8 +22,11 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "fp4q_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_LIB_OMP_PATH = os.path.join(_HERE, "liboracle_omp.so")
 _lock = threading.Lock()
-_lib = None
+_lib = None          # the library the wrappers below call
+_libs: dict = {}     # loaded builds by path
+_use_openmp = False
 
 BF16, FP32 = 0, 1
 ROWWISE, COLWISE = 1, 2
@@ -37,23 +40,40 @@ FP6_E2M3, FP6_E3M2 = 0, 1
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
 
 
-def build(force: bool = False) -> str:
-    """Compile fp4q_oracle.c into liboracle.so (idempotent)."""
+def build(force: bool = False, openmp: bool = False) -> str:
+    """Compile fp4q_oracle.c into liboracle.so (idempotent).  With openmp, the
+    same source with -fopenmp into liboracle_omp.so: its outer loops over
+    rows, columns or tile rows then run on all host cores and produce the
+    same bytes (each iteration writes whole bytes of its own)."""
+    path = _LIB_OMP_PATH if openmp else _LIB_PATH
     with _lock:
-        stale = (not os.path.exists(_LIB_PATH)
-                 or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+        stale = (not os.path.exists(path)
+                 or os.path.getmtime(path) < os.path.getmtime(_SRC))
         if force or stale:
-            tmp = _LIB_PATH + f".{os.getpid()}.tmp"
-            subprocess.check_call(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"])
-            os.replace(tmp, _LIB_PATH)
-    return _LIB_PATH
+            tmp = path + f".{os.getpid()}.tmp"
+            extra = ["-fopenmp"] if openmp else []
+            subprocess.check_call(["gcc", *CFLAGS, *extra, _SRC, "-o", tmp, "-lm"])
+            os.replace(tmp, path)
+    return path
+
+
+def use_openmp(on: bool = True) -> None:
+    """Route the wrappers below to the OpenMP build (all host cores, the
+    thread count from OMP_NUM_THREADS or the core count) or back to the
+    single-threaded build the tests use."""
+    global _lib, _use_openmp
+    _use_openmp = bool(on)
+    _lib = None
 
 
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        build()
-        L = ctypes.CDLL(_LIB_PATH)
+        path = build(openmp=_use_openmp)
+        if path in _libs:
+            _lib = _libs[path]
+            return _lib
+        L = ctypes.CDLL(path)
         P, I64, I, U, U64, F = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
                                 ctypes.c_uint, ctypes.c_uint64, ctypes.c_float)
         sig = {
@@ -106,6 +126,7 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
+        _libs[path] = L
         _lib = L
     return _lib
 

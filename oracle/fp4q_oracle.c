@@ -26,6 +26,11 @@
  *        even matters when converting the shared scale to E8M0.
  * Where the pages are silent the plainest reading is taken; each such place is
  * marked READING below.
+ *
+ * The outer loops over rows, columns or tile rows carry OpenMP pragmas.  Each
+ * iteration writes whole bytes of its own, so a build with -fopenmp (the
+ * all-core CPU baseline) gives the same bytes as the plain single-threaded
+ * build the tests use, where the pragmas are inert.
  */
 #include <float.h>
 #include <math.h>
@@ -293,6 +298,7 @@ int64_t orc_scale_offset(int64_t r, int64_t c, int64_t rows, int64_t cols, int l
 float orc_amax(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld) {
   float m = 0.0f;
   int any_nan = 0;
+#pragma omp parallel for reduction(max : m) reduction(| : any_nan)
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t c = 0; c < cols; ++c) {
       float a = fabsf(load_elem(x, dtype, ld, r, c));
@@ -379,6 +385,7 @@ static int quantize_1x16(const void *x, int dtype, int64_t rows, int64_t cols, i
   if (s_dec_out) *s_dec_out = s_dec;
 
   if (layouts & ORC_ROWWISE) {
+#pragma omp parallel for
     for (int64_t r = 0; r < rows; ++r)
       for (int64_t b = 0; b < cols / 16; ++b) {
         float m = 0.0f;
@@ -398,6 +405,7 @@ static int quantize_1x16(const void *x, int dtype, int64_t rows, int64_t cols, i
       }
   }
   if (layouts & ORC_COLWISE) {
+#pragma omp parallel for
     for (int64_t c = 0; c < cols; ++c)
       for (int64_t b = 0; b < rows / 16; ++b) {
         float m = 0.0f;
@@ -462,6 +470,7 @@ int orc_quantize_mxfp4(const void *x, int dtype, int64_t rows, int64_t cols, int
   if ((layouts & ORC_ROWWISE) && cols % 32 != 0) return 1;
   if ((layouts & ORC_COLWISE) && rows % 32 != 0) return 1;
   if (layouts & ORC_ROWWISE) {
+#pragma omp parallel for
     for (int64_t r = 0; r < rows; ++r)
       for (int64_t b = 0; b < cols / 32; ++b) {
         float m = 0.0f;
@@ -480,6 +489,7 @@ int orc_quantize_mxfp4(const void *x, int dtype, int64_t rows, int64_t cols, int
       }
   }
   if (layouts & ORC_COLWISE) {
+#pragma omp parallel for
     for (int64_t c = 0; c < cols; ++c)
       for (int64_t b = 0; b < rows / 32; ++b) {
         float m = 0.0f;
@@ -519,6 +529,7 @@ int orc_quantize_2d(const void *w, int dtype, int64_t rows, int64_t cols, int64_
   float s_enc, s_dec;
   orc_tensor_scales(amax, &s_enc, &s_dec);
   if (s_dec_out) *s_dec_out = s_dec;
+#pragma omp parallel for
   for (int64_t tr = 0; tr < rows / 16; ++tr)
     for (int64_t tc = 0; tc < cols / 16; ++tc) {
       float m = 0.0f;
@@ -567,11 +578,13 @@ int orc_rht(const void *dy, int dtype, int64_t tokens, int64_t cols, int64_t ld,
             uint64_t seed, float *t_out /* [tokens, cols] */) {
   if (n != 16 && n != 128) return 1;
   if (tokens % n != 0) return 1;
-  float S[128], u[128];
+  float S[128];
   orc_rht_signs(seed, n, S);
   float cn = orc_rht_norm(n);
+#pragma omp parallel for
   for (int64_t j = 0; j < cols; ++j)
     for (int64_t g = 0; g < tokens / n; ++g) {
+      float u[128];
       for (int k = 0; k < n; ++k) u[k] = S[k] * load_elem(dy, dtype, ld, g * n + k, j);
       for (int h = 1; h < n; h *= 2)
         for (int i = 0; i < n; ++i)
@@ -604,6 +617,7 @@ int orc_quantize_rht(const void *dy, int dtype, int64_t tokens, int64_t cols, in
   float s_enc, s_dec;
   orc_tensor_scales(amax, &s_enc, &s_dec);
   if (s_dec_out) *s_dec_out = s_dec;
+#pragma omp parallel for
   for (int64_t c = 0; c < cols; ++c)
     for (int64_t b = 0; b < tokens / 16; ++b) {
       float m = 0.0f;
@@ -657,6 +671,7 @@ int orc_quantize_if4(const void *x, int dtype, int64_t rows, int64_t cols, int64
   orc_tensor_scales(amax, &s_enc, &s_dec);
   if (s_dec_out) *s_dec_out = s_dec;
   const float C76 = orc_if4_c76(), C67 = orc_if4_c67();
+#pragma omp parallel for
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t b = 0; b < cols / 16; ++b) {
       float xv[16], v[16];
@@ -741,6 +756,7 @@ int orc_quantize_mxfp6(const void *x, int dtype, int64_t rows, int64_t cols, int
   float qmax = orc_fp6_value(31, fmt);
   int emax = (fmt == ORC_FP6_E2M3) ? 2 : 4;
   int64_t rb = cols * 3 / 4;                              /* code bytes per row */
+#pragma omp parallel for
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t b = 0; b < cols / 32; ++b) {
       float m = 0.0f;
@@ -799,6 +815,7 @@ int orc_quantize_if6(const void *x, int dtype, int64_t rows, int64_t cols, int64
   if (s_dec_out) *s_dec_out = s_dec;
   const float CU = orc_if6_cu(), CD = orc_if6_cd();
   const int64_t rb = cols * 3 / 4;
+#pragma omp parallel for
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t b = 0; b < cols / 16; ++b) {
       float xv[16];
@@ -904,6 +921,7 @@ int orc_quantize_if3(const void *x, int dtype, int64_t rows, int64_t cols, int64
   if (s_dec_out) *s_dec_out = s_dec;
   const float CU = orc_if3_cu(), CD = orc_if3_cd();
   const int64_t rb = cols * 3 / 8;
+#pragma omp parallel for
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t b = 0; b < cols / 16; ++b) {
       float xv[16];
@@ -972,6 +990,7 @@ int orc_dequantize(int format, const uint8_t *q, const uint8_t *sf, int scale_la
   const int fp6 = (format == ORC_FMT_MXFP6_E2M3 || format == ORC_FMT_MXFP6_E3M2);
   const int six = fp6 || format == ORC_FMT_IF6;             /* 6-bit codes, 4 per 3 bytes */
   const int three = format == ORC_FMT_IF3;                  /* 3-bit codes, 8 per 3 bytes */
+#pragma omp parallel for
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t c = 0; c < cols; ++c) {
       uint8_t code;

@@ -15,6 +15,17 @@
  * The sign is copied and the value converted by round-to-nearest-even with
  * saturation (the hardware conversion; the oracle's RNE stands in for it
  * here), which also maps 8 to 6.
+ *
+ * Method 2 (subnormal scaling): multiplying |v| by 2^-126 maps E2M1's grid
+ * onto float bit patterns with one rule everywhere: [1, 8) becomes three
+ * normal binades whose E2M1 values keep one mantissa bit, and [0, 1) becomes
+ * the subnormal range, whose uniform step 2^-149 makes E2M1's spacing 0.5
+ * (2^-127) exactly 2^22 steps, the same as in [1, 2).  So the magnitude is
+ * rounded by adding 0x3FFFFF - 64 u to bits(w) and clearing the low 22 bits,
+ * for every |v|, with no test of the range.  The product is rounded up
+ * (towards +inf on the non-negative |v|), which keeps "64 u < frac" exact
+ * where the scaling drops low bits of |v| < 1.  The sign is put back, the
+ * value multiplied by 2^126 (exact) and converted as for method 1.
  * Usage: sr_check <n_random> [method] -- prints the number of mismatches. */
 #include <fenv.h>
 #include <math.h>
@@ -55,8 +66,20 @@ static uint32_t method1(float v, uint32_t u16) {
   return orc_e2m1_rne(flt(bits(r) | (raw & 0x80000000u)));
 }
 
+static uint32_t method2(float v, uint32_t u16) {
+  uint32_t raw = bits(v);
+  fesetround(FE_UPWARD);
+  volatile float w = fabsf(v) * 0x1p-126f;
+  fesetround(FE_TONEAREST);
+  uint32_t R = (bits(w) + 0x3FFFFFu - (u16 << 6)) & 0xFFC00000u;
+  volatile float r = flt(R | (raw & 0x80000000u)) * 0x1p126f;
+  return orc_e2m1_rne(r);
+}
+
 static int which = 0;
-static uint32_t pick(float v, uint32_t u16) { return which ? method1(v, u16) : method(v, u16); }
+static uint32_t pick(float v, uint32_t u16) {
+  return which == 2 ? method2(v, u16) : which ? method1(v, u16) : method(v, u16);
+}
 
 static uint64_t s = 0x9E3779B97F4A7C15ull;
 static uint64_t rnd(void) { s ^= s << 13; s ^= s >> 7; s ^= s << 17; return s; }
@@ -79,6 +102,19 @@ int main(int argc, char **argv) {
         if (pick(-v, u) != orc_e2m1_sr(-v, u)) ++bad;
       }
     }
+  /* the extremes that method 2's scaling reaches: subnormal and tiny v
+     (the product drops low bits), the smallest normals, and magnitudes so
+     large that the scaled value rounds up to 2^128 */
+  const uint32_t edge[] = {0x00000001u, 0x00000003u, 0x00012345u, 0x007FFFFFu, 0x00800000u,
+                           0x00800001u, 0x01000000u, 0x0C000001u, 0x33800001u, 0x34000001u,
+                           0x7F7FFFFFu, 0x7F3FFFFFu, 0x7F400000u, 0x7E000001u};
+  if (which == 2)
+    for (unsigned i = 0; i < sizeof edge / sizeof edge[0]; ++i)
+      for (uint32_t u = 0; u < 65536; ++u) {
+        float v = flt(edge[i]);
+        if (pick(v, u) != orc_e2m1_sr(v, u)) ++bad;
+        if (pick(-v, u) != orc_e2m1_sr(-v, u)) ++bad;
+      }
   for (long i = 0; i < n; ++i) {
     uint64_t r = rnd();
     /* magnitudes spread over [2^-30, 16) */

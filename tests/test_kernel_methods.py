@@ -162,10 +162,11 @@ def test_rint_ties_go_to_even():
     assert np.all(np.rint(t) % 2 == 0)
 
 
-@pytest.mark.parametrize("method", [0, 1])
+@pytest.mark.parametrize("method", [0, 1, 2])
 def test_stochastic_rounding_fixed_point_method(tmp_path, method):
     """The kernels' stochastic rounding methods (0: integer codes, 1: rounded
-    values then the round-to-nearest conversion) equal the oracle's rule
+    values then the round-to-nearest conversion, 2: the same after scaling
+    by 2^-126, which needs no range test) equal the oracle's rule
     (round the magnitude up iff u < t * 2^16) on every u for values around
     each E2M1 grid point and midpoint, and on 4M random pairs."""
     exe = str(tmp_path / "sr_check")

@@ -439,3 +439,39 @@ def test_tiny_tensor_clamps_encode_scale_and_block_factor(orc):
                             layouts=orc.COLWISE)
     ccodes = unpack(oc["q_col"].reshape(16, 16))[0]
     assert list(ccodes) == list(want)
+
+
+# ------------------------------------------------ the all-core oracle build
+
+def test_openmp_build_gives_the_same_bytes(orc):
+    """The OpenMP build of the oracle (the all-core CPU baseline) splits only
+    loops whose iterations write bytes of their own, so every output equals
+    the single-threaded build's byte for byte."""
+    from fp4_block_scaled_04_b200 import workloads
+    x = bf16_bits(workloads.activation(rows=256, cols=512))
+    g = bf16_bits(workloads.gradient(tokens=256, cols=256))
+    w = workloads.weight(rows=64, cols=128).numpy()
+    x5 = bf16_bits(workloads.if4_blocks(rows=64, cols=256))
+
+    def run():
+        out = {}
+        out["nv"] = orc.quantize_nvfp4(x, layouts=3, round=orc.SR, seed=3)
+        out["mx"] = orc.quantize_mxfp4(x, layouts=3)
+        out["2d"] = orc.quantize_2d(w)
+        out["rht16"] = orc.quantize_rht(g, 16, round=orc.SR, seed=1)
+        out["rht128"] = orc.quantize_rht(g, 128, round=orc.RNE, seed=1)
+        out["if4"] = orc.quantize_if4(x5)
+        out["deq"] = {"y": orc.dequantize(orc.FMT_IF4, out["if4"]["q"], out["if4"]["sf"], 64, 256,
+                                          s_dec=float(out["if4"]["s_dec"][0]))}
+        return out
+
+    one = run()
+    try:
+        orc.use_openmp(True)
+        many = run()
+    finally:
+        orc.use_openmp(False)
+    for k in one:
+        for name in one[k]:
+            a, b = np.asarray(one[k][name]), np.asarray(many[k][name])
+            assert a.tobytes() == b.tobytes(), (k, name)
