@@ -34,7 +34,7 @@ __all__ = [
     "fp4q_rht_amax", "fp4q_quantize_rht_sr", "fp4q_quantize_if4", "fp4q_dequantize",
     "fp4q_quantize_nvfp4_noalloc", "fp4q_quantize_nvint4", "fp4q_quantize_four_over_six",
     "fp4q_quantize_backward", "fp4q_quantize_mxfp6", "FMT_MXFP6_E2M3", "FMT_MXFP6_E3M2",
-    "FP6_E2M3", "FP6_E3M2", "fp4q_gemm_nvfp4", "fp4q_quantize_if6", "FMT_IF6",
+    "FP6_E2M3", "FP6_E3M2", "fp4q_gemm_nvfp4", "fp4q_gemm_mxfp4", "fp4q_quantize_if6", "FMT_IF6",
     "fp4q_gemm_if4_nvfp4", "fp4q_quantize_if3", "FMT_IF3",
 ]
 
@@ -98,6 +98,7 @@ _SIGNATURES = {
                                          _I, _P, _SZ, _P]),
     "fp4q_quantize_mxfp6": (_I, [_P, _I, _I64, _I64, _I64, _I, _I, _P, _P, _I, _P]),
     "fp4q_gemm_nvfp4": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P, _P]),
+    "fp4q_gemm_mxfp4": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _I, _I64, _P, _P]),
     "fp4q_gemm_nvfp4_withhold_loads": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I,
                                             _I64, _P, _P]),
     "fp4q_gemm_if4_workspace_bytes": (_SZ, [_I64, _I64]),
@@ -329,6 +330,23 @@ def fp4q_gemm_nvfp4(qa: torch.Tensor, sfa: torch.Tensor, qb: torch.Tensor, sfb: 
     _check("fp4q_gemm_nvfp4", lib().fp4q_gemm_nvfp4(
         _ptr(qa), _ptr(sfa), _ptr(tensor_scale_a), _ptr(qb), _ptr(sfb), _ptr(tensor_scale_b),
         M, N, K, _ptr(c), cdt, c.stride(0) if M > 1 else N, _ptr(status), _stream(qa.device)))
+    return c
+
+
+def fp4q_gemm_mxfp4(qa: torch.Tensor, sfa: torch.Tensor, qb: torch.Tensor, sfb: torch.Tensor,
+                    K: int, out_dtype: torch.dtype = torch.float32,
+                    out: torch.Tensor | None = None,
+                    status: torch.Tensor | None = None) -> torch.Tensor:
+    """C [M, N] = A B^T from MXFP4 operands: codes qa [M, K/2], qb [N, K/2] and
+    their swizzled 1x32 E8M0 scales (as fp4q_quantize_mxfp4 writes them)."""
+    if not qa.is_cuda:
+        raise ValueError("qa must be a CUDA tensor")
+    M, N = qa.shape[0], qb.shape[0]
+    c = torch.empty((M, N), dtype=out_dtype, device=qa.device) if out is None else out
+    cdt = _BF16 if c.dtype == torch.bfloat16 else _FP32
+    _check("fp4q_gemm_mxfp4", lib().fp4q_gemm_mxfp4(
+        _ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), M, N, K, _ptr(c), cdt,
+        c.stride(0) if M > 1 else N, _ptr(status), _stream(qa.device)))
     return c
 
 

@@ -593,7 +593,7 @@ namespace {
 fp4q_status gemm_checked(const uint8_t *qa, const uint8_t *sfa, const float *tensor_scale_a,
                          const uint8_t *qb, const uint8_t *sfb, const float *tensor_scale_b,
                          int64_t M, int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
-                         int *status, void *stream, int withhold);
+                         int *status, void *stream, int withhold, bool mx = false);
 }  // namespace
 }  // namespace fp4q
 
@@ -654,6 +654,14 @@ fp4q_status fp4q_gemm_if4_nvfp4(const uint8_t *qa, const uint8_t *sfa, const flo
                                            tensor_scale_b, M, N, K, c, ldc, status, L));
 }
 
+fp4q_status fp4q_gemm_mxfp4(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
+                            const uint8_t *sfb, int64_t M, int64_t N, int64_t K, void *c,
+                            int c_dtype, int64_t ldc, int *status, void *stream) {
+  DeviceGuard guard;
+  return gemm_checked(qa, sfa, nullptr, qb, sfb, nullptr, M, N, K, c, c_dtype, ldc, status,
+                      stream, 0, /*mx=*/true);
+}
+
 fp4q_status fp4q_gemm_nvfp4_withhold_loads(const uint8_t *qa, const uint8_t *sfa,
                                            const float *tensor_scale_a, const uint8_t *qb,
                                            const uint8_t *sfb, const float *tensor_scale_b,
@@ -672,7 +680,7 @@ namespace {
 fp4q_status gemm_checked(const uint8_t *qa, const uint8_t *sfa, const float *tensor_scale_a,
                          const uint8_t *qb, const uint8_t *sfb, const float *tensor_scale_b,
                          int64_t M, int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
-                         int *status, void *stream, int withhold) {
+                         int *status, void *stream, int withhold, bool mx) {
   if (!valid_dtype(c_dtype)) return FP4Q_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4Q_ERR_INVALID_ARG;
   if (M % 128 != 0 || N % 128 != 0 || K % 256 != 0) return FP4Q_ERR_UNSUPPORTED_SHAPE;
@@ -700,6 +708,9 @@ fp4q_status gemm_checked(const uint8_t *qa, const uint8_t *sfa, const float *ten
   FP4Q_TRY(check_dev(tensor_scale_a, true));
   FP4Q_TRY(check_dev(tensor_scale_b, true));
   FP4Q_TRY(check_dev(status, true));
+  if (mx)
+    return cuda_status(
+        launch_gemm_mxfp4(qa, sfa, qb, sfb, M, N, K, c, c_dtype, ldc, status, L));
   GemmOptions opt;
   opt.withhold = withhold;
   return cuda_status(launch_gemm_nvfp4(qa, sfa, tensor_scale_a, qb, sfb, tensor_scale_b, M, N, K,

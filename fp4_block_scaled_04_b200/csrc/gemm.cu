@@ -53,16 +53,20 @@ constexpr int KTILE = 256;                       // K values per stage
 constexpr int KTB = KTILE / 2;                   // 128 code bytes per row per stage
 constexpr int kThreads = 192;                    // producer warp, MMA warp, 4 epilogue warps
 constexpr int SF_TILE = 512;                     // 128 rows x 4 scales
-constexpr int SF_BYTES = (KTILE / 64) * SF_TILE; // 2048: one operand row tile, one K-tile
 constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at the B200's clock
 
 // NA A operands per output tile: 1 (NVFP4), or 3 (the IF4 split: the FP4
 // blocks accumulate into one accumulator, the two E2M1 parts of the INT4
-// blocks into a second; all three share the A scales).
-template <int BN, int NA = 1>
+// blocks into a second; all three share the A scales).  VS is the scale
+// block: 16 values with E4M3 scales (NVFP4, kind::mxf4nvf4 block16) or 32
+// values with E8M0 scales (MXFP4, kind::mxf4 block32).
+template <int BN, int NA = 1, int VS = 16>
 struct Tile {
   static constexpr int STAGES = NA == 1 ? 4 : 3;
   static constexpr int NACC = NA == 1 ? 1 : 2;
+  // one 512-byte 128x4 scale tile covers 4 VS-value blocks of K
+  static constexpr int SF_TILES = KTILE / (4 * VS);            // per K-tile: 4 or 2
+  static constexpr int SF_BYTES = SF_TILES * SF_TILE;          // one operand row tile, one K-tile
   static constexpr int A_BYTES = BM * KTB;                      // 16384 per A operand
   static constexpr int B_BYTES = BN * KTB;                      // 16384 or 32768
   static constexpr int B_OFF = NA * A_BYTES;
@@ -70,18 +74,22 @@ struct Tile {
   static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES + SF_BYTES + SFB_BYTES;
   static constexpr int BAR_BYTES = 128;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-  // tensor memory: NACC accumulators of BN columns, then per stage 16 columns
-  // of A scales and 4 * BN / 32 columns of B scales
+  // tensor memory: NACC accumulators of BN columns, then per stage 4 columns
+  // per A scale tile and 4 per B scale tile
   static constexpr uint32_t SF_COL0 = NACC * BN;
-  static constexpr uint32_t SFB_COLS = 4 * (BN / 32);
-  static constexpr uint32_t STAGE_COLS = 16 + SFB_COLS;
+  static constexpr uint32_t SFA_COLS = 4 * SF_TILES;
+  static constexpr uint32_t SFB_COLS = 4 * SF_TILES * (BN / 128);
+  static constexpr uint32_t STAGE_COLS = SFA_COLS + SFB_COLS;
   static constexpr uint32_t COLS_USED = NACC * BN + STAGES * STAGE_COLS;
   static constexpr uint32_t TMEM_COLS = COLS_USED <= 256 ? 256 : 512;
-  // Instruction descriptor of tcgen05.mma kind::mxf4nvf4 (block-scaled): A and
-  // B E2M1 (format 1), K-major, E4M3 scales (bit 23 = 0), N (bits 17-22 =
-  // N/8), M = 128 (bits 24-28 = M/16), dense, K = 64.
+  // Instruction descriptor of the block-scaled tcgen05.mma: A and B E2M1
+  // (format 1), K-major, N (bits 17-22 = N/8), M = 128 (bits 24-28 = M/16),
+  // dense, K = 64, scale format in bit 23 (0 = E4M3, 1 = E8M0); the scale
+  // byte within each 32-bit tensor-memory cell goes in bits 29-30 (A) and
+  // 4-5 (B) per instruction.
   static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
-                                    (uint32_t(BM >> 4) << 24);
+                                    (VS == 32 ? (1u << 23) : 0u) | (uint32_t(BM >> 4) << 24);
+  static_assert(VS == 16 || VS == 32, "scale block of 16 (NVFP4) or 32 (MXFP4)");
   static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
   static_assert(COLS_USED <= 512, "tensor memory");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -146,15 +154,25 @@ __device__ __forceinline__ void tc_copy_sf(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
                : "memory");
 }
+template <int VS>
 __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
                                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
-      "[%6], p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
-      : "memory");
+  if (VS == 16)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
+        "[%6], p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], "
+        "[%6], p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
 }
 
 // 16 consecutive FP32 accumulator columns of this thread's row (warp w reads
@@ -200,7 +218,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
       : "memory");
 }
 
-template <typename OutT, int BN, int NA>
+template <typename OutT, int BN, int NA, int VS>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
                   const __grid_constant__ CUtensorMap map_a1,
@@ -210,8 +228,9 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
                   const float *__restrict__ s_b, int K, int n_tiles_n, int n_tiles,
                   OutT *__restrict__ c, int64_t ldc, int *__restrict__ status,
                   GemmOptions opt) {
-  using T = Tile<BN, NA>;
+  using T = Tile<BN, NA, VS>;
   constexpr int STAGES = T::STAGES;
+  constexpr int SF_BYTES = T::SF_BYTES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -226,7 +245,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KT = K / KTILE;
-  const int64_t sf_rowtile = static_cast<int64_t>(K / 64) * SF_TILE;   // bytes per 128-row tile
+  // bytes of the scales of one 128-row tile: K / (4 VS) tiles of 512 bytes
+  const int64_t sf_rowtile = static_cast<int64_t>(K / (4 * VS)) * SF_TILE;
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -307,25 +327,34 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
           tc_fence_after();
           const uint32_t st = base + s * T::STAGE_BYTES;
           const uint32_t sfa_col = tmem + T::SF_COL0 + T::STAGE_COLS * s;
-          const uint32_t sfb_col = sfa_col + 16u;
+          const uint32_t sfb_col = sfa_col + T::SFA_COLS;
+          // scale tile t (4 VS-value blocks of K) of every operand row tile
+          // into 4 tensor-memory columns: A at sfa_col + 4 t, B rows
+          // 128 h .. 128 h + 127 at sfb_col + 4 (BN / 128) t + 4 h
 #pragma unroll
-          for (int kb = 0; kb < KTILE / 64; ++kb) {
-            tc_copy_sf(sfa_col + 4u * kb, desc_sf(st + T::B_OFF + T::B_BYTES + kb * SF_TILE));
+          for (int t = 0; t < T::SF_TILES; ++t) {
+            tc_copy_sf(sfa_col + 4u * t, desc_sf(st + T::B_OFF + T::B_BYTES + t * SF_TILE));
 #pragma unroll
-            for (int h = 0; h < BN / 128; ++h)   // B rows 128h .. 128h + 127: columns 4h .. 4h + 3
-              tc_copy_sf(sfb_col + (T::SFB_COLS / 4) * kb + 4u * h,
+            for (int h = 0; h < BN / 128; ++h)
+              tc_copy_sf(sfb_col + 4u * (BN / 128) * t + 4u * h,
                          desc_sf(st + T::B_OFF + T::B_BYTES + SF_BYTES + h * SF_BYTES +
-                                 kb * SF_TILE));
+                                 t * SF_TILE));
           }
           const uint64_t da = desc_sw128(st), db = desc_sw128(st + T::B_OFF);
 #pragma unroll
           for (int kb = 0; kb < KTILE / 64; ++kb) {     // 64 values = 32 bytes = 2 descriptor units
-            const uint32_t sa = sfa_col + 4u * kb, sb = sfb_col + (T::SFB_COLS / 4) * kb;
-            tc_mma(tmem, da + 2u * kb, db + 2u * kb, T::IDESC, sa, sb, (kt | kb) != 0);
+            // the scales of these 64 values: all four bytes of tile kb
+            // (VS 16), or bytes 2 (kb % 2) and up of tile kb / 2 (VS 32); the
+            // byte goes in the address's top bits and in the descriptor
+            const uint32_t t = VS == 16 ? kb : kb / 2, id = VS == 16 ? 0u : 2u * (kb & 1);
+            const uint32_t sa = (sfa_col + 4u * t) | (id << 30);
+            const uint32_t sb = (sfb_col + 4u * (BN / 128) * t) | (id << 30);
+            const uint32_t idesc = T::IDESC | (id << 29) | (id << 4);
+            tc_mma<VS>(tmem, da + 2u * kb, db + 2u * kb, idesc, sa, sb, (kt | kb) != 0);
             if (NA == 3) {                              // both INT4 parts into accumulator 1
               const uint64_t da1 = desc_sw128(st + T::A_BYTES), da2 = desc_sw128(st + 2 * T::A_BYTES);
-              tc_mma(tmem + BN, da1 + 2u * kb, db + 2u * kb, T::IDESC, sa, sb, (kt | kb) != 0);
-              tc_mma(tmem + BN, da2 + 2u * kb, db + 2u * kb, T::IDESC, sa, sb, 1u);
+              tc_mma<VS>(tmem + BN, da1 + 2u * kb, db + 2u * kb, idesc, sa, sb, (kt | kb) != 0);
+              tc_mma<VS>(tmem + BN, da2 + 2u * kb, db + 2u * kb, idesc, sa, sb, 1u);
             }
           }
           tc_commit(empty + 8 * s);
@@ -455,16 +484,16 @@ bool make_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t row_b
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename OutT, int BN, int NA>
+template <typename OutT, int BN, int NA, int VS = 16>
 cudaError_t launch_t(const uint8_t *const (&qa)[3], const uint8_t *sfa, const float *s_a,
                      const uint8_t *qb, const uint8_t *sfb, const float *s_b, int64_t M,
                      int64_t N, int64_t K, void *c, int64_t ldc, int *status, GemmOptions opt,
                      const Launch &L) {
-  using T = Tile<BN, NA>;
+  using T = Tile<BN, NA, VS>;
   static KernelSetup setup;
   int per_sm = 0;
   const cudaError_t e =
-      kernel_setup(setup, reinterpret_cast<const void *>(gemm_nvfp4_kernel<OutT, BN, NA>),
+      kernel_setup(setup, reinterpret_cast<const void *>(gemm_nvfp4_kernel<OutT, BN, NA, VS>),
                    kThreads, T::SMEM_BYTES, &per_sm);
   if (e != cudaSuccess) return e;
   CUtensorMap map_a[3], map_b;
@@ -475,21 +504,21 @@ cudaError_t launch_t(const uint8_t *const (&qa)[3], const uint8_t *sfa, const fl
   // tiles in row-major order, each CTA taking every gridDim-th tile
   const int64_t n_tiles_n = N / BN, n_tiles = (M / BM) * n_tiles_n;
   const int grid = static_cast<int>(n_tiles < L.num_sms ? n_tiles : L.num_sms);
-  gemm_nvfp4_kernel<OutT, BN, NA><<<grid, kThreads, T::SMEM_BYTES, L.stream>>>(
+  gemm_nvfp4_kernel<OutT, BN, NA, VS><<<grid, kThreads, T::SMEM_BYTES, L.stream>>>(
       map_a[0], map_a[1], map_a[2], map_b, sfa, s_a, sfb, s_b, static_cast<int>(K),
       static_cast<int>(n_tiles_n), static_cast<int>(n_tiles), static_cast<OutT *>(c), ldc,
       status, opt);
   return cudaGetLastError();
 }
 
-template <typename OutT>
+template <typename OutT, int VS = 16>
 cudaError_t launch_o(const uint8_t *qa, const uint8_t *sfa, const float *s_a, const uint8_t *qb,
                      const uint8_t *sfb, const float *s_b, int64_t M, int64_t N, int64_t K,
                      void *c, int64_t ldc, int *status, GemmOptions opt, const Launch &L) {
   const uint8_t *const a[3] = {qa, qa, qa};
   if (N % 256 == 0)
-    return launch_t<OutT, 256, 1>(a, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
-  return launch_t<OutT, 128, 1>(a, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
+    return launch_t<OutT, 256, 1, VS>(a, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
+  return launch_t<OutT, 128, 1, VS>(a, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
 }
 
 }  // namespace
@@ -512,6 +541,17 @@ cudaError_t launch_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float
   if (c_dtype == FP4Q_BF16)
     return launch_o<__nv_bfloat16>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
   return launch_o<float>(qa, sfa, s_a, qb, sfb, s_b, M, N, K, c, ldc, status, opt, L);
+}
+
+cudaError_t launch_gemm_mxfp4(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
+                              const uint8_t *sfb, int64_t M, int64_t N, int64_t K, void *c,
+                              int c_dtype, int64_t ldc, int *status, const Launch &L) {
+  GemmOptions opt;
+  if (c_dtype == FP4Q_BF16)
+    return launch_o<__nv_bfloat16, 32>(qa, sfa, nullptr, qb, sfb, nullptr, M, N, K, c, ldc,
+                                       status, opt, L);
+  return launch_o<float, 32>(qa, sfa, nullptr, qb, sfb, nullptr, M, N, K, c, ldc, status, opt,
+                             L);
 }
 
 }  // namespace fp4q

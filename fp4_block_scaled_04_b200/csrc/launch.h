@@ -38,7 +38,7 @@ class DeviceGuard {
 };
 
 // One-time set-up of a kernel on the current device: its dynamic shared
-// memory limit (when it needs more than the default 48 KB) and how many of
+// memory limit and how many of
 // its CTAs fit on one SM.  Function attributes belong to a device, so each
 // device is set up once; std::call_once makes concurrent first calls from
 // several host threads safe.  Devices beyond the first 64 are not cached.
@@ -54,7 +54,7 @@ inline cudaError_t kernel_setup(KernelSetup &ks, const void *kern, int threads, 
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return cudaGetLastError();
   auto run = [&](cudaError_t *err, int *n) {
     *err = cudaSuccess;
-    if (smem > 48 * 1024) {
+    if (smem > 0) {   // the limit counts dynamic shared memory on top of the static
       *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (*err != cudaSuccess) return;
     }
@@ -148,6 +148,12 @@ cudaError_t launch_gemm_nvfp4(const uint8_t *qa, const uint8_t *sfa, const float
                               const uint8_t *qb, const uint8_t *sfb, const float *s_b, int64_t M,
                               int64_t N, int64_t K, void *c, int c_dtype, int64_t ldc,
                               int *status, GemmOptions opt, const Launch &L);
+
+// C[M, N] = A B^T from MXFP4 operands (codes [rows, K/2], E8M0 scales per 32
+// values in the 128x4 tile layout, no tensor scale) on the tensor cores
+cudaError_t launch_gemm_mxfp4(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
+                              const uint8_t *sfb, int64_t M, int64_t N, int64_t K, void *c,
+                              int c_dtype, int64_t ldc, int *status, const Launch &L);
 
 // IF4 x NVFP4 in one pass over the split operands: C = RN(RN(acc_fp * a) +
 // RN(acc_int * RN(a * RN(6/7)))), acc_int accumulating both INT4 parts; FP32

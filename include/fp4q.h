@@ -403,6 +403,26 @@ fp4q_status fp4q_gemm_if4_nvfp4(const uint8_t *qa, const uint8_t *sfa, const flo
                                 float *c, int64_t ldc, void *workspace, size_t ws_bytes,
                                 int *status, void *stream);
 
+/* Block-scaled MXFP4 GEMM on the tensor cores: the consumer of
+ * fp4q_quantize_mxfp4's swizzled outputs.  Ultralytics glossary "FP4",
+ * section "FP4の仕組み" (MXFP4: 32 E2M1 values share one power-of-two E8M0
+ * scale, no tensor scale); the AIBR summary of Quartet (MXFP4 operands in the
+ * linear layers on Blackwell).  With A = dequantize(qa, sfa) and B =
+ * dequantize(qb, sfb):
+ *   C[m, n] = acc[m, n],  acc = A B^T accumulated in FP32 by tcgen05.mma
+ * kind::mxf4 block32 (the order of the FP32 additions is the hardware's; the
+ * result is within FP32 accumulation error of the exact product).
+ *   qa, sfa      A codes [M, K/2] (K-major) and its 1x32 E8M0 scales in
+ *                FP4Q_SCALE_SWIZZLED_128x4, as fp4q_quantize_mxfp4 writes them
+ *                (a column-wise output is the row-wise layout of the transpose)
+ *   qb, sfb      B codes [N, K/2] and scales, the same way
+ *   c, c_dtype, ldc, status  as for fp4q_gemm_nvfp4
+ * Shape: M % 128 == 0, N % 128 == 0, K % 256 == 0; alignment as for
+ * fp4q_gemm_nvfp4.  K == 0 writes zeros.  Nothing is allocated. */
+fp4q_status fp4q_gemm_mxfp4(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
+                            const uint8_t *sfb, int64_t M, int64_t N, int64_t K, void *c,
+                            int c_dtype, int64_t ldc, int *status, void *stream);
+
 /* ---- TEST-ONLY ENTRY POINT: not part of the supported interface ----------
  * Exported so that the failure-detection test can reach it through the C
  * ABI; production code has no reason to call it.
