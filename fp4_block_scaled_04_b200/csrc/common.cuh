@@ -8,6 +8,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -92,11 +93,14 @@ __device__ __forceinline__ uint32_t e2m1x4(float f0, float f1, float f2, float f
 // E4M3 encode / decode (block scales)
 // ---------------------------------------------------------------------------
 
-// s >= 0 -> E4M3 code, round to nearest even, saturating at 448 (0x7E).
+// s >= 0 -> E4M3 code, round to nearest even, saturating at 448 (0x7E).  The
+// code is masked to 7 bits, a no-op for s >= 0 that keeps it a valid index
+// into a 128-entry factor table even for a NaN (lanes outside the matrix may
+// compute on stale values whose results are never stored).
 __device__ __forceinline__ uint32_t e4m3_code(float s) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(s));
-  return r & 0xFFu;
+  return r & 0x7Fu;
 }
 
 // Value of a 7-bit E4M3 magnitude code (sign bit ignored).
@@ -374,6 +378,21 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   return r;
 }
 
+// The E4M3 codes of two block scales at once: the same correctly rounded
+// steps as nvfp4_scale_code lane by lane (RN(m * s_enc), then Markstein's
+// division by 6) as f32x2 operations, and one conversion for both codes:
+// code of a in bits 0..7, of b in bits 8..15.
+__device__ __forceinline__ uint32_t nvfp4_scale_code2(float a, float b, float s_enc) {
+  constexpr float kInv6 = 1.0f / 6.0f;
+  const float2 y = mul2(make_float2(a, b), make_float2(s_enc, s_enc));
+  const float2 q0 = mul2(y, make_float2(kInv6, kInv6));
+  const float2 r = fma2(q0, make_float2(-6.0f, -6.0f), y);
+  const float2 q = fma2(r, make_float2(kInv6, kInv6), q0);
+  uint16_t c;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(q.y), "f"(q.x));
+  return c;
+}
+
 // per 16-bit lane: max(|a|, |b|) of two BF16 pairs (the sign bits of the
 // result are meaningless; mask with 0x7FFF7FFF)
 __device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
@@ -414,6 +433,56 @@ __device__ __forceinline__ float e2m1_sr_value(float v, uint32_t z) {
 // z of the low / high 16-bit uniform of a 32-bit word
 __device__ __forceinline__ uint32_t sr_z_lo(uint32_t w) { return 0x3FFFFFu ^ ((w << 6) & 0x3FFFC0u); }
 __device__ __forceinline__ uint32_t sr_z_hi(uint32_t w) { return 0x3FFFFFu ^ ((w >> 10) & 0x3FFFC0u); }
+
+// Stochastic rounding of v onto the E2M1 grid by scaling (the oracle's rule,
+// checked against it by tests/sr_check.c, method 2): w = RU(|v| * 2^-126)
+// maps the whole E2M1 grid onto float bit patterns that keep the top 2^22
+// ulps of the low bits -- [1, 8) onto normal binades with one mantissa bit
+// kept, [0, 1) onto the subnormals, whose uniform step makes E2M1's 0.5
+// spacing 2^22 steps too -- so adding 0x3FFFFF - 64 u and clearing the low
+// 22 bits rounds the magnitude up exactly when 64 u < frac, with no range
+// test.  Rounding the product up keeps that comparison exact where the
+// scaling drops low bits of |v| < 1.  The sign is put back and the product
+// with 2^126 (exact) is encoded by the round-to-nearest conversion, which
+// maps 8 (and anything larger, including an overflow to infinity) to 6.
+// x64 = 64 u (sr_x_lo / sr_x_hi).
+__device__ __forceinline__ uint32_t sr_scaled_bits(float v, uint32_t x64) {
+  const float w = __fmul_ru(fabsf(v), 0x1p-126f);
+  const uint32_t b = (__float_as_uint(w) + 0x3FFFFFu - x64) & 0xFFC00000u;
+  return b | (__float_as_uint(v) & 0x80000000u);
+}
+__device__ __forceinline__ float e2m1_sr_scaled(float v, uint32_t x64) {
+  return __fmul_rn(__uint_as_float(sr_scaled_bits(v, x64)), 0x1p126f);
+}
+// two values at once; the final exact scaling is one f32x2 product
+__device__ __forceinline__ float2 e2m1_sr_scaled2(float2 v, uint32_t xa, uint32_t xb) {
+  return mul2(make_float2(__uint_as_float(sr_scaled_bits(v.x, xa)),
+                          __uint_as_float(sr_scaled_bits(v.y, xb))),
+              make_float2(0x1p126f, 0x1p126f));
+}
+// 64 u of the low / high 16-bit uniform of a 32-bit word
+__device__ __forceinline__ uint32_t sr_x_lo(uint32_t w) { return (w << 6) & 0x3FFFC0u; }
+__device__ __forceinline__ uint32_t sr_x_hi(uint32_t w) { return (w >> 10) & 0x3FFFC0u; }
+
+// max(|a|, |b|, |c|) in one three-input maximum (inputs finite)
+__device__ __forceinline__ float absmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
+  return r;
+}
+// max over |v[0..N)|, N >= 3 odd or even
+template <int N>
+__device__ __forceinline__ float absmax_n(const float (&v)[N]) {
+  float m = absmax3(v[0], v[1], v[2]);
+#pragma unroll
+  for (int i = 3; i + 1 < N; i += 2) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(m), "f"(fabsf(v[i])), "f"(fabsf(v[i + 1])));
+    m = r;
+  }
+  if ((N - 3) % 2 == 1) m = fmaxf(m, fabsf(v[N - 1]));
+  return m;
+}
 
 // Philox4x32-10 with the round keys held by the caller (they depend only on
 // the seed).
@@ -462,16 +531,17 @@ __device__ __forceinline__ void cp_async_wait() {
 
 // Coordinates (tile row tt, tile column tc) of a linear tile index over a
 // grid of tiles_c tile columns, stepped by a fixed number of tiles without
-// dividing.
-struct TileCursor {
-  int64_t tile, tt, tc;
-  __device__ __forceinline__ void init(int64_t t, int64_t tiles_c) {
+// dividing.  I is the index type: int32_t where the launcher has checked that
+// every index fits, int64_t otherwise.
+template <typename I>
+struct TileCursorT {
+  I tile, tt, tc;
+  __device__ __forceinline__ void init(I t, I tiles_c) {
     tile = t;
     tt = t / tiles_c;
     tc = t - tt * tiles_c;
   }
-  __device__ __forceinline__ void advance(int64_t step, int64_t dtt, int64_t dtc,
-                                          int64_t tiles_c) {
+  __device__ __forceinline__ void advance(I step, I dtt, I dtc, I tiles_c) {
     tile += step;
     tt += dtt;
     tc += dtc;
@@ -481,5 +551,14 @@ struct TileCursor {
     }
   }
 };
+using TileCursor = TileCursorT<int64_t>;
+
+// scale_offset in the index type I
+template <typename I>
+__device__ __forceinline__ I scale_offset_t(I r, I c, I cols, int layout) {
+  if (layout == FP4Q_SCALE_LINEAR) return r * cols + c;
+  const I tile = (r >> 7) * (cols >> 2) + (c >> 2);
+  return tile * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
 
 }  // namespace fp4q

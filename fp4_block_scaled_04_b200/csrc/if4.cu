@@ -10,7 +10,9 @@
 // A lane quantizes two adjacent blocks at once: every elementwise step is one
 // f32x2 instruction whose lanes are (block A element k, block B element k),
 // so each lane still sums its own block's squared errors in order k = 0..15,
-// as the definition requires.
+// as the definition requires.  Products that feed an add or subtract are
+// f32x2 fused multiply-adds with a -0 addend known only at run time, which
+// keeps them from being contracted into the add (see if4_pair).
 //   FP4:  codes by cvt.rn.satfinite.e2m1x2, values back by cvt.f16x2.e2m1x2,
 //         errors RN(g - v) by the mixed-precision sub.f32.f16 (g is exact in
 //         f16; the sign of the difference does not change its square)
@@ -77,8 +79,14 @@ __device__ __forceinline__ uint32_t fp4_codes_diffs(const float (&v)[8], float (
 // Both candidates of blocks A and B (lanes .x / .y of the pairs); picks the
 // smaller error per block (MODE 1, IF4) or keeps INT4 (MODE 2, NVINT4, which
 // needs neither the FP4 candidate nor the errors).
+// nz is -0.0 passed in at run time: fma(a, b, -0) is exactly RN(a * b), signed
+// zeros included, and because the compiler cannot see that the addend is
+// zero it keeps the product a separate fused multiply-add, which it never
+// contracts with the add or subtract that consumes it.  (A plain f32x2
+// multiply followed by an f32x2 add has been seen contracted into one fused
+// operation despite .rn, which rounds once instead of twice.)
 template <bool CLAMP, int MODE>
-__device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float c67,
+__device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float c67, float nz,
                                          uint32_t (&wa)[2], uint32_t (&wb)[2], bool &int_a,
                                          bool &int_b) {
   // FP4 candidates and their differences, in element order
@@ -102,20 +110,18 @@ __device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float
   for (int k = 0; k < 16; ++k) {
     const int h = k >> 3, i = k & 7;
     const float2 vk = v[k];
-    // No product below feeds a packed add or subtract: ptxas may contract a
-    // mul.f32x2 -> add.f32x2 pair into one fused operation even with .rn,
-    // which rounds once instead of twice.  Products that are added to are
-    // scalar __fmul_rn / __fadd_rn / __fsub_rn, which are never fused.
-    float tx = __fmul_rn(vk.x, c76), ty = __fmul_rn(vk.y, c76);
+    // t = RN(v * RN(7/6)) and h = RN(k * RN(6/7)) are products that feed an
+    // add or subtract: each is fma(a, b, -0) with the run-time zero nz
+    float2 t2 = fma2(vk, make_float2(c76, c76), make_float2(nz, nz));
     if (CLAMP) {
-      tx = fminf(fmaxf(tx, -7.25f), 7.25f);
-      ty = fminf(fmaxf(ty, -7.25f), 7.25f);
+      t2.x = fminf(fmaxf(t2.x, -7.25f), 7.25f);
+      t2.y = fminf(fmaxf(t2.y, -7.25f), 7.25f);
     }
-    const float2 tm = make_float2(__fadd_rn(tx, kMagic), __fadd_rn(ty, kMagic));
+    const float2 tm = add2(t2, make_float2(kMagic, kMagic));
     if (MODE == 1) {
       const float2 kf = sub2(tm, make_float2(kMagic, kMagic));    // rint(t), exact
-      const float2 hv = mul2(kf, make_float2(c67, c67));
-      const float2 dint = make_float2(__fsub_rn(vk.x, hv.x), __fsub_rn(vk.y, hv.y));
+      const float2 hv = fma2(kf, make_float2(c67, c67), make_float2(nz, nz));
+      const float2 dint = sub2(vk, hv);
       efp = fma2(make_float2(da[k], db[k]), make_float2(da[k], db[k]), efp);
       eint = fma2(dint, dint, eint);
     }
@@ -137,15 +143,17 @@ __device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float
 
 
 // Position of a lane's pair: row r and first block cb = 2 * pc, advanced by
-// a fixed stride of pairs.
+// a fixed stride of pairs.  I is int32_t where every element and input offset
+// fits (the launcher checks), int64_t otherwise.
+template <typename I>
 struct Cursor {
-  int64_t p, r, pc;
-  __device__ __forceinline__ void init(int64_t p0, int64_t ppr) {
+  I p, r, pc;
+  __device__ __forceinline__ void init(I p0, I ppr) {
     p = p0;
     r = p0 / ppr;
     pc = p0 - r * ppr;
   }
-  __device__ __forceinline__ void advance(int64_t stride, int64_t dr, int64_t dpc, int64_t ppr) {
+  __device__ __forceinline__ void advance(I stride, I dr, I dpc, I ppr) {
     p += stride;
     r += dr;
     pc += dpc;
@@ -156,11 +164,13 @@ struct Cursor {
   }
 };
 
-template <typename T, bool SWZ, int MODE>
+template <typename T, bool SWZ, int MODE, typename I>
 __global__ void __launch_bounds__(kThreads, 4)
-if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
            const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
-           uint8_t *__restrict__ q, uint8_t *__restrict__ sf) {
+           uint8_t *__restrict__ q, uint8_t *__restrict__ sf, float nz) {
+  const I rows = static_cast<I>(rows_), cols = static_cast<I>(cols_), ld = static_cast<I>(ld_);
+  const bool sf_even = (reinterpret_cast<uintptr_t>(sf) & 1u) == 0;
   constexpr int LB = 32 * sizeof(T);          // bytes of a lane's pair
   constexpr int PPL = LB / 16;                // 16-byte pieces per lane
   constexpr int PPB = PPL / 2;                // pieces per block
@@ -178,14 +188,14 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
 
   // work unit: a pair of adjacent blocks (cb, cb + 1) of one row; an odd
   // last block of a row pairs with itself
-  const int64_t bpr = cols / 16, ppr = (bpr + 1) / 2, npairs = rows * ppr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  const int64_t p0 = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-  const int64_t dr = stride / ppr, dpc = stride - dr * ppr;
+  const I bpr = cols / 16, ppr = (bpr + 1) / 2, npairs = rows * ppr;
+  const I stride = static_cast<I>(gridDim.x) * kThreads;
+  const I p0 = static_cast<I>(blockIdx.x) * kThreads + static_cast<I>(threadIdx.x);
+  const I dr = stride / ppr, dpc = stride - dr * ppr;
 
-  auto issue = [&](const Cursor &c, int st) {
+  auto issue = [&](const Cursor<I> &c, int st) {
     if (c.p >= npairs) return;
-    const int64_t cb = 2 * c.pc;
+    const I cb = 2 * c.pc;
     const uint8_t *src = reinterpret_cast<const uint8_t *>(x + c.r * ld + cb * 16);
     const int n = (cb + 1 < bpr) ? PPL : PPB;
     const uint32_t dst = my_s + static_cast<uint32_t>(st * STAGE);
@@ -194,7 +204,7 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
       if (i < n) cp_async16(dst + static_cast<uint32_t>((i ^ swz) * 16), src + 16 * i);
   };
 
-  Cursor ci, cc;
+  Cursor<I> ci, cc;
   ci.init(p0, ppr);
   cc = ci;
 #pragma unroll
@@ -217,7 +227,7 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     ci.advance(stride, dr, dpc, ppr);
     cp_async_wait<kStages - 1>();
 
-    const int64_t r = cc.r, cb = 2 * cc.pc;
+    const I r = cc.r, cb = 2 * cc.pc;
     const bool has_b = cb + 1 < bpr;
     const uint8_t *buf = my_g + st * STAGE;
     float2 v[16];
@@ -272,9 +282,9 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     uint32_t wa[2], wb[2];
     bool ia, ib;
     if (ta < 7.5f && tb < 7.5f)
-      if4_pair<false, MODE>(v, c76, c67, wa, wb, ia, ib);
+      if4_pair<false, MODE>(v, c76, c67, nz, wa, wb, ia, ib);
     else
-      if4_pair<true, MODE>(v, c76, c67, wa, wb, ia, ib);
+      if4_pair<true, MODE>(v, c76, c67, nz, wa, wb, ia, ib);
     uint8_t *qp = q + r * (cols / 2) + cb * 8;
     const uint32_t ba = sa | (ia ? 0x80u : 0u), bb = sb | (ib ? 0x80u : 0u);
     if (has_b) {
@@ -289,11 +299,16 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     }
     if (SWZ) {
       // (cb, cb + 1) are adjacent bytes of one 4-column group (cb even, and
-      // bpr % 4 == 0 gives every block a partner)
-      const int64_t tile = (r >> 7) * (bpr >> 2) + (cb >> 2);
-      const int64_t o = tile * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (cb & 3);
-      sf[o] = static_cast<uint8_t>(ba);
-      sf[o + 1] = static_cast<uint8_t>(bb);
+      // bpr % 4 == 0 gives every block a partner): one 2-byte store when the
+      // scale matrix starts on an even address (the offset o is even)
+      const I tile = (r >> 7) * (bpr >> 2) + (cb >> 2);
+      const I o = tile * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (cb & 3);
+      if (sf_even) {
+        *reinterpret_cast<uint16_t *>(sf + o) = static_cast<uint16_t>(ba | (bb << 8));
+      } else {
+        sf[o] = static_cast<uint8_t>(ba);
+        sf[o + 1] = static_cast<uint8_t>(bb);
+      }
     } else {
       sf[r * bpr + cb] = static_cast<uint8_t>(ba);
       if (has_b) sf[r * bpr + cb + 1] = static_cast<uint8_t>(bb);
@@ -303,11 +318,11 @@ if4_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
   cp_async_wait<0>();
 }
 
-template <typename T, bool SWZ, int MODE>
-cudaError_t launch_t(const T *x, int64_t rows, int64_t cols, int64_t ld, const float *amax,
+template <typename T, bool SWZ, int MODE, typename I>
+cudaError_t launch_i(const T *x, int64_t rows, int64_t cols, int64_t ld, const float *amax,
                      float *s_dec_out, uint8_t *q, uint8_t *sf, const Launch &L) {
   constexpr int SMEM = kWarps * kStages * 32 * 32 * static_cast<int>(sizeof(T));
-  const void *kern = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE>);
+  const void *kern = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE, I>);
   static KernelSetup setup;
   int per_sm = 0;
   const cudaError_t e = kernel_setup(setup, kern, kThreads, SMEM, &per_sm);
@@ -316,9 +331,20 @@ cudaError_t launch_t(const T *x, int64_t rows, int64_t cols, int64_t ld, const f
   const int64_t want = (npairs + kThreads - 1) / kThreads;
   const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
   const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-  if4_kernel<T, SWZ, MODE><<<grid, kThreads, SMEM, L.stream>>>(x, rows, cols, ld, amax, s_dec_out, q,
-                                                         sf);
+  // -0.0 as a run-time value (see if4_pair)
+  if4_kernel<T, SWZ, MODE, I><<<grid, kThreads, SMEM, L.stream>>>(x, rows, cols, ld, amax, s_dec_out, q,
+                                                            sf, -0.0f);
   return cudaGetLastError();
+}
+
+// 32-bit index arithmetic where every element offset and input offset fits
+template <typename T, bool SWZ, int MODE>
+cudaError_t launch_t(const T *x, int64_t rows, int64_t cols, int64_t ld, const float *amax,
+                     float *s_dec_out, uint8_t *q, uint8_t *sf, const Launch &L) {
+  constexpr int64_t kLim = (int64_t{1} << 31) - (int64_t{1} << 24);
+  if (rows * ld < kLim && rows * cols < kLim)
+    return launch_i<T, SWZ, MODE, int32_t>(x, rows, cols, ld, amax, s_dec_out, q, sf, L);
+  return launch_i<T, SWZ, MODE, int64_t>(x, rows, cols, ld, amax, s_dec_out, q, sf, L);
 }
 
 template <typename T, int MODE>

@@ -82,19 +82,21 @@ __device__ __forceinline__ float block_absmax(const uint4 (&u)[BLK * sizeof(T) /
 }
 
 // 16 values scaled by f, stochastic rounding with the bits of one Philox call
-// per 8 values: calls g0 and g0 + 1
+// per 8 values: calls g0 and g0 + 1 (the high counter word g_hi)
 __device__ __forceinline__ void encode_sr16(const float (&v)[16], float f, const PhiloxKey &K,
-                                            uint64_t g0, uint32_t (&w)[2]) {
+                                            uint32_t g0, uint32_t g_hi, uint32_t (&w)[2]) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint64_t g = g0 + h;
-    const U32x4 bits = philox(K, static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u);
+    const U32x4 bits = philox(K, g0 + h, g_hi, 0u, 0u);
     const uint32_t words[4] = {bits.x, bits.y, bits.z, bits.w};
     float t[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t z = (k & 1) ? sr_z_hi(words[k >> 1]) : sr_z_lo(words[k >> 1]);
-      t[k] = e2m1_sr_value(__fmul_rn(v[8 * h + k], f), z);
+    for (int k = 0; k < 8; k += 2) {
+      const float2 r = e2m1_sr_scaled2(
+          mul2(make_float2(v[8 * h + k], v[8 * h + k + 1]), make_float2(f, f)),
+          sr_x_lo(words[k >> 1]), sr_x_hi(words[k >> 1]));
+      t[k] = r.x;
+      t[k + 1] = r.y;
     }
     w[h] = e2m1x8(t);
   }
@@ -116,14 +118,17 @@ __device__ __forceinline__ void encode_rne(const float (&v)[BLK], float f,
   }
 }
 
-template <typename T, bool MX, bool SR, int QMAX>
+template <typename T, bool MX, bool SR, int QMAX, bool I32>
 __global__ void __launch_bounds__(kRowThreads)
-rowwise_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+rowwise_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
                const float *__restrict__ amax_ptr, int e8m0_mode, uint64_t seed,
                float *__restrict__ s_dec_out, uint8_t *__restrict__ q,
                uint8_t *__restrict__ sf, int scale_layout) {
   constexpr int BLK = MX ? 32 : 16;
   constexpr int NV = BLK * sizeof(T) / 16;   // uint4 per block
+  // 32-bit indices where the launcher has checked that they fit
+  using I = typename std::conditional<I32, int32_t, int64_t>::type;
+  const I rows = static_cast<I>(rows_), cols = static_cast<I>(cols_), ld = static_cast<I>(ld_);
   __shared__ float rtab[128];
   TensorScale ts{1.0f, 1.0f};
   if (!MX) {
@@ -133,23 +138,23 @@ rowwise_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     __syncthreads();
   }
   const PhiloxKey K(seed);
-  const int64_t bpr = cols / BLK, nblk = rows * bpr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kRowThreads;
-  int64_t b = static_cast<int64_t>(blockIdx.x) * kRowThreads + threadIdx.x;
+  const I bpr = cols / BLK, nblk = rows * bpr;
+  const I stride = static_cast<I>(gridDim.x) * kRowThreads;
+  I b = static_cast<I>(blockIdx.x) * kRowThreads + threadIdx.x;
   // two independent blocks per iteration keep 2 x BLK x sizeof(T) bytes in flight
   for (; b < nblk; b += 2 * stride) {
-    const int64_t b1 = b + stride;
+    const I b1 = b + stride;
     const bool two = b1 < nblk;
     uint4 u0[NV], u1[NV];
-    const int64_t r0 = b / bpr, cb0 = b - r0 * bpr;
-    const int64_t r1 = two ? b1 / bpr : r0, cb1 = two ? b1 - r1 * bpr : cb0;
+    const I r0 = b / bpr, cb0 = b - r0 * bpr;
+    const I r1 = two ? b1 / bpr : r0, cb1 = two ? b1 - r1 * bpr : cb0;
     load_block<T, BLK>(x + r0 * ld + cb0 * BLK, u0);
     load_block<T, BLK>(x + r1 * ld + cb1 * BLK, u1);
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
       if (s == 1 && !two) break;
       const uint4(&u)[NV] = s == 0 ? u0 : u1;
-      const int64_t r = s == 0 ? r0 : r1, cb = s == 0 ? cb0 : cb1;
+      const I r = s == 0 ? r0 : r1, cb = s == 0 ? cb0 : cb1;
       const float m = block_absmax<T, BLK>(u);
       uint32_t sbyte;
       float f;
@@ -165,8 +170,13 @@ rowwise_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
       uint8_t *qp = q + r * (cols / 2) + cb * (BLK / 2);
       if (BLK == 16) {
         uint32_t w[2];
-        if (SR) encode_sr16(*reinterpret_cast<const float(*)[16]>(v), f, K,
-                            static_cast<uint64_t>(r * cols + cb * 16) / 8, w);
+        if (SR) {
+          // Philox call (r cols + c) / 8; with fewer than 2^35 elements the
+          // counter's high word is 0
+          const uint64_t g0 = static_cast<uint64_t>(r * cols + cb * 16) / 8;
+          encode_sr16(*reinterpret_cast<const float(*)[16]>(v), f, K, static_cast<uint32_t>(g0),
+                      I32 ? 0u : static_cast<uint32_t>(g0 >> 32), w);
+        }
         else encode_rne<16>(*reinterpret_cast<const float(*)[16]>(v), f,
                             *reinterpret_cast<uint32_t(*)[2]>(w));
         *reinterpret_cast<uint2 *>(qp) = make_uint2(w[0], w[1]);
@@ -176,7 +186,7 @@ rowwise_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                        *reinterpret_cast<uint32_t(*)[4]>(w));
         *reinterpret_cast<uint4 *>(qp) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      sf[scale_offset(r, cb, bpr, scale_layout)] = static_cast<uint8_t>(sbyte);
+      sf[scale_offset_t<I>(r, cb, bpr, scale_layout)] = static_cast<uint8_t>(sbyte);
     }
   }
 }
@@ -254,23 +264,26 @@ __device__ __forceinline__ uint32_t block_scale(float m, const TensorScale &ts, 
 constexpr int kRCTileBytes = 64 * 128;            // one warp tile: 64 rows x 128 bytes
 constexpr int kRCSmem = (kRCThreads / 32) * 2 * kRCTileBytes;
 
-template <typename T, bool MX, bool SR, int QMAX>
+template <typename T, bool MX, bool SR, int QMAX, bool I32>
 __global__ void __launch_bounds__(kRCThreads, SR ? 2 : 3)
-rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, unsigned layouts,
+rowcol_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_, unsigned layouts,
               const float *__restrict__ amax_ptr, int e8m0_mode, uint64_t seed,
               float *__restrict__ s_dec_out, uint8_t *__restrict__ q_row,
               uint8_t *__restrict__ sf_row, uint8_t *__restrict__ q_col,
               uint8_t *__restrict__ sf_col, int scale_layout) {
   using G = RCGeom<T, MX>;
   constexpr int CPT = G::CPT, BLK = G::BLK, GR = G::GR;
+  // 32-bit indices where the launcher has checked that they fit
+  using I = typename std::conditional<I32, int32_t, int64_t>::type;
+  const I rows = static_cast<I>(rows_), cols = static_cast<I>(cols_), ld = static_cast<I>(ld_);
   __shared__ float rtab[128];
   const PhiloxKey K(seed);
   const bool do_row = (layouts & FP4Q_ROWWISE) != 0;
   const bool do_col = (layouts & FP4Q_COLWISE) != 0;
   const int lane = threadIdx.x & 31, cc = lane & 7, band = lane >> 3;
-  const int64_t tiles_c = (cols + G::WC - 1) / G::WC;
-  const int64_t ntiles = tiles_c * ((rows + G::WR - 1) / G::WR);
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kRCThreads / 32);
+  const I tiles_c = (cols + G::WC - 1) / G::WC;
+  const I ntiles = tiles_c * ((rows + G::WR - 1) / G::WR);
+  const I nwarps = static_cast<I>(gridDim.x) * (kRCThreads / 32);
   const bool swz = scale_layout == FP4Q_SCALE_SWIZZLED_128x4;
   extern __shared__ __align__(16) uint8_t rc_smem[];
   const int warp = threadIdx.x >> 5;
@@ -280,10 +293,10 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
   // lane L copies the 16-byte pieces L + 32 i: row (L + 32 i) / 8, chunk L % 8
   // row (L >> 3) + 4 i lies in the 16-row band i / 4 for every lane, and rows
   // is a multiple of 16, so the row bound is one test per band
-  auto issue = [&](const TileCursor &t, int st) {
-    const int64_t col = t.tc * G::WC + cc * CPT;
+  auto issue = [&](const TileCursorT<I> &t, int st) {
+    const I col = t.tc * G::WC + cc * CPT;
     if (col >= cols) return;
-    const int64_t row0 = t.tt * G::WR;
+    const I row0 = t.tt * G::WR;
     const T *src = x + (row0 + (lane >> 3)) * ld + col;
     const uint32_t dst =
         stage_s + static_cast<uint32_t>(st * kRCTileBytes + (lane >> 3) * 128 + cc * 16);
@@ -294,9 +307,9 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
       src += 4 * ld;
     }
   };
-  const int64_t dtr = nwarps / tiles_c, dtc = nwarps - dtr * tiles_c;
-  TileCursor cur, nxt;                                    // this tile, the one being copied
-  cur.init(static_cast<int64_t>(blockIdx.x) * (kRCThreads / 32) + warp, tiles_c);
+  const I dtr = nwarps / tiles_c, dtc = nwarps - dtr * tiles_c;
+  TileCursorT<I> cur, nxt;                                    // this tile, the one being copied
+  cur.init(static_cast<I>(blockIdx.x) * (kRCThreads / 32) + warp, tiles_c);
   nxt = cur;
   if (nxt.tile < ntiles) issue(nxt, 0);
   cp_async_commit();
@@ -317,8 +330,8 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
     nxt.advance(nwarps, dtr, dtc, tiles_c);
     cp_async_wait<1>();
     __syncwarp();
-    const int64_t tr = cur.tt, tc = cur.tc;
-    const int64_t r0 = tr * G::WR + band * 16, c0 = tc * G::WC + cc * CPT;
+    const I tr = cur.tt, tc = cur.tc;
+    const I r0 = tr * G::WR + band * 16, c0 = tc * G::WC + cc * CPT;
     const bool valid = r0 < rows && c0 < cols;
     // row k of this thread's 16: tb[8 * k] (rows outside the matrix are never
     // copied; their lanes' values only meet other outside lanes and are not stored)
@@ -380,26 +393,55 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
     {
       // rows r0..r0+15 of one block column: in the swizzled layout they are
       // 16 bytes apart (r0 is a multiple of 16), in the linear one cols/BLK
-      const int64_t step = swz ? 16 : cols / BLK;
-      uint8_t *srow = sf_row + scale_offset(r0, c0 / BLK, cols / BLK, scale_layout) + gi * step;
+      const I step = swz ? 16 : cols / BLK;
+      uint8_t *srow = sf_row + scale_offset_t<I>(r0, c0 / BLK, cols / BLK, scale_layout) + gi * step;
+      float mrow[RPL];
 #pragma unroll
       for (int i = 0; i < RPL; ++i) {
         float m = rmax[i * GR];
 #pragma unroll
         for (int g = 1; g < GR; ++g)
           if (g == gi) m = rmax[i * GR + g];
-        const uint32_t b = block_scale<T, MX, QMAX>(m, ts, rtab, e8m0_mode, own_f[i]);
-        if (valid && do_row) srow[i * GR * step] = static_cast<uint8_t>(b);
+        mrow[i] = m;
+      }
+      if (!MX && QMAX == 6 && RPL % 2 == 0) {
+#pragma unroll
+        for (int i = 0; i < RPL; i += 2) {
+          const uint32_t c2 = nvfp4_scale_code2(mrow[i], mrow[i + 1], ts.enc);
+          own_f[i] = rtab[c2 & 0xFFu];
+          own_f[i + 1] = rtab[c2 >> 8];
+          if (valid && do_row) {
+            srow[i * GR * step] = static_cast<uint8_t>(c2);
+            srow[(i + 1) * GR * step] = static_cast<uint8_t>(c2 >> 8);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+          const uint32_t b = block_scale<T, MX, QMAX>(mrow[i], ts, rtab, e8m0_mode, own_f[i]);
+          if (valid && do_row) srow[i * GR * step] = static_cast<uint8_t>(b);
+        }
       }
     }
 #pragma unroll
     for (int k = 0; k < 16; ++k)
       rf[k] = GR == 1 ? own_f[k] : __shfl_sync(0xFFFFFFFFu, own_f[k / GR], lane - gi + k % GR);
+    if (!MX && QMAX == 6) {
 #pragma unroll
-    for (int j = 0; j < CPT; ++j) cbyte[j] = block_scale<T, MX, QMAX>(cmax[j], ts, rtab, e8m0_mode, cf[j]);
+      for (int j = 0; j < CPT; j += 2) {
+        const uint32_t c2 = nvfp4_scale_code2(cmax[j], cmax[j + 1], ts.enc);
+        cbyte[j] = c2 & 0xFFu;
+        cbyte[j + 1] = c2 >> 8;
+        cf[j] = rtab[cbyte[j]];
+        cf[j + 1] = rtab[cbyte[j + 1]];
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) cbyte[j] = block_scale<T, MX, QMAX>(cmax[j], ts, rtab, e8m0_mode, cf[j]);
+    }
     if (valid && do_col && (!MX || (band & 1) == 0)) {
-      const int64_t base = scale_offset(c0, r0 / BLK, rows / BLK, scale_layout);
-      const int64_t step = swz ? 16 : rows / BLK;
+      const I base = scale_offset_t<I>(c0, r0 / BLK, rows / BLK, scale_layout);
+      const I step = swz ? 16 : rows / BLK;
 #pragma unroll
       for (int j = 0; j < CPT; ++j) sf_col[base + j * step] = static_cast<uint8_t>(cbyte[j]);
     }
@@ -421,13 +463,14 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
         for (int i = 0; i < 4; ++i) {
           const uint64_t idx = static_cast<uint64_t>((r0 + 4 * q4 + i) * cols + c0);
           const uint64_t gi = idx / 8;
-          const U32x4 bits = philox(K, static_cast<uint32_t>(gi), static_cast<uint32_t>(gi >> 32), 0u, 0u);
+          const U32x4 bits = philox(K, static_cast<uint32_t>(gi),
+                                    I32 ? 0u : static_cast<uint32_t>(gi >> 32), 0u, 0u);
           const uint32_t words[4] = {bits.x, bits.y, bits.z, bits.w};
 #pragma unroll
           for (int j = 0; j < CPT; ++j) {
             const int e = static_cast<int>(idx % 8) + j;
             const uint32_t wv = words[(e >> 1) & 3];
-            u[i][j] = (e & 1) ? sr_z_hi(wv) : sr_z_lo(wv);   // z of the 16-bit uniform
+            u[i][j] = (e & 1) ? sr_x_hi(wv) : sr_x_lo(wv);   // 64 times the 16-bit uniform
           }
         }
       }
@@ -440,8 +483,9 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
 #pragma unroll
           for (int j = 0; j < CPT; j += 2) {
             const float2 p = mul2(make_float2(v[i][j], v[i][j + 1]), make_float2(rf[k], rf[k]));
-            t[j] = SR ? e2m1_sr_value(p.x, u[i][j]) : p.x;
-            t[j + 1] = SR ? e2m1_sr_value(p.y, u[i][j + 1]) : p.y;
+            const float2 q = SR ? e2m1_sr_scaled2(p, u[i][j], u[i][j + 1]) : p;
+            t[j] = q.x;
+            t[j + 1] = q.y;
           }
           wr = CPT == 8 ? e2m1x8(t) : e2m1x4(t[0], t[1], t[2 % CPT], t[3 % CPT]);
           if (valid) {
@@ -461,7 +505,7 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
           if (SR) {
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              p[i] = make_float2(e2m1_sr_value(p[i].x, u[i][j]), e2m1_sr_value(p[i].y, u[i][j + 1]));
+              p[i] = e2m1_sr_scaled2(p[i], u[i][j], u[i][j + 1]);
           }
           const uint32_t h0 = e2m1x4(p[0].x, p[1].x, p[2].x, p[3].x);  // column j, rows 4q4..4q4+3
           const uint32_t h1 = e2m1x4(p[0].y, p[1].y, p[2].y, p[3].y);  // column j + 1
@@ -486,8 +530,8 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, u
 }
 
 
-template <typename T, bool MX, bool SR, int QMAX = 6>
-cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, unsigned layouts,
+template <typename T, bool MX, bool SR, int QMAX, bool I32>
+cudaError_t launch_typed2(const T *x, int64_t rows, int64_t cols, int64_t ld, unsigned layouts,
                          const float *amax, int e8m0_mode, uint64_t seed, float *s_dec_out,
                          uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col, uint8_t *sf_col,
                          int scale_layout, const Launch &L) {
@@ -497,18 +541,18 @@ cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, uns
     static KernelSetup setup;
     int per_sm = 0;
     const cudaError_t e = kernel_setup(
-        setup, reinterpret_cast<const void *>(rowwise_kernel<T, MX, SR, QMAX>), kRowThreads, 0,
+        setup, reinterpret_cast<const void *>(rowwise_kernel<T, MX, SR, QMAX, I32>), kRowThreads, 0,
         &per_sm);
     if (e != cudaSuccess) return e;
     const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
     const int64_t want = (nblk + 2 * kRowThreads - 1) / (2 * kRowThreads);
     const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-    rowwise_kernel<T, MX, SR, QMAX><<<grid, kRowThreads, 0, L.stream>>>(
+    rowwise_kernel<T, MX, SR, QMAX, I32><<<grid, kRowThreads, 0, L.stream>>>(
         x, rows, cols, ld, amax, e8m0_mode, seed, s_dec_out, q_row, sf_row, scale_layout);
   } else {
     using G = RCGeom<T, MX>;
     const int64_t ntiles = ((cols + G::WC - 1) / G::WC) * ((rows + G::WR - 1) / G::WR);
-    const void *kern = reinterpret_cast<const void *>(rowcol_kernel<T, MX, SR, QMAX>);
+    const void *kern = reinterpret_cast<const void *>(rowcol_kernel<T, MX, SR, QMAX, I32>);
     static KernelSetup setup;
     int per_sm = 0;
     const cudaError_t e = kernel_setup(setup, kern, kRCThreads, kRCSmem, &per_sm);
@@ -516,11 +560,28 @@ cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, uns
     const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
     const int64_t want = (ntiles + kRCThreads / 32 - 1) / (kRCThreads / 32);
     const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-    rowcol_kernel<T, MX, SR, QMAX><<<grid, kRCThreads, kRCSmem, L.stream>>>(
+    rowcol_kernel<T, MX, SR, QMAX, I32><<<grid, kRCThreads, kRCSmem, L.stream>>>(
         x, rows, cols, ld, layouts, amax, e8m0_mode, seed, s_dec_out, q_row, sf_row, q_col,
         sf_col, scale_layout);
   }
   return cudaGetLastError();
+}
+
+// 32-bit index arithmetic where every element and input offset fits (then
+// every stochastic-rounding counter (r * cols + c) / 8 fits in 32 bits too).
+template <typename T, bool MX, bool SR, int QMAX = 6>
+cudaError_t launch_typed(const T *x, int64_t rows, int64_t cols, int64_t ld, unsigned layouts,
+                         const float *amax, int e8m0_mode, uint64_t seed, float *s_dec_out,
+                         uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col, uint8_t *sf_col,
+                         int scale_layout, const Launch &L) {
+  constexpr int64_t kLim = (int64_t{1} << 31) - (int64_t{1} << 24);
+  if (rows * ld < kLim && rows * cols < kLim)
+    return launch_typed2<T, MX, SR, QMAX, true>(x, rows, cols, ld, layouts, amax, e8m0_mode, seed,
+                                               s_dec_out, q_row, sf_row, q_col, sf_col,
+                                               scale_layout, L);
+  return launch_typed2<T, MX, SR, QMAX, false>(x, rows, cols, ld, layouts, amax, e8m0_mode, seed,
+                                              s_dec_out, q_row, sf_row, q_col, sf_col,
+                                              scale_layout, L);
 }
 
 }  // namespace

@@ -14,21 +14,30 @@
 //     shared memory, so the next tile is in flight while this one computes
 //     (16-byte copies laid out so each warp write is a contiguous 512 bytes;
 //     warp barriers order the copy, the reads and the refill);
-//   * the sign flip is one LOP3 per packed word, the butterfly stages
-//     h = 1, 2, 4, 8 run in registers on f32x2 column pairs;
+//   * the sign flip rides on the BF16 unpacking (one multiply-add and one
+//     LOP3 per packed pair), the butterfly stages h = 1, 2, 4, 8 run in
+//     registers on f32x2 column pairs;
 //   * for n = 128 the stages h = 16, 32, 64 combine the eight groups of a
-//     column quad: butterflies between lanes g and g ^ 1, g ^ 2, g ^ 4 by
-//     shuffle, each output fma(own, +-1, partner) (an exact product, so one
-//     rounding of the sum or difference).  With stochastic rounding, where
-//     registers are short, the warp instead swaps values through an 8 KB
-//     shared buffer (XOR-swizzled so the write and the transposed read both
-//     spread over all banks), runs the three stages and swaps back;
-//   * block maxima are in-thread; stochastic rounding needs one Philox call
-//     per token per 8 columns, which two lanes share (each computes half of
-//     the tokens and passes the other lane its 64 bits by shuffle).  The ten
-//     Philox round keys and the 128 signs come in as kernel parameters.  The
-//     values are rounded stochastically in place (e2m1_sr_value) and then
-//     packed by the same round-to-nearest conversion as the RNE path;
+//     column quad: the warp swaps values through an 8 KB exchange buffer
+//     whose padding keeps both the write and the transposed read on eight
+//     distinct bank groups per eight lanes (every address a lane base plus a
+//     constant), runs the three stages in registers and writes the results
+//     back there;
+//   * the rest runs in two passes over the lane's two column pairs, which
+//     halves the values live at once: scaling by the transform's factor,
+//     block maxima (three-input maximum), block scales, stochastic rounding
+//     or RNE, packing and the stores of the pair's two code rows and scales.
+//     Lanes of odd column quads take their pairs in the opposite order, which
+//     keeps the pass reads of the exchange buffer conflict-free;
+//   * stochastic rounding needs one Philox call per token per 8 columns,
+//     which two lanes share (each computes half of the tokens and passes the
+//     other lane the words it needs by shuffle; the second pass's words wait
+//     in registers).  The ten Philox round keys and the 128 signs come in as
+//     kernel parameters, and the counters are 32-bit arithmetic wherever the
+//     tensor has fewer than 2^35 elements (the high counter word is then 0).
+//     The values are rounded stochastically in place (e2m1_sr_scaled2: the
+//     rounding by scaling with 2^-126) and then packed by the same
+//     round-to-nearest conversion as the RNE path;
 //   * dY^T codes leave as 8 lanes x 8 bytes = 64 contiguous bytes per column.
 #include "common.cuh"
 #include "launch.h"
@@ -78,20 +87,6 @@ __device__ __forceinline__ U32x4 philox_rk(const K &P, uint32_t c0, uint32_t c1)
   return U32x4{c0, c1, c2, c3};
 }
 
-template <int H>
-__device__ __forceinline__ void stage(float2 (&lo)[16], float2 (&hi)[16]) {
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-    if ((i & H) == 0) {
-      const float2 a = lo[i], b = lo[i + H];
-      lo[i] = add2(a, b);
-      lo[i + H] = sub2(a, b);
-      const float2 c = hi[i], d = hi[i + H];
-      hi[i] = add2(c, d);
-      hi[i + H] = sub2(c, d);
-    }
-}
-
 // cross-group stage on (8 groups x 2 offsets) values, index 2 * group + offset
 template <int H>
 __device__ __forceinline__ void xstage(float2 (&lo)[16], float2 (&hi)[16]) {
@@ -110,8 +105,62 @@ __device__ __forceinline__ void xstage(float2 (&lo)[16], float2 (&hi)[16]) {
       }
 }
 
-template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW>
-__global__ void __launch_bounds__(kThreads, (N == 16 && !SR && !ROW) ? 4 : 3)
+// stages h = 1, 2, 4, 8 of one column pair over 16 tokens
+__device__ __forceinline__ void stages16(float2 (&v)[16]) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if ((i & h) == 0) {
+        const float2 a = v[i], b = v[i + h];
+        v[i] = add2(a, b);
+        v[i + h] = sub2(a, b);
+      }
+}
+
+// The exchange buffer of the 128-point transform, in 16-byte units: (token t,
+// column quad q) sits at unit 4 t + q + t / 2 + t / 16, which grows with t
+// (so no two (t, q) share a unit) and whose two pad terms make both access
+// patterns hit eight distinct bank groups per eight lanes: the write of
+// tokens 16 g + k (fixed k, g = 0..7: the unit mod 8 is g + const) and the
+// transposed read of tokens 16 gg + 2 g + o (fixed gg, o: g + const again).
+// Every address is a lane base plus a constant: 73 g + q for the own tokens,
+// 9 g + q for the transposed ones.
+constexpr int kXUnits = 4 * 127 + 127 / 2 + 127 / 16 + 3 + 1;
+__host__ __device__ constexpr int xunit_own(int k) { return 4 * k + (k >> 1); }      // + 73 g + q
+__host__ __device__ constexpr int xunit_tr(int gg, int o) { return 73 * gg + 4 * o; }  // + 9 g + q
+
+// The Philox table of a warp tile: the four words of the call for token t
+// (0..127) and column octet o (0, 1) at byte (2 t + o) * 16 + (t / 16) * 16;
+// the pad puts the eight 16-byte writes of a quarter warp (tokens 16 g + i,
+// g = 0..7) on eight distinct bank groups.
+constexpr int kPTabBytes = (2 * 127 + 1) * 16 + (127 / 16) * 16 + 16;
+static_assert(kPTabBytes <= kUnits * 8, "the table fits in one BF16 input stage");
+__host__ __device__ constexpr int ptab_off(int t, int o) { return (2 * t + o) * 16 + (t >> 4) * 16; }
+
+// Coordinates (tile row tt, tile column tc) of a linear tile index over a grid
+// of tiles_c tile columns, stepped by a fixed number of tiles without
+// dividing; 32-bit.
+struct TileCursor32 {
+  int tile, tt, tc;
+  __device__ __forceinline__ void init(int t, int tiles_c) {
+    tile = t;
+    tt = t / tiles_c;
+    tc = t - tt * tiles_c;
+  }
+  __device__ __forceinline__ void advance(int step, int dtt, int dtc, int tiles_c) {
+    tile += step;
+    tt += dtt;
+    tc += dtc;
+    if (tc >= tiles_c) {
+      tc -= tiles_c;
+      ++tt;
+    }
+  }
+};
+
+template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW, bool I32>
+__global__ void __launch_bounds__(kThreads, ROW ? 3 : 4)
 rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
            const RhtParams P, const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
            unsigned *__restrict__ amax_out, uint8_t *__restrict__ q_t,
@@ -119,10 +168,8 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
            const RowArgs R) {
   constexpr int UB = 4 * sizeof(T);                       // bytes per input chunk
   constexpr int IN_BYTES = 2 * kUnits * UB;               // two stages
-  // with stochastic rounding the 128-point cross-group stages go through a
-  // shared exchange buffer (registers are short); otherwise through shuffles
-  constexpr bool XSMEM = N == 128 && SR;
-  constexpr int WARP_BYTES = IN_BYTES + (XSMEM ? 128 * 16 * 4 : 0);
+  constexpr bool PTAB_IN_STAGE = SR && N == 128 && !ROW;
+  constexpr int WARP_BYTES = IN_BYTES + (N == 128 ? kXUnits * 16 : 0) + ((SR && !PTAB_IN_STAGE) ? kPTabBytes : 0);
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float rtab[128];
   __shared__ float rtab_row[ROW ? 128 : 1];
@@ -130,6 +177,7 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   uint8_t *wbase = smem + warp * WARP_BYTES;
   const uint32_t in_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbase));
   float4 *xbuf = reinterpret_cast<float4 *>(wbase + IN_BYTES);
+  uint8_t *const ptab_own = wbase + IN_BYTES + (N == 128 ? kXUnits * 16 : 0);
   const int my_unit = unit_of(16 * g, cq);                // unit (16 g + k, cq) = my_unit + 4 k
 
   // signs of this lane's 16 tokens
@@ -143,12 +191,13 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   }
   const float cn = N == 16 ? 0.25f : __frsqrt_rn(128.0f);
 
-  const int64_t tiles_c = (cols + 15) / 16;
-  const int64_t ntiles = tiles_c * ((tokens + 127) / 128);
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
-  const int64_t dtt = nwarps / tiles_c, dtc = nwarps - dtt * tiles_c;
-  TileCursor cur, nxt;                                    // this tile, the one being copied
-  cur.init(static_cast<int64_t>(blockIdx.x) * kWarps + warp, tiles_c);
+  // tile counts fit in 32 bits (the launcher checks): a tile is 2048 elements
+  const int tiles_c = static_cast<int>((cols + 15) / 16);
+  const int ntiles = tiles_c * static_cast<int>((tokens + 127) / 128);
+  const int nwarps = static_cast<int>(gridDim.x) * kWarps;
+  const int dtt = nwarps / tiles_c, dtc = nwarps - dtt * tiles_c;
+  TileCursor32 cur, nxt;                                  // this tile, the one being copied
+  cur.init(static_cast<int>(blockIdx.x) * kWarps + warp, tiles_c);
   nxt = cur;
 
   // the copy of a tile is spread differently from the reads: lane L moves the
@@ -165,9 +214,9 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   constexpr int TPI = 32 / PPT;                           // tokens per copy step
   const int tok0 = lane / PPT, pc = lane % PPT;
   const uint32_t lane_dst = in_s + static_cast<uint32_t>(unit_of(tok0, pc * UPP) * UB);
-  auto issue = [&](const TileCursor &t, int st) {
-    const int64_t tbase = t.tt * 128;
-    const int64_t col = t.tc * 16 + pc * (16 / static_cast<int>(sizeof(T)));
+  auto issue = [&](const TileCursor32 &t, int st) {
+    const int64_t tbase = static_cast<int64_t>(t.tt) * 128;
+    const int64_t col = static_cast<int64_t>(t.tc) * 16 + pc * (16 / static_cast<int>(sizeof(T)));
     if (col >= cols) return;
     const T *src = dy + (tbase + tok0) * ld + col;
     const uint32_t dst = lane_dst + static_cast<uint32_t>(st * kUnits * UB);
@@ -198,6 +247,7 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
     if (blockIdx.x == 0 && threadIdx.x == 0 && R.s_dec_out) *R.s_dec_out = tsr.dec;
   }
   __syncthreads();
+  const int half = cq & 1;
   for (int st = 0; cur.tile < ntiles; cur.advance(nwarps, dtt, dtc, tiles_c), st ^= 1) {
     __syncwarp();   // every lane is done with stage st ^ 1 (last tile) before it is refilled
     if (nxt.tile < ntiles) issue(nxt, st ^ 1);
@@ -207,72 +257,90 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
     __syncwarp();
     // a column quad is all-in or all-out (cols % 8 == 0); a 16-token group
     // likewise (tokens % 16 == 0); for n = 128 all groups of a tile are in
-    const int64_t t0 = cur.tt * 128 + 16 * g, c0 = cur.tc * 16 + 4 * cq;
+    const int64_t t0 = static_cast<int64_t>(cur.tt) * 128 + 16 * g;
+    const int64_t c0 = static_cast<int64_t>(cur.tc) * 16 + 4 * cq;
     const bool valid = c0 < cols && t0 < tokens;
-
-    // ---- sign flip and stages h = 1, 2, 4, 8 ----------------------------------
-    float2 lo[16], hi[16];     // columns (c0, c0+1) and (c0+2, c0+3) per token
     const uint8_t *ib = wbase + (st * kUnits + my_unit) * UB;
+    // The tile's stochastic-rounding bits: element (t, c) draws from Philox
+    // call (t cols + c) / 8, one call per token and column octet, 256 per
+    // tile.  This lane computes tokens 16 g + 8 (cq & 1) + i of octet cq / 2
+    // and stores the four words of each in the warp's table; the passes read
+    // back the words of their own columns.  For n = 128 the table sits in the
+    // input stage this tile has finished reading (written after the
+    // transform, so that no transformed values are live meanwhile).
+    uint8_t *const ptab = PTAB_IN_STAGE ? wbase + st * kUnits * UB : ptab_own;
+    auto philox_phase = [&]() {
+      const int o = cq >> 1, tb = 16 * g + 8 * half;
+      const int64_t orow = (static_cast<int64_t>(cur.tt) * 128 + tb) * cols +
+                           static_cast<int64_t>(cur.tc) * 16 + 8 * o;
+      const uint32_t rstep = static_cast<uint32_t>(cols / 8);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      // 0 or 0xFFFFFFFF: token k's sign
-      const uint32_t m = static_cast<uint32_t>(static_cast<int32_t>(signs << (31 - k)) >> 31);
-      if (sizeof(T) == 2) {
-        uint2 w = valid ? *reinterpret_cast<const uint2 *>(ib + 4 * k * UB) : make_uint2(0u, 0u);
-        w.x ^= m & 0x80008000u;
-        w.y ^= m & 0x80008000u;
-        lo[k] = make_float2(bf16_lo(w.x), bf16_hi(w.x));
-        hi[k] = make_float2(bf16_lo(w.y), bf16_hi(w.y));
-      } else {
-        uint4 w = valid ? *reinterpret_cast<const uint4 *>(ib + 4 * k * UB)
-                        : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t s = m & 0x80000000u;
-        lo[k] = make_float2(__uint_as_float(w.x ^ s), __uint_as_float(w.y ^ s));
-        hi[k] = make_float2(__uint_as_float(w.z ^ s), __uint_as_float(w.w ^ s));
-      }
-    }
-    stage<1>(lo, hi);
-    stage<2>(lo, hi);
-    stage<4>(lo, hi);
-    stage<8>(lo, hi);
-
-    if (N == 128 && !XSMEM) {
-      // ---- stages h = 16, 32, 64 across the eight groups ------------------------
-      // token 16 g + k meets token 16 (g ^ m) + k, m = 1, 2, 4: the lane with
-      // bit m of g clear keeps RN(a + b), its partner RN(a - b); both are
-      // fma(own, +-1, partner), whose product is exact
-#pragma unroll
-      for (int sgi = 0; sgi < 3; ++sgi) {
-        const int m = 1 << sgi;
-        const float sg = (g & m) ? -1.0f : 1.0f;
-        const float2 sg2 = make_float2(sg, sg);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float2 pl = make_float2(__shfl_xor_sync(0xFFFFFFFFu, lo[k].x, m),
-                                        __shfl_xor_sync(0xFFFFFFFFu, lo[k].y, m));
-          const float2 ph = make_float2(__shfl_xor_sync(0xFFFFFFFFu, hi[k].x, m),
-                                        __shfl_xor_sync(0xFFFFFFFFu, hi[k].y, m));
-          lo[k] = fma2(lo[k], sg2, pl);
-          hi[k] = fma2(hi[k], sg2, ph);
+      for (int i = 0; i < 8; ++i) {
+        U32x4 b;
+        if (I32) {
+          b = philox_rk(P, static_cast<uint32_t>(orow / 8) + static_cast<uint32_t>(i) * rstep, 0u);
+        } else {
+          const uint64_t gidx = static_cast<uint64_t>(orow / 8) + static_cast<uint64_t>(i) * rstep;
+          b = philox_rk(P, static_cast<uint32_t>(gidx), static_cast<uint32_t>(gidx >> 32));
         }
+        *reinterpret_cast<uint4 *>(ptab + ptab_off(tb + i, o)) = make_uint4(b.x, b.y, b.z, b.w);
       }
-    }
-    if (N == 128 && XSMEM) {
-      // ---- stages h = 16, 32, 64 across the eight groups ------------------------
-      // the 16-byte chunk of (token t, quad q) is 4t + q with its low three
-      // bits XORed with (t/16 ^ t/2) mod 8; s = q ^ g is the lane's part of it
-      const int s = cq ^ g;
+      __syncwarp();
+    };
+    if (SR && !PTAB_IN_STAGE) philox_phase();
+    // token k's sign as a mask for the BF16 / FP32 sign bits
+    auto sign_of = [&](int k) -> uint32_t {
+      return static_cast<uint32_t>(static_cast<int32_t>(signs << (31 - k)) >> 31) & 0x80000000u;
+    };
+    // sign-flipped FP32 values of a raw column pair: for BF16 the low value is
+    // w * 2^16 + s (adding the sign bit flips it), the high one
+    // (w & 0xFFFF0000) ^ s -- one multiply-add and one LOP3 per pair
+    auto unpack_bf16 = [](uint32_t w, uint32_t sg) -> float2 {
+      return make_float2(__uint_as_float(w * 65536u + sg), __uint_as_float((w & 0xFFFF0000u) ^ sg));
+    };
+    auto unpack_f32 = [](uint2 w, uint32_t sg) -> float2 {
+      return make_float2(__uint_as_float(w.x ^ sg), __uint_as_float(w.y ^ sg));
+    };
+
+    // The lane works on its four columns as two column pairs, one per pass.
+    // For n = 128 the order is lane-dependent (pair half in pass 0, pair
+    // half ^ 1 in pass 1), which keeps the pass reads of the exchange buffer
+    // on distinct banks; for n = 16 every lane takes pair 0 first.
+    uint32_t raw1[sizeof(T) == 2 ? 16 : 1];   // BF16: the pass-1 pair, still packed
+    float2 *xb2 = reinterpret_cast<float2 *>(xbuf) + 2 * (73 * g + cq);
+    if (N == 128) {
+      // ---- the whole 128-point transform on all four columns --------------------
+      float2 lo[16], hi[16];
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
-        const int ck = (4 * (k & 1)) ^ ((k >> 1) & 7);
-        xbuf[64 * g + 8 * (k >> 1) + (s ^ ck)] = make_float4(lo[k].x, lo[k].y, hi[k].x, hi[k].y);
+        const uint32_t sg = sign_of(k);
+        // (a lane outside the matrix reads stale shared memory: it shares no
+        // values with lanes inside, and its results are never stored)
+        if (sizeof(T) == 2) {
+          const uint2 w = *reinterpret_cast<const uint2 *>(ib + 4 * k * UB);
+          lo[k] = unpack_bf16(w.x, sg);
+          hi[k] = unpack_bf16(w.y, sg);
+        } else {
+          const uint4 w = *reinterpret_cast<const uint4 *>(ib + 4 * k * UB);
+          lo[k] = unpack_f32(make_uint2(w.x, w.y), sg);
+          hi[k] = unpack_f32(make_uint2(w.z, w.w), sg);
+        }
       }
+      stages16(lo);
+      stages16(hi);
+      // stages h = 16, 32, 64 across the eight groups: swap through the
+      // exchange buffer so that a lane holds tokens 16 gg + 2 g + o of all
+      // eight groups gg, run the stages, and write the results back there
+      float4 *xw = xbuf + (73 * g + cq), *xr = xbuf + (9 * g + cq);
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        xw[xunit_own(k)] = make_float4(lo[k].x, lo[k].y, hi[k].x, hi[k].y);
       __syncwarp();
 #pragma unroll
       for (int gg = 0; gg < 8; ++gg)
 #pragma unroll
         for (int o = 0; o < 2; ++o) {
-          const float4 c = xbuf[64 * gg + 8 * g + (s ^ ((4 * o) ^ gg))];
+          const float4 c = xr[xunit_tr(gg, o)];
           lo[2 * gg + o] = make_float2(c.x, c.y);
           hi[2 * gg + o] = make_float2(c.z, c.w);
         }
@@ -284,116 +352,98 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
 #pragma unroll
         for (int o = 0; o < 2; ++o) {
           const int i = 2 * gg + o;
-          xbuf[64 * gg + 8 * g + (s ^ ((4 * o) ^ gg))] =
-              make_float4(lo[i].x, lo[i].y, hi[i].x, hi[i].y);
+          xr[xunit_tr(gg, o)] = make_float4(lo[i].x, lo[i].y, hi[i].x, hi[i].y);
         }
       __syncwarp();
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int ck = (4 * (k & 1)) ^ ((k >> 1) & 7);
-        const float4 c = xbuf[64 * g + 8 * (k >> 1) + (s ^ ck)];
-        lo[k] = make_float2(c.x, c.y);
-        hi[k] = make_float2(c.z, c.w);
-      }
-      __syncwarp();
-    }
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      lo[k] = mul2(lo[k], make_float2(cn, cn));
-      hi[k] = mul2(hi[k], make_float2(cn, cn));
+      if (PTAB_IN_STAGE) philox_phase();   // the stage's raw values are all read
     }
 
-    // ---- block maxima (16 tokens of each column) ------------------------------
-    float m[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    // ---- two passes over the column pairs ---------------------------------------
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      m[0] = fmaxf(m[0], fabsf(lo[k].x));
-      m[1] = fmaxf(m[1], fabsf(lo[k].y));
-      m[2] = fmaxf(m[2], fabsf(hi[k].x));
-      m[3] = fmaxf(m[3], fabsf(hi[k].y));
-    }
-    if (AMAX_ONLY) {
-      if (valid)
-        amax_bits = max(amax_bits, __float_as_uint(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]))));
-      continue;
-    }
-    if (rht_out && valid) {
+    for (int p = 0; p < 2; ++p) {
+      const int pp = N == 128 ? p ^ half : p;  // the column pair of this pass
+      float2 v[16];
+      if (N == 128) {
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        *reinterpret_cast<float4 *>(rht_out + (t0 + k) * cols + c0) =
-            make_float4(lo[k].x, lo[k].y, hi[k].x, hi[k].y);
-    }
-    uint32_t sbyte[4];
-    float f[4];
+        for (int k = 0; k < 16; ++k) v[k] = xb2[2 * xunit_own(k) + pp];
+        __syncwarp();   // the exchange buffer is rewritten by the next tile
+      } else {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      sbyte[j] = nvfp4_scale_code(m[j], ts.enc);
-      f[j] = rtab[sbyte[j]];
-    }
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      lo[k] = mul2(lo[k], make_float2(f[0], f[1]));
-      hi[k] = mul2(hi[k], make_float2(f[2], f[3]));
-    }
-
-    // ---- encode -----------------------------------------------------------------
-    uint32_t w[4][2];
-    if (SR) {
-      // element (t, c) draws from the Philox call (t * cols + c) / 8, covering
-      // this lane's quad and its neighbour's (lane ^ 8): the even quad computes
-      // tokens 0..7, the odd one 8..15, and each sends the other its half.
-      // The values are rounded in place; the RNE packing below encodes them.
-      const int half = cq & 1;
-      const uint64_t row0 = (static_cast<uint64_t>(t0) * static_cast<uint64_t>(cols) +
-                             static_cast<uint64_t>(c0 - 4 * half)) / 8;
-      const uint64_t rstep = static_cast<uint64_t>(cols) / 8;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint64_t gidx = row0 + static_cast<uint64_t>(i + 8 * half) * rstep;
-        const U32x4 b = philox_rk(P, static_cast<uint32_t>(gidx), static_cast<uint32_t>(gidx >> 32));
-        // words 0,1 serve the even quad (columns 0-3), words 2,3 the odd quad
-        const uint32_t keep0 = half ? b.z : b.x, keep1 = half ? b.w : b.y;
-        const uint32_t send0 = half ? b.x : b.z, send1 = half ? b.y : b.w;
-        const uint32_t got0 = __shfl_xor_sync(0xFFFFFFFFu, send0, 8);
-        const uint32_t got1 = __shfl_xor_sync(0xFFFFFFFFu, send1, 8);
-        // this lane computed token i + 8 half, the partner token i + 8 (1 - half)
-        const uint32_t ti0 = half ? got0 : keep0, ti1 = half ? got1 : keep1;
-        const uint32_t tj0 = half ? keep0 : got0, tj1 = half ? keep1 : got1;
-        lo[i].x = e2m1_sr_value(lo[i].x, sr_z_lo(ti0));
-        lo[i].y = e2m1_sr_value(lo[i].y, sr_z_hi(ti0));
-        hi[i].x = e2m1_sr_value(hi[i].x, sr_z_lo(ti1));
-        hi[i].y = e2m1_sr_value(hi[i].y, sr_z_hi(ti1));
-        lo[i + 8].x = e2m1_sr_value(lo[i + 8].x, sr_z_lo(tj0));
-        lo[i + 8].y = e2m1_sr_value(lo[i + 8].y, sr_z_hi(tj0));
-        hi[i + 8].x = e2m1_sr_value(hi[i + 8].x, sr_z_lo(tj1));
-        hi[i + 8].y = e2m1_sr_value(hi[i + 8].y, sr_z_hi(tj1));
+        for (int k = 0; k < 16; ++k) {
+          const uint32_t sg = sign_of(k);
+          if (sizeof(T) == 2) {
+            uint32_t w;
+            if (p == 0) {
+              const uint2 u = *reinterpret_cast<const uint2 *>(ib + 4 * k * UB);
+              w = u.x;
+              raw1[k] = u.y;
+            } else {
+              w = raw1[k];
+            }
+            v[k] = unpack_bf16(w, sg);
+          } else {
+            const uint2 u = *reinterpret_cast<const uint2 *>(ib + 4 * k * UB + 8 * pp);
+            v[k] = unpack_f32(u, sg);
+          }
+        }
+        stages16(v);
       }
-    }
-    {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) v[k] = mul2(v[k], make_float2(cn, cn));
+
+      // ---- block maxima (16 tokens of each column) ------------------------------
+      float ma, mb;
+      {
+        float a[16], b[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) { a[k] = v[k].x; b[k] = v[k].y; }
+        ma = absmax_n(a);
+        mb = absmax_n(b);
+      }
+      if (AMAX_ONLY) {
+        if (valid) amax_bits = max(amax_bits, __float_as_uint(fmaxf(ma, mb)));
+        continue;
+      }
+      const int64_t c = c0 + 2 * pp;
+      if (rht_out && valid) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          *reinterpret_cast<float2 *>(rht_out + (t0 + k) * cols + c) = v[k];
+      }
+      const uint32_t sa = nvfp4_scale_code(ma, ts.enc), sb = nvfp4_scale_code(mb, ts.enc);
+      const float2 f = make_float2(rtab[sa], rtab[sb]);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) v[k] = mul2(v[k], f);
+
+      if (SR) {
+        // words 0, 1 of a call serve the even quad's pairs, 2, 3 the odd quad's;
+        // token 16 g + k of octet o is at ptab_off(16 g, o) + 32 k
+        const uint8_t *pw = ptab + ptab_off(16 * g, cq >> 1) + 4 * (2 * (cq & 1) + pp);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint32_t w = *reinterpret_cast<const uint32_t *>(pw + 32 * k);
+          v[k] = e2m1_sr_scaled2(v[k], sr_x_lo(w), sr_x_hi(w));
+        }
+      }
+      uint32_t wa[2], wb[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        float a[8], b[8], c[8], d[8];
+        float a[8], b[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          a[k] = lo[8 * h + k].x; b[k] = lo[8 * h + k].y;
-          c[k] = hi[8 * h + k].x; d[k] = hi[8 * h + k].y;
-        }
-        w[0][h] = e2m1x8(a);
-        w[1][h] = e2m1x8(b);
-        w[2][h] = e2m1x8(c);
-        w[3][h] = e2m1x8(d);
+        for (int k = 0; k < 8; ++k) { a[k] = v[8 * h + k].x; b[k] = v[8 * h + k].y; }
+        wa[h] = e2m1x8(a);
+        wb[h] = e2m1x8(b);
       }
-    }
-    if (valid) {
-      // columns c0..c0+3 (c0 % 4 == 0): code rows tokens/2 bytes apart, scale
-      // rows 16 bytes apart in the swizzled layout, tokens/16 in the linear one
-      uint8_t *qp = q_t + c0 * (tokens / 2) + t0 / 2;
-      uint8_t *sp = sf_t + scale_offset(c0, t0 / 16, tokens / 16, scale_layout);
-      const int64_t sstep = scale_layout == FP4Q_SCALE_SWIZZLED_128x4 ? 16 : tokens / 16;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        *reinterpret_cast<uint2 *>(qp + j * (tokens / 2)) = make_uint2(w[j][0], w[j][1]);
-        sp[j * sstep] = static_cast<uint8_t>(sbyte[j]);
+      if (valid) {
+        // columns c, c + 1: code rows tokens/2 bytes apart, scale rows 16 bytes
+        // apart in the swizzled layout, tokens/16 in the linear one
+        uint8_t *qp = q_t + c * (tokens / 2) + t0 / 2;
+        uint8_t *sp = sf_t + scale_offset(c, t0 / 16, tokens / 16, scale_layout);
+        const int64_t sstep = scale_layout == FP4Q_SCALE_SWIZZLED_128x4 ? 16 : tokens / 16;
+        *reinterpret_cast<uint2 *>(qp) = make_uint2(wa[0], wa[1]);
+        *reinterpret_cast<uint2 *>(qp + tokens / 2) = make_uint2(wb[0], wb[1]);
+        sp[0] = static_cast<uint8_t>(sa);
+        sp[sstep] = static_cast<uint8_t>(sb);
       }
     }
     if (ROW) {
@@ -407,7 +457,8 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
       // 16-byte halves of their tokens in opposite order, so eight consecutive
       // lanes hit eight distinct bank groups.
       const uint8_t *sb0 = wbase + st * kUnits * UB;
-      const int64_t tile_t0 = cur.tt * 128, col0 = cur.tc * 16;
+      const int64_t tile_t0 = static_cast<int64_t>(cur.tt) * 128;
+      const int64_t col0 = static_cast<int64_t>(cur.tc) * 16;
       const bool cvalid = col0 < cols;
 #pragma unroll 1
       for (int j = 0; j < 4; ++j) {
@@ -436,9 +487,7 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
             x[4 * p + 2] = __uint_as_float(w.z); x[4 * p + 3] = __uint_as_float(w.w);
           }
         }
-        float m = 0.0f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) m = fmaxf(m, fabsf(x[k]));
+        const float m = absmax_n(x);
         const uint32_t sbr = nvfp4_scale_code(m, tsr.enc);
         const float f = rtab_row[sbr];
 #pragma unroll
@@ -453,11 +502,16 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
           for (int h = 0; h < 2; ++h) {
             const uint64_t gidx = (static_cast<uint64_t>(t) * static_cast<uint64_t>(cols) +
                                    static_cast<uint64_t>(col0 + 8 * h)) / 8;
-            const U32x4 b = philox_rk(R, static_cast<uint32_t>(gidx), static_cast<uint32_t>(gidx >> 32));
+            const U32x4 b = philox_rk(R, static_cast<uint32_t>(gidx),
+                                      I32 ? 0u : static_cast<uint32_t>(gidx >> 32));
             const uint32_t wd[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              x[8 * h + k] = e2m1_sr_value(x[8 * h + k], (k & 1) ? sr_z_hi(wd[k >> 1]) : sr_z_lo(wd[k >> 1]));
+            for (int k = 0; k < 8; k += 2) {
+              const float2 r = e2m1_sr_scaled2(make_float2(x[8 * h + k], x[8 * h + k + 1]),
+                                               sr_x_lo(wd[k >> 1]), sr_x_hi(wd[k >> 1]));
+              x[8 * h + k] = r.x;
+              x[8 * h + k + 1] = r.y;
+            }
           }
         }
         float lo8[8], hi8[8];
@@ -526,27 +580,45 @@ RowArgs make_row_args(const float *amax, float *s_dec_out, uint8_t *q, uint8_t *
   return R;
 }
 
-template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW = false>
-cudaError_t launch_k(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint64_t seed,
-                     const float *amax, float *s_dec_out, unsigned *amax_out, uint8_t *q_t,
-                     uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L,
-                     const RowArgs &R = RowArgs{}) {
+template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW, bool I32>
+cudaError_t launch_k2(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint64_t seed,
+                      const float *amax, float *s_dec_out, unsigned *amax_out, uint8_t *q_t,
+                      uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L,
+                      const RowArgs &R) {
   constexpr int UB = 4 * sizeof(T);
-  constexpr int WARP_BYTES = 2 * kUnits * UB + ((N == 128 && SR) ? 128 * 16 * 4 : 0);
+  constexpr int WARP_BYTES = 2 * kUnits * UB + (N == 128 ? kXUnits * 16 : 0) +
+                             ((SR && !(N == 128 && !ROW)) ? kPTabBytes : 0);
   constexpr int SMEM = kWarps * WARP_BYTES;
-  const void *kern = reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY, ROW>);
+  const void *kern = reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY, ROW, I32>);
   static KernelSetup setup;
   int per_sm = 0;
   const cudaError_t e = kernel_setup(setup, kern, kThreads, SMEM, &per_sm);
   if (e != cudaSuccess) return e;
   const int64_t ntiles = ((cols + 15) / 16) * ((tokens + 127) / 128);
+  if (ntiles > INT32_MAX / 2) return cudaErrorInvalidValue;   // the kernel counts tiles in 32 bits
   const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
   const int64_t want = (ntiles + kWarps - 1) / kWarps;
   const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-  rht_kernel<T, N, SR, AMAX_ONLY, ROW><<<grid, kThreads, SMEM, L.stream>>>(
+  rht_kernel<T, N, SR, AMAX_ONLY, ROW, I32><<<grid, kThreads, SMEM, L.stream>>>(
       dy, tokens, cols, ld, make_params(seed), amax, s_dec_out, amax_out, q_t, sf_t, scale_layout,
       rht_out, R);
   return cudaGetLastError();
+}
+
+// Stochastic rounding draws Philox calls (t * cols + c) / 8: with fewer than
+// 2^35 elements every counter fits in 32 bits.
+template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW = false>
+cudaError_t launch_k(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint64_t seed,
+                     const float *amax, float *s_dec_out, unsigned *amax_out, uint8_t *q_t,
+                     uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L,
+                     const RowArgs &R = RowArgs{}) {
+  if (SR && tokens * cols < (int64_t{1} << 35))
+    return launch_k2<T, N, SR, AMAX_ONLY, ROW, true>(dy, tokens, cols, ld, seed, amax, s_dec_out,
+                                                    amax_out, q_t, sf_t, scale_layout, rht_out,
+                                                    L, R);
+  return launch_k2<T, N, SR, AMAX_ONLY, ROW, false>(dy, tokens, cols, ld, seed, amax, s_dec_out,
+                                                   amax_out, q_t, sf_t, scale_layout, rht_out, L,
+                                                   R);
 }
 
 template <typename T, int N>

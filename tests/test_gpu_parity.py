@@ -289,6 +289,23 @@ def test_if4_spread_and_swizzled(orc):
         assert_same(k, host(got[k]), want[k])
 
 
+@pytest.mark.parametrize("layout", [0, 1])
+def test_if4_scales_at_an_odd_address(orc, layout):
+    """The scale matrix may start anywhere (the ABI asks 16-byte alignment of
+    the codes only): the kernel's paired scale stores fall back to single
+    bytes when it starts on an odd address."""
+    x = randmat(256, 256, torch.bfloat16, seed=33)
+    n = fq.fp4q_scale_bytes(256, 256, 16, layout)
+    buf = torch.full((n + 2,), 0xAB, dtype=torch.uint8, device=DEV)
+    out = {"s_dec": torch.empty(1, dtype=torch.float32, device=DEV),
+           "q": torch.empty((256, 128), dtype=torch.uint8, device=DEV), "sf": buf[1:n + 1]}
+    got = fq.fp4q_quantize_if4(x.to(DEV), scale_layout=layout, out=out)
+    want = orc.quantize_if4(bits(x), scale_layout=layout)
+    for k in ("s_dec", "q", "sf"):
+        assert_same(k, host(got[k]), want[k])
+    assert int(buf[0].item()) == 0xAB and int(buf[n + 1].item()) == 0xAB
+
+
 # ------------------------------------------------------------------ dequant
 
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
