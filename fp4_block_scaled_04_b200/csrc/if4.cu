@@ -90,8 +90,10 @@ __device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float
                                          uint32_t (&wa)[2], uint32_t (&wb)[2], bool &int_a,
                                          bool &int_b) {
   // FP4 candidates and their differences, in element order
+  // (each candidate's squared errors are summed as soon as they exist, in
+  // element order, so no difference outlives its half-block)
   uint32_t fpa[2] = {0u, 0u}, fpb[2] = {0u, 0u};
-  float da[16], db[16];
+  float2 efp = make_float2(0.0f, 0.0f), eint = make_float2(0.0f, 0.0f);
   if (MODE == 1) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -101,10 +103,10 @@ __device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float
       fpa[h] = fp4_codes_diffs(ta, ea);
       fpb[h] = fp4_codes_diffs(tb, eb);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) { da[8 * h + k] = ea[k]; db[8 * h + k] = eb[k]; }
+      for (int k = 0; k < 8; ++k)
+        efp = fma2(make_float2(ea[k], eb[k]), make_float2(ea[k], eb[k]), efp);
     }
   }
-  float2 efp = make_float2(0.0f, 0.0f), eint = make_float2(0.0f, 0.0f);
   uint32_t ia[2] = {0u, 0u}, ib[2] = {0u, 0u};
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
@@ -122,7 +124,6 @@ __device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float
       const float2 kf = sub2(tm, make_float2(kMagic, kMagic));    // rint(t), exact
       const float2 hv = fma2(kf, make_float2(c67, c67), make_float2(nz, nz));
       const float2 dint = sub2(vk, hv);
-      efp = fma2(make_float2(da[k], db[k]), make_float2(da[k], db[k]), efp);
       eint = fma2(dint, dint, eint);
     }
     ia[h] += __float_as_uint(tm.x) << (4 * i);
@@ -165,7 +166,7 @@ struct Cursor {
 };
 
 template <typename T, bool SWZ, int MODE, typename I>
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kThreads, 5)
 if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
            const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
            uint8_t *__restrict__ q, uint8_t *__restrict__ sf, float nz) {
@@ -273,7 +274,8 @@ if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
         mb = fmaxf(mb, fabsf(v[k].y));
       }
     }
-    const uint32_t sa = nvfp4_scale_code(ma, ts.enc), sb = nvfp4_scale_code(mb, ts.enc);
+    const uint32_t sab = nvfp4_scale_code2(ma, mb, ts.enc);
+    const uint32_t sa = sab & 0xFFu, sb = sab >> 8;
     const float fa = rtab[sa], fb = rtab[sb];
 #pragma unroll
     for (int k = 0; k < 16; ++k) v[k] = mul2(v[k], make_float2(fa, fb));
