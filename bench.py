@@ -776,7 +776,8 @@ def main():
             avg_s = time_call(job.run, 1.0)
             gbs = job.bytes / avg_s / 1e9
             entry = {"workload": job.name, "bytes": job.bytes, "us": round(avg_s * 1e6, 2),
-                     "GB/s": round(gbs, 1), "pct_of_peak": round(100 * gbs / peak, 1)}
+                     "GB/s": round(gbs, 1), "pct_of_peak": round(100 * gbs / peak, 1),
+                     "dram_bytes": traffic_for(job.src, job.name)}
             if job.run_amax is not None:
                 entry["us_incl_amax"] = round(time_call(job.run_amax, 5.0) * 1e6, 2)
             extra.append(entry)
@@ -795,7 +796,8 @@ def main():
         entry = {"workload": job.name, "bytes": job.bytes,
                  "us": round(avg_s * 1e6, 2), "GB/s": round(gbs, 1),
                  "pct_of_peak": round(100 * gbs / peak, 1),
-                 "share": round(ms / total_ms, 4)}
+                 "share": round(ms / total_ms, 4),
+                 "dram_bytes": traffic_for(job.src, job.name)}
         if job.name in incl_amax:
             # the algorithmic bytes stay those of the call itself; the amax
             # pre-pass's re-read of the input is overhead, not work
