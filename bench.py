@@ -493,9 +493,11 @@ def torch_uint8():
     return torch.uint8
 
 
-def oracle_sample(rows_fraction: float, inputs=None):
+def oracle_sample(rows_fraction: float, inputs=None, parts=None):
     """Run the oracle over the first rows_fraction of every workload of the
-    suite; returns (algorithmic bytes of the sample, seconds, description)."""
+    suite; returns (algorithmic bytes of the sample, seconds, description).
+    If ``parts`` is a dict, each call's (bytes, seconds) is stored in it under
+    the call's workload name."""
     import numpy as np
     import torch
     import oracle as orc
@@ -509,47 +511,61 @@ def oracle_sample(rows_fraction: float, inputs=None):
     def rows_of(n, align):
         return max(align, int(n * rows_fraction) // align * align)
 
+    total = [0, 0.0]
+
+    def timed(name, nbytes, fn):
+        t0 = time.perf_counter()
+        out = fn()
+        sec = time.perf_counter() - t0
+        total[0] += nbytes
+        total[1] += sec
+        if parts is not None:
+            parts[name] = (nbytes, sec)
+        return out
+
     inputs = inputs or suite_inputs()
     xa, w, g, x5 = inputs["activation"], inputs["weight"], inputs["gradient"], inputs["if4"]
-    total_b, total_s = 0, 0.0
     ra = rows_of(xa.shape[0], 32)
     a = np.ascontiguousarray(bits(xa[:ra]))
     C = xa.shape[1]
-    t0 = time.perf_counter()
-    orc.quantize_nvfp4(a, layouts=3, scale_layout=orc.SCALE_SWIZZLED if ra % 128 == 0 else 0)
-    orc.quantize_mxfp4(a, layouts=3)
-    total_s += time.perf_counter() - t0
-    total_b += ra * C * 2 + 2 * (ra * C // 2) + 2 * (ra * C // 16) + 4
-    total_b += ra * C * 2 + 2 * (ra * C // 2) + 2 * (ra * C // 32)
+    sl = orc.SCALE_SWIZZLED if ra % 128 == 0 else 0
+    timed("activation nvfp4 row+col", ra * C * 2 + 2 * (ra * C // 2) + 2 * (ra * C // 16) + 4,
+          lambda: orc.quantize_nvfp4(a, layouts=3, scale_layout=sl))
+    timed("activation mxfp4 row+col", ra * C * 2 + 2 * (ra * C // 2) + 2 * (ra * C // 32),
+          lambda: orc.quantize_mxfp4(a, layouts=3))
     rw = rows_of(w.shape[0], 16)
     ww = np.ascontiguousarray(bits(w[:rw]))
     C = w.shape[1]
-    t0 = time.perf_counter()
-    orc.quantize_2d(ww)
-    total_s += time.perf_counter() - t0
-    total_b += rw * C * 4 + 2 * (rw * C // 2) + (rw // 16) * (C // 16) + 4
+    timed("weight 2d16x16 w+wt", rw * C * 4 + 2 * (rw * C // 2) + (rw // 16) * (C // 16) + 4,
+          lambda: orc.quantize_2d(ww))
     rg = rows_of(g.shape[0], 128)
     gg = np.ascontiguousarray(bits(g[:rg]))
     C = g.shape[1]
-    t0 = time.perf_counter()
     for n in (16, 128):
-        for rnd in (orc.SR, orc.RNE):
-            orc.quantize_rht(gg, n, round=rnd, seed=0)
-    total_s += time.perf_counter() - t0
-    total_b += 4 * (rg * C * 2 + rg * C // 2 + rg * C // 16 + 4)
+        for rnd, rname in ((orc.SR, "sr"), (orc.RNE, "rne")):
+            timed(f"gradient rht{n}+{rname}", rg * C * 2 + rg * C // 2 + rg * C // 16 + 4,
+                  lambda: orc.quantize_rht(gg, n, round=rnd, seed=0))
     r5 = rows_of(x5.shape[0], 16)
     xx = np.ascontiguousarray(bits(x5[:r5]))
     C = x5.shape[1]
-    t0 = time.perf_counter()
-    o = orc.quantize_if4(xx)
-    orc.dequantize(orc.FMT_IF4, o["q"], o["sf"], r5, C, s_dec=float(o["s_dec"][0]),
-                   out_dtype=orc.BF16)
-    total_s += time.perf_counter() - t0
-    total_b += 2 * (r5 * C * 2 + r5 * C // 2 + r5 * C // 16 + 4)
+    nb5 = r5 * C * 2 + r5 * C // 2 + r5 * C // 16 + 4
+    o = timed("if4 quantize", nb5, lambda: orc.quantize_if4(xx))
+    timed("if4 dequantize to bf16", nb5,
+          lambda: orc.dequantize(orc.FMT_IF4, o["q"], o["sf"], r5, C,
+                                 s_dec=float(o["s_dec"][0]), out_dtype=orc.BF16))
+    xs = inputs.get("small")
+    if xs is not None:                    # the 256x256 parity workload, whole
+        sm = np.ascontiguousarray(bits(xs))
+        Rs, Cs = xs.shape
+        osm = timed("small 256x256 nvfp4 quantize", Rs * Cs * 2 + Rs * Cs // 2 + Rs * Cs // 16 + 4,
+                    lambda: orc.quantize_nvfp4(sm))
+        timed("small 256x256 dequantize to fp32", Rs * Cs // 2 + Rs * Cs // 16 + 4 + Rs * Cs * 4,
+              lambda: orc.dequantize(orc.FMT_NVFP4, osm["q_row"], osm["sf_row"], Rs, Cs,
+                                     s_dec=float(osm["s_dec"][0])))
     desc = (f"oracle (plain C) on the first {rows_fraction:.4g} of the rows of every "
             f"workload of the suite: activation {ra} rows, weight {rw}, gradient {rg}, "
-            f"if4 {r5}")
-    return total_b, total_s, desc
+            f"if4 {r5}" + ("; and the whole 256x256 small workload" if xs is not None else ""))
+    return total[0], total[1], desc
 
 
 def host_info():
@@ -577,15 +593,22 @@ def oracle_baseline(fraction: float, inputs, runs: int = 3):
     import oracle as orc
     cores, model = host_info()
     os.environ.setdefault("OMP_NUM_THREADS", str(cores))
-    out = {}
+    out, per = {}, {}
     try:
         for mode in ("single", "all"):
             orc.use_openmp(mode == "all")
-            times, b, desc = [], 0, ""
+            times, b, desc, runs_parts = [], 0, "", []
             for _ in range(runs):
-                b, sec, desc = oracle_sample(fraction, inputs)
+                parts = {}
+                b, sec, desc = oracle_sample(fraction, inputs, parts)
                 times.append(sec)
+                runs_parts.append(parts)
             out[mode] = (b, statistics.median(times), desc)
+            for name in runs_parts[0]:
+                nb = runs_parts[0][name][0]
+                med = statistics.median(p[name][1] for p in runs_parts)
+                per.setdefault(name, {})["GB/s_1_core" if mode == "single" else "GB/s_all_cores"] = \
+                    round(nb / med / 1e9, 5)
     finally:
         orc.use_openmp(False)
     b1, s1, desc = out["single"]
@@ -596,7 +619,8 @@ def oracle_baseline(fraction: float, inputs, runs: int = 3):
             "seconds": round(sa, 3), "runs": runs, "statistic": "median",
             "host_cores": cores, "cpu_model": model,
             "single_thread": {"value": round(b1 / s1 / 1e9, 5), "unit": "GB/s", "cores": 1,
-                              "seconds": round(s1, 3)}}
+                              "seconds": round(s1, 3)},
+            "per_config": per}
 
 
 # ---------------------------------------------------------------------------
