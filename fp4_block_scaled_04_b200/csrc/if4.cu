@@ -20,9 +20,13 @@
 //         (exact round-half-even for |t| < 2^22; the sum's low bits hold k in
 //         two's complement); the clamp to [-7, 7] only matters when the
 //         block's largest |t| reaches 7.5, which is tested once per block.
-//         Eight nibbles are packed by multiply-adds: the sum of
-//         bits(t + 1.5 * 2^23) * 16^i minus a constant leaves k_i + 8 in
-//         nibble i, and XOR 0x88888888 turns that into k_i mod 16.
+//         IF4 packs four nibbles at a time as an exact float sum: the sum of
+//         k_i * 16^i (|sum| < 2^15, by f32x2 fused multiply-adds on the
+//         integers k_i) plus 8 * 4369 + 2^23 leaves k_i + 8 in nibble i of
+//         the low 16 bits; two such halves make a word, and XOR 0x88888888
+//         turns every k_i + 8 into k_i mod 16.  NVINT4, which has no k as a
+//         float, packs the same way in integers: the sum of
+//         bits(t + 1.5 * 2^23) * 16^i minus a constant.
 //
 // Memory: each warp streams tiles of 32 block pairs through a three-stage
 // cp.async buffer in shared memory (each lane copies and later reads only
@@ -108,6 +112,8 @@ __device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float
     }
   }
   uint32_t ia[2] = {0u, 0u}, ib[2] = {0u, 0u};
+  // IF4: k packed as exact float sums of k_i * 16^i over four elements
+  float2 pk[2][2];
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
     const int h = k >> 3, i = k & 7;
@@ -125,14 +131,27 @@ __device__ __forceinline__ void if4_pair(const float2 (&v)[16], float c76, float
       const float2 hv = fma2(kf, make_float2(c67, c67), make_float2(nz, nz));
       const float2 dint = sub2(vk, hv);
       eint = fma2(dint, dint, eint);
+      const int q = i >> 2, j = i & 3;
+      const float w16 = j == 0 ? 1.0f : j == 1 ? 16.0f : j == 2 ? 256.0f : 4096.0f;
+      pk[h][q] = j == 0 ? kf : fma2(kf, make_float2(w16, w16), pk[h][q]);
+    } else {
+      ia[h] += __float_as_uint(tm.x) << (4 * i);
+      ib[h] += __float_as_uint(tm.y) << (4 * i);
     }
-    ia[h] += __float_as_uint(tm.x) << (4 * i);
-    ib[h] += __float_as_uint(tm.y) << (4 * i);
   }
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    ia[h] = (ia[h] - kPackBias) ^ 0x88888888u;
-    ib[h] = (ib[h] - kPackBias) ^ 0x88888888u;
+    if (MODE == 1) {
+      // sum + 8 * 4369 + 2^23 is exact and leaves k_i + 8 in nibble i of the
+      // low 16 bits
+      const float2 lo = add2(pk[h][0], make_float2(8423560.0f, 8423560.0f));
+      const float2 hi = add2(pk[h][1], make_float2(8423560.0f, 8423560.0f));
+      ia[h] = __byte_perm(__float_as_uint(lo.x), __float_as_uint(hi.x), 0x5410) ^ 0x88888888u;
+      ib[h] = __byte_perm(__float_as_uint(lo.y), __float_as_uint(hi.y), 0x5410) ^ 0x88888888u;
+    } else {
+      ia[h] = (ia[h] - kPackBias) ^ 0x88888888u;
+      ib[h] = (ib[h] - kPackBias) ^ 0x88888888u;
+    }
   }
   int_a = MODE == 2 || eint.x < efp.x;
   int_b = MODE == 2 || eint.y < efp.y;
