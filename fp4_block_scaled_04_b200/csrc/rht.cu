@@ -30,9 +30,11 @@
 //     Lanes of odd column quads take their pairs in the opposite order, which
 //     keeps the pass reads of the exchange buffer conflict-free;
 //   * stochastic rounding needs one Philox call per token per 8 columns,
-//     which two lanes share (each computes half of the tokens and passes the
-//     other lane the words it needs by shuffle; the second pass's words wait
-//     in registers).  The ten Philox round keys and the 128 signs come in as
+//     256 per tile: each lane computes 8 of them and stores their four words
+//     in a per-warp table in shared memory, from which both passes read the
+//     words of their own columns (for n = 128 the table takes the input
+//     stage the tile has finished reading, so the warp's shared memory does
+//     not grow).  The ten Philox round keys and the 128 signs come in as
 //     kernel parameters, and the counters are 32-bit arithmetic wherever the
 //     tensor has fewer than 2^35 elements (the high counter word is then 0).
 //     The values are rounded stochastically in place (e2m1_sr_scaled2: the

@@ -16,6 +16,11 @@ that does almost no work. Together these split a kernel's time into:
   - ``rate``, the slope: the streaming rate once the kernel is running, in
     algorithmic bytes per second.
 
+For scale, a plain device-to-device copy (``Tensor.copy_``, the operation behind
+the measured HBM peak) is timed the same way at each benchmark workload's
+byte count: read plus write equal to the kernel's algorithmic bytes. It shows
+what the same fixed costs leave of the copy bandwidth at that size.
+
 The fit uses the sizes from half the benchmark's shape upward. There the time
 grows linearly with the bytes; smaller launches are still ramping up.
 """
@@ -92,6 +97,18 @@ def main(argv=None) -> int:
     out["tiny_launch_us"] = round(run(tiny), 2)
     del tiny
     print(json.dumps(out), flush=True)
+    for name, nbytes in (("activation 8192x4096 nvfp4 row+col", 104857604),
+                         ("gradient 8192x5120 rht", 107479044),
+                         ("weight 14336x4096 2d", 293830660),
+                         ("if4 16384x8192", 343932932)):
+        n = nbytes // 4                    # BF16 elements: n * 2 read + n * 2 written
+        src = torch.empty(n, dtype=torch.bfloat16, device=dev).normal_()
+        dst = torch.empty_like(src)
+        us = run(lambda: dst.copy_(src))
+        print(json.dumps({"copy_like": name, "bytes": 4 * n, "us": round(us, 2),
+                          "GB/s": round(4 * n / us / 1e3, 1)}), flush=True)
+        del src, dst
+        torch.cuda.empty_cache()
     for op in a.ops.split(","):
         rows, cols, bpe = SWEEP[op]
         pts = []
