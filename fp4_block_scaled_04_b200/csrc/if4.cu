@@ -173,18 +173,23 @@ struct Cursor {
     r = p0 / ppr;
     pc = p0 - r * ppr;
   }
+  // FIXED: the stride is a multiple of the pairs per row, so the lane's
+  // pair column never changes (dpc == 0) and only the row moves
+  template <bool FIXED>
   __device__ __forceinline__ void advance(I stride, I dr, I dpc, I ppr) {
     p += stride;
     r += dr;
-    pc += dpc;
-    if (pc >= ppr) {
-      pc -= ppr;
-      ++r;
+    if (!FIXED) {
+      pc += dpc;
+      if (pc >= ppr) {
+        pc -= ppr;
+        ++r;
+      }
     }
   }
 };
 
-template <typename T, bool SWZ, int MODE, typename I>
+template <typename T, bool SWZ, int MODE, typename I, bool FIXED>
 __global__ void __launch_bounds__(kThreads, 5)
 if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
            const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
@@ -231,7 +236,7 @@ if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
   for (int s = 0; s < kStages - 1; ++s) {
     issue(ci, s);
     cp_async_commit();
-    ci.advance(stride, dr, dpc, ppr);
+    ci.template advance<FIXED>(stride, dr, dpc, ppr);
   }
   // the tensor scale and the factor table are set up while the first tiles
   // are already in flight
@@ -244,7 +249,7 @@ if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
   for (int st = 0; cc.p < npairs; st = (st + 1 == kStages ? 0 : st + 1)) {
     issue(ci, st == 0 ? kStages - 1 : st - 1);
     cp_async_commit();
-    ci.advance(stride, dr, dpc, ppr);
+    ci.template advance<FIXED>(stride, dr, dpc, ppr);
     cp_async_wait<kStages - 1>();
 
     const I r = cc.r, cb = 2 * cc.pc;
@@ -334,7 +339,7 @@ if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
       sf[r * bpr + cb] = static_cast<uint8_t>(ba);
       if (has_b) sf[r * bpr + cb + 1] = static_cast<uint8_t>(bb);
     }
-    cc.advance(stride, dr, dpc, ppr);
+    cc.template advance<FIXED>(stride, dr, dpc, ppr);
   }
   cp_async_wait<0>();
 }
@@ -343,18 +348,35 @@ template <typename T, bool SWZ, int MODE, typename I>
 cudaError_t launch_i(const T *x, int64_t rows, int64_t cols, int64_t ld, const float *amax,
                      float *s_dec_out, uint8_t *q, uint8_t *sf, const Launch &L) {
   constexpr int SMEM = kWarps * kStages * 32 * 32 * static_cast<int>(sizeof(T));
-  const void *kern = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE, I>);
-  static KernelSetup setup;
-  int per_sm = 0;
-  const cudaError_t e = kernel_setup(setup, kern, kThreads, SMEM, &per_sm);
+  // both forms share one occupancy query (same registers and shared memory
+  // by construction: the fixed form only drops work)
+  const void *kern = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE, I, false>);
+  const void *kern_f = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE, I, true>);
+  static KernelSetup setup, setup_f;
+  int per_sm = 0, per_sm_f = 0;
+  cudaError_t e = kernel_setup(setup, kern, kThreads, SMEM, &per_sm);
   if (e != cudaSuccess) return e;
-  const int64_t npairs = rows * ((cols / 16 + 1) / 2);
+  e = kernel_setup(setup_f, kern_f, kThreads, SMEM, &per_sm_f);
+  if (e != cudaSuccess) return e;
+  const int64_t ppr = (cols / 16 + 1) / 2, npairs = rows * ppr;
   const int64_t want = (npairs + kThreads - 1) / kThreads;
-  const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
-  const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+  const int64_t cap = static_cast<int64_t>(per_sm < per_sm_f ? per_sm : per_sm_f) * L.num_sms;
+  int64_t grid = want < 1 ? 1 : (want > cap ? cap : want);
+  // a full grid a little smaller than the cap whose stride is a multiple of
+  // the pairs per row keeps every lane on one pair column
+  bool fixed = (grid * kThreads) % ppr == 0;
+  for (int64_t g = grid; !fixed && grid == cap && g > cap - cap / 8; --g)
+    if ((g * kThreads) % ppr == 0) {
+      grid = g;
+      fixed = true;
+    }
   // -0.0 as a run-time value (see if4_pair)
-  if4_kernel<T, SWZ, MODE, I><<<grid, kThreads, SMEM, L.stream>>>(x, rows, cols, ld, amax, s_dec_out, q,
-                                                            sf, -0.0f);
+  if (fixed)
+    if4_kernel<T, SWZ, MODE, I, true><<<static_cast<int>(grid), kThreads, SMEM, L.stream>>>(
+        x, rows, cols, ld, amax, s_dec_out, q, sf, -0.0f);
+  else
+    if4_kernel<T, SWZ, MODE, I, false><<<static_cast<int>(grid), kThreads, SMEM, L.stream>>>(
+        x, rows, cols, ld, amax, s_dec_out, q, sf, -0.0f);
   return cudaGetLastError();
 }
 

@@ -281,6 +281,20 @@ def test_if4(orc, dtype, shape):
         assert_same(k, host(got[k]), want[k])
 
 
+@pytest.mark.parametrize("shape,layout", [((256, 32288), 0), ((2048, 2048), 1)])
+def test_if4_lanes_walk_several_pairs(orc, shape, layout):
+    """Shapes with more pairs of blocks than the grid has lanes. With 32288
+    columns (1009 pairs per row, a prime that divides no full grid's stride)
+    a lane's pair column changes from one pair to the next. With 2048
+    columns the stride is a multiple of the pairs per row, so every lane
+    stays on one pair column."""
+    x = workloads.if4_blocks(seed=34, rows=shape[0], cols=shape[1])
+    got = fq.fp4q_quantize_if4(x.to(DEV), scale_layout=layout)
+    want = orc.quantize_if4(bits(x), scale_layout=layout)
+    for k in ("s_dec", "q", "sf"):
+        assert_same(k, host(got[k]), want[k])
+
+
 def test_if4_spread_and_swizzled(orc):
     x = randmat(256, 256, torch.bfloat16, seed=32)
     got = fq.fp4q_quantize_if4(x.to(DEV), scale_layout=fq.SCALE_SWIZZLED)
