@@ -11,7 +11,8 @@
 // The codes [rows, cols/2] and the output [rows, cols] are both dense, so the
 // kernel walks the flat element range in units of 8 elements (4 code bytes,
 // one 16-byte BF16 store), consecutive units on consecutive lanes, four
-// units per lane per step so that four loads are in flight.  With a linear
+// units per lane per step, and loads the next step's codes and scale bytes
+// before it decodes this step's, so that eight loads are in flight.  With a linear
 // 1x16 or 1x32 scale matrix the scale index is the flat element index / 16
 // (or / 32), so the walk needs no row and column; the swizzled and
 // 16x16-tile layouts carry (row, column) along with a fixed stride.
@@ -172,25 +173,19 @@ dequant_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ sf,
       c[j] = e - r[j] * cols;
     }
   }
-  for (I base = warp0 * NU * 32 + lane; base < total; base += wstride * NU * 32) {
-    uint32_t cw[NU], sb[NU];
+  // the codes and scale bytes of the lane's NU units of one step; the next
+  // step's are loaded before this step decodes, so the loads overlap the
+  // arithmetic (r, c: the units of the next step to load)
+  uint32_t cw[NU], sb[NU];
+  auto load = [&](I b, uint32_t (&w)[NU], uint32_t (&s8)[NU]) {
 #pragma unroll
     for (int j = 0; j < NU; ++j) {
-      const I u = base + 32 * j;
+      const I u = b + 32 * j;
       if (u < total) {
         const I si = FLAT ? (BLK == 32 ? (u >> 2) : (u >> 1))
                           : unit_scale<BLK, BROWS, SWZ, I>(r[j], c[j], cols);
-        cw[j] = __ldg(qw + u);
-        sb[j] = __ldg(sf + si);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < NU; ++j) {
-      const I u = base + 32 * j;
-      if (u < total) {
-        float2 v[4];
-        decode8<FMT>(cw[j], sb[j], s_dec, c67, v);
-        Store::put(y + static_cast<size_t>(u) * 8, v);
+        w[j] = __ldg(qw + u);
+        s8[j] = __ldg(sf + si);
       }
       if (!FLAT) {
         r[j] += dr;
@@ -200,6 +195,27 @@ dequant_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ sf,
           ++r[j];
         }
       }
+    }
+  };
+  const I step = wstride * NU * 32;
+  I base = warp0 * NU * 32 + lane;
+  if (base < total) load(base, cw, sb);
+  for (; base < total; base += step) {
+    uint32_t cn[NU], sn[NU];
+    if (base + step < total) load(base + step, cn, sn);
+#pragma unroll
+    for (int j = 0; j < NU; ++j) {
+      const I u = base + 32 * j;
+      if (u < total) {
+        float2 v[4];
+        decode8<FMT>(cw[j], sb[j], s_dec, c67, v);
+        Store::put(y + static_cast<size_t>(u) * 8, v);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NU; ++j) {
+      cw[j] = cn[j];
+      sb[j] = sn[j];
     }
   }
 }
