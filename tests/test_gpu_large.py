@@ -6,6 +6,8 @@ checks are the ones that hold at any size: the tensor amax against a planted
 maximum at the very last element, and sampled rows (first, second, middle,
 last) against the oracle run on those rows alone.  The row-wise formats are
 row-independent once the tensor amax is given, so that comparison is exact.
+The formats whose blocks span rows (row+col NVFP4 and MXFP4, 2D, the RHT
+along tokens) are compared on bands of whole blocks (first, middle, last).
 Round to nearest throughout (the stochastic-rounding bits depend on the
 global element index).
 """
@@ -89,3 +91,64 @@ def test_large_if(orc, big, fmt):
     assert_same("s_dec", host(out["s_dec"]), want["s_dec"])
     assert_same("q", sample(out["q"]), want["q"])
     assert_same("sf", sample(out["sf"].view(R, C // 16)), want["sf"])
+
+
+# Row bands for the formats whose blocks or tiles span rows: a band of whole
+# column blocks (16 rows; 32 for MXFP4; the transform's 16- or 128-token
+# groups) gives, on the oracle run on the band alone, the same column-wise
+# codes and scales as the whole tensor once the tensor amax is given.
+def bands(n):
+    return [0, (R // 2 // n) * n + n, R - n]
+
+
+def test_large_nvfp4_rowcol(orc, big):
+    x, amax = big
+    out = fq.fp4q_quantize_nvfp4(x, layouts=fq.ROWWISE | fq.COLWISE, amax=amax)
+    for r0 in bands(16):
+        want = orc.quantize_nvfp4(bits(x[r0:r0 + 16]), layouts=3, amax=PEAK)
+        assert_same("q_row", host(out["q_row"][r0:r0 + 16]), want["q_row"])
+        assert_same("sf_row", host(out["sf_row"].view(R, C // 16)[r0:r0 + 16]), want["sf_row"])
+        assert_same("q_col", host(out["q_col"][:, r0 // 2:r0 // 2 + 8]), want["q_col"])
+        assert_same("sf_col", host(out["sf_col"].view(C, R // 16)[:, r0 // 16:r0 // 16 + 1]),
+                    want["sf_col"])
+
+
+def test_large_mxfp4_rowcol(orc, big):
+    x, _ = big
+    out = fq.fp4q_quantize_mxfp4(x, layouts=fq.ROWWISE | fq.COLWISE)
+    for r0 in bands(32):
+        want = orc.quantize_mxfp4(bits(x[r0:r0 + 32]), layouts=3)
+        assert_same("q_row", host(out["q_row"][r0:r0 + 32]), want["q_row"])
+        assert_same("sf_row", host(out["sf_row"].view(R, C // 32)[r0:r0 + 32]), want["sf_row"])
+        assert_same("q_col", host(out["q_col"][:, r0 // 2:r0 // 2 + 16]), want["q_col"])
+        assert_same("sf_col", host(out["sf_col"].view(C, R // 32)[:, r0 // 32:r0 // 32 + 1]),
+                    want["sf_col"])
+
+
+def test_large_2d(orc, big):
+    x, amax = big
+    out = fq.fp4q_quantize_2d(x, amax=amax)
+    for r0 in bands(16):
+        want = orc.quantize_2d(bits(x[r0:r0 + 16]), amax=PEAK)
+        assert_same("q_w", host(out["q_w"][r0:r0 + 16]), want["q_w"])
+        assert_same("q_wt", host(out["q_wt"][:, r0 // 2:r0 // 2 + 8]), want["q_wt"])
+        assert_same("sf_tiles", host(out["sf_tiles"].view(R // 16, C // 16)[r0 // 16]),
+                    want["sf_tiles"])
+
+
+@pytest.mark.parametrize("n", [16, 128])
+def test_large_rht(orc, big, n):
+    """The transform works within 16- or 128-token groups and its signs repeat
+    per group, so a band of whole groups is transformed and quantized as in
+    the whole tensor; the transform's amax is given (any positive value is a
+    valid caller amax) so that the band needs no global reduction."""
+    x, _ = big
+    a = 16384.0
+    out = fq.fp4q_quantize_rht_sr(x, n, round=fq.RNE,
+                                  amax_rht=torch.tensor([a], dtype=torch.float32, device=DEV))
+    for r0 in bands(n):
+        want = orc.quantize_rht(bits(x[r0:r0 + n]), n, round=orc.RNE, amax_rht=a)
+        assert_same("s_dec", host(out["s_dec"]), want["s_dec"])
+        assert_same("q_t", host(out["q_t"][:, r0 // 2:r0 // 2 + n // 2]), want["q_t"])
+        assert_same("sf_t", host(out["sf_t"].view(C, R // 16)[:, r0 // 16:r0 // 16 + n // 16]),
+                    want["sf_t"])
