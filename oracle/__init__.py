@@ -93,6 +93,8 @@ def lib() -> ctypes.CDLL:
             "orc_amax": (F, [P, I, I64, I64, I64]),
             "orc_tensor_scales": (None, [F, P, P]),
             "orc_quantize_nvfp4": (I, [P, I, I64, I64, I64, U, I, U64, P, P, P, P, P, P, I]),
+            "orc_quantize_nvfp4_rows": (I, [P, I, I64, I64, I64, U, I, U64, P, P, P, P, P, P, I,
+                                            I64]),
             "orc_quantize_mxfp4": (I, [P, I, I64, I64, I64, U, I, P, P, P, P, I]),
             "orc_quantize_mxfp6": (I, [P, I, I64, I64, I64, I, I, P, P, I]),
             "orc_fp6_value": (F, [ctypes.c_uint8, I]),
@@ -101,6 +103,7 @@ def lib() -> ctypes.CDLL:
             "orc_rht_norm": (F, [I]),
             "orc_rht": (I, [P, I, I64, I64, I64, I, U64, P]),
             "orc_quantize_rht": (I, [P, I, I64, I64, I64, I, I, U64, P, P, P, P, I, P]),
+            "orc_quantize_rht_rows": (I, [P, I, I64, I64, I64, I, I, U64, P, P, P, P, I, P, I64]),
             "orc_if4_c76": (F, []),
             "orc_if4_c67": (F, []),
             "orc_quantize_if4": (I, [P, I, I64, I64, I64, P, P, P, P, I, I]),
@@ -275,7 +278,11 @@ def _amax_arg(a):
 
 
 def quantize_nvfp4(x: np.ndarray, layouts: int = ROWWISE, round: int = RNE, seed: int = 0,
-                   amax: float | None = None, scale_layout: int = SCALE_LINEAR) -> dict:
+                   amax: float | None = None, scale_layout: int = SCALE_LINEAR,
+                   row0: int = 0) -> dict:
+    """NVFP4 1x16.  row0 > 0: x is rows row0.. of a larger tensor with the same
+    columns (give its amax); the stochastic-rounding bits then use the whole
+    tensor's flat index."""
     x = np.ascontiguousarray(x)
     rows, cols = x.shape
     out = {"s_dec": np.zeros(1, np.float32)}
@@ -286,10 +293,11 @@ def quantize_nvfp4(x: np.ndarray, layouts: int = ROWWISE, round: int = RNE, seed
         out["q_col"] = np.zeros((cols, rows // 2), np.uint8)
         out["sf_col"] = np.zeros(scale_bytes(cols, rows // 16, scale_layout), np.uint8)
     keep, ap = _amax_arg(amax)
-    rc = lib().orc_quantize_nvfp4(_ptr(x), _dtype_code(x), rows, cols, cols, layouts, round,
-                                  seed, ap, _ptr(out["s_dec"]), _ptr(out.get("q_row")),
-                                  _ptr(out.get("sf_row")), _ptr(out.get("q_col")),
-                                  _ptr(out.get("sf_col")), scale_layout)
+    args = (_ptr(x), _dtype_code(x), rows, cols, cols, layouts, round, seed, ap,
+            _ptr(out["s_dec"]), _ptr(out.get("q_row")), _ptr(out.get("sf_row")),
+            _ptr(out.get("q_col")), _ptr(out.get("sf_col")), scale_layout)
+    rc = (lib().orc_quantize_nvfp4_rows(*args, row0) if row0 else
+          lib().orc_quantize_nvfp4(*args))
     if rc != 0:
         raise ValueError(f"oracle rejected shape {x.shape}")
     return out
@@ -405,7 +413,10 @@ def rht(dy: np.ndarray, n: int, seed: int = 0) -> np.ndarray:
 
 def quantize_rht(dy: np.ndarray, n: int, round: int = SR, seed: int = 0,
                  amax_rht: float | None = None, scale_layout: int = SCALE_LINEAR,
-                 want_rht: bool = False) -> dict:
+                 want_rht: bool = False, token0: int = 0) -> dict:
+    """RHT + column-wise NVFP4.  token0 > 0: dy is tokens token0.. (a multiple of
+    n) of a larger gradient with the same columns (give the transform's amax);
+    the stochastic-rounding bits then use the whole tensor's flat index."""
     dy = np.ascontiguousarray(dy)
     tokens, cols = dy.shape
     out = {"s_dec": np.zeros(1, np.float32),
@@ -414,9 +425,11 @@ def quantize_rht(dy: np.ndarray, n: int, round: int = SR, seed: int = 0,
     if want_rht:
         out["rht"] = np.zeros((tokens, cols), np.float32)
     keep, ap = _amax_arg(amax_rht)
-    rc = lib().orc_quantize_rht(_ptr(dy), _dtype_code(dy), tokens, cols, cols, n, round, seed,
-                                ap, _ptr(out["s_dec"]), _ptr(out["q_t"]), _ptr(out["sf_t"]),
-                                scale_layout, _ptr(out.get("rht")))
+    args = (_ptr(dy), _dtype_code(dy), tokens, cols, cols, n, round, seed, ap,
+            _ptr(out["s_dec"]), _ptr(out["q_t"]), _ptr(out["sf_t"]), scale_layout,
+            _ptr(out.get("rht")))
+    rc = (lib().orc_quantize_rht_rows(*args, token0) if token0 else
+          lib().orc_quantize_rht(*args))
     if rc != 0:
         raise ValueError("oracle rejected RHT arguments")
     return out

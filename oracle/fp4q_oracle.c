@@ -372,11 +372,13 @@ static void put_nibble(uint8_t *q, int64_t byte_index, int high, uint8_t code) {
   else q[byte_index] = (uint8_t)((q[byte_index] & 0xF0) | (code & 0xF));
 }
 
-/* 1x16 quantization with block grid maximum qmax (6: NVFP4, 4: 4/6). */
+/* 1x16 quantization with block grid maximum qmax (6: NVFP4, 4: 4/6).  x is */
+/* rows row0 .. row0 + rows - 1 of a tensor with cols columns (row0 = 0: the */
+/* whole tensor); only the SR bits see row0, through the flat index.        */
 static int quantize_1x16(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                          unsigned layouts, int round, uint64_t seed, const float *amax_in,
                          float *s_dec_out, uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col,
-                         uint8_t *sf_col, int scale_layout, float qmax) {
+                         uint8_t *sf_col, int scale_layout, float qmax, int64_t row0) {
   if ((layouts & ORC_ROWWISE) && cols % 16 != 0) return 1;
   if ((layouts & ORC_COLWISE) && rows % 16 != 0) return 1;
   float amax = amax_in ? *amax_in : orc_amax(x, dtype, rows, cols, ld);
@@ -399,7 +401,7 @@ static int quantize_1x16(const void *x, int dtype, int64_t rows, int64_t cols, i
         for (int k = 0; k < 16; ++k) {
           int64_t c = b * 16 + k;
           float v = load_elem(x, dtype, ld, r, c) * rf;
-          uint8_t code = encode_elem(v, round, seed, (uint64_t)(r * cols + c));
+          uint8_t code = encode_elem(v, round, seed, (uint64_t)((row0 + r) * cols + c));
           put_nibble(q_row, r * (cols / 2) + c / 2, (int)(c & 1), code);
         }
       }
@@ -419,7 +421,7 @@ static int quantize_1x16(const void *x, int dtype, int64_t rows, int64_t cols, i
         for (int k = 0; k < 16; ++k) {
           int64_t r = b * 16 + k;
           float v = load_elem(x, dtype, ld, r, c) * rf;
-          uint8_t code = encode_elem(v, round, seed, (uint64_t)(r * cols + c));
+          uint8_t code = encode_elem(v, round, seed, (uint64_t)((row0 + r) * cols + c));
           put_nibble(q_col, c * (rows / 2) + r / 2, (int)(r & 1), code);
         }
       }
@@ -432,7 +434,20 @@ int orc_quantize_nvfp4(const void *x, int dtype, int64_t rows, int64_t cols, int
                        float *s_dec_out, uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col,
                        uint8_t *sf_col, int scale_layout) {
   return quantize_1x16(x, dtype, rows, cols, ld, layouts, round, seed, amax_in, s_dec_out,
-                       q_row, sf_row, q_col, sf_col, scale_layout, 6.0f);
+                       q_row, sf_row, q_col, sf_col, scale_layout, 6.0f, 0);
+}
+
+/* The same for rows row0 .. row0 + rows - 1 of a larger tensor with cols     */
+/* columns, given its amax: the SR bits use the whole tensor's flat index     */
+/* (row0 + r) * cols + c, everything else is local to the rows (row-wise     */
+/* blocks; column blocks when rows and row0 are multiples of 16).            */
+int orc_quantize_nvfp4_rows(const void *x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                            unsigned layouts, int round, uint64_t seed, const float *amax_in,
+                            float *s_dec_out, uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col,
+                            uint8_t *sf_col, int scale_layout, int64_t row0) {
+  if (row0 < 0) return 1;
+  return quantize_1x16(x, dtype, rows, cols, ld, layouts, round, seed, amax_in, s_dec_out,
+                       q_row, sf_row, q_col, sf_col, scale_layout, 6.0f, row0);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -452,7 +467,7 @@ int orc_quantize_four_over_six(const void *x, int dtype, int64_t rows, int64_t c
                                uint8_t *q_row, uint8_t *sf_row, uint8_t *q_col, uint8_t *sf_col,
                                int scale_layout) {
   return quantize_1x16(x, dtype, rows, cols, ld, layouts, ORC_RNE, 0, amax_in, s_dec_out,
-                       q_row, sf_row, q_col, sf_col, scale_layout, 4.0f);
+                       q_row, sf_row, q_col, sf_col, scale_layout, 4.0f, 0);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -603,11 +618,12 @@ int orc_rht(const void *dy, int dtype, int64_t tokens, int64_t cols, int64_t ld,
  * values), written as dY^T codes [cols, tokens/2] and scales [cols, tokens/16].
  * SR bits use the flat input index token*cols + col.  [Q] "確率的丸め": SR
  * is what helps gradient quantization. */
-int orc_quantize_rht(const void *dy, int dtype, int64_t tokens, int64_t cols, int64_t ld,
-                     int n, int round, uint64_t seed, const float *amax_rht_in,
-                     float *s_dec_out, uint8_t *q_t, uint8_t *sf_t, int scale_layout,
-                     float *rht_out) {
+static int quantize_rht_at(const void *dy, int dtype, int64_t tokens, int64_t cols, int64_t ld,
+                           int n, int round, uint64_t seed, const float *amax_rht_in,
+                           float *s_dec_out, uint8_t *q_t, uint8_t *sf_t, int scale_layout,
+                           float *rht_out, int64_t token0) {
   if (n != 16 && n != 128) return 1;
+  if (token0 < 0) return 1;
   if (tokens % n != 0 || tokens % 16 != 0) return 1;
   float *t = (float *)malloc(sizeof(float) * (size_t)(tokens * cols));
   if (!t) return 2;
@@ -631,12 +647,32 @@ int orc_quantize_rht(const void *dy, int dtype, int64_t tokens, int64_t cols, in
       for (int k = 0; k < 16; ++k) {
         int64_t r = b * 16 + k;
         float v = t[r * cols + c] * rf;
-        uint8_t code = encode_elem(v, round, seed, (uint64_t)(r * cols + c));
+        uint8_t code = encode_elem(v, round, seed, (uint64_t)((token0 + r) * cols + c));
         put_nibble(q_t, c * (tokens / 2) + r / 2, (int)(r & 1), code);
       }
     }
   free(t);
   return 0;
+}
+
+int orc_quantize_rht(const void *dy, int dtype, int64_t tokens, int64_t cols, int64_t ld,
+                     int n, int round, uint64_t seed, const float *amax_rht_in,
+                     float *s_dec_out, uint8_t *q_t, uint8_t *sf_t, int scale_layout,
+                     float *rht_out) {
+  return quantize_rht_at(dy, dtype, tokens, cols, ld, n, round, seed, amax_rht_in, s_dec_out,
+                         q_t, sf_t, scale_layout, rht_out, 0);
+}
+
+/* The same for tokens token0 .. token0 + tokens - 1 of a larger gradient with */
+/* cols columns, given the transform's amax: the SR bits use the whole        */
+/* tensor's flat index (token0 + t) * cols + c; the transform and the blocks  */
+/* are local when token0 is a multiple of n (the signs repeat per group).     */
+int orc_quantize_rht_rows(const void *dy, int dtype, int64_t tokens, int64_t cols, int64_t ld,
+                          int n, int round, uint64_t seed, const float *amax_rht_in,
+                          float *s_dec_out, uint8_t *q_t, uint8_t *sf_t, int scale_layout,
+                          float *rht_out, int64_t token0) {
+  return quantize_rht_at(dy, dtype, tokens, cols, ld, n, round, seed, amax_rht_in, s_dec_out,
+                         q_t, sf_t, scale_layout, rht_out, token0);
 }
 
 /* ------------------------------------------------------------------------ */

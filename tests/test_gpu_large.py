@@ -8,8 +8,9 @@ last) against the oracle run on those rows alone.  The row-wise formats are
 row-independent once the tensor amax is given, so that comparison is exact.
 The formats whose blocks span rows (row+col NVFP4 and MXFP4, 2D, the RHT
 along tokens) are compared on bands of whole blocks (first, middle, last).
-Round to nearest throughout (the stochastic-rounding bits depend on the
-global element index).
+Round to nearest, except in the stochastic-rounding tests: their bits depend
+on the global element index, so the oracle runs on the band with the band's
+first row (row0 / token0) and draws the same bits.
 """
 import pytest
 import torch
@@ -149,6 +150,36 @@ def test_large_rht(orc, big, n):
     for r0 in bands(n):
         want = orc.quantize_rht(bits(x[r0:r0 + n]), n, round=orc.RNE, amax_rht=a)
         assert_same("s_dec", host(out["s_dec"]), want["s_dec"])
+        assert_same("q_t", host(out["q_t"][:, r0 // 2:r0 // 2 + n // 2]), want["q_t"])
+        assert_same("sf_t", host(out["sf_t"].view(C, R // 16)[:, r0 // 16:r0 // 16 + n // 16]),
+                    want["sf_t"])
+
+
+@pytest.mark.parametrize("layouts", [1, 3])
+def test_large_nvfp4_sr(orc, big, layouts):
+    """Stochastic rounding at more than 2^31 elements: the oracle runs on a
+    band with the band's first row, so that its SR bits come from the whole
+    tensor's flat index, as the kernel's do."""
+    x, amax = big
+    out = fq.fp4q_quantize_nvfp4(x, layouts=layouts, round=fq.SR, seed=21, amax=amax)
+    for r0 in bands(16):
+        want = orc.quantize_nvfp4(bits(x[r0:r0 + 16]), layouts=layouts, round=orc.SR, seed=21,
+                                  amax=PEAK, row0=r0)
+        assert_same("q_row", host(out["q_row"][r0:r0 + 16]), want["q_row"])
+        assert_same("sf_row", host(out["sf_row"].view(R, C // 16)[r0:r0 + 16]), want["sf_row"])
+        if layouts & fq.COLWISE:
+            assert_same("q_col", host(out["q_col"][:, r0 // 2:r0 // 2 + 8]), want["q_col"])
+
+
+@pytest.mark.parametrize("n", [16, 128])
+def test_large_rht_sr(orc, big, n):
+    x, _ = big
+    a = 16384.0
+    out = fq.fp4q_quantize_rht_sr(x, n, round=fq.SR, seed=23,
+                                  amax_rht=torch.tensor([a], dtype=torch.float32, device=DEV))
+    for r0 in bands(n):
+        want = orc.quantize_rht(bits(x[r0:r0 + n]), n, round=orc.SR, seed=23, amax_rht=a,
+                                token0=r0)
         assert_same("q_t", host(out["q_t"][:, r0 // 2:r0 // 2 + n // 2]), want["q_t"])
         assert_same("sf_t", host(out["sf_t"].view(C, R // 16)[:, r0 // 16:r0 // 16 + n // 16]),
                     want["sf_t"])

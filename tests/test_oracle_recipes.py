@@ -475,3 +475,41 @@ def test_openmp_build_gives_the_same_bytes(orc):
         for name in one[k]:
             a, b = np.asarray(one[k][name]), np.asarray(many[k][name])
             assert a.tobytes() == b.tobytes(), (k, name)
+
+
+
+def _whole_amax(x_bits):
+    """max |x| of BF16 bit patterns, as a float."""
+    return float(np.abs((x_bits.astype(np.uint32) << 16).view(np.float32)).max())
+
+
+def test_band_of_rows_draws_the_whole_tensors_sr_bits(orc):
+    """The row-offset entries (row0 / token0) exist so that a band of a tensor
+    too large for the oracle can be checked with stochastic rounding: on a
+    band of whole blocks, given the tensor's amax, they must give exactly the
+    band's slice of the whole tensor's outputs, which draw their SR bits from
+    the whole tensor's flat index (Qiita note, "確率的丸め")."""
+    x = bf16_bits(workloads.gradient(tokens=512, cols=96))
+    a = _whole_amax(x)
+    whole = orc.quantize_nvfp4(x, layouts=3, round=orc.SR, seed=11)
+    for r0 in (0, 16, 256, 496):
+        band = orc.quantize_nvfp4(x[r0:r0 + 16], layouts=3, round=orc.SR, seed=11, amax=a,
+                                  row0=r0)
+        assert np.array_equal(band["q_row"], whole["q_row"][r0:r0 + 16])
+        assert np.array_equal(band["sf_row"].reshape(16, -1),
+                              whole["sf_row"].reshape(512, -1)[r0:r0 + 16])
+        assert np.array_equal(band["q_col"], whole["q_col"][:, r0 // 2:r0 // 2 + 8])
+        assert np.array_equal(band["sf_col"].reshape(96, -1),
+                              whole["sf_col"].reshape(96, -1)[:, r0 // 16:r0 // 16 + 1])
+    # the same band drawn with its own local index differs: the offset matters
+    local = orc.quantize_nvfp4(x[256:272], layouts=1, round=orc.SR, seed=11, amax=a)
+    assert not np.array_equal(local["q_row"], whole["q_row"][256:272])
+    for n in (16, 128):
+        t_whole = orc.quantize_rht(x, n, round=orc.SR, seed=5)
+        amax_t = float(np.abs(orc.rht(x, n, 5)).max())
+        for t0 in (0, 256, 512 - n):
+            band = orc.quantize_rht(x[t0:t0 + n], n, round=orc.SR, seed=5, amax_rht=amax_t,
+                                    token0=t0)
+            assert np.array_equal(band["q_t"], t_whole["q_t"][:, t0 // 2:t0 // 2 + n // 2])
+            assert np.array_equal(band["sf_t"].reshape(96, -1),
+                                  t_whole["sf_t"].reshape(96, -1)[:, t0 // 16:t0 // 16 + n // 16])
