@@ -48,6 +48,10 @@ if ROOT not in sys.path:
 METRIC = "quantize throughput GB/s (bytes in+out) and % of B200 HBM peak per config"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
+# the workload both arms name in their "config"
+SUITE_WORKLOAD = ("fp4 quantization suite: activation 8192x4096 nvfp4 row+col and mxfp4 "
+                  "row+col; weight 14336x4096 fp32 2d16x16; gradient 8192x5120 rht16/rht128 x "
+                  "sr/rne; if4 16384x8192 quant + bf16 dequant")
 LEAD_SLEEP_CYCLES = 200_000  # ~0.1 ms at 1.965 GHz, untimed
 
 
@@ -669,7 +673,9 @@ def run_reference(args):
         "ms_per_step": round(1e3 * total / len(times), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": "fp4 quantization suite (bounded row sample per step)",
+        "config": {"workload": SUITE_WORKLOAD,
+                   "sample": f"bounded row sample per step: the first {frac:.4g} of the rows "
+                             "of every workload",
                    "rows_fraction": frac, "l2": "n/a (CPU)", "parallelism": "rank 0 only"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s",
                          "cores": int(os.environ["OMP_NUM_THREADS"]), "kind": "oracle",
@@ -881,10 +887,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "fp4 quantization suite: activation 8192x4096 nvfp4 row+col "
-                                   "and mxfp4 row+col; weight 14336x4096 fp32 2d16x16; gradient "
-                                   "8192x5120 rht16/rht128 x sr/rne; if4 16384x8192 quant + "
-                                   "bf16 dequant",
+            "config": {"workload": SUITE_WORKLOAD,
                        "l2": "flushed before every kernel (256 MiB written then read, untimed)",
                        "launch": "device sleep before each flush hides host launch latency",
                        "amax": "precomputed on the device (headline); per_config "
