@@ -18,11 +18,14 @@
 //     LOP3 per packed pair), the butterfly stages h = 1, 2, 4, 8 run in
 //     registers on f32x2 column pairs;
 //   * for n = 128 the stages h = 16, 32, 64 combine the eight groups of a
-//     column quad: the warp swaps values through an 8 KB exchange buffer
-//     whose padding keeps both the write and the transposed read on eight
-//     distinct bank groups per eight lanes (every address a lane base plus a
-//     constant), runs the three stages in registers and writes the results
-//     back there;
+//     column quad, which sit in lanes g ^ 1, g ^ 2, g ^ 4.  With round to
+//     nearest each stage is a warp shuffle of the partner's values and one
+//     exact fused multiply-add per pair, and the lane keeps its own tokens in
+//     registers.  With stochastic rounding, where the registers are short,
+//     the warp swaps values through an 8 KB exchange buffer whose padding
+//     keeps both the write and the transposed read on eight distinct bank
+//     groups per eight lanes (every address a lane base plus a constant),
+//     runs the three stages in registers and writes the results back there;
 //   * the rest runs in two passes over the lane's two column pairs, which
 //     halves the values live at once: scaling by the transform's factor,
 //     block maxima (three-input maximum), block scales, stochastic rounding
@@ -140,6 +143,16 @@ constexpr int kPTabBytes = (2 * 127 + 1) * 16 + (127 / 16) * 16 + 16;
 static_assert(kPTabBytes <= kUnits * 8, "the table fits in one BF16 input stage");
 __host__ __device__ constexpr int ptab_off(int t, int o) { return (2 * t + o) * 16 + (t >> 4) * 16; }
 
+// The 128-point transform's cross-group stages go by warp shuffles with
+// round to nearest, where the lane keeps its values in registers throughout;
+// with stochastic rounding, whose Philox words need the registers, through
+// the shared exchange buffer.  Its bytes per warp:
+__host__ __device__ constexpr bool rht_shuffle_stages(int n, bool sr) { return n == 128 && !sr; }
+__host__ __device__ constexpr int rht_xbytes(int n, bool sr) {
+  return n == 128 && !rht_shuffle_stages(n, sr) ? kXUnits * 16 : 0;
+}
+
+
 // Coordinates (tile row tt, tile column tc) of a linear tile index over a grid
 // of tiles_c tile columns, stepped by a fixed number of tiles without
 // dividing; 32-bit.
@@ -171,7 +184,8 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   constexpr int UB = 4 * sizeof(T);                       // bytes per input chunk
   constexpr int IN_BYTES = 2 * kUnits * UB;               // two stages
   constexpr bool PTAB_IN_STAGE = SR && N == 128 && !ROW;
-  constexpr int WARP_BYTES = IN_BYTES + (N == 128 ? kXUnits * 16 : 0) + ((SR && !PTAB_IN_STAGE) ? kPTabBytes : 0);
+  constexpr bool XSHFL = rht_shuffle_stages(N, SR);
+  constexpr int WARP_BYTES = IN_BYTES + rht_xbytes(N, SR) + ((SR && !PTAB_IN_STAGE) ? kPTabBytes : 0);
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float rtab[128];
   __shared__ float rtab_row[ROW ? 128 : 1];
@@ -179,7 +193,7 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   uint8_t *wbase = smem + warp * WARP_BYTES;
   const uint32_t in_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbase));
   float4 *xbuf = reinterpret_cast<float4 *>(wbase + IN_BYTES);
-  uint8_t *const ptab_own = wbase + IN_BYTES + (N == 128 ? kXUnits * 16 : 0);
+  uint8_t *const ptab_own = wbase + IN_BYTES + rht_xbytes(N, SR);
   const int my_unit = unit_of(16 * g, cq);                // unit (16 g + k, cq) = my_unit + 4 k
 
   // signs of this lane's 16 tokens
@@ -310,9 +324,9 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
     // on distinct banks; for n = 16 every lane takes pair 0 first.
     uint32_t raw1[sizeof(T) == 2 ? 16 : 1];   // BF16: the pass-1 pair, still packed
     float2 *xb2 = reinterpret_cast<float2 *>(xbuf) + 2 * (73 * g + cq);
+    float2 lo[16], hi[16];   // n = 128: the lane's four columns (unused for n = 16)
     if (N == 128) {
       // ---- the whole 128-point transform on all four columns --------------------
-      float2 lo[16], hi[16];
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         const uint32_t sg = sign_of(k);
@@ -330,6 +344,30 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
       }
       stages16(lo);
       stages16(hi);
+    }
+    if (N == 128 && XSHFL) {
+      // ---- stages h = 16, 32, 64 across the eight groups, by warp shuffles -------
+      // token 16 g + k meets token 16 (g ^ m) + k, m = 1, 2, 4, which sits in
+      // lane ^ m: the lane with bit m of g clear keeps RN(a + b), its partner
+      // RN(a - b); both are fma(own, +-1, partner), whose product is exact, so
+      // the lane keeps its own 16 tokens and nothing is written back
+#pragma unroll
+      for (int sgi = 0; sgi < 3; ++sgi) {
+        const int m = 1 << sgi;
+        const float sgn = (g & m) ? -1.0f : 1.0f;
+        const float2 sg2 = make_float2(sgn, sgn);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float2 pl = make_float2(__shfl_xor_sync(0xFFFFFFFFu, lo[k].x, m),
+                                        __shfl_xor_sync(0xFFFFFFFFu, lo[k].y, m));
+          const float2 ph = make_float2(__shfl_xor_sync(0xFFFFFFFFu, hi[k].x, m),
+                                        __shfl_xor_sync(0xFFFFFFFFu, hi[k].y, m));
+          lo[k] = fma2(lo[k], sg2, pl);
+          hi[k] = fma2(hi[k], sg2, ph);
+        }
+      }
+    }
+    if (N == 128 && !XSHFL) {
       // stages h = 16, 32, 64 across the eight groups: swap through the
       // exchange buffer so that a lane holds tokens 16 gg + 2 g + o of all
       // eight groups gg, run the stages, and write the results back there
@@ -363,9 +401,12 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
     // ---- two passes over the column pairs ---------------------------------------
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
-      const int pp = N == 128 ? p ^ half : p;  // the column pair of this pass
+      const int pp = (N == 128 && !XSHFL) ? p ^ half : p;  // the column pair of this pass
       float2 v[16];
-      if (N == 128) {
+      if (N == 128 && XSHFL) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = p == 0 ? lo[k] : hi[k];
+      } else if (N == 128) {
 #pragma unroll
         for (int k = 0; k < 16; ++k) v[k] = xb2[2 * xunit_own(k) + pp];
         __syncwarp();   // the exchange buffer is rewritten by the next tile
@@ -588,7 +629,7 @@ cudaError_t launch_k2(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uin
                       uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L,
                       const RowArgs &R) {
   constexpr int UB = 4 * sizeof(T);
-  constexpr int WARP_BYTES = 2 * kUnits * UB + (N == 128 ? kXUnits * 16 : 0) +
+  constexpr int WARP_BYTES = 2 * kUnits * UB + rht_xbytes(N, SR) +
                              ((SR && !(N == 128 && !ROW)) ? kPTabBytes : 0);
   constexpr int SMEM = kWarps * WARP_BYTES;
   const void *kern = reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY, ROW, I32>);
