@@ -18,20 +18,17 @@
 //     LOP3 per packed pair), the butterfly stages h = 1, 2, 4, 8 run in
 //     registers on f32x2 column pairs;
 //   * for n = 128 the stages h = 16, 32, 64 combine the eight groups of a
-//     column quad, which sit in lanes g ^ 1, g ^ 2, g ^ 4.  With round to
-//     nearest each stage is a warp shuffle of the partner's values and one
-//     exact fused multiply-add per pair, and the lane keeps its own tokens in
-//     registers.  With stochastic rounding, where the registers are short,
-//     the warp swaps values through an 8 KB exchange buffer whose padding
-//     keeps both the write and the transposed read on eight distinct bank
-//     groups per eight lanes (every address a lane base plus a constant),
-//     runs the three stages in registers and writes the results back there;
-//   * the rest runs in two passes over the lane's two column pairs, which
-//     halves the values live at once: scaling by the transform's factor,
-//     block maxima (three-input maximum), block scales, stochastic rounding
-//     or RNE, packing and the stores of the pair's two code rows and scales.
-//     Lanes of odd column quads take their pairs in the opposite order, which
-//     keeps the pass reads of the exchange buffer conflict-free;
+//     column quad, which sit in lanes g ^ 1, g ^ 2, g ^ 4: each stage is a
+//     warp shuffle of the partner's values and one exact fused multiply-add
+//     per pair, so the lane keeps its own tokens in registers throughout;
+//   * three CTAs per SM for n = 128, stochastic rounding and the fused
+//     backward (the register budget that avoids spills), four for the
+//     16-point transform with round to nearest;
+//   * the rest runs in two passes over the lane's two column pairs (for
+//     n = 16 each pass also transforms its pair, which halves the values live
+//     at once): scaling by the transform's factor, block maxima (three-input
+//     maximum), block scales, stochastic rounding or RNE, packing and the
+//     stores of the pair's two code rows and scales;
 //   * stochastic rounding needs one Philox call per token per 8 columns,
 //     256 per tile: each lane computes 8 of them and stores their four words
 //     in a per-warp table in shared memory, from which both passes read the
@@ -92,24 +89,6 @@ __device__ __forceinline__ U32x4 philox_rk(const K &P, uint32_t c0, uint32_t c1)
   return U32x4{c0, c1, c2, c3};
 }
 
-// cross-group stage on (8 groups x 2 offsets) values, index 2 * group + offset
-template <int H>
-__device__ __forceinline__ void xstage(float2 (&lo)[16], float2 (&hi)[16]) {
-#pragma unroll
-  for (int g = 0; g < 8; ++g)
-    if ((g & H) == 0)
-#pragma unroll
-      for (int o = 0; o < 2; ++o) {
-        const int i = 2 * g + o, j = 2 * (g + H) + o;
-        const float2 a = lo[i], b = lo[j];
-        lo[i] = add2(a, b);
-        lo[j] = sub2(a, b);
-        const float2 c = hi[i], d = hi[j];
-        hi[i] = add2(c, d);
-        hi[j] = sub2(c, d);
-      }
-}
-
 // stages h = 1, 2, 4, 8 of one column pair over 16 tokens
 __device__ __forceinline__ void stages16(float2 (&v)[16]) {
 #pragma unroll
@@ -123,18 +102,6 @@ __device__ __forceinline__ void stages16(float2 (&v)[16]) {
       }
 }
 
-// The exchange buffer of the 128-point transform, in 16-byte units: (token t,
-// column quad q) sits at unit 4 t + q + t / 2 + t / 16, which grows with t
-// (so no two (t, q) share a unit) and whose two pad terms make both access
-// patterns hit eight distinct bank groups per eight lanes: the write of
-// tokens 16 g + k (fixed k, g = 0..7: the unit mod 8 is g + const) and the
-// transposed read of tokens 16 gg + 2 g + o (fixed gg, o: g + const again).
-// Every address is a lane base plus a constant: 73 g + q for the own tokens,
-// 9 g + q for the transposed ones.
-constexpr int kXUnits = 4 * 127 + 127 / 2 + 127 / 16 + 3 + 1;
-__host__ __device__ constexpr int xunit_own(int k) { return 4 * k + (k >> 1); }      // + 73 g + q
-__host__ __device__ constexpr int xunit_tr(int gg, int o) { return 73 * gg + 4 * o; }  // + 9 g + q
-
 // The Philox table of a warp tile: the four words of the call for token t
 // (0..127) and column octet o (0, 1) at byte (2 t + o) * 16 + (t / 16) * 16;
 // the pad puts the eight 16-byte writes of a quarter warp (tokens 16 g + i,
@@ -142,15 +109,6 @@ __host__ __device__ constexpr int xunit_tr(int gg, int o) { return 73 * gg + 4 *
 constexpr int kPTabBytes = (2 * 127 + 1) * 16 + (127 / 16) * 16 + 16;
 static_assert(kPTabBytes <= kUnits * 8, "the table fits in one BF16 input stage");
 __host__ __device__ constexpr int ptab_off(int t, int o) { return (2 * t + o) * 16 + (t >> 4) * 16; }
-
-// The 128-point transform's cross-group stages go by warp shuffles with
-// round to nearest, where the lane keeps its values in registers throughout;
-// with stochastic rounding, whose Philox words need the registers, through
-// the shared exchange buffer.  Its bytes per warp:
-__host__ __device__ constexpr bool rht_shuffle_stages(int n, bool sr) { return n == 128 && !sr; }
-__host__ __device__ constexpr int rht_xbytes(int n, bool sr) {
-  return n == 128 && !rht_shuffle_stages(n, sr) ? kXUnits * 16 : 0;
-}
 
 
 // Coordinates (tile row tt, tile column tc) of a linear tile index over a grid
@@ -175,7 +133,7 @@ struct TileCursor32 {
 };
 
 template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW, bool I32>
-__global__ void __launch_bounds__(kThreads, ROW ? 3 : 4)
+__global__ void __launch_bounds__(kThreads, (ROW || SR || N == 128) ? 3 : 4)
 rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
            const RhtParams P, const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
            unsigned *__restrict__ amax_out, uint8_t *__restrict__ q_t,
@@ -184,16 +142,14 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   constexpr int UB = 4 * sizeof(T);                       // bytes per input chunk
   constexpr int IN_BYTES = 2 * kUnits * UB;               // two stages
   constexpr bool PTAB_IN_STAGE = SR && N == 128 && !ROW;
-  constexpr bool XSHFL = rht_shuffle_stages(N, SR);
-  constexpr int WARP_BYTES = IN_BYTES + rht_xbytes(N, SR) + ((SR && !PTAB_IN_STAGE) ? kPTabBytes : 0);
+  constexpr int WARP_BYTES = IN_BYTES + ((SR && !PTAB_IN_STAGE) ? kPTabBytes : 0);
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float rtab[128];
   __shared__ float rtab_row[ROW ? 128 : 1];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane & 7, cq = lane >> 3;
   uint8_t *wbase = smem + warp * WARP_BYTES;
   const uint32_t in_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbase));
-  float4 *xbuf = reinterpret_cast<float4 *>(wbase + IN_BYTES);
-  uint8_t *const ptab_own = wbase + IN_BYTES + rht_xbytes(N, SR);
+  uint8_t *const ptab_own = wbase + IN_BYTES;
   const int my_unit = unit_of(16 * g, cq);                // unit (16 g + k, cq) = my_unit + 4 k
 
   // signs of this lane's 16 tokens
@@ -319,11 +275,7 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
     };
 
     // The lane works on its four columns as two column pairs, one per pass.
-    // For n = 128 the order is lane-dependent (pair half in pass 0, pair
-    // half ^ 1 in pass 1), which keeps the pass reads of the exchange buffer
-    // on distinct banks; for n = 16 every lane takes pair 0 first.
     uint32_t raw1[sizeof(T) == 2 ? 16 : 1];   // BF16: the pass-1 pair, still packed
-    float2 *xb2 = reinterpret_cast<float2 *>(xbuf) + 2 * (73 * g + cq);
     float2 lo[16], hi[16];   // n = 128: the lane's four columns (unused for n = 16)
     if (N == 128) {
       // ---- the whole 128-point transform on all four columns --------------------
@@ -345,7 +297,7 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
       stages16(lo);
       stages16(hi);
     }
-    if (N == 128 && XSHFL) {
+    if (N == 128) {
       // ---- stages h = 16, 32, 64 across the eight groups, by warp shuffles -------
       // token 16 g + k meets token 16 (g ^ m) + k, m = 1, 2, 4, which sits in
       // lane ^ m: the lane with bit m of g clear keeps RN(a + b), its partner
@@ -367,49 +319,19 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
         }
       }
     }
-    if (N == 128 && !XSHFL) {
-      // stages h = 16, 32, 64 across the eight groups: swap through the
-      // exchange buffer so that a lane holds tokens 16 gg + 2 g + o of all
-      // eight groups gg, run the stages, and write the results back there
-      float4 *xw = xbuf + (73 * g + cq), *xr = xbuf + (9 * g + cq);
-#pragma unroll
-      for (int k = 0; k < 16; ++k)
-        xw[xunit_own(k)] = make_float4(lo[k].x, lo[k].y, hi[k].x, hi[k].y);
+    if (PTAB_IN_STAGE) {   // the stage's raw values are all read
       __syncwarp();
-#pragma unroll
-      for (int gg = 0; gg < 8; ++gg)
-#pragma unroll
-        for (int o = 0; o < 2; ++o) {
-          const float4 c = xr[xunit_tr(gg, o)];
-          lo[2 * gg + o] = make_float2(c.x, c.y);
-          hi[2 * gg + o] = make_float2(c.z, c.w);
-        }
-      xstage<1>(lo, hi);   // h = 16
-      xstage<2>(lo, hi);   // h = 32
-      xstage<4>(lo, hi);   // h = 64
-#pragma unroll
-      for (int gg = 0; gg < 8; ++gg)
-#pragma unroll
-        for (int o = 0; o < 2; ++o) {
-          const int i = 2 * gg + o;
-          xr[xunit_tr(gg, o)] = make_float4(lo[i].x, lo[i].y, hi[i].x, hi[i].y);
-        }
-      __syncwarp();
-      if (PTAB_IN_STAGE) philox_phase();   // the stage's raw values are all read
+      philox_phase();
     }
 
     // ---- two passes over the column pairs ---------------------------------------
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
-      const int pp = (N == 128 && !XSHFL) ? p ^ half : p;  // the column pair of this pass
+      const int pp = p;                      // the column pair of this pass
       float2 v[16];
-      if (N == 128 && XSHFL) {
+      if (N == 128) {
 #pragma unroll
         for (int k = 0; k < 16; ++k) v[k] = p == 0 ? lo[k] : hi[k];
-      } else if (N == 128) {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = xb2[2 * xunit_own(k) + pp];
-        __syncwarp();   // the exchange buffer is rewritten by the next tile
       } else {
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -629,7 +551,7 @@ cudaError_t launch_k2(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uin
                       uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L,
                       const RowArgs &R) {
   constexpr int UB = 4 * sizeof(T);
-  constexpr int WARP_BYTES = 2 * kUnits * UB + rht_xbytes(N, SR) +
+  constexpr int WARP_BYTES = 2 * kUnits * UB +
                              ((SR && !(N == 128 && !ROW)) ? kPTabBytes : 0);
   constexpr int SMEM = kWarps * WARP_BYTES;
   const void *kern = reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY, ROW, I32>);

@@ -183,39 +183,6 @@ def _rht_source():
     return open(os.path.join(HERE, "..", "fp4_block_scaled_04_b200", "csrc", "rht.cu")).read()
 
 
-def test_rht128_exchange_layout_is_one_to_one_and_conflict_free():
-    """The n = 128 exchange buffer of the RHT kernel: unit (token t, column
-    quad q) = 4 t + q + t / 2 + t / 16 (16-byte units). Each unit holds at
-    most one (t, q). The two access patterns each put eight lanes on eight
-    distinct bank groups (unit mod 8): the write of tokens 16 g + k (fixed k
-    and q) and the transposed read of tokens 16 gg + 2 g + o (fixed gg, o,
-    q). Both are a lane base plus a constant, as the kernel computes them:
-    73 g + q + xunit_own(k) and 9 g + q + xunit_tr(gg, o)."""
-    src = _rht_source()
-    assert "constexpr int kXUnits = 4 * 127 + 127 / 2 + 127 / 16 + 3 + 1;" in src
-    assert "xunit_own(int k) { return 4 * k + (k >> 1); }" in src
-    assert "xunit_tr(int gg, int o) { return 73 * gg + 4 * o; }" in src
-    n_units = 4 * 127 + 127 // 2 + 127 // 16 + 3 + 1
-    unit = lambda t, q: 4 * t + q + t // 2 + t // 16
-    seen = {}
-    for t in range(128):
-        for q in range(4):
-            u = unit(t, q)
-            assert 0 <= u < n_units
-            assert u not in seen, (t, q, seen.get(u))
-            seen[u] = (t, q)
-    for q in range(4):
-        for k in range(16):
-            units = [unit(16 * g + k, q) for g in range(8)]
-            assert units == [73 * g + q + 4 * k + (k >> 1) for g in range(8)]
-            assert len({u % 8 for u in units}) == 8, (q, k)
-        for gg in range(8):
-            for o in range(2):
-                units = [unit(16 * gg + 2 * g + o, q) for g in range(8)]
-                assert units == [9 * g + q + 73 * gg + 4 * o for g in range(8)]
-                assert len({u % 8 for u in units}) == 8, (q, gg, o)
-
-
 def test_rht_philox_table_layout():
     """The per-warp Philox table of the SR transform: the four words of the
     call for token t and column octet o at byte (2 t + o) * 16 + (t / 16) * 16.
