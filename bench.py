@@ -53,6 +53,7 @@ SUITE_WORKLOAD = ("fp4 quantization suite: activation 8192x4096 nvfp4 row+col an
                   "row+col; weight 14336x4096 fp32 2d16x16; gradient 8192x5120 rht16/rht128 x "
                   "sr/rne; if4 16384x8192 quant + bf16 dequant")
 LEAD_SLEEP_CYCLES = 200_000  # ~0.1 ms at 1.965 GHz, untimed
+FIRST_LEAD_CYCLES = 4_000_000  # ~2 ms, untimed, before the first timed job
 
 
 def hbm_peak():
@@ -758,6 +759,11 @@ def main():
     torch.cuda.synchronize(device)
     wall0 = time.perf_counter()
     with ClockSampler(local) as clocks:
+        # an untimed device sleep of about 2 ms first: the host then enqueues
+        # the first jobs while the device waits, so neither the sampler
+        # thread's start nor the loop's first host steps reach the first
+        # job's events
+        torch.cuda._sleep(FIRST_LEAD_CYCLES)
         for s in range(args.steps):
             step(events[s])
         torch.cuda.synchronize(device)
@@ -781,6 +787,7 @@ def main():
             run()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
+        torch.cuda._sleep(FIRST_LEAD_CYCLES)
         for a, b in ev:
             torch.cuda._sleep(LEAD_SLEEP_CYCLES)
             flush.fill_(tag + 1.0)

@@ -61,6 +61,7 @@ def timer(reps: int, dev):
         torch.cuda.synchronize(dev)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(reps)]
+        torch.cuda._sleep(4_000_000)   # ~2 ms, untimed: the host gets ahead of the device
         for i, (a, b) in enumerate(ev):
             torch.cuda._sleep(200000)
             flush.fill_(float(i))
