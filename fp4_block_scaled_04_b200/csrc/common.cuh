@@ -89,6 +89,31 @@ __device__ __forceinline__ uint32_t e2m1x4(float f0, float f1, float f2, float f
   return r;
 }
 
+// The truncating forms of e2m1x8 and e2m1x4: each value goes to the largest
+// E2M1 magnitude not above |v| (6 for anything larger, infinity included),
+// with its sign.  This is cvt.rs.satfinite with zero random bits: the
+// stochastic conversion adds its random bits below the kept ones before
+// dropping them, so with none it truncates.  The stochastic-rounding paths
+// feed it the dithered values of e2m1_sr_dithered2.  The first operand of
+// the x4 conversion lands in the top nibble.
+__device__ __forceinline__ uint32_t e2m1x8_rz(const float (&v)[8]) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 h0, h1;\n\t"
+      "cvt.rs.satfinite.e2m1x4.f32 h0, {%4, %3, %2, %1}, %9;\n\t"
+      "cvt.rs.satfinite.e2m1x4.f32 h1, {%8, %7, %6, %5}, %9;\n\t"
+      "mov.b32 %0, {h0, h1};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+        "f"(v[7]), "r"(0u));
+  return r;
+}
+__device__ __forceinline__ uint32_t e2m1x4_rz(float f0, float f1, float f2, float f3) {
+  uint16_t h;
+  asm("cvt.rs.satfinite.e2m1x4.f32 %0, {%4, %3, %2, %1}, %5;"
+      : "=h"(h) : "f"(f0), "f"(f1), "f"(f2), "f"(f3), "r"(0u));
+  return h;
+}
+
 // ---------------------------------------------------------------------------
 // E4M3 encode / decode (block scales)
 // ---------------------------------------------------------------------------
@@ -413,51 +438,34 @@ __device__ __forceinline__ float absmax8(uint4 u) {
   return bf16x2_hmax(maxabs_bf16x2(maxabs_bf16x2(u.x, u.y), maxabs_bf16x2(u.z, u.w)));
 }
 
-// Stochastic rounding of v onto the E2M1 grid, returned as a float that the
-// round-to-nearest conversion (cvt.rn.satfinite.e2m1x2) then encodes exactly
-// (the oracle's rule: the magnitude goes up iff u < t * 2^16).  On
-// [1, 8) E2M1 is a float with one mantissa bit, so adding 0x3FFFFF - 64 u to
-// the bits and clearing the low 22 rounds up exactly when 64 u < frac; below
-// 1 the spacing 0.5 equals that of [1, 2), so w = RU(|v| + 1) is rounded the
-// same way and 1 subtracted again (rounding the sum up keeps the comparison
-// with the integer 64 u exact).  Values rounded to 8 saturate to 6 in the
-// conversion; the sign is copied.  Checked against the oracle by
-// tests/sr_check.c (method 1).  z = 0x3FFFFF - 64 u.
-__device__ __forceinline__ float e2m1_sr_value(float v, uint32_t z) {
-  const float av = fabsf(v);
-  const float a = av < 1.0f ? 1.0f : 0.0f;
-  const float w = __fadd_ru(av, a);
-  const float r = __fsub_rn(__uint_as_float((__float_as_uint(w) + z) & 0xFFC00000u), a);
-  return __uint_as_float(__float_as_uint(r) | (__float_as_uint(v) & 0x80000000u));
-}
-// z of the low / high 16-bit uniform of a 32-bit word
-__device__ __forceinline__ uint32_t sr_z_lo(uint32_t w) { return 0x3FFFFFu ^ ((w << 6) & 0x3FFFC0u); }
-__device__ __forceinline__ uint32_t sr_z_hi(uint32_t w) { return 0x3FFFFFu ^ ((w >> 10) & 0x3FFFC0u); }
-
-// Stochastic rounding of v onto the E2M1 grid by scaling (the oracle's rule,
-// checked against it by tests/sr_check.c, method 2): w = RU(|v| * 2^-126)
-// maps the whole E2M1 grid onto float bit patterns that keep the top 2^22
-// ulps of the low bits -- [1, 8) onto normal binades with one mantissa bit
-// kept, [0, 1) onto the subnormals, whose uniform step makes E2M1's 0.5
-// spacing 2^22 steps too -- so adding 0x3FFFFF - 64 u and clearing the low
-// 22 bits rounds the magnitude up exactly when 64 u < frac, with no range
-// test.  Rounding the product up keeps that comparison exact where the
-// scaling drops low bits of |v| < 1.  The sign is put back and the product
-// with 2^126 (exact) is encoded by the round-to-nearest conversion, which
-// maps 8 (and anything larger, including an overflow to infinity) to 6.
-// x64 = 64 u (sr_x_lo / sr_x_hi).
-__device__ __forceinline__ uint32_t sr_scaled_bits(float v, uint32_t x64) {
-  const float w = __fmul_ru(fabsf(v), 0x1p-126f);
-  const uint32_t b = (__float_as_uint(w) + 0x3FFFFFu - x64) & 0xFFC00000u;
-  return b | (__float_as_uint(v) & 0x80000000u);
-}
-__device__ __forceinline__ float e2m1_sr_scaled(float v, uint32_t x64) {
-  return __fmul_rn(__uint_as_float(sr_scaled_bits(v, x64)), 0x1p126f);
+// Stochastic rounding of v onto the E2M1 grid by scaling (the oracle's rule:
+// the magnitude goes up iff u < t * 2^16, with u the 16-bit uniform and t the
+// position of |v| between its two grid neighbours).  w = |v| * 2^-126 maps
+// the whole grid onto float bit patterns that keep the top 2^22 ulps of the
+// low bits: [1, 8) onto normal binades with one mantissa bit kept, [0, 1)
+// onto the subnormals, whose uniform step makes E2M1's 0.5 spacing 2^22 steps
+// too.  Adding 0x3FFFFF - 64 u to the bits of w therefore carries into the
+// kept bit exactly when 64 u < frac, with no test of the range; rounding the
+// product up keeps that comparison exact where the scaling drops low bits of
+// |v| < 1.  The sign of v is put back and the value multiplied by 2^126
+// (exact).  The bits below the kept one are not cleared here: the truncating
+// conversion (e2m1x8_rz, e2m1x4_rz) drops them, and maps 8 and above to 6.
+// The values the kernels pass stay below about 6.5 (the factor is s_enc / S
+// for the block's own rounded scale S), but unmasked an infinite |v| would
+// become a NaN pattern, so the scaled product saturates at 1 (mul.rp.sat, at
+// no cost): any |v| >= 2^126 lands in [1, 1.5) * 2^126, which the conversion
+// saturates to 6 as the oracle does.  Checked against the oracle by
+// tests/sr_check.c, method 3, infinity included.  x64 = 64 u (sr_x_lo /
+// sr_x_hi).
+__device__ __forceinline__ uint32_t sr_dither_bits(float v, uint32_t x64) {
+  float w;
+  asm("mul.rp.sat.f32 %0, %1, %2;" : "=f"(w) : "f"(fabsf(v)), "f"(0x1p-126f));
+  return (__float_as_uint(w) + 0x3FFFFFu - x64) | (__float_as_uint(v) & 0x80000000u);
 }
 // two values at once; the final exact scaling is one f32x2 product
-__device__ __forceinline__ float2 e2m1_sr_scaled2(float2 v, uint32_t xa, uint32_t xb) {
-  return mul2(make_float2(__uint_as_float(sr_scaled_bits(v.x, xa)),
-                          __uint_as_float(sr_scaled_bits(v.y, xb))),
+__device__ __forceinline__ float2 e2m1_sr_dithered2(float2 v, uint32_t xa, uint32_t xb) {
+  return mul2(make_float2(__uint_as_float(sr_dither_bits(v.x, xa)),
+                          __uint_as_float(sr_dither_bits(v.y, xb))),
               make_float2(0x1p126f, 0x1p126f));
 }
 // 64 u of the low / high 16-bit uniform of a 32-bit word

@@ -92,13 +92,13 @@ __device__ __forceinline__ void encode_sr16(const float (&v)[16], float f, const
     float t[8];
 #pragma unroll
     for (int k = 0; k < 8; k += 2) {
-      const float2 r = e2m1_sr_scaled2(
+      const float2 r = e2m1_sr_dithered2(
           mul2(make_float2(v[8 * h + k], v[8 * h + k + 1]), make_float2(f, f)),
           sr_x_lo(words[k >> 1]), sr_x_hi(words[k >> 1]));
       t[k] = r.x;
       t[k + 1] = r.y;
     }
-    w[h] = e2m1x8(t);
+    w[h] = e2m1x8_rz(t);
   }
 }
 
@@ -483,11 +483,14 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_
 #pragma unroll
           for (int j = 0; j < CPT; j += 2) {
             const float2 p = mul2(make_float2(v[i][j], v[i][j + 1]), make_float2(rf[k], rf[k]));
-            const float2 q = SR ? e2m1_sr_scaled2(p, u[i][j], u[i][j + 1]) : p;
+            const float2 q = SR ? e2m1_sr_dithered2(p, u[i][j], u[i][j + 1]) : p;
             t[j] = q.x;
             t[j + 1] = q.y;
           }
-          wr = CPT == 8 ? e2m1x8(t) : e2m1x4(t[0], t[1], t[2 % CPT], t[3 % CPT]);
+          if (SR)
+            wr = CPT == 8 ? e2m1x8_rz(t) : e2m1x4_rz(t[0], t[1], t[2 % CPT], t[3 % CPT]);
+          else
+            wr = CPT == 8 ? e2m1x8(t) : e2m1x4(t[0], t[1], t[2 % CPT], t[3 % CPT]);
           if (valid) {
             uint8_t *qa = q_row + (r0 + k) * (cols / 2) + c0 / 2;
             if (CPT == 8) *reinterpret_cast<uint32_t *>(qa) = wr;
@@ -505,10 +508,13 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_
           if (SR) {
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              p[i] = e2m1_sr_scaled2(p[i], u[i][j], u[i][j + 1]);
+              p[i] = e2m1_sr_dithered2(p[i], u[i][j], u[i][j + 1]);
           }
-          const uint32_t h0 = e2m1x4(p[0].x, p[1].x, p[2].x, p[3].x);  // column j, rows 4q4..4q4+3
-          const uint32_t h1 = e2m1x4(p[0].y, p[1].y, p[2].y, p[3].y);  // column j + 1
+          // column j, rows 4q4..4q4+3, and column j + 1
+          const uint32_t h0 = SR ? e2m1x4_rz(p[0].x, p[1].x, p[2].x, p[3].x)
+                                 : e2m1x4(p[0].x, p[1].x, p[2].x, p[3].x);
+          const uint32_t h1 = SR ? e2m1x4_rz(p[0].y, p[1].y, p[2].y, p[3].y)
+                                 : e2m1x4(p[0].y, p[1].y, p[2].y, p[3].y);
           if (q4 & 1) {
             colw[j][q4 >> 1] |= h0 << 16;
             colw[j + 1][q4 >> 1] |= h1 << 16;

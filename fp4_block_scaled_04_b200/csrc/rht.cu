@@ -37,9 +37,9 @@
 //     not grow).  The ten Philox round keys and the 128 signs come in as
 //     kernel parameters, and the counters are 32-bit arithmetic wherever the
 //     tensor has fewer than 2^35 elements (the high counter word is then 0).
-//     The values are rounded stochastically in place (e2m1_sr_scaled2: the
-//     rounding by scaling with 2^-126) and then packed by the same
-//     round-to-nearest conversion as the RNE path;
+//     The values are dithered in place (e2m1_sr_dithered2: the rounding by
+//     scaling with 2^-126) and then packed by the truncating conversion,
+//     which drops the bits below the kept one;
 //   * dY^T codes leave as 8 lanes x 8 bytes = 64 contiguous bytes per column.
 #include "common.cuh"
 #include "launch.h"
@@ -387,7 +387,7 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
           const uint32_t w = *reinterpret_cast<const uint32_t *>(pw + 32 * k);
-          v[k] = e2m1_sr_scaled2(v[k], sr_x_lo(w), sr_x_hi(w));
+          v[k] = e2m1_sr_dithered2(v[k], sr_x_lo(w), sr_x_hi(w));
         }
       }
       uint32_t wa[2], wb[2];
@@ -396,8 +396,8 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
         float a[8], b[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) { a[k] = v[8 * h + k].x; b[k] = v[8 * h + k].y; }
-        wa[h] = e2m1x8(a);
-        wb[h] = e2m1x8(b);
+        wa[h] = SR ? e2m1x8_rz(a) : e2m1x8(a);
+        wb[h] = SR ? e2m1x8_rz(b) : e2m1x8(b);
       }
       if (valid) {
         // columns c, c + 1: code rows tokens/2 bytes apart, scale rows 16 bytes
@@ -472,8 +472,8 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
             const uint32_t wd[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
             for (int k = 0; k < 8; k += 2) {
-              const float2 r = e2m1_sr_scaled2(make_float2(x[8 * h + k], x[8 * h + k + 1]),
-                                               sr_x_lo(wd[k >> 1]), sr_x_hi(wd[k >> 1]));
+              const float2 r = e2m1_sr_dithered2(make_float2(x[8 * h + k], x[8 * h + k + 1]),
+                                                 sr_x_lo(wd[k >> 1]), sr_x_hi(wd[k >> 1]));
               x[8 * h + k] = r.x;
               x[8 * h + k + 1] = r.y;
             }
@@ -483,7 +483,8 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
 #pragma unroll
         for (int k = 0; k < 8; ++k) { lo8[k] = x[k]; hi8[k] = x[8 + k]; }
         if (tv) {
-          *reinterpret_cast<uint2 *>(R.q + t * (cols / 2) + col0 / 2) = make_uint2(e2m1x8(lo8), e2m1x8(hi8));
+          *reinterpret_cast<uint2 *>(R.q + t * (cols / 2) + col0 / 2) =
+              SR ? make_uint2(e2m1x8_rz(lo8), e2m1x8_rz(hi8)) : make_uint2(e2m1x8(lo8), e2m1x8(hi8));
           R.sf[scale_offset(t, cur.tc, cols / 16, scale_layout)] = static_cast<uint8_t>(sbr);
         }
       }

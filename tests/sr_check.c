@@ -26,6 +26,16 @@
  * (towards +inf on the non-negative |v|), which keeps "64 u < frac" exact
  * where the scaling drops low bits of |v| < 1.  The sign is put back, the
  * value multiplied by 2^126 (exact) and converted as for method 1.
+ *
+ * Method 3 (method 2 with a truncating conversion): the low 22 bits are left
+ * as they are and the conversion truncates towards zero onto the E2M1 grid,
+ * saturating at 6 (cvt.rs.satfinite.e2m1x4 with zero random bits, which adds
+ * nothing below the kept bits).  Everything below the kept mantissa bit is
+ * then dropped by the conversion instead of the mask.  Without the mask an
+ * infinite |v| would turn into a NaN pattern, so the scaled product saturates
+ * at 1 (mul.rp.sat): every |v| >= 2^126 maps to [1, 1.5) * 2^126, which the
+ * conversion saturates to 6 like the oracle.
+
  * Usage: sr_check <n_random> [method] -- prints the number of mismatches. */
 #include <fenv.h>
 #include <math.h>
@@ -76,13 +86,37 @@ static uint32_t method2(float v, uint32_t u16) {
   return orc_e2m1_rne(r);
 }
 
-static int which = 0;
-static uint32_t pick(float v, uint32_t u16) {
-  return which == 2 ? method2(v, u16) : which ? method1(v, u16) : method(v, u16);
+/* truncation of x towards zero onto the E2M1 grid, saturating at 6 */
+static uint32_t e2m1_trunc(float x) {
+  static const float grid[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  float a = fabsf(x);
+  uint32_t c = 0;
+  for (uint32_t k = 0; k < 8; ++k)
+    if (grid[k] <= a) c = k;
+  return c | (signbit(x) ? 8u : 0u);
+}
+
+static uint32_t method3(float v, uint32_t u16) {
+  uint32_t raw = bits(v);
+  fesetround(FE_UPWARD);
+  volatile float w = fabsf(v) * 0x1p-126f;
+  fesetround(FE_TONEAREST);
+  float ws = w > 1.0f ? 1.0f : w;            /* .sat */
+  uint32_t T = bits(ws) + 0x3FFFFFu - (u16 << 6);
+  volatile float r = flt(T | (raw & 0x80000000u)) * 0x1p126f;
+  return e2m1_trunc(r);
 }
 
 static uint64_t s = 0x9E3779B97F4A7C15ull;
 static uint64_t rnd(void) { s ^= s << 13; s ^= s >> 7; s ^= s << 17; return s; }
+
+static int which = 0;
+static uint32_t pick(float v, uint32_t u16) {
+  return which == 3   ? method3(v, u16)
+         : which == 2 ? method2(v, u16)
+         : which      ? method1(v, u16)
+                      : method(v, u16);
+}
 
 int main(int argc, char **argv) {
   long n = atol(argv[1]);
@@ -107,8 +141,9 @@ int main(int argc, char **argv) {
      large that the scaled value rounds up to 2^128 */
   const uint32_t edge[] = {0x00000001u, 0x00000003u, 0x00012345u, 0x007FFFFFu, 0x00800000u,
                            0x00800001u, 0x01000000u, 0x0C000001u, 0x33800001u, 0x34000001u,
-                           0x7F7FFFFFu, 0x7F3FFFFFu, 0x7F400000u, 0x7E000001u};
-  if (which == 2)
+                           0x7F7FFFFFu, 0x7F3FFFFFu, 0x7F400000u, 0x7E000001u,
+                           0x7F800000u, 0x7E800000u, 0x7E7FFFFFu, 0x40FFFFFFu, 0x41000000u};
+  if (which >= 2)
     for (unsigned i = 0; i < sizeof edge / sizeof edge[0]; ++i)
       for (uint32_t u = 0; u < 65536; ++u) {
         float v = flt(edge[i]);

@@ -47,6 +47,14 @@ def test_backward_linear(orc, dtype, rnd, n, shape):
 
 @pytest.mark.parametrize("rnd", [0, 1])
 @pytest.mark.parametrize("n", [16, 128])
+def test_backward_zero_scale_blocks(orc, rnd, n):
+    """Blocks whose scale code is 0 (factor 0: signed zeros) in both outputs."""
+    from test_gpu_parity import wide_range
+    check(orc, wide_range(256, 48, torch.bfloat16, seed=43), n, rnd, 0)
+
+
+@pytest.mark.parametrize("rnd", [0, 1])
+@pytest.mark.parametrize("n", [16, 128])
 def test_backward_swizzled_given_amaxes(orc, rnd, n):
     dy = randmat(256, 128, torch.bfloat16, seed=72)
     a = float(torch.abs(dy.float()).max().item())

@@ -162,6 +162,42 @@ def test_nvfp4_degenerate(orc, kind):
             assert_same(f"{kind}/{k}", host(got[k]), want[k])
 
 
+def wide_range(rows, cols, dtype, seed):
+    """Values of about 100 and one of 4e10 at [0, 0].  The tensor scale
+    s_enc = 2688 / amax is then so small that a block whose largest magnitude
+    is a few hundred gets the scale code 0, whose factor is 0: its values
+    encode as zeros, negative ones as -0 (code 8), under both roundings."""
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(rows, cols, generator=g) * 100.0
+    x[0, 0] = 4e10
+    return x.to(dtype)
+
+
+@pytest.mark.parametrize("layouts", [1, 3])
+@pytest.mark.parametrize("rnd", [0, 1])
+def test_nvfp4_zero_scale_blocks(orc, layouts, rnd):
+    for dtype in DTYPES:
+        x = wide_range(64, 96, dtype, seed=41)
+        got = fq.fp4q_quantize_nvfp4(x.to(DEV), layouts=layouts, round=rnd, seed=77)
+        want = orc.quantize_nvfp4(bits(x), layouts=layouts, round=rnd, seed=77)
+        assert (want["sf_row"] == 0).sum() > 0
+        for k in ("s_dec", "q_row", "sf_row") + (("q_col", "sf_col") if layouts & 2 else ()):
+            assert_same(f"{dtype}/{k}", host(got[k]), want[k])
+
+
+@pytest.mark.parametrize("n", [16, 128])
+@pytest.mark.parametrize("rnd", [0, 1])
+def test_rht_zero_scale_blocks(orc, n, rnd):
+    """The same through the transform: the huge value stays in column 0,
+    whose blocks set the amax, and the other columns' blocks get scale 0."""
+    dy = wide_range(256, 48, torch.bfloat16, seed=42)
+    got = fq.fp4q_quantize_rht_sr(dy.to(DEV), n, round=rnd, seed=5)
+    want = orc.quantize_rht(bits(dy), n, round=rnd, seed=5)
+    assert (want["sf_t"] == 0).sum() > 0
+    for k in ("s_dec", "q_t", "sf_t"):
+        assert_same(k, host(got[k]), want[k])
+
+
 def test_empty_inputs():
     x = torch.empty(0, 32, dtype=torch.bfloat16, device=DEV)
     out = fq.fp4q_quantize_nvfp4(x, layouts=3)

@@ -162,11 +162,13 @@ def test_rint_ties_go_to_even():
     assert np.all(np.rint(t) % 2 == 0)
 
 
-@pytest.mark.parametrize("method", [0, 1, 2])
+@pytest.mark.parametrize("method", [0, 1, 2, 3])
 def test_stochastic_rounding_fixed_point_method(tmp_path, method):
     """The kernels' stochastic rounding methods (0: integer codes, 1: rounded
     values then the round-to-nearest conversion, 2: the same after scaling
-    by 2^-126, which needs no range test) equal the oracle's rule
+    by 2^-126, which needs no range test, 3: method 2 with the product
+    saturated at 1 and the low bits dropped by a truncating conversion
+    instead of a mask) equal the oracle's rule
     (round the magnitude up iff u < t * 2^16) on every u for values around
     each E2M1 grid point and midpoint, and on 4M random pairs."""
     exe = str(tmp_path / "sr_check")
