@@ -189,7 +189,10 @@ struct Cursor {
   }
 };
 
-template <typename T, bool SWZ, int MODE, typename I, bool FIXED>
+// EVEN: cols % 32 == 0 and an even scale address, so every block has a
+// partner, code rows are 16-byte aligned and both scale bytes of a pair go
+// out as one 2-byte store (the runtime tests of those cases drop out).
+template <typename T, bool SWZ, int MODE, typename I, bool FIXED, bool EVEN>
 __global__ void __launch_bounds__(kThreads, 5)
 if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
            const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
@@ -222,11 +225,11 @@ if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
     if (c.p >= npairs) return;
     const I cb = 2 * c.pc;
     const uint8_t *src = reinterpret_cast<const uint8_t *>(x + c.r * ld + cb * 16);
-    const int n = (cb + 1 < bpr) ? PPL : PPB;
+    const int n = (EVEN || cb + 1 < bpr) ? PPL : PPB;
     const uint32_t dst = my_s + static_cast<uint32_t>(st * STAGE);
 #pragma unroll
     for (int i = 0; i < PPL; ++i)
-      if (i < n) cp_async16(dst + static_cast<uint32_t>((i ^ swz) * 16), src + 16 * i);
+      if (EVEN || i < n) cp_async16(dst + static_cast<uint32_t>((i ^ swz) * 16), src + 16 * i);
   };
 
   Cursor<I> ci, cc;
@@ -253,7 +256,7 @@ if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
     cp_async_wait<kStages - 1>();
 
     const I r = cc.r, cb = 2 * cc.pc;
-    const bool has_b = cb + 1 < bpr;
+    const bool has_b = EVEN || cb + 1 < bpr;
     const uint8_t *buf = my_g + st * STAGE;
     float2 v[16];
     float ma, mb;
@@ -314,7 +317,7 @@ if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
     uint8_t *qp = q + r * (cols / 2) + cb * 8;
     const uint32_t ba = sa | (ia ? 0x80u : 0u), bb = sb | (ib ? 0x80u : 0u);
     if (has_b) {
-      if ((cols & 31) == 0) {
+      if (EVEN || (cols & 31) == 0) {
         *reinterpret_cast<uint4 *>(qp) = make_uint4(wa[0], wa[1], wb[0], wb[1]);
       } else {  // rows of codes are only 8-byte aligned
         *reinterpret_cast<uint2 *>(qp) = make_uint2(wa[0], wa[1]);
@@ -329,12 +332,14 @@ if4_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_,
       // scale matrix starts on an even address (the offset o is even)
       const I tile = (r >> 7) * (bpr >> 2) + (cb >> 2);
       const I o = tile * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (cb & 3);
-      if (sf_even) {
+      if (EVEN || sf_even) {
         *reinterpret_cast<uint16_t *>(sf + o) = static_cast<uint16_t>(ba | (bb << 8));
       } else {
         sf[o] = static_cast<uint8_t>(ba);
         sf[o + 1] = static_cast<uint8_t>(bb);
       }
+    } else if (EVEN) {   // r * bpr + cb is even
+      *reinterpret_cast<uint16_t *>(sf + r * bpr + cb) = static_cast<uint16_t>(ba | (bb << 8));
     } else {
       sf[r * bpr + cb] = static_cast<uint8_t>(ba);
       if (has_b) sf[r * bpr + cb + 1] = static_cast<uint8_t>(bb);
@@ -348,16 +353,21 @@ template <typename T, bool SWZ, int MODE, typename I>
 cudaError_t launch_i(const T *x, int64_t rows, int64_t cols, int64_t ld, const float *amax,
                      float *s_dec_out, uint8_t *q, uint8_t *sf, const Launch &L) {
   constexpr int SMEM = kWarps * kStages * 32 * 32 * static_cast<int>(sizeof(T));
-  // both forms share one occupancy query (same registers and shared memory
-  // by construction: the fixed form only drops work)
-  const void *kern = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE, I, false>);
-  const void *kern_f = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE, I, true>);
-  static KernelSetup setup, setup_f;
-  int per_sm = 0, per_sm_f = 0;
+  // the three forms have the same shared memory and nearly the same
+  // registers (the fixed and even forms only drop work); the grid is sized
+  // by the smallest occupancy of the forms it may launch
+  const void *kern = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE, I, false, false>);
+  const void *kern_f = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE, I, true, false>);
+  const void *kern_e = reinterpret_cast<const void *>(if4_kernel<T, SWZ, MODE, I, true, true>);
+  static KernelSetup setup, setup_f, setup_e;
+  int per_sm = 0, per_sm_f = 0, per_sm_e = 0;
   cudaError_t e = kernel_setup(setup, kern, kThreads, SMEM, &per_sm);
   if (e != cudaSuccess) return e;
   e = kernel_setup(setup_f, kern_f, kThreads, SMEM, &per_sm_f);
   if (e != cudaSuccess) return e;
+  e = kernel_setup(setup_e, kern_e, kThreads, SMEM, &per_sm_e);
+  if (e != cudaSuccess) return e;
+  if (per_sm_e < per_sm_f) per_sm_f = per_sm_e;
   const int64_t ppr = (cols / 16 + 1) / 2, npairs = rows * ppr;
   const int64_t want = (npairs + kThreads - 1) / kThreads;
   const int64_t cap = static_cast<int64_t>(per_sm < per_sm_f ? per_sm : per_sm_f) * L.num_sms;
@@ -370,12 +380,16 @@ cudaError_t launch_i(const T *x, int64_t rows, int64_t cols, int64_t ld, const f
       grid = g;
       fixed = true;
     }
+  const bool even = cols % 32 == 0 && (reinterpret_cast<uintptr_t>(sf) & 1u) == 0;
   // -0.0 as a run-time value (see if4_pair)
-  if (fixed)
-    if4_kernel<T, SWZ, MODE, I, true><<<static_cast<int>(grid), kThreads, SMEM, L.stream>>>(
+  if (fixed && even)
+    if4_kernel<T, SWZ, MODE, I, true, true><<<static_cast<int>(grid), kThreads, SMEM, L.stream>>>(
+        x, rows, cols, ld, amax, s_dec_out, q, sf, -0.0f);
+  else if (fixed)
+    if4_kernel<T, SWZ, MODE, I, true, false><<<static_cast<int>(grid), kThreads, SMEM, L.stream>>>(
         x, rows, cols, ld, amax, s_dec_out, q, sf, -0.0f);
   else
-    if4_kernel<T, SWZ, MODE, I, false><<<static_cast<int>(grid), kThreads, SMEM, L.stream>>>(
+    if4_kernel<T, SWZ, MODE, I, false, false><<<static_cast<int>(grid), kThreads, SMEM, L.stream>>>(
         x, rows, cols, ld, amax, s_dec_out, q, sf, -0.0f);
   return cudaGetLastError();
 }

@@ -317,13 +317,15 @@ def test_if4(orc, dtype, shape):
         assert_same(k, host(got[k]), want[k])
 
 
-@pytest.mark.parametrize("shape,layout", [((256, 32288), 0), ((2048, 2048), 1)])
+@pytest.mark.parametrize("shape,layout", [((256, 32288), 0), ((2048, 2048), 1), ((2048, 2048), 0)])
 def test_if4_lanes_walk_several_pairs(orc, shape, layout):
     """Shapes with more pairs of blocks than the grid has lanes. With 32288
     columns (1009 pairs per row, a prime that divides no full grid's stride)
     a lane's pair column changes from one pair to the next. With 2048
     columns the stride is a multiple of the pairs per row, so every lane
-    stays on one pair column."""
+    stays on one pair column; the columns are also a multiple of 32, so the
+    kernel's even form runs (no lone trailing block, both scale bytes of a
+    pair in one store), in both scale layouts."""
     x = workloads.if4_blocks(seed=34, rows=shape[0], cols=shape[1])
     got = fq.fp4q_quantize_if4(x.to(DEV), scale_layout=layout)
     want = orc.quantize_if4(bits(x), scale_layout=layout)
