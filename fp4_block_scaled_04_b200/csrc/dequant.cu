@@ -145,7 +145,12 @@ __device__ __forceinline__ I unit_scale(I r, I c, I cols) {
 // A warp takes NU x 32 consecutive 8-element units per step, lane l the units
 // l, l + 32, ...: every code load and output store of the warp is then one
 // contiguous stretch, and a thread has NU independent loads in flight.
-template <int FMT, int BROWS, bool SWZ, typename I, typename OutT>
+// ROWAL: cols % (NU * 32 * 8) == 0, so every row holds whole steps of a
+// warp: the NU * 32 units of a warp's step lie in one row, lane l's at
+// columns c + 256 j, all inside the matrix or all outside it, and the scale
+// byte of unit j sits DS j bytes after that of unit 0.  One cursor step, one
+// scale offset and one bound test per step then serve all NU units.
+template <int FMT, int BROWS, bool SWZ, typename I, bool ROWAL, typename OutT>
 __global__ void __launch_bounds__(kThreads)
 dequant_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ sf,
                const float *__restrict__ s_dec_ptr, I rows, I cols, OutT *__restrict__ y) {
@@ -159,6 +164,55 @@ dequant_kernel(const uint8_t *__restrict__ q, const uint8_t *__restrict__ sf,
   const I warp0 = (static_cast<I>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
   const I wstride = static_cast<I>(gridDim.x) * (kThreads / 32);
   const uint32_t *qw = reinterpret_cast<const uint32_t *>(q);
+  if (ROWAL) {
+    constexpr I DS = SWZ ? (BLK == 32 ? 1024 : 2048) : (BLK == 32 ? 8 : 16);
+    I rr = 0, cc = 0, dr1 = 0, dc1 = 0;               // row and column of unit 0
+    if (!FLAT) {
+      const I estride = wstride * NU * 32 * 8;
+      dr1 = estride / cols;
+      dc1 = estride - dr1 * cols;
+      const I e = (warp0 * NU * 32 + lane) * 8;
+      rr = e / cols;
+      cc = e - rr * cols;
+    }
+    auto load1 = [&](I b, uint32_t (&w)[NU], uint32_t (&s8)[NU]) {
+      const I si0 = FLAT ? (BLK == 32 ? (b >> 2) : (b >> 1))
+                         : unit_scale<BLK, BROWS, SWZ, I>(rr, cc, cols);
+#pragma unroll
+      for (int j = 0; j < NU; ++j) {
+        w[j] = __ldg(qw + b + 32 * j);
+        s8[j] = __ldg(sf + si0 + DS * j);
+      }
+      if (!FLAT) {
+        rr += dr1;
+        cc += dc1;
+        if (cc >= cols) {
+          cc -= cols;
+          ++rr;
+        }
+      }
+    };
+    const I step = wstride * NU * 32;
+    uint32_t cw[NU], sb[NU];
+    I base = warp0 * NU * 32 + lane;
+    if (base < total) load1(base, cw, sb);
+    for (; base < total; base += step) {
+      uint32_t cn[NU], sn[NU];
+      if (base + step < total) load1(base + step, cn, sn);
+#pragma unroll
+      for (int j = 0; j < NU; ++j) {
+        float2 v[4];
+        decode8<FMT>(cw[j], sb[j], s_dec, c67, v);
+        Store::put(y + static_cast<size_t>(base + 32 * j) * 8, v);
+      }
+#pragma unroll
+      for (int j = 0; j < NU; ++j) {
+        cw[j] = cn[j];
+        sb[j] = sn[j];
+      }
+    }
+    return;
+  }
   // (row, column) of each of the lane's NU units, advanced by a fixed stride
   I r[NU], c[NU];
   I dr = 0, dc = 0;
@@ -231,22 +285,30 @@ cudaError_t launch_fmt(const uint8_t *q, const uint8_t *sf, const float *s_dec, 
   // element index of a row start and the scale offsets all stay below 2^31
   const bool narrow = units + static_cast<int64_t>(grid) * 4 * kThreads < (int64_t(1) << 31) &&
                       rows * cols < (int64_t(1) << 31);
+  const bool rowal = cols % (4 * 32 * 8) == 0;        // whole warp steps per row
+  const uint32_t r32 = static_cast<uint32_t>(rows), c32 = static_cast<uint32_t>(cols);
   if (y_dtype == FP4Q_BF16) {
     auto *yp = static_cast<__nv_bfloat16 *>(y);
-    if (narrow)
-      dequant_kernel<FMT, BROWS, SWZ, uint32_t><<<grid, kThreads, 0, L.stream>>>(
-          q, sf, s_dec, static_cast<uint32_t>(rows), static_cast<uint32_t>(cols), yp);
+    if (narrow && rowal)
+      dequant_kernel<FMT, BROWS, SWZ, uint32_t, true><<<grid, kThreads, 0, L.stream>>>(
+          q, sf, s_dec, r32, c32, yp);
+    else if (narrow)
+      dequant_kernel<FMT, BROWS, SWZ, uint32_t, false><<<grid, kThreads, 0, L.stream>>>(
+          q, sf, s_dec, r32, c32, yp);
     else
-      dequant_kernel<FMT, BROWS, SWZ, int64_t><<<grid, kThreads, 0, L.stream>>>(q, sf, s_dec, rows,
-                                                                               cols, yp);
+      dequant_kernel<FMT, BROWS, SWZ, int64_t, false><<<grid, kThreads, 0, L.stream>>>(
+          q, sf, s_dec, rows, cols, yp);
   } else {
     auto *yp = static_cast<float *>(y);
-    if (narrow)
-      dequant_kernel<FMT, BROWS, SWZ, uint32_t><<<grid, kThreads, 0, L.stream>>>(
-          q, sf, s_dec, static_cast<uint32_t>(rows), static_cast<uint32_t>(cols), yp);
+    if (narrow && rowal)
+      dequant_kernel<FMT, BROWS, SWZ, uint32_t, true><<<grid, kThreads, 0, L.stream>>>(
+          q, sf, s_dec, r32, c32, yp);
+    else if (narrow)
+      dequant_kernel<FMT, BROWS, SWZ, uint32_t, false><<<grid, kThreads, 0, L.stream>>>(
+          q, sf, s_dec, r32, c32, yp);
     else
-      dequant_kernel<FMT, BROWS, SWZ, int64_t><<<grid, kThreads, 0, L.stream>>>(q, sf, s_dec, rows,
-                                                                               cols, yp);
+      dequant_kernel<FMT, BROWS, SWZ, int64_t, false><<<grid, kThreads, 0, L.stream>>>(
+          q, sf, s_dec, rows, cols, yp);
   }
   return cudaGetLastError();
 }

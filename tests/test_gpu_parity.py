@@ -360,34 +360,40 @@ def test_if4_scales_at_an_odd_address(orc, layout):
 
 # ------------------------------------------------------------------ dequant
 
+@pytest.mark.parametrize("cols", [256, 2048])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_dequant_all_formats(orc, out_dtype):
+def test_dequant_all_formats(orc, out_dtype, cols):
+    """Every format, both scale layouts, both output types.  With 2048
+    columns (a multiple of 1024) the kernel's row-aligned form runs: a warp's
+    step lies in one row, one scale offset and one bound test per step."""
     od = orc.FP32 if out_dtype == torch.float32 else orc.BF16
-    x = randmat(256, 256, torch.bfloat16, seed=41).to(DEV)
+    R, C = 256, cols
+    x = randmat(R, C, torch.bfloat16, seed=41).to(DEV)
     for layout in (fq.SCALE_LINEAR, fq.SCALE_SWIZZLED):
         nv = fq.fp4q_quantize_nvfp4(x, layouts=3, scale_layout=layout)
-        y = fq.fp4q_dequantize(fq.FMT_NVFP4, nv["q_row"], nv["sf_row"], 256, 256,
+        y = fq.fp4q_dequantize(fq.FMT_NVFP4, nv["q_row"], nv["sf_row"], R, C,
                                tensor_scale=nv["s_dec"], scale_layout=layout, out_dtype=out_dtype)
-        want = orc.dequantize(orc.FMT_NVFP4, host(nv["q_row"]), host(nv["sf_row"]), 256, 256,
+        want = orc.dequantize(orc.FMT_NVFP4, host(nv["q_row"]), host(nv["sf_row"]), R, C,
                               s_dec=float(host(nv["s_dec"])[0]), scale_layout=layout, out_dtype=od)
         assert_same("nvfp4 deq", host(y), want)
         mx = fq.fp4q_quantize_mxfp4(x, layouts=1, scale_layout=layout)
-        y = fq.fp4q_dequantize(fq.FMT_MXFP4, mx["q_row"], mx["sf_row"], 256, 256, 1, 32,
+        y = fq.fp4q_dequantize(fq.FMT_MXFP4, mx["q_row"], mx["sf_row"], R, C, 1, 32,
                                scale_layout=layout, out_dtype=out_dtype)
-        want = orc.dequantize(orc.FMT_MXFP4, host(mx["q_row"]), host(mx["sf_row"]), 256, 256, 1,
+        want = orc.dequantize(orc.FMT_MXFP4, host(mx["q_row"]), host(mx["sf_row"]), R, C, 1,
                               32, scale_layout=layout, out_dtype=od)
         assert_same("mxfp4 deq", host(y), want)
         i4 = fq.fp4q_quantize_if4(x, scale_layout=layout)
-        y = fq.fp4q_dequantize(fq.FMT_IF4, i4["q"], i4["sf"], 256, 256, tensor_scale=i4["s_dec"],
+        y = fq.fp4q_dequantize(fq.FMT_IF4, i4["q"], i4["sf"], R, C, tensor_scale=i4["s_dec"],
                                scale_layout=layout, out_dtype=out_dtype)
-        want = orc.dequantize(orc.FMT_IF4, host(i4["q"]), host(i4["sf"]), 256, 256,
+        want = orc.dequantize(orc.FMT_IF4, host(i4["q"]), host(i4["sf"]), R, C,
                               s_dec=float(host(i4["s_dec"])[0]), scale_layout=layout, out_dtype=od)
         assert_same("if4 deq", host(y), want)
-    w = randmat(128, 64, torch.float32, seed=42).to(DEV)
+    WC = 64 if cols == 256 else 1024
+    w = randmat(128, WC, torch.float32, seed=42).to(DEV)
     q2 = fq.fp4q_quantize_2d(w)
-    y = fq.fp4q_dequantize(fq.FMT_NVFP4, q2["q_w"], q2["sf_tiles"], 128, 64, 16, 16,
+    y = fq.fp4q_dequantize(fq.FMT_NVFP4, q2["q_w"], q2["sf_tiles"], 128, WC, 16, 16,
                            tensor_scale=q2["s_dec"], out_dtype=out_dtype)
-    want = orc.dequantize(orc.FMT_NVFP4, host(q2["q_w"]), host(q2["sf_tiles"]), 128, 64, 16, 16,
+    want = orc.dequantize(orc.FMT_NVFP4, host(q2["q_w"]), host(q2["sf_tiles"]), 128, WC, 16, 16,
                           s_dec=float(host(q2["s_dec"])[0]), out_dtype=od)
     assert_same("2d deq", host(y), want)
 
