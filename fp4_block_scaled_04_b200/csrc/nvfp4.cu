@@ -264,7 +264,9 @@ __device__ __forceinline__ uint32_t block_scale(float m, const TensorScale &ts, 
 constexpr int kRCTileBytes = 64 * 128;            // one warp tile: 64 rows x 128 bytes
 constexpr int kRCSmem = (kRCThreads / 32) * 2 * kRCTileBytes;
 
-template <typename T, bool MX, bool SR, int QMAX, bool I32>
+// EVEN: rows % 64 == 0 and cols % WC == 0, so every warp tile lies wholly
+// inside the matrix and the bound tests of the copies and stores drop out.
+template <typename T, bool MX, bool SR, int QMAX, bool I32, bool EVEN>
 __global__ void __launch_bounds__(kRCThreads, SR ? 2 : 3)
 rowcol_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_, unsigned layouts,
               const float *__restrict__ amax_ptr, int e8m0_mode, uint64_t seed,
@@ -295,14 +297,14 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_
   // is a multiple of 16, so the row bound is one test per band
   auto issue = [&](const TileCursorT<I> &t, int st) {
     const I col = t.tc * G::WC + cc * CPT;
-    if (col >= cols) return;
+    if (!EVEN && col >= cols) return;
     const I row0 = t.tt * G::WR;
     const T *src = x + (row0 + (lane >> 3)) * ld + col;
     const uint32_t dst =
         stage_s + static_cast<uint32_t>(st * kRCTileBytes + (lane >> 3) * 128 + cc * 16);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      if (row0 + 16 * (i / 4) >= rows) break;
+      if (!EVEN && row0 + 16 * (i / 4) >= rows) break;
       cp_async16(dst + static_cast<uint32_t>(i * 512), src);
       src += 4 * ld;
     }
@@ -332,7 +334,7 @@ rowcol_kernel(const T *__restrict__ x, int64_t rows_, int64_t cols_, int64_t ld_
     __syncwarp();
     const I tr = cur.tt, tc = cur.tc;
     const I r0 = tr * G::WR + band * 16, c0 = tc * G::WC + cc * CPT;
-    const bool valid = r0 < rows && c0 < cols;
+    const bool valid = EVEN || (r0 < rows && c0 < cols);
     // row k of this thread's 16: tb[8 * k] (rows outside the matrix are never
     // copied; their lanes' values only meet other outside lanes and are not stored)
     const uint4 *tb = stage_g + st * (kRCTileBytes / 16) + band * 16 * 8 + cc;
@@ -558,17 +560,25 @@ cudaError_t launch_typed2(const T *x, int64_t rows, int64_t cols, int64_t ld, un
   } else {
     using G = RCGeom<T, MX>;
     const int64_t ntiles = ((cols + G::WC - 1) / G::WC) * ((rows + G::WR - 1) / G::WR);
-    const void *kern = reinterpret_cast<const void *>(rowcol_kernel<T, MX, SR, QMAX, I32>);
-    static KernelSetup setup;
+    const bool even = rows % G::WR == 0 && cols % G::WC == 0;   // whole warp tiles only
+    const void *kern = even
+        ? reinterpret_cast<const void *>(rowcol_kernel<T, MX, SR, QMAX, I32, true>)
+        : reinterpret_cast<const void *>(rowcol_kernel<T, MX, SR, QMAX, I32, false>);
+    static KernelSetup setup, setup_e;
     int per_sm = 0;
-    const cudaError_t e = kernel_setup(setup, kern, kRCThreads, kRCSmem, &per_sm);
+    const cudaError_t e = kernel_setup(even ? setup_e : setup, kern, kRCThreads, kRCSmem, &per_sm);
     if (e != cudaSuccess) return e;
     const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
     const int64_t want = (ntiles + kRCThreads / 32 - 1) / (kRCThreads / 32);
     const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-    rowcol_kernel<T, MX, SR, QMAX, I32><<<grid, kRCThreads, kRCSmem, L.stream>>>(
-        x, rows, cols, ld, layouts, amax, e8m0_mode, seed, s_dec_out, q_row, sf_row, q_col,
-        sf_col, scale_layout);
+    if (even)
+      rowcol_kernel<T, MX, SR, QMAX, I32, true><<<grid, kRCThreads, kRCSmem, L.stream>>>(
+          x, rows, cols, ld, layouts, amax, e8m0_mode, seed, s_dec_out, q_row, sf_row, q_col,
+          sf_col, scale_layout);
+    else
+      rowcol_kernel<T, MX, SR, QMAX, I32, false><<<grid, kRCThreads, kRCSmem, L.stream>>>(
+          x, rows, cols, ld, layouts, amax, e8m0_mode, seed, s_dec_out, q_row, sf_row, q_col,
+          sf_col, scale_layout);
   }
   return cudaGetLastError();
 }
