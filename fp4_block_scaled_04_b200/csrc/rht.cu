@@ -132,7 +132,9 @@ struct TileCursor32 {
   }
 };
 
-template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW, bool I32>
+// EVEN: tokens % 128 == 0 and cols % 16 == 0, so every warp tile lies wholly
+// inside the matrix and the bound tests of the copies and stores drop out.
+template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW, bool I32, bool EVEN>
 __global__ void __launch_bounds__(kThreads, (ROW || SR || N == 128) ? 3 : 4)
 rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
            const RhtParams P, const float *__restrict__ amax_ptr, float *__restrict__ s_dec_out,
@@ -189,12 +191,12 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
   auto issue = [&](const TileCursor32 &t, int st) {
     const int64_t tbase = static_cast<int64_t>(t.tt) * 128;
     const int64_t col = static_cast<int64_t>(t.tc) * 16 + pc * (16 / static_cast<int>(sizeof(T)));
-    if (col >= cols) return;
+    if (!EVEN && col >= cols) return;
     const T *src = dy + (tbase + tok0) * ld + col;
     const uint32_t dst = lane_dst + static_cast<uint32_t>(st * kUnits * UB);
 #pragma unroll
     for (int i = 0; i < 4 * PPT; ++i) {
-      if (tbase + 16 * ((TPI * i) / 16) >= tokens) break;
+      if (!EVEN && tbase + 16 * ((TPI * i) / 16) >= tokens) break;
       // unit_of(tok0 + TPI i, .) - unit_of(tok0, .) = 4 TPI i + 2 ((TPI i) / 16)
       cp_async16(dst + static_cast<uint32_t>((4 * TPI * i + 2 * ((TPI * i) / 16)) * UB), src);
       src += TPI * ld;
@@ -231,7 +233,7 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
     // likewise (tokens % 16 == 0); for n = 128 all groups of a tile are in
     const int64_t t0 = static_cast<int64_t>(cur.tt) * 128 + 16 * g;
     const int64_t c0 = static_cast<int64_t>(cur.tc) * 16 + 4 * cq;
-    const bool valid = c0 < cols && t0 < tokens;
+    const bool valid = EVEN || (c0 < cols && t0 < tokens);
     const uint8_t *ib = wbase + (st * kUnits + my_unit) * UB;
     // The tile's stochastic-rounding bits: element (t, c) draws from Philox
     // call (t cols + c) / 8, one call per token and column octet, 256 per
@@ -424,12 +426,12 @@ rht_kernel(const T *__restrict__ dy, int64_t tokens, int64_t cols, int64_t ld,
       const uint8_t *sb0 = wbase + st * kUnits * UB;
       const int64_t tile_t0 = static_cast<int64_t>(cur.tt) * 128;
       const int64_t col0 = static_cast<int64_t>(cur.tc) * 16;
-      const bool cvalid = col0 < cols;
+      const bool cvalid = EVEN || col0 < cols;
 #pragma unroll 1
       for (int j = 0; j < 4; ++j) {
         const int tok = lane + 32 * j;
         const int64_t t = tile_t0 + tok;
-        const bool tv = cvalid && t < tokens;
+        const bool tv = cvalid && (EVEN || t < tokens);
         const uint8_t *src = sb0 + unit_of(tok, 0) * UB;    // 16 values, 16 * sizeof(T) bytes
         float x[16];
         if (sizeof(T) == 2) {
@@ -546,7 +548,7 @@ RowArgs make_row_args(const float *amax, float *s_dec_out, uint8_t *q, uint8_t *
   return R;
 }
 
-template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW, bool I32>
+template <typename T, int N, bool SR, bool AMAX_ONLY, bool ROW, bool I32, bool EVEN>
 cudaError_t launch_k2(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint64_t seed,
                       const float *amax, float *s_dec_out, unsigned *amax_out, uint8_t *q_t,
                       uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L,
@@ -555,7 +557,8 @@ cudaError_t launch_k2(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uin
   constexpr int WARP_BYTES = 2 * kUnits * UB +
                              ((SR && !(N == 128 && !ROW)) ? kPTabBytes : 0);
   constexpr int SMEM = kWarps * WARP_BYTES;
-  const void *kern = reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY, ROW, I32>);
+  const void *kern =
+      reinterpret_cast<const void *>(rht_kernel<T, N, SR, AMAX_ONLY, ROW, I32, EVEN>);
   static KernelSetup setup;
   int per_sm = 0;
   const cudaError_t e = kernel_setup(setup, kern, kThreads, SMEM, &per_sm);
@@ -565,7 +568,7 @@ cudaError_t launch_k2(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uin
   const int64_t cap = static_cast<int64_t>(per_sm) * L.num_sms;
   const int64_t want = (ntiles + kWarps - 1) / kWarps;
   const int grid = static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
-  rht_kernel<T, N, SR, AMAX_ONLY, ROW, I32><<<grid, kThreads, SMEM, L.stream>>>(
+  rht_kernel<T, N, SR, AMAX_ONLY, ROW, I32, EVEN><<<grid, kThreads, SMEM, L.stream>>>(
       dy, tokens, cols, ld, make_params(seed), amax, s_dec_out, amax_out, q_t, sf_t, scale_layout,
       rht_out, R);
   return cudaGetLastError();
@@ -578,13 +581,27 @@ cudaError_t launch_k(const T *dy, int64_t tokens, int64_t cols, int64_t ld, uint
                      const float *amax, float *s_dec_out, unsigned *amax_out, uint8_t *q_t,
                      uint8_t *sf_t, int scale_layout, float *rht_out, const Launch &L,
                      const RowArgs &R = RowArgs{}) {
-  if (SR && tokens * cols < (int64_t{1} << 35))
-    return launch_k2<T, N, SR, AMAX_ONLY, ROW, true>(dy, tokens, cols, ld, seed, amax, s_dec_out,
-                                                    amax_out, q_t, sf_t, scale_layout, rht_out,
-                                                    L, R);
-  return launch_k2<T, N, SR, AMAX_ONLY, ROW, false>(dy, tokens, cols, ld, seed, amax, s_dec_out,
-                                                   amax_out, q_t, sf_t, scale_layout, rht_out, L,
-                                                   R);
+  const bool i32 = SR && tokens * cols < (int64_t{1} << 35);
+  // whole warp tiles only; not for the 128-point transform with stochastic
+  // rounding, whose even form spills registers and measured no faster
+  if constexpr (!(N == 128 && SR)) {
+    if (tokens % 128 == 0 && cols % 16 == 0) {
+      if (i32)
+        return launch_k2<T, N, SR, AMAX_ONLY, ROW, true, true>(
+            dy, tokens, cols, ld, seed, amax, s_dec_out, amax_out, q_t, sf_t, scale_layout,
+            rht_out, L, R);
+      return launch_k2<T, N, SR, AMAX_ONLY, ROW, false, true>(
+          dy, tokens, cols, ld, seed, amax, s_dec_out, amax_out, q_t, sf_t, scale_layout,
+          rht_out, L, R);
+    }
+  }
+  if (i32)
+    return launch_k2<T, N, SR, AMAX_ONLY, ROW, true, false>(
+        dy, tokens, cols, ld, seed, amax, s_dec_out, amax_out, q_t, sf_t, scale_layout, rht_out,
+        L, R);
+  return launch_k2<T, N, SR, AMAX_ONLY, ROW, false, false>(
+      dy, tokens, cols, ld, seed, amax, s_dec_out, amax_out, q_t, sf_t, scale_layout, rht_out, L,
+      R);
 }
 
 template <typename T, int N>
